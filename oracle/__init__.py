@@ -1,0 +1,156 @@
+"""fp64 CPU oracle of the causal sliding-window attention layer (RoPE -> RMS QK-norm ->
+gated value embedding -> causal windowed softmax attention).
+
+TEST INFRASTRUCTURE.  Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It shares no code with the CUDA library and never
+imports it.
+
+Two independent implementations live here:
+
+* ``forward`` / ``prologue``: the C oracle (``swa_oracle.c``), one query row at a time, fp64.
+* ``brute.py``: a NumPy fp64 restatement that materialises the full T x T score matrix, used
+  as the brute-force pin of the C oracle on small shapes.
+
+Each function cites the passage of the pages it follows in ``swa_oracle.c``'s header.
+Readings taken where the pages are silent (pair layout and sign of RoPE, window boundary,
+eps placement, gate shape) are stated there and in the design notes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _configure(lib):
+    P = ctypes.c_void_p
+    lib.swa_oracle_forward.restype = ctypes.c_int
+    lib.swa_oracle_forward.argtypes = [P, P, P, P, P, ctypes.c_int, P, ctypes.c_int, P,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_double, ctypes.c_double,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       P, ctypes.c_int64, P, P]
+    lib.swa_oracle_prologue.restype = ctypes.c_int
+    lib.swa_oracle_prologue.argtypes = [P, P, P, P, P, ctypes.c_int, P, ctypes.c_int, P,
+                                        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_double, ctypes.c_double,
+                                        ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P]
+    lib.swa_oracle_threads.restype = ctypes.c_int
+    lib.swa_oracle_round_bf16.restype = ctypes.c_double
+    lib.swa_oracle_round_bf16.argtypes = [ctypes.c_double]
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _configure(ctypes.CDLL(_build.build()))
+    return _lib
+
+
+def _swap_library(path: Optional[str]):
+    """Test hook: load another build of swa_oracle.c (e.g. one with a planted mistake).
+    ``None`` restores the regular build.  Returns the previously loaded library."""
+    global _lib
+    prev = _lib
+    _lib = None if path is None else _configure(ctypes.CDLL(path))
+    return prev
+
+
+def threads() -> int:
+    return int(_load().swa_oracle_threads())
+
+
+def round_bf16(x: float) -> float:
+    return float(_load().swa_oracle_round_bf16(float(x)))
+
+
+def _bits(t) -> np.ndarray:
+    """bf16 tensor/array -> contiguous uint16 bit patterns (no value conversion)."""
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        assert t.dtype == np.uint16
+        return np.ascontiguousarray(t)
+    import torch
+    assert t.dtype == torch.bfloat16, t.dtype
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _ve_args(inputs: Dict):
+    if inputs.get("ids") is None:
+        return None, None, 0, None, 0, None
+    import torch
+    ids = inputs["ids"]
+    ids = ids.cpu().contiguous().numpy().astype(np.int64) if isinstance(ids, torch.Tensor) else np.ascontiguousarray(ids, dtype=np.int64)
+    table = _bits(inputs["table"])
+    x = _bits(inputs["x"])
+    Wg = _bits(inputs["Wg"])
+    return ids, table, int(table.shape[0]), x, int(x.shape[-1]), Wg
+
+
+def forward(inputs: Dict, window: int, rope_base: float = 10000.0, eps: float = 1e-6, *,
+            parity: bool = True, rope: bool = True, qknorm: bool = True,
+            window_convention: int = 0, rows=None):
+    """Attention forward of one layer.
+
+    inputs: dict with q, k, v bf16 (B,T,H,D) and, for value-embedding layers, ids (B,T),
+    table [vocab, H*D], x (B,T,C), Wg [32,H].
+    parity=True rounds qhat, khat, v' to bf16 after the fp64 prologue (pure fp64 otherwise).
+    rope/qknorm switch the prologue steps off (test-only, for the library special case).
+    rows: None for every row, else flat query ids ((b*H + h)*T + i).
+
+    Returns (out, lse): out fp64 (B,T,H,D) and lse fp64 (B,H,T) when rows is None, else
+    out [n_rows, D] and lse [n_rows] in the sorted order of ``rows``.
+    """
+    lib = _load()
+    q, k, v = _bits(inputs["q"]), _bits(inputs["k"]), _bits(inputs["v"])
+    B, T, H, D = q.shape
+    ids, table, vocab, x, C, Wg = _ve_args(inputs)
+    if rows is None:
+        rows_a = None
+        n = 0
+        out = np.empty((B, T, H, D), dtype=np.float64)
+        lse = np.empty((B, H, T), dtype=np.float64)
+    else:
+        rows_a = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        if rows_a.size > 1 and np.any(np.diff(rows_a) < 0):
+            raise ValueError("rows must be sorted ascending")
+        n = int(rows_a.size)
+        out = np.empty((n, D), dtype=np.float64)
+        lse = np.empty((n,), dtype=np.float64)
+    rc = lib.swa_oracle_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(ids), _ptr(table), vocab,
+                                _ptr(x), C, _ptr(Wg), B, T, H, D, int(window),
+                                float(rope_base), float(eps), int(parity), int(rope), int(qknorm),
+                                int(window_convention), _ptr(rows_a), n, _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return out, lse
+
+
+def prologue(inputs: Dict, rope_base: float = 10000.0, eps: float = 1e-6, *,
+             parity: bool = False, rope: bool = True, qknorm: bool = True):
+    """qhat, khat, v' as fp64 (B,T,H,D) arrays (the steps before the attention)."""
+    lib = _load()
+    q, k, v = _bits(inputs["q"]), _bits(inputs["k"]), _bits(inputs["v"])
+    B, T, H, D = q.shape
+    ids, table, vocab, x, C, Wg = _ve_args(inputs)
+    qh = np.empty((B, T, H, D), dtype=np.float64)
+    kh = np.empty_like(qh)
+    vp = np.empty_like(qh)
+    rc = lib.swa_oracle_prologue(_ptr(q), _ptr(k), _ptr(v), _ptr(ids), _ptr(table), vocab,
+                                 _ptr(x), C, _ptr(Wg), B, T, H, D, float(rope_base), float(eps),
+                                 int(parity), int(rope), int(qknorm), _ptr(qh), _ptr(kh), _ptr(vp))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return qh, kh, vp

@@ -1,0 +1,268 @@
+/*
+ * swa_oracle.c -- plain fp64 CPU oracle of the causal sliding-window attention layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may include, link, load or call
+ * this file; only the tests, the smoke check and the benchmark's CPU-baseline leg use it.
+ * It shares no code with the CUDA library.
+ *
+ * What it computes, in the order the pages state it, one query row at a time:
+ *
+ *   1. RoPE on q and k  (intelliparadigm "GPT-2 for $73", section 2.2, the QK-norm snippet
+ *      "q, k = normalize(apply_rope(q)), normalize(apply_rope(k))"; kongchang speedrun explainer,
+ *      "RoPE" paragraph: rotation matrices that make scores depend on relative position).
+ *      Reading taken where the pages are silent: pairs are (i, i + D/2) for i < D/2, the
+ *      frequency of pair i is theta_i = base^(-2i/D), and position t rotates the pair
+ *      (a, b) -> (a cos(t theta_i) - b sin(t theta_i), a sin(t theta_i) + b cos(t theta_i)).
+ *      Angles and their cos/sin are taken in fp64.
+ *   2. Parameter-free RMS normalisation after RoPE (same section 2.1/2.2: RMSNorm with no
+ *      gamma/beta; PaperWeekly repost, "QK Normalization ... after RoPE"):
+ *      xhat = x / sqrt(mean_D(x^2) + eps).
+ *   3. Gated value embedding on VE layers (PaperWeekly repost, "Value Embeddings"
+ *      paragraph: ve = value_embeds[layer](token_ids); gate = 2*sigmoid(ve_gate(x[:, :, :32]));
+ *      v = v + gate*ve).  Reading: ve_gate is a bias-free linear map Wg [32, H], one gate per
+ *      head, broadcast over D.  This oracle does its own lookup ve = table[ids].
+ *   4. Scaled dot-product attention with the causal mask including the diagonal ("Let's
+ *      reproduce GPT-2 (124M)" notes, section 3, the attention listing and the paragraph on
+ *      the lower-triangular mask): s_j = qhat_i . khat_j / sqrt(D), softmax over the visible
+ *      keys, out_i = sum_j p_j v'_j.  The window (intelliparadigm section 3.2, "local window
+ *      (1024 tokens)") is read as W keys including the query itself: key j is visible to
+ *      query i iff 0 <= i - j < W; window <= 0 or >= T means full causal.
+ *   5. The log-sum-exp of the scaled scores per row (natural log): lse_i = M + ln(sum exp(s - M)).
+ *
+ * Nothing is blocked, fused or reordered beyond this definition.  The only parallelism is
+ * an OpenMP split over independent (position) and (query row) indices.
+ *
+ * Parity mode (round_bf16 = 1) rounds qhat, khat and v' to bf16 (round to nearest even)
+ * after the fp64 prologue, because the tensor-core operands of the GPU path are bf16; the
+ * attention itself stays fp64.  Pure mode (round_bf16 = 0) is fp64 throughout.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* bf16 bit pattern -> double, exactly (bf16 is the top half of an IEEE binary32). */
+static double bf16_to_double(uint16_t h) {
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* double -> nearest bf16 value (ties to even), returned as a double.  bf16 keeps 8
+ * significant bits; frexp gives x = m * 2^e with 0.5 <= |m| < 1, so m * 2^8 lies in
+ * [128, 256) and rounding it to an integer in the current (nearest-even) mode rounds x to
+ * 8 significant bits in one step, with no intermediate float rounding. */
+static double round_to_bf16(double x) {
+    if (x == 0.0 || !isfinite(x)) return x;
+    int e;
+    double m = frexp(x, &e);
+    double r = nearbyint(ldexp(m, 8));
+    return ldexp(r, e - 8);
+}
+
+static void rope_inplace(double* x, int D, int t, double base) {
+    const int half = D / 2;
+    for (int i = 0; i < half; ++i) {
+        double theta = pow(base, -2.0 * (double)i / (double)D);
+        double ang = (double)t * theta;
+        double c = cos(ang), s = sin(ang);
+        double a = x[i], b = x[i + half];
+        x[i] = a * c - b * s;
+        x[i + half] = a * s + b * c;
+    }
+}
+
+static void rmsnorm_inplace(double* x, int D, double eps) {
+    double ss = 0.0;
+    for (int d = 0; d < D; ++d) ss += x[d] * x[d];
+    double r = 1.0 / sqrt(ss / (double)D + eps);
+    for (int d = 0; d < D; ++d) x[d] *= r;
+}
+
+/* q or k row (b, t, h) -> qhat/khat in out[D]. */
+static void prologue_qk(const uint16_t* src, int T, int H, int D, int b, int t, int h,
+                        double base, double eps, int use_rope, int use_qknorm, int round_bf16,
+                        double* out) {
+    const uint16_t* row = src + (((size_t)b * T + t) * H + h) * (size_t)D;
+    for (int d = 0; d < D; ++d) out[d] = bf16_to_double(row[d]);
+    if (use_rope) rope_inplace(out, D, t, base);
+    if (use_qknorm) rmsnorm_inplace(out, D, eps);
+    if (round_bf16)
+        for (int d = 0; d < D; ++d) out[d] = round_to_bf16(out[d]);
+}
+
+/* v row (b, t, h) -> v' = v + 2 sigmoid(x[b,t,:32] . Wg[:, h]) * table[ids[b,t], h*D:(h+1)*D]. */
+static void prologue_v(const uint16_t* v, const int64_t* ids, const uint16_t* table,
+                       const uint16_t* x, int C, const uint16_t* Wg,
+                       int T, int H, int D, int b, int t, int h, int round_bf16, double* out) {
+    const uint16_t* row = v + (((size_t)b * T + t) * H + h) * (size_t)D;
+    for (int d = 0; d < D; ++d) out[d] = bf16_to_double(row[d]);
+    if (ids != NULL) {
+        const uint16_t* xr = x + ((size_t)b * T + t) * (size_t)C;
+        double z = 0.0;
+        for (int c = 0; c < 32; ++c) z += bf16_to_double(xr[c]) * bf16_to_double(Wg[c * H + h]);
+        double gate = 2.0 / (1.0 + exp(-z));
+        int64_t id = ids[(size_t)b * T + t];
+        const uint16_t* ve = table + (size_t)id * (size_t)H * D + (size_t)h * D;
+        for (int d = 0; d < D; ++d) out[d] += gate * bf16_to_double(ve[d]);
+    }
+    if (round_bf16)
+        for (int d = 0; d < D; ++d) out[d] = round_to_bf16(out[d]);
+}
+
+static int ids_in_range(const int64_t* ids, int64_t n, int vocab) {
+    for (int64_t i = 0; i < n; ++i)
+        if (ids[i] < 0 || ids[i] >= vocab) return 0;
+    return 1;
+}
+
+static int visible(int i, int j, int W, int convention) {
+    int diff = i - j;
+    if (diff < 0) return 0;
+    return convention == 0 ? (diff < W) : (diff <= W);
+}
+
+/* One attention row: qhat_i against khat[0..T), v'[0..T) of one (b, h). */
+static void attention_row(const double* qh, const double* kh, const double* vp, int T, int D,
+                          int i, int W, int convention, double* out, double* lse, double* s) {
+    const double scale = 1.0 / sqrt((double)D);
+    double M = -INFINITY;
+    for (int j = 0; j < T; ++j) {
+        if (!visible(i, j, W, convention)) continue;
+        double acc = 0.0;
+        for (int d = 0; d < D; ++d) acc += qh[d] * kh[(size_t)j * D + d];
+        s[j] = acc * scale;
+        if (s[j] > M) M = s[j];
+    }
+    double L = 0.0;
+    for (int j = 0; j < T; ++j)
+        if (visible(i, j, W, convention)) L += exp(s[j] - M);
+    for (int d = 0; d < D; ++d) out[d] = 0.0;
+    for (int j = 0; j < T; ++j) {
+        if (!visible(i, j, W, convention)) continue;
+        double p = exp(s[j] - M) / L;
+        for (int d = 0; d < D; ++d) out[d] += p * vp[(size_t)j * D + d];
+    }
+    *lse = M + log(L);
+}
+
+int swa_oracle_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * q, k, v       bf16 bit patterns, (B, T, H, D) contiguous.
+ * ids, table    VE token ids (B, T) and table [vocab, H*D] bf16; ids == NULL means no VE.
+ * x, C          x (B, T, C) bf16; the gate reads channels 0..31.
+ * Wg            [32, H] bf16.
+ * window        <= 0 or >= T: full causal.
+ * rows/n_rows   flat query ids ((b*H + h)*T + i), sorted ascending; rows == NULL: every row.
+ * out           rows == NULL: (B, T, H, D) fp64; else [n_rows, D].
+ * lse           rows == NULL: (B, H, T) fp64;   else [n_rows].
+ * Returns 0, or -1 on bad arguments / allocation failure.
+ */
+int swa_oracle_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                       const int64_t* ids, const uint16_t* table, int vocab,
+                       const uint16_t* x, int C, const uint16_t* Wg,
+                       int B, int T, int H, int D, int window, double rope_base, double eps,
+                       int round_bf16, int use_rope, int use_qknorm, int window_convention,
+                       const int64_t* rows, int64_t n_rows, double* out, double* lse) {
+    if (B < 1 || T < 1 || H < 1 || D < 2 || (D % 2) != 0) return -1;
+    if (ids != NULL && (table == NULL || x == NULL || Wg == NULL || C < 32 || vocab < 1)) return -1;
+    if (ids != NULL && !ids_in_range(ids, (int64_t)B * T, vocab)) return -1;
+    const int W = (window <= 0 || window >= T) ? T : window;
+    const int64_t total_rows = (int64_t)B * H * T;
+    if (rows == NULL) n_rows = total_rows;
+
+    double* kh = (double*)malloc(sizeof(double) * (size_t)T * D);
+    double* vp = (double*)malloc(sizeof(double) * (size_t)T * D);
+    if (!kh || !vp) { free(kh); free(vp); return -1; }
+    int rc = 0;
+
+    int64_t r0 = 0;
+    while (r0 < n_rows) {
+        /* The run of requested rows that share one (b, h). */
+        int64_t id0 = rows ? rows[r0] : r0;
+        if (id0 < 0 || id0 >= total_rows) { rc = -1; break; }
+        int64_t bh = id0 / T;
+        int64_t r1 = r0 + 1;
+        while (r1 < n_rows && (rows ? rows[r1] : r1) / T == bh) ++r1;
+        const int b = (int)(bh / H), h = (int)(bh % H);
+
+        #pragma omp parallel for schedule(static)
+        for (int t = 0; t < T; ++t) {
+            prologue_qk(k, T, H, D, b, t, h, rope_base, eps, use_rope, use_qknorm, round_bf16,
+                        kh + (size_t)t * D);
+            prologue_v(v, ids, table, x, C, Wg, T, H, D, b, t, h, round_bf16, vp + (size_t)t * D);
+        }
+
+        int bad = 0;
+        #pragma omp parallel
+        {
+            double* qh = (double*)malloc(sizeof(double) * (size_t)D);
+            double* s = (double*)malloc(sizeof(double) * (size_t)T);
+            double* o = (double*)malloc(sizeof(double) * (size_t)D);
+            const int ok = (qh != NULL && s != NULL && o != NULL);
+            #pragma omp for schedule(dynamic, 16)
+            for (int64_t r = r0; r < r1; ++r) {
+                if (!ok) {
+                    #pragma omp atomic write
+                    bad = 1;
+                    continue;
+                }
+                int64_t id = rows ? rows[r] : r;
+                int i = (int)(id % T);
+                double l;
+                prologue_qk(q, T, H, D, b, i, h, rope_base, eps, use_rope, use_qknorm,
+                            round_bf16, qh);
+                attention_row(qh, kh, vp, T, D, i, W, window_convention, o, &l, s);
+                if (rows) {
+                    memcpy(out + (size_t)r * D, o, sizeof(double) * (size_t)D);
+                    lse[r] = l;
+                } else {
+                    memcpy(out + (((size_t)b * T + i) * H + h) * (size_t)D, o,
+                           sizeof(double) * (size_t)D);
+                    lse[((size_t)b * H + h) * T + i] = l;
+                }
+            }
+            free(qh); free(s); free(o);
+        }
+        if (bad) { rc = -1; break; }
+        r0 = r1;
+    }
+    free(kh); free(vp);
+    return rc;
+}
+
+/* The prologue alone, for the pins on RoPE / RMS / gate: qhat, khat, v' as fp64 (B,T,H,D). */
+int swa_oracle_prologue(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                        const int64_t* ids, const uint16_t* table, int vocab,
+                        const uint16_t* x, int C, const uint16_t* Wg,
+                        int B, int T, int H, int D, double rope_base, double eps,
+                        int round_bf16, int use_rope, int use_qknorm,
+                        double* qh, double* kh, double* vp) {
+    if (B < 1 || T < 1 || H < 1 || D < 2 || (D % 2) != 0) return -1;
+    if (ids != NULL && (table == NULL || x == NULL || Wg == NULL || C < 32 || vocab < 1)) return -1;
+    if (ids != NULL && !ids_in_range(ids, (int64_t)B * T, vocab)) return -1;
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t)
+            for (int h = 0; h < H; ++h) {
+                size_t off = (((size_t)b * T + t) * H + h) * (size_t)D;
+                prologue_qk(q, T, H, D, b, t, h, rope_base, eps, use_rope, use_qknorm, round_bf16, qh + off);
+                prologue_qk(k, T, H, D, b, t, h, rope_base, eps, use_rope, use_qknorm, round_bf16, kh + off);
+                prologue_v(v, ids, table, x, C, Wg, T, H, D, b, t, h, round_bf16, vp + off);
+            }
+    return 0;
+}
+
+/* Exposed for the rounding pin: double -> bf16 value, ties to even. */
+double swa_oracle_round_bf16(double x) { return round_to_bf16(x); }
