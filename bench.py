@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark of the causal sliding-window attention forward on B200.
+
+Metric: attention-forward TFLOP/s counted over unmasked (query, key) pairs (4*D flops per pair:
+2D for q.k, 2D for p*v), with tokens/s and the fraction of the dense-BF16 tensor peak, on the
+nanochat d24 full-window layer with value embeddings (B=16, T=2048, H=12, D=128, W=2048).
+
+One step = one whole layer forward (RoPE + RMS QK-norm + VE gate prologue, then the windowed
+attention with its LSE) on inputs already resident in HBM.  Inputs are seeded synthetic
+N(0,1) bf16 tensors shaped like the layer; they are larger than the 126 MB L2, so no flush
+is needed between steps.
+
+  python bench.py [--gpus N --steps K --warmup W]            # our CUDA path
+  python bench.py --impl reference [--steps K --warmup W]    # the fp64 CPU oracle, same metric
+
+With N > 1 (torchrun), every rank runs its own batch shard of 16 sequences (weak scaling, no
+collective on the data path); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+WORKLOADS = {
+    "d24_L_VE": workloads.D24_L_VE,
+    "d24_S": workloads.D24_S,
+    "gpt2_124m": workloads.GPT2,
+    "tiny": workloads.TINY,
+}
+METRIC = "attention fwd TFLOP/s (unmasked pairs) & tokens/s, d24 T=2048; % of BF16 peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["causal_sliding_window_swa_b200/csrc/attn_fwd.cuh",
+                  "causal_sliding_window_swa_b200/csrc/ptx.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
+
+
+# ------------------------------------------------------------------ host-side helpers
+
+def flops_per_step(s: workloads.LayerShape) -> float:
+    return 4.0 * s.D * s.unmasked_pairs()
+
+
+def shard_shape(s: workloads.LayerShape, rank: int) -> workloads.LayerShape:
+    """Rank r's batch shard: same per-GPU shape, its own seed (rank 0 keeps the workload's)."""
+    import dataclasses
+    return dataclasses.replace(s, seed=s.seed + 1000 * rank)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload: str):
+    """dram__bytes_read.sum + dram__bytes_write.sum per launch of the attention kernel from the
+    committed ncu summary, or None if absent or taken on a different kernel source."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            doc = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = doc.get(workload)
+    if not ent or ent.get("kernel_sha256") != kernel_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def reduce_max(x: float, device=None) -> float:
+    """Max of a scalar over all ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.index = index
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        self.ok = False
+
+    def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            return self
+        self._thr = threading.Thread(target=self._run, daemon=True)
+        self._thr.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                bits = get(self._h)
+                for b, name in self.REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def stop(self):
+        self._stop.set()
+        if self._thr is not None:
+            self._thr.join()
+        return {"sm_mhz": (statistics.median(self.samples) if self.samples else None),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def cpu_baseline(s: workloads.LayerShape, d, budget_s: float):
+    """The fp64 oracle, as it stands, on whole (b, h) slices of the workload (every query row of
+    the slice) until ~budget_s seconds of CPU work are done.  Returns the metric in TFLOP/s."""
+    import numpy as np
+    import oracle
+    W = s.eff_window()
+    pairs_per_bh = W * (W + 1) // 2 + (s.T - W) * W
+    done = 0
+    t0 = time.perf_counter()
+    for bh in range(s.B * s.H):
+        rows = np.arange(bh * s.T, (bh + 1) * s.T, dtype=np.int64)
+        oracle.forward(d, s.window, parity=True, rows=rows)
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    flops = 4.0 * s.D * pairs_per_bh * done
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{done} of {s.B * s.H} (b,h) slices of {s.name}, every query row of each "
+                      f"({done * pairs_per_bh} unmasked pairs), {dt:.1f} s",
+            "tokens_per_s": done * s.T / s.H / dt}
+
+
+def config_of(s: workloads.LayerShape, world: int):
+    return {"workload": s.name, "B_per_gpu": s.B, "T": s.T, "H": s.H, "D": s.D,
+            "window": s.eff_window(), "value_embeddings": s.ve, "global_batch": s.B * world,
+            "seq_len": s.T, "parallelism": f"dp{world} (batch shards, no collective)",
+            "l2": "no flush: inputs (q,k,v" + (",ve" if s.ve else "") +
+                  f") = {(4 if s.ve else 3) * s.n_elems * 2 / 1e6:.0f} MB > 126 MB L2"}
+
+
+# ------------------------------------------------------------------------ reference arm
+
+def run_reference(args, s):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import numpy as np
+    import oracle
+    d = workloads.make_layer(s)
+    W = s.eff_window()
+    total_steps = args.steps + args.warmup
+    per_step_budget = max(0.02, args.reference_budget_s / max(1, total_steps))
+    g = np.random.default_rng(1234)
+
+    def step(n_rows):
+        bh = int(g.integers(0, s.B * s.H))
+        i = np.sort(g.choice(s.T, size=n_rows, replace=False)).astype(np.int64)
+        rows = bh * s.T + i
+        t0 = time.perf_counter()
+        oracle.forward(d, s.window, parity=True, rows=rows)
+        dt = time.perf_counter() - t0
+        pairs = int(np.minimum(i + 1, W).sum())
+        return dt, pairs
+
+    # calibrate the rows per step to the per-step budget
+    dt, _ = step(32)
+    n_rows = int(max(1, min(s.T, 32 * per_step_budget / max(dt, 1e-6))))
+    for _ in range(args.warmup):
+        step(n_rows)
+    tot_t, tot_pairs = 0.0, 0
+    for _ in range(args.steps):
+        dt, pairs = step(n_rows)
+        tot_t += dt
+        tot_pairs += pairs
+    value = 4.0 * s.D * tot_pairs / tot_t / 1e12
+    cores = oracle.threads()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(s, world), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {n_rows} seeded query rows of one random (b,h) slice "
+                                   f"of {s.name} (with that slice's prologue)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- our arm
+
+def run_ours(args, s0):
+    import torch
+    import torch.distributed as dist
+    import causal_sliding_window_swa_b200 as swa
+
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    s = shard_shape(s0, rank)
+
+    d = workloads.make_layer(s)
+    g = workloads.gpu_side_inputs(d)
+    host = {k: (None if v is None else v.contiguous().pin_memory()) for k, v in g.items()}
+    x = {k: (None if v is None else v.to(dev, non_blocking=True)) for k, v in host.items()}
+    out = torch.empty_like(x["q"])
+    lse = torch.empty((s.B, s.H, s.T), dtype=torch.float32, device=dev)
+    nbytes = swa.swa_attn_workspace_bytes(s.B, s.T, s.H, s.D, int(s.ve))
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    st = stream.cuda_stream
+    P = lambda t: None if t is None else t.data_ptr()
+    args_pro = (P(x["q"]), P(x["k"]), P(x["v"]), P(x["ve"]), P(x["gate_x"]), P(x["Wg"]),
+                s.B, s.T, s.H, s.D, 10000.0, 1e-6, ws.data_ptr(), nbytes, st)
+    args_att = (P(x["v"]), int(s.ve), out.data_ptr(), lse.data_ptr(), s.B, s.T, s.H, s.D, s.window,
+                ws.data_ptr(), nbytes, st)
+
+    def check(rc, what):
+        if rc != 0:
+            raise swa.SwaError(rc, what)
+
+    # The RoPE table depends only on (T, D, base): built once, like a model's rotary cache.
+    check(swa.swa_attn_rope_table(s.B, s.T, s.H, s.D, int(s.ve), 10000.0, ws.data_ptr(), nbytes, st),
+          "swa_attn_rope_table")
+
+    K, Wm = args.steps, args.warmup
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+
+    def step(e=None):
+        if e is not None:
+            e[0].record(stream)
+        check(swa.swa_attn_prologue(*args_pro), "swa_attn_prologue")
+        if e is not None:
+            e[1].record(stream)
+        check(swa.swa_attn_attention(*args_att), "swa_attn_attention")
+        if e is not None:
+            e[2].record(stream)
+
+    for _ in range(Wm):
+        step()
+    torch.cuda.synchronize(dev)
+    swa.check_device_status(stream)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local).start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(K):
+        step(ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    swa.check_device_status(stream)
+    ms_local = t_start.elapsed_time(t_end) / K
+    pro_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
+    att_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    ms = reduce_max(ms_local, dev)
+    att_ms_max = reduce_max(att_ms, dev)
+    pro_ms_max = reduce_max(pro_ms, dev)
+
+    # ---------------- end to end through the public call, host buffers, copies inside
+    E = max(1, min(args.e2e_steps, K))
+    h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h_lse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    xin = {k: (None if v is None else torch.empty_like(v)) for k, v in x.items()}
+
+    def e2e_step():
+        for k, v in host.items():
+            if v is not None:
+                xin[k].copy_(v, non_blocking=True)
+        swa.forward(xin["q"], xin["k"], xin["v"], s.window, xin["ve"], xin["gate_x"], xin["Wg"],
+                    out=out, lse=lse)
+        h_out.copy_(out, non_blocking=True)
+        h_lse.copy_(lse, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    swa.check_device_status(stream)
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / E, dev)
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+
+    # ---------------- roll-up
+    fl = flops_per_step(s)
+    value = world * fl / (ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = fl / (att_ms_max * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": Wm,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 q,k,v; VE table/ids/x/Wg as the "
+                                  "layer's shapes)",
+        "config": config_of(s, world),
+        "tokens_per_s": world * s.B * s.T / (ms * 1e-3),
+        "pct_bf16_peak": 100.0 * value / world / peak,
+        "peak_source": f"{peak_src} bf16_tflops (burst)",
+        "stage_ms": {"prologue": pro_ms_max, "attention": att_ms_max},
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": recorded_traffic(args.workload),
+                     "note": f"4*D flops per unmasked pair / mean attention launch time; peak = "
+                             f"{peak_src} dense bf16 (burst)"},
+        "prologue_roofline": {"bound": "hbm", "achieved": prologue_bytes(s) / (pro_ms_max * 1e-3) / 1e9,
+                              "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                              "frac": prologue_bytes(s) / (pro_ms_max * 1e-3) / 1e9 / float(peaks["hbm_gbs"])},
+        "e2e": {"value": world * fl / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(s, d, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def prologue_bytes(s: workloads.LayerShape) -> float:
+    """Algorithmic bytes of the prologue: read q, k, v (+ ve, gate_x, Wg), write qhat, khat
+    (+ v')."""
+    n = s.n_elems * 2
+    b = 2 * n + 2 * n           # q, k in; qhat, khat out
+    if s.ve:
+        b += 3 * n + s.B * s.T * 32 * 2 + 32 * s.H * 2   # v, ve in; v' out; gate_x, Wg
+    return float(b)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="d24_L_VE")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-budget-s", type=float, default=90.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    s = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, s)
+    return run_ours(args, s)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

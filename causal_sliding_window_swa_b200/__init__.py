@@ -1,0 +1,212 @@
+"""B200 (sm_100a) causal sliding-window attention forward: Python binding of the C ABI in
+``include/swa_attn.h``.
+
+This module only marshals arguments: every step of the layer (RoPE, RMS QK-norm, the value-
+embedding gate, the windowed attention, the log-sum-exp) runs in the CUDA kernels of
+``libswa_attn.so``.  There is no CPU path: the first call loads the library and raises if it
+is not built (``load()`` does that eagerly).
+
+Functions with the C names take raw device pointers (ints) and return the status code.
+``forward`` is the tensor-level convenience call: it checks dtypes and layouts, allocates the
+outputs with torch and raises ``SwaError`` on a non-zero status.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libswa_attn.so")
+
+SWA_OK = 0
+SWA_ERR_INVALID_ARG = -1
+SWA_ERR_UNSUPPORTED = -2
+SWA_ERR_MISALIGNED = -3
+SWA_ERR_CUDA = -4
+SWA_ERR_TIMEOUT = -5
+SWA_ERR_NO_MEMORY = -6
+SWA_ERR_NO_DEVICE = -7
+
+
+class SwaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {swa_attn_strerror(status)} (status {status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m causal_sliding_window_swa_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.swa_attn_fwd.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, F, F, P]
+    lib.swa_attn_fwd.restype = I
+    lib.swa_attn_fwd_ws.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, F, F, P, Z, P]
+    lib.swa_attn_fwd_ws.restype = I
+    lib.swa_attn_workspace_bytes.argtypes = [I, I, I, I, I]
+    lib.swa_attn_workspace_bytes.restype = Z
+    lib.swa_attn_workspace_offset.argtypes = [I, I, I, I, I, I]
+    lib.swa_attn_workspace_offset.restype = Z
+    lib.swa_attn_rope_table.argtypes = [I, I, I, I, I, F, P, Z, P]
+    lib.swa_attn_rope_table.restype = I
+    lib.swa_attn_prologue.argtypes = [P, P, P, P, P, P, I, I, I, I, F, F, P, Z, P]
+    lib.swa_attn_prologue.restype = I
+    lib.swa_attn_attention.argtypes = [P, I, P, P, I, I, I, I, I, P, Z, P]
+    lib.swa_attn_attention.restype = I
+    lib.swa_attn_strerror.argtypes = [I]
+    lib.swa_attn_strerror.restype = ctypes.c_char_p
+    lib.swa_attn_last_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
+    lib.swa_attn_last_device_status.restype = I
+    lib.swa_attn_set_wait_limit_ms.argtypes = [I]
+    lib.swa_attn_set_wait_limit_ms.restype = I
+    lib.swa_attn_version.argtypes = []
+    lib.swa_attn_version.restype = I
+    return lib
+
+
+_lib_handle: Optional[ctypes.CDLL] = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libswa_attn.so (once); raises ImportError/OSError if it is missing or stale."""
+    global _lib_handle
+    if _lib_handle is None:
+        _lib_handle = _load()
+    return _lib_handle
+
+
+class _LazyLib:
+    def __getattr__(self, name):
+        return getattr(load(), name)
+
+
+_lib = _LazyLib()
+
+
+# ------------------------------------------------------------------ the C entry points
+
+def swa_attn_fwd(q, k, v, ve, gate_x, Wg, out, lse, B, T, H, D, window, rope_base, eps, stream) -> int:
+    return _lib.swa_attn_fwd(q, k, v, ve, gate_x, Wg, out, lse, B, T, H, D, window, rope_base, eps, stream)
+
+
+def swa_attn_fwd_ws(q, k, v, ve, gate_x, Wg, out, lse, B, T, H, D, window, rope_base, eps,
+                    workspace, ws_bytes, stream) -> int:
+    return _lib.swa_attn_fwd_ws(q, k, v, ve, gate_x, Wg, out, lse, B, T, H, D, window, rope_base, eps,
+                                workspace, ws_bytes, stream)
+
+
+def swa_attn_workspace_bytes(B, T, H, D, has_ve) -> int:
+    return int(_lib.swa_attn_workspace_bytes(B, T, H, D, int(has_ve)))
+
+
+SWA_WS_QHAT, SWA_WS_KHAT, SWA_WS_VPRIME, SWA_WS_ROPE_TABLE = 0, 1, 2, 3
+
+
+def swa_attn_workspace_offset(B, T, H, D, has_ve, section) -> int:
+    return int(_lib.swa_attn_workspace_offset(B, T, H, D, int(has_ve), int(section)))
+
+
+def swa_attn_rope_table(B, T, H, D, has_ve, rope_base, workspace, ws_bytes, stream) -> int:
+    return _lib.swa_attn_rope_table(B, T, H, D, int(has_ve), rope_base, workspace, ws_bytes, stream)
+
+
+def swa_attn_prologue(q, k, v, ve, gate_x, Wg, B, T, H, D, rope_base, eps, workspace, ws_bytes, stream) -> int:
+    return _lib.swa_attn_prologue(q, k, v, ve, gate_x, Wg, B, T, H, D, rope_base, eps, workspace, ws_bytes, stream)
+
+
+def swa_attn_attention(v, has_ve, out, lse, B, T, H, D, window, workspace, ws_bytes, stream) -> int:
+    return _lib.swa_attn_attention(v, int(has_ve), out, lse, B, T, H, D, window, workspace, ws_bytes, stream)
+
+
+def swa_attn_strerror(status: int) -> str:
+    return _lib.swa_attn_strerror(int(status)).decode()
+
+
+def swa_attn_last_device_status(stream=None) -> Tuple[int, int]:
+    detail = ctypes.c_uint(0)
+    rc = _lib.swa_attn_last_device_status(stream, ctypes.byref(detail))
+    return int(rc), int(detail.value)
+
+
+def swa_attn_set_wait_limit_ms(ms: int) -> int:
+    return int(_lib.swa_attn_set_wait_limit_ms(int(ms)))
+
+
+def swa_attn_version() -> int:
+    return int(_lib.swa_attn_version())
+
+
+# ------------------------------------------------------------- tensor-level convenience
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+def _check_qkv(q, k, v, ve, gate_x, Wg):
+    import torch
+    if q.dim() != 4:
+        raise ValueError("q, k, v must be (B, T, H, D)")
+    for name, t in (("q", q), ("k", k), ("v", v), ("ve", ve)):
+        if t is None:
+            continue
+        if t.shape != q.shape or t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {tuple(q.shape)}")
+    B, T, H, D = q.shape
+    if ve is not None:
+        if gate_x is None or Wg is None:
+            raise ValueError("ve, gate_x and Wg go together")
+        if tuple(gate_x.shape) != (B, T, 32) or gate_x.dtype != torch.bfloat16 or not gate_x.is_contiguous():
+            raise ValueError("gate_x must be a contiguous bf16 (B, T, 32) tensor")
+        if tuple(Wg.shape) != (32, H) or Wg.dtype != torch.bfloat16 or not Wg.is_contiguous():
+            raise ValueError("Wg must be a contiguous bf16 [32, H] tensor")
+    elif gate_x is not None or Wg is not None:
+        raise ValueError("ve, gate_x and Wg go together")
+    return B, T, H, D
+
+
+def forward(q, k, v, window: int = 0, ve=None, gate_x=None, Wg=None, rope_base: float = 10000.0,
+            eps: float = 1e-6, *, out=None, lse=None, with_lse: bool = True, workspace=None,
+            stream=None):
+    """One attention layer.  q, k, v (and ve) bf16 (B,T,H,D) CUDA tensors; gate_x (B,T,32);
+    Wg [32,H].  Returns (out bf16 (B,T,H,D), lse fp32 (B,H,T) or None).
+    ``workspace``: optional uint8 CUDA tensor of at least ``swa_attn_workspace_bytes`` bytes
+    (then nothing is allocated by the library)."""
+    import torch
+    B, T, H, D = _check_qkv(q, k, v, ve, gate_x, Wg)
+    if out is None:
+        out = torch.empty_like(q)
+    if with_lse and lse is None:
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    st = _stream_handle(stream)
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(out), _ptr(lse),
+            B, T, H, D, int(window), float(rope_base), float(eps))
+    if workspace is None:
+        rc = swa_attn_fwd(*args, st)
+    else:
+        rc = swa_attn_fwd_ws(*args, _ptr(workspace), workspace.numel() * workspace.element_size(), st)
+    if rc != SWA_OK:
+        raise SwaError(rc, "swa_attn_fwd")
+    return out, lse
+
+
+def check_device_status(stream=None) -> None:
+    """Synchronise and raise SwaError if a kernel recorded an error (e.g. a wait timeout)."""
+    rc, detail = swa_attn_last_device_status(_stream_handle(stream))
+    if rc != SWA_OK:
+        raise SwaError(rc, f"device status word 0x{detail:08x}")
+
+
+__all__ = [
+    "forward", "check_device_status", "SwaError", "LIB_PATH", "load",
+    "swa_attn_fwd", "swa_attn_fwd_ws", "swa_attn_workspace_bytes", "swa_attn_workspace_offset", "swa_attn_rope_table", "swa_attn_prologue",
+    "swa_attn_attention", "swa_attn_strerror", "swa_attn_last_device_status",
+    "swa_attn_set_wait_limit_ms", "swa_attn_version",
+]

@@ -1,0 +1,434 @@
+// swa_attn.cu -- host side of the C ABI declared in include/swa_attn.h: argument checks,
+// workspace management, TMA descriptors and the two kernel launches (prologue, attention).
+// All kernels are in this translation unit (ptx.cuh, prologue.cuh, attn_fwd.cuh).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "swa_attn.h"
+#include "attn_fwd.cuh"
+#include "prologue.cuh"
+
+namespace {
+
+constexpr int kVersion = 100;   // 0.1.0
+
+// ------------------------------------------------------------------ configuration knobs
+
+std::mutex g_cache_mu;                          // guards the per-device workspace cache
+std::atomic<unsigned long long> g_wait_limit_ns{0};   // 0 = not yet initialised
+
+unsigned long long wait_limit_ns() {
+    unsigned long long v = g_wait_limit_ns.load(std::memory_order_relaxed);
+    if (v != 0) return v;
+    long ms = 2000;
+    if (const char* e = std::getenv("SWA_WAIT_LIMIT_MS")) {
+        const long x = std::strtol(e, nullptr, 10);
+        if (x >= 1) ms = x;
+    }
+    unsigned long long expected = 0;
+    const unsigned long long want = (unsigned long long)ms * 1000000ull;
+    g_wait_limit_ns.compare_exchange_strong(expected, want);
+    return g_wait_limit_ns.load(std::memory_order_relaxed);
+}
+
+// ---------------------------------------------------------------------- argument checks
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct Shape {
+    int B, T, H, D;
+    long long n;          // B*T*H*D
+};
+
+int check_sizes(int B, int T, int H, int D, Shape* s) {
+    if (B < 1 || T < 1 || H < 1) return SWA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
+    const long long n = (long long)B * T * H * D;
+    if (n >= (1ll << 31)) return SWA_ERR_UNSUPPORTED;
+    if (B > 65535 || H > 65535) return SWA_ERR_UNSUPPORTED;   // grid y/z limits
+    *s = Shape{B, T, H, D, n};
+    return SWA_OK;
+}
+
+int check_layer_args(const void* q, const void* k, const void* v, const void* ve,
+                     const void* gate_x, const void* Wg, float rope_base, float eps) {
+    if (!q || !k || !v) return SWA_ERR_INVALID_ARG;
+    const int n_ve = (ve != nullptr) + (gate_x != nullptr) + (Wg != nullptr);
+    if (n_ve != 0 && n_ve != 3) return SWA_ERR_INVALID_ARG;
+    if (!std::isfinite(rope_base) || !(rope_base > 0.f)) return SWA_ERR_INVALID_ARG;
+    if (!std::isfinite(eps) || eps < 0.f) return SWA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return SWA_ERR_MISALIGNED;
+    if (n_ve == 3 && (!aligned(ve, 16) || !aligned(gate_x, 2) || !aligned(Wg, 2)))
+        return SWA_ERR_MISALIGNED;
+    return SWA_OK;
+}
+
+int check_outputs(const void* out, const float* lse) {
+    if (!out) return SWA_ERR_INVALID_ARG;
+    if (!aligned(out, 16) || (lse && !aligned(lse, 4))) return SWA_ERR_MISALIGNED;
+    return SWA_OK;
+}
+
+// ---------------------------------------------------------------------- workspace layout
+
+constexpr size_t kAlign = 1024;
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct WsLayout {
+    size_t qh, kh, vp, tab32, tab64, total;
+};
+
+// qhat | khat | v' (value-embedding layers only) | RoPE table fp32 pieces | RoPE table fp64,
+// each section 1024-byte aligned.
+WsLayout ws_layout(const Shape& s, bool has_ve) {
+    WsLayout w{};
+    const size_t tensor = round_up((size_t)s.n * 2);
+    const size_t pairs = (size_t)s.T * (s.D / 2);
+    w.qh = 0;
+    w.kh = w.qh + tensor;
+    w.vp = w.kh + tensor;
+    w.tab32 = w.vp + (has_ve ? tensor : 0);
+    w.tab64 = w.tab32 + round_up(pairs * sizeof(float4));
+    w.total = w.tab64 + round_up(pairs * sizeof(double2));
+    return w;
+}
+
+// ---------------------------------------------------------------------------- device
+
+int device_ready(int* dev_out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return SWA_ERR_NO_DEVICE;
+    }
+    static int checked[64] = {0};   // 0 unknown, 1 ok, 2 unsupported
+    if (dev < 0 || dev >= 64) return SWA_ERR_UNSUPPORTED;
+    if (checked[dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return SWA_ERR_CUDA;
+        }
+        checked[dev] = (major == 10 && minor == 0) ? 1 : 2;
+        if (checked[dev] == 1) {
+            if (cudaFuncSetAttribute(swa::attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     swa::FwdCfg<64>::SMEM_TOTAL) != cudaSuccess ||
+                cudaFuncSetAttribute(swa::attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     swa::FwdCfg<128>::SMEM_TOTAL) != cudaSuccess) {
+                cudaGetLastError();
+                checked[dev] = 0;
+                return SWA_ERR_CUDA;
+            }
+        }
+    }
+    *dev_out = dev;
+    return checked[dev] == 1 ? SWA_OK : SWA_ERR_UNSUPPORTED;
+}
+
+// ---------------------------------------------------------------------- TMA descriptors
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// A (B,T,H,D) bf16 tensor seen as 4-D {D, H, T, B}; box = 64 features x 1 head x 128 positions,
+// 128-byte swizzle (the canonical K-major / MN-major shared-memory atom of the tensor core).
+// Positions past T read as zeros.
+bool make_tile_map(CUtensorMap* m, const void* base, const Shape& s) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)s.D, (cuuint64_t)s.H, (cuuint64_t)s.T, (cuuint64_t)s.B};
+    const cuuint64_t strides[3] = {(cuuint64_t)s.D * 2, (cuuint64_t)s.H * s.D * 2,
+                                   (cuuint64_t)s.T * s.H * s.D * 2};
+    const cuuint32_t box[4] = {64, 1, 128, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------- launches
+
+int launch_rope_table(uint8_t* ws, const WsLayout& L, const Shape& s, float rope_base, cudaStream_t st) {
+    const long long n = (long long)s.T * (s.D / 2);
+    const int threads = 256;
+    const long long blocks = std::min<long long>((n + threads - 1) / threads, 148ll * 16);
+    swa::rope_table_kernel<<<(unsigned)blocks, threads, 0, st>>>(
+        reinterpret_cast<float4*>(ws + L.tab32), reinterpret_cast<double2*>(ws + L.tab64), s.T, s.D,
+        (double)rope_base);
+    return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+int launch_prologue(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                    const void* Wg, uint8_t* ws, const WsLayout& L, const Shape& s, float eps,
+                    cudaStream_t st) {
+    using bf = __nv_bfloat16;
+    const bool has_ve = ve != nullptr;
+    const long long n_rows = (long long)s.B * s.T * s.H;
+    const long long threads_total = n_rows * (s.D / 16);
+    const int threads = 256;
+    const long long blocks = std::min<long long>((threads_total + threads - 1) / threads, 148ll * 8);
+    const bf* qp = static_cast<const bf*>(q);
+    const bf* kp = static_cast<const bf*>(k);
+    const bf* vpi = static_cast<const bf*>(v);
+    const bf* vep = static_cast<const bf*>(ve);
+    const bf* gx = static_cast<const bf*>(gate_x);
+    const bf* wg = static_cast<const bf*>(Wg);
+    bf* qh = reinterpret_cast<bf*>(ws + L.qh);
+    bf* kh = reinterpret_cast<bf*>(ws + L.kh);
+    bf* vp = reinterpret_cast<bf*>(ws + L.vp);
+    const float4* t32 = reinterpret_cast<const float4*>(ws + L.tab32);
+    const double2* t64 = reinterpret_cast<const double2*>(ws + L.tab64);
+    const unsigned g = (unsigned)blocks;
+    if (s.D == 128) {
+        if (has_ve)
+            swa::prologue_kernel<128, true><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gx, wg, qh, kh, vp, t32, t64, n_rows, s.T, s.H, (double)eps);
+        else
+            swa::prologue_kernel<128, false><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gx, wg, qh, kh, vp, t32, t64, n_rows, s.T, s.H, (double)eps);
+    } else {
+        if (has_ve)
+            swa::prologue_kernel<64, true><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gx, wg, qh, kh, vp, t32, t64, n_rows, s.T, s.H, (double)eps);
+        else
+            swa::prologue_kernel<64, false><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gx, wg, qh, kh, vp, t32, t64, n_rows, s.T, s.H, (double)eps);
+    }
+    return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+int launch_attention(const void* v, bool has_ve, void* out, float* lse, const Shape& s, int window,
+                     uint8_t* ws, const WsLayout& L, cudaStream_t st) {
+    CUtensorMap tq, tk, tv;
+    const void* vsrc = has_ve ? static_cast<const void*>(ws + L.vp) : v;
+    if (!make_tile_map(&tq, ws + L.qh, s) || !make_tile_map(&tk, ws + L.kh, s) ||
+        !make_tile_map(&tv, vsrc, s))
+        return SWA_ERR_CUDA;
+    swa::FwdParams p{};
+    p.B = s.B;
+    p.T = s.T;
+    p.H = s.H;
+    p.W = (window <= 0 || window >= s.T) ? s.T : window;
+    const int n_qtiles = (s.T + 127) / 128;
+    p.n_pairs = (n_qtiles + 1) / 2;
+    const double log2e = 1.4426950408889634;
+    const double m0 = std::sqrt((double)s.D) * (1.0 + 1.0 / 64.0);
+    p.c1 = (float)(log2e / std::sqrt((double)s.D));
+    p.c2 = (float)(m0 * log2e);
+    p.m0 = (float)m0;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    p.wait_limit_ns = wait_limit_ns();
+    const dim3 grid((unsigned)p.n_pairs, (unsigned)s.H, (unsigned)s.B);
+    if (s.D == 128)
+        swa::attn_fwd_kernel<128><<<grid, swa::FwdCfg<128>::THREADS, swa::FwdCfg<128>::SMEM_TOTAL, st>>>(tq, tk, tv, p);
+    else
+        swa::attn_fwd_kernel<64><<<grid, swa::FwdCfg<64>::THREADS, swa::FwdCfg<64>::SMEM_TOTAL, st>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------- library-owned workspace
+
+struct DevCache {
+    void* ptr = nullptr;
+    size_t bytes = 0;
+    int tab_T = -1, tab_D = -1;
+    float tab_base = 0.f;
+    size_t tab_off = (size_t)-1;
+};
+DevCache g_cache[64];
+
+}  // namespace
+
+extern "C" {
+
+int swa_attn_version(void) { return kVersion; }
+
+const char* swa_attn_strerror(int status) {
+    switch (status) {
+        case SWA_OK: return "ok";
+        case SWA_ERR_INVALID_ARG: return "invalid argument";
+        case SWA_ERR_UNSUPPORTED: return "unsupported size, head dim or device";
+        case SWA_ERR_MISALIGNED: return "pointer not aligned (tensors and workspace need 16 bytes)";
+        case SWA_ERR_CUDA: return "CUDA call failed";
+        case SWA_ERR_TIMEOUT: return "a bounded wait inside a kernel expired";
+        case SWA_ERR_NO_MEMORY: return "workspace too small or allocation failed";
+        case SWA_ERR_NO_DEVICE: return "no CUDA device";
+        default: return "unknown status";
+    }
+}
+
+int swa_attn_set_wait_limit_ms(int ms) {
+    const unsigned long long prev = wait_limit_ns();
+    if (ms >= 1) g_wait_limit_ns.store((unsigned long long)ms * 1000000ull);
+    return (int)(prev / 1000000ull);
+}
+
+size_t swa_attn_workspace_offset(int B, int T, int H, int D, int has_ve, int section) {
+    Shape s;
+    if (check_sizes(B, T, H, D, &s) != SWA_OK) return (size_t)-1;
+    const WsLayout L = ws_layout(s, has_ve != 0);
+    switch (section) {
+        case SWA_WS_QHAT: return L.qh;
+        case SWA_WS_KHAT: return L.kh;
+        case SWA_WS_VPRIME: return has_ve ? L.vp : (size_t)-1;
+        case SWA_WS_ROPE_TABLE: return L.tab32;
+        default: return (size_t)-1;
+    }
+}
+
+size_t swa_attn_workspace_bytes(int B, int T, int H, int D, int has_ve) {
+    Shape s;
+    if (check_sizes(B, T, H, D, &s) != SWA_OK) return 0;
+    return ws_layout(s, has_ve != 0).total;
+}
+
+int swa_attn_rope_table(int B, int T, int H, int D, int has_ve, float rope_base, void* workspace,
+                        size_t ws_bytes, swa_stream_t stream) {
+    Shape s;
+    int rc = check_sizes(B, T, H, D, &s);
+    if (rc != SWA_OK) return rc;
+    if (!std::isfinite(rope_base) || !(rope_base > 0.f) || !workspace) return SWA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return SWA_ERR_MISALIGNED;
+    const WsLayout L = ws_layout(s, has_ve != 0);
+    if (ws_bytes < L.total) return SWA_ERR_NO_MEMORY;
+    int dev;
+    if ((rc = device_ready(&dev)) != SWA_OK) return rc;
+    return launch_rope_table(static_cast<uint8_t*>(workspace), L, s, rope_base,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+int swa_attn_prologue(const void* q, const void* k, const void* v, const void* ve,
+                      const void* gate_x, const void* Wg, int B, int T, int H, int D,
+                      float rope_base, float eps, void* workspace, size_t ws_bytes,
+                      swa_stream_t stream) {
+    Shape s;
+    int rc = check_sizes(B, T, H, D, &s);
+    if (rc == SWA_OK) rc = check_layer_args(q, k, v, ve, gate_x, Wg, rope_base, eps);
+    if (rc != SWA_OK) return rc;
+    if (!workspace) return SWA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return SWA_ERR_MISALIGNED;
+    const WsLayout L = ws_layout(s, ve != nullptr);
+    if (ws_bytes < L.total) return SWA_ERR_NO_MEMORY;
+    int dev;
+    if ((rc = device_ready(&dev)) != SWA_OK) return rc;
+    return launch_prologue(q, k, v, ve, gate_x, Wg, static_cast<uint8_t*>(workspace), L, s, eps,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+int swa_attn_attention(const void* v, int has_ve, void* out, float* lse, int B, int T, int H, int D,
+                       int window, void* workspace, size_t ws_bytes, swa_stream_t stream) {
+    Shape s;
+    int rc = check_sizes(B, T, H, D, &s);
+    if (rc != SWA_OK) return rc;
+    if (!workspace || (!has_ve && !v)) return SWA_ERR_INVALID_ARG;
+    if ((rc = check_outputs(out, lse)) != SWA_OK) return rc;
+    if (!aligned(workspace, 16) || (!has_ve && !aligned(v, 16))) return SWA_ERR_MISALIGNED;
+    const WsLayout L = ws_layout(s, has_ve != 0);
+    if (ws_bytes < L.total) return SWA_ERR_NO_MEMORY;
+    int dev;
+    if ((rc = device_ready(&dev)) != SWA_OK) return rc;
+    return launch_attention(v, has_ve != 0, out, lse, s, window, static_cast<uint8_t*>(workspace), L,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+int swa_attn_fwd_ws(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                    const void* Wg, void* out, float* lse, int B, int T, int H, int D, int window,
+                    float rope_base, float eps, void* workspace, size_t ws_bytes,
+                    swa_stream_t stream) {
+    Shape s;
+    int rc = check_sizes(B, T, H, D, &s);
+    if (rc == SWA_OK) rc = check_layer_args(q, k, v, ve, gate_x, Wg, rope_base, eps);
+    if (rc == SWA_OK) rc = check_outputs(out, lse);
+    if (rc != SWA_OK) return rc;
+    rc = swa_attn_rope_table(B, T, H, D, ve != nullptr, rope_base, workspace, ws_bytes, stream);
+    if (rc != SWA_OK) return rc;
+    rc = swa_attn_prologue(q, k, v, ve, gate_x, Wg, B, T, H, D, rope_base, eps, workspace, ws_bytes,
+                           stream);
+    if (rc != SWA_OK) return rc;
+    return swa_attn_attention(v, ve != nullptr, out, lse, B, T, H, D, window, workspace, ws_bytes,
+                              stream);
+}
+
+int swa_attn_fwd(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                 const void* Wg, void* out, float* lse, int B, int T, int H, int D, int window,
+                 float rope_base, float eps, swa_stream_t stream) {
+    Shape s;
+    int rc = check_sizes(B, T, H, D, &s);
+    if (rc == SWA_OK) rc = check_layer_args(q, k, v, ve, gate_x, Wg, rope_base, eps);
+    if (rc == SWA_OK) rc = check_outputs(out, lse);
+    if (rc != SWA_OK) return rc;
+    int dev;
+    if ((rc = device_ready(&dev)) != SWA_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const bool has_ve = ve != nullptr;
+    const WsLayout L = ws_layout(s, has_ve);
+
+    const unsigned long long limit = wait_limit_ns();   // read before taking the cache lock
+    (void)limit;
+    std::lock_guard<std::mutex> lk(g_cache_mu);
+    DevCache& c = g_cache[dev];
+    if (c.bytes < L.total) {
+        if (c.ptr) cudaFreeAsync(c.ptr, st);
+        c.ptr = nullptr;
+        c.bytes = 0;
+        c.tab_T = -1;
+        void* p = nullptr;
+        if (cudaMallocAsync(&p, L.total, st) != cudaSuccess) {
+            cudaGetLastError();
+            return SWA_ERR_NO_MEMORY;
+        }
+        c.ptr = p;
+        c.bytes = L.total;
+    }
+    uint8_t* ws = static_cast<uint8_t*>(c.ptr);
+    if (c.tab_T != T || c.tab_D != D || c.tab_base != rope_base || c.tab_off != L.tab32) {
+        if ((rc = launch_rope_table(ws, L, s, rope_base, st)) != SWA_OK) return rc;
+        c.tab_T = T;
+        c.tab_D = D;
+        c.tab_base = rope_base;
+        c.tab_off = L.tab32;
+    }
+    if ((rc = launch_prologue(q, k, v, ve, gate_x, Wg, ws, L, s, eps, st)) != SWA_OK) return rc;
+    return launch_attention(v, has_ve, out, lse, s, window, ws, L, st);
+}
+
+int swa_attn_last_device_status(swa_stream_t stream, unsigned int* detail) {
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) {
+        cudaGetLastError();
+        return SWA_ERR_CUDA;
+    }
+    unsigned int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, swa::g_status, sizeof word) != cudaSuccess ||
+        cudaMemcpyToSymbol(swa::g_status, &zero, sizeof zero) != cudaSuccess) {
+        cudaGetLastError();
+        return SWA_ERR_CUDA;
+    }
+    if (detail) *detail = word;
+    if (word == 0) return SWA_OK;
+    return (word & 0xffu) == swa::kErrTimeout ? SWA_ERR_TIMEOUT : SWA_ERR_CUDA;
+}
+
+}  // extern "C"

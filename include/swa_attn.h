@@ -1,0 +1,170 @@
+/*
+ * swa_attn.h -- C ABI of the B200 (sm_100a) causal sliding-window attention forward.
+ *
+ * The layer (one call = one attention layer of the nanochat / modded-NanoGPT speedrun model):
+ *
+ *   qhat = rms(rope(q)),  khat = rms(rope(k))
+ *        intelliparadigm "GPT-2 for $73", section 2.2 (q, k = norm(rope(q)), norm(rope(k)));
+ *        section 2.1 (parameter-free RMSNorm); kongchang speedrun explainer, "RoPE" paragraph.
+ *        rope: pairs (i, i + D/2), theta_i = rope_base^(-2i/D), position t = 0..T-1 rotates
+ *        (a, b) -> (a cos(t theta_i) - b sin(t theta_i), a sin(t theta_i) + b cos(t theta_i)).
+ *        rms:  x / sqrt(mean_D(x^2) + eps), no learned scale.
+ *   v'   = v + 2 sigmoid(gate_x[b,t,:] . Wg[:, h]) * ve        (value-embedding layers only)
+ *        PaperWeekly repost of the nanochat write-up, "Value Embeddings" paragraph.
+ *   out  = softmax(qhat khat^T / sqrt(D) + mask) v'
+ *        "Let's reproduce GPT-2 (124M)" notes, section 3 (scores, lower-triangular mask that
+ *        includes the diagonal, softmax over keys, weighted sum of values).
+ *        mask: key j is visible to query i iff 0 <= i - j < W, W = window (intelliparadigm
+ *        section 3.2: local windows of 1024 tokens, a full window of 2048 every fourth layer);
+ *        window <= 0 or window >= T means full causal.
+ *   lse  = ln sum_j exp(qhat_i . khat_j / sqrt(D)) over the visible keys (natural log).
+ *
+ * Layouts (all row-major, contiguous, no strides):
+ *   q, k, v, ve, out : bf16 (B, T, H, D)        -- the native layout (intelliparadigm 3.1)
+ *   gate_x           : bf16 (B, T, 32)          -- x[..., :32].contiguous()
+ *   Wg               : bf16 [32, H]             -- one gate per head, no bias
+ *   lse              : fp32 (B, H, T)
+ *
+ * Ownership: every pointer is a DEVICE pointer owned by the caller, except where stated.
+ * The library never frees a caller pointer and never writes q, k, v, ve, gate_x or Wg.
+ *
+ * Streams: calls are asynchronous on `stream` (NULL = the legacy default stream) and never
+ * synchronise the host, except swa_attn_last_device_status().
+ *
+ * Errors: a negative swa_status.  Arguments are validated before anything is enqueued; a
+ * rejected call has no effect.  Waits inside the kernels are bounded: if one expires, the
+ * kernel records SWA_ERR_TIMEOUT in a per-device status word and exits cleanly; read it with
+ * swa_attn_last_device_status().
+ */
+#ifndef SWA_ATTN_H_
+#define SWA_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SWA_API __attribute__((visibility("default")))
+#else
+#define SWA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* swa_stream_t;
+
+typedef enum swa_status {
+    SWA_OK = 0,
+    SWA_ERR_INVALID_ARG = -1,  /* null pointer, size < 1, bad eps / rope_base, ve/gate_x/Wg partly set */
+    SWA_ERR_UNSUPPORTED = -2,  /* D not in {64, 128}, sizes beyond int32 indexing, device not sm_100 */
+    SWA_ERR_MISALIGNED = -3,   /* a tensor pointer or the workspace is not 16-byte aligned */
+    SWA_ERR_CUDA = -4,         /* a CUDA runtime / driver call failed (launch, allocation by CUDA) */
+    SWA_ERR_TIMEOUT = -5,      /* a bounded wait inside a kernel expired (read via last_device_status) */
+    SWA_ERR_NO_MEMORY = -6,    /* workspace too small (swa_attn_fwd_ws) or allocation failed */
+    SWA_ERR_NO_DEVICE = -7     /* no CUDA device is visible */
+} swa_status;
+
+/*
+ * Full layer forward.  Steps: RoPE + RMS norm of q and k, gate + add of the value embedding,
+ * windowed causal attention, bf16 out and fp32 lse.
+ *
+ * q, k, v      bf16 (B,T,H,D), read only.
+ * ve, gate_x, Wg  value-embedding inputs; all three NULL for a layer without value embeddings,
+ *              otherwise all three set (else SWA_ERR_INVALID_ARG).
+ * out          bf16 (B,T,H,D), written.
+ * lse          fp32 (B,H,T), written; NULL skips it.
+ * B, T, H      >= 1;  D in {64, 128};  B*T*H*D < 2^31.
+ * window       keys visible to a query, counting itself; <= 0 or >= T is full causal.
+ * rope_base    > 0 and finite (10000 in the pages' models).
+ * eps          >= 0 and finite (1e-6 here).
+ * stream       CUDA stream (NULL = legacy default stream).
+ *
+ * Scratch: the library keeps one workspace per device (qhat, khat, v' and the RoPE table),
+ * grown on demand with stream-ordered allocation on `stream` and kept until the library is
+ * unloaded.  Calls that may overlap on different streams must use swa_attn_fwd_ws() with
+ * separate workspaces.
+ */
+SWA_API int swa_attn_fwd(const void* q, const void* k, const void* v,
+                 const void* ve, const void* gate_x, const void* Wg,
+                 void* out, float* lse,
+                 int B, int T, int H, int D, int window,
+                 float rope_base, float eps, swa_stream_t stream);
+
+/* Bytes of caller workspace swa_attn_fwd_ws() needs for these sizes (0 on invalid sizes). */
+SWA_API size_t swa_attn_workspace_bytes(int B, int T, int H, int D, int has_ve);
+
+/*
+ * Byte offset of one section of the workspace, for callers that read the prologue's results
+ * (e.g. to keep them for a backward pass) after swa_attn_prologue():
+ *   SWA_WS_QHAT, SWA_WS_KHAT   bf16 (B,T,H,D): rms(rope(q)), rms(rope(k)), each element the
+ *                              correctly rounded bf16 (nearest, ties to even) of its exact value;
+ *   SWA_WS_VPRIME              bf16 (B,T,H,D): v + 2 sigmoid(gate_x . Wg) ve, same rounding
+ *                              (value-embedding layers only);
+ *   SWA_WS_ROPE_TABLE          the RoPE table (internal format).
+ * Returns (size_t)-1 for invalid sizes or a section that does not exist.
+ */
+enum swa_ws_section { SWA_WS_QHAT = 0, SWA_WS_KHAT = 1, SWA_WS_VPRIME = 2, SWA_WS_ROPE_TABLE = 3 };
+SWA_API size_t swa_attn_workspace_offset(int B, int T, int H, int D, int has_ve, int section);
+
+/*
+ * Same as swa_attn_fwd() with caller-owned device scratch: `workspace` (16-byte aligned,
+ * at least swa_attn_workspace_bytes() bytes) holds qhat, khat, v' and the RoPE table, which
+ * is rebuilt on every call (one small extra kernel).  Nothing is allocated.  SWA_ERR_NO_MEMORY if ws_bytes is too small.
+ */
+SWA_API int swa_attn_fwd_ws(const void* q, const void* k, const void* v,
+                    const void* ve, const void* gate_x, const void* Wg,
+                    void* out, float* lse,
+                    int B, int T, int H, int D, int window,
+                    float rope_base, float eps,
+                    void* workspace, size_t ws_bytes, swa_stream_t stream);
+
+/*
+ * The steps of swa_attn_fwd_ws(), exposed for per-stage timing and tests.
+ *
+ * swa_attn_rope_table: fill the workspace's RoPE table, cos/sin(t * rope_base^(-2i/D)) for
+ *   t < T, i < D/2, evaluated in fp64 and stored as fp32.  It depends only on T, D and
+ *   rope_base, so a caller that keeps one workspace for many calls of the same T, D and base
+ *   builds it once (swa_attn_fwd does that with its own workspace).
+ * swa_attn_prologue: RoPE + RMS norm of q and k, gate + add of the value embedding, into the
+ *   workspace (same sizes and rules as swa_attn_fwd_ws).  Uses the table already in the
+ *   workspace; it does not rebuild it.
+ * swa_attn_attention: the windowed attention on a workspace that swa_attn_prologue() filled
+ *   for the same B, T, H, D and value-embedding setting (`v` is read directly when has_ve == 0).
+ */
+SWA_API int swa_attn_rope_table(int B, int T, int H, int D, int has_ve, float rope_base,
+                                void* workspace, size_t ws_bytes, swa_stream_t stream);
+
+SWA_API int swa_attn_prologue(const void* q, const void* k, const void* v,
+                      const void* ve, const void* gate_x, const void* Wg,
+                      int B, int T, int H, int D, float rope_base, float eps,
+                      void* workspace, size_t ws_bytes, swa_stream_t stream);
+
+SWA_API int swa_attn_attention(const void* v, int has_ve, void* out, float* lse,
+                       int B, int T, int H, int D, int window,
+                       void* workspace, size_t ws_bytes, swa_stream_t stream);
+
+/* Static description of a status code (never NULL). */
+SWA_API const char* swa_attn_strerror(int status);
+
+/*
+ * Synchronises `stream`, then returns and clears the current device's status word:
+ * SWA_OK, SWA_ERR_TIMEOUT (a bounded wait expired in some kernel since the last read) or
+ * SWA_ERR_CUDA (the stream reported an error).  If `detail` is not NULL it receives the raw
+ * word (bits 0-7 kind, 8-15 wait site, 16-31 block index).
+ */
+SWA_API int swa_attn_last_device_status(swa_stream_t stream, unsigned int* detail);
+
+/* Upper bound, in milliseconds, on any single wait inside the kernels (default 2000).
+ * Returns the previous value.  Values < 1 are ignored. */
+SWA_API int swa_attn_set_wait_limit_ms(int ms);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+SWA_API int swa_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWA_ATTN_H_ */

@@ -1,0 +1,106 @@
+"""The C-ABI library loads and exports every entry point its header declares, and rejects bad
+arguments before touching the device.  CPU only: every call below fails validation, so no
+kernel is launched and no pointer is dereferenced (the fake addresses are never used)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import causal_sliding_window_swa_b200 as swa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+A = 0x7f0000000000          # a 16-byte aligned fake address, never dereferenced
+
+
+def _declared_symbols():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if f.endswith(".h"):
+            txt = open(os.path.join(inc, f)).read()
+            names |= set(re.findall(r"SWA_API\s+[\w\s\*]+?\b(swa_\w+)\s*\(", txt))
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared_symbols()
+    assert len(names) >= 9
+    lib = ctypes.CDLL(swa.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_version_and_strerror():
+    assert swa.swa_attn_version() >= 100
+    for code in range(-7, 1):
+        assert swa.swa_attn_strerror(code)
+    assert swa.swa_attn_strerror(-99) == "unknown status"
+
+
+def test_workspace_bytes():
+    n = 16 * 2048 * 12 * 128
+    b0 = swa.swa_attn_workspace_bytes(16, 2048, 12, 128, 0)
+    b1 = swa.swa_attn_workspace_bytes(16, 2048, 12, 128, 1)
+    assert b0 >= 2 * 2 * n and b1 >= 3 * 2 * n and b1 - b0 == 2 * n
+    assert swa.swa_attn_workspace_bytes(0, 2048, 12, 128, 0) == 0
+    assert swa.swa_attn_workspace_bytes(1, 16, 1, 96, 0) == 0
+
+
+def _fwd(**kw):
+    args = dict(q=A, k=A, v=A, ve=None, gate_x=None, Wg=None, out=A, lse=A, B=1, T=16, H=1, D=64,
+                window=0, rope_base=1e4, eps=1e-6, stream=None)
+    args.update(kw)
+    return swa.swa_attn_fwd(*args.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), swa.SWA_ERR_INVALID_ARG),
+    (dict(T=0), swa.SWA_ERR_INVALID_ARG),
+    (dict(H=-1), swa.SWA_ERR_INVALID_ARG),
+    (dict(D=96), swa.SWA_ERR_UNSUPPORTED),
+    (dict(D=256), swa.SWA_ERR_UNSUPPORTED),
+    (dict(B=1 << 14, T=1 << 14, H=1, D=128), swa.SWA_ERR_UNSUPPORTED),   # 2^35 elements
+    (dict(q=None), swa.SWA_ERR_INVALID_ARG),
+    (dict(v=None), swa.SWA_ERR_INVALID_ARG),
+    (dict(out=None), swa.SWA_ERR_INVALID_ARG),
+    (dict(ve=A), swa.SWA_ERR_INVALID_ARG),                  # ve without gate_x / Wg
+    (dict(ve=A, gate_x=A), swa.SWA_ERR_INVALID_ARG),
+    (dict(eps=-1.0), swa.SWA_ERR_INVALID_ARG),
+    (dict(eps=float("nan")), swa.SWA_ERR_INVALID_ARG),
+    (dict(rope_base=0.0), swa.SWA_ERR_INVALID_ARG),
+    (dict(rope_base=float("inf")), swa.SWA_ERR_INVALID_ARG),
+    (dict(q=A + 2), swa.SWA_ERR_MISALIGNED),
+    (dict(k=A + 8), swa.SWA_ERR_MISALIGNED),
+    (dict(out=A + 4), swa.SWA_ERR_MISALIGNED),
+    (dict(lse=A + 2), swa.SWA_ERR_MISALIGNED),
+    (dict(ve=A + 2, gate_x=A, Wg=A), swa.SWA_ERR_MISALIGNED),
+])
+def test_fwd_rejects_bad_arguments(kw, code):
+    assert _fwd(**kw) == code
+
+
+def test_fwd_ws_rejects_small_or_misaligned_workspace():
+    need = swa.swa_attn_workspace_bytes(1, 16, 1, 64, 0)
+    base = (A, A, A, None, None, None, A, A, 1, 16, 1, 64, 0, 1e4, 1e-6)
+    assert swa.swa_attn_fwd_ws(*base, A, need - 1, None) == swa.SWA_ERR_NO_MEMORY
+    assert swa.swa_attn_fwd_ws(*base, A + 8, need, None) == swa.SWA_ERR_MISALIGNED
+    assert swa.swa_attn_fwd_ws(*base, None, need, None) == swa.SWA_ERR_INVALID_ARG
+
+
+def test_stage_entry_points_reject_bad_arguments():
+    need = swa.swa_attn_workspace_bytes(1, 16, 1, 64, 0)
+    assert swa.swa_attn_prologue(A, A, A, None, None, None, 1, 16, 1, 64, 1e4, 1e-6, A, need - 1, None) \
+        == swa.SWA_ERR_NO_MEMORY
+    assert swa.swa_attn_rope_table(1, 16, 1, 64, 0, 1e4, A, need - 1, None) == swa.SWA_ERR_NO_MEMORY
+    assert swa.swa_attn_rope_table(1, 16, 1, 64, 0, -1.0, A, need, None) == swa.SWA_ERR_INVALID_ARG
+    assert swa.swa_attn_attention(None, 0, A, A, 1, 16, 1, 64, 0, A, need, None) == swa.SWA_ERR_INVALID_ARG
+    assert swa.swa_attn_attention(A, 0, A, A, 1, 16, 1, 64, 0, A, need - 1, None) == swa.SWA_ERR_NO_MEMORY
+    assert swa.swa_attn_attention(A, 0, A, A, 1, 16, 1, 80, 0, A, need, None) == swa.SWA_ERR_UNSUPPORTED
+
+
+def test_wait_limit_setter():
+    prev = swa.swa_attn_set_wait_limit_ms(1500)
+    assert prev >= 1
+    assert swa.swa_attn_set_wait_limit_ms(0) == 1500      # ignored, returns current
+    swa.swa_attn_set_wait_limit_ms(prev)
