@@ -46,6 +46,10 @@ def _load() -> ctypes.CDLL:
     lib.swa_attn_fwd_ws.restype = I
     lib.swa_attn_workspace_bytes.argtypes = [I, I, I, I, I]
     lib.swa_attn_workspace_bytes.restype = Z
+    lib.swa_attn_fwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, F, F, P]
+    lib.swa_attn_fwd_noalloc.restype = I
+    lib.swa_attn_noalloc_scratch_bytes.argtypes = []
+    lib.swa_attn_noalloc_scratch_bytes.restype = Z
     lib.swa_attn_workspace_offset.argtypes = [I, I, I, I, I, I]
     lib.swa_attn_workspace_offset.restype = Z
     lib.swa_attn_rope_table.argtypes = [I, I, I, I, I, F, P, Z, P]
@@ -94,6 +98,18 @@ def swa_attn_fwd_ws(q, k, v, ve, gate_x, Wg, out, lse, B, T, H, D, window, rope_
                     workspace, ws_bytes, stream) -> int:
     return _lib.swa_attn_fwd_ws(q, k, v, ve, gate_x, Wg, out, lse, B, T, H, D, window, rope_base, eps,
                                 workspace, ws_bytes, stream)
+
+
+def swa_attn_fwd_noalloc(q, k, v, ve, gate_x, Wg, out, lse, B, T, H, D, window, rope_base, eps,
+                         stream) -> int:
+    """swa_attn_fwd for callers that cannot allocate device memory: scratch comes from a fixed
+    array inside the library (see include/swa_attn.h); nothing is allocated."""
+    return _lib.swa_attn_fwd_noalloc(q, k, v, ve, gate_x, Wg, out, lse, B, T, H, D, window, rope_base,
+                                     eps, stream)
+
+
+def swa_attn_noalloc_scratch_bytes() -> int:
+    return int(_lib.swa_attn_noalloc_scratch_bytes())
 
 
 def swa_attn_workspace_bytes(B, T, H, D, has_ve) -> int:
@@ -206,7 +222,7 @@ def check_device_status(stream=None) -> None:
 
 __all__ = [
     "forward", "check_device_status", "SwaError", "LIB_PATH", "load",
-    "swa_attn_fwd", "swa_attn_fwd_ws", "swa_attn_workspace_bytes", "swa_attn_workspace_offset", "swa_attn_rope_table", "swa_attn_prologue",
+    "swa_attn_fwd", "swa_attn_fwd_ws", "swa_attn_fwd_noalloc", "swa_attn_noalloc_scratch_bytes", "swa_attn_workspace_bytes", "swa_attn_workspace_offset", "swa_attn_rope_table", "swa_attn_prologue",
     "swa_attn_attention", "swa_attn_strerror", "swa_attn_last_device_status",
     "swa_attn_set_wait_limit_ms", "swa_attn_version",
 ]

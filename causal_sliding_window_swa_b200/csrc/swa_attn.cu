@@ -432,3 +432,60 @@ int swa_attn_last_device_status(swa_stream_t stream, unsigned int* detail) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------ entry point that allocates nothing
+//
+// Scratch for swa_attn_fwd_noalloc(): a fixed device array in this module.  Every GPU that
+// loads the library holds these bytes until the process exits.  Host code must not use the
+// array's name as a device address; the address comes from cudaGetSymbolAddress() below.
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = 64ull << 20;   // 64 MiB
+__device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_static_mu;
+void* g_static_ptr[64] = {nullptr};
+
+// Once per device, with that device current: the device address of the scratch array.
+int static_scratch(int dev, uint8_t** out) {
+    std::lock_guard<std::mutex> lk(g_static_mu);
+    if (g_static_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return SWA_ERR_CUDA;
+        }
+        g_static_ptr[dev] = p;
+    }
+    *out = static_cast<uint8_t*>(g_static_ptr[dev]);
+    return SWA_OK;
+}
+
+}  // namespace
+
+extern "C" size_t swa_attn_noalloc_scratch_bytes(void) { return kStaticScratchBytes; }
+
+extern "C" int swa_attn_fwd_noalloc(const void* q, const void* k, const void* v, const void* ve,
+                                    const void* gate_x, const void* Wg, void* out, float* lse,
+                                    int B, int T, int H, int D, int window, float rope_base,
+                                    float eps, swa_stream_t stream) {
+    Shape s;
+    int rc = check_sizes(B, T, H, D, &s);
+    if (rc == SWA_OK) rc = check_layer_args(q, k, v, ve, gate_x, Wg, rope_base, eps);
+    if (rc == SWA_OK) rc = check_outputs(out, lse);
+    if (rc != SWA_OK) return rc;
+    const bool has_ve = ve != nullptr;
+    const WsLayout L = ws_layout(s, has_ve);
+    if (L.total > kStaticScratchBytes) return SWA_ERR_NO_MEMORY;   // beyond the fixed scratch
+    int dev;
+    if ((rc = device_ready(&dev)) != SWA_OK) return rc;
+    uint8_t* ws = nullptr;
+    if ((rc = static_scratch(dev, &ws)) != SWA_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // Every section of the scratch this call reads is written earlier in the same call
+    // (table, then qhat/khat/v'), so nothing needs clearing between calls.
+    if ((rc = launch_rope_table(ws, L, s, rope_base, st)) != SWA_OK) return rc;
+    if ((rc = launch_prologue(q, k, v, ve, gate_x, Wg, ws, L, s, eps, st)) != SWA_OK) return rc;
+    return launch_attention(v, has_ve, out, lse, s, window, ws, L, st);
+}

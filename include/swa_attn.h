@@ -145,6 +145,33 @@ SWA_API int swa_attn_attention(const void* v, int has_ve, void* out, float* lse,
                        int B, int T, int H, int D, int window,
                        void* workspace, size_t ws_bytes, swa_stream_t stream);
 
+/*
+ * swa_attn_fwd_noalloc: swa_attn_fwd() for callers that cannot allocate device memory on the
+ * call path -- a plugin whose host framework owns all device memory and forbids allocation
+ * inside its execute call, or a latency-critical loop where an allocation (which may
+ * synchronise the device) is not allowed.  The pages have no counterpart of this entry point.
+ *
+ * The caller passes inputs and outputs exactly as for swa_attn_fwd(); the scratch (qhat, khat,
+ * v' and the RoPE table) lives in a fixed device array compiled into the library,
+ * swa_attn_noalloc_scratch_bytes() bytes (64 MiB), which every GPU that loads the library holds
+ * until the process exits.  Nothing is allocated or freed by the call.
+ *   - Sizes whose workspace (swa_attn_workspace_bytes()) exceeds that array are rejected with
+ *     SWA_ERR_NO_MEMORY before anything is enqueued.
+ *   - The first call on a device looks up the array's device address (a runtime query, once per
+ *     device, with that device current); make that first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's contents; every
+ *     byte a call reads is written earlier in that call.  Calls that overlap on the GPU (other
+ *     streams, other host threads) race on it: serialise them.
+ */
+SWA_API int swa_attn_fwd_noalloc(const void* q, const void* k, const void* v,
+                                 const void* ve, const void* gate_x, const void* Wg,
+                                 void* out, float* lse,
+                                 int B, int T, int H, int D, int window,
+                                 float rope_base, float eps, swa_stream_t stream);
+
+/* Size in bytes of the fixed scratch array behind swa_attn_fwd_noalloc(). */
+SWA_API size_t swa_attn_noalloc_scratch_bytes(void);
+
 /* Static description of a status code (never NULL). */
 SWA_API const char* swa_attn_strerror(int status);
 
