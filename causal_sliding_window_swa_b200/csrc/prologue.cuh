@@ -7,27 +7,33 @@
 // (a, b) -> (a cos - b sin, a sin + b cos).
 //
 // Rounding.  Every output element is the correctly rounded bf16 (nearest, ties to even) of the
-// exact value of its definition.  The common path runs in fp32 with a rigorous bound E on its
-// error; an element whose fp32 value lies within E of a bf16 rounding midpoint (about 1e-4 of
-// them) is recomputed in fp64.  So the tensor-core operands do not depend on how the arithmetic
-// was organised (an fp32-only pipeline flips the last bf16 bit of ~1e-4 of the elements, which
-// moves single attention scores by ~1e-3).
-//   rotation: cos and sin are stored as two 16-bit-significand pieces (hi + lo, remainder below
-//     2^-33), so a * hi and a * lo are exact in fp32 for a bf16 input a; ra = (a c_hi - b s_hi)
-//     + (a c_lo - b s_lo) carries an error of at most 2^-23 |ra| + 2^-32 (|a| + |b|).
-//   norm: the sum of squares is taken over the raw inputs (the rotation preserves it) in fp64,
-//     where each square is exact; r = 1 / sqrt(ss / D + eps) in fp64, rounded once to fp32.
-//   gate: the 32-term dot product and 2 sigmoid(z) in fp64, rounded once to fp32.
+// exact value of its definition, so the tensor-core operands do not depend on how the arithmetic
+// is organised (an fp32-only pipeline flips the last bf16 bit of ~1e-4 of the elements, which
+// moves single attention scores by ~1e-3).  The common path runs in fp32 with a proven error
+// bound; a pair whose fp32 result could round differently from the exact one is recomputed in
+// fp64 (a fraction of a percent of them).
+//   norm: r = 1 / sqrt(ss / D + eps) from the sum of squares of the raw inputs (the rotation
+//     preserves it) in fp64, where each square and the sum are exact; the inverse square root by
+//     two Newton-Raphson steps from the hardware estimate, then rounded once to fp32.
+//   rotation: cos and sin are stored as two pieces with 16-bit significands (remainder below
+//     2^-33), so every product a * piece is exact in fp32 for a bf16 input a; x = ra * r is then
+//     within 4 of its own ulps of the exact value whenever |x| >= 2^-8 r (|a| + |b|).  The test
+//     window is 8 ulps, and smaller |x| (partial cancellation) always take the fp64 path.
+//   gate: z = x[:32] . Wg[:, h] and g = 2 sigmoid(z) in fp64, split as g_hi + g_lo (fp32);
+//     v' = (v + g_hi ve) + g_lo ve with two fp32 roundings: within 1 ulp of the exact value
+//     unless |v'| < 2^-16 |g ve|.
 #pragma once
 
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace swa {
 
 // RoPE tables, one entry per (t, i):
 //   tab32[t*D/2 + i] = (c_hi, c_lo, s_hi, s_lo) fp32, each piece with a 16-bit significand;
-//   tab64[t*D/2 + i] = (cos, sin) fp64, read only when an element falls back to fp64.
+//   tab64[t*D/2 + i] = (cos, sin) fp64, read only by the fp64 path.
 __device__ __forceinline__ float round_sig16(double x) {
     // nearest float with at most 16 significant bits (8 low mantissa bits cleared)
     const float f = (float)x;
@@ -70,6 +76,21 @@ __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
     }
 }
 
+__device__ __forceinline__ uint2 ldg_stream8(const void* p) {
+    uint2 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
+                 : "=r"(r.x), "=r"(r.y)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void unpack4(const uint2& u, float (&f)[4]) {
+    f[0] = __uint_as_float(u.x << 16);
+    f[1] = __uint_as_float(u.x & 0xffff0000u);
+    f[2] = __uint_as_float(u.y << 16);
+    f[3] = __uint_as_float(u.y & 0xffff0000u);
+}
+
 __device__ __forceinline__ uint16_t bf16_rn_bits(float x) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
@@ -78,120 +99,135 @@ __device__ __forceinline__ uint16_t bf16_rn_bits(double x) {
     return __bfloat16_as_ushort(__double2bfloat16(x));
 }
 
-__device__ __forceinline__ uint4 pack8_bits(const uint16_t (&o)[8]) {
-    uint4 r;
-    r.x = o[0] | ((uint32_t)o[1] << 16);
-    r.y = o[2] | ((uint32_t)o[3] << 16);
-    r.z = o[4] | ((uint32_t)o[5] << 16);
-    r.w = o[6] | ((uint32_t)o[7] << 16);
+// 1 / sqrt(y) for y > 0 in fp64: the hardware fp32 estimate refined by two Newton-Raphson steps
+// for the inverse square root, r <- r (3 - y r^2) / 2 (each step squares the relative error:
+// ~2^-22 -> 2^-44 -> below 2^-52).
+__device__ __forceinline__ double rsqrt_newton(double y) {
+    double r = (double)rsqrtf((float)y);
+    r = r * fma(-0.5 * y, r * r, 1.5);
+    r = r * fma(-0.5 * y, r * r, 1.5);
     return r;
 }
 
-// True if |x - m| <= E for the bf16 rounding midpoint m just above |x|'s bf16 truncation: the
-// only midpoint within reach of an error much smaller than half a bf16 ulp.
-__device__ __forceinline__ bool near_bf16_midpoint(float x, float E) {
-    const float m = __uint_as_float((__float_as_uint(x) & 0xffff0000u) | 0x8000u);
-    return fabsf(x - m) <= E;
+// True if the low 16 bits of x are within 8 of 0x8000: a bf16 rounding midpoint lies within
+// [-8, +7] fp32 ulps of x.
+__device__ __forceinline__ bool near_midpoint_8ulp(float x) {
+    return ((__float_as_uint(x) + 8u - 0x8000u) & 0xfff0u) == 0u;
 }
 
-// One group of D/16 consecutive threads handles one (b, t, h) row of D elements.  Thread c of
-// the group owns elements [8c, 8c+8) and their rotation partners [8c + D/2, 8c + D/2 + 8):
-// two 16-byte loads per tensor; the sum of squares is reduced over the group with shuffles.
+// True if a bf16 rounding midpoint lies within [-16, +15] fp32 ulps of x.
+__device__ __forceinline__ bool near_midpoint_16ulp(float x) {
+    return ((__float_as_uint(x) + 16u - 0x8000u) & 0xffe0u) == 0u;
+}
+
+// One group of D/8 consecutive threads handles one (b, t, h) row.  Thread c of the group owns
+// pairs i in [4c, 4c+4): elements i (in `lo_raw`) and i + D/2 (in `hi_raw`).
 template <int D>
-__device__ __forceinline__ void rope_rms_row(const __nv_bfloat16* __restrict__ src,
-                                             __nv_bfloat16* __restrict__ dst, long long off,
-                                             int i0, const float4 (&cs)[8],
-                                             const double2* __restrict__ tab64_row, double eps,
-                                             bool valid) {
-    constexpr int HALF = D / 2;
-    constexpr int TPR = D / 16;
-    float a[8], b[8];
-    if (valid) {
-        unpack8(ldg_stream(src + off + i0), a);
-        unpack8(ldg_stream(src + off + HALF + i0), b);
-    } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) a[e] = b[e] = 0.f;
-    }
+__device__ __forceinline__ void rope_rms_pairs4(const uint2& lo_raw, const uint2& hi_raw,
+                                                const float4 (&cs)[4],
+                                                const double2* __restrict__ tab64, double eps,
+                                                uint2& out_lo, uint2& out_hi) {
+    constexpr int TPR = D / 8;
+    float a[4], b[4];
+    unpack4(lo_raw, a);
+    unpack4(hi_raw, b);
     double ss = 0.0;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const double ad = (double)a[e], bd = (double)b[e];
-        ss = fma(ad, ad, ss);
-        ss = fma(bd, bd, ss);
+    for (int e = 0; e < 4; ++e) {
+        ss = fma((double)a[e], (double)a[e], ss);
+        ss = fma((double)b[e], (double)b[e], ss);
     }
 #pragma unroll
     for (int m = TPR / 2; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-    const double r64 = 1.0 / sqrt(ss / (double)D + eps);
+    const double r64 = rsqrt_newton(ss * (1.0 / (double)D) + eps);
     const float r = (float)r64;
-
-    uint16_t oa[8], ob[8];
-    bool slow = false;
+    uint32_t wa[2], wb[2];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const float4 w = cs[e];   // (c_hi, c_lo, s_hi, s_lo)
-        const float ra = fmaf(a[e], w.x, -(b[e] * w.z)) + fmaf(a[e], w.y, -(b[e] * w.w));
-        const float rb = fmaf(a[e], w.z, b[e] * w.x) + fmaf(a[e], w.w, b[e] * w.y);
-        const float xa = ra * r, xb = rb * r;
-        const float K = r * (fabsf(a[e]) + fabsf(b[e])) * 0x1p-31f;
-        slow |= near_bf16_midpoint(xa, fmaf(fabsf(xa), 0x1p-21f, K));
-        slow |= near_bf16_midpoint(xb, fmaf(fabsf(xb), 0x1p-21f, K));
-        oa[e] = bf16_rn_bits(xa);
-        ob[e] = bf16_rn_bits(xb);
-    }
-    if (slow) {
-        // Rare: recompute this thread's elements in fp64 and round once.
+    for (int e = 0; e < 4; e += 2) {
+        float xa[2], xb[2];
+        bool slow = false;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const double2 w = tab64_row[i0 + e];
-            const double ad = (double)a[e], bd = (double)b[e];
-            oa[e] = bf16_rn_bits((ad * w.x - bd * w.y) * r64);
-            ob[e] = bf16_rn_bits((ad * w.y + bd * w.x) * r64);
+        for (int u = 0; u < 2; ++u) {
+            const float4 w = cs[e + u];   // (c_hi, c_lo, s_hi, s_lo)
+            const float A = a[e + u], Bv = b[e + u];
+            // products with a 16-bit piece are exact; one rounding per fma, one per add
+            const float ra = fmaf(A, w.x, -(Bv * w.z)) + fmaf(A, w.y, -(Bv * w.w));
+            const float rb = fmaf(A, w.z, Bv * w.x) + fmaf(A, w.w, Bv * w.y);
+            xa[u] = ra * r;
+            xb[u] = rb * r;
+            const float small = r * (fabsf(A) + fabsf(Bv)) * 0x1p-8f;
+            slow |= near_midpoint_8ulp(xa[u]) | near_midpoint_8ulp(xb[u]) |
+                    (fabsf(xa[u]) < small) | (fabsf(xb[u]) < small);
+        }
+        wa[e >> 1] = pack_bf16x2(xa[0], xa[1]);
+        wb[e >> 1] = pack_bf16x2(xb[0], xb[1]);
+        if (slow) {
+            // Rare: these two pairs in fp64, rounded once.
+            uint16_t oa[2], ob[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const double2 w = tab64[e + u];
+                const double A = (double)a[e + u], Bv = (double)b[e + u];
+                oa[u] = bf16_rn_bits((A * w.x - Bv * w.y) * r64);
+                ob[u] = bf16_rn_bits((A * w.y + Bv * w.x) * r64);
+            }
+            wa[e >> 1] = oa[0] | ((uint32_t)oa[1] << 16);
+            wb[e >> 1] = ob[0] | ((uint32_t)ob[1] << 16);
         }
     }
-    if (valid) {
-        *reinterpret_cast<uint4*>(dst + off + i0) = pack8_bits(oa);
-        *reinterpret_cast<uint4*>(dst + off + HALF + i0) = pack8_bits(ob);
-    }
+    out_lo = make_uint2(wa[0], wa[1]);
+    out_hi = make_uint2(wb[0], wb[1]);
 }
 
-// v' = v + g ve for 8 elements: fp32 fma with error at most 2^-23 (|g ve| + |v'|); fp64 when
-// close to a bf16 rounding midpoint.
-__device__ __forceinline__ uint4 gated_add8(const uint4& vw, const uint4& ew, float gf, double g64) {
-    float v[8], e8[8];
-    unpack8(vw, v);
-    unpack8(ew, e8);
-    uint16_t o[8];
+// v' = v + g ve for 4 elements: (v + g_hi ve) + g_lo ve in fp32 (two roundings, within 1 ulp
+// unless |v'| < 2^-16 |g ve|); fp64 when that could cross a bf16 rounding midpoint.
+__device__ __forceinline__ uint2 gated_add4(const uint2& vw, const uint2& ew, float g_hi, float g_lo,
+                                            double g64) {
+    float v[4], e4[4];
+    unpack4(vw, v);
+    unpack4(ew, e4);
+    uint32_t w[2];
     bool slow = false;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const float x = fmaf(gf, e8[e], v[e]);
-        slow |= near_bf16_midpoint(x, (fabsf(gf * e8[e]) + fabsf(x)) * 0x1p-22f);
-        o[e] = bf16_rn_bits(x);
+    for (int e = 0; e < 4; e += 2) {
+        float x[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            x[u] = fmaf(g_lo, e4[e + u], fmaf(g_hi, e4[e + u], v[e + u]));
+            slow |= near_midpoint_8ulp(x[u]) | (fabsf(x[u]) < fabsf(g_hi * e4[e + u]) * 0x1p-16f);
+        }
+        w[e >> 1] = pack_bf16x2(x[0], x[1]);
     }
     if (slow) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = bf16_rn_bits(fma(g64, (double)e8[e], (double)v[e]));
+        for (int e = 0; e < 4; e += 2)
+            w[e >> 1] = (uint32_t)bf16_rn_bits(fma(g64, (double)e4[e], (double)v[e])) |
+                        ((uint32_t)bf16_rn_bits(fma(g64, (double)e4[e + 1], (double)v[e + 1])) << 16);
     }
-    return pack8_bits(o);
+    return make_uint2(w[0], w[1]);
 }
 
 template <int D, bool HAS_VE>
-__global__ void __launch_bounds__(256) prologue_kernel(
+__global__ void __launch_bounds__(256, 3) prologue_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
     const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ ve,
     const __nv_bfloat16* __restrict__ gate_x, const __nv_bfloat16* __restrict__ Wg,
     __nv_bfloat16* __restrict__ qh, __nv_bfloat16* __restrict__ kh, __nv_bfloat16* __restrict__ vp,
-    const float4* __restrict__ tab32, const double2* __restrict__ tab64, long long n_rows, int T,
-    int H, double eps) {
-    constexpr int TPR = D / 16;          // threads per row (8 or 4); divides 32
+    const float4* __restrict__ tab32, const double2* __restrict__ tab64, int* __restrict__ sched,
+    long long n_rows, int T, int H, double eps) {
+    constexpr int TPR = D / 8;           // threads per row (16 or 8); divides 32
     constexpr int HALF = D / 2;
-    constexpr int GCH = 32 / TPR;        // gate channels per thread
+    constexpr int GCH = 32 / TPR;        // gate channels per thread (2 or 4)
     const long long gtid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
     const long long stride = (long long)gridDim.x * blockDim.x;
-    // Every thread of a warp runs the same number of iterations, so the shuffles below always
-    // see the full warp; rows past the end are computed on zeros and not stored.
+    // Every thread of a warp runs the same number of iterations, so the shuffles always see the
+    // full warp; rows past the end are computed on zeros and not stored.
     const long long n_iter = (n_rows * TPR + stride - 1) / stride;
+    // The attention kernel that follows takes its work items from this counter.
+    if (gtid == 0) {
+        sched[0] = 0;
+        sched[1] = 0;
+    }
     for (long long it = 0; it < n_iter; ++it) {
         const long long tid = gtid + it * stride;
         const long long row = tid / TPR;          // (b*T + t)*H + h
@@ -201,18 +237,42 @@ __global__ void __launch_bounds__(256) prologue_kernel(
         const int h = (int)(rr % H);
         const long long bt = rr / H;
         const int t = (int)(bt % T);
-        const int i0 = 8 * c;
+        const int i0 = 4 * c;
         const long long off = rr * D;
 
-        float4 cs[8];
+        // Every load of this row chunk is issued before any arithmetic.
+        uint2 raw[8];
+        if (valid) {
+            raw[0] = ldg_stream8(q + off + i0);
+            raw[1] = ldg_stream8(q + off + HALF + i0);
+            raw[2] = ldg_stream8(k + off + i0);
+            raw[3] = ldg_stream8(k + off + HALF + i0);
+            if (HAS_VE) {
+                raw[4] = ldg_stream8(v + off + i0);
+                raw[5] = ldg_stream8(v + off + HALF + i0);
+                raw[6] = ldg_stream8(ve + off + i0);
+                raw[7] = ldg_stream8(ve + off + HALF + i0);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) raw[e] = make_uint2(0u, 0u);
+        }
+        float4 cs[4];
         {
             const float4* tp = tab32 + (long long)t * HALF + i0;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) cs[e] = __ldg(tp + e);
+            for (int e = 0; e < 4; ++e) cs[e] = __ldg(tp + e);
         }
-        const double2* t64 = tab64 + (long long)t * HALF;
-        rope_rms_row<D>(q, qh, off, i0, cs, t64, eps, valid);
-        rope_rms_row<D>(k, kh, off, i0, cs, t64, eps, valid);
+        const double2* t64 = tab64 + (long long)t * HALF + i0;
+        uint2 o0, o1, o2, o3;
+        rope_rms_pairs4<D>(raw[0], raw[1], cs, t64, eps, o0, o1);
+        rope_rms_pairs4<D>(raw[2], raw[3], cs, t64, eps, o2, o3);
+        if (valid) {
+            *reinterpret_cast<uint2*>(qh + off + i0) = o0;
+            *reinterpret_cast<uint2*>(qh + off + HALF + i0) = o1;
+            *reinterpret_cast<uint2*>(kh + off + i0) = o2;
+            *reinterpret_cast<uint2*>(kh + off + HALF + i0) = o3;
+        }
 
         if constexpr (HAS_VE) {
             double z = 0.0;
@@ -226,13 +286,11 @@ __global__ void __launch_bounds__(256) prologue_kernel(
 #pragma unroll
             for (int m = TPR / 2; m >= 1; m >>= 1) z += __shfl_xor_sync(0xffffffffu, z, m);
             const double g64 = 2.0 / (1.0 + exp(-z));
-            const float gf = (float)g64;
+            const float g_hi = (float)g64;
+            const float g_lo = (float)(g64 - (double)g_hi);
             if (valid) {
-                const uint4 oa = gated_add8(ldg_stream(v + off + i0), ldg_stream(ve + off + i0), gf, g64);
-                const uint4 ob = gated_add8(ldg_stream(v + off + HALF + i0),
-                                            ldg_stream(ve + off + HALF + i0), gf, g64);
-                *reinterpret_cast<uint4*>(vp + off + i0) = oa;
-                *reinterpret_cast<uint4*>(vp + off + HALF + i0) = ob;
+                *reinterpret_cast<uint2*>(vp + off + i0) = gated_add4(raw[4], raw[6], g_hi, g_lo, g64);
+                *reinterpret_cast<uint2*>(vp + off + HALF + i0) = gated_add4(raw[5], raw[7], g_hi, g_lo, g64);
             }
         }
     }

@@ -82,11 +82,11 @@ constexpr size_t kAlign = 1024;
 size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct WsLayout {
-    size_t qh, kh, vp, tab32, tab64, total;
+    size_t qh, kh, vp, tab32, tab64, sched, total;
 };
 
-// qhat | khat | v' (value-embedding layers only) | RoPE table fp32 pieces | RoPE table fp64,
-// each section 1024-byte aligned.
+// qhat | khat | v' (value-embedding layers only) | RoPE table fp32 pieces | RoPE table fp64 |
+// attention scheduler counters, each section 1024-byte aligned.
 WsLayout ws_layout(const Shape& s, bool has_ve) {
     WsLayout w{};
     const size_t tensor = round_up((size_t)s.n * 2);
@@ -96,11 +96,14 @@ WsLayout ws_layout(const Shape& s, bool has_ve) {
     w.vp = w.kh + tensor;
     w.tab32 = w.vp + (has_ve ? tensor : 0);
     w.tab64 = w.tab32 + round_up(pairs * sizeof(float4));
-    w.total = w.tab64 + round_up(pairs * sizeof(double2));
+    w.sched = w.tab64 + round_up(pairs * sizeof(double2));
+    w.total = w.sched + kAlign;
     return w;
 }
 
 // ---------------------------------------------------------------------------- device
+
+int g_num_sms[64] = {0};
 
 int device_ready(int* dev_out) {
     int dev = -1;
@@ -118,6 +121,11 @@ int device_ready(int* dev_out) {
             return SWA_ERR_CUDA;
         }
         checked[dev] = (major == 10 && minor == 0) ? 1 : 2;
+        if (cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            checked[dev] = 0;
+            return SWA_ERR_CUDA;
+        }
         if (checked[dev] == 1) {
             if (cudaFuncSetAttribute(swa::attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      swa::FwdCfg<64>::SMEM_TOTAL) != cudaSuccess ||
@@ -189,9 +197,9 @@ int launch_prologue(const void* q, const void* k, const void* v, const void* ve,
     using bf = __nv_bfloat16;
     const bool has_ve = ve != nullptr;
     const long long n_rows = (long long)s.B * s.T * s.H;
-    const long long threads_total = n_rows * (s.D / 16);
+    const long long threads_total = n_rows * (s.D / 8);
     const int threads = 256;
-    const long long blocks = std::min<long long>((threads_total + threads - 1) / threads, 148ll * 8);
+    const long long blocks = std::min<long long>((threads_total + threads - 1) / threads, 148ll * 3 * 4);
     const bf* qp = static_cast<const bf*>(q);
     const bf* kp = static_cast<const bf*>(k);
     const bf* vpi = static_cast<const bf*>(v);
@@ -203,23 +211,24 @@ int launch_prologue(const void* q, const void* k, const void* v, const void* ve,
     bf* vp = reinterpret_cast<bf*>(ws + L.vp);
     const float4* t32 = reinterpret_cast<const float4*>(ws + L.tab32);
     const double2* t64 = reinterpret_cast<const double2*>(ws + L.tab64);
+    int* sched = reinterpret_cast<int*>(ws + L.sched);
     const unsigned g = (unsigned)blocks;
     if (s.D == 128) {
         if (has_ve)
-            swa::prologue_kernel<128, true><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gx, wg, qh, kh, vp, t32, t64, n_rows, s.T, s.H, (double)eps);
+            swa::prologue_kernel<128, true><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gx, wg, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, (double)eps);
         else
-            swa::prologue_kernel<128, false><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gx, wg, qh, kh, vp, t32, t64, n_rows, s.T, s.H, (double)eps);
+            swa::prologue_kernel<128, false><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gx, wg, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, (double)eps);
     } else {
         if (has_ve)
-            swa::prologue_kernel<64, true><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gx, wg, qh, kh, vp, t32, t64, n_rows, s.T, s.H, (double)eps);
+            swa::prologue_kernel<64, true><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gx, wg, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, (double)eps);
         else
-            swa::prologue_kernel<64, false><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gx, wg, qh, kh, vp, t32, t64, n_rows, s.T, s.H, (double)eps);
+            swa::prologue_kernel<64, false><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gx, wg, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, (double)eps);
     }
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
-int launch_attention(const void* v, bool has_ve, void* out, float* lse, const Shape& s, int window,
-                     uint8_t* ws, const WsLayout& L, cudaStream_t st) {
+int launch_attention(int dev, const void* v, bool has_ve, void* out, float* lse, const Shape& s,
+                     int window, uint8_t* ws, const WsLayout& L, cudaStream_t st) {
     CUtensorMap tq, tk, tv;
     const void* vsrc = has_ve ? static_cast<const void*>(ws + L.vp) : v;
     if (!make_tile_map(&tq, ws + L.qh, s) || !make_tile_map(&tk, ws + L.kh, s) ||
@@ -232,6 +241,10 @@ int launch_attention(const void* v, bool has_ve, void* out, float* lse, const Sh
     p.W = (window <= 0 || window >= s.T) ? s.T : window;
     const int n_qtiles = (s.T + 127) / 128;
     p.n_pairs = (n_qtiles + 1) / 2;
+    p.n_items = p.n_pairs * s.H * s.B;
+    // Scheduling chunks of (b, h) slices whose K/V (about 4 T D bytes each) fit in ~40 MB of L2.
+    const long long slice_bytes = 4ll * s.T * s.D;
+    p.chunk_bh = (int)std::max<long long>(1, std::min<long long>((40ll << 20) / slice_bytes, (long long)s.B * s.H));
     const double log2e = 1.4426950408889634;
     const double m0 = std::sqrt((double)s.D) * (1.0 + 1.0 / 64.0);
     p.c1 = (float)(log2e / std::sqrt((double)s.D));
@@ -239,8 +252,9 @@ int launch_attention(const void* v, bool has_ve, void* out, float* lse, const Sh
     p.m0 = (float)m0;
     p.out = static_cast<__nv_bfloat16*>(out);
     p.lse = lse;
+    p.sched = reinterpret_cast<int*>(ws + L.sched);
     p.wait_limit_ns = wait_limit_ns();
-    const dim3 grid((unsigned)p.n_pairs, (unsigned)s.H, (unsigned)s.B);
+    const dim3 grid((unsigned)std::min(p.n_items, g_num_sms[dev]));
     if (s.D == 128)
         swa::attn_fwd_kernel<128><<<grid, swa::FwdCfg<128>::THREADS, swa::FwdCfg<128>::SMEM_TOTAL, st>>>(tq, tk, tv, p);
     else
@@ -349,7 +363,7 @@ int swa_attn_attention(const void* v, int has_ve, void* out, float* lse, int B, 
     if (ws_bytes < L.total) return SWA_ERR_NO_MEMORY;
     int dev;
     if ((rc = device_ready(&dev)) != SWA_OK) return rc;
-    return launch_attention(v, has_ve != 0, out, lse, s, window, static_cast<uint8_t*>(workspace), L,
+    return launch_attention(dev, v, has_ve != 0, out, lse, s, window, static_cast<uint8_t*>(workspace), L,
                             reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -411,7 +425,7 @@ int swa_attn_fwd(const void* q, const void* k, const void* v, const void* ve, co
         c.tab_off = L.tab32;
     }
     if ((rc = launch_prologue(q, k, v, ve, gate_x, Wg, ws, L, s, eps, st)) != SWA_OK) return rc;
-    return launch_attention(v, has_ve, out, lse, s, window, ws, L, st);
+    return launch_attention(dev, v, has_ve, out, lse, s, window, ws, L, st);
 }
 
 int swa_attn_last_device_status(swa_stream_t stream, unsigned int* detail) {
@@ -487,5 +501,5 @@ extern "C" int swa_attn_fwd_noalloc(const void* q, const void* k, const void* v,
     // (table, then qhat/khat/v'), so nothing needs clearing between calls.
     if ((rc = launch_rope_table(ws, L, s, rope_base, st)) != SWA_OK) return rc;
     if ((rc = launch_prologue(q, k, v, ve, gate_x, Wg, ws, L, s, eps, st)) != SWA_OK) return rc;
-    return launch_attention(v, has_ve, out, lse, s, window, ws, L, st);
+    return launch_attention(dev, v, has_ve, out, lse, s, window, ws, L, st);
 }
