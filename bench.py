@@ -383,7 +383,7 @@ def run_ours(args, s0):
                               "frac": prologue_bytes(s) / (pro_ms_max * 1e-3) / 1e9 / float(peaks["hbm_gbs"])},
         "e2e": {"value": world * fl / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": 2 * K,
+        "gpu_launches": (3 if s.ve else 2) * K,   # (gate,) prologue, attention
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -397,7 +397,7 @@ def run_ours(args, s0):
 
 
 def prologue_bytes(s: workloads.LayerShape) -> float:
-    """Algorithmic bytes of the prologue: read q, k, v (+ ve, gate_x, Wg), write qhat, khat
+    """Algorithmic bytes of the prologue stage: read q, k, v (+ ve, gate_x, Wg), write qhat, khat
     (+ v')."""
     n = s.n_elems * 2
     b = 2 * n + 2 * n           # q, k in; qhat, khat out

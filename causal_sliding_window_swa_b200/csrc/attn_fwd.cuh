@@ -11,10 +11,10 @@
 // are never loaded.  The kernel is persistent: one CTA per SM takes items from a global counter
 // (ordered in L2-sized chunks of (b, h) slices, heaviest first inside a chunk) until none is left.
 // Warp roles (320 threads):
-//   warps 0-3  softmax + epilogue for query tile 0 (thread r owns row r: TMEM lane r)
-//   warps 4-7  softmax + epilogue for query tile 1
-//   warp  8    scheduler + TMA producer: Q tiles, then K_j, V_j through an NS-stage mbarrier ring
-//   warp  9    TMEM allocator and the single thread that issues tcgen05.mma
+//   warp  0    TMEM allocator and the single thread that issues tcgen05.mma
+//   warp  1    scheduler + TMA producer: Q tiles, then K_j, V_j through an NS-stage mbarrier ring
+//   warps 2-5  softmax + epilogue for query tile 0 (warp w owns rows 32 (w % 4) .. +31: TMEM lanes)
+//   warps 6-9  softmax + epilogue for query tile 1
 // Tensor memory (512 columns): S0 | S1 (128 fp32 columns each) | O0 | O1 (D columns each).
 // P (bf16) is written over the first 64 columns of its S buffer and fed to the PV product
 // straight from tensor memory.
@@ -212,9 +212,14 @@ __global__ void __maxnreg__(168)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    constexpr uint32_t kItemConsumers = 1 + 8;  // the MMA thread and lane 0 of each softmax warp
+    // The MMA thread gets the lowest warp id: among ready warps the issue logic tends to favour
+    // lower ids, and the tensor core idles whenever this thread waits for an issue slot.
+    constexpr int kMmaWarp = 0;
+    constexpr int kProducerWarp = 1;
+    constexpr int kSoftmaxWarp0 = 2;             // warps 2-5: tile 0, warps 6-9: tile 1
+    constexpr uint32_t kItemConsumers = 1 + 8;   // the MMA thread and lane 0 of each softmax warp
 
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 32) {
         for (int g = 0; g < 2; ++g) {
             mbar_init(smem_u32(b_qfull + g), 1);
             mbar_init(smem_u32(b_qempty + g), 1);
@@ -232,11 +237,11 @@ __global__ void __maxnreg__(168)
         }
         fence_barrier_init();
     }
-    if (warp == 9) {
+    if (warp == kMmaWarp) {
         tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
         tmem_relinquish();
     }
-    if (warp == 8 && lane == 0) {
+    if (warp == kProducerWarp && lane == 0) {
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
@@ -247,7 +252,7 @@ __global__ void __maxnreg__(168)
     const uint32_t tmem = *tmem_slot;
     const unsigned long long lim = p.wait_limit_ns;
 
-    if (warp == 8) {
+    if (warp == kProducerWarp) {
         // ========================= scheduler + TMA producer =========================
         if (lane == 0) {
             uint32_t stage = 0, phase = 0;
@@ -256,6 +261,33 @@ __global__ void __maxnreg__(168)
             for (int s = 0; s < C::NS; ++s) filled[s] = false, filled_phase[s] = 0;
             uint32_t q_uses[2] = {0u, 0u};
             bool ok = true;
+            auto load_kv = [&](const CUtensorMap* tm, const Item<D>& m, int j) -> bool {
+                if (!mbar_wait(smem_u32(b_kvempty + stage), phase ^ 1u, lim, kSiteKvEmpty)) return false;
+                const uint32_t fb = smem_u32(b_kvfull + stage);
+                mbar_arrive_expect_tx(fb, (uint32_t)C::TILE_BYTES);
+                for (int ch = 0; ch < C::NCHUNK; ++ch)
+                    tma_load_4d(smem_u32(sKV + stage * C::TILE_BYTES + ch * C::CHUNK_BYTES), tm, fb, ch * 64,
+                                m.h, j * C::BN, m.b);
+                filled[stage] = true;
+                filled_phase[stage] = phase;
+                if (++stage == (uint32_t)C::NS) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                return true;
+            };
+            auto load_q = [&](const Item<D>& m, int g) -> bool {
+                if (q_uses[g] > 0 &&
+                    !mbar_wait(smem_u32(b_qempty + g), (q_uses[g] - 1) & 1u, lim, kSiteQEmpty))
+                    return false;
+                const uint32_t qb = smem_u32(b_qfull + g);
+                mbar_arrive_expect_tx(qb, (uint32_t)C::TILE_BYTES);
+                for (int ch = 0; ch < C::NCHUNK; ++ch)
+                    tma_load_4d(smem_u32(sQ + g * C::TILE_BYTES + ch * C::CHUNK_BYTES), &tm_q, qb, ch * 64,
+                                m.h, m.q0[g], m.b);
+                ++q_uses[g];
+                return true;
+            };
             for (uint32_t k = 0; ok; ++k) {
                 int it = atomicAdd(p.sched, 1);
                 if (it >= p.n_items) it = -1;
@@ -265,36 +297,14 @@ __global__ void __maxnreg__(168)
                 mbar_arrive(smem_u32(b_itfull + slot));
                 if (it < 0) break;
                 const Item<D> m = decode_item<D>(p, it);
-                for (int g = 0; ok && g < 2; ++g) {
-                    if (!m.valid[g]) continue;
-                    if (q_uses[g] > 0 &&
-                        !(ok = mbar_wait(smem_u32(b_qempty + g), (q_uses[g] - 1) & 1u, lim, kSiteQEmpty)))
-                        break;
-                    const uint32_t qb = smem_u32(b_qfull + g);
-                    mbar_arrive_expect_tx(qb, (uint32_t)C::TILE_BYTES);
-                    for (int ch = 0; ch < C::NCHUNK; ++ch)
-                        tma_load_4d(smem_u32(sQ + g * C::TILE_BYTES + ch * C::CHUNK_BYTES), &tm_q, qb,
-                                    ch * 64, m.h, m.q0[g], m.b);
-                    ++q_uses[g];
-                }
-                for (int j = m.lo; ok && j <= m.hi; ++j) {
-                    for (int which = 0; which < 2; ++which) {
-                        if (!(ok = mbar_wait(smem_u32(b_kvempty + stage), phase ^ 1u, lim, kSiteKvEmpty)))
-                            break;
-                        const uint32_t fb = smem_u32(b_kvfull + stage);
-                        mbar_arrive_expect_tx(fb, (uint32_t)C::TILE_BYTES);
-                        const CUtensorMap* tm = which == 0 ? &tm_k : &tm_v;
-                        for (int ch = 0; ch < C::NCHUNK; ++ch)
-                            tma_load_4d(smem_u32(sKV + stage * C::TILE_BYTES + ch * C::CHUNK_BYTES), tm, fb,
-                                        ch * 64, m.h, j * C::BN, m.b);
-                        filled[stage] = true;
-                        filled_phase[stage] = phase;
-                        if (++stage == (uint32_t)C::NS) {
-                            stage = 0;
-                            phase ^= 1u;
-                        }
-                    }
-                }
+                // Warm L2 with this item's query tiles while the previous item finishes.
+                for (int g = 0; g < 2; ++g)
+                    if (m.valid[g])
+                        for (int ch = 0; ch < C::NCHUNK; ++ch) tma_prefetch_4d(&tm_q, ch * 64, m.h, m.q0[g], m.b);
+                // Order: Q0, K_lo, Q1, V_lo, then K/V of the rest, so tile 0 can start before tile 1.
+                ok = load_q(m, 0) && load_kv(&tm_k, m, m.lo) && (!m.valid[1] || load_q(m, 1)) &&
+                     load_kv(&tm_v, m, m.lo);
+                for (int j = m.lo + 1; ok && j <= m.hi; ++j) ok = load_kv(&tm_k, m, j) && load_kv(&tm_v, m, j);
             }
             // The last CTA to run out of items resets the counters for the next launch.
             if (ok && atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1) {
@@ -307,16 +317,18 @@ __global__ void __maxnreg__(168)
             for (int s = 0; s < C::NS; ++s)
                 if (filled[s]) mbar_wait(smem_u32(b_kvfull + s), filled_phase[s], lim, kSiteDrain);
         }
-    } else if (warp == 9) {
+    } else if (warp == kMmaWarp) {
         // ============================== MMA issuer ==============================
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, C::BN, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-            const uint32_t sQ_addr = smem_u32(sQ);
-            const uint32_t sKV_addr = smem_u32(sKV);
+            const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+            const uint64_t dkv = smem_desc_sw128(smem_u32(sKV), 16, 1024);
+            const uint64_t dv = smem_desc_sw128(smem_u32(sKV), C::CHUNK_BYTES, 1024);
             uint32_t stage = 0, phase = 0;
             uint32_t p_phase[2] = {0u, 0u};
             uint32_t uses[2] = {0u, 0u};     // items in which each query tile was valid
+            // K/V ring slot; the data arrived by TMA, so the barrier wait alone orders the reads.
             auto acquire = [&](uint32_t& s) -> bool {
                 s = stage;
                 const bool r = mbar_wait(smem_u32(b_kvfull + stage), phase, lim, kSiteKvFull);
@@ -326,29 +338,28 @@ __global__ void __maxnreg__(168)
                 }
                 return r;
             };
-            // S_g = Q_g K^T : M=128, N=BN, K=D in steps of 16 (32 bytes inside a swizzle chunk).
+            // S_g = Q_g K^T : M=128, N=BN, K=D in steps of 16 (32 bytes inside a 128-byte swizzle
+            // chunk; the descriptor start address advances in 16-byte units).
             auto issue_s = [&](int g, uint32_t sk) {
-                const uint32_t a0 = sQ_addr + g * C::TILE_BYTES;
-                const uint32_t b0 = sKV_addr + sk * C::TILE_BYTES;
+                const uint64_t da = dq + (uint64_t)((g * C::TILE_BYTES) >> 4);
+                const uint64_t db = dkv + (uint64_t)((sk * C::TILE_BYTES) >> 4);
                 const uint32_t d = tmem + (g == 0 ? C::COL_S0 : C::COL_S1);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
-                    mma_ss(d, smem_desc_sw128(a0 + off, 16, 1024), smem_desc_sw128(b0 + off, 16, 1024),
-                           idesc_qk, kk > 0 ? 1u : 0u);
+                    const uint32_t off = ((kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32) >> 4;
+                    mma_ss(d, da + off, db + off, idesc_qk, kk > 0 ? 1u : 0u);
                 }
             };
             // O_g += P_g V : M=128, N=D, K=BN in steps of 16 key rows.  P from tensor memory
             // (8 columns of packed bf16 pairs per step), V MN-major from shared memory.
             auto issue_pv = [&](int g, uint32_t sv, bool acc) {
                 const uint32_t pa = tmem + (g == 0 ? C::COL_S0 : C::COL_S1);
-                const uint32_t b0 = sKV_addr + sv * C::TILE_BYTES;
                 const uint32_t d = tmem + (g == 0 ? C::COL_O0 : C::COL_O1);
+                const uint64_t db = dv + (uint64_t)((sv * C::TILE_BYTES) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk) {
-                    mma_ts(d, pa + kk * 8, smem_desc_sw128(b0 + kk * 16 * 128, C::CHUNK_BYTES, 1024),
-                           idesc_pv, (acc || kk > 0) ? 1u : 0u);
-                }
+                for (int kk = 0; kk < C::BN / 16; ++kk)
+                    mma_ts(d, pa + kk * 8, db + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv,
+                           (acc || kk > 0) ? 1u : 0u);
             };
             // S_g(j), then release Q_g once its last S product of the item is issued.
             auto s_step = [&](const Item<D>& m, int g, uint32_t sk, int j) {
@@ -378,25 +389,24 @@ __global__ void __maxnreg__(168)
                 mbar_arrive(smem_u32(b_itempty + slot));
                 if (it < 0) break;
                 const Item<D> m = decode_item<D>(p, it);
-                for (int g = 0; ok && g < 2; ++g)
-                    if (m.valid[g]) ok = mbar_wait(smem_u32(b_qfull + g), uses[g] & 1u, lim, kSiteQFull);
+                // Tile 0 starts as soon as its Q and the first K are in; tile 1 waits for its Q
+                // only when its first product is due.
                 uint32_t sk = 0;
-                if (ok) ok = acquire(sk);
-                if (!ok) break;
-                tc_fence_after();
-                for (int g = 0; g < 2; ++g)
-                    if (m.active(g, m.lo)) s_step(m, g, sk, m.lo);
+                if (!(ok = mbar_wait(smem_u32(b_qfull + 0), uses[0] & 1u, lim, kSiteQFull))) break;
+                if (!(ok = acquire(sk))) break;
+                if (m.active(0, m.lo)) s_step(m, 0, sk, m.lo);
+                if (m.valid[1] && !(ok = mbar_wait(smem_u32(b_qfull + 1), uses[1] & 1u, lim, kSiteQFull)))
+                    break;
+                if (m.active(1, m.lo)) s_step(m, 1, sk, m.lo);
                 mma_commit(smem_u32(b_kvempty + sk));
                 for (int j = m.lo; ok && j <= m.hi; ++j) {
                     uint32_t sv = 0;
                     if (!(ok = acquire(sv))) break;
-                    tc_fence_after();
                     if (m.active(0, j) && !(ok = pv_step(m, 0, sv, j))) break;
                     const bool next = j + 1 <= m.hi;
                     uint32_t sk2 = 0;
                     if (next) {
                         if (!(ok = acquire(sk2))) break;
-                        tc_fence_after();
                         if (m.active(0, j + 1)) s_step(m, 0, sk2, j + 1);
                     }
                     if (m.active(1, j) && !(ok = pv_step(m, 1, sv, j))) break;
@@ -416,8 +426,9 @@ __global__ void __maxnreg__(168)
         __syncwarp();
     } else {
         // ============================ softmax + epilogue ============================
-        const int g = warp >> 2;                  // query tile of this warpgroup
-        const int r = ((warp & 3) << 5) + lane;   // row within the tile == TMEM lane
+        const int g = (warp - kSoftmaxWarp0) >> 2;   // query tile of this warpgroup
+        // A warp reaches the TMEM lanes of its quarter, 32 (warp % 4) .. + 31: row r of the tile.
+        const int r = ((warp & 3) << 5) + lane;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t colS = g == 0 ? C::COL_S0 : C::COL_S1;
         const uint32_t colO = g == 0 ? C::COL_O0 : C::COL_O1;
@@ -520,36 +531,36 @@ __global__ void __maxnreg__(168)
             const float inv_l = 1.0f / lr;
             const bool row_ok = qi < p.T;
             __nv_bfloat16* orow = p.out + (((long long)m.b * p.T + qi) * p.H + m.h) * D;
+            // Read all of O, then release it to the next item, then convert and store.
+            uint32_t ov[D / 32][32];
 #pragma unroll
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t ov[32];
-                tmem_ld32(tmem + lane_base + colO + cc * 32, ov);
-                tmem_ld_wait();
-                if (row_ok) {
+            for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tmem + lane_base + colO + cc * 32, ov[cc]);
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(smem_u32(b_oempty + g));
+            ++o_uses;
+            if (row_ok) {
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t w16[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
-                        w16[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l,
-                                             __uint_as_float(ov[2 * e + 1]) * inv_l);
+                        w16[e] = pack_bf16x2(__uint_as_float(ov[cc][2 * e]) * inv_l,
+                                             __uint_as_float(ov[cc][2 * e + 1]) * inv_l);
                     uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         dst[e] = make_uint4(w16[4 * e], w16[4 * e + 1], w16[4 * e + 2], w16[4 * e + 3]);
                 }
+                if (p.lse != nullptr) p.lse[((long long)m.b * p.H + m.h) * p.T + qi] = p.m0 + logf(l);
             }
-            // O of this tile has been read: the next item's first PV may overwrite it.
-            tc_fence_before();
-            mbar_arrive(smem_u32(b_oempty + g));
-            ++o_uses;
-            if (row_ok && p.lse != nullptr)
-                p.lse[((long long)m.b * p.H + m.h) * p.T + qi] = p.m0 + logf(l);
         }
     }
 
     // ---- teardown: all tensor-memory traffic of this CTA is finished before the free.
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }

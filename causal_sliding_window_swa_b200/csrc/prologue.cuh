@@ -19,9 +19,9 @@
 //     2^-33), so every product a * piece is exact in fp32 for a bf16 input a; x = ra * r is then
 //     within 4 of its own ulps of the exact value whenever |x| >= 2^-8 r (|a| + |b|).  The test
 //     window is 8 ulps, and smaller |x| (partial cancellation) always take the fp64 path.
-//   gate: z = x[:32] . Wg[:, h] and g = 2 sigmoid(z) in fp64, split as g_hi + g_lo (fp32);
-//     v' = (v + g_hi ve) + g_lo ve with two fp32 roundings: within 1 ulp of the exact value
-//     unless |v'| < 2^-16 |g ve|.
+//   gate: z = x[:32] . Wg[:, h] and g = 2 sigmoid(z) in fp64 by a separate one-thread-per-row
+//     kernel, stored split as g_hi + g_lo (fp32); v' = (v + g_hi ve) + g_lo ve with two fp32
+//     roundings: within 1 ulp of the exact value unless |v'| < 2^-16 |g ve|.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -30,6 +30,37 @@
 #include "ptx.cuh"
 
 namespace swa {
+
+// Division by a loop-invariant divisor d for 0 <= n < 2^31: q = (n * m) >> k with
+// k = 32 + ceil(log2 d) and m = ceil(2^k / d) (Granlund and Montgomery, "Division by invariant
+// integers using multiplication", 1994: the error term n (m d - 2^k) / (d 2^k) stays below 1/d).
+struct FastDiv {
+    unsigned long long m;
+    int k;
+    int d;
+};
+
+__device__ __forceinline__ int fdiv(int n, const FastDiv& f) {
+    return (int)(((unsigned long long)(unsigned)n * f.m) >> f.k);
+}
+
+// Gate of every (b, t, h) row: g = 2 sigmoid(sum_{c<32} x[b,t,c] Wg[c,h]) in fp64, stored as
+// (g_hi, g_lo) = (fp32(g), fp32(g - g_hi)).
+__global__ void gate_kernel(const __nv_bfloat16* __restrict__ gate_x, const __nv_bfloat16* __restrict__ Wg,
+                            float2* __restrict__ gate, int n_rows, int H, FastDiv divH) {
+    for (int row = blockIdx.x * blockDim.x + threadIdx.x; row < n_rows; row += gridDim.x * blockDim.x) {
+        const int bt = fdiv(row, divH);
+        const int h = row - bt * H;
+        const __nv_bfloat16* xr = gate_x + (long long)bt * 32;
+        double z = 0.0;
+#pragma unroll 8
+        for (int c = 0; c < 32; ++c)
+            z = fma((double)__bfloat162float(xr[c]), (double)__bfloat162float(Wg[c * H + h]), z);
+        const double g = 2.0 / (1.0 + exp(-z));
+        const float g_hi = (float)g;
+        gate[row] = make_float2(g_hi, (float)(g - (double)g_hi));
+    }
+}
 
 // RoPE tables, one entry per (t, i):
 //   tab32[t*D/2 + i] = (c_hi, c_lo, s_hi, s_lo) fp32, each piece with a 16-bit significand;
@@ -211,18 +242,18 @@ template <int D, bool HAS_VE>
 __global__ void __launch_bounds__(256, 3) prologue_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
     const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ ve,
-    const __nv_bfloat16* __restrict__ gate_x, const __nv_bfloat16* __restrict__ Wg,
+    const float2* __restrict__ gate,
     __nv_bfloat16* __restrict__ qh, __nv_bfloat16* __restrict__ kh, __nv_bfloat16* __restrict__ vp,
     const float4* __restrict__ tab32, const double2* __restrict__ tab64, int* __restrict__ sched,
-    long long n_rows, int T, int H, double eps) {
+    int n_rows, int T, int H, FastDiv divT, FastDiv divH, double eps) {
     constexpr int TPR = D / 8;           // threads per row (16 or 8); divides 32
+    constexpr int LOG_TPR = (D == 128) ? 4 : 3;
     constexpr int HALF = D / 2;
-    constexpr int GCH = 32 / TPR;        // gate channels per thread (2 or 4)
     const long long gtid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
     const long long stride = (long long)gridDim.x * blockDim.x;
     // Every thread of a warp runs the same number of iterations, so the shuffles always see the
     // full warp; rows past the end are computed on zeros and not stored.
-    const long long n_iter = (n_rows * TPR + stride - 1) / stride;
+    const long long n_iter = ((long long)n_rows * TPR + stride - 1) / stride;
     // The attention kernel that follows takes its work items from this counter.
     if (gtid == 0) {
         sched[0] = 0;
@@ -230,18 +261,18 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(
     }
     for (long long it = 0; it < n_iter; ++it) {
         const long long tid = gtid + it * stride;
-        const long long row = tid / TPR;          // (b*T + t)*H + h
-        const int c = (int)(tid % TPR);
-        const bool valid = row < n_rows;
-        const long long rr = valid ? row : 0;
-        const int h = (int)(rr % H);
-        const long long bt = rr / H;
-        const int t = (int)(bt % T);
+        const int row_raw = (int)(tid >> LOG_TPR);           // (b*T + t)*H + h, < 2^31
+        const int c = (int)(tid & (TPR - 1));
+        const bool valid = row_raw < n_rows;
+        const int row = valid ? row_raw : 0;
+        const int bt = fdiv(row, divH);
+        const int t = bt - fdiv(bt, divT) * T;
         const int i0 = 4 * c;
-        const long long off = rr * D;
+        const long long off = (long long)row * D;
 
         // Every load of this row chunk is issued before any arithmetic.
         uint2 raw[8];
+        float2 gw = make_float2(0.f, 0.f);
         if (valid) {
             raw[0] = ldg_stream8(q + off + i0);
             raw[1] = ldg_stream8(q + off + HALF + i0);
@@ -252,6 +283,7 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(
                 raw[5] = ldg_stream8(v + off + HALF + i0);
                 raw[6] = ldg_stream8(ve + off + i0);
                 raw[7] = ldg_stream8(ve + off + HALF + i0);
+                gw = __ldg(gate + row);
             }
         } else {
 #pragma unroll
@@ -272,25 +304,10 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(
             *reinterpret_cast<uint2*>(qh + off + HALF + i0) = o1;
             *reinterpret_cast<uint2*>(kh + off + i0) = o2;
             *reinterpret_cast<uint2*>(kh + off + HALF + i0) = o3;
-        }
-
-        if constexpr (HAS_VE) {
-            double z = 0.0;
-            if (valid) {
-                const __nv_bfloat16* xr = gate_x + bt * 32 + c * GCH;
-#pragma unroll
-                for (int e = 0; e < GCH; ++e)
-                    z = fma((double)__bfloat162float(xr[e]),
-                            (double)__bfloat162float(Wg[(c * GCH + e) * H + h]), z);
-            }
-#pragma unroll
-            for (int m = TPR / 2; m >= 1; m >>= 1) z += __shfl_xor_sync(0xffffffffu, z, m);
-            const double g64 = 2.0 / (1.0 + exp(-z));
-            const float g_hi = (float)g64;
-            const float g_lo = (float)(g64 - (double)g_hi);
-            if (valid) {
-                *reinterpret_cast<uint2*>(vp + off + i0) = gated_add4(raw[4], raw[6], g_hi, g_lo, g64);
-                *reinterpret_cast<uint2*>(vp + off + HALF + i0) = gated_add4(raw[5], raw[7], g_hi, g_lo, g64);
+            if (HAS_VE) {
+                const double g64 = (double)gw.x + (double)gw.y;
+                *reinterpret_cast<uint2*>(vp + off + i0) = gated_add4(raw[4], raw[6], gw.x, gw.y, g64);
+                *reinterpret_cast<uint2*>(vp + off + HALF + i0) = gated_add4(raw[5], raw[7], gw.x, gw.y, g64);
             }
         }
     }

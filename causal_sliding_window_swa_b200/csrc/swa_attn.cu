@@ -82,11 +82,11 @@ constexpr size_t kAlign = 1024;
 size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct WsLayout {
-    size_t qh, kh, vp, tab32, tab64, sched, total;
+    size_t qh, kh, vp, gate, tab32, tab64, sched, total;
 };
 
-// qhat | khat | v' (value-embedding layers only) | RoPE table fp32 pieces | RoPE table fp64 |
-// attention scheduler counters, each section 1024-byte aligned.
+// qhat | khat | v' and gate (value-embedding layers only) | RoPE table fp32 pieces |
+// RoPE table fp64 | attention scheduler counters, each section 1024-byte aligned.
 WsLayout ws_layout(const Shape& s, bool has_ve) {
     WsLayout w{};
     const size_t tensor = round_up((size_t)s.n * 2);
@@ -94,7 +94,8 @@ WsLayout ws_layout(const Shape& s, bool has_ve) {
     w.qh = 0;
     w.kh = w.qh + tensor;
     w.vp = w.kh + tensor;
-    w.tab32 = w.vp + (has_ve ? tensor : 0);
+    w.gate = w.vp + (has_ve ? tensor : 0);
+    w.tab32 = w.gate + (has_ve ? round_up((size_t)s.B * s.T * s.H * sizeof(float2)) : 0);
     w.tab64 = w.tab32 + round_up(pairs * sizeof(float4));
     w.sched = w.tab64 + round_up(pairs * sizeof(double2));
     w.total = w.sched + kAlign;
@@ -181,6 +182,17 @@ bool make_tile_map(CUtensorMap* m, const void* base, const Shape& s) {
 
 // ---------------------------------------------------------------------------- launches
 
+swa::FastDiv make_fastdiv(int d) {
+    int l = 0;
+    while ((1ll << l) < d) ++l;          // ceil(log2 d)
+    const int k = 32 + l;
+    swa::FastDiv f;
+    f.m = (unsigned long long)((((unsigned __int128)1 << k) + (unsigned)d - 1) / (unsigned)d);
+    f.k = k;
+    f.d = d;
+    return f;
+}
+
 int launch_rope_table(uint8_t* ws, const WsLayout& L, const Shape& s, float rope_base, cudaStream_t st) {
     const long long n = (long long)s.T * (s.D / 2);
     const int threads = 256;
@@ -196,16 +208,21 @@ int launch_prologue(const void* q, const void* k, const void* v, const void* ve,
                     cudaStream_t st) {
     using bf = __nv_bfloat16;
     const bool has_ve = ve != nullptr;
-    const long long n_rows = (long long)s.B * s.T * s.H;
-    const long long threads_total = n_rows * (s.D / 8);
+    const int n_rows = s.B * s.T * s.H;
+    const swa::FastDiv divH = make_fastdiv(s.H), divT = make_fastdiv(s.T);
+    float2* gate = reinterpret_cast<float2*>(ws + L.gate);
+    if (has_ve) {
+        const int gblocks = (int)std::min<long long>(((long long)n_rows + 255) / 256, 148ll * 8);
+        swa::gate_kernel<<<gblocks, 256, 0, st>>>(static_cast<const bf*>(gate_x), static_cast<const bf*>(Wg),
+                                                   gate, n_rows, s.H, divH);
+    }
+    const long long threads_total = (long long)n_rows * (s.D / 8);
     const int threads = 256;
     const long long blocks = std::min<long long>((threads_total + threads - 1) / threads, 148ll * 3 * 4);
     const bf* qp = static_cast<const bf*>(q);
     const bf* kp = static_cast<const bf*>(k);
     const bf* vpi = static_cast<const bf*>(v);
     const bf* vep = static_cast<const bf*>(ve);
-    const bf* gx = static_cast<const bf*>(gate_x);
-    const bf* wg = static_cast<const bf*>(Wg);
     bf* qh = reinterpret_cast<bf*>(ws + L.qh);
     bf* kh = reinterpret_cast<bf*>(ws + L.kh);
     bf* vp = reinterpret_cast<bf*>(ws + L.vp);
@@ -213,16 +230,17 @@ int launch_prologue(const void* q, const void* k, const void* v, const void* ve,
     const double2* t64 = reinterpret_cast<const double2*>(ws + L.tab64);
     int* sched = reinterpret_cast<int*>(ws + L.sched);
     const unsigned g = (unsigned)blocks;
+    const double e = (double)eps;
     if (s.D == 128) {
         if (has_ve)
-            swa::prologue_kernel<128, true><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gx, wg, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, (double)eps);
+            swa::prologue_kernel<128, true><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, divT, divH, e);
         else
-            swa::prologue_kernel<128, false><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gx, wg, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, (double)eps);
+            swa::prologue_kernel<128, false><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, divT, divH, e);
     } else {
         if (has_ve)
-            swa::prologue_kernel<64, true><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gx, wg, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, (double)eps);
+            swa::prologue_kernel<64, true><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, divT, divH, e);
         else
-            swa::prologue_kernel<64, false><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gx, wg, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, (double)eps);
+            swa::prologue_kernel<64, false><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, divT, divH, e);
     }
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
