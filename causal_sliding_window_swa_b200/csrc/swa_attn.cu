@@ -247,19 +247,18 @@ int launch_prologue(const void* q, const void* k, const void* v, const void* ve,
 
 int launch_attention(int dev, const void* v, bool has_ve, void* out, float* lse, const Shape& s,
                      int window, uint8_t* ws, const WsLayout& L, cudaStream_t st) {
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     const void* vsrc = has_ve ? static_cast<const void*>(ws + L.vp) : v;
     if (!make_tile_map(&tq, ws + L.qh, s) || !make_tile_map(&tk, ws + L.kh, s) ||
-        !make_tile_map(&tv, vsrc, s))
+        !make_tile_map(&tv, vsrc, s) || !make_tile_map(&to, out, s))
         return SWA_ERR_CUDA;
     swa::FwdParams p{};
     p.B = s.B;
     p.T = s.T;
     p.H = s.H;
     p.W = (window <= 0 || window >= s.T) ? s.T : window;
-    const int n_qtiles = (s.T + 127) / 128;
-    p.n_pairs = (n_qtiles + 1) / 2;
-    p.n_items = p.n_pairs * s.H * s.B;
+    p.n_qtiles = (s.T + 127) / 128;
+    p.n_items = p.n_qtiles * s.H * s.B;
     // Scheduling chunks of (b, h) slices whose K/V (about 4 T D bytes each) fit in ~40 MB of L2.
     const long long slice_bytes = 4ll * s.T * s.D;
     p.chunk_bh = (int)std::max<long long>(1, std::min<long long>((40ll << 20) / slice_bytes, (long long)s.B * s.H));
@@ -274,9 +273,9 @@ int launch_attention(int dev, const void* v, bool has_ve, void* out, float* lse,
     p.wait_limit_ns = wait_limit_ns();
     const dim3 grid((unsigned)std::min(p.n_items, g_num_sms[dev]));
     if (s.D == 128)
-        swa::attn_fwd_kernel<128><<<grid, swa::FwdCfg<128>::THREADS, swa::FwdCfg<128>::SMEM_TOTAL, st>>>(tq, tk, tv, p);
+        swa::attn_fwd_kernel<128><<<grid, swa::FwdCfg<128>::THREADS, swa::FwdCfg<128>::SMEM_TOTAL, st>>>(tq, tk, tv, to, p);
     else
-        swa::attn_fwd_kernel<64><<<grid, swa::FwdCfg<64>::THREADS, swa::FwdCfg<64>::SMEM_TOTAL, st>>>(tq, tk, tv, p);
+        swa::attn_fwd_kernel<64><<<grid, swa::FwdCfg<64>::THREADS, swa::FwdCfg<64>::SMEM_TOTAL, st>>>(tq, tk, tv, to, p);
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 

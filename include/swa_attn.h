@@ -60,7 +60,8 @@ typedef enum swa_status {
     SWA_ERR_INVALID_ARG = -1,  /* null pointer, size < 1, bad eps / rope_base, ve/gate_x/Wg partly set */
     SWA_ERR_UNSUPPORTED = -2,  /* D not in {64, 128}, sizes beyond int32 indexing, device not sm_100 */
     SWA_ERR_MISALIGNED = -3,   /* a tensor pointer or the workspace is not 16-byte aligned */
-    SWA_ERR_CUDA = -4,         /* a CUDA runtime / driver call failed (launch, allocation by CUDA) */
+    SWA_ERR_CUDA = -4,         /* a CUDA runtime / driver call failed (launch, allocation by CUDA),
+                                  or a kernel found its shared memory misaligned and did nothing */
     SWA_ERR_TIMEOUT = -5,      /* a bounded wait inside a kernel expired (read via last_device_status) */
     SWA_ERR_NO_MEMORY = -6,    /* workspace too small (swa_attn_fwd_ws) or allocation failed */
     SWA_ERR_NO_DEVICE = -7     /* no CUDA device is visible */
