@@ -62,6 +62,8 @@ def _load() -> ctypes.CDLL:
     lib.swa_attn_strerror.restype = ctypes.c_char_p
     lib.swa_attn_last_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
     lib.swa_attn_last_device_status.restype = I
+    lib.swa_attn_selftest_wait.argtypes = [I, P]
+    lib.swa_attn_selftest_wait.restype = I
     lib.swa_attn_set_wait_limit_ms.argtypes = [I]
     lib.swa_attn_set_wait_limit_ms.restype = I
     lib.swa_attn_version.argtypes = []
@@ -145,6 +147,10 @@ def swa_attn_last_device_status(stream=None) -> Tuple[int, int]:
     return int(rc), int(detail.value)
 
 
+def swa_attn_selftest_wait(limit_ms: int, stream=None) -> int:
+    return int(_lib.swa_attn_selftest_wait(int(limit_ms), stream))
+
+
 def swa_attn_set_wait_limit_ms(ms: int) -> int:
     return int(_lib.swa_attn_set_wait_limit_ms(int(ms)))
 
@@ -224,5 +230,5 @@ __all__ = [
     "forward", "check_device_status", "SwaError", "LIB_PATH", "load",
     "swa_attn_fwd", "swa_attn_fwd_ws", "swa_attn_fwd_noalloc", "swa_attn_noalloc_scratch_bytes", "swa_attn_workspace_bytes", "swa_attn_workspace_offset", "swa_attn_rope_table", "swa_attn_prologue",
     "swa_attn_attention", "swa_attn_strerror", "swa_attn_last_device_status",
-    "swa_attn_set_wait_limit_ms", "swa_attn_version",
+    "swa_attn_set_wait_limit_ms", "swa_attn_selftest_wait", "swa_attn_version",
 ]

@@ -15,6 +15,23 @@
 #include "attn_fwd.cuh"
 #include "prologue.cuh"
 
+// ------------------------------------------------------------------ failure-detection self-test
+
+namespace swa {
+// Waits, through the same bounded wait the kernels use, on an mbarrier that nothing ever
+// completes: after `limit_ns` the wait gives up and records a timeout at site kSiteSelfTest.
+constexpr unsigned int kSiteSelfTest = 30;
+__global__ void wait_selftest_kernel(unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    mbar_wait(smem_u32(&bar), 0u, limit_ns, kSiteSelfTest);
+}
+}  // namespace swa
+
 namespace {
 
 constexpr int kVersion = 100;   // 0.1.0
@@ -443,6 +460,16 @@ int swa_attn_fwd(const void* q, const void* k, const void* v, const void* ve, co
     }
     if ((rc = launch_prologue(q, k, v, ve, gate_x, Wg, ws, L, s, eps, st)) != SWA_OK) return rc;
     return launch_attention(dev, v, has_ve, out, lse, s, window, ws, L, st);
+}
+
+int swa_attn_selftest_wait(int limit_ms, swa_stream_t stream) {
+    if (limit_ms < 1 || limit_ms > 10000) return SWA_ERR_INVALID_ARG;
+    int dev;
+    int rc = device_ready(&dev);
+    if (rc != SWA_OK) return rc;
+    swa::wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        (unsigned long long)limit_ms * 1000000ull);
+    return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
 int swa_attn_last_device_status(swa_stream_t stream, unsigned int* detail) {

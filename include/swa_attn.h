@@ -184,6 +184,16 @@ SWA_API const char* swa_attn_strerror(int status);
  */
 SWA_API int swa_attn_last_device_status(swa_stream_t stream, unsigned int* detail);
 
+/*
+ * Failure-detection self-test (no counterpart in the pages).  Enqueues on `stream` one block of
+ * 32 threads that waits, through the bounded wait every kernel here uses, on an mbarrier that
+ * nothing ever completes.  After `limit_ms` (1..10000) the wait gives up, records SWA_ERR_TIMEOUT
+ * at wait site 30 in the device status word and the kernel returns normally: the device context
+ * stays usable.  Read the result with swa_attn_last_device_status().  Returns SWA_OK once the
+ * kernel is enqueued, SWA_ERR_INVALID_ARG for a limit out of range, else as the other calls.
+ */
+SWA_API int swa_attn_selftest_wait(int limit_ms, swa_stream_t stream);
+
 /* Upper bound, in milliseconds, on any single wait inside the kernels (default 2000).
  * Returns the previous value.  Values < 1 are ignored. */
 SWA_API int swa_attn_set_wait_limit_ms(int ms);

@@ -106,3 +106,9 @@ def test_wait_limit_setter():
     assert prev >= 1
     assert swa.swa_attn_set_wait_limit_ms(0) == 1500      # ignored, returns current
     swa.swa_attn_set_wait_limit_ms(prev)
+
+
+def test_selftest_wait_rejects_limits_out_of_range():
+    # validated before any device query, so this runs without a GPU
+    assert swa.swa_attn_selftest_wait(0, None) == swa.SWA_ERR_INVALID_ARG
+    assert swa.swa_attn_selftest_wait(10001, None) == swa.SWA_ERR_INVALID_ARG
