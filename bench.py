@@ -406,6 +406,93 @@ def prologue_bytes(s: workloads.LayerShape) -> float:
     return float(b)
 
 
+def run_decode(args, s):
+    """One generation step per timed iteration (swa_attn_decode) at the last position of the
+    workload's sequence: the new token of each of the B sequences attends to min(W, T) cached keys.
+    The caches are filled once by the prefill prologue, so they hold real khat / v'.  Metric: the
+    step's algorithmic bytes (K and V window reads, the new token's inputs and cache writes, out)
+    per second; HBM-bound."""
+    import torch
+    import causal_sliding_window_swa_b200 as swa
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU path)")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    d = workloads.make_layer(s)
+    g = {k: (None if v is None else v.to(dev)) for k, v in workloads.gpu_side_inputs(d).items()}
+    B, T, H, D = s.B, s.T, s.H, s.D
+    stream = torch.cuda.current_stream(dev)
+    st = stream.cuda_stream
+    P = lambda t: None if t is None else t.data_ptr()
+    # caches = the prefill prologue's khat / v' of every position
+    nbytes = swa.swa_attn_workspace_bytes(B, T, H, D, int(s.ve))
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    for rc, what in ((swa.swa_attn_rope_table(B, T, H, D, int(s.ve), 10000.0, ws.data_ptr(), nbytes, st), "rope"),
+                     (swa.swa_attn_prologue(P(g["q"]), P(g["k"]), P(g["v"]), P(g["ve"]), P(g["gate_x"]), P(g["Wg"]),
+                                            B, T, H, D, 10000.0, 1e-6, ws.data_ptr(), nbytes, st), "prologue")):
+        if rc != 0:
+            raise swa.SwaError(rc, what)
+    sec = lambda i: swa.swa_attn_workspace_offset(B, T, H, D, int(s.ve), i)
+    n = B * T * H * D
+    k_cache = ws[sec(1):sec(1) + 2 * n].view(torch.bfloat16).view(B, T, H, D).clone()
+    v_cache = (ws[sec(2):sec(2) + 2 * n].view(torch.bfloat16).view(B, T, H, D).clone() if s.ve else g["v"].clone())
+    pos = T - 1
+    tok = {k: (None if g[k] is None else g[k][:, pos].contiguous()) for k in ("q", "k", "v", "ve", "gate_x")}
+    out = torch.empty((B, H, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    need = swa.swa_attn_decode_workspace_bytes(B, T, H, D, int(s.ve), s.window)
+    dws = torch.empty(need, dtype=torch.uint8, device=dev)
+    argsd = (P(tok["q"]), P(tok["k"]), P(tok["v"]), P(tok["ve"]), P(tok["gate_x"]), P(g["Wg"]), P(k_cache),
+             P(v_cache), pos, P(out), P(lse), B, T, H, D, s.window, 10000.0, 1e-6, P(dws), need, st)
+
+    def step():
+        rc = swa.swa_attn_decode(*argsd)
+        if rc != 0:
+            raise swa.SwaError(rc, "swa_attn_decode")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    swa.check_device_status(stream)
+    # L2 (126 MB) holds part of the 201 MB window: flush it between steps with a 256 MB write.
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(0).start()
+    for i in range(K):
+        flush.fill_(i & 0xff)
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    swa.check_device_status(stream)
+    ms = sum(a.elapsed_time(b) for a, b in evs) / K
+    W = T if s.window <= 0 or s.window >= T else s.window
+    keys = min(W, pos + 1)
+    bytes_step = (2.0 * B * keys * H * D * 2          # K and V window reads
+                  + B * H * D * 2 * (3 + 2 + 1)       # q, k, v in; khat, v' cache writes; out
+                  + (B * H * D * 2 + B * 32 * 2 if s.ve else 0))
+    gbs = bytes_step / (ms * 1e-3) / 1e9
+    peaks, peak_src = load_peaks()
+    line = {
+        "metric": "decode step, KV-cache window read bandwidth (d24 shape, last position)",
+        "value": gbs, "unit": "GB/s", "n_gpus": 1, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 in/out, fp32 scores and sums", "data": "synthetic (seeded), caches from the prefill prologue",
+        "config": {"workload": f"decode {args.workload}: B={B} Tmax={T} H={H} D={D} W={W} pos={pos} ve={s.ve}",
+                   "l2": "flushed between steps (256 MB write, outside the timed events)"},
+        "tokens_per_s": B / (ms * 1e-3),
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src},
+        "gpu_launches": (5 if s.ve else 4) * K,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -417,10 +504,14 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--reference-budget-s", type=float, default=90.0)
+    ap.add_argument("--mode", choices=["forward", "decode"], default="forward",
+                    help="decode: time one KV-cache generation step instead of the layer forward")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     s = WORKLOADS[args.workload]
+    if args.mode == "decode":
+        return run_decode(args, s)
     if args.impl == "reference":
         return run_reference(args, s)
     return run_ours(args, s)

@@ -62,6 +62,10 @@ def _load() -> ctypes.CDLL:
     lib.swa_attn_strerror.restype = ctypes.c_char_p
     lib.swa_attn_last_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
     lib.swa_attn_last_device_status.restype = I
+    lib.swa_attn_decode_workspace_bytes.argtypes = [I, I, I, I, I, I]
+    lib.swa_attn_decode_workspace_bytes.restype = Z
+    lib.swa_attn_decode.argtypes = [P, P, P, P, P, P, P, P, I, P, P, I, I, I, I, I, F, F, P, Z, P]
+    lib.swa_attn_decode.restype = I
     lib.swa_attn_selftest_wait.argtypes = [I, P]
     lib.swa_attn_selftest_wait.restype = I
     lib.swa_attn_set_wait_limit_ms.argtypes = [I]
@@ -147,6 +151,16 @@ def swa_attn_last_device_status(stream=None) -> Tuple[int, int]:
     return int(rc), int(detail.value)
 
 
+def swa_attn_decode_workspace_bytes(B, Tmax, H, D, has_ve, window) -> int:
+    return int(_lib.swa_attn_decode_workspace_bytes(B, Tmax, H, D, int(has_ve), window))
+
+
+def swa_attn_decode(q, k, v, ve, gate_x, Wg, k_cache, v_cache, pos, out, lse, B, Tmax, H, D, window,
+                    rope_base, eps, workspace, ws_bytes, stream) -> int:
+    return _lib.swa_attn_decode(q, k, v, ve, gate_x, Wg, k_cache, v_cache, pos, out, lse, B, Tmax, H, D,
+                                window, rope_base, eps, workspace, ws_bytes, stream)
+
+
 def swa_attn_selftest_wait(limit_ms: int, stream=None) -> int:
     return int(_lib.swa_attn_selftest_wait(int(limit_ms), stream))
 
@@ -219,6 +233,31 @@ def forward(q, k, v, window: int = 0, ve=None, gate_x=None, Wg=None, rope_base: 
     return out, lse
 
 
+def decode(q, k, v, k_cache, v_cache, pos: int, window: int, ve=None, gate_x=None, Wg=None,
+           rope_base: float = 1e4, eps: float = 1e-6, out=None, lse=None, workspace=None, stream=None):
+    """One generation step (C call swa_attn_decode) on torch tensors: q, k, v (B,H,D) bf16 of the
+    new token at position ``pos``; k_cache, v_cache (B,Tmax,H,D) bf16, updated in place at ``pos``.
+    Returns (out (B,H,D) bf16, lse (B,H) fp32).  Raises SwaError on a nonzero status."""
+    import torch
+    B, H, D = q.shape
+    Tmax = k_cache.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    need = swa_attn_decode_workspace_bytes(B, Tmax, H, D, ve is not None, window)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = _stream_handle(stream)
+    rc = swa_attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(k_cache),
+                         _ptr(v_cache), int(pos), _ptr(out), _ptr(lse), B, Tmax, H, D, int(window),
+                         float(rope_base), float(eps), _ptr(workspace),
+                         workspace.numel() * workspace.element_size(), st)
+    if rc != SWA_OK:
+        raise SwaError(rc, "swa_attn_decode")
+    return out, lse
+
+
 def check_device_status(stream=None) -> None:
     """Synchronise and raise SwaError if a kernel recorded an error (e.g. a wait timeout)."""
     rc, detail = swa_attn_last_device_status(_stream_handle(stream))
@@ -227,8 +266,9 @@ def check_device_status(stream=None) -> None:
 
 
 __all__ = [
-    "forward", "check_device_status", "SwaError", "LIB_PATH", "load",
+    "forward", "decode", "check_device_status", "SwaError", "LIB_PATH", "load",
     "swa_attn_fwd", "swa_attn_fwd_ws", "swa_attn_fwd_noalloc", "swa_attn_noalloc_scratch_bytes", "swa_attn_workspace_bytes", "swa_attn_workspace_offset", "swa_attn_rope_table", "swa_attn_prologue",
     "swa_attn_attention", "swa_attn_strerror", "swa_attn_last_device_status",
     "swa_attn_set_wait_limit_ms", "swa_attn_selftest_wait", "swa_attn_version",
+    "swa_attn_decode", "swa_attn_decode_workspace_bytes",
 ]

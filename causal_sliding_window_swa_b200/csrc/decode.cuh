@@ -1,0 +1,210 @@
+// decode.cuh -- one generation step with a key/value cache: the new token at position `pos` of
+// every sequence goes through the layer's prologue (RoPE, RMS QK-norm, gated value embedding;
+// intelliparadigm "GPT-2 for $73", sections 2.1, 2.2 and the "Value Embeddings" paragraph of
+// the PaperWeekly repost), its k-hat and v' are appended to the caches, and its query attends
+// to the cached keys inside its window ("Let's reproduce GPT-2 (124M)" notes, section 19, which
+// lists a KV cache among the missing pieces):
+//   out[b,h,:] = sum_{j in J} softmax_j(qhat . khat_j / sqrt(D)) v'_j,  J = [max(0, pos-W+1), pos].
+//
+// The per-element arithmetic of the prologue is the prefill path's (prologue.cuh), so the cache
+// entries are bit-identical to the k-hat / v' the prefill path writes for the same token.
+// Attention: the window's keys are cut into chunks of CK keys, one CTA per (chunk, b, h).  The
+// softmax offset is fixed at M0 = sqrt(D) (1 + 2^-6) (the QK-norm bound used by the prefill
+// kernel), so chunk results need no rescaling: each chunk writes sum_j p_j v'_j and sum_j p_j,
+// and a second kernel adds the chunks in order (deterministic) and divides.  Scores, exponentials
+// and the weighted sums are fp32; nothing goes through bf16 except the final output.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "prologue.cuh"
+#include "ptx.cuh"
+
+namespace swa {
+
+constexpr int kDecodeChunk = 128;        // keys per CTA of the attention kernel
+
+// Prologue of the new token: rows r = b*H + h; D/8 threads per row as in the prefill prologue.
+// The block first builds the RoPE row of position `pos` in shared memory, with the same split as
+// the prefill table (16-bit-significand pieces and the fp64 pair for the fallback).
+template <int D, bool HAS_VE>
+__global__ void __launch_bounds__(256) decode_prologue_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+    const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ ve,
+    const float2* __restrict__ gate, __nv_bfloat16* __restrict__ qh,
+    __nv_bfloat16* __restrict__ k_cache, __nv_bfloat16* __restrict__ v_cache, int n_rows, int H,
+    int Tmax, int pos, double base, double eps) {
+    constexpr int TPR = D / 8;
+    constexpr int HALF = D / 2;
+    __shared__ float4 s_tab32[HALF];
+    __shared__ double2 s_tab64[HALF];
+    for (int i = threadIdx.x; i < HALF; i += blockDim.x) {
+        const double theta = pow(base, -2.0 * (double)i / (double)D);
+        double sn, cs;
+        sincos((double)pos * theta, &sn, &cs);
+        const float c_hi = round_sig16(cs), s_hi = round_sig16(sn);
+        const float c_lo = round_sig16(cs - (double)c_hi), s_lo = round_sig16(sn - (double)s_hi);
+        s_tab32[i] = make_float4(c_hi, c_lo, s_hi, s_lo);
+        s_tab64[i] = make_double2(cs, sn);
+    }
+    __syncthreads();
+    const int rows_per_block = blockDim.x / TPR;
+    const int c = threadIdx.x % TPR;
+    const int i0 = 4 * c;
+    // Every thread of a warp runs the same number of iterations (rows past the end compute on
+    // zeros and store nothing), so the shuffles inside the row functions see the whole warp.
+    for (int row0 = blockIdx.x * rows_per_block; row0 < n_rows; row0 += gridDim.x * rows_per_block) {
+        const int row_raw = row0 + (int)threadIdx.x / TPR;
+        const bool valid = row_raw < n_rows;
+        const int row = valid ? row_raw : 0;
+        const int b = row / H;
+        const int h = row - b * H;
+        const long long in_off = (long long)row * D;
+        const long long cache_off = (((long long)b * Tmax + pos) * H + h) * D;
+        uint2 raw[8];
+        float2 gw = make_float2(0.f, 0.f);
+        if (valid) {
+            raw[0] = ldg_stream8(q + in_off + i0);
+            raw[1] = ldg_stream8(q + in_off + HALF + i0);
+            raw[2] = ldg_stream8(k + in_off + i0);
+            raw[3] = ldg_stream8(k + in_off + HALF + i0);
+            raw[4] = ldg_stream8(v + in_off + i0);
+            raw[5] = ldg_stream8(v + in_off + HALF + i0);
+            if (HAS_VE) {
+                raw[6] = ldg_stream8(ve + in_off + i0);
+                raw[7] = ldg_stream8(ve + in_off + HALF + i0);
+                gw = gate[row];
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) raw[e] = make_uint2(0u, 0u);
+        }
+        float4 cs4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) cs4[e] = s_tab32[i0 + e];
+        uint2 o0, o1, o2, o3;
+        rope_rms_pairs4<D>(raw[0], raw[1], cs4, s_tab64 + i0, eps, o0, o1);
+        rope_rms_pairs4<D>(raw[2], raw[3], cs4, s_tab64 + i0, eps, o2, o3);
+        if (valid) {
+            *reinterpret_cast<uint2*>(qh + in_off + i0) = o0;
+            *reinterpret_cast<uint2*>(qh + in_off + HALF + i0) = o1;
+            *reinterpret_cast<uint2*>(k_cache + cache_off + i0) = o2;
+            *reinterpret_cast<uint2*>(k_cache + cache_off + HALF + i0) = o3;
+            if (HAS_VE) {
+                const double g64 = (double)gw.x + (double)gw.y;
+                *reinterpret_cast<uint2*>(v_cache + cache_off + i0) = gated_add4(raw[4], raw[6], gw.x, gw.y, g64);
+                *reinterpret_cast<uint2*>(v_cache + cache_off + HALF + i0) =
+                    gated_add4(raw[5], raw[7], gw.x, gw.y, g64);
+            } else {
+                *reinterpret_cast<uint2*>(v_cache + cache_off + i0) = raw[4];
+                *reinterpret_cast<uint2*>(v_cache + cache_off + HALF + i0) = raw[5];
+            }
+        }
+    }
+}
+
+// bf16 bits -> fp32 for DPL consecutive elements starting at p (DPL = 4 or 2).
+template <int DPL>
+__device__ __forceinline__ void load_bf16(const __nv_bfloat16* p, float (&f)[DPL]) {
+    if constexpr (DPL == 4) {
+        const uint2 u = *reinterpret_cast<const uint2*>(p);
+        f[0] = __uint_as_float(u.x << 16);
+        f[1] = __uint_as_float(u.x & 0xffff0000u);
+        f[2] = __uint_as_float(u.y << 16);
+        f[3] = __uint_as_float(u.y & 0xffff0000u);
+    } else {
+        const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+        f[0] = __uint_as_float(u << 16);
+        f[1] = __uint_as_float(u & 0xffff0000u);
+    }
+}
+
+// Attention of the new token over one chunk of cached keys.  Grid B*H*n_chunks, 4 warps; the
+// lanes of a warp split the D features (D/32 each), and each warp takes every fourth key of the
+// chunk, four keys at a time so the four dot-product reductions overlap.  Partial results:
+// part[(row * n_chunks + chunk) * (D + 2) + d] = sum_j p_j v'_j[d], [.. + D] = sum_j p_j.
+template <int D>
+__global__ void __launch_bounds__(128) decode_attn_kernel(
+    const __nv_bfloat16* __restrict__ qh, const __nv_bfloat16* __restrict__ k_cache,
+    const __nv_bfloat16* __restrict__ v_cache, float* __restrict__ part, int H, int Tmax, int lo,
+    int n_keys, int n_chunks, float c1, float c2) {
+    constexpr int DPL = D / 32;          // features per lane
+    const int row = (int)(blockIdx.x / (unsigned)n_chunks);    // b*H + h
+    const int chunk = (int)(blockIdx.x - (unsigned)row * (unsigned)n_chunks);
+    const int b = row / H;
+    const int h = row - b * H;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __shared__ float s_o[4][D];
+    __shared__ float s_l[4];
+    float qf[DPL];
+    load_bf16<DPL>(qh + (long long)row * D + lane * DPL, qf);
+    float o[DPL];
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) o[e] = 0.f;
+    float l = 0.f;
+    const int key_begin = chunk * kDecodeChunk;
+    const int key_end = min(key_begin + kDecodeChunk, n_keys);
+    const long long stride = (long long)H * D;              // between consecutive positions
+    const __nv_bfloat16* kbase = k_cache + ((long long)b * Tmax + lo) * stride + (long long)h * D + lane * DPL;
+    const __nv_bfloat16* vbase = v_cache + ((long long)b * Tmax + lo) * stride + (long long)h * D + lane * DPL;
+    for (int j0 = key_begin + warp; j0 < key_end; j0 += 16) {
+        float s[4];
+        bool live[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = j0 + 4 * u;
+            live[u] = j < key_end;
+            s[u] = 0.f;
+            if (live[u]) {
+                float kf[DPL];
+                load_bf16<DPL>(kbase + (long long)j * stride, kf);
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) s[u] = fmaf(qf[e], kf[e], s[u]);
+            }
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) s[u] += __shfl_xor_sync(0xffffffffu, s[u], m);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (!live[u]) continue;
+            const int j = j0 + 4 * u;
+            const float p = ex2_approx(fmaf(s[u], c1, -c2));
+            l += p;
+            float vf[DPL];
+            load_bf16<DPL>(vbase + (long long)j * stride, vf);
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) o[e] = fmaf(p, vf[e], o[e]);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) s_o[warp][lane * DPL + e] = o[e];
+    if (lane == 0) s_l[warp] = l;
+    __syncthreads();
+    float* dst = part + ((long long)row * n_chunks + chunk) * (D + 2);
+    for (int d = threadIdx.x; d < D; d += blockDim.x)
+        dst[d] = (s_o[0][d] + s_o[1][d]) + (s_o[2][d] + s_o[3][d]);
+    if (threadIdx.x == 0) dst[D] = (s_l[0] + s_l[1]) + (s_l[2] + s_l[3]);
+}
+
+// Adds the chunks of each row in order and writes out = o / l (bf16) and lse = M0 + ln l.
+template <int D>
+__global__ void __launch_bounds__(D) decode_combine_kernel(const float* __restrict__ part,
+                                                          __nv_bfloat16* __restrict__ out,
+                                                          float* __restrict__ lse, int n_chunks,
+                                                          float m0) {
+    const int row = blockIdx.x;
+    const int d = threadIdx.x;
+    const float* src = part + (long long)row * n_chunks * (D + 2);
+    float o = 0.f, l = 0.f;
+    for (int c = 0; c < n_chunks; ++c) {
+        o += src[(long long)c * (D + 2) + d];
+        l += src[(long long)c * (D + 2) + D];
+    }
+    out[(long long)row * D + d] = __float2bfloat16_rn(o / l);
+    if (d == 0 && lse != nullptr) lse[row] = m0 + logf(l);
+}
+
+}  // namespace swa

@@ -13,6 +13,7 @@
 
 #include "swa_attn.h"
 #include "attn_fwd.cuh"
+#include "decode.cuh"
 #include "prologue.cuh"
 
 // ------------------------------------------------------------------ failure-detection self-test
@@ -460,6 +461,95 @@ int swa_attn_fwd(const void* q, const void* k, const void* v, const void* ve, co
     }
     if ((rc = launch_prologue(q, k, v, ve, gate_x, Wg, ws, L, s, eps, st)) != SWA_OK) return rc;
     return launch_attention(dev, v, has_ve, out, lse, s, window, ws, L, st);
+}
+
+// ------------------------------------------------------------- decode step with a KV cache
+//
+// Workspace: qhat of the new token (B*H*D bf16) | gate (B*H float2, value-embedding layers) |
+// chunk partials (B*H*n_chunks*(D+2) fp32), each section 1024-byte aligned; n_chunks covers the
+// largest window the call can see, min(window, Tmax) keys.
+
+size_t swa_attn_decode_workspace_bytes(int B, int Tmax, int H, int D, int has_ve, int window) {
+    Shape s;
+    if (check_sizes(B, Tmax, H, D, &s) != SWA_OK) return 0;
+    const long long rows = (long long)B * H;
+    const int W = (window <= 0 || window >= Tmax) ? Tmax : window;
+    const long long n_chunks = (W + swa::kDecodeChunk - 1) / swa::kDecodeChunk;
+    return round_up((size_t)rows * D * 2) + (has_ve ? round_up((size_t)rows * sizeof(float2)) : 0) +
+           round_up((size_t)(rows * n_chunks * (D + 2)) * sizeof(float));
+}
+
+int swa_attn_decode(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                    const void* Wg, void* k_cache, void* v_cache, int pos, void* out, float* lse,
+                    int B, int Tmax, int H, int D, int window, float rope_base, float eps,
+                    void* workspace, size_t ws_bytes, swa_stream_t stream) {
+    Shape s;
+    int rc = check_sizes(B, Tmax, H, D, &s);
+    if (rc == SWA_OK) rc = check_layer_args(q, k, v, ve, gate_x, Wg, rope_base, eps);
+    if (rc == SWA_OK) rc = check_outputs(out, lse);
+    if (rc != SWA_OK) return rc;
+    if (pos < 0 || pos >= Tmax || !k_cache || !v_cache || !workspace) return SWA_ERR_INVALID_ARG;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(workspace, 16)) return SWA_ERR_MISALIGNED;
+    const bool has_ve = ve != nullptr;
+    if (ws_bytes < swa_attn_decode_workspace_bytes(B, Tmax, H, D, has_ve, window)) return SWA_ERR_NO_MEMORY;
+    int dev;
+    if ((rc = device_ready(&dev)) != SWA_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    using bf = __nv_bfloat16;
+    const int rows = B * H;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    bf* qh = reinterpret_cast<bf*>(ws);
+    float2* gate = reinterpret_cast<float2*>(ws + round_up((size_t)rows * D * 2));
+    float* part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(gate) +
+                                           (has_ve ? round_up((size_t)rows * sizeof(float2)) : 0));
+    if (has_ve) {
+        // the gate rows of one step are (b, h): gate_x is (B, 32)
+        const int gblocks = std::max(1, std::min((rows + 255) / 256, 148 * 8));
+        swa::gate_kernel<<<gblocks, 256, 0, st>>>(static_cast<const bf*>(gate_x), static_cast<const bf*>(Wg),
+                                                   gate, rows, H, make_fastdiv(H));
+    }
+    {
+        const int rows_per_block = 256 / (D / 8);
+        const int blocks = std::max(1, std::min((rows + rows_per_block - 1) / rows_per_block, 148 * 8));
+        const bf* qp = static_cast<const bf*>(q);
+        const bf* kp = static_cast<const bf*>(k);
+        const bf* vp = static_cast<const bf*>(v);
+        const bf* vep = static_cast<const bf*>(ve);
+        bf* kc = static_cast<bf*>(k_cache);
+        bf* vc = static_cast<bf*>(v_cache);
+        const double base = (double)rope_base, e = (double)eps;
+        if (D == 128) {
+            if (has_ve)
+                swa::decode_prologue_kernel<128, true><<<blocks, 256, 0, st>>>(qp, kp, vp, vep, gate, qh, kc, vc, rows, H, Tmax, pos, base, e);
+            else
+                swa::decode_prologue_kernel<128, false><<<blocks, 256, 0, st>>>(qp, kp, vp, vep, gate, qh, kc, vc, rows, H, Tmax, pos, base, e);
+        } else {
+            if (has_ve)
+                swa::decode_prologue_kernel<64, true><<<blocks, 256, 0, st>>>(qp, kp, vp, vep, gate, qh, kc, vc, rows, H, Tmax, pos, base, e);
+            else
+                swa::decode_prologue_kernel<64, false><<<blocks, 256, 0, st>>>(qp, kp, vp, vep, gate, qh, kc, vc, rows, H, Tmax, pos, base, e);
+        }
+    }
+    const int W = (window <= 0 || window >= Tmax) ? Tmax : window;
+    const int lo = std::max(0, pos - W + 1);
+    const int n_keys = pos - lo + 1;
+    const int n_chunks = (n_keys + swa::kDecodeChunk - 1) / swa::kDecodeChunk;
+    const double log2e = 1.4426950408889634;
+    const double m0 = std::sqrt((double)D) * (1.0 + 1.0 / 64.0);
+    const float c1 = (float)(log2e / std::sqrt((double)D)), c2 = (float)(m0 * log2e);
+    const unsigned grid = (unsigned)((long long)rows * n_chunks);
+    const bf* qc = qh;
+    const bf* kcc = static_cast<const bf*>(k_cache);
+    const bf* vcc = static_cast<const bf*>(v_cache);
+    bf* o = static_cast<bf*>(out);
+    if (D == 128) {
+        swa::decode_attn_kernel<128><<<grid, 128, 0, st>>>(qc, kcc, vcc, part, H, Tmax, lo, n_keys, n_chunks, c1, c2);
+        swa::decode_combine_kernel<128><<<rows, 128, 0, st>>>(part, o, lse, n_chunks, (float)m0);
+    } else {
+        swa::decode_attn_kernel<64><<<grid, 128, 0, st>>>(qc, kcc, vcc, part, H, Tmax, lo, n_keys, n_chunks, c1, c2);
+        swa::decode_combine_kernel<64><<<rows, 64, 0, st>>>(part, o, lse, n_chunks, (float)m0);
+    }
+    return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
 int swa_attn_selftest_wait(int limit_ms, swa_stream_t stream) {

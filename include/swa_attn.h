@@ -185,6 +185,39 @@ SWA_API const char* swa_attn_strerror(int status);
 SWA_API int swa_attn_last_device_status(swa_stream_t stream, unsigned int* detail);
 
 /*
+ * One generation step with a key/value cache (the pages list a KV cache among the missing
+ * pieces: "Let's reproduce GPT-2 (124M)" notes, section 19).  For the new token of every
+ * sequence, at position `pos` (the same for all b):
+ *   1. the prologue of swa_attn_fwd at position pos: qhat = RMS(RoPE(q, pos)),
+ *      khat = RMS(RoPE(k, pos)), v' = v + 2 sigmoid(gate_x . Wg[:, h]) ve (value-embedding
+ *      layers) or v; khat and v' are written to k_cache[b, pos, h, :] and v_cache[b, pos, h, :],
+ *      bit-identical to what the prefill path computes for that token;
+ *   2. attention of qhat over the cached keys j in [max(0, pos - W + 1), pos] (W = Tmax if
+ *      window <= 0 or window >= Tmax): out[b,h,:] = sum_j softmax_j(qhat . khat_j / sqrt(D)) v'_j,
+ *      lse[b,h] = ln sum_j exp(qhat . khat_j / sqrt(D)).
+ * Arguments:
+ *   q, k, v      bf16 (B, H, D): the new token's raw projections.
+ *   ve, gate_x, Wg  bf16 (B, H, D) / (B, 32) / (32, H), all set (value-embedding layer) or all NULL.
+ *   k_cache, v_cache  bf16 (B, Tmax, H, D), caller-owned: entries j < pos (inside the window) must
+ *                hold khat / v' of earlier positions (as written by earlier calls or by the prefill
+ *                path); entry pos is written.
+ *   out          bf16 (B, H, D), written.   lse  fp32 (B, H) or NULL.
+ *   workspace    device memory of at least swa_attn_decode_workspace_bytes(B, Tmax, H, D, has_ve,
+ *                window) bytes, 16-byte aligned, caller-owned and not retained.
+ * Scores, exponentials and weighted sums are fp32 (no bf16 rounding of the weights).  The call is
+ * asynchronous on `stream` (five small kernels); arguments are validated before anything is
+ * enqueued.  Errors: SWA_ERR_INVALID_ARG (null pointer, pos outside [0, Tmax), bad rope_base /
+ * eps, partial value-embedding set), SWA_ERR_UNSUPPORTED (D not 64/128, sizes beyond int32),
+ * SWA_ERR_MISALIGNED, SWA_ERR_NO_MEMORY (workspace too small), SWA_ERR_CUDA.
+ */
+SWA_API size_t swa_attn_decode_workspace_bytes(int B, int Tmax, int H, int D, int has_ve, int window);
+SWA_API int swa_attn_decode(const void* q, const void* k, const void* v, const void* ve,
+                            const void* gate_x, const void* Wg, void* k_cache, void* v_cache,
+                            int pos, void* out, float* lse, int B, int Tmax, int H, int D,
+                            int window, float rope_base, float eps, void* workspace,
+                            size_t ws_bytes, swa_stream_t stream);
+
+/*
  * Failure-detection self-test (no counterpart in the pages).  Enqueues on `stream` one block of
  * 32 threads that waits, through the bounded wait every kernel here uses, on an mbarrier that
  * nothing ever completes.  After `limit_ms` (1..10000) the wait gives up, records SWA_ERR_TIMEOUT

@@ -112,3 +112,29 @@ def test_selftest_wait_rejects_limits_out_of_range():
     # validated before any device query, so this runs without a GPU
     assert swa.swa_attn_selftest_wait(0, None) == swa.SWA_ERR_INVALID_ARG
     assert swa.swa_attn_selftest_wait(10001, None) == swa.SWA_ERR_INVALID_ARG
+
+
+def test_decode_workspace_and_validation():
+    # qhat (B*H*D bf16) + chunk partials for the largest window, each section 1024-byte aligned
+    n = swa.swa_attn_decode_workspace_bytes(2, 1000, 3, 64, 0, 0)
+    chunks = (1000 + 127) // 128
+    assert n == 1024 + ((2 * 3 * chunks * 66 * 4 + 1023) // 1024) * 1024
+    assert swa.swa_attn_decode_workspace_bytes(2, 1000, 3, 64, 1, 200) > swa.swa_attn_decode_workspace_bytes(2, 1000, 3, 64, 0, 200)
+    assert swa.swa_attn_decode_workspace_bytes(2, 1000, 3, 96, 0, 0) == 0
+    need = swa.swa_attn_decode_workspace_bytes(1, 16, 1, 64, 0, 0)
+    base = dict(q=A, k=A, v=A, ve=None, gate_x=None, Wg=None, k_cache=A, v_cache=A, out=A, lse=A,
+                B=1, Tmax=16, H=1, D=64, window=0, rope_base=1e4, eps=1e-6, workspace=A, ws_bytes=need, stream=None)
+
+    def call(**kw):
+        a = dict(base, **kw)
+        return swa.swa_attn_decode(a["q"], a["k"], a["v"], a["ve"], a["gate_x"], a["Wg"], a["k_cache"],
+                                   a["v_cache"], a.get("pos", 3), a["out"], a["lse"], a["B"], a["Tmax"],
+                                   a["H"], a["D"], a["window"], a["rope_base"], a["eps"], a["workspace"],
+                                   a["ws_bytes"], a["stream"])
+    assert call(pos=16) == swa.SWA_ERR_INVALID_ARG
+    assert call(pos=-1) == swa.SWA_ERR_INVALID_ARG
+    assert call(k_cache=None) == swa.SWA_ERR_INVALID_ARG
+    assert call(ve=A) == swa.SWA_ERR_INVALID_ARG
+    assert call(v_cache=A + 8) == swa.SWA_ERR_MISALIGNED
+    assert call(ws_bytes=need - 1) == swa.SWA_ERR_NO_MEMORY
+    assert call(D=80) == swa.SWA_ERR_UNSUPPORTED
