@@ -486,7 +486,7 @@ def run_decode(args, s):
         "tokens_per_s": B / (ms * 1e-3),
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src},
-        "gpu_launches": (5 if s.ve else 4) * K,
+        "gpu_launches": 3 * K,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

@@ -11,7 +11,7 @@
 // Attention: the window's keys are cut into chunks of CK keys, one CTA per (chunk, b, h).  The
 // softmax offset is fixed at M0 = sqrt(D) (1 + 2^-6) (the QK-norm bound used by the prefill
 // kernel), so chunk results need no rescaling: each chunk writes sum_j p_j v'_j and sum_j p_j,
-// and a second kernel adds the chunks in order (deterministic) and divides.  Scores, exponentials
+// and a third kernel adds the chunks in order (deterministic) and divides.  Scores, exponentials
 // and the weighted sums are fp32; nothing goes through bf16 except the final output.
 #pragma once
 
@@ -27,14 +27,17 @@ constexpr int kDecodeChunk = 128;        // keys per CTA of the attention kernel
 
 // Prologue of the new token: rows r = b*H + h; D/8 threads per row as in the prefill prologue.
 // The block first builds the RoPE row of position `pos` in shared memory, with the same split as
-// the prefill table (16-bit-significand pieces and the fp64 pair for the fallback).
+// the prefill table (16-bit-significand pieces and the fp64 pair for the fallback).  On
+// value-embedding layers the first thread of each row computes the gate 2 sigmoid(x . Wg[:, h]) in
+// fp64 in the order of the prefill gate kernel, so the value is the same.
 template <int D, bool HAS_VE>
 __global__ void __launch_bounds__(256) decode_prologue_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
     const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ ve,
-    const float2* __restrict__ gate, __nv_bfloat16* __restrict__ qh,
-    __nv_bfloat16* __restrict__ k_cache, __nv_bfloat16* __restrict__ v_cache, int n_rows, int H,
-    int Tmax, int pos, double base, double eps) {
+    const __nv_bfloat16* __restrict__ gate_x, const __nv_bfloat16* __restrict__ Wg,
+    __nv_bfloat16* __restrict__ qh, __nv_bfloat16* __restrict__ k_cache,
+    __nv_bfloat16* __restrict__ v_cache, int n_rows, int H, int Tmax, int pos, double base,
+    double eps) {
     constexpr int TPR = D / 8;
     constexpr int HALF = D / 2;
     __shared__ float4 s_tab32[HALF];
@@ -64,6 +67,21 @@ __global__ void __launch_bounds__(256) decode_prologue_kernel(
         const long long cache_off = (((long long)b * Tmax + pos) * H + h) * D;
         uint2 raw[8];
         float2 gw = make_float2(0.f, 0.f);
+        if (HAS_VE) {
+            // gate of this row by its first thread, then shared with the row's other threads
+            if (c == 0 && valid) {
+                const __nv_bfloat16* xr = gate_x + (long long)b * 32;
+                double z = 0.0;
+                for (int cc = 0; cc < 32; ++cc)
+                    z = fma((double)__bfloat162float(xr[cc]), (double)__bfloat162float(Wg[cc * H + h]), z);
+                const double g = 2.0 / (1.0 + exp(-z));
+                gw.x = (float)g;
+                gw.y = (float)(g - (double)gw.x);
+            }
+            const int src = ((int)(threadIdx.x & 31u) / TPR) * TPR;
+            gw.x = __shfl_sync(0xffffffffu, gw.x, src);
+            gw.y = __shfl_sync(0xffffffffu, gw.y, src);
+        }
         if (valid) {
             raw[0] = ldg_stream8(q + in_off + i0);
             raw[1] = ldg_stream8(q + in_off + HALF + i0);
@@ -74,7 +92,6 @@ __global__ void __launch_bounds__(256) decode_prologue_kernel(
             if (HAS_VE) {
                 raw[6] = ldg_stream8(ve + in_off + i0);
                 raw[7] = ldg_stream8(ve + in_off + HALF + i0);
-                gw = gate[row];
             }
         } else {
 #pragma unroll
@@ -104,32 +121,45 @@ __global__ void __launch_bounds__(256) decode_prologue_kernel(
     }
 }
 
-// bf16 bits -> fp32 for DPL consecutive elements starting at p (DPL = 4 or 2).
+// DPL consecutive bf16 features as raw bits: 8 bytes (DPL = 4) or 4 bytes (DPL = 2).
 template <int DPL>
-__device__ __forceinline__ void load_bf16(const __nv_bfloat16* p, float (&f)[DPL]) {
-    if constexpr (DPL == 4) {
-        const uint2 u = *reinterpret_cast<const uint2*>(p);
+struct Raw;
+template <>
+struct Raw<4> {
+    uint2 u;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = *reinterpret_cast<const uint2*>(p); }
+    __device__ __forceinline__ void zero() { u = make_uint2(0u, 0u); }
+    __device__ __forceinline__ void unpack(float (&f)[4]) const {
         f[0] = __uint_as_float(u.x << 16);
         f[1] = __uint_as_float(u.x & 0xffff0000u);
         f[2] = __uint_as_float(u.y << 16);
         f[3] = __uint_as_float(u.y & 0xffff0000u);
-    } else {
-        const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+    }
+};
+template <>
+struct Raw<2> {
+    uint32_t u;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = *reinterpret_cast<const uint32_t*>(p); }
+    __device__ __forceinline__ void zero() { u = 0u; }
+    __device__ __forceinline__ void unpack(float (&f)[2]) const {
         f[0] = __uint_as_float(u << 16);
         f[1] = __uint_as_float(u & 0xffff0000u);
     }
-}
+};
 
 // Attention of the new token over one chunk of cached keys.  Grid B*H*n_chunks, 4 warps; the
-// lanes of a warp split the D features (D/32 each), and each warp takes every fourth key of the
-// chunk, four keys at a time so the four dot-product reductions overlap.  Partial results:
-// part[(row * n_chunks + chunk) * (D + 2) + d] = sum_j p_j v'_j[d], [.. + D] = sum_j p_j.
+// lanes of a warp split the D features (D/32 each).  Per iteration the block takes 32 keys, eight
+// per warp (keys w, w+4, ..., w+28 of the block): the warp loads their K and V pieces first, then
+// reduces the eight dot products together, so sixteen loads per lane are in flight at once.
+// Partial results: part[(row * n_chunks + chunk) * (D + 2) + d] = sum_j p_j v'_j[d],
+// [.. + D] = sum_j p_j.
 template <int D>
 __global__ void __launch_bounds__(128) decode_attn_kernel(
     const __nv_bfloat16* __restrict__ qh, const __nv_bfloat16* __restrict__ k_cache,
     const __nv_bfloat16* __restrict__ v_cache, float* __restrict__ part, int H, int Tmax, int lo,
     int n_keys, int n_chunks, float c1, float c2) {
     constexpr int DPL = D / 32;          // features per lane
+    constexpr int U = 8;                 // keys per warp per iteration
     const int row = (int)(blockIdx.x / (unsigned)n_chunks);    // b*H + h
     const int chunk = (int)(blockIdx.x - (unsigned)row * (unsigned)n_chunks);
     const int b = row / H;
@@ -138,7 +168,11 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
     __shared__ float s_o[4][D];
     __shared__ float s_l[4];
     float qf[DPL];
-    load_bf16<DPL>(qh + (long long)row * D + lane * DPL, qf);
+    {
+        Raw<DPL> rq;
+        rq.load(qh + (long long)row * D + lane * DPL);
+        rq.unpack(qf);
+    }
     float o[DPL];
 #pragma unroll
     for (int e = 0; e < DPL; ++e) o[e] = 0.f;
@@ -148,33 +182,39 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
     const long long stride = (long long)H * D;              // between consecutive positions
     const __nv_bfloat16* kbase = k_cache + ((long long)b * Tmax + lo) * stride + (long long)h * D + lane * DPL;
     const __nv_bfloat16* vbase = v_cache + ((long long)b * Tmax + lo) * stride + (long long)h * D + lane * DPL;
-    for (int j0 = key_begin + warp; j0 < key_end; j0 += 16) {
-        float s[4];
-        bool live[4];
+    for (int j0 = key_begin + warp; j0 < key_end; j0 += 4 * U) {
+        Raw<DPL> rk[U], rv[U];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < U; ++u) {
             const int j = j0 + 4 * u;
-            live[u] = j < key_end;
-            s[u] = 0.f;
-            if (live[u]) {
-                float kf[DPL];
-                load_bf16<DPL>(kbase + (long long)j * stride, kf);
-#pragma unroll
-                for (int e = 0; e < DPL; ++e) s[u] = fmaf(qf[e], kf[e], s[u]);
+            if (j < key_end) {
+                rk[u].load(kbase + (long long)j * stride);
+                rv[u].load(vbase + (long long)j * stride);
+            } else {
+                rk[u].zero();
+                rv[u].zero();
             }
+        }
+        float s[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            float kf[DPL];
+            rk[u].unpack(kf);
+            s[u] = 0.f;
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) s[u] = fmaf(qf[e], kf[e], s[u]);
         }
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1)
 #pragma unroll
-            for (int u = 0; u < 4; ++u) s[u] += __shfl_xor_sync(0xffffffffu, s[u], m);
+            for (int u = 0; u < U; ++u) s[u] += __shfl_xor_sync(0xffffffffu, s[u], m);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            if (!live[u]) continue;
-            const int j = j0 + 4 * u;
+        for (int u = 0; u < U; ++u) {
+            if (j0 + 4 * u >= key_end) continue;
             const float p = ex2_approx(fmaf(s[u], c1, -c2));
             l += p;
             float vf[DPL];
-            load_bf16<DPL>(vbase + (long long)j * stride, vf);
+            rv[u].unpack(vf);
 #pragma unroll
             for (int e = 0; e < DPL; ++e) o[e] = fmaf(p, vf[e], o[e]);
         }

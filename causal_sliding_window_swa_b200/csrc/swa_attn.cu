@@ -465,9 +465,9 @@ int swa_attn_fwd(const void* q, const void* k, const void* v, const void* ve, co
 
 // ------------------------------------------------------------- decode step with a KV cache
 //
-// Workspace: qhat of the new token (B*H*D bf16) | gate (B*H float2, value-embedding layers) |
-// chunk partials (B*H*n_chunks*(D+2) fp32), each section 1024-byte aligned; n_chunks covers the
-// largest window the call can see, min(window, Tmax) keys.
+// Workspace: qhat of the new token (B*H*D bf16) | chunk partials (B*H*n_chunks*(D+2) fp32), each
+// section 1024-byte aligned; n_chunks covers the largest window the call can see, min(window,
+// Tmax) keys.
 
 size_t swa_attn_decode_workspace_bytes(int B, int Tmax, int H, int D, int has_ve, int window) {
     Shape s;
@@ -475,8 +475,8 @@ size_t swa_attn_decode_workspace_bytes(int B, int Tmax, int H, int D, int has_ve
     const long long rows = (long long)B * H;
     const int W = (window <= 0 || window >= Tmax) ? Tmax : window;
     const long long n_chunks = (W + swa::kDecodeChunk - 1) / swa::kDecodeChunk;
-    return round_up((size_t)rows * D * 2) + (has_ve ? round_up((size_t)rows * sizeof(float2)) : 0) +
-           round_up((size_t)(rows * n_chunks * (D + 2)) * sizeof(float));
+    (void)has_ve;
+    return round_up((size_t)rows * D * 2) + round_up((size_t)(rows * n_chunks * (D + 2)) * sizeof(float));
 }
 
 int swa_attn_decode(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
@@ -499,15 +499,7 @@ int swa_attn_decode(const void* q, const void* k, const void* v, const void* ve,
     const int rows = B * H;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     bf* qh = reinterpret_cast<bf*>(ws);
-    float2* gate = reinterpret_cast<float2*>(ws + round_up((size_t)rows * D * 2));
-    float* part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(gate) +
-                                           (has_ve ? round_up((size_t)rows * sizeof(float2)) : 0));
-    if (has_ve) {
-        // the gate rows of one step are (b, h): gate_x is (B, 32)
-        const int gblocks = std::max(1, std::min((rows + 255) / 256, 148 * 8));
-        swa::gate_kernel<<<gblocks, 256, 0, st>>>(static_cast<const bf*>(gate_x), static_cast<const bf*>(Wg),
-                                                   gate, rows, H, make_fastdiv(H));
-    }
+    float* part = reinterpret_cast<float*>(ws + round_up((size_t)rows * D * 2));
     {
         const int rows_per_block = 256 / (D / 8);
         const int blocks = std::max(1, std::min((rows + rows_per_block - 1) / rows_per_block, 148 * 8));
@@ -515,20 +507,26 @@ int swa_attn_decode(const void* q, const void* k, const void* v, const void* ve,
         const bf* kp = static_cast<const bf*>(k);
         const bf* vp = static_cast<const bf*>(v);
         const bf* vep = static_cast<const bf*>(ve);
+        const bf* gx = static_cast<const bf*>(gate_x);
+        const bf* wg = static_cast<const bf*>(Wg);
         bf* kc = static_cast<bf*>(k_cache);
         bf* vc = static_cast<bf*>(v_cache);
         const double base = (double)rope_base, e = (double)eps;
+#define SWA_DEC_PRO(DD, VE)                                                                           \
+    swa::decode_prologue_kernel<DD, VE><<<blocks, 256, 0, st>>>(qp, kp, vp, vep, gx, wg, qh, kc, vc, rows, H, \
+                                                                Tmax, pos, base, e)
         if (D == 128) {
             if (has_ve)
-                swa::decode_prologue_kernel<128, true><<<blocks, 256, 0, st>>>(qp, kp, vp, vep, gate, qh, kc, vc, rows, H, Tmax, pos, base, e);
+                SWA_DEC_PRO(128, true);
             else
-                swa::decode_prologue_kernel<128, false><<<blocks, 256, 0, st>>>(qp, kp, vp, vep, gate, qh, kc, vc, rows, H, Tmax, pos, base, e);
+                SWA_DEC_PRO(128, false);
         } else {
             if (has_ve)
-                swa::decode_prologue_kernel<64, true><<<blocks, 256, 0, st>>>(qp, kp, vp, vep, gate, qh, kc, vc, rows, H, Tmax, pos, base, e);
+                SWA_DEC_PRO(64, true);
             else
-                swa::decode_prologue_kernel<64, false><<<blocks, 256, 0, st>>>(qp, kp, vp, vep, gate, qh, kc, vc, rows, H, Tmax, pos, base, e);
+                SWA_DEC_PRO(64, false);
         }
+#undef SWA_DEC_PRO
     }
     const int W = (window <= 0 || window >= Tmax) ? Tmax : window;
     const int lo = std::max(0, pos - W + 1);

@@ -119,7 +119,7 @@ def test_decode_workspace_and_validation():
     n = swa.swa_attn_decode_workspace_bytes(2, 1000, 3, 64, 0, 0)
     chunks = (1000 + 127) // 128
     assert n == 1024 + ((2 * 3 * chunks * 66 * 4 + 1023) // 1024) * 1024
-    assert swa.swa_attn_decode_workspace_bytes(2, 1000, 3, 64, 1, 200) > swa.swa_attn_decode_workspace_bytes(2, 1000, 3, 64, 0, 200)
+    assert swa.swa_attn_decode_workspace_bytes(2, 1000, 3, 64, 0, 200) < n
     assert swa.swa_attn_decode_workspace_bytes(2, 1000, 3, 96, 0, 0) == 0
     need = swa.swa_attn_decode_workspace_bytes(1, 16, 1, 64, 0, 0)
     base = dict(q=A, k=A, v=A, ve=None, gate_x=None, Wg=None, k_cache=A, v_cache=A, out=A, lse=A,
