@@ -90,23 +90,6 @@ __global__ void rope_table_kernel(float4* __restrict__ tab32, double2* __restric
     }
 }
 
-__device__ __forceinline__ uint4 ldg_stream(const void* p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
-
-__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-    }
-}
-
 __device__ __forceinline__ uint2 ldg_stream8(const void* p) {
     uint2 r;
     asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
@@ -144,11 +127,6 @@ __device__ __forceinline__ double rsqrt_newton(double y) {
 // [-8, +7] fp32 ulps of x.
 __device__ __forceinline__ bool near_midpoint_8ulp(float x) {
     return ((__float_as_uint(x) + 8u - 0x8000u) & 0xfff0u) == 0u;
-}
-
-// True if a bf16 rounding midpoint lies within [-16, +15] fp32 ulps of x.
-__device__ __forceinline__ bool near_midpoint_16ulp(float x) {
-    return ((__float_as_uint(x) + 16u - 0x8000u) & 0xffe0u) == 0u;
 }
 
 // One group of D/8 consecutive threads handles one (b, t, h) row.  Thread c of the group owns
