@@ -41,6 +41,17 @@ def _configure(lib):
                                         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_double, ctypes.c_double,
                                         ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P]
+    lib.swa_oracle_forward_gqa.restype = ctypes.c_int
+    lib.swa_oracle_forward_gqa.argtypes = [P, P, P, P, P, ctypes.c_int, P, ctypes.c_int, P,
+                                           ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                           ctypes.c_double, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, ctypes.c_int, P, ctypes.c_int64, P, P]
+    lib.swa_oracle_prologue_gqa.restype = ctypes.c_int
+    lib.swa_oracle_prologue_gqa.argtypes = [P, P, P, P, P, ctypes.c_int, P, ctypes.c_int, P,
+                                            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, ctypes.c_double, ctypes.c_double,
+                                            ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P]
     lib.swa_oracle_threads.restype = ctypes.c_int
     lib.swa_oracle_round_bf16.restype = ctypes.c_double
     lib.swa_oracle_round_bf16.argtypes = [ctypes.c_double]
@@ -104,8 +115,9 @@ def forward(inputs: Dict, window: int, rope_base: float = 10000.0, eps: float = 
             window_convention: int = 0, rows=None):
     """Attention forward of one layer.
 
-    inputs: dict with q, k, v bf16 (B,T,H,D) and, for value-embedding layers, ids (B,T),
-    table [vocab, H*D], x (B,T,C), Wg [32,H].
+    inputs: dict with q bf16 (B,T,H,D), k, v bf16 (B,T,Hkv,D) (Hkv divides H; query head h reads
+    key/value head h // (H // Hkv); Hkv == H is the multi-head layer) and, for value-embedding
+    layers, ids (B,T), table [vocab, Hkv*D], x (B,T,C), Wg [32,Hkv].
     parity=True rounds qhat, khat, v' to bf16 after the fp64 prologue (pure fp64 otherwise).
     rope/qknorm switch the prologue steps off (test-only, for the library special case).
     rows: None for every row, else flat query ids ((b*H + h)*T + i).
@@ -129,10 +141,18 @@ def forward(inputs: Dict, window: int, rope_base: float = 10000.0, eps: float = 
         n = int(rows_a.size)
         out = np.empty((n, D), dtype=np.float64)
         lse = np.empty((n,), dtype=np.float64)
-    rc = lib.swa_oracle_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(ids), _ptr(table), vocab,
-                                _ptr(x), C, _ptr(Wg), B, T, H, D, int(window),
-                                float(rope_base), float(eps), int(parity), int(rope), int(qknorm),
-                                int(window_convention), _ptr(rows_a), n, _ptr(out), _ptr(lse))
+    Hkv = int(k.shape[2])
+    if Hkv == H:
+        rc = lib.swa_oracle_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(ids), _ptr(table), vocab,
+                                    _ptr(x), C, _ptr(Wg), B, T, H, D, int(window),
+                                    float(rope_base), float(eps), int(parity), int(rope), int(qknorm),
+                                    int(window_convention), _ptr(rows_a), n, _ptr(out), _ptr(lse))
+    else:
+        rc = lib.swa_oracle_forward_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(ids), _ptr(table), vocab,
+                                        _ptr(x), C, _ptr(Wg), B, T, H, Hkv, D, int(window),
+                                        float(rope_base), float(eps), int(parity), int(rope),
+                                        int(qknorm), int(window_convention), _ptr(rows_a), n,
+                                        _ptr(out), _ptr(lse))
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     return out, lse
@@ -140,17 +160,24 @@ def forward(inputs: Dict, window: int, rope_base: float = 10000.0, eps: float = 
 
 def prologue(inputs: Dict, rope_base: float = 10000.0, eps: float = 1e-6, *,
              parity: bool = False, rope: bool = True, qknorm: bool = True):
-    """qhat, khat, v' as fp64 (B,T,H,D) arrays (the steps before the attention)."""
+    """qhat (B,T,H,D), khat and v' (B,T,Hkv,D) as fp64 arrays (the steps before the attention)."""
     lib = _load()
     q, k, v = _bits(inputs["q"]), _bits(inputs["k"]), _bits(inputs["v"])
     B, T, H, D = q.shape
+    Hkv = int(k.shape[2])
     ids, table, vocab, x, C, Wg = _ve_args(inputs)
     qh = np.empty((B, T, H, D), dtype=np.float64)
-    kh = np.empty_like(qh)
-    vp = np.empty_like(qh)
-    rc = lib.swa_oracle_prologue(_ptr(q), _ptr(k), _ptr(v), _ptr(ids), _ptr(table), vocab,
-                                 _ptr(x), C, _ptr(Wg), B, T, H, D, float(rope_base), float(eps),
-                                 int(parity), int(rope), int(qknorm), _ptr(qh), _ptr(kh), _ptr(vp))
+    kh = np.empty((B, T, Hkv, D), dtype=np.float64)
+    vp = np.empty_like(kh)
+    if Hkv == H:
+        rc = lib.swa_oracle_prologue(_ptr(q), _ptr(k), _ptr(v), _ptr(ids), _ptr(table), vocab,
+                                     _ptr(x), C, _ptr(Wg), B, T, H, D, float(rope_base), float(eps),
+                                     int(parity), int(rope), int(qknorm), _ptr(qh), _ptr(kh), _ptr(vp))
+    else:
+        rc = lib.swa_oracle_prologue_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(ids), _ptr(table), vocab,
+                                         _ptr(x), C, _ptr(Wg), B, T, H, Hkv, D, float(rope_base),
+                                         float(eps), int(parity), int(rope), int(qknorm), _ptr(qh),
+                                         _ptr(kh), _ptr(vp))
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     return qh, kh, vp

@@ -159,23 +159,29 @@ int swa_oracle_threads(void) {
 }
 
 /*
- * q, k, v       bf16 bit patterns, (B, T, H, D) contiguous.
- * ids, table    VE token ids (B, T) and table [vocab, H*D] bf16; ids == NULL means no VE.
+ * q             bf16 bit patterns, (B, T, H, D) contiguous: H query heads.
+ * k, v          bf16 bit patterns, (B, T, Hkv, D): Hkv key/value heads, Hkv divides H; query head
+ *               h reads key/value head h / (H / Hkv) (grouped-query attention; Hkv == H is the
+ *               ordinary multi-head layer).
+ * ids, table    VE token ids (B, T) and table [vocab, Hkv*D] bf16; ids == NULL means no VE.
  * x, C          x (B, T, C) bf16; the gate reads channels 0..31.
- * Wg            [32, H] bf16.
+ * Wg            [32, Hkv] bf16.
  * window        <= 0 or >= T: full causal.
  * rows/n_rows   flat query ids ((b*H + h)*T + i), sorted ascending; rows == NULL: every row.
  * out           rows == NULL: (B, T, H, D) fp64; else [n_rows, D].
  * lse           rows == NULL: (B, H, T) fp64;   else [n_rows].
  * Returns 0, or -1 on bad arguments / allocation failure.
  */
-int swa_oracle_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                       const int64_t* ids, const uint16_t* table, int vocab,
-                       const uint16_t* x, int C, const uint16_t* Wg,
-                       int B, int T, int H, int D, int window, double rope_base, double eps,
-                       int round_bf16, int use_rope, int use_qknorm, int window_convention,
-                       const int64_t* rows, int64_t n_rows, double* out, double* lse) {
+int swa_oracle_forward_gqa(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                           const int64_t* ids, const uint16_t* table, int vocab,
+                           const uint16_t* x, int C, const uint16_t* Wg,
+                           int B, int T, int H, int Hkv, int D, int window, double rope_base,
+                           double eps, int round_bf16, int use_rope, int use_qknorm,
+                           int window_convention, const int64_t* rows, int64_t n_rows,
+                           double* out, double* lse) {
     if (B < 1 || T < 1 || H < 1 || D < 2 || (D % 2) != 0) return -1;
+    if (Hkv < 1 || Hkv > H || (H % Hkv) != 0) return -1;
+    const int G = H / Hkv;
     if (ids != NULL && (table == NULL || x == NULL || Wg == NULL || C < 32 || vocab < 1)) return -1;
     if (ids != NULL && !ids_in_range(ids, (int64_t)B * T, vocab)) return -1;
     const int W = (window <= 0 || window >= T) ? T : window;
@@ -196,12 +202,13 @@ int swa_oracle_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v,
         int64_t r1 = r0 + 1;
         while (r1 < n_rows && (rows ? rows[r1] : r1) / T == bh) ++r1;
         const int b = (int)(bh / H), h = (int)(bh % H);
+        const int hk = h / G;                       /* this query head's key/value head */
 
         #pragma omp parallel for schedule(static)
         for (int t = 0; t < T; ++t) {
-            prologue_qk(k, T, H, D, b, t, h, rope_base, eps, use_rope, use_qknorm, round_bf16,
+            prologue_qk(k, T, Hkv, D, b, t, hk, rope_base, eps, use_rope, use_qknorm, round_bf16,
                         kh + (size_t)t * D);
-            prologue_v(v, ids, table, x, C, Wg, T, H, D, b, t, h, round_bf16, vp + (size_t)t * D);
+            prologue_v(v, ids, table, x, C, Wg, T, Hkv, D, b, t, hk, round_bf16, vp + (size_t)t * D);
         }
 
         int bad = 0;
@@ -242,26 +249,53 @@ int swa_oracle_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v,
     return rc;
 }
 
-/* The prologue alone, for the pins on RoPE / RMS / gate: qhat, khat, v' as fp64 (B,T,H,D). */
+/* The multi-head layer: every tensor has H heads. */
+int swa_oracle_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                       const int64_t* ids, const uint16_t* table, int vocab,
+                       const uint16_t* x, int C, const uint16_t* Wg,
+                       int B, int T, int H, int D, int window, double rope_base, double eps,
+                       int round_bf16, int use_rope, int use_qknorm, int window_convention,
+                       const int64_t* rows, int64_t n_rows, double* out, double* lse) {
+    return swa_oracle_forward_gqa(q, k, v, ids, table, vocab, x, C, Wg, B, T, H, H, D, window,
+                                  rope_base, eps, round_bf16, use_rope, use_qknorm,
+                                  window_convention, rows, n_rows, out, lse);
+}
+
+/* The prologue alone, for the pins on RoPE / RMS / gate: qhat (B,T,H,D), khat and v'
+ * (B,T,Hkv,D) as fp64. */
+int swa_oracle_prologue_gqa(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                            const int64_t* ids, const uint16_t* table, int vocab,
+                            const uint16_t* x, int C, const uint16_t* Wg,
+                            int B, int T, int H, int Hkv, int D, double rope_base, double eps,
+                            int round_bf16, int use_rope, int use_qknorm,
+                            double* qh, double* kh, double* vp) {
+    if (B < 1 || T < 1 || H < 1 || D < 2 || (D % 2) != 0) return -1;
+    if (Hkv < 1 || Hkv > H || (H % Hkv) != 0) return -1;
+    if (ids != NULL && (table == NULL || x == NULL || Wg == NULL || C < 32 || vocab < 1)) return -1;
+    if (ids != NULL && !ids_in_range(ids, (int64_t)B * T, vocab)) return -1;
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t) {
+            for (int h = 0; h < H; ++h)
+                prologue_qk(q, T, H, D, b, t, h, rope_base, eps, use_rope, use_qknorm, round_bf16,
+                            qh + (((size_t)b * T + t) * H + h) * (size_t)D);
+            for (int h = 0; h < Hkv; ++h) {
+                size_t off = (((size_t)b * T + t) * Hkv + h) * (size_t)D;
+                prologue_qk(k, T, Hkv, D, b, t, h, rope_base, eps, use_rope, use_qknorm, round_bf16, kh + off);
+                prologue_v(v, ids, table, x, C, Wg, T, Hkv, D, b, t, h, round_bf16, vp + off);
+            }
+        }
+    return 0;
+}
+
 int swa_oracle_prologue(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                         const int64_t* ids, const uint16_t* table, int vocab,
                         const uint16_t* x, int C, const uint16_t* Wg,
                         int B, int T, int H, int D, double rope_base, double eps,
                         int round_bf16, int use_rope, int use_qknorm,
                         double* qh, double* kh, double* vp) {
-    if (B < 1 || T < 1 || H < 1 || D < 2 || (D % 2) != 0) return -1;
-    if (ids != NULL && (table == NULL || x == NULL || Wg == NULL || C < 32 || vocab < 1)) return -1;
-    if (ids != NULL && !ids_in_range(ids, (int64_t)B * T, vocab)) return -1;
-    #pragma omp parallel for collapse(2) schedule(static)
-    for (int b = 0; b < B; ++b)
-        for (int t = 0; t < T; ++t)
-            for (int h = 0; h < H; ++h) {
-                size_t off = (((size_t)b * T + t) * H + h) * (size_t)D;
-                prologue_qk(q, T, H, D, b, t, h, rope_base, eps, use_rope, use_qknorm, round_bf16, qh + off);
-                prologue_qk(k, T, H, D, b, t, h, rope_base, eps, use_rope, use_qknorm, round_bf16, kh + off);
-                prologue_v(v, ids, table, x, C, Wg, T, H, D, b, t, h, round_bf16, vp + off);
-            }
-    return 0;
+    return swa_oracle_prologue_gqa(q, k, v, ids, table, vocab, x, C, Wg, B, T, H, H, D, rope_base,
+                                   eps, round_bf16, use_rope, use_qknorm, qh, kh, vp);
 }
 
 /* Exposed for the rounding pin: double -> bf16 value, ties to even. */

@@ -29,6 +29,7 @@ MUTANTS = {
     "lse drops max": ("*lse = M + log(L);", "*lse = log(L);"),
     "bf16 rounding truncates": ("double r = nearbyint(ldexp(m, 8));", "double r = trunc(ldexp(m, 8));"),
     "rope second component swapped": ("x[i + half] = a * s + b * c;", "x[i + half] = b * s + a * c;"),
+    "gqa head mapping modulo": ("const int hk = h / G;", "const int hk = h % Hkv;"),
 }
 
 PIN_FUNCS = [
@@ -44,6 +45,7 @@ PIN_FUNCS = [
     pins.test_rms_unit_when_eps_zero_and_closed_form_otherwise,
     pins.test_gate_is_two_sigmoid_per_head_in_open_interval,
     pins.test_round_bf16_ties_to_even_without_double_rounding,
+    lambda: pins.test_gqa_equals_multihead_with_repeated_kv_heads(6, 2, 13, True),
 ]
 
 

@@ -322,3 +322,43 @@ def test_row_subset_equals_full_rows():
     h = (rows // s.T) % s.H
     i = rows % s.T
     assert np.array_equal(o, full[b, i, h]) and np.array_equal(l, lfull[b, h, i])
+
+
+# ---------------------------------------------------------------- grouped-query attention
+# With Hkv key/value heads shared by groups of H / Hkv query heads, query head h reads key/value
+# head h // (H / Hkv).  Repeating every key/value head (and its value-embedding table block and
+# gate column) H / Hkv times gives a multi-head layer with the same arithmetic in the same order:
+# the two must agree bit for bit.
+
+def _repeat_kv(d, G):
+    r = dict(d)
+    r["k"] = d["k"].repeat_interleave(G, dim=2)
+    r["v"] = d["v"].repeat_interleave(G, dim=2)
+    if "table" in d:
+        V, HkvD = d["table"].shape
+        Hkv = d["Wg"].shape[1]
+        D = HkvD // Hkv
+        r["table"] = d["table"].view(V, Hkv, D).repeat_interleave(G, dim=1).reshape(V, Hkv * G * D).contiguous()
+        r["Wg"] = d["Wg"].repeat_interleave(G, dim=1).contiguous()
+    return r
+
+
+@pytest.mark.parametrize("H,Hkv,window,ve", [(6, 2, 13, True), (4, 1, 0, False), (6, 3, 1, True)])
+def test_gqa_equals_multihead_with_repeated_kv_heads(H, Hkv, window, ve):
+    s = workloads.LayerShape(B=2, T=40, H=H, D=16, window=window, ve=ve, seed=31, kv_heads=Hkv, vocab=50,
+                             model_dim=48)
+    d = workloads.make_layer(s)
+    assert d["k"].shape[2] == Hkv and d["q"].shape[2] == H
+    o_g, l_g = oracle.forward(d, window, parity=True)
+    o_m, l_m = oracle.forward(_repeat_kv(d, H // Hkv), window, parity=True)
+    assert np.array_equal(o_g, o_m) and np.array_equal(l_g, l_m)
+    qh, kh, vp = oracle.prologue(d, parity=True)
+    qm, km, vm = oracle.prologue(_repeat_kv(d, H // Hkv), parity=True)
+    assert kh.shape[2] == Hkv and np.array_equal(qh, qm)
+    assert np.array_equal(kh, km[:, :, :: H // Hkv]) and np.array_equal(vp, vm[:, :, :: H // Hkv])
+
+
+def test_gqa_rejects_heads_that_do_not_divide():
+    s = workloads.LayerShape(B=1, T=8, H=6, D=16, window=0, ve=False, seed=1, kv_heads=4)
+    with pytest.raises(ValueError):
+        oracle.forward(workloads.make_layer(s), 0)

@@ -44,6 +44,11 @@ class LayerShape:
     name: str = ""
     vocab: int = VOCAB
     model_dim: int = 0   # channels of x (defaults to H*D)
+    kv_heads: int = 0    # key/value heads (grouped-query attention); 0 means H
+
+    @property
+    def Hkv(self) -> int:
+        return self.kv_heads if self.kv_heads > 0 else self.H
 
     @property
     def C(self) -> int:
@@ -99,19 +104,21 @@ def _bf16_normal(gen: torch.Generator, shape, std: float = 1.0) -> torch.Tensor:
 def draw_layer(gen: torch.Generator, s: LayerShape) -> Dict[str, torch.Tensor]:
     """Draw one layer's inputs from ``gen`` in a fixed order: q, k, v, then (VE) ids, table, x, Wg.
 
-    Returns CPU tensors: q, k, v bf16 (B,T,H,D); for VE layers also ids int64 (B,T),
-    table bf16 [vocab, H*D], x bf16 (B,T,C), Wg bf16 [32, H].
+    Returns CPU tensors: q bf16 (B,T,H,D), k, v bf16 (B,T,Hkv,D); for VE layers also ids int64
+    (B,T), table bf16 [vocab, Hkv*D], x bf16 (B,T,C), Wg bf16 [32, Hkv].  With Hkv == H (the
+    default) the draws are those of the multi-head layer.
     """
     shp = (s.B, s.T, s.H, s.D)
+    kv_shp = (s.B, s.T, s.Hkv, s.D)
     d: Dict[str, torch.Tensor] = {}
     d["q"] = _bf16_normal(gen, shp)
-    d["k"] = _bf16_normal(gen, shp)
-    d["v"] = _bf16_normal(gen, shp)
+    d["k"] = _bf16_normal(gen, kv_shp)
+    d["v"] = _bf16_normal(gen, kv_shp)
     if s.ve:
         d["ids"] = torch.randint(0, s.vocab, (s.B, s.T), generator=gen, dtype=torch.int64)
-        d["table"] = _bf16_normal(gen, (s.vocab, s.H * s.D))
+        d["table"] = _bf16_normal(gen, (s.vocab, s.Hkv * s.D))
         d["x"] = _bf16_normal(gen, (s.B, s.T, s.C))
-        d["Wg"] = _bf16_normal(gen, (GATE_CHANNELS, s.H), std=WG_STD)
+        d["Wg"] = _bf16_normal(gen, (GATE_CHANNELS, s.Hkv), std=WG_STD)
     return d
 
 
@@ -136,8 +143,8 @@ def gpu_side_inputs(d: Dict[str, torch.Tensor]) -> Dict[str, Optional[torch.Tens
     q, k, v = d["q"], d["k"], d["v"]
     if "ids" not in d:
         return dict(q=q, k=k, v=v, ve=None, gate_x=None, Wg=None)
-    B, T, H, D = q.shape
-    ve = d["table"][d["ids"]].view(B, T, H, D)
+    B, T, Hkv, D = k.shape
+    ve = d["table"][d["ids"]].view(B, T, Hkv, D)
     gate_x = d["x"][..., :GATE_CHANNELS].contiguous()
     return dict(q=q, k=k, v=v, ve=ve, gate_x=gate_x, Wg=d["Wg"].contiguous())
 
