@@ -62,6 +62,8 @@ def _load() -> ctypes.CDLL:
     lib.swa_attn_strerror.restype = ctypes.c_char_p
     lib.swa_attn_last_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
     lib.swa_attn_last_device_status.restype = I
+    lib.swa_attn_fwd_gqa.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, F, P]
+    lib.swa_attn_fwd_gqa.restype = I
     lib.swa_attn_decode_workspace_bytes.argtypes = [I, I, I, I, I, I]
     lib.swa_attn_decode_workspace_bytes.restype = Z
     lib.swa_attn_decode.argtypes = [P, P, P, P, P, P, P, P, I, P, P, I, I, I, I, I, F, F, P, Z, P]
@@ -151,6 +153,12 @@ def swa_attn_last_device_status(stream=None) -> Tuple[int, int]:
     return int(rc), int(detail.value)
 
 
+def swa_attn_fwd_gqa(q, k, v, ve, gate_x, Wg, out, lse, B, T, H, Hkv, D, window, rope_base, eps,
+                     stream) -> int:
+    return _lib.swa_attn_fwd_gqa(q, k, v, ve, gate_x, Wg, out, lse, B, T, H, Hkv, D, window, rope_base,
+                                 eps, stream)
+
+
 def swa_attn_decode_workspace_bytes(B, Tmax, H, D, has_ve, window) -> int:
     return int(_lib.swa_attn_decode_workspace_bytes(B, Tmax, H, D, int(has_ve), window))
 
@@ -187,36 +195,43 @@ def _stream_handle(stream):
 
 
 def _check_qkv(q, k, v, ve, gate_x, Wg):
+    """Shapes of a layer call: q (B,T,H,D); k, v and ve (B,T,Hkv,D) with Hkv dividing H (Hkv == H
+    for the multi-head layer); gate_x (B,T,32); Wg [32,Hkv].  Returns (B, T, H, Hkv, D)."""
     import torch
-    if q.dim() != 4:
+    if q.dim() != 4 or k.dim() != 4:
         raise ValueError("q, k, v must be (B, T, H, D)")
-    for name, t in (("q", q), ("k", k), ("v", v), ("ve", ve)):
+    B, T, H, D = q.shape
+    Hkv = k.shape[2]
+    kv_shape = (B, T, Hkv, D)
+    for name, t, shp in (("q", q, tuple(q.shape)), ("k", k, kv_shape), ("v", v, kv_shape), ("ve", ve, kv_shape)):
         if t is None:
             continue
-        if t.shape != q.shape or t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {tuple(q.shape)}")
-    B, T, H, D = q.shape
+        if tuple(t.shape) != shp or t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {shp}")
+    if Hkv < 1 or H % Hkv != 0:
+        raise ValueError("the key/value head count must divide the query head count")
     if ve is not None:
         if gate_x is None or Wg is None:
             raise ValueError("ve, gate_x and Wg go together")
         if tuple(gate_x.shape) != (B, T, 32) or gate_x.dtype != torch.bfloat16 or not gate_x.is_contiguous():
             raise ValueError("gate_x must be a contiguous bf16 (B, T, 32) tensor")
-        if tuple(Wg.shape) != (32, H) or Wg.dtype != torch.bfloat16 or not Wg.is_contiguous():
-            raise ValueError("Wg must be a contiguous bf16 [32, H] tensor")
+        if tuple(Wg.shape) != (32, Hkv) or Wg.dtype != torch.bfloat16 or not Wg.is_contiguous():
+            raise ValueError(f"Wg must be a contiguous bf16 [32, {Hkv}] tensor")
     elif gate_x is not None or Wg is not None:
         raise ValueError("ve, gate_x and Wg go together")
-    return B, T, H, D
+    return B, T, H, Hkv, D
 
 
 def forward(q, k, v, window: int = 0, ve=None, gate_x=None, Wg=None, rope_base: float = 10000.0,
             eps: float = 1e-6, *, out=None, lse=None, with_lse: bool = True, workspace=None,
             stream=None):
-    """One attention layer.  q, k, v (and ve) bf16 (B,T,H,D) CUDA tensors; gate_x (B,T,32);
-    Wg [32,H].  Returns (out bf16 (B,T,H,D), lse fp32 (B,H,T) or None).
+    """One attention layer.  q bf16 (B,T,H,D); k, v (and ve) bf16 (B,T,Hkv,D) CUDA tensors, Hkv
+    dividing H (grouped-query attention when Hkv < H: C call swa_attn_fwd_gqa); gate_x (B,T,32);
+    Wg [32,Hkv].  Returns (out bf16 (B,T,H,D), lse fp32 (B,H,T) or None).
     ``workspace``: optional uint8 CUDA tensor of at least ``swa_attn_workspace_bytes`` bytes
-    (then nothing is allocated by the library)."""
+    (then nothing is allocated by the library; multi-head layers only)."""
     import torch
-    B, T, H, D = _check_qkv(q, k, v, ve, gate_x, Wg)
+    B, T, H, Hkv, D = _check_qkv(q, k, v, ve, gate_x, Wg)
     if out is None:
         out = torch.empty_like(q)
     if with_lse and lse is None:
@@ -224,6 +239,14 @@ def forward(q, k, v, window: int = 0, ve=None, gate_x=None, Wg=None, rope_base: 
     st = _stream_handle(stream)
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(out), _ptr(lse),
             B, T, H, D, int(window), float(rope_base), float(eps))
+    if Hkv != H:
+        if workspace is not None:
+            raise ValueError("a caller workspace is supported for multi-head layers only")
+        rc = swa_attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(out),
+                              _ptr(lse), B, T, H, Hkv, D, int(window), float(rope_base), float(eps), st)
+        if rc != SWA_OK:
+            raise SwaError(rc, "swa_attn_fwd_gqa")
+        return out, lse
     if workspace is None:
         rc = swa_attn_fwd(*args, st)
     else:
@@ -270,5 +293,5 @@ __all__ = [
     "swa_attn_fwd", "swa_attn_fwd_ws", "swa_attn_fwd_noalloc", "swa_attn_noalloc_scratch_bytes", "swa_attn_workspace_bytes", "swa_attn_workspace_offset", "swa_attn_rope_table", "swa_attn_prologue",
     "swa_attn_attention", "swa_attn_strerror", "swa_attn_last_device_status",
     "swa_attn_set_wait_limit_ms", "swa_attn_selftest_wait", "swa_attn_version",
-    "swa_attn_decode", "swa_attn_decode_workspace_bytes",
+    "swa_attn_decode", "swa_attn_decode_workspace_bytes", "swa_attn_fwd_gqa",
 ]

@@ -79,6 +79,7 @@ struct FwdParams {
     int n_qtiles;          // ceil(T / 128)
     int n_items;           // n_qtiles * H * B
     int chunk_bh;          // (b, h) slices per scheduling chunk
+    int G;                 // query heads per key/value head (1: multi-head; >1: grouped-query)
     float c1;              // log2(e) / sqrt(D): raw score -> log2 units
     float c2;              // M0 * log2(e)
     float m0;              // M0 (natural-log units), added back into the LSE
@@ -288,7 +289,7 @@ __global__ void __launch_bounds__(576, 1)
                 mbar_arrive_expect_tx(fb, (uint32_t)C::TILE_BYTES);
                 for (int ch = 0; ch < C::NCHUNK; ++ch)
                     tma_load_4d(smem_u32(sKV + stage * C::TILE_BYTES + ch * C::CHUNK_BYTES), tm, fb, ch * 64,
-                                m.h, j * C::BN, m.b);
+                                m.h / p.G, j * C::BN, m.b);
                 filled[stage] = true;
                 filled_phase[stage] = phase;
                 if (++stage == (uint32_t)C::NS) {

@@ -216,7 +216,11 @@ __device__ __forceinline__ uint2 gated_add4(const uint2& vw, const uint2& ew, fl
     return make_uint2(w[0], w[1]);
 }
 
-template <int D, bool HAS_VE>
+// PARTS selects the outputs: bit 0 qhat, bit 1 khat and v' (v' only on value-embedding layers).
+// The multi-head layer runs both in one pass (PARTS = 3, rows (b,t,h) of all inputs); with
+// grouped-query attention the query rows (H heads) and the key/value rows (Hkv heads) are two
+// passes over their own row sets, `H` being that pass's head count.
+template <int D, bool HAS_VE, int PARTS = 3>
 __global__ void __launch_bounds__(256, 3) prologue_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
     const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ ve,
@@ -249,14 +253,19 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(
         const long long off = (long long)row * D;
 
         // Every load of this row chunk is issued before any arithmetic.
+        constexpr bool DO_Q = (PARTS & 1) != 0, DO_KV = (PARTS & 2) != 0;
         uint2 raw[8];
         float2 gw = make_float2(0.f, 0.f);
         if (valid) {
-            raw[0] = ldg_stream8(q + off + i0);
-            raw[1] = ldg_stream8(q + off + HALF + i0);
-            raw[2] = ldg_stream8(k + off + i0);
-            raw[3] = ldg_stream8(k + off + HALF + i0);
-            if (HAS_VE) {
+            if (DO_Q) {
+                raw[0] = ldg_stream8(q + off + i0);
+                raw[1] = ldg_stream8(q + off + HALF + i0);
+            }
+            if (DO_KV) {
+                raw[2] = ldg_stream8(k + off + i0);
+                raw[3] = ldg_stream8(k + off + HALF + i0);
+            }
+            if (HAS_VE && DO_KV) {
                 raw[4] = ldg_stream8(v + off + i0);
                 raw[5] = ldg_stream8(v + off + HALF + i0);
                 raw[6] = ldg_stream8(ve + off + i0);
@@ -267,6 +276,11 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(
 #pragma unroll
             for (int e = 0; e < 8; ++e) raw[e] = make_uint2(0u, 0u);
         }
+        if (!DO_Q) raw[0] = raw[1] = make_uint2(0u, 0u);
+        if (!DO_KV || !HAS_VE)
+#pragma unroll
+            for (int e = 4; e < 8; ++e) raw[e] = make_uint2(0u, 0u);
+        if (!DO_KV) raw[2] = raw[3] = make_uint2(0u, 0u);
         float4 cs[4];
         {
             const float4* tp = tab32 + (long long)t * HALF + i0;
@@ -275,14 +289,18 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(
         }
         const double2* t64 = tab64 + (long long)t * HALF + i0;
         uint2 o0, o1, o2, o3;
-        rope_rms_pairs4<D>(raw[0], raw[1], cs, t64, eps, o0, o1);
-        rope_rms_pairs4<D>(raw[2], raw[3], cs, t64, eps, o2, o3);
+        if (DO_Q) rope_rms_pairs4<D>(raw[0], raw[1], cs, t64, eps, o0, o1);
+        if (DO_KV) rope_rms_pairs4<D>(raw[2], raw[3], cs, t64, eps, o2, o3);
         if (valid) {
-            *reinterpret_cast<uint2*>(qh + off + i0) = o0;
-            *reinterpret_cast<uint2*>(qh + off + HALF + i0) = o1;
-            *reinterpret_cast<uint2*>(kh + off + i0) = o2;
-            *reinterpret_cast<uint2*>(kh + off + HALF + i0) = o3;
-            if (HAS_VE) {
+            if (DO_Q) {
+                *reinterpret_cast<uint2*>(qh + off + i0) = o0;
+                *reinterpret_cast<uint2*>(qh + off + HALF + i0) = o1;
+            }
+            if (DO_KV) {
+                *reinterpret_cast<uint2*>(kh + off + i0) = o2;
+                *reinterpret_cast<uint2*>(kh + off + HALF + i0) = o3;
+            }
+            if (HAS_VE && DO_KV) {
                 const double g64 = (double)gw.x + (double)gw.y;
                 *reinterpret_cast<uint2*>(vp + off + i0) = gated_add4(raw[4], raw[6], gw.x, gw.y, g64);
                 *reinterpret_cast<uint2*>(vp + off + HALF + i0) = gated_add4(raw[5], raw[7], gw.x, gw.y, g64);

@@ -63,6 +63,7 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 struct Shape {
     int B, T, H, D;
     long long n;          // B*T*H*D
+    int Hkv;              // key/value heads (H unless grouped-query attention)
 };
 
 int check_sizes(int B, int T, int H, int D, Shape* s) {
@@ -71,7 +72,14 @@ int check_sizes(int B, int T, int H, int D, Shape* s) {
     const long long n = (long long)B * T * H * D;
     if (n >= (1ll << 31)) return SWA_ERR_UNSUPPORTED;
     if (B > 65535 || H > 65535) return SWA_ERR_UNSUPPORTED;   // grid y/z limits
-    *s = Shape{B, T, H, D, n};
+    *s = Shape{B, T, H, D, n, H};
+    return SWA_OK;
+}
+
+// Grouped-query attention: Hkv key/value heads, 1 <= Hkv <= H, Hkv divides H.
+int check_kv_heads(int Hkv, Shape* s) {
+    if (Hkv < 1 || Hkv > s->H || (s->H % Hkv) != 0) return SWA_ERR_INVALID_ARG;
+    s->Hkv = Hkv;
     return SWA_OK;
 }
 
@@ -108,12 +116,13 @@ struct WsLayout {
 WsLayout ws_layout(const Shape& s, bool has_ve) {
     WsLayout w{};
     const size_t tensor = round_up((size_t)s.n * 2);
+    const size_t kv_tensor = round_up((size_t)s.B * s.T * s.Hkv * s.D * 2);
     const size_t pairs = (size_t)s.T * (s.D / 2);
     w.qh = 0;
     w.kh = w.qh + tensor;
-    w.vp = w.kh + tensor;
-    w.gate = w.vp + (has_ve ? tensor : 0);
-    w.tab32 = w.gate + (has_ve ? round_up((size_t)s.B * s.T * s.H * sizeof(float2)) : 0);
+    w.vp = w.kh + kv_tensor;
+    w.gate = w.vp + (has_ve ? kv_tensor : 0);
+    w.tab32 = w.gate + (has_ve ? round_up((size_t)s.B * s.T * s.Hkv * sizeof(float2)) : 0);
     w.tab64 = w.tab32 + round_up(pairs * sizeof(float4));
     w.sched = w.tab64 + round_up(pairs * sizeof(double2));
     w.total = w.sched + kAlign;
@@ -182,15 +191,15 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// A (B,T,H,D) bf16 tensor seen as 4-D {D, H, T, B}; box = 64 features x 1 head x 128 positions,
+// A (B,T,heads,D) bf16 tensor seen as 4-D {D, heads, T, B}; box = 64 features x 1 head x 128 positions,
 // 128-byte swizzle (the canonical K-major / MN-major shared-memory atom of the tensor core).
 // Positions past T read as zeros.
-bool make_tile_map(CUtensorMap* m, const void* base, const Shape& s) {
+bool make_tile_map(CUtensorMap* m, const void* base, const Shape& s, int heads) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    const cuuint64_t dims[4] = {(cuuint64_t)s.D, (cuuint64_t)s.H, (cuuint64_t)s.T, (cuuint64_t)s.B};
-    const cuuint64_t strides[3] = {(cuuint64_t)s.D * 2, (cuuint64_t)s.H * s.D * 2,
-                                   (cuuint64_t)s.T * s.H * s.D * 2};
+    const cuuint64_t dims[4] = {(cuuint64_t)s.D, (cuuint64_t)heads, (cuuint64_t)s.T, (cuuint64_t)s.B};
+    const cuuint64_t strides[3] = {(cuuint64_t)s.D * 2, (cuuint64_t)heads * s.D * 2,
+                                   (cuuint64_t)s.T * heads * s.D * 2};
     const cuuint32_t box[4] = {64, 1, 128, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
@@ -227,12 +236,13 @@ int launch_prologue(const void* q, const void* k, const void* v, const void* ve,
     using bf = __nv_bfloat16;
     const bool has_ve = ve != nullptr;
     const int n_rows = s.B * s.T * s.H;
+    const int n_kv_rows = s.B * s.T * s.Hkv;
     const swa::FastDiv divH = make_fastdiv(s.H), divT = make_fastdiv(s.T);
     float2* gate = reinterpret_cast<float2*>(ws + L.gate);
     if (has_ve) {
-        const int gblocks = (int)std::min<long long>(((long long)n_rows + 255) / 256, 148ll * 8);
+        const int gblocks = (int)std::min<long long>(((long long)n_kv_rows + 255) / 256, 148ll * 8);
         swa::gate_kernel<<<gblocks, 256, 0, st>>>(static_cast<const bf*>(gate_x), static_cast<const bf*>(Wg),
-                                                   gate, n_rows, s.H, divH);
+                                                   gate, n_kv_rows, s.Hkv, make_fastdiv(s.Hkv));
     }
     const long long threads_total = (long long)n_rows * (s.D / 8);
     const int threads = 256;
@@ -249,6 +259,33 @@ int launch_prologue(const void* q, const void* k, const void* v, const void* ve,
     int* sched = reinterpret_cast<int*>(ws + L.sched);
     const unsigned g = (unsigned)blocks;
     const double e = (double)eps;
+    if (s.Hkv != s.H) {
+        // Grouped-query attention: the query rows (H heads) and the key/value rows (Hkv heads) are
+        // two passes over their own rows.
+        const swa::FastDiv divK = make_fastdiv(s.Hkv);
+        const unsigned gk = (unsigned)std::min<long long>(((long long)n_kv_rows * (s.D / 8) + threads - 1) / threads,
+                                                          148ll * 3 * 4);
+#define SWA_PRO_GQA(DD, VE)                                                                                  \
+    swa::prologue_kernel<DD, VE, 1><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, \
+                                                           n_rows, s.T, s.H, divT, divH, e);                 \
+    swa::prologue_kernel<DD, VE, 2><<<gk, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, \
+                                                            n_kv_rows, s.T, s.Hkv, divT, divK, e)
+        if (s.D == 128) {
+            if (has_ve) {
+                SWA_PRO_GQA(128, true);
+            } else {
+                SWA_PRO_GQA(128, false);
+            }
+        } else {
+            if (has_ve) {
+                SWA_PRO_GQA(64, true);
+            } else {
+                SWA_PRO_GQA(64, false);
+            }
+        }
+#undef SWA_PRO_GQA
+        return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+    }
     if (s.D == 128) {
         if (has_ve)
             swa::prologue_kernel<128, true><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, divT, divH, e);
@@ -267,14 +304,16 @@ int launch_attention(int dev, const void* v, bool has_ve, void* out, float* lse,
                      int window, uint8_t* ws, const WsLayout& L, cudaStream_t st) {
     CUtensorMap tq, tk, tv, to;
     const void* vsrc = has_ve ? static_cast<const void*>(ws + L.vp) : v;
-    if (!make_tile_map(&tq, ws + L.qh, s) || !make_tile_map(&tk, ws + L.kh, s) ||
-        !make_tile_map(&tv, vsrc, s) || !make_tile_map(&to, out, s))
+    // q and out have H heads, k and v Hkv heads
+    if (!make_tile_map(&tq, ws + L.qh, s, s.H) || !make_tile_map(&tk, ws + L.kh, s, s.Hkv) ||
+        !make_tile_map(&tv, vsrc, s, s.Hkv) || !make_tile_map(&to, out, s, s.H))
         return SWA_ERR_CUDA;
     swa::FwdParams p{};
     p.B = s.B;
     p.T = s.T;
     p.H = s.H;
     p.W = (window <= 0 || window >= s.T) ? s.T : window;
+    p.G = s.H / s.Hkv;
     p.n_qtiles = (s.T + 127) / 128;
     p.n_items = p.n_qtiles * s.H * s.B;
     // Scheduling chunks of (b, h) slices whose K/V (about 4 T D bytes each) fit in ~40 MB of L2.
@@ -420,11 +459,12 @@ int swa_attn_fwd_ws(const void* q, const void* k, const void* v, const void* ve,
                               stream);
 }
 
-int swa_attn_fwd(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
-                 const void* Wg, void* out, float* lse, int B, int T, int H, int D, int window,
-                 float rope_base, float eps, swa_stream_t stream) {
+int swa_attn_fwd_gqa(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                     const void* Wg, void* out, float* lse, int B, int T, int H, int Hkv, int D,
+                     int window, float rope_base, float eps, swa_stream_t stream) {
     Shape s;
     int rc = check_sizes(B, T, H, D, &s);
+    if (rc == SWA_OK) rc = check_kv_heads(Hkv, &s);
     if (rc == SWA_OK) rc = check_layer_args(q, k, v, ve, gate_x, Wg, rope_base, eps);
     if (rc == SWA_OK) rc = check_outputs(out, lse);
     if (rc != SWA_OK) return rc;
@@ -461,6 +501,13 @@ int swa_attn_fwd(const void* q, const void* k, const void* v, const void* ve, co
     }
     if ((rc = launch_prologue(q, k, v, ve, gate_x, Wg, ws, L, s, eps, st)) != SWA_OK) return rc;
     return launch_attention(dev, v, has_ve, out, lse, s, window, ws, L, st);
+}
+
+int swa_attn_fwd(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                 const void* Wg, void* out, float* lse, int B, int T, int H, int D, int window,
+                 float rope_base, float eps, swa_stream_t stream) {
+    return swa_attn_fwd_gqa(q, k, v, ve, gate_x, Wg, out, lse, B, T, H, H, D, window, rope_base, eps,
+                            stream);
 }
 
 // ------------------------------------------------------------- decode step with a KV cache

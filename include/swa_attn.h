@@ -93,6 +93,20 @@ SWA_API int swa_attn_fwd(const void* q, const void* k, const void* v,
                  int B, int T, int H, int D, int window,
                  float rope_base, float eps, swa_stream_t stream);
 
+/*
+ * Grouped-query attention (the pages size the key/value projection separately, as kv_dim:
+ * intelliparadigm "GPT-2 for $73", model section): as swa_attn_fwd, with q (B,T,H,D) and k, v, ve
+ * (B,T,Hkv,D), gate_x
+ * (B,T,32), Wg [32,Hkv]; Hkv divides H and query head h attends with key/value head h / (H/Hkv).
+ * The prologue runs on the Hkv key/value heads once (not per query head).  Hkv == H is exactly
+ * swa_attn_fwd.  Errors as swa_attn_fwd; SWA_ERR_INVALID_ARG if Hkv does not divide H.
+ */
+SWA_API int swa_attn_fwd_gqa(const void* q, const void* k, const void* v,
+                             const void* ve, const void* gate_x, const void* Wg,
+                             void* out, float* lse,
+                             int B, int T, int H, int Hkv, int D, int window,
+                             float rope_base, float eps, swa_stream_t stream);
+
 /* Bytes of caller workspace swa_attn_fwd_ws() needs for these sizes (0 on invalid sizes). */
 SWA_API size_t swa_attn_workspace_bytes(int B, int T, int H, int D, int has_ve);
 
