@@ -68,6 +68,8 @@ def _load() -> ctypes.CDLL:
     lib.swa_attn_decode_workspace_bytes.restype = Z
     lib.swa_attn_decode.argtypes = [P, P, P, P, P, P, P, P, I, P, P, I, I, I, I, I, F, F, P, Z, P]
     lib.swa_attn_decode.restype = I
+    lib.swa_attn_decode_gqa.argtypes = [P, P, P, P, P, P, P, P, I, P, P, I, I, I, I, I, I, F, F, P, Z, P]
+    lib.swa_attn_decode_gqa.restype = I
     lib.swa_attn_selftest_wait.argtypes = [I, P]
     lib.swa_attn_selftest_wait.restype = I
     lib.swa_attn_set_wait_limit_ms.argtypes = [I]
@@ -258,11 +260,13 @@ def forward(q, k, v, window: int = 0, ve=None, gate_x=None, Wg=None, rope_base: 
 
 def decode(q, k, v, k_cache, v_cache, pos: int, window: int, ve=None, gate_x=None, Wg=None,
            rope_base: float = 1e4, eps: float = 1e-6, out=None, lse=None, workspace=None, stream=None):
-    """One generation step (C call swa_attn_decode) on torch tensors: q, k, v (B,H,D) bf16 of the
-    new token at position ``pos``; k_cache, v_cache (B,Tmax,H,D) bf16, updated in place at ``pos``.
+    """One generation step (C call swa_attn_decode, or swa_attn_decode_gqa when k has fewer heads
+    than q) on torch tensors: q (B,H,D), k, v (B,Hkv,D) bf16 of the new token at position ``pos``;
+    k_cache, v_cache (B,Tmax,Hkv,D) bf16, updated in place at ``pos``.
     Returns (out (B,H,D) bf16, lse (B,H) fp32).  Raises SwaError on a nonzero status."""
     import torch
     B, H, D = q.shape
+    Hkv = k.shape[1]
     Tmax = k_cache.shape[1]
     if out is None:
         out = torch.empty_like(q)
@@ -272,10 +276,16 @@ def decode(q, k, v, k_cache, v_cache, pos: int, window: int, ve=None, gate_x=Non
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     st = _stream_handle(stream)
-    rc = swa_attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(k_cache),
-                         _ptr(v_cache), int(pos), _ptr(out), _ptr(lse), B, Tmax, H, D, int(window),
-                         float(rope_base), float(eps), _ptr(workspace),
-                         workspace.numel() * workspace.element_size(), st)
+    if Hkv == H:
+        rc = swa_attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(k_cache),
+                             _ptr(v_cache), int(pos), _ptr(out), _ptr(lse), B, Tmax, H, D, int(window),
+                             float(rope_base), float(eps), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), st)
+    else:
+        rc = _lib.swa_attn_decode_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg),
+                                      _ptr(k_cache), _ptr(v_cache), int(pos), _ptr(out), _ptr(lse), B,
+                                      Tmax, H, Hkv, D, int(window), float(rope_base), float(eps),
+                                      _ptr(workspace), workspace.numel() * workspace.element_size(), st)
     if rc != SWA_OK:
         raise SwaError(rc, "swa_attn_decode")
     return out, lse

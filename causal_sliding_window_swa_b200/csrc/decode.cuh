@@ -25,12 +25,14 @@ namespace swa {
 
 constexpr int kDecodeChunk = 128;        // keys per CTA of the attention kernel
 
-// Prologue of the new token: rows r = b*H + h; D/8 threads per row as in the prefill prologue.
+// Prologue of the new token: rows r = b*H + h (H = the head count of this pass); D/8 threads per
+// row as in the prefill prologue.  PARTS: bit 0 qhat (to the workspace), bit 1 khat and v' (to the
+// caches); grouped-query layers run the query rows and the key/value rows as two passes.
 // The block first builds the RoPE row of position `pos` in shared memory, with the same split as
 // the prefill table (16-bit-significand pieces and the fp64 pair for the fallback).  On
 // value-embedding layers the first thread of each row computes the gate 2 sigmoid(x . Wg[:, h]) in
 // fp64 in the order of the prefill gate kernel, so the value is the same.
-template <int D, bool HAS_VE>
+template <int D, bool HAS_VE, int PARTS = 3>
 __global__ void __launch_bounds__(256) decode_prologue_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
     const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ ve,
@@ -65,9 +67,10 @@ __global__ void __launch_bounds__(256) decode_prologue_kernel(
         const int h = row - b * H;
         const long long in_off = (long long)row * D;
         const long long cache_off = (((long long)b * Tmax + pos) * H + h) * D;
+        constexpr bool DO_Q = (PARTS & 1) != 0, DO_KV = (PARTS & 2) != 0;
         uint2 raw[8];
         float2 gw = make_float2(0.f, 0.f);
-        if (HAS_VE) {
+        if (HAS_VE && DO_KV) {
             // gate of this row by its first thread, then shared with the row's other threads
             if (c == 0 && valid) {
                 const __nv_bfloat16* xr = gate_x + (long long)b * 32;
@@ -82,30 +85,35 @@ __global__ void __launch_bounds__(256) decode_prologue_kernel(
             gw.x = __shfl_sync(0xffffffffu, gw.x, src);
             gw.y = __shfl_sync(0xffffffffu, gw.y, src);
         }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) raw[e] = make_uint2(0u, 0u);
         if (valid) {
-            raw[0] = ldg_stream8(q + in_off + i0);
-            raw[1] = ldg_stream8(q + in_off + HALF + i0);
-            raw[2] = ldg_stream8(k + in_off + i0);
-            raw[3] = ldg_stream8(k + in_off + HALF + i0);
-            raw[4] = ldg_stream8(v + in_off + i0);
-            raw[5] = ldg_stream8(v + in_off + HALF + i0);
-            if (HAS_VE) {
+            if (DO_Q) {
+                raw[0] = ldg_stream8(q + in_off + i0);
+                raw[1] = ldg_stream8(q + in_off + HALF + i0);
+            }
+            if (DO_KV) {
+                raw[2] = ldg_stream8(k + in_off + i0);
+                raw[3] = ldg_stream8(k + in_off + HALF + i0);
+                raw[4] = ldg_stream8(v + in_off + i0);
+                raw[5] = ldg_stream8(v + in_off + HALF + i0);
+            }
+            if (HAS_VE && DO_KV) {
                 raw[6] = ldg_stream8(ve + in_off + i0);
                 raw[7] = ldg_stream8(ve + in_off + HALF + i0);
             }
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) raw[e] = make_uint2(0u, 0u);
         }
         float4 cs4[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) cs4[e] = s_tab32[i0 + e];
         uint2 o0, o1, o2, o3;
-        rope_rms_pairs4<D>(raw[0], raw[1], cs4, s_tab64 + i0, eps, o0, o1);
-        rope_rms_pairs4<D>(raw[2], raw[3], cs4, s_tab64 + i0, eps, o2, o3);
-        if (valid) {
+        if (DO_Q) rope_rms_pairs4<D>(raw[0], raw[1], cs4, s_tab64 + i0, eps, o0, o1);
+        if (DO_KV) rope_rms_pairs4<D>(raw[2], raw[3], cs4, s_tab64 + i0, eps, o2, o3);
+        if (valid && DO_Q) {
             *reinterpret_cast<uint2*>(qh + in_off + i0) = o0;
             *reinterpret_cast<uint2*>(qh + in_off + HALF + i0) = o1;
+        }
+        if (valid && DO_KV) {
             *reinterpret_cast<uint2*>(k_cache + cache_off + i0) = o2;
             *reinterpret_cast<uint2*>(k_cache + cache_off + HALF + i0) = o3;
             if (HAS_VE) {
@@ -156,8 +164,8 @@ struct Raw<2> {
 template <int D>
 __global__ void __launch_bounds__(128) decode_attn_kernel(
     const __nv_bfloat16* __restrict__ qh, const __nv_bfloat16* __restrict__ k_cache,
-    const __nv_bfloat16* __restrict__ v_cache, float* __restrict__ part, int H, int Tmax, int lo,
-    int n_keys, int n_chunks, float c1, float c2) {
+    const __nv_bfloat16* __restrict__ v_cache, float* __restrict__ part, int H, int Hkv, int Tmax,
+    int lo, int n_keys, int n_chunks, float c1, float c2) {
     constexpr int DPL = D / 32;          // features per lane
     constexpr int U = 8;                 // keys per warp per iteration
     const int row = (int)(blockIdx.x / (unsigned)n_chunks);    // b*H + h
@@ -179,9 +187,10 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
     float l = 0.f;
     const int key_begin = chunk * kDecodeChunk;
     const int key_end = min(key_begin + kDecodeChunk, n_keys);
-    const long long stride = (long long)H * D;              // between consecutive positions
-    const __nv_bfloat16* kbase = k_cache + ((long long)b * Tmax + lo) * stride + (long long)h * D + lane * DPL;
-    const __nv_bfloat16* vbase = v_cache + ((long long)b * Tmax + lo) * stride + (long long)h * D + lane * DPL;
+    const int hk = h / (H / Hkv);                           // key/value head of this query head
+    const long long stride = (long long)Hkv * D;            // between consecutive positions
+    const __nv_bfloat16* kbase = k_cache + ((long long)b * Tmax + lo) * stride + (long long)hk * D + lane * DPL;
+    const __nv_bfloat16* vbase = v_cache + ((long long)b * Tmax + lo) * stride + (long long)hk * D + lane * DPL;
     for (int j0 = key_begin + warp; j0 < key_end; j0 += 4 * U) {
         Raw<DPL> rk[U], rv[U];
 #pragma unroll

@@ -526,12 +526,14 @@ size_t swa_attn_decode_workspace_bytes(int B, int Tmax, int H, int D, int has_ve
     return round_up((size_t)rows * D * 2) + round_up((size_t)(rows * n_chunks * (D + 2)) * sizeof(float));
 }
 
-int swa_attn_decode(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
-                    const void* Wg, void* k_cache, void* v_cache, int pos, void* out, float* lse,
-                    int B, int Tmax, int H, int D, int window, float rope_base, float eps,
-                    void* workspace, size_t ws_bytes, swa_stream_t stream) {
+int swa_attn_decode_gqa(const void* q, const void* k, const void* v, const void* ve,
+                        const void* gate_x, const void* Wg, void* k_cache, void* v_cache, int pos,
+                        void* out, float* lse, int B, int Tmax, int H, int Hkv, int D, int window,
+                        float rope_base, float eps, void* workspace, size_t ws_bytes,
+                        swa_stream_t stream) {
     Shape s;
     int rc = check_sizes(B, Tmax, H, D, &s);
+    if (rc == SWA_OK) rc = check_kv_heads(Hkv, &s);
     if (rc == SWA_OK) rc = check_layer_args(q, k, v, ve, gate_x, Wg, rope_base, eps);
     if (rc == SWA_OK) rc = check_outputs(out, lse);
     if (rc != SWA_OK) return rc;
@@ -559,9 +561,21 @@ int swa_attn_decode(const void* q, const void* k, const void* v, const void* ve,
         bf* kc = static_cast<bf*>(k_cache);
         bf* vc = static_cast<bf*>(v_cache);
         const double base = (double)rope_base, e = (double)eps;
-#define SWA_DEC_PRO(DD, VE)                                                                           \
-    swa::decode_prologue_kernel<DD, VE><<<blocks, 256, 0, st>>>(qp, kp, vp, vep, gx, wg, qh, kc, vc, rows, H, \
-                                                                Tmax, pos, base, e)
+        // grouped-query layers: the query rows and the key/value rows (Hkv heads) as two passes
+        const int kv_rows = B * Hkv;
+        const int kv_blocks = std::max(1, std::min((kv_rows + rows_per_block - 1) / rows_per_block, 148 * 8));
+#define SWA_DEC_PRO(DD, VE)                                                                               \
+    do {                                                                                                  \
+    if (Hkv == H) {                                                                                       \
+        swa::decode_prologue_kernel<DD, VE><<<blocks, 256, 0, st>>>(qp, kp, vp, vep, gx, wg, qh, kc, vc, rows, \
+                                                                    H, Tmax, pos, base, e);               \
+    } else {                                                                                              \
+        swa::decode_prologue_kernel<DD, VE, 1><<<blocks, 256, 0, st>>>(qp, kp, vp, vep, gx, wg, qh, kc, vc,   \
+                                                                       rows, H, Tmax, pos, base, e);      \
+        swa::decode_prologue_kernel<DD, VE, 2><<<kv_blocks, 256, 0, st>>>(qp, kp, vp, vep, gx, wg, qh, kc, vc, \
+                                                                          kv_rows, Hkv, Tmax, pos, base, e); \
+    }                                                                                                     \
+    } while (0)
         if (D == 128) {
             if (has_ve)
                 SWA_DEC_PRO(128, true);
@@ -588,13 +602,21 @@ int swa_attn_decode(const void* q, const void* k, const void* v, const void* ve,
     const bf* vcc = static_cast<const bf*>(v_cache);
     bf* o = static_cast<bf*>(out);
     if (D == 128) {
-        swa::decode_attn_kernel<128><<<grid, 128, 0, st>>>(qc, kcc, vcc, part, H, Tmax, lo, n_keys, n_chunks, c1, c2);
+        swa::decode_attn_kernel<128><<<grid, 128, 0, st>>>(qc, kcc, vcc, part, H, Hkv, Tmax, lo, n_keys, n_chunks, c1, c2);
         swa::decode_combine_kernel<128><<<rows, 128, 0, st>>>(part, o, lse, n_chunks, (float)m0);
     } else {
-        swa::decode_attn_kernel<64><<<grid, 128, 0, st>>>(qc, kcc, vcc, part, H, Tmax, lo, n_keys, n_chunks, c1, c2);
+        swa::decode_attn_kernel<64><<<grid, 128, 0, st>>>(qc, kcc, vcc, part, H, Hkv, Tmax, lo, n_keys, n_chunks, c1, c2);
         swa::decode_combine_kernel<64><<<rows, 64, 0, st>>>(part, o, lse, n_chunks, (float)m0);
     }
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+int swa_attn_decode(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                    const void* Wg, void* k_cache, void* v_cache, int pos, void* out, float* lse,
+                    int B, int Tmax, int H, int D, int window, float rope_base, float eps,
+                    void* workspace, size_t ws_bytes, swa_stream_t stream) {
+    return swa_attn_decode_gqa(q, k, v, ve, gate_x, Wg, k_cache, v_cache, pos, out, lse, B, Tmax, H, H, D,
+                               window, rope_base, eps, workspace, ws_bytes, stream);
 }
 
 int swa_attn_selftest_wait(int limit_ms, swa_stream_t stream) {

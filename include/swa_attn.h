@@ -229,6 +229,15 @@ SWA_API int swa_attn_decode(const void* q, const void* k, const void* v, const v
                             int pos, void* out, float* lse, int B, int Tmax, int H, int D,
                             int window, float rope_base, float eps, void* workspace,
                             size_t ws_bytes, swa_stream_t stream);
+/* Grouped-query decode step: as swa_attn_decode with q (B, H, D) and k, v, ve (B, Hkv, D),
+ * gate_x (B, 32), Wg (32, Hkv), caches (B, Tmax, Hkv, D); Hkv divides H and query head h attends
+ * with key/value head h / (H / Hkv).  The workspace size is that of swa_attn_decode for (B, Tmax,
+ * H, D).  SWA_ERR_INVALID_ARG if Hkv does not divide H. */
+SWA_API int swa_attn_decode_gqa(const void* q, const void* k, const void* v, const void* ve,
+                                const void* gate_x, const void* Wg, void* k_cache, void* v_cache,
+                                int pos, void* out, float* lse, int B, int Tmax, int H, int Hkv,
+                                int D, int window, float rope_base, float eps, void* workspace,
+                                size_t ws_bytes, swa_stream_t stream);
 
 /*
  * Failure-detection self-test (no counterpart in the pages).  Enqueues on `stream` one block of

@@ -19,6 +19,9 @@ CASES = [
     workloads.LayerShape(B=2, T=200, H=2, D=128, window=48, ve=True, seed=12, name="decode D128 W48 VE"),
     workloads.LayerShape(B=1, T=300, H=2, D=128, window=1, ve=False, seed=13, name="decode D128 W1"),
     workloads.LayerShape(B=1, T=260, H=1, D=64, window=129, ve=True, seed=14, name="decode D64 W129 VE"),
+    # grouped-query layers: caches with Hkv heads, query head h reads key/value head h / (H/Hkv)
+    workloads.LayerShape(B=2, T=180, H=4, D=64, window=50, ve=True, seed=15, kv_heads=2, name="decode gqa D64 H4/2 W50 VE"),
+    workloads.LayerShape(B=1, T=260, H=6, D=128, window=0, ve=False, seed=16, kv_heads=3, name="decode gqa D128 H6/3 full"),
 ]
 
 
@@ -36,7 +39,7 @@ def _bits(x: np.ndarray) -> torch.Tensor:
 
 def _generate(s, dev):
     B, T, H, D = s.B, s.T, s.H, s.D
-    k_cache = torch.zeros((B, T, H, D), dtype=torch.bfloat16, device="cuda")
+    k_cache = torch.zeros((B, T, s.Hkv, D), dtype=torch.bfloat16, device="cuda")
     v_cache = torch.zeros_like(k_cache)
     out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
