@@ -8,6 +8,8 @@ imports it.
 Two independent implementations live here:
 
 * ``forward`` / ``prologue``: the C oracle (``swa_oracle.c``), one query row at a time, fp64.
+* ``backward``: the gradient of the same layer (chain rule through the five steps in
+  reverse), also in ``swa_oracle.c``.
 * ``brute.py``: a NumPy fp64 restatement that materialises the full T x T score matrix, used
   as the brute-force pin of the C oracle on small shapes.
 
@@ -52,6 +54,12 @@ def _configure(lib):
                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                             ctypes.c_int, ctypes.c_double, ctypes.c_double,
                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P]
+    lib.swa_oracle_backward_gqa.restype = ctypes.c_int
+    lib.swa_oracle_backward_gqa.argtypes = [P, P, P, P, P, ctypes.c_int, P, ctypes.c_int, P,
+                                            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                            ctypes.c_double, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, ctypes.c_int, P, P, P, P, P, P, P, P]
     lib.swa_oracle_threads.restype = ctypes.c_int
     lib.swa_oracle_round_bf16.restype = ctypes.c_double
     lib.swa_oracle_round_bf16.argtypes = [ctypes.c_double]
@@ -181,3 +189,53 @@ def prologue(inputs: Dict, rope_base: float = 10000.0, eps: float = 1e-6, *,
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     return qh, kh, vp
+
+
+def backward(inputs: Dict, dout, window: int, dlse=None, rope_base: float = 10000.0,
+             eps: float = 1e-6, *, parity: bool = False, rope: bool = True, qknorm: bool = True,
+             window_convention: int = 0):
+    """Gradient of ``sum(dout * out) + sum(dlse * lse)`` with respect to the layer's inputs.
+
+    inputs as for ``forward``; dout (B,T,H,D) and dlse (B,H,T) (None for zero) are taken as
+    fp64.  parity=False (the default) is the exact gradient of the fp64 layer; parity=True
+    rounds qhat, khat, v' to bf16 as the forward's parity mode does and passes the gradient
+    straight through the rounding.
+
+    Returns a dict of fp64 arrays: dq (B,T,H,D); dk, dv (B,T,Hkv,D); on value-embedding layers
+    also dve (B,T,Hkv,D) (gradient of the looked-up table row at each position), dx (B,T,32)
+    (the gate's input channels) and dWg [32,Hkv].
+    """
+    lib = _load()
+    q, k, v = _bits(inputs["q"]), _bits(inputs["k"]), _bits(inputs["v"])
+    B, T, H, D = q.shape
+    Hkv = int(k.shape[2])
+    ids, table, vocab, x, C, Wg = _ve_args(inputs)
+    go = np.ascontiguousarray(_as_f64(dout))
+    if go.shape != (B, T, H, D):
+        raise ValueError("dout must be (B, T, H, D)")
+    gl = None
+    if dlse is not None:
+        gl = np.ascontiguousarray(_as_f64(dlse))
+        if gl.shape != (B, H, T):
+            raise ValueError("dlse must be (B, H, T)")
+    grads = dict(dq=np.empty((B, T, H, D)), dk=np.empty((B, T, Hkv, D)),
+                 dv=np.empty((B, T, Hkv, D)))
+    if ids is not None:
+        grads.update(dve=np.empty((B, T, Hkv, D)), dx=np.empty((B, T, 32)),
+                     dWg=np.empty((32, Hkv)))
+    rc = lib.swa_oracle_backward_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(ids), _ptr(table), vocab,
+                                     _ptr(x), C, _ptr(Wg), B, T, H, Hkv, D, int(window),
+                                     float(rope_base), float(eps), int(parity), int(rope),
+                                     int(qknorm), int(window_convention), _ptr(go), _ptr(gl),
+                                     _ptr(grads["dq"]), _ptr(grads["dk"]), _ptr(grads["dv"]),
+                                     _ptr(grads.get("dve")), _ptr(grads.get("dx")),
+                                     _ptr(grads.get("dWg")))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return grads
+
+
+def _as_f64(a) -> np.ndarray:
+    if isinstance(a, np.ndarray):
+        return a.astype(np.float64, copy=False)
+    return a.detach().cpu().double().numpy()

@@ -300,3 +300,285 @@ int swa_oracle_prologue(const uint16_t* q, const uint16_t* k, const uint16_t* v,
 
 /* Exposed for the rounding pin: double -> bf16 value, ties to even. */
 double swa_oracle_round_bf16(double x) { return round_to_bf16(x); }
+
+/* -----------------------------------------------------------------------------------------
+ * Backward: the gradient of the layer, for training.
+ *
+ * The pages train this layer (the speedrun explainer's attention section and the GPT-2
+ * notes train end to end; the forward keeps the log-sum-exp so the backward can rebuild the
+ * softmax).  The backward is the chain rule through the five forward steps above, taken in
+ * reverse, for the scalar loss
+ *
+ *     loss = sum_{b,t,h,d} dout[b,t,h,d] * out[b,t,h,d] + sum_{b,h,t} dlse[b,h,t] * lse[b,h,t].
+ *
+ *   5/4. Attention.  For query row i with visible keys J: P_ij = exp(s_ij - lse_i),
+ *        dP_ij = dout_i . v'_j, delta_i = sum_j P_ij dP_ij (the softmax Jacobian's rank-one
+ *        term), dS_ij = P_ij (dP_ij - delta_i) + P_ij dlse_i (d lse_i / d s_ij = P_ij).
+ *        Then dqhat_i = sum_j dS_ij khat_j / sqrt(D), dkhat_j = sum_i dS_ij qhat_i / sqrt(D),
+ *        dv'_j = sum_i P_ij dout_i.  Under grouped-query attention the key/value gradients
+ *        sum over the query heads that read the head.
+ *   3.   Gate: v' = v + g ve with g = 2 sigma(z), z = sum_{c<32} x_c Wg[c, h]:
+ *        dv = dv', dve = g dv', dz = (dv' . ve) * 2 sigma(z)(1 - sigma(z)),
+ *        dx_c = sum_h dz_h Wg[c, h], dWg[c, h] = sum_{b,t} dz[b,t,h] x[b,t,c].
+ *   2.   RMS: y = r x with r = (mean(x^2) + eps)^(-1/2); d r / d x_e = -r^3 x_e / D, so
+ *        dx = r dy - (r^3 / D) (x . dy) x.
+ *   1.   RoPE rotates each pair by +t theta_i; its transpose rotates by -t theta_i.
+ *
+ * Parity mode (round_bf16 = 1) recomputes qhat, khat, v' rounded to bf16 as the forward does
+ * and passes the gradient straight through the rounding (it has no derivative); pure mode is
+ * the exact gradient of the fp64 layer.
+ * ----------------------------------------------------------------------------------------- */
+
+/* The transpose of rope_inplace.  Rotation by -a equals F R(a) F with F = diag(1, -1) on each
+ * pair, so the second half is negated around the forward rotation (negation is exact). */
+static void rope_transpose_inplace(double* g, int D, int t, double base) {
+    const int half = D / 2;
+    for (int i = half; i < D; ++i) g[i] = -g[i];
+    rope_inplace(g, D, t, base);
+    for (int i = half; i < D; ++i) g[i] = -g[i];
+}
+
+/* dL/d(row of q or k) from dy = dL/d(qhat or khat) for row (b, t, h): rebuilds the rotated,
+ * un-normalised row xr (scratch of D) and applies the RMS and RoPE steps in reverse. */
+static void prologue_qk_backward(const uint16_t* src, int T, int H, int D, int b, int t, int h,
+                                 double base, double eps, int use_rope, int use_qknorm,
+                                 const double* dy, double* dx, double* xr) {
+    const uint16_t* row = src + (((size_t)b * T + t) * H + h) * (size_t)D;
+    for (int d = 0; d < D; ++d) xr[d] = bf16_to_double(row[d]);
+    if (use_rope) rope_inplace(xr, D, t, base);
+    if (use_qknorm) {
+        double sq = 0.0, xdy = 0.0;
+        for (int d = 0; d < D; ++d) {
+            sq += xr[d] * xr[d];
+            xdy += xr[d] * dy[d];
+        }
+        const double r = 1.0 / sqrt(sq / (double)D + eps);
+        const double coef = r * r * r * xdy / (double)D;
+        for (int d = 0; d < D; ++d) dx[d] = r * dy[d] - coef * xr[d];
+    } else {
+        for (int d = 0; d < D; ++d) dx[d] = dy[d];
+    }
+    if (use_rope) rope_transpose_inplace(dx, D, t, base);
+}
+
+static double dot_d(const double* a, const double* b, int D) {
+    double acc = 0.0;
+    for (int d = 0; d < D; ++d) acc += a[d] * b[d];
+    return acc;
+}
+
+/*
+ * Inputs as swa_oracle_forward_gqa, plus
+ *   dout   fp64 (B, T, H, D): dL/d out.
+ *   dlse   fp64 (B, H, T):    dL/d lse, or NULL for zero.
+ * Outputs (fp64, written in full):
+ *   dq            (B, T, H, D)
+ *   dk, dv        (B, T, Hkv, D)
+ *   dve           (B, T, Hkv, D): dL/d(the looked-up value-embedding row at (b, t)); the table's
+ *                 gradient is its scatter-add over ids.  VE layers only (NULL otherwise).
+ *   dx            (B, T, 32): dL/d x[b, t, c] for the 32 gate channels (channels >= 32 do not
+ *                 reach the layer).  VE layers only.
+ *   dWg           [32, Hkv].  VE layers only.
+ * Returns 0, or -1 on bad arguments / allocation failure.
+ */
+int swa_oracle_backward_gqa(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                            const int64_t* ids, const uint16_t* table, int vocab,
+                            const uint16_t* x, int C, const uint16_t* Wg,
+                            int B, int T, int H, int Hkv, int D, int window, double rope_base,
+                            double eps, int round_bf16, int use_rope, int use_qknorm,
+                            int window_convention, const double* dout, const double* dlse,
+                            double* dq, double* dk, double* dv, double* dve, double* dx,
+                            double* dWg) {
+    if (B < 1 || T < 1 || H < 1 || D < 2 || (D % 2) != 0) return -1;
+    if (Hkv < 1 || Hkv > H || (H % Hkv) != 0) return -1;
+    if (dout == NULL || dq == NULL || dk == NULL || dv == NULL) return -1;
+    if (ids != NULL && (table == NULL || x == NULL || Wg == NULL || C < 32 || vocab < 1)) return -1;
+    if (ids != NULL && (dve == NULL || dx == NULL || dWg == NULL)) return -1;
+    if (ids != NULL && !ids_in_range(ids, (int64_t)B * T, vocab)) return -1;
+    const int G = H / Hkv;
+    const int W = (window <= 0 || window >= T) ? T : window;
+    /* Keys j visible to query i are those with i in [j, j + reach]. */
+    const int reach = window_convention == 0 ? W - 1 : W;
+    const double inv_sqrt_d = 1.0 / sqrt((double)D);
+    const size_t TD = (size_t)T * D;
+
+    double* kh = (double*)malloc(sizeof(double) * TD);
+    double* vp = (double*)malloc(sizeof(double) * TD);
+    double* qh = (double*)malloc(sizeof(double) * TD);
+    double* dkh = (double*)malloc(sizeof(double) * TD);
+    double* dvp = (double*)malloc(sizeof(double) * TD);
+    double* dqh = (double*)malloc(sizeof(double) * TD);
+    double* lse = (double*)malloc(sizeof(double) * (size_t)T);
+    double* delta = (double*)malloc(sizeof(double) * (size_t)T);
+    double* dz = (double*)calloc((size_t)B * T * Hkv, sizeof(double));
+    int rc = 0;
+    if (!kh || !vp || !qh || !dkh || !dvp || !dqh || !lse || !delta || !dz) { rc = -1; goto done; }
+
+    for (int b = 0; b < B && rc == 0; ++b) {
+        for (int hk = 0; hk < Hkv && rc == 0; ++hk) {
+            #pragma omp parallel for schedule(static)
+            for (int t = 0; t < T; ++t) {
+                prologue_qk(k, T, Hkv, D, b, t, hk, rope_base, eps, use_rope, use_qknorm,
+                            round_bf16, kh + (size_t)t * D);
+                prologue_v(v, ids, table, x, C, Wg, T, Hkv, D, b, t, hk, round_bf16,
+                           vp + (size_t)t * D);
+            }
+            memset(dkh, 0, sizeof(double) * TD);
+            memset(dvp, 0, sizeof(double) * TD);
+
+            for (int g = 0; g < G; ++g) {
+                const int h = hk * G + g;
+                #pragma omp parallel for schedule(static)
+                for (int i = 0; i < T; ++i)
+                    prologue_qk(q, T, H, D, b, i, h, rope_base, eps, use_rope, use_qknorm,
+                                round_bf16, qh + (size_t)i * D);
+
+                /* Row pass: lse_i, delta_i and dqhat_i, one query row at a time. */
+                int bad = 0;
+                #pragma omp parallel
+                {
+                    double* s = (double*)malloc(sizeof(double) * (size_t)T);
+                    #pragma omp for schedule(dynamic, 8)
+                    for (int i = 0; i < T; ++i) {
+                        if (s == NULL) {
+                            #pragma omp atomic write
+                            bad = 1;
+                            continue;
+                        }
+                        const double* qi = qh + (size_t)i * D;
+                        const double* gi = dout + (((size_t)b * T + i) * H + h) * (size_t)D;
+                        const double gl = dlse ? dlse[((size_t)b * H + h) * T + i] : 0.0;
+                        double M = -INFINITY;
+                        for (int j = 0; j < T; ++j) {
+                            if (!visible(i, j, W, window_convention)) continue;
+                            s[j] = dot_d(qi, kh + (size_t)j * D, D) * inv_sqrt_d;
+                            if (s[j] > M) M = s[j];
+                        }
+                        double L = 0.0;
+                        for (int j = 0; j < T; ++j)
+                            if (visible(i, j, W, window_convention)) L += exp(s[j] - M);
+                        const double li = M + log(L);
+                        double dl = 0.0;
+                        for (int j = 0; j < T; ++j)
+                            if (visible(i, j, W, window_convention))
+                                dl += exp(s[j] - li) * dot_d(gi, vp + (size_t)j * D, D);
+                        lse[i] = li;
+                        delta[i] = dl;
+                        double* dqi = dqh + (size_t)i * D;
+                        for (int d = 0; d < D; ++d) dqi[d] = 0.0;
+                        for (int j = 0; j < T; ++j) {
+                            if (!visible(i, j, W, window_convention)) continue;
+                            const double p = exp(s[j] - li);
+                            const double ds = p * (dot_d(gi, vp + (size_t)j * D, D) - dl) + p * gl;
+                            for (int d = 0; d < D; ++d) dqi[d] += ds * kh[(size_t)j * D + d] * inv_sqrt_d;
+                        }
+                    }
+                    free(s);
+                }
+                if (bad) { rc = -1; break; }
+
+                /* Key pass: dkhat_j and dv'_j, one key row at a time, over the queries that
+                 * see key j. */
+                #pragma omp parallel for schedule(dynamic, 8)
+                for (int j = 0; j < T; ++j) {
+                    const double* kj = kh + (size_t)j * D;
+                    const double* vj = vp + (size_t)j * D;
+                    double* dkj = dkh + (size_t)j * D;
+                    double* dvj = dvp + (size_t)j * D;
+                    const int i_end = (j + reach < T - 1) ? j + reach : T - 1;
+                    for (int i = j; i <= i_end; ++i) {
+                        const double* qi = qh + (size_t)i * D;
+                        const double* gi = dout + (((size_t)b * T + i) * H + h) * (size_t)D;
+                        const double gl = dlse ? dlse[((size_t)b * H + h) * T + i] : 0.0;
+                        const double p = exp(dot_d(qi, kj, D) * inv_sqrt_d - lse[i]);
+                        const double ds = p * (dot_d(gi, vj, D) - delta[i]) + p * gl;
+                        for (int d = 0; d < D; ++d) {
+                            dkj[d] += ds * qi[d] * inv_sqrt_d;
+                            dvj[d] += p * gi[d];
+                        }
+                    }
+                }
+
+                /* dq rows of head h. */
+                #pragma omp parallel
+                {
+                    double* xr = (double*)malloc(sizeof(double) * (size_t)D);
+                    #pragma omp for schedule(static)
+                    for (int i = 0; i < T; ++i) {
+                        if (xr == NULL) {
+                            #pragma omp atomic write
+                            bad = 1;
+                            continue;
+                        }
+                        prologue_qk_backward(q, T, H, D, b, i, h, rope_base, eps, use_rope,
+                                             use_qknorm, dqh + (size_t)i * D,
+                                             dq + (((size_t)b * T + i) * H + h) * (size_t)D, xr);
+                    }
+                    free(xr);
+                }
+                if (bad) { rc = -1; break; }
+            }
+            if (rc != 0) break;
+
+            /* dk, dv and the gate of key/value head hk. */
+            int bad = 0;
+            #pragma omp parallel
+            {
+                double* xr = (double*)malloc(sizeof(double) * (size_t)D);
+                #pragma omp for schedule(static)
+                for (int t = 0; t < T; ++t) {
+                    if (xr == NULL) {
+                        #pragma omp atomic write
+                        bad = 1;
+                        continue;
+                    }
+                    const size_t off = (((size_t)b * T + t) * Hkv + hk) * (size_t)D;
+                    const double* dvt = dvp + (size_t)t * D;
+                    prologue_qk_backward(k, T, Hkv, D, b, t, hk, rope_base, eps, use_rope,
+                                         use_qknorm, dkh + (size_t)t * D, dk + off, xr);
+                    for (int d = 0; d < D; ++d) dv[off + d] = dvt[d];
+                    if (ids != NULL) {
+                        const uint16_t* xt = x + ((size_t)b * T + t) * (size_t)C;
+                        double z = 0.0;
+                        for (int c = 0; c < 32; ++c)
+                            z += bf16_to_double(xt[c]) * bf16_to_double(Wg[(size_t)c * Hkv + hk]);
+                        const double sig = 1.0 / (1.0 + exp(-z));
+                        const int64_t id = ids[(size_t)b * T + t];
+                        const uint16_t* ve = table + (size_t)id * (size_t)Hkv * D + (size_t)hk * D;
+                        double dgate = 0.0;
+                        for (int d = 0; d < D; ++d) {
+                            dve[off + d] = 2.0 * sig * dvt[d];
+                            dgate += dvt[d] * bf16_to_double(ve[d]);
+                        }
+                        dz[((size_t)b * T + t) * Hkv + hk] = dgate * 2.0 * sig * (1.0 - sig);
+                    }
+                }
+                free(xr);
+            }
+            if (bad) rc = -1;
+        }
+    }
+
+    if (rc == 0 && ids != NULL) {
+        /* Gate inputs and weights from dz: dx sums over heads, dWg over positions. */
+        #pragma omp parallel for schedule(static)
+        for (int64_t bt = 0; bt < (int64_t)B * T; ++bt)
+            for (int c = 0; c < 32; ++c) {
+                double acc = 0.0;
+                for (int hk = 0; hk < Hkv; ++hk)
+                    acc += dz[(size_t)bt * Hkv + hk] * bf16_to_double(Wg[(size_t)c * Hkv + hk]);
+                dx[(size_t)bt * 32 + c] = acc;
+            }
+        for (int c = 0; c < 32; ++c)
+            for (int hk = 0; hk < Hkv; ++hk) {
+                double acc = 0.0;
+                for (int64_t bt = 0; bt < (int64_t)B * T; ++bt)
+                    acc += dz[(size_t)bt * Hkv + hk] * bf16_to_double(x[(size_t)bt * C + c]);
+                dWg[(size_t)c * Hkv + hk] = acc;
+            }
+    }
+
+done:
+    free(kh); free(vp); free(qh); free(dkh); free(dvp); free(dqh); free(lse); free(delta); free(dz);
+    return rc;
+}

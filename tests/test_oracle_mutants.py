@@ -11,6 +11,7 @@ import pytest
 
 import oracle
 from oracle import build as obuild
+import tests.test_oracle_backward_pins as bpins
 import tests.test_oracle_pins as pins
 
 MUTANTS = {
@@ -49,14 +50,88 @@ PIN_FUNCS = [
 ]
 
 
-def _failing_pins():
+# Mistakes in the backward (the gradient of the layer); the forward stays correct.
+BACKWARD_MUTANTS = {
+    "bwd row pass drops delta": ("p * (dot_d(gi, vp + (size_t)j * D, D) - dl) + p * gl",
+                                 "p * dot_d(gi, vp + (size_t)j * D, D) + p * gl"),
+    "bwd key pass drops delta": ("p * (dot_d(gi, vj, D) - delta[i]) + p * gl",
+                                 "p * dot_d(gi, vj, D) + p * gl"),
+    "bwd row pass drops dlse": ("- dl) + p * gl;", "- dl);"),
+    "bwd key pass drops dlse": ("- delta[i]) + p * gl;", "- delta[i]);"),
+    "bwd rms correction sign": ("dx[d] = r * dy[d] - coef * xr[d];", "dx[d] = r * dy[d] + coef * xr[d];"),
+    "bwd rms r squared": ("const double coef = r * r * r * xdy", "const double coef = r * r * xdy"),
+    "bwd rope not transposed": (
+        "    for (int i = half; i < D; ++i) g[i] = -g[i];\n    rope_inplace(g, D, t, base);\n"
+        "    for (int i = half; i < D; ++i) g[i] = -g[i];\n",
+        "    rope_inplace(g, D, t, base);\n"),
+    "bwd gate derivative without 1 - sigma": ("dgate * 2.0 * sig * (1.0 - sig)", "dgate * 2.0 * sig"),
+    "bwd ve gradient without gate": ("dve[off + d] = 2.0 * sig * dvt[d];", "dve[off + d] = dvt[d];"),
+    "bwd dx reads Wg transposed": (
+        "acc += dz[(size_t)bt * Hkv + hk] * bf16_to_double(Wg[(size_t)c * Hkv + hk]);",
+        "acc += dz[(size_t)bt * Hkv + hk] * bf16_to_double(Wg[(size_t)hk * 32 + c]);"),
+    "bwd dWg reads x with stride 32": ("bf16_to_double(x[(size_t)bt * C + c])",
+                                       "bf16_to_double(x[(size_t)bt * 32 + c])"),
+    "bwd key pass window off by one": ("const int reach = window_convention == 0 ? W - 1 : W;",
+                                       "const int reach = window_convention == 0 ? W : W;"),
+    "bwd gqa group sum dropped": (
+        "            memset(dkh, 0, sizeof(double) * TD);\n            memset(dvp, 0, sizeof(double) * TD);\n\n"
+        "            for (int g = 0; g < G; ++g) {\n",
+        "            for (int g = 0; g < G; ++g) {\n"
+        "            memset(dkh, 0, sizeof(double) * TD);\n            memset(dvp, 0, sizeof(double) * TD);\n"),
+    "bwd dk without scale": ("dkj[d] += ds * qi[d] * inv_sqrt_d;", "dkj[d] += ds * qi[d];"),
+    "bwd dv weighted by dS": ("dvj[d] += p * gi[d];", "dvj[d] += ds * gi[d];"),
+    "bwd dq from queries": ("dqi[d] += ds * kh[(size_t)j * D + d] * inv_sqrt_d;",
+                            "dqi[d] += ds * qh[(size_t)j * D + d] * inv_sqrt_d;"),
+    "bwd keys not rounded in parity mode": ("                            round_bf16, kh + (size_t)t * D);",
+                                            "                            0, kh + (size_t)t * D);"),
+}
+
+BACKWARD_PIN_FUNCS = [
+    lambda: bpins.test_backward_matches_central_differences(1, 7, 1, 8, 3, True, True, True, True),
+    lambda: bpins.test_backward_matches_central_differences(2, 5, 2, 4, 2, False, True, True, True),
+    lambda: bpins.test_backward_matches_torch_autograd(4, 2, 5, True),
+    lambda: bpins.test_parity_mode_backward_is_straight_through_rounding(2),
+    bpins.test_window_one_closed_form,
+    bpins.test_lse_only_cotangent_leaves_values_untouched,
+    lambda: bpins.test_rms_scale_invariance_makes_dq_orthogonal_to_q(True),
+    lambda: bpins.test_gqa_gradients_are_group_sums_of_repeated_head_gradients(6, 2),
+]
+
+
+def _failing_pins(funcs=None):
     failed = 0
-    for f in PIN_FUNCS:
+    for f in (PIN_FUNCS if funcs is None else funcs):
         try:
             f()
         except (AssertionError, ValueError, FloatingPointError):
             failed += 1
     return failed
+
+
+def _build_mutant(old, new, tmp):
+    src = open(obuild.SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not found: {old!r}"
+    c = os.path.join(tmp, "mutant.c")
+    so = os.path.join(tmp, "libmutant.so")
+    open(c, "w").write(src.replace(old, new))
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fPIC",
+                    "-shared", "-o", so, c, "-lm"], check=True)
+    return so
+
+
+@pytest.mark.parametrize("name", sorted(BACKWARD_MUTANTS))
+def test_planted_backward_mistake_is_caught(name):
+    old, new = BACKWARD_MUTANTS[name]
+    with tempfile.TemporaryDirectory() as tmp:
+        oracle._swap_library(_build_mutant(old, new, tmp))
+        try:
+            assert _failing_pins(BACKWARD_PIN_FUNCS) >= 1, f"no pin caught the planted mistake: {name}"
+        finally:
+            oracle._swap_library(None)
+
+
+def test_unmutated_backward_passes_every_backward_pin():
+    assert _failing_pins(BACKWARD_PIN_FUNCS) == 0
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
