@@ -1,4 +1,4 @@
-"""B200 (sm_100a) causal sliding-window attention forward: Python binding of the C ABI in
+"""B200 (sm_100a) causal sliding-window attention (forward, backward, decode): Python binding of the C ABI in
 ``include/swa_attn.h``.
 
 This module only marshals arguments: every step of the layer (RoPE, RMS QK-norm, the value-
@@ -70,6 +70,14 @@ def _load() -> ctypes.CDLL:
     lib.swa_attn_decode.restype = I
     lib.swa_attn_decode_gqa.argtypes = [P, P, P, P, P, P, P, P, I, P, P, I, I, I, I, I, I, F, F, P, Z, P]
     lib.swa_attn_decode_gqa.restype = I
+    lib.swa_attn_bwd_workspace_bytes.argtypes = [I, I, I, I, I, I]
+    lib.swa_attn_bwd_workspace_bytes.restype = Z
+    lib.swa_attn_bwd_gqa.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
+                                     I, I, I, I, I, I, F, F, P, Z, P]
+    lib.swa_attn_bwd_gqa.restype = I
+    lib.swa_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
+                                 I, I, I, I, I, F, F, P, Z, P]
+    lib.swa_attn_bwd.restype = I
     lib.swa_attn_selftest_wait.argtypes = [I, P]
     lib.swa_attn_selftest_wait.restype = I
     lib.swa_attn_set_wait_limit_ms.argtypes = [I]
@@ -169,6 +177,22 @@ def swa_attn_decode(q, k, v, ve, gate_x, Wg, k_cache, v_cache, pos, out, lse, B,
                     rope_base, eps, workspace, ws_bytes, stream) -> int:
     return _lib.swa_attn_decode(q, k, v, ve, gate_x, Wg, k_cache, v_cache, pos, out, lse, B, Tmax, H, D,
                                 window, rope_base, eps, workspace, ws_bytes, stream)
+
+
+def swa_attn_bwd_workspace_bytes(B, T, H, Hkv, D, has_ve) -> int:
+    return int(_lib.swa_attn_bwd_workspace_bytes(B, T, H, Hkv, D, int(has_ve)))
+
+
+def swa_attn_bwd_gqa(q, k, v, ve, gate_x, Wg, out, lse, dout, dlse, dq, dk, dv, dve, dgate_x, dWg,
+                     B, T, H, Hkv, D, window, rope_base, eps, workspace, ws_bytes, stream) -> int:
+    return _lib.swa_attn_bwd_gqa(q, k, v, ve, gate_x, Wg, out, lse, dout, dlse, dq, dk, dv, dve, dgate_x,
+                                 dWg, B, T, H, Hkv, D, window, rope_base, eps, workspace, ws_bytes, stream)
+
+
+def swa_attn_bwd(q, k, v, ve, gate_x, Wg, out, lse, dout, dlse, dq, dk, dv, dve, dgate_x, dWg,
+                 B, T, H, D, window, rope_base, eps, workspace, ws_bytes, stream) -> int:
+    return _lib.swa_attn_bwd(q, k, v, ve, gate_x, Wg, out, lse, dout, dlse, dq, dk, dv, dve, dgate_x, dWg,
+                             B, T, H, D, window, rope_base, eps, workspace, ws_bytes, stream)
 
 
 def swa_attn_selftest_wait(limit_ms: int, stream=None) -> int:
@@ -291,6 +315,42 @@ def decode(q, k, v, k_cache, v_cache, pos: int, window: int, ve=None, gate_x=Non
     return out, lse
 
 
+def backward(q, k, v, out, lse, dout, window: int = 0, dlse=None, ve=None, gate_x=None, Wg=None,
+             rope_base: float = 10000.0, eps: float = 1e-6, *, workspace=None, stream=None):
+    """Gradient of one layer (C call swa_attn_bwd_gqa) for the loss sum(dout * out) +
+    sum(dlse * lse).  q, k, v, ve, gate_x, Wg as for ``forward``; out bf16 (B,T,H,D) and lse fp32
+    (B,H,T) are that call's outputs; dout bf16 (B,T,H,D); dlse fp32 (B,H,T) or None.
+    Returns a dict: dq bf16 (B,T,H,D), dk, dv bf16 (B,T,Hkv,D) and, on value-embedding layers,
+    dve bf16 (B,T,Hkv,D), dgate_x fp32 (B,T,32), dWg fp32 [32,Hkv].  Raises SwaError on a nonzero
+    status."""
+    import torch
+    B, T, H, Hkv, D = _check_qkv(q, k, v, ve, gate_x, Wg)
+    for name, t in (("out", out), ("dout", dout)):
+        if tuple(t.shape) != (B, T, H, D) or t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {(B, T, H, D)}")
+    for name, t in (("lse", lse), ("dlse", dlse)):
+        if t is None and name == "dlse":
+            continue
+        if tuple(t.shape) != (B, H, T) or t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA fp32 tensor of shape {(B, H, T)}")
+    g = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v))
+    if ve is not None:
+        g.update(dve=torch.empty_like(ve),
+                 dgate_x=torch.empty((B, T, 32), dtype=torch.float32, device=q.device),
+                 dWg=torch.empty((32, Hkv), dtype=torch.float32, device=q.device))
+    need = swa_attn_bwd_workspace_bytes(B, T, H, Hkv, D, ve is not None)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    rc = swa_attn_bwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(out), _ptr(lse),
+                          _ptr(dout), _ptr(dlse), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g.get("dve")),
+                          _ptr(g.get("dgate_x")), _ptr(g.get("dWg")), B, T, H, Hkv, D, int(window),
+                          float(rope_base), float(eps), _ptr(workspace),
+                          workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    if rc != SWA_OK:
+        raise SwaError(rc, "swa_attn_bwd_gqa")
+    return g
+
+
 def check_device_status(stream=None) -> None:
     """Synchronise and raise SwaError if a kernel recorded an error (e.g. a wait timeout)."""
     rc, detail = swa_attn_last_device_status(_stream_handle(stream))
@@ -299,9 +359,10 @@ def check_device_status(stream=None) -> None:
 
 
 __all__ = [
-    "forward", "decode", "check_device_status", "SwaError", "LIB_PATH", "load",
+    "forward", "decode", "backward", "check_device_status", "SwaError", "LIB_PATH", "load",
     "swa_attn_fwd", "swa_attn_fwd_ws", "swa_attn_fwd_noalloc", "swa_attn_noalloc_scratch_bytes", "swa_attn_workspace_bytes", "swa_attn_workspace_offset", "swa_attn_rope_table", "swa_attn_prologue",
     "swa_attn_attention", "swa_attn_strerror", "swa_attn_last_device_status",
     "swa_attn_set_wait_limit_ms", "swa_attn_selftest_wait", "swa_attn_version",
     "swa_attn_decode", "swa_attn_decode_workspace_bytes", "swa_attn_fwd_gqa",
+    "swa_attn_bwd", "swa_attn_bwd_gqa", "swa_attn_bwd_workspace_bytes",
 ]

@@ -1,0 +1,938 @@
+// attn_bwd.cuh -- gradient of the causal sliding-window attention layer on the sm_100a tensor cores.
+//
+// The layer ("Let's reproduce GPT-2 (124M)" notes, section 3; intelliparadigm "GPT-2 for $73",
+// sections 2.2 and 3.2; PaperWeekly repost, "Value Embeddings" paragraph) is
+//   qhat, khat = rms(rope(q)), rms(rope(k));  v' = v + 2 sigmoid(x[:32] . Wg) ve;
+//   out_i = sum_{j in J_i} P_ij v'_j,  P_ij = exp(s_ij - lse_i),  s_ij = qhat_i . khat_j / sqrt(D),
+//   J_i = { j : 0 <= i - j < W }.
+// For the loss sum(dout * out) + sum(dlse * lse) the chain rule gives, per visible pair,
+//   dP_ij = dout_i . v'_j,  dS_ij = P_ij (dP_ij - (delta_i - dlse_i)),  delta_i = dout_i . out_i,
+//   dqhat_i = sum_j dS_ij khat_j / sqrt(D),  dkhat_j = sum_i dS_ij qhat_i / sqrt(D),
+//   dv'_j = sum_i P_ij dout_i,
+// and then the prologue in reverse (RMS, RoPE, gate).  The softmax is rebuilt from the saved
+// log-sum-exp, so no running maximum or sum is needed.
+//
+// Kernels, in launch order (after the forward prologue has recomputed qhat, khat, v'):
+//   bwd_rowstat_kernel    per query row: (lse log2 e, delta - dlse), padded to whole tiles
+//                         with (+inf, 0) so that rows past T get P = 0.
+//   attn_bwd_dq_kernel    one 128-row query tile per item: S = Q K^T and dP = dO V'^T (Q and dO
+//                         copied into tensor memory, K and V' from shared memory), dS by 16
+//                         warps, dQ += dS K with dS fed from tensor memory and K read MN-major.
+//   attn_bwd_dkv_kernel   one 128-row key tile per item, over every query tile (and, under
+//                         grouped-query attention, every query head of the group) that sees it:
+//                         S^T = K Q^T and dP^T = V' dO^T from shared memory, P^T and dS^T by 16
+//                         warps, dV += P^T dO and dK += dS^T Q with P^T / dS^T from tensor memory.
+//   bwd_qk_rows_kernel    dq (dk) = RoPE^T applied to the RMS backward of dqhat (dkhat).
+//   bwd_v_rows_kernel     dv = dv', dve = g dv', dz = (dv' . ve) g (1 - g / 2) per row.
+//   bwd_gate_x_kernel, bwd_wg_partial_kernel, bwd_wg_final_kernel
+//                         dgate_x = dz Wg^T and dWg = gate_x^T dz (fixed summation order).
+// The two tensor-core kernels use seven products per (query tile, key tile) pair instead of
+// five so that neither needs fp32 atomics: dQ is owned by the query-tile kernel, dK and dV by the
+// key-tile kernel.  Every tensor-core operand form here (A from tensor memory or shared memory, B
+// K-major or MN-major, P-style bf16 pairs in tensor memory) is one the forward kernel uses.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace swa {
+
+// 1-D bulk copy global -> shared memory, completing `bytes` on the mbarrier.  Both addresses
+// 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+template <int D>
+struct BwdCfg {
+    static constexpr int NCHUNK = D / 64;              // 128-byte swizzle chunks per row
+    static constexpr int CHUNK_BYTES = 128 * 128;      // 128 rows x 128 B
+    static constexpr int TILE_BYTES = 128 * D * 2;     // one 128 x D bf16 tile
+    static constexpr int SMEM_BAR = 512;
+    static constexpr int THREADS = 576;
+    static constexpr int SOFTMAX_THREADS = 512;
+    static constexpr uint32_t TMEM_COLS = 512;
+    // query-tile kernel: Q | dO | NS-stage ring of K and V' tiles | barriers
+    static constexpr int DQ_NS = (D == 128) ? 4 : 10;
+    static constexpr int DQ_SMEM = 2 * TILE_BYTES + DQ_NS * TILE_BYTES + SMEM_BAR;
+    static constexpr uint32_t DQ_COL_S = 0;            // S, then dS as bf16 pairs
+    static constexpr uint32_t DQ_COL_DP = 128;
+    static constexpr uint32_t DQ_COL_DQ = 256;         // D fp32 columns
+    static constexpr uint32_t DQ_COL_Q = 256 + D;      // D / 2 columns of bf16 pairs
+    static constexpr uint32_t DQ_COL_DO = 256 + D + D / 2;
+    // key-tile kernel: K | V' | NS stages of (Q tile, dO tile, 128 row statistics) | barriers
+    static constexpr int STAGE_BYTES = 2 * TILE_BYTES + 1024;
+    static constexpr int KV_NS = (D == 128) ? 2 : 5;
+    static constexpr int KV_SMEM = 2 * TILE_BYTES + KV_NS * STAGE_BYTES + SMEM_BAR;
+    static constexpr uint32_t KV_COL_ST = 0;           // S^T, then P^T as bf16 pairs
+    static constexpr uint32_t KV_COL_DPT = 128;        // dP^T, then dS^T as bf16 pairs
+    static constexpr uint32_t KV_COL_DV = 256;
+    static constexpr uint32_t KV_COL_DK = 256 + D;
+    static_assert(DQ_COL_DO + D / 2 <= TMEM_COLS, "query-tile kernel exceeds tensor memory");
+    static_assert(KV_COL_DK + D <= TMEM_COLS, "key-tile kernel exceeds tensor memory");
+    static_assert(DQ_SMEM <= 227 * 1024 && KV_SMEM <= 227 * 1024, "shared memory per CTA");
+};
+
+struct BwdParams {
+    int B, T, H, Hkv, G;   // G = H / Hkv query heads per key/value head
+    int W;                 // effective window, 1..T
+    int n_tiles;           // ceil(T / 128): query tiles = key tiles
+    int Tp;                // n_tiles * 128, the row-statistics stride
+    int n_items;
+    int chunk_bh;          // (b, head) slices per scheduling chunk
+    float c1;              // log2(e) / sqrt(D): raw score -> log2 units
+    float inv_sqrt_d;
+    const float2* rowstat; // (B, H, Tp): (lse log2 e, delta - dlse); padding rows (+inf, 0)
+    float* dqh;            // (B, T, H, D) fp32: dL/dqhat
+    float* dkh;            // (B, T, Hkv, D) fp32: dL/dkhat
+    float* dvp;            // (B, T, Hkv, D) fp32: dL/dv'
+    int* sched;            // [0] next item, [1] CTAs done; zero before the launch, reset after
+    unsigned long long wait_limit_ns;
+};
+
+// Wait sites recorded in the status word on timeout (distinct from the forward's).
+enum : unsigned int {
+    kSiteBwdQFull = 40, kSiteBwdQEmpty = 41, kSiteBwdKvFull = 42, kSiteBwdKvEmpty = 43,
+    kSiteBwdSFull = 44, kSiteBwdPFull = 45, kSiteBwdOFull = 46, kSiteBwdOEmpty = 47,
+    kSiteBwdItem = 48, kSiteBwdDrain = 49, kSiteBwdStage = 50
+};
+
+// Query-tile item: tile [q0, q0 + 127] of (b, h) and the key tiles lo..hi of its band; order as
+// in the forward (chunks of (b, h) slices, heaviest tiles first inside a chunk).
+struct BwdQItem {
+    int b, h, q0, lo, hi;
+};
+
+__device__ __forceinline__ BwdQItem bwd_q_item(const BwdParams& p, int it) {
+    BwdQItem m;
+    const int per_chunk = p.chunk_bh * p.n_tiles;
+    const int chunk = it / per_chunk;
+    const int rem = it - chunk * per_chunk;
+    const int first_bh = chunk * p.chunk_bh;
+    const int n_bh = min(p.chunk_bh, p.B * p.H - first_bh);
+    const int qt = p.n_tiles - 1 - rem / n_bh;
+    const int bh = first_bh + rem % n_bh;
+    m.b = bh / p.H;
+    m.h = bh - m.b * p.H;
+    m.q0 = qt * 128;
+    m.lo = max(0, m.q0 - p.W + 1) / 128;
+    m.hi = min(m.q0 + 127, p.T - 1) / 128;
+    return m;
+}
+
+// Key-tile item: tile [k0, k0 + 127] of (b, hk); the queries that see it lie in
+// [k0, k0 + 127 + W - 1], query tiles lo..hi, for each of the G query heads hk G .. hk G + G - 1.
+// Under the causal mask the first key tiles are seen by the most queries, so they go first.
+struct BwdKvItem {
+    int b, hk, k0, lo, hi;
+};
+
+__device__ __forceinline__ BwdKvItem bwd_kv_item(const BwdParams& p, int it) {
+    BwdKvItem m;
+    const int per_chunk = p.chunk_bh * p.n_tiles;
+    const int chunk = it / per_chunk;
+    const int rem = it - chunk * per_chunk;
+    const int first_bh = chunk * p.chunk_bh;
+    const int n_bh = min(p.chunk_bh, p.B * p.Hkv - first_bh);
+    const int kt = rem / n_bh;
+    const int bh = first_bh + rem % n_bh;
+    m.b = bh / p.Hkv;
+    m.hk = bh - m.b * p.Hkv;
+    m.k0 = kt * 128;
+    m.lo = kt;
+    m.hi = min(m.k0 + 127 + p.W - 1, p.T - 1) / 128;
+    return m;
+}
+
+// Byte offset (>> 4) of k-step kk (16 elements of the contraction) inside a K-major tile: 32 bytes
+// inside a 128-byte swizzle chunk, chunks CHUNK_BYTES apart.
+template <int D>
+__device__ __forceinline__ uint64_t kmajor_step(int kk) {
+    return (uint64_t)(((kk >> 2) * BwdCfg<D>::CHUNK_BYTES + (kk & 3) * 32) >> 4);
+}
+
+// ------------------------------------------------------------------- row statistics
+
+// One warp per (b, h, t), t < Tp: delta = dout . out over D (fp32), stored with the log-sum-exp in
+// log2 units.  Block 0 also zeroes the scheduler counters of the two tensor-core kernels.
+template <int D>
+__global__ void bwd_rowstat_kernel(const __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ dout,
+                                   const float* __restrict__ lse, const float* __restrict__ dlse,
+                                   float2* __restrict__ rowstat, int B, int T, int H, int Tp,
+                                   int* __restrict__ sched4) {
+    if (blockIdx.x == 0 && threadIdx.x < 4) sched4[threadIdx.x] = 0;
+    constexpr int E = D / 32;   // elements per lane: 4 or 2
+    const int lane = threadIdx.x & 31;
+    const long long n = (long long)B * H * Tp;
+    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long f = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); f < n; f += warps) {
+        const int t = (int)(f % Tp);
+        const long long bh = f / Tp;
+        if (t >= T) {
+            if (lane == 0) rowstat[f] = make_float2(__int_as_float(0x7f800000), 0.f);
+            continue;
+        }
+        const int h = (int)(bh % H);
+        const long long b = bh / H;
+        const long long row = ((b * T + t) * H + h) * D + lane * E;
+        float acc = 0.f;
+        if constexpr (E == 4) {
+            const uint2 a = *reinterpret_cast<const uint2*>(out + row);
+            const uint2 g = *reinterpret_cast<const uint2*>(dout + row);
+            acc = __uint_as_float(a.x << 16) * __uint_as_float(g.x << 16) +
+                  __uint_as_float(a.x & 0xffff0000u) * __uint_as_float(g.x & 0xffff0000u) +
+                  __uint_as_float(a.y << 16) * __uint_as_float(g.y << 16) +
+                  __uint_as_float(a.y & 0xffff0000u) * __uint_as_float(g.y & 0xffff0000u);
+        } else {
+            const uint32_t a = *reinterpret_cast<const uint32_t*>(out + row);
+            const uint32_t g = *reinterpret_cast<const uint32_t*>(dout + row);
+            acc = __uint_as_float(a << 16) * __uint_as_float(g << 16) +
+                  __uint_as_float(a & 0xffff0000u) * __uint_as_float(g & 0xffff0000u);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) {
+            const long long li = bh * T + t;
+            const float gl = dlse ? dlse[li] : 0.f;
+            rowstat[f] = make_float2(lse[li] * 1.4426950408889634f, acc - gl);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ query-tile kernel (dQ)
+
+template <int D>
+__global__ void __launch_bounds__(576, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                       const BwdParams p) {
+    using C = BwdCfg<D>;
+    constexpr int NS = C::DQ_NS;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    if ((smem_u32(smem_raw) & 1023u) != 0u) {   // uniform: every thread leaves before any barrier
+        if (threadIdx.x == 0) record_error(kErrLayout, 0);
+        return;
+    }
+    uint8_t* sQ = smem_raw;
+    uint8_t* sdO = sQ + C::TILE_BYTES;
+    uint8_t* sKV = sdO + C::TILE_BYTES;          // NS tiles: K_j, V'_j alternately
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NS * C::TILE_BYTES);
+    uint64_t* b_qfull = bars + 0;                // Q and dO tiles landed
+    uint64_t* b_qempty = bars + 1;               // both copied into tensor memory
+    uint64_t* b_ofull = bars + 2;                // dQ of the item complete
+    uint64_t* b_oempty = bars + 3;               // dQ read by the epilogue
+    uint64_t* b_mdrain = bars + 4;
+    uint64_t* b_itfull = bars + 5;               // [2]
+    uint64_t* b_itempty = bars + 7;              // [2]
+    uint64_t* b_sfull = bars + 9;                // S and dP of the current key tile ready
+    uint64_t* b_pfull = bars + 10;               // dS written to tensor memory
+    uint64_t* b_kvfull = bars + 11;              // [NS]
+    uint64_t* b_kvempty = bars + 11 + NS;        // [NS]
+    int* s_item = reinterpret_cast<int*>(bars + 11 + 2 * NS);   // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_item + 2);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    constexpr int kMmaWarp = 0;
+    constexpr int kProducerWarp = 1;
+    constexpr int kSoftmaxWarp0 = 2;
+    constexpr uint32_t kItemConsumers = 1 + 16;
+
+    if (threadIdx.x == 32) {
+        mbar_init(smem_u32(b_qfull), 1);
+        mbar_init(smem_u32(b_qempty), 1);
+        mbar_init(smem_u32(b_ofull), 1);
+        mbar_init(smem_u32(b_oempty), C::SOFTMAX_THREADS);
+        mbar_init(smem_u32(b_mdrain), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(b_itfull + i), 1);
+            mbar_init(smem_u32(b_itempty + i), kItemConsumers);
+        }
+        mbar_init(smem_u32(b_sfull), 1);
+        mbar_init(smem_u32(b_pfull), C::SOFTMAX_THREADS);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(smem_u32(b_kvfull + s), 1);
+            mbar_init(smem_u32(b_kvempty + s), 1);
+        }
+        fence_barrier_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == kProducerWarp && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_do);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const unsigned long long lim = p.wait_limit_ns;
+
+    if (warp == kProducerWarp) {
+        // ========================= scheduler + TMA producer =========================
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            uint32_t filled_phase[NS];
+            bool filled[NS];
+            for (int s = 0; s < NS; ++s) filled[s] = false, filled_phase[s] = 0;
+            uint32_t q_uses = 0;
+            bool ok = true;
+            auto load_kv = [&](const CUtensorMap* tm, const BwdQItem& m, int j) -> bool {
+                if (!mbar_wait(smem_u32(b_kvempty + stage), phase ^ 1u, lim, kSiteBwdKvEmpty)) return false;
+                const uint32_t fb = smem_u32(b_kvfull + stage);
+                mbar_arrive_expect_tx(fb, (uint32_t)C::TILE_BYTES);
+                for (int ch = 0; ch < C::NCHUNK; ++ch)
+                    tma_load_4d(smem_u32(sKV + stage * C::TILE_BYTES + ch * C::CHUNK_BYTES), tm, fb, ch * 64,
+                                m.h / p.G, j * 128, m.b);
+                filled[stage] = true;
+                filled_phase[stage] = phase;
+                if (++stage == (uint32_t)NS) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                return true;
+            };
+            for (uint32_t k = 0; ok; ++k) {
+                int it = atomicAdd(p.sched, 1);
+                if (it >= p.n_items) it = -1;
+                const uint32_t slot = k & 1u;
+                if (!(ok = mbar_wait(smem_u32(b_itempty + slot), ((k >> 1) & 1u) ^ 1u, lim, kSiteBwdItem))) break;
+                s_item[slot] = it;
+                mbar_arrive(smem_u32(b_itfull + slot));
+                if (it < 0) break;
+                const BwdQItem m = bwd_q_item(p, it);
+                if (q_uses > 0 && !(ok = mbar_wait(smem_u32(b_qempty), (q_uses - 1) & 1u, lim, kSiteBwdQEmpty)))
+                    break;
+                {
+                    const uint32_t qb = smem_u32(b_qfull);
+                    mbar_arrive_expect_tx(qb, 2u * (uint32_t)C::TILE_BYTES);
+                    for (int ch = 0; ch < C::NCHUNK; ++ch) {
+                        tma_load_4d(smem_u32(sQ + ch * C::CHUNK_BYTES), &tm_q, qb, ch * 64, m.h, m.q0, m.b);
+                        tma_load_4d(smem_u32(sdO + ch * C::CHUNK_BYTES), &tm_do, qb, ch * 64, m.h, m.q0, m.b);
+                    }
+                    ++q_uses;
+                }
+                // The MMA thread's order: K_j, then V'_j, for each key tile j.
+                for (int j = m.lo; ok && j <= m.hi; ++j) ok = load_kv(&tm_k, m, j) && load_kv(&tm_v, m, j);
+            }
+            if (ok && atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1) {
+                p.sched[0] = 0;
+                p.sched[1] = 0;
+            }
+            if (q_uses > 0) mbar_wait(smem_u32(b_qfull), (q_uses - 1) & 1u, lim, kSiteBwdDrain);
+            for (int s = 0; s < NS; ++s)
+                if (filled[s]) mbar_wait(smem_u32(b_kvfull + s), filled_phase[s], lim, kSiteBwdDrain);
+        }
+    } else if (warp == kMmaWarp) {
+        // ============================== MMA issuer ==============================
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);   // S, dP: N = 128 keys
+            constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, true);     // dQ: B = K MN-major
+            const uint64_t dq_src = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+            const uint64_t ddo_src = smem_desc_sw128(smem_u32(sdO), 16, 1024);
+            const uint64_t dkv_k = smem_desc_sw128(smem_u32(sKV), 16, 1024);
+            const uint64_t dkv_mn = smem_desc_sw128(smem_u32(sKV), C::CHUNK_BYTES, 1024);
+            uint32_t stage = 0, phase = 0;
+            uint32_t p_cnt = 0;   // dS hand-overs consumed
+            uint32_t uses = 0;    // items done
+            auto acquire = [&](uint32_t& s) -> bool {
+                s = stage;
+                const bool r = mbar_wait(smem_u32(b_kvfull + stage), phase, lim, kSiteBwdKvFull);
+                if (++stage == (uint32_t)NS) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                return r;
+            };
+            bool ok = true;
+            for (uint32_t k = 0; ok; ++k) {
+                const uint32_t slot = k & 1u;
+                if (!(ok = mbar_wait(smem_u32(b_itfull + slot), (k >> 1) & 1u, lim, kSiteBwdItem))) break;
+                const int it = s_item[slot];
+                mbar_arrive(smem_u32(b_itempty + slot));
+                if (it < 0) break;
+                const BwdQItem m = bwd_q_item(p, it);
+                // Q and dO into tensor memory (after the previous item's products on the same pipe).
+                if (!(ok = mbar_wait(smem_u32(b_qfull), uses & 1u, lim, kSiteBwdQFull))) break;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    tmem_cp_128x256b(tmem + C::DQ_COL_Q + 8u * kk, dq_src + kmajor_step<D>(kk));
+                    tmem_cp_128x256b(tmem + C::DQ_COL_DO + 8u * kk, ddo_src + kmajor_step<D>(kk));
+                }
+                mma_commit(smem_u32(b_qempty));
+                for (int j = m.lo; ok && j <= m.hi; ++j) {
+                    uint32_t sk = 0, sv = 0;
+                    if (!(ok = acquire(sk))) break;
+                    const uint64_t bk = dkv_k + (uint64_t)((sk * C::TILE_BYTES) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ts(tmem + C::DQ_COL_S, tmem + C::DQ_COL_Q + 8u * kk, bk + kmajor_step<D>(kk), idesc_s,
+                               kk > 0 ? 1u : 0u);
+                    if (!(ok = acquire(sv))) break;
+                    const uint64_t bv = dkv_k + (uint64_t)((sv * C::TILE_BYTES) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ts(tmem + C::DQ_COL_DP, tmem + C::DQ_COL_DO + 8u * kk, bv + kmajor_step<D>(kk), idesc_s,
+                               kk > 0 ? 1u : 0u);
+                    mma_commit(smem_u32(b_sfull));
+                    mma_commit(smem_u32(b_kvempty + sv));
+                    if (!(ok = mbar_wait(smem_u32(b_pfull), p_cnt & 1u, lim, kSiteBwdPFull))) break;
+                    ++p_cnt;
+                    if (j == m.lo && uses > 0 &&
+                        !(ok = mbar_wait(smem_u32(b_oempty), (uses - 1) & 1u, lim, kSiteBwdOEmpty)))
+                        break;
+                    tc_fence_after();
+                    // dQ += dS K_j: K = 128 keys in steps of 16; dS of keys 32 c + i at column 32 c + i / 2.
+                    const uint64_t bkm = dkv_mn + (uint64_t)((sk * C::TILE_BYTES) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tmem + C::DQ_COL_DQ, tmem + C::DQ_COL_S + (kk >> 1) * 32 + (kk & 1) * 8,
+                               bkm + (uint64_t)((kk * 16 * 128) >> 4), idesc_dq, (j > m.lo || kk > 0) ? 1u : 0u);
+                    mma_commit(smem_u32(b_kvempty + sk));
+                    if (j == m.hi) mma_commit(smem_u32(b_ofull));
+                }
+                ++uses;
+            }
+            mma_commit(smem_u32(b_mdrain));
+            mbar_wait(smem_u32(b_mdrain), 0, lim, kSiteBwdDrain);
+        }
+        __syncwarp();
+    } else {
+        // ============================ dS + epilogue ============================
+        const int cq = (warp - kSoftmaxWarp0) >> 2;   // key / output column quarter
+        const int r = ((warp & 3) << 5) + lane;       // tile row = tensor-memory lane
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        uint32_t s_cnt = 0, o_uses = 0;
+        bool ok = true;
+        for (uint32_t k = 0; ok; ++k) {
+            const uint32_t slot = k & 1u;
+            int it = 0;
+            if (lane == 0) {
+                ok = mbar_wait(smem_u32(b_itfull + slot), (k >> 1) & 1u, lim, kSiteBwdItem);
+                it = s_item[slot];
+                mbar_arrive(smem_u32(b_itempty + slot));
+            }
+            ok = __all_sync(0xffffffffu, ok);
+            it = __shfl_sync(0xffffffffu, it, 0);
+            if (!ok || it < 0) break;
+            const BwdQItem m = bwd_q_item(p, it);
+            const int qi = m.q0 + r;
+            const float2 rs = p.rowstat[((long long)m.b * p.H + m.h) * p.Tp + qi];
+            const float nl = -rs.x, dl = rs.y;
+            for (int j = m.lo; j <= m.hi; ++j) {
+                const bool w = mbar_wait(smem_u32(b_sfull), s_cnt & 1u, lim, kSiteBwdSFull);
+                ok = __all_sync(0xffffffffu, w);
+                if (!ok) break;
+                ++s_cnt;
+                tc_fence_after();
+                const int k0 = j * 128 + 32 * cq;
+                uint32_t sv[2][16], dv[2][16], pk[16];
+                const uint32_t colS = C::DQ_COL_S + 32u * (uint32_t)cq;
+                const uint32_t colP = C::DQ_COL_DP + 32u * (uint32_t)cq;
+                tmem_ld16(tmem + lane_base + colS, sv[0]);
+                tmem_ld16(tmem + lane_base + colS + 16u, sv[1]);
+                tmem_ld16(tmem + lane_base + colP, dv[0]);
+                tmem_ld16(tmem + lane_base + colP + 16u, dv[1]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {
+#pragma unroll
+                    for (int e = 0; e < 16; e += 2) {
+                        const int kv = k0 + 16 * hb + e;
+                        float p0 = ex2_approx(fmaf(__uint_as_float(sv[hb][e]), p.c1, nl));
+                        float p1 = ex2_approx(fmaf(__uint_as_float(sv[hb][e + 1]), p.c1, nl));
+                        if ((unsigned)(qi - kv) >= (unsigned)p.W) p0 = 0.f;
+                        if ((unsigned)(qi - kv - 1) >= (unsigned)p.W) p1 = 0.f;
+                        const float d0 = p0 * (__uint_as_float(dv[hb][e]) - dl);
+                        const float d1 = p1 * (__uint_as_float(dv[hb][e + 1]) - dl);
+                        pk[8 * hb + (e >> 1)] = pack_bf16x2(d0, d1);
+                    }
+                }
+                tmem_st16(tmem + lane_base + colS, pk);
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(smem_u32(b_pfull));
+            }
+            if (!ok) break;
+            {
+                const bool w = mbar_wait(smem_u32(b_ofull), o_uses & 1u, lim, kSiteBwdOFull);
+                ok = __all_sync(0xffffffffu, w);
+            }
+            if (!ok) break;
+            tc_fence_after();
+            constexpr int OQ = D / 4;   // output columns per thread: 32 or 16
+            uint32_t ov[OQ];
+            tmem_ld16(tmem + lane_base + C::DQ_COL_DQ + (uint32_t)(OQ * cq), *reinterpret_cast<uint32_t(*)[16]>(ov));
+            if constexpr (OQ == 32)
+                tmem_ld16(tmem + lane_base + C::DQ_COL_DQ + (uint32_t)(OQ * cq) + 16u,
+                          *reinterpret_cast<uint32_t(*)[16]>(ov + 16));
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(smem_u32(b_oempty));
+            ++o_uses;
+            if (qi < p.T) {
+                float4* dst = reinterpret_cast<float4*>(p.dqh + (((long long)m.b * p.T + qi) * p.H + m.h) * D + OQ * cq);
+#pragma unroll
+                for (int e = 0; e < OQ / 4; ++e)
+                    dst[e] = make_float4(__uint_as_float(ov[4 * e]) * p.inv_sqrt_d,
+                                         __uint_as_float(ov[4 * e + 1]) * p.inv_sqrt_d,
+                                         __uint_as_float(ov[4 * e + 2]) * p.inv_sqrt_d,
+                                         __uint_as_float(ov[4 * e + 3]) * p.inv_sqrt_d);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- key-tile kernel (dK, dV)
+
+template <int D>
+__global__ void __launch_bounds__(576, 1)
+    attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                        const BwdParams p) {
+    using C = BwdCfg<D>;
+    constexpr int NS = C::KV_NS;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    if ((smem_u32(smem_raw) & 1023u) != 0u) {
+        if (threadIdx.x == 0) record_error(kErrLayout, 0);
+        return;
+    }
+    uint8_t* sK = smem_raw;
+    uint8_t* sV = sK + C::TILE_BYTES;
+    uint8_t* sSt = sV + C::TILE_BYTES;           // NS stages: Q tile | dO tile | 128 x float2
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sSt + NS * C::STAGE_BYTES);
+    uint64_t* b_kfull = bars + 0;                // K and V' tiles of the item landed
+    uint64_t* b_kempty = bars + 1;               // the item's products are done with them
+    uint64_t* b_ofull = bars + 2;
+    uint64_t* b_oempty = bars + 3;
+    uint64_t* b_mdrain = bars + 4;
+    uint64_t* b_itfull = bars + 5;               // [2]
+    uint64_t* b_itempty = bars + 7;              // [2]
+    uint64_t* b_sfull = bars + 9;
+    uint64_t* b_pfull = bars + 10;
+    uint64_t* b_stfull = bars + 11;              // [NS]
+    uint64_t* b_stempty = bars + 11 + NS;        // [NS]
+    int* s_item = reinterpret_cast<int*>(bars + 11 + 2 * NS);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_item + 2);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    constexpr int kMmaWarp = 0;
+    constexpr int kProducerWarp = 1;
+    constexpr int kSoftmaxWarp0 = 2;
+    constexpr uint32_t kItemConsumers = 1 + 16;
+
+    if (threadIdx.x == 32) {
+        mbar_init(smem_u32(b_kfull), 1);
+        mbar_init(smem_u32(b_kempty), 1);
+        mbar_init(smem_u32(b_ofull), 1);
+        mbar_init(smem_u32(b_oempty), C::SOFTMAX_THREADS);
+        mbar_init(smem_u32(b_mdrain), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(b_itfull + i), 1);
+            mbar_init(smem_u32(b_itempty + i), kItemConsumers);
+        }
+        mbar_init(smem_u32(b_sfull), 1);
+        mbar_init(smem_u32(b_pfull), C::SOFTMAX_THREADS);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(smem_u32(b_stfull + s), 1);
+            mbar_init(smem_u32(b_stempty + s), 1);
+        }
+        fence_barrier_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == kProducerWarp && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_do);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const unsigned long long lim = p.wait_limit_ns;
+
+    if (warp == kProducerWarp) {
+        // ========================= scheduler + TMA producer =========================
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            uint32_t filled_phase[NS];
+            bool filled[NS];
+            for (int s = 0; s < NS; ++s) filled[s] = false, filled_phase[s] = 0;
+            uint32_t kv_uses = 0;
+            bool ok = true;
+            for (uint32_t k = 0; ok; ++k) {
+                int it = atomicAdd(p.sched, 1);
+                if (it >= p.n_items) it = -1;
+                const uint32_t slot = k & 1u;
+                if (!(ok = mbar_wait(smem_u32(b_itempty + slot), ((k >> 1) & 1u) ^ 1u, lim, kSiteBwdItem))) break;
+                s_item[slot] = it;
+                mbar_arrive(smem_u32(b_itfull + slot));
+                if (it < 0) break;
+                const BwdKvItem m = bwd_kv_item(p, it);
+                if (kv_uses > 0 && !(ok = mbar_wait(smem_u32(b_kempty), (kv_uses - 1) & 1u, lim, kSiteBwdKvEmpty)))
+                    break;
+                {
+                    const uint32_t kb = smem_u32(b_kfull);
+                    mbar_arrive_expect_tx(kb, 2u * (uint32_t)C::TILE_BYTES);
+                    for (int ch = 0; ch < C::NCHUNK; ++ch) {
+                        tma_load_4d(smem_u32(sK + ch * C::CHUNK_BYTES), &tm_k, kb, ch * 64, m.hk, m.k0, m.b);
+                        tma_load_4d(smem_u32(sV + ch * C::CHUNK_BYTES), &tm_v, kb, ch * 64, m.hk, m.k0, m.b);
+                    }
+                    ++kv_uses;
+                }
+                for (int g = 0; ok && g < p.G; ++g) {
+                    const int h = m.hk * p.G + g;
+                    for (int i = m.lo; ok && i <= m.hi; ++i) {
+                        if (!(ok = mbar_wait(smem_u32(b_stempty + stage), phase ^ 1u, lim, kSiteBwdStage))) break;
+                        const uint32_t fb = smem_u32(b_stfull + stage);
+                        uint8_t* base = sSt + stage * C::STAGE_BYTES;
+                        mbar_arrive_expect_tx(fb, 2u * (uint32_t)C::TILE_BYTES + 1024u);
+                        for (int ch = 0; ch < C::NCHUNK; ++ch) {
+                            tma_load_4d(smem_u32(base + ch * C::CHUNK_BYTES), &tm_q, fb, ch * 64, h, i * 128, m.b);
+                            tma_load_4d(smem_u32(base + C::TILE_BYTES + ch * C::CHUNK_BYTES), &tm_do, fb, ch * 64, h,
+                                        i * 128, m.b);
+                        }
+                        bulk_load_1d(smem_u32(base + 2 * C::TILE_BYTES),
+                                     p.rowstat + ((long long)m.b * p.H + h) * p.Tp + (long long)i * 128, 1024u, fb);
+                        filled[stage] = true;
+                        filled_phase[stage] = phase;
+                        if (++stage == (uint32_t)NS) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                }
+            }
+            if (ok && atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1) {
+                p.sched[0] = 0;
+                p.sched[1] = 0;
+            }
+            if (kv_uses > 0) mbar_wait(smem_u32(b_kfull), (kv_uses - 1) & 1u, lim, kSiteBwdDrain);
+            for (int s = 0; s < NS; ++s)
+                if (filled[s]) mbar_wait(smem_u32(b_stfull + s), filled_phase[s], lim, kSiteBwdDrain);
+        }
+    } else if (warp == kMmaWarp) {
+        // ============================== MMA issuer ==============================
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);   // S^T, dP^T: N = 128 queries
+            constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, true);      // dV, dK: B MN-major
+            const uint64_t a_k = smem_desc_sw128(smem_u32(sK), 16, 1024);
+            const uint64_t a_v = smem_desc_sw128(smem_u32(sV), 16, 1024);
+            const uint64_t b_kmaj = smem_desc_sw128(smem_u32(sSt), 16, 1024);
+            const uint64_t b_mn = smem_desc_sw128(smem_u32(sSt), C::CHUNK_BYTES, 1024);
+            uint32_t stage = 0, phase = 0;
+            uint32_t p_cnt = 0, uses = 0;
+            bool ok = true;
+            for (uint32_t k = 0; ok; ++k) {
+                const uint32_t slot = k & 1u;
+                if (!(ok = mbar_wait(smem_u32(b_itfull + slot), (k >> 1) & 1u, lim, kSiteBwdItem))) break;
+                const int it = s_item[slot];
+                mbar_arrive(smem_u32(b_itempty + slot));
+                if (it < 0) break;
+                const BwdKvItem m = bwd_kv_item(p, it);
+                if (!(ok = mbar_wait(smem_u32(b_kfull), uses & 1u, lim, kSiteBwdKvFull))) break;
+                const int n_steps = p.G * (m.hi - m.lo + 1);
+                for (int s = 0; ok && s < n_steps; ++s) {
+                    const uint32_t sg = stage;
+                    if (!(ok = mbar_wait(smem_u32(b_stfull + stage), phase, lim, kSiteBwdStage))) break;
+                    if (++stage == (uint32_t)NS) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                    const uint64_t qoff = (uint64_t)((sg * C::STAGE_BYTES) >> 4);
+                    const uint64_t dooff = (uint64_t)((sg * C::STAGE_BYTES + C::TILE_BYTES) >> 4);
+                    // S^T = K Q^T and dP^T = V' dO^T: M = 128 keys, N = 128 queries, K = D.
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ss(tmem + C::KV_COL_ST, a_k + kmajor_step<D>(kk), b_kmaj + qoff + kmajor_step<D>(kk),
+                               idesc_s, kk > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_ss(tmem + C::KV_COL_DPT, a_v + kmajor_step<D>(kk), b_kmaj + dooff + kmajor_step<D>(kk),
+                               idesc_s, kk > 0 ? 1u : 0u);
+                    mma_commit(smem_u32(b_sfull));
+                    if (!(ok = mbar_wait(smem_u32(b_pfull), p_cnt & 1u, lim, kSiteBwdPFull))) break;
+                    ++p_cnt;
+                    if (s == 0 && uses > 0 && !(ok = mbar_wait(smem_u32(b_oempty), (uses - 1) & 1u, lim, kSiteBwdOEmpty)))
+                        break;
+                    tc_fence_after();
+                    // dV += P^T dO and dK += dS^T Q: K = 128 queries in steps of 16; P^T / dS^T of
+                    // queries 32 c + i at column 32 c + i / 2 of their buffers.
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tmem + C::KV_COL_DV, tmem + C::KV_COL_ST + (kk >> 1) * 32 + (kk & 1) * 8,
+                               b_mn + dooff + (uint64_t)((kk * 16 * 128) >> 4), idesc_g, (s > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tmem + C::KV_COL_DK, tmem + C::KV_COL_DPT + (kk >> 1) * 32 + (kk & 1) * 8,
+                               b_mn + qoff + (uint64_t)((kk * 16 * 128) >> 4), idesc_g, (s > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(smem_u32(b_stempty + sg));
+                }
+                if (!ok) break;
+                mma_commit(smem_u32(b_ofull));
+                mma_commit(smem_u32(b_kempty));
+                ++uses;
+            }
+            mma_commit(smem_u32(b_mdrain));
+            mbar_wait(smem_u32(b_mdrain), 0, lim, kSiteBwdDrain);
+        }
+        __syncwarp();
+    } else {
+        // ========================= P^T, dS^T + epilogue =========================
+        const int cq = (warp - kSoftmaxWarp0) >> 2;   // query / output column quarter
+        const int r = ((warp & 3) << 5) + lane;       // key row = tensor-memory lane
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        uint32_t stage = 0, phase = 0;
+        uint32_t s_cnt = 0, o_uses = 0;
+        bool ok = true;
+        for (uint32_t k = 0; ok; ++k) {
+            const uint32_t slot = k & 1u;
+            int it = 0;
+            if (lane == 0) {
+                ok = mbar_wait(smem_u32(b_itfull + slot), (k >> 1) & 1u, lim, kSiteBwdItem);
+                it = s_item[slot];
+                mbar_arrive(smem_u32(b_itempty + slot));
+            }
+            ok = __all_sync(0xffffffffu, ok);
+            it = __shfl_sync(0xffffffffu, it, 0);
+            if (!ok || it < 0) break;
+            const BwdKvItem m = bwd_kv_item(p, it);
+            const int key = m.k0 + r;
+            const int nq = m.hi - m.lo + 1;
+            const int n_steps = p.G * nq;
+            for (int s = 0; s < n_steps; ++s) {
+                const int i = m.lo + s % nq;
+                const uint32_t sg = stage;
+                // The score products of this step are complete, and (through the stage's own
+                // barrier, still in this phase) so is the copy of its row statistics.
+                bool w = mbar_wait(smem_u32(b_sfull), s_cnt & 1u, lim, kSiteBwdSFull);
+                w = w && mbar_wait(smem_u32(b_stfull + sg), phase, lim, kSiteBwdStage);
+                ok = __all_sync(0xffffffffu, w);
+                if (!ok) break;
+                ++s_cnt;
+                if (++stage == (uint32_t)NS) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                tc_fence_after();
+                const float2* rs = reinterpret_cast<const float2*>(sSt + sg * C::STAGE_BYTES + 2 * C::TILE_BYTES) + 32 * cq;
+                const int qc0 = i * 128 + 32 * cq;      // first query column of this thread
+                uint32_t sv[2][16], dv[2][16], pp[16], pd[16];
+                const uint32_t colS = C::KV_COL_ST + 32u * (uint32_t)cq;
+                const uint32_t colP = C::KV_COL_DPT + 32u * (uint32_t)cq;
+                tmem_ld16(tmem + lane_base + colS, sv[0]);
+                tmem_ld16(tmem + lane_base + colS + 16u, sv[1]);
+                tmem_ld16(tmem + lane_base + colP, dv[0]);
+                tmem_ld16(tmem + lane_base + colP + 16u, dv[1]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {
+#pragma unroll
+                    for (int e = 0; e < 16; e += 2) {
+                        const int c = 16 * hb + e;
+                        const float2 r0 = rs[c], r1 = rs[c + 1];
+                        float p0 = ex2_approx(fmaf(__uint_as_float(sv[hb][e]), p.c1, -r0.x));
+                        float p1 = ex2_approx(fmaf(__uint_as_float(sv[hb][e + 1]), p.c1, -r1.x));
+                        if ((unsigned)(qc0 + c - key) >= (unsigned)p.W) p0 = 0.f;
+                        if ((unsigned)(qc0 + c + 1 - key) >= (unsigned)p.W) p1 = 0.f;
+                        const float d0 = p0 * (__uint_as_float(dv[hb][e]) - r0.y);
+                        const float d1 = p1 * (__uint_as_float(dv[hb][e + 1]) - r1.y);
+                        pp[8 * hb + (e >> 1)] = pack_bf16x2(p0, p1);
+                        pd[8 * hb + (e >> 1)] = pack_bf16x2(d0, d1);
+                    }
+                }
+                tmem_st16(tmem + lane_base + colS, pp);
+                tmem_st16(tmem + lane_base + colP, pd);
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(smem_u32(b_pfull));
+            }
+            if (!ok) break;
+            {
+                const bool w = mbar_wait(smem_u32(b_ofull), o_uses & 1u, lim, kSiteBwdOFull);
+                ok = __all_sync(0xffffffffu, w);
+            }
+            if (!ok) break;
+            tc_fence_after();
+            constexpr int OQ = D / 4;
+            uint32_t ovv[OQ], okk[OQ];
+            tmem_ld16(tmem + lane_base + C::KV_COL_DV + (uint32_t)(OQ * cq), *reinterpret_cast<uint32_t(*)[16]>(ovv));
+            tmem_ld16(tmem + lane_base + C::KV_COL_DK + (uint32_t)(OQ * cq), *reinterpret_cast<uint32_t(*)[16]>(okk));
+            if constexpr (OQ == 32) {
+                tmem_ld16(tmem + lane_base + C::KV_COL_DV + (uint32_t)(OQ * cq) + 16u,
+                          *reinterpret_cast<uint32_t(*)[16]>(ovv + 16));
+                tmem_ld16(tmem + lane_base + C::KV_COL_DK + (uint32_t)(OQ * cq) + 16u,
+                          *reinterpret_cast<uint32_t(*)[16]>(okk + 16));
+            }
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(smem_u32(b_oempty));
+            ++o_uses;
+            if (key < p.T) {
+                const long long off = (((long long)m.b * p.T + key) * p.Hkv + m.hk) * D + OQ * cq;
+                float4* dvd = reinterpret_cast<float4*>(p.dvp + off);
+                float4* dkd = reinterpret_cast<float4*>(p.dkh + off);
+#pragma unroll
+                for (int e = 0; e < OQ / 4; ++e) {
+                    dvd[e] = make_float4(__uint_as_float(ovv[4 * e]), __uint_as_float(ovv[4 * e + 1]),
+                                         __uint_as_float(ovv[4 * e + 2]), __uint_as_float(ovv[4 * e + 3]));
+                    dkd[e] = make_float4(__uint_as_float(okk[4 * e]) * p.inv_sqrt_d,
+                                         __uint_as_float(okk[4 * e + 1]) * p.inv_sqrt_d,
+                                         __uint_as_float(okk[4 * e + 2]) * p.inv_sqrt_d,
+                                         __uint_as_float(okk[4 * e + 3]) * p.inv_sqrt_d);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------- the prologue in reverse
+
+// dL/d(raw row) of q or k from dy = dL/d(normalised row), one warp per (b, t, head) row.
+// With x the raw row, R_t the rotation at position t, r = (|x|^2 / D + eps)^(-1/2) (the rotation
+// keeps the norm) and u = R_t^T dy:  dx = r u - (r^3 / D) (x . u) x.  Lane l holds the pairs
+// (i, i + D/2) for i = l P .. l P + P - 1, P = D / 64.
+template <int D>
+__global__ void bwd_qk_rows_kernel(const __nv_bfloat16* __restrict__ src, const float* __restrict__ dy,
+                                   __nv_bfloat16* __restrict__ dx, const double2* __restrict__ tab64,
+                                   int n_rows, int T, int heads, float eps) {
+    constexpr int P = D / 64;
+    constexpr int HALF = D / 2;
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    for (int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < n_rows; row += warps) {
+        const int t = (row / heads) % T;
+        const long long base = (long long)row * D;
+        const int i0 = lane * P;
+        float xa[P], xb[P], ua[P], ub[P];
+        float ss = 0.f, xu = 0.f;
+#pragma unroll
+        for (int e = 0; e < P; ++e) {
+            const int i = i0 + e;
+            xa[e] = __bfloat162float(src[base + i]);
+            xb[e] = __bfloat162float(src[base + i + HALF]);
+            const float ga = dy[base + i], gb = dy[base + i + HALF];
+            const double2 cs = tab64[(long long)t * HALF + i];
+            const float c = (float)cs.x, s = (float)cs.y;
+            ua[e] = ga * c + gb * s;
+            ub[e] = gb * c - ga * s;
+            ss += xa[e] * xa[e] + xb[e] * xb[e];
+            xu += xa[e] * ua[e] + xb[e] * ub[e];
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            xu += __shfl_xor_sync(0xffffffffu, xu, o);
+        }
+        const float rr = rsqrtf(ss / (float)D + eps);
+        const float coef = rr * rr * rr * xu / (float)D;
+#pragma unroll
+        for (int e = 0; e < P; ++e) {
+            const int i = i0 + e;
+            dx[base + i] = __float2bfloat16_rn(rr * ua[e] - coef * xa[e]);
+            dx[base + i + HALF] = __float2bfloat16_rn(rr * ub[e] - coef * xb[e]);
+        }
+    }
+}
+
+// dv = dv'; on value-embedding layers dve = g dv' and dz = (dv' . ve) g (1 - g / 2), the
+// derivative of g = 2 sigmoid(z) being 2 sigmoid (1 - sigmoid).  One warp per (b, t, hk) row.
+template <int D, bool HAS_VE>
+__global__ void bwd_v_rows_kernel(const float* __restrict__ dvp, const __nv_bfloat16* __restrict__ ve,
+                                  const float2* __restrict__ gate, __nv_bfloat16* __restrict__ dv,
+                                  __nv_bfloat16* __restrict__ dve, float* __restrict__ dz, int n_rows) {
+    constexpr int E = D / 32;
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    for (int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < n_rows; row += warps) {
+        const long long base = (long long)row * D + lane * E;
+        float g = 0.f;
+        if constexpr (HAS_VE) {
+            const float2 gg = gate[row];
+            g = gg.x + gg.y;
+        }
+        float acc = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const float d = dvp[base + e];
+            dv[base + e] = __float2bfloat16_rn(d);
+            if constexpr (HAS_VE) {
+                dve[base + e] = __float2bfloat16_rn(g * d);
+                acc += d * __bfloat162float(ve[base + e]);
+            }
+        }
+        if constexpr (HAS_VE) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (lane == 0) dz[row] = acc * g * (1.f - 0.5f * g);
+        }
+    }
+}
+
+// dgate_x[bt, c] = sum_hk dz[bt, hk] Wg[c, hk]: one thread per (bt, c).
+__global__ void bwd_gate_x_kernel(const float* __restrict__ dz, const __nv_bfloat16* __restrict__ Wg,
+                                  float* __restrict__ dgx, long long n_bt, int Hkv) {
+    const long long n = n_bt * 32;
+    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
+         idx += (long long)gridDim.x * blockDim.x) {
+        const long long bt = idx >> 5;
+        const int c = (int)(idx & 31);
+        float acc = 0.f;
+        for (int hk = 0; hk < Hkv; ++hk) acc += dz[bt * Hkv + hk] * __bfloat162float(Wg[c * Hkv + hk]);
+        dgx[idx] = acc;
+    }
+}
+
+// dWg in two passes with a fixed order: block blk sums rows [blk R, blk R + R) into
+// part[blk][c Hkv + hk]; the final pass adds the blocks in index order.
+__global__ void bwd_wg_partial_kernel(const float* __restrict__ dz, const __nv_bfloat16* __restrict__ gate_x,
+                                      float* __restrict__ part, long long n_bt, int Hkv, int rows_per_block) {
+    const int n = 32 * Hkv;
+    const long long r0 = (long long)blockIdx.x * rows_per_block;
+    const long long r1 = min(r0 + rows_per_block, n_bt);
+    for (int idx = threadIdx.x; idx < n; idx += blockDim.x) {
+        const int c = idx / Hkv;
+        const int hk = idx - c * Hkv;
+        float acc = 0.f;
+        for (long long bt = r0; bt < r1; ++bt) acc += dz[bt * Hkv + hk] * __bfloat162float(gate_x[bt * 32 + c]);
+        part[(long long)blockIdx.x * n + idx] = acc;
+    }
+}
+
+__global__ void bwd_wg_final_kernel(const float* __restrict__ part, float* __restrict__ dWg, int n_blocks, int n) {
+    for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < n; idx += gridDim.x * blockDim.x) {
+        float acc = 0.f;
+        for (int b = 0; b < n_blocks; ++b) acc += part[(long long)b * n + idx];
+        dWg[idx] = acc;
+    }
+}
+
+}  // namespace swa

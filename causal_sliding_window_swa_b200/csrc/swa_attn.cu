@@ -1,6 +1,7 @@
 // swa_attn.cu -- host side of the C ABI declared in include/swa_attn.h: argument checks,
 // workspace management, TMA descriptors and the two kernel launches (prologue, attention).
-// All kernels are in this translation unit (ptx.cuh, prologue.cuh, attn_fwd.cuh).
+// All kernels are in this translation unit (ptx.cuh, prologue.cuh, attn_fwd.cuh, attn_bwd.cuh,
+// decode.cuh).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -12,6 +13,7 @@
 #include <mutex>
 
 #include "swa_attn.h"
+#include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
 #include "decode.cuh"
 #include "prologue.cuh"
@@ -155,10 +157,19 @@ int device_ready(int* dev_out) {
             return SWA_ERR_CUDA;
         }
         if (checked[dev] == 1) {
+            const int smem_attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
             if (cudaFuncSetAttribute(swa::attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      swa::FwdCfg<64>::SMEM_TOTAL) != cudaSuccess ||
                 cudaFuncSetAttribute(swa::attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     swa::FwdCfg<128>::SMEM_TOTAL) != cudaSuccess) {
+                                     swa::FwdCfg<128>::SMEM_TOTAL) != cudaSuccess ||
+                cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<64>, (cudaFuncAttribute)smem_attr,
+                                     swa::BwdCfg<64>::DQ_SMEM) != cudaSuccess ||
+                cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<128>, (cudaFuncAttribute)smem_attr,
+                                     swa::BwdCfg<128>::DQ_SMEM) != cudaSuccess ||
+                cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<64>, (cudaFuncAttribute)smem_attr,
+                                     swa::BwdCfg<64>::KV_SMEM) != cudaSuccess ||
+                cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<128>, (cudaFuncAttribute)smem_attr,
+                                     swa::BwdCfg<128>::KV_SMEM) != cudaSuccess) {
                 cudaGetLastError();
                 checked[dev] = 0;
                 return SWA_ERR_CUDA;
@@ -336,6 +347,149 @@ int launch_attention(int dev, const void* v, bool has_ve, void* out, float* lse,
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------- backward
+
+// The forward's sections (qhat, khat, v', gate, RoPE tables, counters; the prologue rewrites them)
+// followed by the backward's: row statistics (B, H, Tp) float2 | dqhat (B,T,H,D) fp32 |
+// dkhat, dv' (B,T,Hkv,D) fp32 | dz (B,T,Hkv) fp32 and the dWg partial sums (value-embedding
+// layers only).  The backward kernels' scheduler counters are ints 4..7 of the counter section.
+struct BwdLayout {
+    WsLayout f;
+    size_t rowstat, dqh, dkh, dvp, dz, wgp, total;
+    int Tp, wg_blocks, wg_rows;
+};
+
+BwdLayout bwd_layout(const Shape& s, bool has_ve) {
+    BwdLayout w{};
+    w.f = ws_layout(s, has_ve);
+    w.Tp = ((s.T + 127) / 128) * 128;
+    const long long n_bt = (long long)s.B * s.T;
+    const size_t kv_f32 = round_up((size_t)n_bt * s.Hkv * s.D * 4);
+    w.wg_rows = 256;
+    w.wg_blocks = has_ve ? (int)((n_bt + w.wg_rows - 1) / w.wg_rows) : 0;
+    size_t o = w.f.total;
+    w.rowstat = o;
+    o += round_up((size_t)s.B * s.H * w.Tp * sizeof(float2));
+    w.dqh = o;
+    o += round_up((size_t)s.n * 4);
+    w.dkh = o;
+    o += kv_f32;
+    w.dvp = o;
+    o += kv_f32;
+    w.dz = o;
+    o += has_ve ? round_up((size_t)n_bt * s.Hkv * 4) : 0;
+    w.wgp = o;
+    o += has_ve ? round_up((size_t)w.wg_blocks * 32 * s.Hkv * 4) : 0;
+    w.total = o;
+    return w;
+}
+
+int launch_backward(int dev, const void* q, const void* k, const void* v, const void* ve,
+                    const void* gate_x, const void* Wg, const void* out, const float* lse,
+                    const void* dout, const float* dlse, void* dq, void* dk, void* dv, void* dve,
+                    float* dgate_x, float* dWg, const Shape& s, int window, float rope_base, float eps,
+                    uint8_t* ws, const BwdLayout& L, cudaStream_t st) {
+    using bf = __nv_bfloat16;
+    const bool has_ve = ve != nullptr;
+    int rc;
+    // qhat, khat, v' and the gate exactly as the forward computed them.
+    if ((rc = launch_rope_table(ws, L.f, s, rope_base, st)) != SWA_OK) return rc;
+    if ((rc = launch_prologue(q, k, v, ve, gate_x, Wg, ws, L.f, s, eps, st)) != SWA_OK) return rc;
+
+    int* sched4 = reinterpret_cast<int*>(ws + L.f.sched) + 4;
+    float2* rowstat = reinterpret_cast<float2*>(ws + L.rowstat);
+    {
+        const long long rows = (long long)s.B * s.H * L.Tp;
+        const int blocks = (int)std::min<long long>((rows + 7) / 8, 148ll * 16);
+        if (s.D == 128)
+            swa::bwd_rowstat_kernel<128><<<blocks, 256, 0, st>>>(static_cast<const bf*>(out), static_cast<const bf*>(dout),
+                                                                 lse, dlse, rowstat, s.B, s.T, s.H, L.Tp, sched4);
+        else
+            swa::bwd_rowstat_kernel<64><<<blocks, 256, 0, st>>>(static_cast<const bf*>(out), static_cast<const bf*>(dout),
+                                                                lse, dlse, rowstat, s.B, s.T, s.H, L.Tp, sched4);
+    }
+
+    CUtensorMap tq, tk, tv, tdo;
+    const void* vsrc = has_ve ? static_cast<const void*>(ws + L.f.vp) : v;
+    if (!make_tile_map(&tq, ws + L.f.qh, s, s.H) || !make_tile_map(&tk, ws + L.f.kh, s, s.Hkv) ||
+        !make_tile_map(&tv, vsrc, s, s.Hkv) || !make_tile_map(&tdo, dout, s, s.H))
+        return SWA_ERR_CUDA;
+    swa::BwdParams p{};
+    p.B = s.B;
+    p.T = s.T;
+    p.H = s.H;
+    p.Hkv = s.Hkv;
+    p.G = s.H / s.Hkv;
+    p.W = (window <= 0 || window >= s.T) ? s.T : window;
+    p.n_tiles = (s.T + 127) / 128;
+    p.Tp = L.Tp;
+    p.c1 = (float)(1.4426950408889634 / std::sqrt((double)s.D));
+    p.inv_sqrt_d = (float)(1.0 / std::sqrt((double)s.D));
+    p.rowstat = rowstat;
+    p.dqh = reinterpret_cast<float*>(ws + L.dqh);
+    p.dkh = reinterpret_cast<float*>(ws + L.dkh);
+    p.dvp = reinterpret_cast<float*>(ws + L.dvp);
+    p.wait_limit_ns = wait_limit_ns();
+    const long long slice_bytes = 4ll * s.T * s.D;   // two bf16 (T, D) slices
+    // Query tiles: chunks of (b, h) slices whose K and V' fit in ~40 MB of L2.
+    swa::BwdParams pq = p;
+    pq.n_items = p.n_tiles * s.H * s.B;
+    pq.chunk_bh = (int)std::max<long long>(1, std::min<long long>((40ll << 20) / slice_bytes, (long long)s.B * s.H));
+    pq.sched = sched4;
+    // Key tiles: chunks of (b, hk) slices whose G query heads of Q and dO fit likewise.
+    swa::BwdParams pk = p;
+    pk.n_items = p.n_tiles * s.Hkv * s.B;
+    pk.chunk_bh = (int)std::max<long long>(
+        1, std::min<long long>((40ll << 20) / (slice_bytes * p.G), (long long)s.B * s.Hkv));
+    pk.sched = sched4 + 2;
+    const dim3 gq((unsigned)std::min(pq.n_items, g_num_sms[dev]));
+    const dim3 gk((unsigned)std::min(pk.n_items, g_num_sms[dev]));
+    if (s.D == 128) {
+        using C = swa::BwdCfg<128>;
+        swa::attn_bwd_dq_kernel<128><<<gq, C::THREADS, C::DQ_SMEM, st>>>(tq, tk, tv, tdo, pq);
+        swa::attn_bwd_dkv_kernel<128><<<gk, C::THREADS, C::KV_SMEM, st>>>(tq, tk, tv, tdo, pk);
+    } else {
+        using C = swa::BwdCfg<64>;
+        swa::attn_bwd_dq_kernel<64><<<gq, C::THREADS, C::DQ_SMEM, st>>>(tq, tk, tv, tdo, pq);
+        swa::attn_bwd_dkv_kernel<64><<<gk, C::THREADS, C::KV_SMEM, st>>>(tq, tk, tv, tdo, pk);
+    }
+
+    // The prologue in reverse.
+    const double2* t64 = reinterpret_cast<const double2*>(ws + L.f.tab64);
+    const int n_q = s.B * s.T * s.H, n_kv = s.B * s.T * s.Hkv;
+    const int bq = std::min((n_q + 7) / 8, 148 * 16), bkv = std::min((n_kv + 7) / 8, 148 * 16);
+    const float2* gate = reinterpret_cast<const float2*>(ws + L.f.gate);
+    float* dz = reinterpret_cast<float*>(ws + L.dz);
+#define SWA_BWD_ROWS(DD)                                                                                          \
+    swa::bwd_qk_rows_kernel<DD><<<bq, 256, 0, st>>>(static_cast<const bf*>(q), p.dqh, static_cast<bf*>(dq), t64,  \
+                                                   n_q, s.T, s.H, eps);                                            \
+    swa::bwd_qk_rows_kernel<DD><<<bkv, 256, 0, st>>>(static_cast<const bf*>(k), p.dkh, static_cast<bf*>(dk), t64, \
+                                                    n_kv, s.T, s.Hkv, eps);                                        \
+    if (has_ve)                                                                                                   \
+        swa::bwd_v_rows_kernel<DD, true><<<bkv, 256, 0, st>>>(p.dvp, static_cast<const bf*>(ve), gate,            \
+                                                             static_cast<bf*>(dv), static_cast<bf*>(dve), dz, n_kv); \
+    else                                                                                                          \
+        swa::bwd_v_rows_kernel<DD, false><<<bkv, 256, 0, st>>>(p.dvp, nullptr, nullptr, static_cast<bf*>(dv),     \
+                                                              nullptr, nullptr, n_kv)
+    if (s.D == 128) {
+        SWA_BWD_ROWS(128);
+    } else {
+        SWA_BWD_ROWS(64);
+    }
+#undef SWA_BWD_ROWS
+    if (has_ve) {
+        const long long n_bt = (long long)s.B * s.T;
+        const int bgx = (int)std::min<long long>((n_bt * 32 + 255) / 256, 148ll * 16);
+        swa::bwd_gate_x_kernel<<<bgx, 256, 0, st>>>(dz, static_cast<const bf*>(Wg), dgate_x, n_bt, s.Hkv);
+        float* part = reinterpret_cast<float*>(ws + L.wgp);
+        swa::bwd_wg_partial_kernel<<<L.wg_blocks, 256, 0, st>>>(dz, static_cast<const bf*>(gate_x), part, n_bt,
+                                                                s.Hkv, L.wg_rows);
+        const int n = 32 * s.Hkv;
+        swa::bwd_wg_final_kernel<<<(n + 255) / 256, 256, 0, st>>>(part, dWg, L.wg_blocks, n);
+    }
+    return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
 // ------------------------------------------------------------- library-owned workspace
 
 struct DevCache {
@@ -508,6 +662,50 @@ int swa_attn_fwd(const void* q, const void* k, const void* v, const void* ve, co
                  float rope_base, float eps, swa_stream_t stream) {
     return swa_attn_fwd_gqa(q, k, v, ve, gate_x, Wg, out, lse, B, T, H, H, D, window, rope_base, eps,
                             stream);
+}
+
+// ---------------------------------------------------------------------------- backward
+
+size_t swa_attn_bwd_workspace_bytes(int B, int T, int H, int Hkv, int D, int has_ve) {
+    Shape s;
+    if (check_sizes(B, T, H, D, &s) != SWA_OK || check_kv_heads(Hkv, &s) != SWA_OK) return 0;
+    return bwd_layout(s, has_ve != 0).total;
+}
+
+int swa_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                     const void* Wg, const void* out, const float* lse, const void* dout,
+                     const float* dlse, void* dq, void* dk, void* dv, void* dve, float* dgate_x,
+                     float* dWg, int B, int T, int H, int Hkv, int D, int window, float rope_base,
+                     float eps, void* workspace, size_t ws_bytes, swa_stream_t stream) {
+    Shape s;
+    int rc = check_sizes(B, T, H, D, &s);
+    if (rc == SWA_OK) rc = check_kv_heads(Hkv, &s);
+    if (rc == SWA_OK) rc = check_layer_args(q, k, v, ve, gate_x, Wg, rope_base, eps);
+    if (rc != SWA_OK) return rc;
+    const bool has_ve = ve != nullptr;
+    if (!out || !lse || !dout || !dq || !dk || !dv || !workspace) return SWA_ERR_INVALID_ARG;
+    const int n_vegrad = (dve != nullptr) + (dgate_x != nullptr) + (dWg != nullptr);
+    if (n_vegrad != (has_ve ? 3 : 0)) return SWA_ERR_INVALID_ARG;
+    if (!aligned(out, 16) || !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+        !aligned(lse, 4) || (dlse && !aligned(dlse, 4)) || !aligned(workspace, 16))
+        return SWA_ERR_MISALIGNED;
+    if (has_ve && (!aligned(dve, 16) || !aligned(dgate_x, 4) || !aligned(dWg, 4))) return SWA_ERR_MISALIGNED;
+    const BwdLayout L = bwd_layout(s, has_ve);
+    if (ws_bytes < L.total) return SWA_ERR_NO_MEMORY;
+    int dev;
+    if ((rc = device_ready(&dev)) != SWA_OK) return rc;
+    return launch_backward(dev, q, k, v, ve, gate_x, Wg, out, lse, dout, dlse, dq, dk, dv, dve, dgate_x, dWg, s,
+                           window, rope_base, eps, static_cast<uint8_t*>(workspace), L,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+int swa_attn_bwd(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                 const void* Wg, const void* out, const float* lse, const void* dout, const float* dlse,
+                 void* dq, void* dk, void* dv, void* dve, float* dgate_x, float* dWg, int B, int T, int H,
+                 int D, int window, float rope_base, float eps, void* workspace, size_t ws_bytes,
+                 swa_stream_t stream) {
+    return swa_attn_bwd_gqa(q, k, v, ve, gate_x, Wg, out, lse, dout, dlse, dq, dk, dv, dve, dgate_x, dWg, B, T,
+                            H, H, D, window, rope_base, eps, workspace, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------- decode step with a KV cache

@@ -240,6 +240,50 @@ SWA_API int swa_attn_decode_gqa(const void* q, const void* k, const void* v, con
                                 size_t ws_bytes, swa_stream_t stream);
 
 /*
+ * Backward of the layer: the gradient of loss = sum(dout * out) + sum(dlse * lse) for the layer of
+ * swa_attn_fwd / swa_attn_fwd_gqa (the pages train it end to end; the log-sum-exp the forward
+ * writes lets the backward rebuild the softmax: "Let's reproduce GPT-2 (124M)" notes, the
+ * attention-kernel discussion in section 19).  Per visible pair (i, j) with P_ij = exp(s_ij - lse_i):
+ *   dP_ij = dout_i . v'_j,  delta_i = dout_i . out_i,  dS_ij = P_ij (dP_ij - delta_i + dlse_i),
+ *   dqhat_i = sum_j dS_ij khat_j / sqrt(D),  dkhat_j = sum_i dS_ij qhat_i / sqrt(D),
+ *   dv'_j = sum_i P_ij dout_i  (summed over the query heads of a key/value head's group),
+ * then the prologue in reverse: dq = RoPE^T(r dqhat - (r^3/D)(x . dqhat) x) per row (likewise dk),
+ * dv = dv', dve = g dv', dz = (dv' . ve) 2 sigmoid(z)(1 - sigmoid(z)), dgate_x = dz Wg^T,
+ * dWg = gate_x^T dz.
+ * Arguments (device pointers, caller-owned, all read-only except the gradients and workspace):
+ *   q, k, v, ve, gate_x, Wg   the forward's inputs, shapes as swa_attn_fwd_gqa.
+ *   out, lse                  the forward's outputs for these inputs: bf16 (B,T,H,D), fp32 (B,H,T).
+ *   dout                      bf16 (B,T,H,D).   dlse  fp32 (B,H,T), or NULL for zero.
+ *   dq                        bf16 (B,T,H,D), written.   dk, dv  bf16 (B,T,Hkv,D), written.
+ *   dve                       bf16 (B,T,Hkv,D): gradient of the looked-up value-embedding rows.
+ *   dgate_x                   fp32 (B,T,32).   dWg  fp32 (32,Hkv).
+ *                             These three are set on value-embedding layers and NULL otherwise.
+ *   workspace                 at least swa_attn_bwd_workspace_bytes(B,T,H,Hkv,D,has_ve) bytes,
+ *                             16-byte aligned; nothing in it is kept between calls.
+ * qhat, khat and v' are recomputed by the forward's prologue (bit-identical to the forward's);
+ * P and dS enter the tensor-core products as bf16 (round to nearest), accumulation is fp32.
+ * Asynchronous on `stream` (about ten kernels); arguments are validated before anything is
+ * enqueued.  Errors: SWA_ERR_INVALID_ARG (null pointer, value-embedding gradients not matching the
+ * inputs, Hkv not dividing H, bad rope_base / eps), SWA_ERR_UNSUPPORTED, SWA_ERR_MISALIGNED,
+ * SWA_ERR_NO_MEMORY (workspace too small), SWA_ERR_CUDA; bounded-wait timeouts inside the kernels
+ * are reported by swa_attn_last_device_status().
+ */
+SWA_API size_t swa_attn_bwd_workspace_bytes(int B, int T, int H, int Hkv, int D, int has_ve);
+SWA_API int swa_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* ve,
+                             const void* gate_x, const void* Wg, const void* out, const float* lse,
+                             const void* dout, const float* dlse, void* dq, void* dk, void* dv,
+                             void* dve, float* dgate_x, float* dWg, int B, int T, int H, int Hkv,
+                             int D, int window, float rope_base, float eps, void* workspace,
+                             size_t ws_bytes, swa_stream_t stream);
+/* The multi-head layer: swa_attn_bwd_gqa with Hkv = H. */
+SWA_API int swa_attn_bwd(const void* q, const void* k, const void* v, const void* ve,
+                         const void* gate_x, const void* Wg, const void* out, const float* lse,
+                         const void* dout, const float* dlse, void* dq, void* dk, void* dv, void* dve,
+                         float* dgate_x, float* dWg, int B, int T, int H, int D, int window,
+                         float rope_base, float eps, void* workspace, size_t ws_bytes,
+                         swa_stream_t stream);
+
+/*
  * Failure-detection self-test (no counterpart in the pages).  Enqueues on `stream` one block of
  * 32 threads that waits, through the bounded wait every kernel here uses, on an mbarrier that
  * nothing ever completes.  After `limit_ms` (1..10000) the wait gives up, records SWA_ERR_TIMEOUT

@@ -138,3 +138,37 @@ def test_decode_workspace_and_validation():
     assert call(v_cache=A + 8) == swa.SWA_ERR_MISALIGNED
     assert call(ws_bytes=need - 1) == swa.SWA_ERR_NO_MEMORY
     assert call(D=80) == swa.SWA_ERR_UNSUPPORTED
+
+
+def test_backward_workspace_and_validation():
+    # forward sections + row statistics (B*H*Tp float2) + dqhat (fp32) + dkhat, dv' (fp32, Hkv heads)
+    # [+ dz and the dWg partial sums on value-embedding layers], each section 1024-byte aligned
+    B, T, H, Hkv, D = 2, 200, 4, 2, 64
+    up = lambda x: (x + 1023) // 1024 * 1024
+    fwd = swa.swa_attn_workspace_bytes(B, T, H, D, 0)
+    n0 = swa.swa_attn_bwd_workspace_bytes(B, T, H, Hkv, D, 0)
+    Tp = 256
+    kv_fwd = up(B * T * Hkv * D * 2)
+    assert n0 == (fwd - 2 * up(B * T * H * D * 2) + 2 * kv_fwd + up(B * T * H * D * 2) - kv_fwd
+                  + up(B * H * Tp * 8) + up(B * T * H * D * 4) + 2 * up(B * T * Hkv * D * 4))
+    n1 = swa.swa_attn_bwd_workspace_bytes(B, T, H, Hkv, D, 1)
+    assert n1 > n0 + up(B * T * Hkv * 4)
+    assert swa.swa_attn_bwd_workspace_bytes(B, T, H, 3, D, 0) == 0     # 3 does not divide 4
+    assert swa.swa_attn_bwd_workspace_bytes(B, T, H, Hkv, 96, 0) == 0
+    base = dict(q=A, k=A, v=A, ve=None, gate_x=None, Wg=None, out=A, lse=A, dout=A, dlse=None, dq=A, dk=A,
+                dv=A, dve=None, dgate_x=None, dWg=None, B=B, T=T, H=H, Hkv=Hkv, D=D, window=0,
+                rope_base=1e4, eps=1e-6, workspace=A, ws_bytes=n0, stream=None)
+
+    def call(**kw):
+        return swa.swa_attn_bwd_gqa(*dict(base, **kw).values())
+    assert call(dout=None) == swa.SWA_ERR_INVALID_ARG
+    assert call(lse=None) == swa.SWA_ERR_INVALID_ARG
+    assert call(dq=None) == swa.SWA_ERR_INVALID_ARG
+    assert call(Hkv=3) == swa.SWA_ERR_INVALID_ARG
+    assert call(dve=A) == swa.SWA_ERR_INVALID_ARG                      # VE gradients without VE
+    assert call(ve=A, gate_x=A, Wg=A, ws_bytes=n1) == swa.SWA_ERR_INVALID_ARG   # VE without its gradients
+    assert call(dk=A + 8) == swa.SWA_ERR_MISALIGNED
+    assert call(workspace=A + 8) == swa.SWA_ERR_MISALIGNED
+    assert call(ws_bytes=n0 - 1) == swa.SWA_ERR_NO_MEMORY
+    assert call(D=80) == swa.SWA_ERR_UNSUPPORTED
+    assert call(eps=-1.0) == swa.SWA_ERR_INVALID_ARG
