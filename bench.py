@@ -493,6 +493,74 @@ def run_decode(args, s):
     return 0
 
 
+def run_backward(args, s):
+    """The layer's backward per timed iteration (swa_attn_bwd: prologue recompute, row
+    statistics, the dQ and dK/dV tensor-core kernels, the prologue in reverse and the gate
+    gradients) on the workload, with out / lse from the forward and seeded dout / dlse.
+    Metric: algorithmic backward FLOP/s, 10 D flops per visible (query, key) pair (the five
+    products of the gradient, 2.5 times the forward's 4 D)."""
+    import torch
+    import causal_sliding_window_swa_b200 as swa
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU path)")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    d = workloads.make_layer(s)
+    g = {k: (None if v is None else v.to(dev)) for k, v in workloads.gpu_side_inputs(d).items()}
+    B, T, H, D = s.B, s.T, s.H, s.D
+    stream = torch.cuda.current_stream(dev)
+    out, lse = swa.forward(g["q"], g["k"], g["v"], s.window, ve=g["ve"], gate_x=g["gate_x"], Wg=g["Wg"])
+    gen = torch.Generator().manual_seed(s.seed + 1000)
+    dout = torch.randn((B, T, H, D), generator=gen).to(torch.bfloat16).to(dev)
+    dlse = torch.randn((B, H, T), generator=gen).to(dev)
+    need = swa.swa_attn_bwd_workspace_bytes(B, T, H, H, D, int(s.ve))
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+
+    def step():
+        swa.backward(g["q"], g["k"], g["v"], out, lse, dout, s.window, dlse=dlse, ve=g["ve"],
+                     gate_x=g["gate_x"], Wg=g["Wg"], workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    swa.check_device_status(stream)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(0).start()
+    for i in range(K):
+        flush.fill_(i & 0xff)
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    swa.check_device_status(stream)
+    ms = sum(a.elapsed_time(b) for a, b in evs) / K
+    flops = 2.5 * flops_per_step(s)
+    tf = flops / (ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    # RoPE table, prologue, row statistics, dQ, dK/dV, two q/k row passes, the v row pass; on
+    # value-embedding layers also the gate and the three gate-gradient kernels
+    launches = 8 + (4 if s.ve else 0)
+    line = {
+        "metric": "attention backward TFLOP/s (10 D flops per visible pair)",
+        "value": tf, "unit": "TFLOP/s", "n_gpus": 1, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 operands, fp32 accumulate", "data": "synthetic (seeded)",
+        "config": {"workload": f"backward {args.workload}: B={B} T={T} H={H} D={D} W={s.window} ve={s.ve}",
+                   "l2": "flushed between steps (256 MB write, outside the timed events)"},
+        "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": tf / peaks["bf16_tflops"], "traffic": None, "peak_source": peak_src,
+                     "note": "whole backward call; the tensor-core kernels do 7 products per tile pair"},
+        "gpu_launches": launches * K,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -504,14 +572,17 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--reference-budget-s", type=float, default=90.0)
-    ap.add_argument("--mode", choices=["forward", "decode"], default="forward",
-                    help="decode: time one KV-cache generation step instead of the layer forward")
+    ap.add_argument("--mode", choices=["forward", "decode", "backward"], default="forward",
+                    help="decode: time one KV-cache generation step; backward: time the layer's "
+                         "gradient; default: the layer forward")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     s = WORKLOADS[args.workload]
     if args.mode == "decode":
         return run_decode(args, s)
+    if args.mode == "backward":
+        return run_backward(args, s)
     if args.impl == "reference":
         return run_reference(args, s)
     return run_ours(args, s)
