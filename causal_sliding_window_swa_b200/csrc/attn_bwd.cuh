@@ -15,13 +15,16 @@
 // Kernels, in launch order (after the forward prologue has recomputed qhat, khat, v'):
 //   bwd_rowstat_kernel    per query row: (lse log2 e, delta - dlse), padded to whole tiles
 //                         with (+inf, 0) so that rows past T get P = 0.
-//   attn_bwd_dq_kernel    one 128-row query tile per item: S = Q K^T and dP = dO V'^T (Q and dO
-//                         copied into tensor memory, K and V' from shared memory), dS by 16
-//                         warps, dQ += dS K with dS fed from tensor memory and K read MN-major.
+//   attn_bwd_dq_kernel    one 128-row query tile per item: S = Q K^T (two buffers in tensor
+//                         memory) and dP = dO V'^T from shared-memory operands, dS by 16 warps,
+//                         dQ += dS K with dS fed from tensor memory and K read MN-major; the next
+//                         tile's S is computed while the warps work on this one.
 //   attn_bwd_dkv_kernel   one 128-row key tile per item, over every query tile (and, under
 //                         grouped-query attention, every query head of the group) that sees it:
-//                         S^T = K Q^T and dP^T = V' dO^T from shared memory, P^T and dS^T by 16
-//                         warps, dV += P^T dO and dK += dS^T Q with P^T / dS^T from tensor memory.
+//                         S^T = K Q^T and dP^T = V' dO^T from shared memory; the 16 warps write
+//                         P^T first and dS^T second, so that dV += P^T dO and the next S^T run
+//                         while dS^T is formed, and dK += dS^T Q and the next dP^T while the next
+//                         P^T is.
 //   bwd_qk_rows_kernel    dq (dk) = RoPE^T applied to the RMS backward of dqhat (dkhat).
 //   bwd_v_rows_kernel     dv = dv', dve = g dv', dz = (dv' . ve) g (1 - g / 2) per row.
 //   bwd_gate_x_kernel, bwd_wg_partial_kernel, bwd_wg_final_kernel
@@ -60,11 +63,9 @@ struct BwdCfg {
     // query-tile kernel: Q | dO | NS-stage ring of K and V' tiles | barriers
     static constexpr int DQ_NS = (D == 128) ? 4 : 10;
     static constexpr int DQ_SMEM = 2 * TILE_BYTES + DQ_NS * TILE_BYTES + SMEM_BAR;
-    static constexpr uint32_t DQ_COL_S = 0;            // S, then dS as bf16 pairs
-    static constexpr uint32_t DQ_COL_DP = 128;
-    static constexpr uint32_t DQ_COL_DQ = 256;         // D fp32 columns
-    static constexpr uint32_t DQ_COL_Q = 256 + D;      // D / 2 columns of bf16 pairs
-    static constexpr uint32_t DQ_COL_DO = 256 + D + D / 2;
+    static constexpr uint32_t DQ_COL_S = 0;            // S(0) | S(1), each then dS as bf16 pairs
+    static constexpr uint32_t DQ_COL_DP = 256;
+    static constexpr uint32_t DQ_COL_DQ = 384;         // D fp32 columns
     // key-tile kernel: K | V' | NS stages of (Q tile, dO tile, 128 row statistics) | barriers
     static constexpr int STAGE_BYTES = 2 * TILE_BYTES + 1024;
     static constexpr int KV_NS = (D == 128) ? 2 : 5;
@@ -73,7 +74,7 @@ struct BwdCfg {
     static constexpr uint32_t KV_COL_DPT = 128;        // dP^T, then dS^T as bf16 pairs
     static constexpr uint32_t KV_COL_DV = 256;
     static constexpr uint32_t KV_COL_DK = 256 + D;
-    static_assert(DQ_COL_DO + D / 2 <= TMEM_COLS, "query-tile kernel exceeds tensor memory");
+    static_assert(DQ_COL_DQ + D <= TMEM_COLS, "query-tile kernel exceeds tensor memory");
     static_assert(KV_COL_DK + D <= TMEM_COLS, "key-tile kernel exceeds tensor memory");
     static_assert(DQ_SMEM <= 227 * 1024 && KV_SMEM <= 227 * 1024, "shared memory per CTA");
 };
@@ -158,46 +159,43 @@ __device__ __forceinline__ uint64_t kmajor_step(int kk) {
 
 // ------------------------------------------------------------------- row statistics
 
-// One warp per (b, h, t), t < Tp: delta = dout . out over D (fp32), stored with the log-sum-exp in
-// log2 units.  Block 0 also zeroes the scheduler counters of the two tensor-core kernels.
+// delta = dout . out over D (fp32) for every (b, h, t), t < Tp, stored with the log-sum-exp in
+// log2 units.  L = D / 8 consecutive lanes share a row, one 16-byte load of each tensor per lane.
+// Block 0 also zeroes the scheduler counters of the two tensor-core kernels.
 template <int D>
 __global__ void bwd_rowstat_kernel(const __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ dout,
                                    const float* __restrict__ lse, const float* __restrict__ dlse,
                                    float2* __restrict__ rowstat, int B, int T, int H, int Tp,
                                    int* __restrict__ sched4) {
     if (blockIdx.x == 0 && threadIdx.x < 4) sched4[threadIdx.x] = 0;
-    constexpr int E = D / 32;   // elements per lane: 4 or 2
-    const int lane = threadIdx.x & 31;
-    const long long n = (long long)B * H * Tp;
-    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
-    for (long long f = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); f < n; f += warps) {
-        const int t = (int)(f % Tp);
-        const long long bh = f / Tp;
-        if (t >= T) {
-            if (lane == 0) rowstat[f] = make_float2(__int_as_float(0x7f800000), 0.f);
-            continue;
-        }
-        const int h = (int)(bh % H);
-        const long long b = bh / H;
-        const long long row = ((b * T + t) * H + h) * D + lane * E;
-        float acc = 0.f;
-        if constexpr (E == 4) {
-            const uint2 a = *reinterpret_cast<const uint2*>(out + row);
-            const uint2 g = *reinterpret_cast<const uint2*>(dout + row);
-            acc = __uint_as_float(a.x << 16) * __uint_as_float(g.x << 16) +
-                  __uint_as_float(a.x & 0xffff0000u) * __uint_as_float(g.x & 0xffff0000u) +
-                  __uint_as_float(a.y << 16) * __uint_as_float(g.y << 16) +
-                  __uint_as_float(a.y & 0xffff0000u) * __uint_as_float(g.y & 0xffff0000u);
-        } else {
-            const uint32_t a = *reinterpret_cast<const uint32_t*>(out + row);
-            const uint32_t g = *reinterpret_cast<const uint32_t*>(dout + row);
-            acc = __uint_as_float(a << 16) * __uint_as_float(g << 16) +
-                  __uint_as_float(a & 0xffff0000u) * __uint_as_float(g & 0xffff0000u);
-        }
+    constexpr int L = D / 8;   // lanes per row: 16 or 8
+    const int sub = threadIdx.x & (L - 1);
+    const int n = B * H * Tp;
+    const int f = (int)((blockIdx.x * (long long)blockDim.x + threadIdx.x) / L);
+    // every lane of a row group takes the same branch; groups are aligned inside the warp
+    const bool live = f < n;
+    const int t = live ? f % Tp : 0;
+    const int bh = live ? f / Tp : 0;
+    float acc = 0.f;
+    if (live && t < T) {
+        const int h = bh % H;
+        const int b = bh / H;
+        const long long e0 = (((long long)b * T + t) * H + h) * D + sub * 8;
+        const uint4 a = *reinterpret_cast<const uint4*>(out + e0);
+        const uint4 g = *reinterpret_cast<const uint4*>(dout + e0);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, gw[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) {
-            const long long li = bh * T + t;
+        for (int w = 0; w < 4; ++w)
+            acc += __uint_as_float(aw[w] << 16) * __uint_as_float(gw[w] << 16) +
+                   __uint_as_float(aw[w] & 0xffff0000u) * __uint_as_float(gw[w] & 0xffff0000u);
+    }
+#pragma unroll
+    for (int o = L / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (live && sub == 0) {
+        if (t >= T) {
+            rowstat[f] = make_float2(__int_as_float(0x7f800000), 0.f);
+        } else {
+            const long long li = (long long)bh * T + t;
             const float gl = dlse ? dlse[li] : 0.f;
             rowstat[f] = make_float2(lse[li] * 1.4426950408889634f, acc - gl);
         }
@@ -206,6 +204,14 @@ __global__ void bwd_rowstat_kernel(const __nv_bfloat16* __restrict__ out, const 
 
 // ------------------------------------------------------------------ query-tile kernel (dQ)
 
+// Per item (query tile of (b, h), key tiles lo..hi; g counts tiles over the CTA's items):
+//   S(g) = Q K_j^T into S buffer g % 2 and dP(g) = dO V_j^T, both with Q / dO and K / V' read
+//   from shared memory; the 16 warps turn S(g), dP(g) into dS(g) (bf16, over S(g)'s columns);
+//   dQ += dS(g) K_j with K read MN-major.  Issue order of the MMA thread:
+//     S(0) dP(0) | S(1) [wait dS(0)] dP(1) dQ(0) | S(2) [wait dS(1)] dP(2) dQ(1) | ...
+//   so while the warps work on tile g the tensor pipe runs dQ(g - 1) and S(g + 1), and only dP(g + 1)
+//   waits for them.  S(g + 2) overwrites the buffer whose dS(g) the dQ(g) product issued just
+//   before it reads (products execute in issue order).
 template <int D>
 __global__ void __launch_bounds__(576, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -223,14 +229,14 @@ __global__ void __launch_bounds__(576, 1)
     uint8_t* sKV = sdO + C::TILE_BYTES;          // NS tiles: K_j, V'_j alternately
     uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NS * C::TILE_BYTES);
     uint64_t* b_qfull = bars + 0;                // Q and dO tiles landed
-    uint64_t* b_qempty = bars + 1;               // both copied into tensor memory
+    uint64_t* b_qempty = bars + 1;               // the item's products are done reading them
     uint64_t* b_ofull = bars + 2;                // dQ of the item complete
     uint64_t* b_oempty = bars + 3;               // dQ read by the epilogue
     uint64_t* b_mdrain = bars + 4;
     uint64_t* b_itfull = bars + 5;               // [2]
     uint64_t* b_itempty = bars + 7;              // [2]
-    uint64_t* b_sfull = bars + 9;                // S and dP of the current key tile ready
-    uint64_t* b_pfull = bars + 10;               // dS written to tensor memory
+    uint64_t* b_sfull = bars + 9;                // S(g) and dP(g) complete
+    uint64_t* b_pfull = bars + 10;               // dS(g) written to tensor memory
     uint64_t* b_kvfull = bars + 11;              // [NS]
     uint64_t* b_kvempty = bars + 11 + NS;        // [NS]
     int* s_item = reinterpret_cast<int*>(bars + 11 + 2 * NS);   // [2]
@@ -310,6 +316,11 @@ __global__ void __launch_bounds__(576, 1)
                 mbar_arrive(smem_u32(b_itfull + slot));
                 if (it < 0) break;
                 const BwdQItem m = bwd_q_item(p, it);
+                // Warm L2 with this item's Q and dO while the previous item finishes with its own.
+                for (int ch = 0; ch < C::NCHUNK; ++ch) {
+                    tma_prefetch_4d(&tm_q, ch * 64, m.h, m.q0, m.b);
+                    tma_prefetch_4d(&tm_do, ch * 64, m.h, m.q0, m.b);
+                }
                 if (q_uses > 0 && !(ok = mbar_wait(smem_u32(b_qempty), (q_uses - 1) & 1u, lim, kSiteBwdQEmpty)))
                     break;
                 {
@@ -337,12 +348,12 @@ __global__ void __launch_bounds__(576, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);   // S, dP: N = 128 keys
             constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, true);     // dQ: B = K MN-major
-            const uint64_t dq_src = smem_desc_sw128(smem_u32(sQ), 16, 1024);
-            const uint64_t ddo_src = smem_desc_sw128(smem_u32(sdO), 16, 1024);
+            const uint64_t a_q = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+            const uint64_t a_do = smem_desc_sw128(smem_u32(sdO), 16, 1024);
             const uint64_t dkv_k = smem_desc_sw128(smem_u32(sKV), 16, 1024);
             const uint64_t dkv_mn = smem_desc_sw128(smem_u32(sKV), C::CHUNK_BYTES, 1024);
             uint32_t stage = 0, phase = 0;
-            uint32_t p_cnt = 0;   // dS hand-overs consumed
+            uint32_t g = 0;       // tiles over this CTA's items: S buffer g & 1, barrier parities
             uint32_t uses = 0;    // items done
             auto acquire = [&](uint32_t& s) -> bool {
                 s = stage;
@@ -353,6 +364,22 @@ __global__ void __launch_bounds__(576, 1)
                 }
                 return r;
             };
+            auto s_mma = [&](uint32_t buf, uint32_t sk) {
+                const uint64_t bk = dkv_k + (uint64_t)((sk * C::TILE_BYTES) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(tmem + C::DQ_COL_S + 128u * buf, a_q + kmajor_step<D>(kk), bk + kmajor_step<D>(kk), idesc_s,
+                           kk > 0 ? 1u : 0u);
+            };
+            auto dp_mma = [&](uint32_t sv) {
+                const uint64_t bv = dkv_k + (uint64_t)((sv * C::TILE_BYTES) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(tmem + C::DQ_COL_DP, a_do + kmajor_step<D>(kk), bv + kmajor_step<D>(kk), idesc_s,
+                           kk > 0 ? 1u : 0u);
+                mma_commit(smem_u32(b_sfull));
+                mma_commit(smem_u32(b_kvempty + sv));
+            };
             bool ok = true;
             for (uint32_t k = 0; ok; ++k) {
                 const uint32_t slot = k & 1u;
@@ -361,45 +388,43 @@ __global__ void __launch_bounds__(576, 1)
                 mbar_arrive(smem_u32(b_itempty + slot));
                 if (it < 0) break;
                 const BwdQItem m = bwd_q_item(p, it);
-                // Q and dO into tensor memory (after the previous item's products on the same pipe).
                 if (!(ok = mbar_wait(smem_u32(b_qfull), uses & 1u, lim, kSiteBwdQFull))) break;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    tmem_cp_128x256b(tmem + C::DQ_COL_Q + 8u * kk, dq_src + kmajor_step<D>(kk));
-                    tmem_cp_128x256b(tmem + C::DQ_COL_DO + 8u * kk, ddo_src + kmajor_step<D>(kk));
-                }
-                mma_commit(smem_u32(b_qempty));
-                for (int j = m.lo; ok && j <= m.hi; ++j) {
-                    uint32_t sk = 0, sv = 0;
-                    if (!(ok = acquire(sk))) break;
-                    const uint64_t bk = dkv_k + (uint64_t)((sk * C::TILE_BYTES) >> 4);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ts(tmem + C::DQ_COL_S, tmem + C::DQ_COL_Q + 8u * kk, bk + kmajor_step<D>(kk), idesc_s,
-                               kk > 0 ? 1u : 0u);
-                    if (!(ok = acquire(sv))) break;
-                    const uint64_t bv = dkv_k + (uint64_t)((sv * C::TILE_BYTES) >> 4);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ts(tmem + C::DQ_COL_DP, tmem + C::DQ_COL_DO + 8u * kk, bv + kmajor_step<D>(kk), idesc_s,
-                               kk > 0 ? 1u : 0u);
-                    mma_commit(smem_u32(b_sfull));
-                    mma_commit(smem_u32(b_kvempty + sv));
-                    if (!(ok = mbar_wait(smem_u32(b_pfull), p_cnt & 1u, lim, kSiteBwdPFull))) break;
-                    ++p_cnt;
-                    if (j == m.lo && uses > 0 &&
+                const int n = m.hi - m.lo + 1;
+                uint32_t sk_cur = 0, sk_next = 0, sv = 0;
+                if (!(ok = acquire(sk_cur))) break;
+                s_mma(g & 1u, sk_cur);
+                if (!(ok = acquire(sv))) break;
+                dp_mma(sv);
+                for (int t = 0; ok && t < n; ++t) {
+                    const bool more = t + 1 < n;
+                    if (more) {
+                        if (!(ok = acquire(sk_next))) break;
+                        s_mma((g + 1u) & 1u, sk_next);
+                    }
+                    if (!(ok = mbar_wait(smem_u32(b_pfull), g & 1u, lim, kSiteBwdPFull))) break;
+                    if (t == 0 && uses > 0 &&
                         !(ok = mbar_wait(smem_u32(b_oempty), (uses - 1) & 1u, lim, kSiteBwdOEmpty)))
                         break;
                     tc_fence_after();
-                    // dQ += dS K_j: K = 128 keys in steps of 16; dS of keys 32 c + i at column 32 c + i / 2.
-                    const uint64_t bkm = dkv_mn + (uint64_t)((sk * C::TILE_BYTES) >> 4);
+                    if (more) {
+                        if (!(ok = acquire(sv))) break;
+                        dp_mma(sv);
+                    }
+                    // dQ += dS K_j: K = 128 keys in steps of 16; dS of keys 32 c + i at column
+                    // 32 c + i / 2 of the tile's S buffer.
+                    const uint64_t bkm = dkv_mn + (uint64_t)((sk_cur * C::TILE_BYTES) >> 4);
+                    const uint32_t a_ds = tmem + C::DQ_COL_S + 128u * (g & 1u);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_ts(tmem + C::DQ_COL_DQ, tmem + C::DQ_COL_S + (kk >> 1) * 32 + (kk & 1) * 8,
-                               bkm + (uint64_t)((kk * 16 * 128) >> 4), idesc_dq, (j > m.lo || kk > 0) ? 1u : 0u);
-                    mma_commit(smem_u32(b_kvempty + sk));
-                    if (j == m.hi) mma_commit(smem_u32(b_ofull));
+                        mma_ts(tmem + C::DQ_COL_DQ, a_ds + (kk >> 1) * 32 + (kk & 1) * 8,
+                               bkm + (uint64_t)((kk * 16 * 128) >> 4), idesc_dq, (t > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(smem_u32(b_kvempty + sk_cur));
+                    sk_cur = sk_next;
+                    ++g;
                 }
+                if (!ok) break;
+                mma_commit(smem_u32(b_qempty));
+                mma_commit(smem_u32(b_ofull));
                 ++uses;
             }
             mma_commit(smem_u32(b_mdrain));
@@ -411,7 +436,7 @@ __global__ void __launch_bounds__(576, 1)
         const int cq = (warp - kSoftmaxWarp0) >> 2;   // key / output column quarter
         const int r = ((warp & 3) << 5) + lane;       // tile row = tensor-memory lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        uint32_t s_cnt = 0, o_uses = 0;
+        uint32_t g = 0, o_uses = 0;
         bool ok = true;
         for (uint32_t k = 0; ok; ++k) {
             const uint32_t slot = k & 1u;
@@ -428,15 +453,14 @@ __global__ void __launch_bounds__(576, 1)
             const int qi = m.q0 + r;
             const float2 rs = p.rowstat[((long long)m.b * p.H + m.h) * p.Tp + qi];
             const float nl = -rs.x, dl = rs.y;
-            for (int j = m.lo; j <= m.hi; ++j) {
-                const bool w = mbar_wait(smem_u32(b_sfull), s_cnt & 1u, lim, kSiteBwdSFull);
+            for (int j = m.lo; j <= m.hi; ++j, ++g) {
+                const bool w = mbar_wait(smem_u32(b_sfull), g & 1u, lim, kSiteBwdSFull);
                 ok = __all_sync(0xffffffffu, w);
                 if (!ok) break;
-                ++s_cnt;
                 tc_fence_after();
                 const int k0 = j * 128 + 32 * cq;
                 uint32_t sv[2][16], dv[2][16], pk[16];
-                const uint32_t colS = C::DQ_COL_S + 32u * (uint32_t)cq;
+                const uint32_t colS = C::DQ_COL_S + 128u * (g & 1u) + 32u * (uint32_t)cq;
                 const uint32_t colP = C::DQ_COL_DP + 32u * (uint32_t)cq;
                 tmem_ld16(tmem + lane_base + colS, sv[0]);
                 tmem_ld16(tmem + lane_base + colS + 16u, sv[1]);
@@ -501,6 +525,13 @@ __global__ void __launch_bounds__(576, 1)
 
 // ---------------------------------------------------------------- key-tile kernel (dK, dV)
 
+// Per item (key tile of (b, hk); steps s over the G query heads x query tiles that see it):
+//   S^T(s) = K Q_s^T and dP^T(s) = V' dO_s^T (shared-memory operands), then the 16 warps in two
+//   phases: A turns S^T into P^T (bf16, over S^T's columns; P stays in registers), B turns dP^T
+//   into dS^T = P^T (dP^T - (delta - dlse)) (bf16, over dP^T's columns).  Issue order:
+//     S^T(0) dP^T(0) | [P^T(0)] dV(0) S^T(1) [dS^T(0)] dK(0) dP^T(1) | [P^T(1)] dV(1) S^T(2) ...
+//   so phase A of step s + 1 waits only for dV(s) and S^T(s + 1), and phase B for dK(s) and
+//   dP^T(s + 1); each overwrite of a buffer follows, in issue order, the product that reads it.
 template <int D>
 __global__ void __launch_bounds__(576, 1)
     attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -524,11 +555,13 @@ __global__ void __launch_bounds__(576, 1)
     uint64_t* b_mdrain = bars + 4;
     uint64_t* b_itfull = bars + 5;               // [2]
     uint64_t* b_itempty = bars + 7;              // [2]
-    uint64_t* b_sfull = bars + 9;
-    uint64_t* b_pfull = bars + 10;
-    uint64_t* b_stfull = bars + 11;              // [NS]
-    uint64_t* b_stempty = bars + 11 + NS;        // [NS]
-    int* s_item = reinterpret_cast<int*>(bars + 11 + 2 * NS);
+    uint64_t* b_stready = bars + 9;              // S^T(s) complete
+    uint64_t* b_dpready = bars + 10;             // dP^T(s) complete
+    uint64_t* b_pready = bars + 11;              // P^T(s) written
+    uint64_t* b_dsready = bars + 12;             // dS^T(s) written
+    uint64_t* b_stfull = bars + 13;              // [NS]
+    uint64_t* b_stempty = bars + 13 + NS;        // [NS]
+    int* s_item = reinterpret_cast<int*>(bars + 13 + 2 * NS);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_item + 2);
 
     const int warp = threadIdx.x >> 5;
@@ -548,8 +581,10 @@ __global__ void __launch_bounds__(576, 1)
             mbar_init(smem_u32(b_itfull + i), 1);
             mbar_init(smem_u32(b_itempty + i), kItemConsumers);
         }
-        mbar_init(smem_u32(b_sfull), 1);
-        mbar_init(smem_u32(b_pfull), C::SOFTMAX_THREADS);
+        mbar_init(smem_u32(b_stready), 1);
+        mbar_init(smem_u32(b_dpready), 1);
+        mbar_init(smem_u32(b_pready), C::SOFTMAX_THREADS);
+        mbar_init(smem_u32(b_dsready), C::SOFTMAX_THREADS);
         for (int s = 0; s < NS; ++s) {
             mbar_init(smem_u32(b_stfull + s), 1);
             mbar_init(smem_u32(b_stempty + s), 1);
@@ -590,6 +625,11 @@ __global__ void __launch_bounds__(576, 1)
                 mbar_arrive(smem_u32(b_itfull + slot));
                 if (it < 0) break;
                 const BwdKvItem m = bwd_kv_item(p, it);
+                // Warm L2 with this item's K and V' while the previous item still uses its own.
+                for (int ch = 0; ch < C::NCHUNK; ++ch) {
+                    tma_prefetch_4d(&tm_k, ch * 64, m.hk, m.k0, m.b);
+                    tma_prefetch_4d(&tm_v, ch * 64, m.hk, m.k0, m.b);
+                }
                 if (kv_uses > 0 && !(ok = mbar_wait(smem_u32(b_kempty), (kv_uses - 1) & 1u, lim, kSiteBwdKvEmpty)))
                     break;
                 {
@@ -642,7 +682,32 @@ __global__ void __launch_bounds__(576, 1)
             const uint64_t b_kmaj = smem_desc_sw128(smem_u32(sSt), 16, 1024);
             const uint64_t b_mn = smem_desc_sw128(smem_u32(sSt), C::CHUNK_BYTES, 1024);
             uint32_t stage = 0, phase = 0;
-            uint32_t p_cnt = 0, uses = 0;
+            uint32_t g = 0, uses = 0;   // steps over this CTA's items (barrier parities); items done
+            auto acquire = [&](uint32_t& sg) -> bool {
+                sg = stage;
+                const bool r = mbar_wait(smem_u32(b_stfull + stage), phase, lim, kSiteBwdStage);
+                if (++stage == (uint32_t)NS) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                return r;
+            };
+            auto st_mma = [&](uint32_t sg) {
+                const uint64_t qoff = (uint64_t)((sg * C::STAGE_BYTES) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(tmem + C::KV_COL_ST, a_k + kmajor_step<D>(kk), b_kmaj + qoff + kmajor_step<D>(kk),
+                           idesc_s, kk > 0 ? 1u : 0u);
+                mma_commit(smem_u32(b_stready));
+            };
+            auto dpt_mma = [&](uint32_t sg) {
+                const uint64_t dooff = (uint64_t)((sg * C::STAGE_BYTES + C::TILE_BYTES) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(tmem + C::KV_COL_DPT, a_v + kmajor_step<D>(kk), b_kmaj + dooff + kmajor_step<D>(kk),
+                           idesc_s, kk > 0 ? 1u : 0u);
+                mma_commit(smem_u32(b_dpready));
+            };
             bool ok = true;
             for (uint32_t k = 0; ok; ++k) {
                 const uint32_t slot = k & 1u;
@@ -653,41 +718,39 @@ __global__ void __launch_bounds__(576, 1)
                 const BwdKvItem m = bwd_kv_item(p, it);
                 if (!(ok = mbar_wait(smem_u32(b_kfull), uses & 1u, lim, kSiteBwdKvFull))) break;
                 const int n_steps = p.G * (m.hi - m.lo + 1);
+                uint32_t sg = 0, sg_next = 0;
+                if (!(ok = acquire(sg))) break;
+                st_mma(sg);
+                dpt_mma(sg);
                 for (int s = 0; ok && s < n_steps; ++s) {
-                    const uint32_t sg = stage;
-                    if (!(ok = mbar_wait(smem_u32(b_stfull + stage), phase, lim, kSiteBwdStage))) break;
-                    if (++stage == (uint32_t)NS) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    const bool more = s + 1 < n_steps;
                     const uint64_t qoff = (uint64_t)((sg * C::STAGE_BYTES) >> 4);
                     const uint64_t dooff = (uint64_t)((sg * C::STAGE_BYTES + C::TILE_BYTES) >> 4);
-                    // S^T = K Q^T and dP^T = V' dO^T: M = 128 keys, N = 128 queries, K = D.
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ss(tmem + C::KV_COL_ST, a_k + kmajor_step<D>(kk), b_kmaj + qoff + kmajor_step<D>(kk),
-                               idesc_s, kk > 0 ? 1u : 0u);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ss(tmem + C::KV_COL_DPT, a_v + kmajor_step<D>(kk), b_kmaj + dooff + kmajor_step<D>(kk),
-                               idesc_s, kk > 0 ? 1u : 0u);
-                    mma_commit(smem_u32(b_sfull));
-                    if (!(ok = mbar_wait(smem_u32(b_pfull), p_cnt & 1u, lim, kSiteBwdPFull))) break;
-                    ++p_cnt;
-                    if (s == 0 && uses > 0 && !(ok = mbar_wait(smem_u32(b_oempty), (uses - 1) & 1u, lim, kSiteBwdOEmpty)))
+                    if (!(ok = mbar_wait(smem_u32(b_pready), g & 1u, lim, kSiteBwdPFull))) break;
+                    if (s == 0 && uses > 0 &&
+                        !(ok = mbar_wait(smem_u32(b_oempty), (uses - 1) & 1u, lim, kSiteBwdOEmpty)))
                         break;
                     tc_fence_after();
-                    // dV += P^T dO and dK += dS^T Q: K = 128 queries in steps of 16; P^T / dS^T of
-                    // queries 32 c + i at column 32 c + i / 2 of their buffers.
+                    // dV += P^T dO: K = 128 queries in steps of 16; P^T of queries 32 c + i at
+                    // column 32 c + i / 2 of the S^T buffer.
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         mma_ts(tmem + C::KV_COL_DV, tmem + C::KV_COL_ST + (kk >> 1) * 32 + (kk & 1) * 8,
                                b_mn + dooff + (uint64_t)((kk * 16 * 128) >> 4), idesc_g, (s > 0 || kk > 0) ? 1u : 0u);
+                    if (more) {
+                        if (!(ok = acquire(sg_next))) break;
+                        st_mma(sg_next);
+                    }
+                    if (!(ok = mbar_wait(smem_u32(b_dsready), g & 1u, lim, kSiteBwdSFull))) break;
+                    tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         mma_ts(tmem + C::KV_COL_DK, tmem + C::KV_COL_DPT + (kk >> 1) * 32 + (kk & 1) * 8,
                                b_mn + qoff + (uint64_t)((kk * 16 * 128) >> 4), idesc_g, (s > 0 || kk > 0) ? 1u : 0u);
                     mma_commit(smem_u32(b_stempty + sg));
+                    if (more) dpt_mma(sg_next);
+                    sg = sg_next;
+                    ++g;
                 }
                 if (!ok) break;
                 mma_commit(smem_u32(b_ofull));
@@ -703,8 +766,10 @@ __global__ void __launch_bounds__(576, 1)
         const int cq = (warp - kSoftmaxWarp0) >> 2;   // query / output column quarter
         const int r = ((warp & 3) << 5) + lane;       // key row = tensor-memory lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t colS = C::KV_COL_ST + 32u * (uint32_t)cq;
+        const uint32_t colP = C::KV_COL_DPT + 32u * (uint32_t)cq;
         uint32_t stage = 0, phase = 0;
-        uint32_t s_cnt = 0, o_uses = 0;
+        uint32_t g = 0, o_uses = 0;
         bool ok = true;
         for (uint32_t k = 0; ok; ++k) {
             const uint32_t slot = k & 1u;
@@ -721,16 +786,15 @@ __global__ void __launch_bounds__(576, 1)
             const int key = m.k0 + r;
             const int nq = m.hi - m.lo + 1;
             const int n_steps = p.G * nq;
-            for (int s = 0; s < n_steps; ++s) {
+            for (int s = 0; s < n_steps; ++s, ++g) {
                 const int i = m.lo + s % nq;
                 const uint32_t sg = stage;
-                // The score products of this step are complete, and (through the stage's own
-                // barrier, still in this phase) so is the copy of its row statistics.
-                bool w = mbar_wait(smem_u32(b_sfull), s_cnt & 1u, lim, kSiteBwdSFull);
+                // Phase A: S^T(s) is complete, and (through the stage's own barrier, still in this
+                // phase) so is the copy of its row statistics.
+                bool w = mbar_wait(smem_u32(b_stready), g & 1u, lim, kSiteBwdSFull);
                 w = w && mbar_wait(smem_u32(b_stfull + sg), phase, lim, kSiteBwdStage);
                 ok = __all_sync(0xffffffffu, w);
                 if (!ok) break;
-                ++s_cnt;
                 if (++stage == (uint32_t)NS) {
                     stage = 0;
                     phase ^= 1u;
@@ -738,35 +802,49 @@ __global__ void __launch_bounds__(576, 1)
                 tc_fence_after();
                 const float2* rs = reinterpret_cast<const float2*>(sSt + sg * C::STAGE_BYTES + 2 * C::TILE_BYTES) + 32 * cq;
                 const int qc0 = i * 128 + 32 * cq;      // first query column of this thread
-                uint32_t sv[2][16], dv[2][16], pp[16], pd[16];
-                const uint32_t colS = C::KV_COL_ST + 32u * (uint32_t)cq;
-                const uint32_t colP = C::KV_COL_DPT + 32u * (uint32_t)cq;
-                tmem_ld16(tmem + lane_base + colS, sv[0]);
-                tmem_ld16(tmem + lane_base + colS + 16u, sv[1]);
-                tmem_ld16(tmem + lane_base + colP, dv[0]);
-                tmem_ld16(tmem + lane_base + colP + 16u, dv[1]);
-                tmem_ld_wait();
+                float pv[32];
+                {
+                    uint32_t sv[2][16], pp[16];
+                    tmem_ld16(tmem + lane_base + colS, sv[0]);
+                    tmem_ld16(tmem + lane_base + colS + 16u, sv[1]);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int hb = 0; hb < 2; ++hb) {
-#pragma unroll
-                    for (int e = 0; e < 16; e += 2) {
-                        const int c = 16 * hb + e;
+                    for (int c = 0; c < 32; c += 2) {
                         const float2 r0 = rs[c], r1 = rs[c + 1];
-                        float p0 = ex2_approx(fmaf(__uint_as_float(sv[hb][e]), p.c1, -r0.x));
-                        float p1 = ex2_approx(fmaf(__uint_as_float(sv[hb][e + 1]), p.c1, -r1.x));
+                        float p0 = ex2_approx(fmaf(__uint_as_float(sv[c >> 4][c & 15]), p.c1, -r0.x));
+                        float p1 = ex2_approx(fmaf(__uint_as_float(sv[c >> 4][(c & 15) + 1]), p.c1, -r1.x));
                         if ((unsigned)(qc0 + c - key) >= (unsigned)p.W) p0 = 0.f;
                         if ((unsigned)(qc0 + c + 1 - key) >= (unsigned)p.W) p1 = 0.f;
-                        const float d0 = p0 * (__uint_as_float(dv[hb][e]) - r0.y);
-                        const float d1 = p1 * (__uint_as_float(dv[hb][e + 1]) - r1.y);
-                        pp[8 * hb + (e >> 1)] = pack_bf16x2(p0, p1);
-                        pd[8 * hb + (e >> 1)] = pack_bf16x2(d0, d1);
+                        pv[c] = p0;
+                        pv[c + 1] = p1;
+                        pp[c >> 1] = pack_bf16x2(p0, p1);
                     }
+                    tmem_st16(tmem + lane_base + colS, pp);
+                    tmem_st_wait();
                 }
-                tmem_st16(tmem + lane_base + colS, pp);
-                tmem_st16(tmem + lane_base + colP, pd);
-                tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(smem_u32(b_pfull));
+                mbar_arrive(smem_u32(b_pready));
+                // Phase B: dP^T(s) is complete.
+                w = mbar_wait(smem_u32(b_dpready), g & 1u, lim, kSiteBwdSFull);
+                ok = __all_sync(0xffffffffu, w);
+                if (!ok) break;
+                tc_fence_after();
+                {
+                    uint32_t dv[2][16], pd[16];
+                    tmem_ld16(tmem + lane_base + colP, dv[0]);
+                    tmem_ld16(tmem + lane_base + colP + 16u, dv[1]);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < 32; c += 2) {
+                        const float d0 = pv[c] * (__uint_as_float(dv[c >> 4][c & 15]) - rs[c].y);
+                        const float d1 = pv[c + 1] * (__uint_as_float(dv[c >> 4][(c & 15) + 1]) - rs[c + 1].y);
+                        pd[c >> 1] = pack_bf16x2(d0, d1);
+                    }
+                    tmem_st16(tmem + lane_base + colP, pd);
+                    tmem_st_wait();
+                }
+                tc_fence_before();
+                mbar_arrive(smem_u32(b_dsready));
             }
             if (!ok) break;
             {
@@ -912,7 +990,8 @@ __global__ void bwd_gate_x_kernel(const float* __restrict__ dz, const __nv_bfloa
 }
 
 // dWg in two passes with a fixed order: block blk sums rows [blk R, blk R + R) into
-// part[blk][c Hkv + hk]; the final pass adds the blocks in index order.
+// part[blk][c Hkv + hk]; the final pass gives each output one block, whose threads add strided
+// partials and then combine them by a tree in shared memory.
 __global__ void bwd_wg_partial_kernel(const float* __restrict__ dz, const __nv_bfloat16* __restrict__ gate_x,
                                       float* __restrict__ part, long long n_bt, int Hkv, int rows_per_block) {
     const int n = 32 * Hkv;
@@ -922,17 +1001,25 @@ __global__ void bwd_wg_partial_kernel(const float* __restrict__ dz, const __nv_b
         const int c = idx / Hkv;
         const int hk = idx - c * Hkv;
         float acc = 0.f;
+#pragma unroll 8
         for (long long bt = r0; bt < r1; ++bt) acc += dz[bt * Hkv + hk] * __bfloat162float(gate_x[bt * 32 + c]);
         part[(long long)blockIdx.x * n + idx] = acc;
     }
 }
 
+// One block of 256 threads per output index.
 __global__ void bwd_wg_final_kernel(const float* __restrict__ part, float* __restrict__ dWg, int n_blocks, int n) {
-    for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < n; idx += gridDim.x * blockDim.x) {
-        float acc = 0.f;
-        for (int b = 0; b < n_blocks; ++b) acc += part[(long long)b * n + idx];
-        dWg[idx] = acc;
+    __shared__ float red[256];
+    const int idx = blockIdx.x;
+    float acc = 0.f;
+    for (int b = threadIdx.x; b < n_blocks; b += 256) acc += part[(long long)b * n + idx];
+    red[threadIdx.x] = acc;
+    __syncthreads();
+    for (int w = 128; w > 0; w >>= 1) {
+        if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+        __syncthreads();
     }
+    if (threadIdx.x == 0) dWg[idx] = red[0];
 }
 
 }  // namespace swa

@@ -365,7 +365,7 @@ BwdLayout bwd_layout(const Shape& s, bool has_ve) {
     w.Tp = ((s.T + 127) / 128) * 128;
     const long long n_bt = (long long)s.B * s.T;
     const size_t kv_f32 = round_up((size_t)n_bt * s.Hkv * s.D * 4);
-    w.wg_rows = 256;
+    w.wg_rows = 32;
     w.wg_blocks = has_ve ? (int)((n_bt + w.wg_rows - 1) / w.wg_rows) : 0;
     size_t o = w.f.total;
     w.rowstat = o;
@@ -400,7 +400,7 @@ int launch_backward(int dev, const void* q, const void* k, const void* v, const 
     float2* rowstat = reinterpret_cast<float2*>(ws + L.rowstat);
     {
         const long long rows = (long long)s.B * s.H * L.Tp;
-        const int blocks = (int)std::min<long long>((rows + 7) / 8, 148ll * 16);
+        const int blocks = (int)((rows * (s.D / 8) + 255) / 256);   // D / 8 lanes per row
         if (s.D == 128)
             swa::bwd_rowstat_kernel<128><<<blocks, 256, 0, st>>>(static_cast<const bf*>(out), static_cast<const bf*>(dout),
                                                                  lse, dlse, rowstat, s.B, s.T, s.H, L.Tp, sched4);
@@ -485,7 +485,7 @@ int launch_backward(int dev, const void* q, const void* k, const void* v, const 
         swa::bwd_wg_partial_kernel<<<L.wg_blocks, 256, 0, st>>>(dz, static_cast<const bf*>(gate_x), part, n_bt,
                                                                 s.Hkv, L.wg_rows);
         const int n = 32 * s.Hkv;
-        swa::bwd_wg_final_kernel<<<(n + 255) / 256, 256, 0, st>>>(part, dWg, L.wg_blocks, n);
+        swa::bwd_wg_final_kernel<<<n, 256, 0, st>>>(part, dWg, L.wg_blocks, n);
     }
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
