@@ -9,7 +9,7 @@ Two independent implementations live here:
 
 * ``forward`` / ``prologue``: the C oracle (``swa_oracle.c``), one query row at a time, fp64.
 * ``backward``: the gradient of the same layer (chain rule through the five steps in
-  reverse), also in ``swa_oracle.c``.
+  reverse), also in ``swa_oracle.c``; ``backward_rows`` gives the same values at sampled rows.
 * ``brute.py``: a NumPy fp64 restatement that materialises the full T x T score matrix, used
   as the brute-force pin of the C oracle on small shapes.
 
@@ -60,6 +60,13 @@ def _configure(lib):
                                             ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                             ctypes.c_double, ctypes.c_int, ctypes.c_int,
                                             ctypes.c_int, ctypes.c_int, P, P, P, P, P, P, P, P]
+    lib.swa_oracle_backward_rows_gqa.restype = ctypes.c_int
+    lib.swa_oracle_backward_rows_gqa.argtypes = [P, P, P, P, P, ctypes.c_int, P, ctypes.c_int, P,
+                                                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                 ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                                 ctypes.c_double, ctypes.c_int, ctypes.c_int,
+                                                 ctypes.c_int, ctypes.c_int, P, P,
+                                                 P, ctypes.c_int64, P, P, ctypes.c_int64, P, P, P]
     lib.swa_oracle_threads.restype = ctypes.c_int
     lib.swa_oracle_round_bf16.restype = ctypes.c_double
     lib.swa_oracle_round_bf16.argtypes = [ctypes.c_double]
@@ -233,6 +240,39 @@ def backward(inputs: Dict, dout, window: int, dlse=None, rope_base: float = 1000
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     return grads
+
+
+def backward_rows(inputs: Dict, dout, window: int, dlse=None, *, qrows=(), krows=(),
+                  rope_base: float = 10000.0, eps: float = 1e-6, parity: bool = True,
+                  rope: bool = True, qknorm: bool = True, window_convention: int = 0):
+    """``backward`` at sampled rows, bit for bit: qrows are flat query ids ((b*H + h)*T + i),
+    krows flat key/value ids ((b*Hkv + hk)*T + j).  Returns dq [len(qrows), D] and dk, dv (and dve
+    on value-embedding layers) [len(krows), D], in the order of the requests."""
+    lib = _load()
+    q, k, v = _bits(inputs["q"]), _bits(inputs["k"]), _bits(inputs["v"])
+    B, T, H, D = q.shape
+    Hkv = int(k.shape[2])
+    ids, table, vocab, x, C, Wg = _ve_args(inputs)
+    go = np.ascontiguousarray(_as_f64(dout))
+    if go.shape != (B, T, H, D):
+        raise ValueError("dout must be (B, T, H, D)")
+    gl = None if dlse is None else np.ascontiguousarray(_as_f64(dlse))
+    if gl is not None and gl.shape != (B, H, T):
+        raise ValueError("dlse must be (B, H, T)")
+    qa = np.ascontiguousarray(np.asarray(qrows, dtype=np.int64).reshape(-1))
+    ka = np.ascontiguousarray(np.asarray(krows, dtype=np.int64).reshape(-1))
+    out = dict(dq=np.empty((qa.size, D)), dk=np.empty((ka.size, D)), dv=np.empty((ka.size, D)))
+    if ids is not None:
+        out["dve"] = np.empty((ka.size, D))
+    rc = lib.swa_oracle_backward_rows_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(ids), _ptr(table), vocab,
+                                          _ptr(x), C, _ptr(Wg), B, T, H, Hkv, D, int(window),
+                                          float(rope_base), float(eps), int(parity), int(rope),
+                                          int(qknorm), int(window_convention), _ptr(go), _ptr(gl),
+                                          _ptr(qa), int(qa.size), _ptr(out["dq"]), _ptr(ka), int(ka.size),
+                                          _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out.get("dve")))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return out
 
 
 def _as_f64(a) -> np.ndarray:

@@ -367,6 +367,83 @@ static double dot_d(const double* a, const double* b, int D) {
     return acc;
 }
 
+/* Row pass for query row i of one (b, h): scores against the visible keys (scratch s of T),
+ * lse_i, delta_i = sum_j P_ij dP_ij and, if dqi is not NULL, dqhat_i = sum_j dS_ij khat_j / sqrt(D).
+ * gi is dout of the row, gl its dlse. */
+static void bwd_query_row(const double* qi, const double* gi, double gl, const double* kh,
+                          const double* vp, int T, int D, int i, int W, int window_convention,
+                          double inv_sqrt_d, double* s, double* lse_i, double* delta_i, double* dqi) {
+    double M = -INFINITY;
+    for (int j = 0; j < T; ++j) {
+        if (!visible(i, j, W, window_convention)) continue;
+        s[j] = dot_d(qi, kh + (size_t)j * D, D) * inv_sqrt_d;
+        if (s[j] > M) M = s[j];
+    }
+    double L = 0.0;
+    for (int j = 0; j < T; ++j)
+        if (visible(i, j, W, window_convention)) L += exp(s[j] - M);
+    const double li = M + log(L);
+    double dl = 0.0;
+    for (int j = 0; j < T; ++j)
+        if (visible(i, j, W, window_convention))
+            dl += exp(s[j] - li) * dot_d(gi, vp + (size_t)j * D, D);
+    *lse_i = li;
+    *delta_i = dl;
+    if (dqi == NULL) return;
+    for (int d = 0; d < D; ++d) dqi[d] = 0.0;
+    for (int j = 0; j < T; ++j) {
+        if (!visible(i, j, W, window_convention)) continue;
+        const double p = exp(s[j] - li);
+        const double ds = p * (dot_d(gi, vp + (size_t)j * D, D) - dl) + p * gl;
+        for (int d = 0; d < D; ++d) dqi[d] += ds * kh[(size_t)j * D + d] * inv_sqrt_d;
+    }
+}
+
+/* Key pass for key row j of one (b, h): adds sum_i dS_ij qhat_i / sqrt(D) to dkj and
+ * sum_i P_ij dout_i to dvj over the queries i in [j, i_end] that see key j.  qh, lse, delta are
+ * indexed by query position; dout / dlse are the full tensors. */
+static void bwd_key_row(const double* kj, const double* vj, const double* qh, const double* lse,
+                        const double* delta, const double* dout, const double* dlse, int b, int h,
+                        int T, int H, int D, int j, int i_end, double inv_sqrt_d, double* dkj,
+                        double* dvj) {
+    for (int i = j; i <= i_end; ++i) {
+        const double* qi = qh + (size_t)i * D;
+        const double* gi = dout + (((size_t)b * T + i) * H + h) * (size_t)D;
+        const double gl = dlse ? dlse[((size_t)b * H + h) * T + i] : 0.0;
+        const double p = exp(dot_d(qi, kj, D) * inv_sqrt_d - lse[i]);
+        const double ds = p * (dot_d(gi, vj, D) - delta[i]) + p * gl;
+        for (int d = 0; d < D; ++d) {
+            dkj[d] += ds * qi[d] * inv_sqrt_d;
+            dvj[d] += p * gi[d];
+        }
+    }
+}
+
+/* dk, dv (and on value-embedding layers dve and dz) of key/value row (b, t, hk) from its dkhat and
+ * dv'.  dk_out / dv_out / dve_out receive D values; *dz_out the gate-logit gradient. */
+static void bwd_kv_outputs(const uint16_t* k, const int64_t* ids, const uint16_t* table,
+                           const uint16_t* x, int C, const uint16_t* Wg, int T, int Hkv, int D,
+                           int b, int t, int hk, double rope_base, double eps, int use_rope,
+                           int use_qknorm, const double* dkt, const double* dvt, double* dk_out,
+                           double* dv_out, double* dve_out, double* dz_out, double* xr) {
+    prologue_qk_backward(k, T, Hkv, D, b, t, hk, rope_base, eps, use_rope, use_qknorm, dkt, dk_out, xr);
+    for (int d = 0; d < D; ++d) dv_out[d] = dvt[d];
+    if (ids == NULL) return;
+    const uint16_t* xt = x + ((size_t)b * T + t) * (size_t)C;
+    double z = 0.0;
+    for (int c = 0; c < 32; ++c)
+        z += bf16_to_double(xt[c]) * bf16_to_double(Wg[(size_t)c * Hkv + hk]);
+    const double sig = 1.0 / (1.0 + exp(-z));
+    const int64_t id = ids[(size_t)b * T + t];
+    const uint16_t* ve = table + (size_t)id * (size_t)Hkv * D + (size_t)hk * D;
+    double dgate = 0.0;
+    for (int d = 0; d < D; ++d) {
+        dve_out[d] = 2.0 * sig * dvt[d];
+        dgate += dvt[d] * bf16_to_double(ve[d]);
+    }
+    *dz_out = dgate * 2.0 * sig * (1.0 - sig);
+}
+
 /*
  * Inputs as swa_oracle_forward_gqa, plus
  *   dout   fp64 (B, T, H, D): dL/d out.
@@ -445,33 +522,10 @@ int swa_oracle_backward_gqa(const uint16_t* q, const uint16_t* k, const uint16_t
                             bad = 1;
                             continue;
                         }
-                        const double* qi = qh + (size_t)i * D;
                         const double* gi = dout + (((size_t)b * T + i) * H + h) * (size_t)D;
                         const double gl = dlse ? dlse[((size_t)b * H + h) * T + i] : 0.0;
-                        double M = -INFINITY;
-                        for (int j = 0; j < T; ++j) {
-                            if (!visible(i, j, W, window_convention)) continue;
-                            s[j] = dot_d(qi, kh + (size_t)j * D, D) * inv_sqrt_d;
-                            if (s[j] > M) M = s[j];
-                        }
-                        double L = 0.0;
-                        for (int j = 0; j < T; ++j)
-                            if (visible(i, j, W, window_convention)) L += exp(s[j] - M);
-                        const double li = M + log(L);
-                        double dl = 0.0;
-                        for (int j = 0; j < T; ++j)
-                            if (visible(i, j, W, window_convention))
-                                dl += exp(s[j] - li) * dot_d(gi, vp + (size_t)j * D, D);
-                        lse[i] = li;
-                        delta[i] = dl;
-                        double* dqi = dqh + (size_t)i * D;
-                        for (int d = 0; d < D; ++d) dqi[d] = 0.0;
-                        for (int j = 0; j < T; ++j) {
-                            if (!visible(i, j, W, window_convention)) continue;
-                            const double p = exp(s[j] - li);
-                            const double ds = p * (dot_d(gi, vp + (size_t)j * D, D) - dl) + p * gl;
-                            for (int d = 0; d < D; ++d) dqi[d] += ds * kh[(size_t)j * D + d] * inv_sqrt_d;
-                        }
+                        bwd_query_row(qh + (size_t)i * D, gi, gl, kh, vp, T, D, i, W, window_convention,
+                                      inv_sqrt_d, s, &lse[i], &delta[i], dqh + (size_t)i * D);
                     }
                     free(s);
                 }
@@ -481,22 +535,9 @@ int swa_oracle_backward_gqa(const uint16_t* q, const uint16_t* k, const uint16_t
                  * see key j. */
                 #pragma omp parallel for schedule(dynamic, 8)
                 for (int j = 0; j < T; ++j) {
-                    const double* kj = kh + (size_t)j * D;
-                    const double* vj = vp + (size_t)j * D;
-                    double* dkj = dkh + (size_t)j * D;
-                    double* dvj = dvp + (size_t)j * D;
                     const int i_end = (j + reach < T - 1) ? j + reach : T - 1;
-                    for (int i = j; i <= i_end; ++i) {
-                        const double* qi = qh + (size_t)i * D;
-                        const double* gi = dout + (((size_t)b * T + i) * H + h) * (size_t)D;
-                        const double gl = dlse ? dlse[((size_t)b * H + h) * T + i] : 0.0;
-                        const double p = exp(dot_d(qi, kj, D) * inv_sqrt_d - lse[i]);
-                        const double ds = p * (dot_d(gi, vj, D) - delta[i]) + p * gl;
-                        for (int d = 0; d < D; ++d) {
-                            dkj[d] += ds * qi[d] * inv_sqrt_d;
-                            dvj[d] += p * gi[d];
-                        }
-                    }
+                    bwd_key_row(kh + (size_t)j * D, vp + (size_t)j * D, qh, lse, delta, dout, dlse, b, h,
+                                T, H, D, j, i_end, inv_sqrt_d, dkh + (size_t)j * D, dvp + (size_t)j * D);
                 }
 
                 /* dq rows of head h. */
@@ -533,25 +574,11 @@ int swa_oracle_backward_gqa(const uint16_t* q, const uint16_t* k, const uint16_t
                         continue;
                     }
                     const size_t off = (((size_t)b * T + t) * Hkv + hk) * (size_t)D;
-                    const double* dvt = dvp + (size_t)t * D;
-                    prologue_qk_backward(k, T, Hkv, D, b, t, hk, rope_base, eps, use_rope,
-                                         use_qknorm, dkh + (size_t)t * D, dk + off, xr);
-                    for (int d = 0; d < D; ++d) dv[off + d] = dvt[d];
-                    if (ids != NULL) {
-                        const uint16_t* xt = x + ((size_t)b * T + t) * (size_t)C;
-                        double z = 0.0;
-                        for (int c = 0; c < 32; ++c)
-                            z += bf16_to_double(xt[c]) * bf16_to_double(Wg[(size_t)c * Hkv + hk]);
-                        const double sig = 1.0 / (1.0 + exp(-z));
-                        const int64_t id = ids[(size_t)b * T + t];
-                        const uint16_t* ve = table + (size_t)id * (size_t)Hkv * D + (size_t)hk * D;
-                        double dgate = 0.0;
-                        for (int d = 0; d < D; ++d) {
-                            dve[off + d] = 2.0 * sig * dvt[d];
-                            dgate += dvt[d] * bf16_to_double(ve[d]);
-                        }
-                        dz[((size_t)b * T + t) * Hkv + hk] = dgate * 2.0 * sig * (1.0 - sig);
-                    }
+                    double dzt = 0.0;
+                    bwd_kv_outputs(k, ids, table, x, C, Wg, T, Hkv, D, b, t, hk, rope_base, eps, use_rope,
+                                   use_qknorm, dkh + (size_t)t * D, dvp + (size_t)t * D, dk + off, dv + off,
+                                   ids ? dve + off : NULL, &dzt, xr);
+                    if (ids != NULL) dz[((size_t)b * T + t) * Hkv + hk] = dzt;
                 }
                 free(xr);
             }
@@ -580,5 +607,150 @@ int swa_oracle_backward_gqa(const uint16_t* q, const uint16_t* k, const uint16_t
 
 done:
     free(kh); free(vp); free(qh); free(dkh); free(dvp); free(dqh); free(lse); free(delta); free(dz);
+    return rc;
+}
+
+/*
+ * The same gradient at sampled rows only, for checks at sizes where the full backward is too slow:
+ *   qrows[n_q]  flat query ids ((b*H + h)*T + i): dq of those rows -> dq_rows [n_q, D];
+ *   krows[n_k]  flat key/value ids ((b*Hkv + hk)*T + j): dk, dv (and dve on value-embedding
+ *               layers) of those rows -> dk_rows, dv_rows, dve_rows [n_k, D].
+ * Each requested value is computed by the same helpers, in the same order, as in
+ * swa_oracle_backward_gqa, from the query rows it depends on (those of its own row, or, for a
+ * key row j, the queries in [j, j + W - 1] of every query head of its group), so it equals the full
+ * backward's value bit for bit.  Returns 0, or -1 on bad arguments / allocation failure.
+ */
+int swa_oracle_backward_rows_gqa(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                 const int64_t* ids, const uint16_t* table, int vocab,
+                                 const uint16_t* x, int C, const uint16_t* Wg,
+                                 int B, int T, int H, int Hkv, int D, int window, double rope_base,
+                                 double eps, int round_bf16, int use_rope, int use_qknorm,
+                                 int window_convention, const double* dout, const double* dlse,
+                                 const int64_t* qrows, int64_t n_q, double* dq_rows,
+                                 const int64_t* krows, int64_t n_k, double* dk_rows,
+                                 double* dv_rows, double* dve_rows) {
+    if (B < 1 || T < 1 || H < 1 || D < 2 || (D % 2) != 0) return -1;
+    if (Hkv < 1 || Hkv > H || (H % Hkv) != 0) return -1;
+    if (dout == NULL || n_q < 0 || n_k < 0) return -1;
+    if (n_q > 0 && (qrows == NULL || dq_rows == NULL)) return -1;
+    if (n_k > 0 && (krows == NULL || dk_rows == NULL || dv_rows == NULL)) return -1;
+    if (ids != NULL && (table == NULL || x == NULL || Wg == NULL || C < 32 || vocab < 1)) return -1;
+    if (ids != NULL && n_k > 0 && dve_rows == NULL) return -1;
+    if (ids != NULL && !ids_in_range(ids, (int64_t)B * T, vocab)) return -1;
+    for (int64_t r = 0; r < n_q; ++r)
+        if (qrows[r] < 0 || qrows[r] >= (int64_t)B * H * T) return -1;
+    for (int64_t r = 0; r < n_k; ++r)
+        if (krows[r] < 0 || krows[r] >= (int64_t)B * Hkv * T) return -1;
+    const int G = H / Hkv;
+    const int W = (window <= 0 || window >= T) ? T : window;
+    const int reach = window_convention == 0 ? W - 1 : W;
+    const double inv_sqrt_d = 1.0 / sqrt((double)D);
+    const size_t TD = (size_t)T * D;
+
+    double* kh = (double*)malloc(sizeof(double) * TD);
+    double* vp = (double*)malloc(sizeof(double) * TD);
+    double* qh = (double*)malloc(sizeof(double) * TD);
+    double* dkh = (double*)malloc(sizeof(double) * TD);
+    double* dvp = (double*)malloc(sizeof(double) * TD);
+    double* dqh = (double*)malloc(sizeof(double) * TD);
+    double* lse = (double*)malloc(sizeof(double) * (size_t)T);
+    double* delta = (double*)malloc(sizeof(double) * (size_t)T);
+    char* need = (char*)malloc((size_t)T);       /* 1: lse/delta needed; 2: dqhat needed too */
+    char* kneed = (char*)malloc((size_t)T);      /* requested key rows of this (b, hk) */
+    int rc = 0;
+    if (!kh || !vp || !qh || !dkh || !dvp || !dqh || !lse || !delta || !need || !kneed) { rc = -1; goto done; }
+
+    for (int b = 0; b < B && rc == 0; ++b) {
+        for (int hk = 0; hk < Hkv && rc == 0; ++hk) {
+            int any = 0;
+            memset(kneed, 0, (size_t)T);
+            for (int64_t r = 0; r < n_k; ++r)
+                if (krows[r] / T == (int64_t)b * Hkv + hk) { kneed[krows[r] % T] = 1; any = 1; }
+            for (int64_t r = 0; r < n_q && !any; ++r) {
+                const int64_t bh = qrows[r] / T;
+                if (bh / H == b && (int)(bh % H) / G == hk) any = 1;
+            }
+            if (!any) continue;
+            #pragma omp parallel for schedule(static)
+            for (int t = 0; t < T; ++t) {
+                prologue_qk(k, T, Hkv, D, b, t, hk, rope_base, eps, use_rope, use_qknorm,
+                            round_bf16, kh + (size_t)t * D);
+                prologue_v(v, ids, table, x, C, Wg, T, Hkv, D, b, t, hk, round_bf16,
+                           vp + (size_t)t * D);
+            }
+            memset(dkh, 0, sizeof(double) * TD);
+            memset(dvp, 0, sizeof(double) * TD);
+            for (int g = 0; g < G; ++g) {
+                const int h = hk * G + g;
+                memset(need, 0, (size_t)T);
+                int any_h = 0;
+                for (int64_t r = 0; r < n_q; ++r)
+                    if (qrows[r] / T == (int64_t)b * H + h) { need[qrows[r] % T] = 2; any_h = 1; }
+                for (int j = 0; j < T; ++j) {
+                    if (!kneed[j]) continue;
+                    const int i_end = (j + reach < T - 1) ? j + reach : T - 1;
+                    for (int i = j; i <= i_end; ++i)
+                        if (need[i] == 0) need[i] = 1;
+                    any_h = 1;
+                }
+                if (!any_h) continue;
+                int bad = 0;
+                #pragma omp parallel
+                {
+                    double* s = (double*)malloc(sizeof(double) * (size_t)T);
+                    #pragma omp for schedule(dynamic, 8)
+                    for (int i = 0; i < T; ++i) {
+                        if (!need[i]) continue;
+                        if (s == NULL) {
+                            #pragma omp atomic write
+                            bad = 1;
+                            continue;
+                        }
+                        prologue_qk(q, T, H, D, b, i, h, rope_base, eps, use_rope, use_qknorm,
+                                    round_bf16, qh + (size_t)i * D);
+                        const double* gi = dout + (((size_t)b * T + i) * H + h) * (size_t)D;
+                        const double gl = dlse ? dlse[((size_t)b * H + h) * T + i] : 0.0;
+                        bwd_query_row(qh + (size_t)i * D, gi, gl, kh, vp, T, D, i, W, window_convention,
+                                      inv_sqrt_d, s, &lse[i], &delta[i],
+                                      need[i] == 2 ? dqh + (size_t)i * D : NULL);
+                    }
+                    free(s);
+                }
+                if (bad) { rc = -1; break; }
+                #pragma omp parallel for schedule(dynamic, 1)
+                for (int j = 0; j < T; ++j) {
+                    if (!kneed[j]) continue;
+                    const int i_end = (j + reach < T - 1) ? j + reach : T - 1;
+                    bwd_key_row(kh + (size_t)j * D, vp + (size_t)j * D, qh, lse, delta, dout, dlse, b, h,
+                                T, H, D, j, i_end, inv_sqrt_d, dkh + (size_t)j * D, dvp + (size_t)j * D);
+                }
+                double* xr = (double*)malloc(sizeof(double) * (size_t)D);
+                if (xr == NULL) { rc = -1; break; }
+                for (int64_t r = 0; r < n_q; ++r)
+                    if (qrows[r] / T == (int64_t)b * H + h) {
+                        const int i = (int)(qrows[r] % T);
+                        prologue_qk_backward(q, T, H, D, b, i, h, rope_base, eps, use_rope, use_qknorm,
+                                             dqh + (size_t)i * D, dq_rows + (size_t)r * D, xr);
+                    }
+                free(xr);
+            }
+            if (rc != 0) break;
+            double* xr = (double*)malloc(sizeof(double) * (size_t)D);
+            if (xr == NULL) { rc = -1; break; }
+            for (int64_t r = 0; r < n_k; ++r) {
+                if (krows[r] / T != (int64_t)b * Hkv + hk) continue;
+                const int j = (int)(krows[r] % T);
+                double dzj = 0.0;
+                bwd_kv_outputs(k, ids, table, x, C, Wg, T, Hkv, D, b, j, hk, rope_base, eps, use_rope,
+                               use_qknorm, dkh + (size_t)j * D, dvp + (size_t)j * D, dk_rows + (size_t)r * D,
+                               dv_rows + (size_t)r * D, ids ? dve_rows + (size_t)r * D : NULL, &dzj, xr);
+            }
+            free(xr);
+        }
+    }
+
+done:
+    free(kh); free(vp); free(qh); free(dkh); free(dvp); free(dqh); free(lse); free(delta);
+    free(need); free(kneed);
     return rc;
 }

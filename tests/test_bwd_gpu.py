@@ -102,3 +102,49 @@ def test_backward_without_dlse_and_single_row():
     assert np.abs(ref["dq"]).max() == 0.0 and np.abs(ref["dk"]).max() == 0.0
     assert np.abs(got["dq"]).max() < 1e-3 and np.abs(got["dk"]).max() < 1e-3
     _compare(got, ref, skip=("dq", "dk"))
+
+
+FULL = {"d24_L_VE": workloads.D24_L_VE, "d24_S": workloads.D24_S}
+
+
+@pytest.mark.parametrize("name", sorted(FULL))
+def test_backward_full_size_sampled_rows(name):
+    """The whole d24 backward (B=16, T=2048, H=12, D=128) on the GPU, checked against the oracle at
+    sampled rows: edge and random query rows (dq) and key rows (dk, dv, dve) of a few (b, head)
+    slices; the oracle computes each sampled value exactly as its full backward would."""
+    s = FULL[name]
+    d = workloads.make_layer(s)
+    gen = torch.Generator().manual_seed(60_000 + s.seed)
+    dout = torch.randn((s.B, s.T, s.H, s.D), generator=gen).to(torch.bfloat16)
+    dlse = torch.randn((s.B, s.H, s.T), generator=gen)
+    got = _run(s, d, dout, dlse)
+    W = s.eff_window()
+    g = torch.Generator().manual_seed(s.seed)
+    edges = sorted({0, 1, 127, 128, W - 1, W, s.T - 128, s.T - 1} & set(range(s.T)))
+    qrows, krows = [], []
+    for (b, h) in [(0, 0), (s.B - 1, s.H - 1), (5, 7)]:
+        for i in edges + torch.randint(0, s.T, (3,), generator=g).tolist():
+            qrows.append((b * s.H + h) * s.T + i)
+    for (b, hk) in [(0, 0), (s.B - 1, s.Hkv - 1)]:
+        for j in edges + torch.randint(0, s.T, (2,), generator=g).tolist():
+            krows.append((b * s.Hkv + hk) * s.T + j)
+    ref = oracle.backward_rows(d, dout, s.window, dlse=dlse, qrows=qrows, krows=krows, parity=True)
+
+    def pick(t, rows, heads):
+        out = []
+        for r in rows:
+            bh, i = divmod(r, s.T)
+            b, h = divmod(bh, heads)
+            out.append(t[b, i, h])
+        return np.stack(out).astype(np.float64)
+
+    pairs = [("dq", pick(got["dq"], qrows, s.H)), ("dk", pick(got["dk"], krows, s.Hkv)),
+             ("dv", pick(got["dv"], krows, s.Hkv))]
+    if s.ve:
+        pairs.append(("dve", pick(got["dve"], krows, s.Hkv)))
+    for key, a in pairs:
+        b = ref[key]
+        rel_l2 = float(np.linalg.norm(a - b) / np.linalg.norm(b))
+        max_rel = float(np.abs(a - b).max() / np.abs(b).max())
+        print(f"{name} {key}: rel_l2={rel_l2:.3e} max_rel={max_rel:.3e}")
+        assert rel_l2 <= REL_L2 and max_rel <= MAX_REL, (key, rel_l2, max_rel)

@@ -308,3 +308,39 @@ def test_backward_rejects_bad_arguments():
     three = dict(q=_draw(1, 4, 3, 8)["q"], k=d["k"], v=d["v"])   # Hkv = 2 does not divide H = 3
     with pytest.raises(ValueError):
         oracle.backward(three, np.zeros((1, 4, 3, 8)), 0)
+
+
+# --------------------------------------------------------------- sampled rows = full backward
+
+@pytest.mark.parametrize("B,T,H,Hkv,D,window,ve,parity", [
+    (2, 37, 4, 4, 16, 5, True, False),
+    (1, 60, 6, 2, 8, 0, True, True),
+    (2, 45, 3, 1, 16, 1, False, True),
+    (1, 130, 2, 2, 32, 40, True, True),
+])
+def test_sampled_rows_equal_the_full_backward_bit_for_bit(B, T, H, Hkv, D, window, ve, parity):
+    d = _draw(B, T, H, D, Hkv=Hkv, ve=ve, seed=T + H, unique_ids=False)
+    dout, dlse = _cotangents(B, T, H, D, seed=T)
+    full = oracle.backward(d, dout, window, dlse=dlse, parity=parity)
+    g = torch.Generator().manual_seed(T)
+    qrows = torch.randint(0, B * H * T, (9,), generator=g).tolist() + [0, B * H * T - 1]
+    krows = torch.randint(0, B * Hkv * T, (9,), generator=g).tolist() + [0, B * Hkv * T - 1, 3]
+    rows = oracle.backward_rows(d, dout, window, dlse=dlse, qrows=qrows, krows=krows, parity=parity)
+    for n, r in enumerate(qrows):
+        bh, i = divmod(r, T)
+        b, h = divmod(bh, H)
+        assert np.array_equal(rows["dq"][n], full["dq"][b, i, h]), ("dq", r)
+    for n, r in enumerate(krows):
+        bh, j = divmod(r, T)
+        b, hk = divmod(bh, Hkv)
+        for key in ("dk", "dv") + (("dve",) if ve else ()):
+            assert np.array_equal(rows[key][n], full[key][b, j, hk]), (key, r)
+
+
+def test_sampled_rows_reject_out_of_range_ids():
+    d = _draw(1, 8, 2, 8, seed=2)
+    dout, _ = _cotangents(1, 8, 2, 8, seed=2)
+    with pytest.raises(ValueError):
+        oracle.backward_rows(d, dout, 0, qrows=[16])
+    with pytest.raises(ValueError):
+        oracle.backward_rows(d, dout, 0, krows=[-1])
