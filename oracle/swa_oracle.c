@@ -367,6 +367,26 @@ static double dot_d(const double* a, const double* b, int D) {
     return acc;
 }
 
+/* Keys j visible to query i are those with i in [j, j + reach]. */
+static int key_reach(int W, int window_convention) {
+    return window_convention == 0 ? W - 1 : W;
+}
+
+/* khat and v' of every position of key/value head hk of batch row b, as the forward computes
+ * them (rounded to bf16 in parity mode). */
+static void bwd_kv_prologue(const uint16_t* k, const uint16_t* v, const int64_t* ids,
+                            const uint16_t* table, const uint16_t* x, int C, const uint16_t* Wg,
+                            int T, int Hkv, int D, int b, int hk, double rope_base, double eps,
+                            int round_bf16, int use_rope, int use_qknorm, double* kh, double* vp) {
+    #pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        prologue_qk(k, T, Hkv, D, b, t, hk, rope_base, eps, use_rope, use_qknorm,
+                    round_bf16, kh + (size_t)t * D);
+        prologue_v(v, ids, table, x, C, Wg, T, Hkv, D, b, t, hk, round_bf16,
+                   vp + (size_t)t * D);
+    }
+}
+
 /* Row pass for query row i of one (b, h): scores against the visible keys (scratch s of T),
  * lse_i, delta_i = sum_j P_ij dP_ij and, if dqi is not NULL, dqhat_i = sum_j dS_ij khat_j / sqrt(D).
  * gi is dout of the row, gl its dlse. */
@@ -474,8 +494,7 @@ int swa_oracle_backward_gqa(const uint16_t* q, const uint16_t* k, const uint16_t
     if (ids != NULL && !ids_in_range(ids, (int64_t)B * T, vocab)) return -1;
     const int G = H / Hkv;
     const int W = (window <= 0 || window >= T) ? T : window;
-    /* Keys j visible to query i are those with i in [j, j + reach]. */
-    const int reach = window_convention == 0 ? W - 1 : W;
+    const int reach = key_reach(W, window_convention);
     const double inv_sqrt_d = 1.0 / sqrt((double)D);
     const size_t TD = (size_t)T * D;
 
@@ -493,13 +512,8 @@ int swa_oracle_backward_gqa(const uint16_t* q, const uint16_t* k, const uint16_t
 
     for (int b = 0; b < B && rc == 0; ++b) {
         for (int hk = 0; hk < Hkv && rc == 0; ++hk) {
-            #pragma omp parallel for schedule(static)
-            for (int t = 0; t < T; ++t) {
-                prologue_qk(k, T, Hkv, D, b, t, hk, rope_base, eps, use_rope, use_qknorm,
-                            round_bf16, kh + (size_t)t * D);
-                prologue_v(v, ids, table, x, C, Wg, T, Hkv, D, b, t, hk, round_bf16,
-                           vp + (size_t)t * D);
-            }
+            bwd_kv_prologue(k, v, ids, table, x, C, Wg, T, Hkv, D, b, hk, rope_base, eps, round_bf16,
+                            use_rope, use_qknorm, kh, vp);
             memset(dkh, 0, sizeof(double) * TD);
             memset(dvp, 0, sizeof(double) * TD);
 
@@ -643,7 +657,7 @@ int swa_oracle_backward_rows_gqa(const uint16_t* q, const uint16_t* k, const uin
         if (krows[r] < 0 || krows[r] >= (int64_t)B * Hkv * T) return -1;
     const int G = H / Hkv;
     const int W = (window <= 0 || window >= T) ? T : window;
-    const int reach = window_convention == 0 ? W - 1 : W;
+    const int reach = key_reach(W, window_convention);
     const double inv_sqrt_d = 1.0 / sqrt((double)D);
     const size_t TD = (size_t)T * D;
 
@@ -671,13 +685,8 @@ int swa_oracle_backward_rows_gqa(const uint16_t* q, const uint16_t* k, const uin
                 if (bh / H == b && (int)(bh % H) / G == hk) any = 1;
             }
             if (!any) continue;
-            #pragma omp parallel for schedule(static)
-            for (int t = 0; t < T; ++t) {
-                prologue_qk(k, T, Hkv, D, b, t, hk, rope_base, eps, use_rope, use_qknorm,
-                            round_bf16, kh + (size_t)t * D);
-                prologue_v(v, ids, table, x, C, Wg, T, Hkv, D, b, t, hk, round_bf16,
-                           vp + (size_t)t * D);
-            }
+            bwd_kv_prologue(k, v, ids, table, x, C, Wg, T, Hkv, D, b, hk, rope_base, eps, round_bf16,
+                            use_rope, use_qknorm, kh, vp);
             memset(dkh, 0, sizeof(double) * TD);
             memset(dvp, 0, sizeof(double) * TD);
             for (int g = 0; g < G; ++g) {

@@ -65,14 +65,14 @@ BACKWARD_MUTANTS = {
         "    for (int i = half; i < D; ++i) g[i] = -g[i];\n",
         "    rope_inplace(g, D, t, base);\n"),
     "bwd gate derivative without 1 - sigma": ("dgate * 2.0 * sig * (1.0 - sig)", "dgate * 2.0 * sig"),
-    "bwd ve gradient without gate": ("dve[off + d] = 2.0 * sig * dvt[d];", "dve[off + d] = dvt[d];"),
+    "bwd ve gradient without gate": ("dve_out[d] = 2.0 * sig * dvt[d];", "dve_out[d] = dvt[d];"),
     "bwd dx reads Wg transposed": (
         "acc += dz[(size_t)bt * Hkv + hk] * bf16_to_double(Wg[(size_t)c * Hkv + hk]);",
         "acc += dz[(size_t)bt * Hkv + hk] * bf16_to_double(Wg[(size_t)hk * 32 + c]);"),
     "bwd dWg reads x with stride 32": ("bf16_to_double(x[(size_t)bt * C + c])",
                                        "bf16_to_double(x[(size_t)bt * 32 + c])"),
-    "bwd key pass window off by one": ("const int reach = window_convention == 0 ? W - 1 : W;",
-                                       "const int reach = window_convention == 0 ? W : W;"),
+    "bwd key pass window off by one": ("return window_convention == 0 ? W - 1 : W;",
+                                       "return window_convention == 0 ? W : W;"),
     "bwd gqa group sum dropped": (
         "            memset(dkh, 0, sizeof(double) * TD);\n            memset(dvp, 0, sizeof(double) * TD);\n\n"
         "            for (int g = 0; g < G; ++g) {\n",
@@ -81,9 +81,9 @@ BACKWARD_MUTANTS = {
     "bwd dk without scale": ("dkj[d] += ds * qi[d] * inv_sqrt_d;", "dkj[d] += ds * qi[d];"),
     "bwd dv weighted by dS": ("dvj[d] += p * gi[d];", "dvj[d] += ds * gi[d];"),
     "bwd dq from queries": ("dqi[d] += ds * kh[(size_t)j * D + d] * inv_sqrt_d;",
-                            "dqi[d] += ds * qh[(size_t)j * D + d] * inv_sqrt_d;"),
-    "bwd keys not rounded in parity mode": ("                            round_bf16, kh + (size_t)t * D);",
-                                            "                            0, kh + (size_t)t * D);"),
+                            "dqi[d] += ds * qi[d] * inv_sqrt_d;"),
+    "bwd keys not rounded in parity mode": ("                    round_bf16, kh + (size_t)t * D);",
+                                            "                    0, kh + (size_t)t * D);"),
 }
 
 BACKWARD_PIN_FUNCS = [
