@@ -8,6 +8,8 @@ imports it.
 Two independent implementations live here:
 
 * ``forward`` / ``prologue``: the C oracle (``swa_oracle.c``), one query row at a time, fp64.
+* ``qkv_prologue``: the bias-free q, k, v projection of the layer input x followed by the same
+  prologue (the fused projection).
 * ``backward``: the gradient of the same layer (chain rule through the five steps in
   reverse), also in ``swa_oracle.c``; ``backward_rows`` gives the same values at sampled rows.
 * ``brute.py``: a NumPy fp64 restatement that materialises the full T x T score matrix, used
@@ -67,6 +69,12 @@ def _configure(lib):
                                                  ctypes.c_double, ctypes.c_int, ctypes.c_int,
                                                  ctypes.c_int, ctypes.c_int, P, P,
                                                  P, ctypes.c_int64, P, P, ctypes.c_int64, P, P, P]
+    lib.swa_oracle_qkv_prologue_gqa.restype = ctypes.c_int
+    lib.swa_oracle_qkv_prologue_gqa.argtypes = [P, ctypes.c_int, P, P, P, ctypes.c_int, P,
+                                                ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                                ctypes.c_double, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int, P, P, P]
     lib.swa_oracle_threads.restype = ctypes.c_int
     lib.swa_oracle_round_bf16.restype = ctypes.c_double
     lib.swa_oracle_round_bf16.argtypes = [ctypes.c_double]
@@ -279,3 +287,35 @@ def _as_f64(a) -> np.ndarray:
     if isinstance(a, np.ndarray):
         return a.astype(np.float64, copy=False)
     return a.detach().cpu().double().numpy()
+
+
+def qkv_prologue(x, Wqkv, H: int, Hkv: int, D: int, ids=None, table=None, Wg=None,
+                 rope_base: float = 10000.0, eps: float = 1e-6, *, parity: bool = False,
+                 rope: bool = True, qknorm: bool = True):
+    """q, k, v = x Wqkv^T (x (B,T,C) bf16, Wqkv [(H + 2 Hkv) D, C] bf16, the linear layer's layout;
+    rows: q heads, k heads, v heads), then RoPE / RMS on q and k and the gated value embedding on
+    v (ids (B,T), table [vocab, Hkv D], Wg [32, Hkv]; the gate reads x[..., :32]).
+    Returns qhat (B,T,H,D), khat and v' (B,T,Hkv,D) as fp64 (rounded to bf16 values if parity)."""
+    lib = _load()
+    xb, wb = _bits(x), _bits(Wqkv)
+    B, T, C = xb.shape
+    if wb.shape != ((H + 2 * Hkv) * D, C):
+        raise ValueError("Wqkv must be [(H + 2 Hkv) D, C]")
+    import torch
+    if ids is not None:
+        ids_a = ids.cpu().contiguous().numpy().astype(np.int64) if isinstance(ids, torch.Tensor) \
+            else np.ascontiguousarray(ids, dtype=np.int64)
+        tb, gw = _bits(table), _bits(Wg)
+        vocab = int(tb.shape[0])
+    else:
+        ids_a = tb = gw = None
+        vocab = 0
+    qh = np.empty((B, T, H, D))
+    kh = np.empty((B, T, Hkv, D))
+    vp = np.empty((B, T, Hkv, D))
+    rc = lib.swa_oracle_qkv_prologue_gqa(_ptr(xb), C, _ptr(wb), _ptr(ids_a), _ptr(tb), vocab, _ptr(gw),
+                                         B, T, H, Hkv, D, float(rope_base), float(eps), int(parity),
+                                         int(rope), int(qknorm), _ptr(qh), _ptr(kh), _ptr(vp))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return qh, kh, vp

@@ -763,3 +763,80 @@ done:
     free(need); free(kneed);
     return rc;
 }
+
+/* -----------------------------------------------------------------------------------------
+ * The projection before the path, fused with the prologue: q, k, v = x Wqkv^T, then RoPE, RMS and
+ * the value-embedding gate as above.
+ *
+ * The pages build q, k, v of each layer with bias-free linear maps of the layer input x ("Let's
+ * reproduce GPT-2 (124M)" notes, section 3, the attention listing: one projection to 3C split
+ * into q, k, v; the speedrun explainer and intelliparadigm "GPT-2 for $73", section 2: separate
+ * bias-free q, k, v maps, key/value width kv_dim).  Reading: one weight in the linear layer's
+ * layout, Wqkv [(H + 2 Hkv) D, C] (rows 0 .. H D - 1 give q, then Hkv D rows of k, then Hkv D of
+ * v), y[n] = sum_c x[c] Wqkv[n, c] summed in fp64 over c in order; the gate reads the first 32
+ * channels of the same x.  Outputs as swa_oracle_prologue_gqa: qhat (B,T,H,D), khat and v'
+ * (B,T,Hkv,D) in fp64, rounded to bf16 in parity mode.
+ * ----------------------------------------------------------------------------------------- */
+
+/* x[b,t,:] . Wqkv[n,:] in fp64, c in order. */
+static double proj_dot(const uint16_t* xr, const uint16_t* Wqkv, int C, int n) {
+    const uint16_t* w = Wqkv + (size_t)n * C;
+    double acc = 0.0;
+    for (int c = 0; c < C; ++c) acc += bf16_to_double(xr[c]) * bf16_to_double(w[c]);
+    return acc;
+}
+
+int swa_oracle_qkv_prologue_gqa(const uint16_t* x, int C, const uint16_t* Wqkv,
+                                const int64_t* ids, const uint16_t* table, int vocab,
+                                const uint16_t* Wg, int B, int T, int H, int Hkv, int D,
+                                double rope_base, double eps, int round_bf16, int use_rope,
+                                int use_qknorm, double* qh, double* kh, double* vp) {
+    if (B < 1 || T < 1 || H < 1 || D < 2 || (D % 2) != 0 || C < 1 || x == NULL || Wqkv == NULL) return -1;
+    if (Hkv < 1 || Hkv > H || (H % Hkv) != 0) return -1;
+    if (ids != NULL && (table == NULL || Wg == NULL || C < 32 || vocab < 1)) return -1;
+    if (ids != NULL && !ids_in_range(ids, (int64_t)B * T, vocab)) return -1;
+    int bad = 0;
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t) {
+            const uint16_t* xr = x + ((size_t)b * T + t) * (size_t)C;
+            double* row = (double*)malloc(sizeof(double) * (size_t)D);
+            if (row == NULL) {
+                #pragma omp atomic write
+                bad = 1;
+                continue;
+            }
+            /* q heads, then k heads: projection, RoPE, RMS */
+            for (int part = 0; part < 2; ++part) {
+                const int heads = part == 0 ? H : Hkv;
+                const int n0 = part == 0 ? 0 : H * D;
+                double* dst = part == 0 ? qh : kh;
+                for (int h = 0; h < heads; ++h) {
+                    for (int d = 0; d < D; ++d) row[d] = proj_dot(xr, Wqkv, C, n0 + h * D + d);
+                    if (use_rope) rope_inplace(row, D, t, rope_base);
+                    if (use_qknorm) rmsnorm_inplace(row, D, eps);
+                    double* o = dst + (((size_t)b * T + t) * heads + h) * (size_t)D;
+                    for (int d = 0; d < D; ++d) o[d] = round_bf16 ? round_to_bf16(row[d]) : row[d];
+                }
+            }
+            /* v heads: projection plus the gated value embedding */
+            for (int h = 0; h < Hkv; ++h) {
+                double gate = 0.0;
+                const uint16_t* ve = NULL;
+                if (ids != NULL) {
+                    double z = 0.0;
+                    for (int c = 0; c < 32; ++c) z += bf16_to_double(xr[c]) * bf16_to_double(Wg[c * Hkv + h]);
+                    gate = 2.0 / (1.0 + exp(-z));
+                    ve = table + (size_t)ids[(size_t)b * T + t] * (size_t)Hkv * D + (size_t)h * D;
+                }
+                double* o = vp + (((size_t)b * T + t) * Hkv + h) * (size_t)D;
+                for (int d = 0; d < D; ++d) {
+                    double val = proj_dot(xr, Wqkv, C, (H + Hkv) * D + h * D + d);
+                    if (ve != NULL) val += gate * bf16_to_double(ve[d]);
+                    o[d] = round_bf16 ? round_to_bf16(val) : val;
+                }
+            }
+            free(row);
+        }
+    return bad ? -1 : 0;
+}

@@ -13,6 +13,7 @@ import oracle
 from oracle import build as obuild
 import tests.test_oracle_backward_pins as bpins
 import tests.test_oracle_pins as pins
+import tests.test_oracle_qkv_pins as qpins
 
 MUTANTS = {
     "rope sign": ("x[i] = a * c - b * s;", "x[i] = a * c + b * s;"),
@@ -98,6 +99,24 @@ BACKWARD_PIN_FUNCS = [
 ]
 
 
+# Mistakes in the fused projection + prologue (every planted index stays inside its array).
+QKV_MUTANTS = {
+    "proj weight row stride": ("const uint16_t* w = Wqkv + (size_t)n * C;", "const uint16_t* w = Wqkv + (size_t)n * (C - 1);"),
+    "proj k rows start at Hkv D": ("const int n0 = part == 0 ? 0 : H * D;", "const int n0 = part == 0 ? 0 : Hkv * D;"),
+    "proj v reads the k rows": ("proj_dot(xr, Wqkv, C, (H + Hkv) * D + h * D + d)", "proj_dot(xr, Wqkv, C, H * D + h * D + d)"),
+    "proj gate column reversed": ("bf16_to_double(Wg[c * Hkv + h]);\n                    gate = 2.0",
+                                  "bf16_to_double(Wg[c * Hkv + (Hkv - 1 - h)]);\n                    gate = 2.0"),
+    "proj rope position from b": ("if (use_rope) rope_inplace(row, D, t, rope_base);", "if (use_rope) rope_inplace(row, D, b, rope_base);"),
+}
+
+QKV_PIN_FUNCS = [
+    lambda: qpins.test_permutation_weights_reduce_to_the_prologue_bit_for_bit(2, 2, 16, True, False),
+    lambda: qpins.test_permutation_weights_reduce_to_the_prologue_bit_for_bit(4, 2, 8, True, True),
+    qpins.test_projection_alone_equals_numpy_matmul,
+    qpins.test_doubling_the_weights_leaves_the_normalised_rows_unchanged,
+]
+
+
 def _failing_pins(funcs=None):
     failed = 0
     for f in (PIN_FUNCS if funcs is None else funcs):
@@ -128,6 +147,21 @@ def test_planted_backward_mistake_is_caught(name):
             assert _failing_pins(BACKWARD_PIN_FUNCS) >= 1, f"no pin caught the planted mistake: {name}"
         finally:
             oracle._swap_library(None)
+
+
+@pytest.mark.parametrize("name", sorted(QKV_MUTANTS))
+def test_planted_projection_mistake_is_caught(name):
+    old, new = QKV_MUTANTS[name]
+    with tempfile.TemporaryDirectory() as tmp:
+        oracle._swap_library(_build_mutant(old, new, tmp))
+        try:
+            assert _failing_pins(QKV_PIN_FUNCS) >= 1, f"no pin caught the planted mistake: {name}"
+        finally:
+            oracle._swap_library(None)
+
+
+def test_unmutated_projection_passes_every_projection_pin():
+    assert _failing_pins(QKV_PIN_FUNCS) == 0
 
 
 def test_unmutated_backward_passes_every_backward_pin():
