@@ -78,6 +78,12 @@ def _load() -> ctypes.CDLL:
     lib.swa_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
                                  I, I, I, I, I, F, F, P, Z, P]
     lib.swa_attn_bwd.restype = I
+    lib.swa_attn_fwd_x_workspace_bytes.argtypes = [I, I, I, I, I]
+    lib.swa_attn_fwd_x_workspace_bytes.restype = Z
+    lib.swa_attn_qkv_prologue.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, F, P, Z, P]
+    lib.swa_attn_qkv_prologue.restype = I
+    lib.swa_attn_fwd_x.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, F, P, Z, P]
+    lib.swa_attn_fwd_x.restype = I
     lib.swa_attn_selftest_wait.argtypes = [I, P]
     lib.swa_attn_selftest_wait.restype = I
     lib.swa_attn_set_wait_limit_ms.argtypes = [I]
@@ -193,6 +199,22 @@ def swa_attn_bwd(q, k, v, ve, gate_x, Wg, out, lse, dout, dlse, dq, dk, dv, dve,
                  B, T, H, D, window, rope_base, eps, workspace, ws_bytes, stream) -> int:
     return _lib.swa_attn_bwd(q, k, v, ve, gate_x, Wg, out, lse, dout, dlse, dq, dk, dv, dve, dgate_x, dWg,
                              B, T, H, D, window, rope_base, eps, workspace, ws_bytes, stream)
+
+
+def swa_attn_fwd_x_workspace_bytes(B, T, H, Hkv, D) -> int:
+    return int(_lib.swa_attn_fwd_x_workspace_bytes(B, T, H, Hkv, D))
+
+
+def swa_attn_qkv_prologue(x, Wqkv, ve, Wg, qh, kh, vp, B, T, C, H, Hkv, D, rope_base, eps, workspace,
+                          ws_bytes, stream) -> int:
+    return _lib.swa_attn_qkv_prologue(x, Wqkv, ve, Wg, qh, kh, vp, B, T, C, H, Hkv, D, rope_base, eps,
+                                      workspace, ws_bytes, stream)
+
+
+def swa_attn_fwd_x(x, Wqkv, ve, Wg, out, lse, B, T, C, H, Hkv, D, window, rope_base, eps, workspace,
+                   ws_bytes, stream) -> int:
+    return _lib.swa_attn_fwd_x(x, Wqkv, ve, Wg, out, lse, B, T, C, H, Hkv, D, window, rope_base, eps,
+                               workspace, ws_bytes, stream)
 
 
 def swa_attn_selftest_wait(limit_ms: int, stream=None) -> int:
@@ -351,6 +373,61 @@ def backward(q, k, v, out, lse, dout, window: int = 0, dlse=None, ve=None, gate_
     return g
 
 
+def _check_x_w(x, Wqkv, H, Hkv, D, ve, Wg):
+    import torch
+    if x.dim() != 3 or x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA bf16 (B, T, C) tensor")
+    B, T, C = x.shape
+    N = (H + 2 * Hkv) * D
+    if tuple(Wqkv.shape) != (N, C) or Wqkv.dtype != torch.bfloat16 or not Wqkv.is_contiguous():
+        raise ValueError(f"Wqkv must be a contiguous bf16 [{N}, {C}] tensor")
+    if (ve is None) != (Wg is None):
+        raise ValueError("ve and Wg go together")
+    if ve is not None:
+        if tuple(ve.shape) != (B, T, Hkv, D) or ve.dtype != torch.bfloat16 or not ve.is_contiguous():
+            raise ValueError(f"ve must be a contiguous bf16 {(B, T, Hkv, D)} tensor")
+        if tuple(Wg.shape) != (32, Hkv) or Wg.dtype != torch.bfloat16 or not Wg.is_contiguous():
+            raise ValueError(f"Wg must be a contiguous bf16 [32, {Hkv}] tensor")
+    return B, T, C
+
+
+def qkv_prologue(x, Wqkv, H: int, Hkv: int, D: int, ve=None, Wg=None, rope_base: float = 10000.0,
+                 eps: float = 1e-6, *, stream=None):
+    """q, k, v = x Wqkv^T fused with RoPE / RMS / the gated value embedding (C call
+    swa_attn_qkv_prologue).  Returns (qhat (B,T,H,D), khat (B,T,Hkv,D), v' (B,T,Hkv,D)), bf16."""
+    import torch
+    B, T, C = _check_x_w(x, Wqkv, H, Hkv, D, ve, Wg)
+    qh = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=x.device)
+    kh = torch.empty((B, T, Hkv, D), dtype=torch.bfloat16, device=x.device)
+    vp = torch.empty((B, T, Hkv, D), dtype=torch.bfloat16, device=x.device)
+    need = swa_attn_fwd_x_workspace_bytes(B, T, H, Hkv, D)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    rc = swa_attn_qkv_prologue(_ptr(x), _ptr(Wqkv), _ptr(ve), _ptr(Wg), _ptr(qh), _ptr(kh), _ptr(vp), B, T, C, H,
+                               Hkv, D, float(rope_base), float(eps), _ptr(ws), need, _stream_handle(stream))
+    if rc != SWA_OK:
+        raise SwaError(rc, "swa_attn_qkv_prologue")
+    return qh, kh, vp
+
+
+def forward_x(x, Wqkv, H: int, Hkv: int, D: int, window: int = 0, ve=None, Wg=None,
+              rope_base: float = 10000.0, eps: float = 1e-6, *, workspace=None, stream=None):
+    """The layer from its input x (C call swa_attn_fwd_x): fused projection + prologue, then the
+    windowed attention.  Returns (out bf16 (B,T,H,D), lse fp32 (B,H,T))."""
+    import torch
+    B, T, C = _check_x_w(x, Wqkv, H, Hkv, D, ve, Wg)
+    out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=x.device)
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=x.device)
+    need = swa_attn_fwd_x_workspace_bytes(B, T, H, Hkv, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    rc = swa_attn_fwd_x(_ptr(x), _ptr(Wqkv), _ptr(ve), _ptr(Wg), _ptr(out), _ptr(lse), B, T, C, H, Hkv, D,
+                        int(window), float(rope_base), float(eps), _ptr(workspace),
+                        workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    if rc != SWA_OK:
+        raise SwaError(rc, "swa_attn_fwd_x")
+    return out, lse
+
+
 def check_device_status(stream=None) -> None:
     """Synchronise and raise SwaError if a kernel recorded an error (e.g. a wait timeout)."""
     rc, detail = swa_attn_last_device_status(_stream_handle(stream))
@@ -359,10 +436,11 @@ def check_device_status(stream=None) -> None:
 
 
 __all__ = [
-    "forward", "decode", "backward", "check_device_status", "SwaError", "LIB_PATH", "load",
+    "forward", "decode", "backward", "qkv_prologue", "forward_x", "check_device_status", "SwaError", "LIB_PATH", "load",
     "swa_attn_fwd", "swa_attn_fwd_ws", "swa_attn_fwd_noalloc", "swa_attn_noalloc_scratch_bytes", "swa_attn_workspace_bytes", "swa_attn_workspace_offset", "swa_attn_rope_table", "swa_attn_prologue",
     "swa_attn_attention", "swa_attn_strerror", "swa_attn_last_device_status",
     "swa_attn_set_wait_limit_ms", "swa_attn_selftest_wait", "swa_attn_version",
     "swa_attn_decode", "swa_attn_decode_workspace_bytes", "swa_attn_fwd_gqa",
     "swa_attn_bwd", "swa_attn_bwd_gqa", "swa_attn_bwd_workspace_bytes",
+    "swa_attn_fwd_x", "swa_attn_qkv_prologue", "swa_attn_fwd_x_workspace_bytes",
 ]

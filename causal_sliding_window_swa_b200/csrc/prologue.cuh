@@ -45,13 +45,14 @@ __device__ __forceinline__ int fdiv(int n, const FastDiv& f) {
 }
 
 // Gate of every (b, t, h) row: g = 2 sigmoid(sum_{c<32} x[b,t,c] Wg[c,h]) in fp64, stored as
-// (g_hi, g_lo) = (fp32(g), fp32(g - g_hi)).
+// (g_hi, g_lo) = (fp32(g), fp32(g - g_hi)).  Token bt's 32 gate channels start at
+// gate_x + bt * x_stride (32 for the contiguous slice, C for the full layer input).
 __global__ void gate_kernel(const __nv_bfloat16* __restrict__ gate_x, const __nv_bfloat16* __restrict__ Wg,
-                            float2* __restrict__ gate, int n_rows, int H, FastDiv divH) {
+                            float2* __restrict__ gate, int n_rows, int H, FastDiv divH, int x_stride) {
     for (int row = blockIdx.x * blockDim.x + threadIdx.x; row < n_rows; row += gridDim.x * blockDim.x) {
         const int bt = fdiv(row, divH);
         const int h = row - bt * H;
-        const __nv_bfloat16* xr = gate_x + (long long)bt * 32;
+        const __nv_bfloat16* xr = gate_x + (long long)bt * x_stride;
         double z = 0.0;
 #pragma unroll 8
         for (int c = 0; c < 32; ++c)

@@ -17,6 +17,7 @@
 #include "attn_fwd.cuh"
 #include "decode.cuh"
 #include "prologue.cuh"
+#include "qkv_gemm.cuh"
 
 // ------------------------------------------------------------------ failure-detection self-test
 
@@ -135,6 +136,19 @@ WsLayout ws_layout(const Shape& s, bool has_ve) {
 
 int g_num_sms[64] = {0};
 
+// Dynamic shared memory of every instantiation of the fused projection kernel.
+bool set_qkv_smem() {
+    const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
+    return cudaFuncSetAttribute(swa::qkv_gemm_kernel<128, 256, true>, a, swa::QkvCfg<256>::SMEM_TOTAL) == cudaSuccess &&
+           cudaFuncSetAttribute(swa::qkv_gemm_kernel<128, 256, false>, a, swa::QkvCfg<256>::SMEM_TOTAL) == cudaSuccess &&
+           cudaFuncSetAttribute(swa::qkv_gemm_kernel<128, 128, true>, a, swa::QkvCfg<128>::SMEM_TOTAL) == cudaSuccess &&
+           cudaFuncSetAttribute(swa::qkv_gemm_kernel<128, 128, false>, a, swa::QkvCfg<128>::SMEM_TOTAL) == cudaSuccess &&
+           cudaFuncSetAttribute(swa::qkv_gemm_kernel<64, 256, true>, a, swa::QkvCfg<256>::SMEM_TOTAL) == cudaSuccess &&
+           cudaFuncSetAttribute(swa::qkv_gemm_kernel<64, 256, false>, a, swa::QkvCfg<256>::SMEM_TOTAL) == cudaSuccess &&
+           cudaFuncSetAttribute(swa::qkv_gemm_kernel<64, 128, true>, a, swa::QkvCfg<128>::SMEM_TOTAL) == cudaSuccess &&
+           cudaFuncSetAttribute(swa::qkv_gemm_kernel<64, 128, false>, a, swa::QkvCfg<128>::SMEM_TOTAL) == cudaSuccess;
+}
+
 int device_ready(int* dev_out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -169,7 +183,8 @@ int device_ready(int* dev_out) {
                 cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<64>, (cudaFuncAttribute)smem_attr,
                                      swa::BwdCfg<64>::KV_SMEM) != cudaSuccess ||
                 cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<128>, (cudaFuncAttribute)smem_attr,
-                                     swa::BwdCfg<128>::KV_SMEM) != cudaSuccess) {
+                                     swa::BwdCfg<128>::KV_SMEM) != cudaSuccess ||
+                !set_qkv_smem()) {
                 cudaGetLastError();
                 checked[dev] = 0;
                 return SWA_ERR_CUDA;
@@ -253,7 +268,7 @@ int launch_prologue(const void* q, const void* k, const void* v, const void* ve,
     if (has_ve) {
         const int gblocks = (int)std::min<long long>(((long long)n_kv_rows + 255) / 256, 148ll * 8);
         swa::gate_kernel<<<gblocks, 256, 0, st>>>(static_cast<const bf*>(gate_x), static_cast<const bf*>(Wg),
-                                                   gate, n_kv_rows, s.Hkv, make_fastdiv(s.Hkv));
+                                                   gate, n_kv_rows, s.Hkv, make_fastdiv(s.Hkv), 32);
     }
     const long long threads_total = (long long)n_rows * (s.D / 8);
     const int threads = 256;
@@ -344,6 +359,87 @@ int launch_attention(int dev, const void* v, bool has_ve, void* out, float* lse,
         swa::attn_fwd_kernel<128><<<grid, swa::FwdCfg<128>::THREADS, swa::FwdCfg<128>::SMEM_TOTAL, st>>>(tq, tk, tv, to, p);
     else
         swa::attn_fwd_kernel<64><<<grid, swa::FwdCfg<64>::THREADS, swa::FwdCfg<64>::SMEM_TOTAL, st>>>(tq, tk, tv, to, p);
+    return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+// --------------------------------------------------------------- fused q/k/v projection
+
+// A (rows, cols) row-major bf16 matrix as a 2-D tensor map {cols, rows}; box = 64 columns (one
+// 128-byte swizzle atom) x box_rows rows.  Rows and columns past the end read as zeros.
+bool make_matrix_map(CUtensorMap* m, const void* base, long long rows, int cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int check_qkv_args(const void* x, const void* Wqkv, const void* ve, const void* Wg, int C, float rope_base,
+                   float eps) {
+    if (!x || !Wqkv) return SWA_ERR_INVALID_ARG;
+    if ((ve == nullptr) != (Wg == nullptr)) return SWA_ERR_INVALID_ARG;
+    if (C < 8 || (C % 8) != 0) return SWA_ERR_UNSUPPORTED;   // 16-byte rows for the tensor maps
+    if (ve != nullptr && C < 32) return SWA_ERR_INVALID_ARG;  // the gate reads 32 channels
+    if (!std::isfinite(rope_base) || !(rope_base > 0.f)) return SWA_ERR_INVALID_ARG;
+    if (!std::isfinite(eps) || eps < 0.f) return SWA_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(Wqkv, 16) || (ve && (!aligned(ve, 16) || !aligned(Wg, 2))))
+        return SWA_ERR_MISALIGNED;
+    return SWA_OK;
+}
+
+// Gate (value-embedding layers), then the fused projection kernel writing qhat, khat, v' to
+// qh / kh / vp.  The RoPE table must already be in the workspace.
+int launch_qkv(int dev, const void* x, const void* Wqkv, const void* ve, const void* Wg, int C, const Shape& s,
+               float eps, uint8_t* ws, const WsLayout& L, void* qh, void* kh, void* vp, int* sched_zero,
+               cudaStream_t st) {
+    using bf = __nv_bfloat16;
+    const bool has_ve = ve != nullptr;
+    const long long M = (long long)s.B * s.T;
+    if (M * C >= (1ll << 31) || M >= (1ll << 31) / std::max(1, s.H * s.D)) return SWA_ERR_UNSUPPORTED;
+    float2* gate = reinterpret_cast<float2*>(ws + L.gate);
+    if (has_ve) {
+        const int n_kv_rows = (int)(M * s.Hkv);
+        const int gblocks = (int)std::min<long long>(((long long)n_kv_rows + 255) / 256, 148ll * 8);
+        swa::gate_kernel<<<gblocks, 256, 0, st>>>(static_cast<const bf*>(x), static_cast<const bf*>(Wg), gate,
+                                                   n_kv_rows, s.Hkv, make_fastdiv(s.Hkv), C);
+    }
+    const int N = (s.H + 2 * s.Hkv) * s.D;
+    const int BN = ((s.H * s.D) % 256 == 0 && (s.Hkv * s.D) % 256 == 0) ? 256 : 128;
+    CUtensorMap tx, tw;
+    if (!make_matrix_map(&tx, x, M, C, 128) || !make_matrix_map(&tw, Wqkv, N, C, BN)) return SWA_ERR_CUDA;
+    swa::QkvParams p{};
+    p.M = (int)M;
+    p.T = s.T;
+    p.C = C;
+    p.H = s.H;
+    p.Hkv = s.Hkv;
+    p.N = N;
+    p.n_ntiles = (N + BN - 1) / BN;
+    p.n_tiles = (int)((M + 127) / 128) * p.n_ntiles;
+    p.eps = eps;
+    p.tab32 = reinterpret_cast<const float4*>(ws + L.tab32);
+    p.gate = has_ve ? gate : nullptr;
+    p.ve = static_cast<const bf*>(ve);
+    p.qh = static_cast<bf*>(qh);
+    p.kh = static_cast<bf*>(kh);
+    p.vp = static_cast<bf*>(vp);
+    p.sched_zero = sched_zero;
+    p.wait_limit_ns = wait_limit_ns();
+    const dim3 grid((unsigned)std::min(p.n_tiles, g_num_sms[dev]));
+#define SWA_QKV(DD, BB, VE) \
+    swa::qkv_gemm_kernel<DD, BB, VE><<<grid, swa::QkvCfg<BB>::THREADS, swa::QkvCfg<BB>::SMEM_TOTAL, st>>>(tx, tw, p)
+    if (s.D == 128) {
+        if (BN == 256) { if (has_ve) SWA_QKV(128, 256, true); else SWA_QKV(128, 256, false); }
+        else { if (has_ve) SWA_QKV(128, 128, true); else SWA_QKV(128, 128, false); }
+    } else {
+        if (BN == 256) { if (has_ve) SWA_QKV(64, 256, true); else SWA_QKV(64, 256, false); }
+        else { if (has_ve) SWA_QKV(64, 128, true); else SWA_QKV(64, 128, false); }
+    }
+#undef SWA_QKV
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
@@ -662,6 +758,58 @@ int swa_attn_fwd(const void* q, const void* k, const void* v, const void* ve, co
                  float rope_base, float eps, swa_stream_t stream) {
     return swa_attn_fwd_gqa(q, k, v, ve, gate_x, Wg, out, lse, B, T, H, H, D, window, rope_base, eps,
                             stream);
+}
+
+// --------------------------------------------------------------- fused q/k/v projection
+
+size_t swa_attn_fwd_x_workspace_bytes(int B, int T, int H, int Hkv, int D) {
+    Shape s;
+    if (check_sizes(B, T, H, D, &s) != SWA_OK || check_kv_heads(Hkv, &s) != SWA_OK) return 0;
+    return ws_layout(s, true).total;   // v' always lives in the workspace on this path
+}
+
+int swa_attn_qkv_prologue(const void* x, const void* Wqkv, const void* ve, const void* Wg, void* qh, void* kh,
+                          void* vp, int B, int T, int C, int H, int Hkv, int D, float rope_base, float eps,
+                          void* workspace, size_t ws_bytes, swa_stream_t stream) {
+    Shape s;
+    int rc = check_sizes(B, T, H, D, &s);
+    if (rc == SWA_OK) rc = check_kv_heads(Hkv, &s);
+    if (rc == SWA_OK) rc = check_qkv_args(x, Wqkv, ve, Wg, C, rope_base, eps);
+    if (rc != SWA_OK) return rc;
+    if (!qh || !kh || !vp || !workspace) return SWA_ERR_INVALID_ARG;
+    if (!aligned(qh, 16) || !aligned(kh, 16) || !aligned(vp, 16) || !aligned(workspace, 16)) return SWA_ERR_MISALIGNED;
+    const WsLayout L = ws_layout(s, true);
+    if (ws_bytes < L.total) return SWA_ERR_NO_MEMORY;
+    int dev;
+    if ((rc = device_ready(&dev)) != SWA_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if ((rc = launch_rope_table(ws, L, s, rope_base, st)) != SWA_OK) return rc;
+    return launch_qkv(dev, x, Wqkv, ve, Wg, C, s, eps, ws, L, qh, kh, vp, nullptr, st);
+}
+
+int swa_attn_fwd_x(const void* x, const void* Wqkv, const void* ve, const void* Wg, void* out, float* lse, int B,
+                   int T, int C, int H, int Hkv, int D, int window, float rope_base, float eps, void* workspace,
+                   size_t ws_bytes, swa_stream_t stream) {
+    Shape s;
+    int rc = check_sizes(B, T, H, D, &s);
+    if (rc == SWA_OK) rc = check_kv_heads(Hkv, &s);
+    if (rc == SWA_OK) rc = check_qkv_args(x, Wqkv, ve, Wg, C, rope_base, eps);
+    if (rc == SWA_OK) rc = check_outputs(out, lse);
+    if (rc != SWA_OK) return rc;
+    if (!workspace) return SWA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return SWA_ERR_MISALIGNED;
+    const WsLayout L = ws_layout(s, true);
+    if (ws_bytes < L.total) return SWA_ERR_NO_MEMORY;
+    int dev;
+    if ((rc = device_ready(&dev)) != SWA_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if ((rc = launch_rope_table(ws, L, s, rope_base, st)) != SWA_OK) return rc;
+    if ((rc = launch_qkv(dev, x, Wqkv, ve, Wg, C, s, eps, ws, L, ws + L.qh, ws + L.kh, ws + L.vp,
+                         reinterpret_cast<int*>(ws + L.sched), st)) != SWA_OK)
+        return rc;
+    return launch_attention(dev, nullptr, true, out, lse, s, window, ws, L, st);
 }
 
 // ---------------------------------------------------------------------------- backward

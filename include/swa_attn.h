@@ -240,6 +240,37 @@ SWA_API int swa_attn_decode_gqa(const void* q, const void* k, const void* v, con
                                 size_t ws_bytes, swa_stream_t stream);
 
 /*
+ * The layer from its input x: the bias-free q, k, v projection fused with the prologue, then the
+ * attention of swa_attn_fwd_gqa.  The pages form q, k, v of each layer as linear maps of the
+ * layer input ("Let's reproduce GPT-2 (124M)" notes, section 3, the attention listing;
+ * intelliparadigm "GPT-2 for $73", section 2: separate bias-free maps, key/value width kv_dim):
+ *   y = x Wqkv^T (fp32 tensor-core accumulation, never rounded or stored), then
+ *   qhat = RMS(RoPE(y_q)), khat = RMS(RoPE(y_k)), v' = y_v + 2 sigmoid(x[..., :32] . Wg[:, h]) ve.
+ * Arguments (device pointers, caller-owned):
+ *   x        bf16 (B, T, C) contiguous, C a multiple of 8 (at least 32 with the value embedding).
+ *   Wqkv     bf16 [(H + 2 Hkv) D, C], the linear layer's layout: rows 0 .. H D - 1 give q (head h at
+ *            rows h D ..), then Hkv D rows of k, then Hkv D rows of v.
+ *   ve, Wg   bf16 (B, T, Hkv, D) gathered value-embedding rows and [32, Hkv], both set or both NULL.
+ * swa_attn_qkv_prologue writes qh bf16 (B, T, H, D), kh and vp bf16 (B, T, Hkv, D) (caller buffers);
+ * swa_attn_fwd_x writes out bf16 (B, T, H, D) and lse fp32 (B, H, T) (NULL = skip) with qhat, khat,
+ * v' kept in the workspace.  workspace: at least swa_attn_fwd_x_workspace_bytes(B, T, H, Hkv, D)
+ * bytes, 16-byte aligned, nothing kept between calls.  Asynchronous on `stream`; arguments are
+ * validated before anything is enqueued.  Errors: SWA_ERR_INVALID_ARG (null pointer, ve / Wg not
+ * both set, C < 32 with the value embedding, Hkv not dividing H, bad rope_base / eps),
+ * SWA_ERR_UNSUPPORTED (D not 64 / 128, C not a multiple of 8, sizes beyond int32),
+ * SWA_ERR_MISALIGNED, SWA_ERR_NO_MEMORY, SWA_ERR_CUDA.
+ */
+SWA_API size_t swa_attn_fwd_x_workspace_bytes(int B, int T, int H, int Hkv, int D);
+SWA_API int swa_attn_qkv_prologue(const void* x, const void* Wqkv, const void* ve, const void* Wg,
+                                  void* qh, void* kh, void* vp, int B, int T, int C, int H, int Hkv,
+                                  int D, float rope_base, float eps, void* workspace, size_t ws_bytes,
+                                  swa_stream_t stream);
+SWA_API int swa_attn_fwd_x(const void* x, const void* Wqkv, const void* ve, const void* Wg, void* out,
+                           float* lse, int B, int T, int C, int H, int Hkv, int D, int window,
+                           float rope_base, float eps, void* workspace, size_t ws_bytes,
+                           swa_stream_t stream);
+
+/*
  * Backward of the layer: the gradient of loss = sum(dout * out) + sum(dlse * lse) for the layer of
  * swa_attn_fwd / swa_attn_fwd_gqa (the pages train it end to end; the log-sum-exp the forward
  * writes lets the backward rebuild the softmax: "Let's reproduce GPT-2 (124M)" notes, the

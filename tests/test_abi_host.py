@@ -172,3 +172,27 @@ def test_backward_workspace_and_validation():
     assert call(ws_bytes=n0 - 1) == swa.SWA_ERR_NO_MEMORY
     assert call(D=80) == swa.SWA_ERR_UNSUPPORTED
     assert call(eps=-1.0) == swa.SWA_ERR_INVALID_ARG
+
+
+def test_fused_projection_workspace_and_validation():
+    B, T, H, Hkv, D, C = 2, 100, 4, 2, 64, 256
+    n = swa.swa_attn_fwd_x_workspace_bytes(B, T, H, Hkv, D)
+    assert n > 0 and swa.swa_attn_fwd_x_workspace_bytes(B, T, H, 3, D) == 0
+    base = dict(x=A, W=A, ve=None, Wg=None, out=A, lse=A, B=B, T=T, C=C, H=H, Hkv=Hkv, D=D, window=0,
+                rope_base=1e4, eps=1e-6, workspace=A, ws_bytes=n, stream=None)
+
+    def call(**kw):
+        a = dict(base, **kw)
+        return swa.swa_attn_fwd_x(a["x"], a["W"], a["ve"], a["Wg"], a["out"], a["lse"], a["B"], a["T"], a["C"],
+                                  a["H"], a["Hkv"], a["D"], a["window"], a["rope_base"], a["eps"],
+                                  a["workspace"], a["ws_bytes"], a["stream"])
+    assert call(x=None) == swa.SWA_ERR_INVALID_ARG
+    assert call(ve=A) == swa.SWA_ERR_INVALID_ARG                 # ve without Wg
+    assert call(C=12) == swa.SWA_ERR_UNSUPPORTED                 # C not a multiple of 8
+    assert call(ve=A, Wg=A, C=16) == swa.SWA_ERR_INVALID_ARG     # the gate needs 32 channels
+    assert call(W=A + 8) == swa.SWA_ERR_MISALIGNED
+    assert call(ws_bytes=n - 1) == swa.SWA_ERR_NO_MEMORY
+    assert call(Hkv=3) == swa.SWA_ERR_INVALID_ARG
+    assert call(D=96) == swa.SWA_ERR_UNSUPPORTED
+    assert swa.swa_attn_qkv_prologue(A, A, None, None, None, A, A, B, T, C, H, Hkv, D, 1e4, 1e-6, A, n,
+                                     None) == swa.SWA_ERR_INVALID_ARG
