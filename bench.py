@@ -561,6 +561,72 @@ def run_backward(args, s):
     return 0
 
 
+def run_forward_x(args, s):
+    """The layer from its input x per timed iteration (swa_attn_fwd_x: the fused q/k/v projection +
+    prologue kernel, then the attention kernel) on the workload's shapes, x (B, T, H D) and a
+    random-init Wqkv [3 H D, H D] (std (H D)^-1/2).  Metric: FLOP/s of the projection
+    (2 M N C) plus the attention (4 D per visible pair)."""
+    import torch
+    import causal_sliding_window_swa_b200 as swa
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU path)")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    B, T, H, D = s.B, s.T, s.H, s.D
+    C = H * D
+    gen = torch.Generator().manual_seed(s.seed + 2000)
+    x = torch.randn((B, T, C), generator=gen).to(torch.bfloat16).to(dev)
+    W = (torch.randn((3 * H * D, C), generator=gen) * C ** -0.5).to(torch.bfloat16).to(dev)
+    ve = Wg = None
+    if s.ve:
+        ve = torch.randn((B, T, H, D), generator=gen).to(torch.bfloat16).to(dev)
+        Wg = (torch.randn((32, H), generator=gen) * workloads.WG_STD).to(torch.bfloat16).to(dev)
+    need = swa.swa_attn_fwd_x_workspace_bytes(B, T, H, H, D)
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        swa.forward_x(x, W, H, H, D, s.window, ve=ve, Wg=Wg, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    swa.check_device_status(stream)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(0).start()
+    for i in range(K):
+        flush.fill_(i & 0xff)
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    swa.check_device_status(stream)
+    ms = sum(a.elapsed_time(b) for a, b in evs) / K
+    proj = 2.0 * B * T * (3 * H * D) * C
+    flops = proj + flops_per_step(s)
+    tf = flops / (ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    line = {
+        "metric": "layer forward from x TFLOP/s (projection 2 M N C + attention 4 D per visible pair)",
+        "value": tf, "unit": "TFLOP/s", "n_gpus": 1, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 operands, fp32 accumulate", "data": "synthetic (seeded), random-init Wqkv",
+        "config": {"workload": f"forward_x {args.workload}: B={B} T={T} C={C} H={H} D={D} W={s.window} ve={s.ve}",
+                   "l2": "flushed between steps (256 MB write, outside the timed events)"},
+        "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": tf / peaks["bf16_tflops"], "traffic": None, "peak_source": peak_src,
+                     "note": "whole call: rope table, gate, fused projection kernel, attention kernel"},
+        "gpu_launches": (4 if s.ve else 3) * K,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -572,9 +638,10 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--reference-budget-s", type=float, default=90.0)
-    ap.add_argument("--mode", choices=["forward", "decode", "backward"], default="forward",
+    ap.add_argument("--mode", choices=["forward", "decode", "backward", "forward_x"], default="forward",
                     help="decode: time one KV-cache generation step; backward: time the layer's "
-                         "gradient; default: the layer forward")
+                         "gradient; forward_x: the layer from its input x (fused projection); "
+                         "default: the layer forward")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -583,6 +650,8 @@ def main(argv=None):
         return run_decode(args, s)
     if args.mode == "backward":
         return run_backward(args, s)
+    if args.mode == "forward_x":
+        return run_forward_x(args, s)
     if args.impl == "reference":
         return run_reference(args, s)
     return run_ours(args, s)
