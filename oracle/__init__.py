@@ -51,6 +51,12 @@ def _configure(lib):
                                            ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                            ctypes.c_double, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int, ctypes.c_int, P, ctypes.c_int64, P, P]
+    lib.swa_oracle_forward_doc_gqa.restype = ctypes.c_int
+    lib.swa_oracle_forward_doc_gqa.argtypes = [P, P, P, P, P, ctypes.c_int, P, ctypes.c_int, P,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                               ctypes.c_double, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int, P, P, ctypes.c_int64, P, P]
     lib.swa_oracle_prologue_gqa.restype = ctypes.c_int
     lib.swa_oracle_prologue_gqa.argtypes = [P, P, P, P, P, ctypes.c_int, P, ctypes.c_int, P,
                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -135,7 +141,7 @@ def _ve_args(inputs: Dict):
 
 def forward(inputs: Dict, window: int, rope_base: float = 10000.0, eps: float = 1e-6, *,
             parity: bool = True, rope: bool = True, qknorm: bool = True,
-            window_convention: int = 0, rows=None):
+            window_convention: int = 0, rows=None, doc=None):
     """Attention forward of one layer.
 
     inputs: dict with q bf16 (B,T,H,D), k, v bf16 (B,T,Hkv,D) (Hkv divides H; query head h reads
@@ -144,6 +150,8 @@ def forward(inputs: Dict, window: int, rope_base: float = 10000.0, eps: float = 
     parity=True rounds qhat, khat, v' to bf16 after the fp64 prologue (pure fp64 otherwise).
     rope/qknorm switch the prologue steps off (test-only, for the library special case).
     rows: None for every row, else flat query ids ((b*H + h)*T + i).
+    doc: None, or document ids (B,T): key j is then visible to query i only within the same
+    document as well (a document-boundary mask; RoPE positions stay the sequence positions).
 
     Returns (out, lse): out fp64 (B,T,H,D) and lse fp64 (B,H,T) when rows is None, else
     out [n_rows, D] and lse [n_rows] in the sorted order of ``rows``.
@@ -165,7 +173,18 @@ def forward(inputs: Dict, window: int, rope_base: float = 10000.0, eps: float = 
         out = np.empty((n, D), dtype=np.float64)
         lse = np.empty((n,), dtype=np.float64)
     Hkv = int(k.shape[2])
-    if Hkv == H:
+    if doc is not None:
+        import torch
+        doc_a = doc.cpu().contiguous().numpy().astype(np.int64) if isinstance(doc, torch.Tensor) \
+            else np.ascontiguousarray(doc, dtype=np.int64)
+        if doc_a.shape != (B, T):
+            raise ValueError("doc must be (B, T)")
+        rc = lib.swa_oracle_forward_doc_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(ids), _ptr(table), vocab,
+                                            _ptr(x), C, _ptr(Wg), B, T, H, Hkv, D, int(window),
+                                            float(rope_base), float(eps), int(parity), int(rope),
+                                            int(qknorm), int(window_convention), _ptr(doc_a), _ptr(rows_a),
+                                            n, _ptr(out), _ptr(lse))
+    elif Hkv == H:
         rc = lib.swa_oracle_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(ids), _ptr(table), vocab,
                                     _ptr(x), C, _ptr(Wg), B, T, H, D, int(window),
                                     float(rope_base), float(eps), int(parity), int(rope), int(qknorm),

@@ -44,7 +44,8 @@ def window_mask(T: int, window: int, convention: int = 0) -> np.ndarray:
 
 
 def forward(inputs, window: int, rope_base: float = 10000.0, eps: float = 1e-6, *,
-            rope: bool = True, qknorm: bool = True, convention: int = 0, return_weights=False):
+            rope: bool = True, qknorm: bool = True, convention: int = 0, return_weights=False,
+            doc=None):
     q, k, v = _f64(inputs["q"]), _f64(inputs["k"]), _f64(inputs["v"])
     B, T, H, D = q.shape
     if rope:
@@ -60,8 +61,11 @@ def forward(inputs, window: int, rope_base: float = 10000.0, eps: float = 1e-6, 
         gate = 2.0 * expit(np.einsum("btc,ch->bth", x, Wg))             # (B,T,H)
         v = v + gate[..., None] * ve
     s = np.einsum("bihd,bjhd->bhij", q, k) / np.sqrt(D)                # (B,H,T,T)
-    mask = window_mask(T, window, convention)
-    s = np.where(mask[None, None], s, -np.inf)
+    mask = np.broadcast_to(window_mask(T, window, convention)[None], (B, T, T))
+    if doc is not None:                                                 # same document only
+        dd = np.asarray(doc.cpu().numpy() if hasattr(doc, "cpu") else doc)
+        mask = mask & (dd[:, :, None] == dd[:, None, :])
+    s = np.where(mask[:, None], s, -np.inf)
     p = softmax(s, axis=-1)
     out = np.einsum("bhij,bjhd->bihd", p, v)
     lse = logsumexp(s, axis=-1)                                         # (B,H,T)

@@ -126,13 +126,20 @@ static int visible(int i, int j, int W, int convention) {
     return convention == 0 ? (diff < W) : (diff <= W);
 }
 
+/* Key j is visible to query i: inside the causal window and, when document ids are given (doc_b,
+ * the ids of this batch row), in the same document. */
+static int visible_doc(int i, int j, int W, int convention, const int64_t* doc_b) {
+    return visible(i, j, W, convention) && (doc_b == NULL || doc_b[j] == doc_b[i]);
+}
+
 /* One attention row: qhat_i against khat[0..T), v'[0..T) of one (b, h). */
 static void attention_row(const double* qh, const double* kh, const double* vp, int T, int D,
-                          int i, int W, int convention, double* out, double* lse, double* s) {
+                          int i, int W, int convention, const int64_t* doc_b, double* out,
+                          double* lse, double* s) {
     const double scale = 1.0 / sqrt((double)D);
     double M = -INFINITY;
     for (int j = 0; j < T; ++j) {
-        if (!visible(i, j, W, convention)) continue;
+        if (!visible_doc(i, j, W, convention, doc_b)) continue;
         double acc = 0.0;
         for (int d = 0; d < D; ++d) acc += qh[d] * kh[(size_t)j * D + d];
         s[j] = acc * scale;
@@ -140,10 +147,10 @@ static void attention_row(const double* qh, const double* kh, const double* vp, 
     }
     double L = 0.0;
     for (int j = 0; j < T; ++j)
-        if (visible(i, j, W, convention)) L += exp(s[j] - M);
+        if (visible_doc(i, j, W, convention, doc_b)) L += exp(s[j] - M);
     for (int d = 0; d < D; ++d) out[d] = 0.0;
     for (int j = 0; j < T; ++j) {
-        if (!visible(i, j, W, convention)) continue;
+        if (!visible_doc(i, j, W, convention, doc_b)) continue;
         double p = exp(s[j] - M) / L;
         for (int d = 0; d < D; ++d) out[d] += p * vp[(size_t)j * D + d];
     }
@@ -167,18 +174,21 @@ int swa_oracle_threads(void) {
  * x, C          x (B, T, C) bf16; the gate reads channels 0..31.
  * Wg            [32, Hkv] bf16.
  * window        <= 0 or >= T: full causal.
+ * doc           (swa_oracle_forward_doc_gqa) document ids (B, T) or NULL: key j is visible to
+ *               query i only if doc[b, j] == doc[b, i] as well (a document-boundary mask; RoPE
+ *               positions stay the positions t in the sequence).
  * rows/n_rows   flat query ids ((b*H + h)*T + i), sorted ascending; rows == NULL: every row.
  * out           rows == NULL: (B, T, H, D) fp64; else [n_rows, D].
  * lse           rows == NULL: (B, H, T) fp64;   else [n_rows].
  * Returns 0, or -1 on bad arguments / allocation failure.
  */
-int swa_oracle_forward_gqa(const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                           const int64_t* ids, const uint16_t* table, int vocab,
-                           const uint16_t* x, int C, const uint16_t* Wg,
-                           int B, int T, int H, int Hkv, int D, int window, double rope_base,
-                           double eps, int round_bf16, int use_rope, int use_qknorm,
-                           int window_convention, const int64_t* rows, int64_t n_rows,
-                           double* out, double* lse) {
+int swa_oracle_forward_doc_gqa(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                               const int64_t* ids, const uint16_t* table, int vocab,
+                               const uint16_t* x, int C, const uint16_t* Wg,
+                               int B, int T, int H, int Hkv, int D, int window, double rope_base,
+                               double eps, int round_bf16, int use_rope, int use_qknorm,
+                               int window_convention, const int64_t* doc, const int64_t* rows,
+                               int64_t n_rows, double* out, double* lse) {
     if (B < 1 || T < 1 || H < 1 || D < 2 || (D % 2) != 0) return -1;
     if (Hkv < 1 || Hkv > H || (H % Hkv) != 0) return -1;
     const int G = H / Hkv;
@@ -230,7 +240,8 @@ int swa_oracle_forward_gqa(const uint16_t* q, const uint16_t* k, const uint16_t*
                 double l;
                 prologue_qk(q, T, H, D, b, i, h, rope_base, eps, use_rope, use_qknorm,
                             round_bf16, qh);
-                attention_row(qh, kh, vp, T, D, i, W, window_convention, o, &l, s);
+                attention_row(qh, kh, vp, T, D, i, W, window_convention,
+                              doc ? doc + (size_t)b * T : NULL, o, &l, s);
                 if (rows) {
                     memcpy(out + (size_t)r * D, o, sizeof(double) * (size_t)D);
                     lse[r] = l;
@@ -247,6 +258,19 @@ int swa_oracle_forward_gqa(const uint16_t* q, const uint16_t* k, const uint16_t*
     }
     free(kh); free(vp);
     return rc;
+}
+
+/* Without document ids: the causal window alone. */
+int swa_oracle_forward_gqa(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                           const int64_t* ids, const uint16_t* table, int vocab,
+                           const uint16_t* x, int C, const uint16_t* Wg,
+                           int B, int T, int H, int Hkv, int D, int window, double rope_base,
+                           double eps, int round_bf16, int use_rope, int use_qknorm,
+                           int window_convention, const int64_t* rows, int64_t n_rows,
+                           double* out, double* lse) {
+    return swa_oracle_forward_doc_gqa(q, k, v, ids, table, vocab, x, C, Wg, B, T, H, Hkv, D, window,
+                                      rope_base, eps, round_bf16, use_rope, use_qknorm,
+                                      window_convention, NULL, rows, n_rows, out, lse);
 }
 
 /* The multi-head layer: every tensor has H heads. */

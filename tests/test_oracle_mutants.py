@@ -13,6 +13,7 @@ import oracle
 from oracle import build as obuild
 import tests.test_oracle_backward_pins as bpins
 import tests.test_oracle_pins as pins
+import tests.test_oracle_doc_pins as dpins
 import tests.test_oracle_qkv_pins as qpins
 
 MUTANTS = {
@@ -109,6 +110,17 @@ QKV_MUTANTS = {
     "proj rope position from b": ("if (use_rope) rope_inplace(row, D, t, rope_base);", "if (use_rope) rope_inplace(row, D, b, rope_base);"),
 }
 
+DOC_MUTANTS = {
+    "doc compared with the first position": ("doc_b[j] == doc_b[i]", "doc_b[j] == doc_b[0]"),
+    "previous document leaks in": ("doc_b[j] == doc_b[i]", "(doc_b[j] == doc_b[i] || doc_b[j] + 1 == doc_b[i])"),
+}
+
+DOC_PIN_FUNCS = [
+    lambda: dpins.test_documents_match_bruteforce(7, True),
+    dpins.test_each_document_is_the_layer_on_its_own_slice,
+    dpins.test_first_row_of_each_document_is_its_own_value,
+]
+
 QKV_PIN_FUNCS = [
     lambda: qpins.test_permutation_weights_reduce_to_the_prologue_bit_for_bit(2, 2, 16, True, False),
     lambda: qpins.test_permutation_weights_reduce_to_the_prologue_bit_for_bit(4, 2, 8, True, True),
@@ -156,6 +168,17 @@ def test_planted_projection_mistake_is_caught(name):
         oracle._swap_library(_build_mutant(old, new, tmp))
         try:
             assert _failing_pins(QKV_PIN_FUNCS) >= 1, f"no pin caught the planted mistake: {name}"
+        finally:
+            oracle._swap_library(None)
+
+
+@pytest.mark.parametrize("name", sorted(DOC_MUTANTS))
+def test_planted_document_mask_mistake_is_caught(name):
+    old, new = DOC_MUTANTS[name]
+    with tempfile.TemporaryDirectory() as tmp:
+        oracle._swap_library(_build_mutant(old, new, tmp))
+        try:
+            assert _failing_pins(DOC_PIN_FUNCS) >= 1, f"no pin caught the planted mistake: {name}"
         finally:
             oracle._swap_library(None)
 
