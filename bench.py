@@ -646,6 +646,8 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     s = WORKLOADS[args.workload]
+    if args.mode != "forward" and (dist_env()[1] > 1 or args.gpus > 1):
+        ap.error(f"--mode {args.mode} runs on one GPU (the forward mode shards across ranks)")
     if args.mode == "decode":
         return run_decode(args, s)
     if args.mode == "backward":
