@@ -46,3 +46,17 @@ def test_frozen_oracle_rows():
     out, lse = oracle.forward(d, s.window, parity=True, rows=doc["rows"])
     assert np.abs(out - np.array(doc["out"])).max() < 1e-12
     assert np.abs(lse - np.array(doc["lse"])).max() < 1e-12
+
+
+def test_frozen_oracle_gradients_and_projection():
+    import tests.golden.make_golden_grads as mg
+    doc = _load("small_oracle_grads.json")
+    d, dout, dlse, W = mg.inputs()
+    assert workloads.sha256_of(d) == doc["input_sha256"], "seeded input generator changed"
+    g = oracle.backward(d, dout, mg.SHAPE.window, dlse=dlse, parity=True)
+    for k, v in doc["grads"].items():
+        assert np.abs(g[k].reshape(-1) - np.array(v)).max() < 1e-12, k
+    qh, kh, vp = oracle.qkv_prologue(d["x"], W, mg.SHAPE.H, mg.SHAPE.Hkv, mg.SHAPE.D, ids=d["ids"],
+                                     table=d["table"], Wg=d["Wg"], parity=True)
+    for k, v in (("qhat", qh), ("khat", kh), ("vprime", vp)):
+        assert np.array_equal(v.reshape(-1), np.array(doc["qkv"][k])), k
