@@ -136,7 +136,8 @@ WsLayout ws_layout(const Shape& s, bool has_ve) {
 
 int g_num_sms[64] = {0};
 
-// Dynamic shared memory of every instantiation of the fused projection kernel.
+// Dynamic shared memory of every instantiation of the fused projection kernel (set on the first
+// fused-projection call on each device, so the other entry points never depend on it).
 bool set_qkv_smem() {
     const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
     return cudaFuncSetAttribute(swa::qkv_gemm_kernel<128, 256, true>, a, swa::QkvCfg<256>::SMEM_TOTAL) == cudaSuccess &&
@@ -183,8 +184,7 @@ int device_ready(int* dev_out) {
                 cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<64>, (cudaFuncAttribute)smem_attr,
                                      swa::BwdCfg<64>::KV_SMEM) != cudaSuccess ||
                 cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<128>, (cudaFuncAttribute)smem_attr,
-                                     swa::BwdCfg<128>::KV_SMEM) != cudaSuccess ||
-                !set_qkv_smem()) {
+                                     swa::BwdCfg<128>::KV_SMEM) != cudaSuccess) {
                 cudaGetLastError();
                 checked[dev] = 0;
                 return SWA_ERR_CUDA;
@@ -400,6 +400,15 @@ int launch_qkv(int dev, const void* x, const void* Wqkv, const void* ve, const v
     const bool has_ve = ve != nullptr;
     const long long M = (long long)s.B * s.T;
     if (M * C >= (1ll << 31) || M >= (1ll << 31) / std::max(1, s.H * s.D)) return SWA_ERR_UNSUPPORTED;
+    {
+        static std::once_flag once[64];
+        static bool ok[64] = {false};
+        std::call_once(once[dev], [&] { ok[dev] = set_qkv_smem(); });
+        if (!ok[dev]) {
+            cudaGetLastError();
+            return SWA_ERR_CUDA;
+        }
+    }
     float2* gate = reinterpret_cast<float2*>(ws + L.gate);
     if (has_ve) {
         const int n_kv_rows = (int)(M * s.Hkv);
