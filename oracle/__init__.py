@@ -68,6 +68,12 @@ def _configure(lib):
                                             ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                             ctypes.c_double, ctypes.c_int, ctypes.c_int,
                                             ctypes.c_int, ctypes.c_int, P, P, P, P, P, P, P, P]
+    lib.swa_oracle_backward_doc_gqa.restype = ctypes.c_int
+    lib.swa_oracle_backward_doc_gqa.argtypes = [P, P, P, P, P, ctypes.c_int, P, ctypes.c_int, P,
+                                                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                                ctypes.c_double, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int, ctypes.c_int, P, P, P, P, P, P, P, P, P]
     lib.swa_oracle_backward_rows_gqa.restype = ctypes.c_int
     lib.swa_oracle_backward_rows_gqa.argtypes = [P, P, P, P, P, ctypes.c_int, P, ctypes.c_int, P,
                                                  ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -227,7 +233,7 @@ def prologue(inputs: Dict, rope_base: float = 10000.0, eps: float = 1e-6, *,
 
 def backward(inputs: Dict, dout, window: int, dlse=None, rope_base: float = 10000.0,
              eps: float = 1e-6, *, parity: bool = False, rope: bool = True, qknorm: bool = True,
-             window_convention: int = 0):
+             window_convention: int = 0, doc=None):
     """Gradient of ``sum(dout * out) + sum(dlse * lse)`` with respect to the layer's inputs.
 
     inputs as for ``forward``; dout (B,T,H,D) and dlse (B,H,T) (None for zero) are taken as
@@ -237,7 +243,7 @@ def backward(inputs: Dict, dout, window: int, dlse=None, rope_base: float = 1000
 
     Returns a dict of fp64 arrays: dq (B,T,H,D); dk, dv (B,T,Hkv,D); on value-embedding layers
     also dve (B,T,Hkv,D) (gradient of the looked-up table row at each position), dx (B,T,32)
-    (the gate's input channels) and dWg [32,Hkv].
+    (the gate's input channels) and dWg [32,Hkv].  doc: document ids (B,T) as in ``forward``.
     """
     lib = _load()
     q, k, v = _bits(inputs["q"]), _bits(inputs["k"]), _bits(inputs["v"])
@@ -257,10 +263,17 @@ def backward(inputs: Dict, dout, window: int, dlse=None, rope_base: float = 1000
     if ids is not None:
         grads.update(dve=np.empty((B, T, Hkv, D)), dx=np.empty((B, T, 32)),
                      dWg=np.empty((32, Hkv)))
-    rc = lib.swa_oracle_backward_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(ids), _ptr(table), vocab,
+    doc_a = None
+    if doc is not None:
+        import torch
+        doc_a = doc.cpu().contiguous().numpy().astype(np.int64) if isinstance(doc, torch.Tensor) \
+            else np.ascontiguousarray(doc, dtype=np.int64)
+        if doc_a.shape != (B, T):
+            raise ValueError("doc must be (B, T)")
+    rc = lib.swa_oracle_backward_doc_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(ids), _ptr(table), vocab,
                                      _ptr(x), C, _ptr(Wg), B, T, H, Hkv, D, int(window),
                                      float(rope_base), float(eps), int(parity), int(rope),
-                                     int(qknorm), int(window_convention), _ptr(go), _ptr(gl),
+                                     int(qknorm), int(window_convention), _ptr(doc_a), _ptr(go), _ptr(gl),
                                      _ptr(grads["dq"]), _ptr(grads["dk"]), _ptr(grads["dv"]),
                                      _ptr(grads.get("dve")), _ptr(grads.get("dx")),
                                      _ptr(grads.get("dWg")))

@@ -413,30 +413,31 @@ static void bwd_kv_prologue(const uint16_t* k, const uint16_t* v, const int64_t*
 
 /* Row pass for query row i of one (b, h): scores against the visible keys (scratch s of T),
  * lse_i, delta_i = sum_j P_ij dP_ij and, if dqi is not NULL, dqhat_i = sum_j dS_ij khat_j / sqrt(D).
- * gi is dout of the row, gl its dlse. */
+ * gi is dout of the row, gl its dlse; doc_b, if not NULL, the document ids of this batch row. */
 static void bwd_query_row(const double* qi, const double* gi, double gl, const double* kh,
                           const double* vp, int T, int D, int i, int W, int window_convention,
-                          double inv_sqrt_d, double* s, double* lse_i, double* delta_i, double* dqi) {
+                          const int64_t* doc_b, double inv_sqrt_d, double* s, double* lse_i,
+                          double* delta_i, double* dqi) {
     double M = -INFINITY;
     for (int j = 0; j < T; ++j) {
-        if (!visible(i, j, W, window_convention)) continue;
+        if (!visible_doc(i, j, W, window_convention, doc_b)) continue;
         s[j] = dot_d(qi, kh + (size_t)j * D, D) * inv_sqrt_d;
         if (s[j] > M) M = s[j];
     }
     double L = 0.0;
     for (int j = 0; j < T; ++j)
-        if (visible(i, j, W, window_convention)) L += exp(s[j] - M);
+        if (visible_doc(i, j, W, window_convention, doc_b)) L += exp(s[j] - M);
     const double li = M + log(L);
     double dl = 0.0;
     for (int j = 0; j < T; ++j)
-        if (visible(i, j, W, window_convention))
+        if (visible_doc(i, j, W, window_convention, doc_b))
             dl += exp(s[j] - li) * dot_d(gi, vp + (size_t)j * D, D);
     *lse_i = li;
     *delta_i = dl;
     if (dqi == NULL) return;
     for (int d = 0; d < D; ++d) dqi[d] = 0.0;
     for (int j = 0; j < T; ++j) {
-        if (!visible(i, j, W, window_convention)) continue;
+        if (!visible_doc(i, j, W, window_convention, doc_b)) continue;
         const double p = exp(s[j] - li);
         const double ds = p * (dot_d(gi, vp + (size_t)j * D, D) - dl) + p * gl;
         for (int d = 0; d < D; ++d) dqi[d] += ds * kh[(size_t)j * D + d] * inv_sqrt_d;
@@ -444,13 +445,15 @@ static void bwd_query_row(const double* qi, const double* gi, double gl, const d
 }
 
 /* Key pass for key row j of one (b, h): adds sum_i dS_ij qhat_i / sqrt(D) to dkj and
- * sum_i P_ij dout_i to dvj over the queries i in [j, i_end] that see key j.  qh, lse, delta are
- * indexed by query position; dout / dlse are the full tensors. */
+ * sum_i P_ij dout_i to dvj over the queries i in [j, i_end] that see key j (and, with document
+ * ids, share its document).  qh, lse, delta are indexed by query position; dout / dlse are the
+ * full tensors. */
 static void bwd_key_row(const double* kj, const double* vj, const double* qh, const double* lse,
                         const double* delta, const double* dout, const double* dlse, int b, int h,
-                        int T, int H, int D, int j, int i_end, double inv_sqrt_d, double* dkj,
-                        double* dvj) {
+                        int T, int H, int D, int j, int i_end, const int64_t* doc_b,
+                        double inv_sqrt_d, double* dkj, double* dvj) {
     for (int i = j; i <= i_end; ++i) {
+        if (doc_b != NULL && doc_b[i] != doc_b[j]) continue;    /* another document */
         const double* qi = qh + (size_t)i * D;
         const double* gi = dout + (((size_t)b * T + i) * H + h) * (size_t)D;
         const double gl = dlse ? dlse[((size_t)b * H + h) * T + i] : 0.0;
@@ -500,16 +503,17 @@ static void bwd_kv_outputs(const uint16_t* k, const int64_t* ids, const uint16_t
  *   dx            (B, T, 32): dL/d x[b, t, c] for the 32 gate channels (channels >= 32 do not
  *                 reach the layer).  VE layers only.
  *   dWg           [32, Hkv].  VE layers only.
+ *   doc           (swa_oracle_backward_doc_gqa) document ids (B, T) or NULL, as in the forward.
  * Returns 0, or -1 on bad arguments / allocation failure.
  */
-int swa_oracle_backward_gqa(const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                            const int64_t* ids, const uint16_t* table, int vocab,
-                            const uint16_t* x, int C, const uint16_t* Wg,
-                            int B, int T, int H, int Hkv, int D, int window, double rope_base,
-                            double eps, int round_bf16, int use_rope, int use_qknorm,
-                            int window_convention, const double* dout, const double* dlse,
-                            double* dq, double* dk, double* dv, double* dve, double* dx,
-                            double* dWg) {
+int swa_oracle_backward_doc_gqa(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                const int64_t* ids, const uint16_t* table, int vocab,
+                                const uint16_t* x, int C, const uint16_t* Wg,
+                                int B, int T, int H, int Hkv, int D, int window, double rope_base,
+                                double eps, int round_bf16, int use_rope, int use_qknorm,
+                                int window_convention, const int64_t* doc, const double* dout,
+                                const double* dlse, double* dq, double* dk, double* dv, double* dve,
+                                double* dx, double* dWg) {
     if (B < 1 || T < 1 || H < 1 || D < 2 || (D % 2) != 0) return -1;
     if (Hkv < 1 || Hkv > H || (H % Hkv) != 0) return -1;
     if (dout == NULL || dq == NULL || dk == NULL || dv == NULL) return -1;
@@ -563,7 +567,8 @@ int swa_oracle_backward_gqa(const uint16_t* q, const uint16_t* k, const uint16_t
                         const double* gi = dout + (((size_t)b * T + i) * H + h) * (size_t)D;
                         const double gl = dlse ? dlse[((size_t)b * H + h) * T + i] : 0.0;
                         bwd_query_row(qh + (size_t)i * D, gi, gl, kh, vp, T, D, i, W, window_convention,
-                                      inv_sqrt_d, s, &lse[i], &delta[i], dqh + (size_t)i * D);
+                                      doc ? doc + (size_t)b * T : NULL, inv_sqrt_d, s, &lse[i], &delta[i],
+                                      dqh + (size_t)i * D);
                     }
                     free(s);
                 }
@@ -575,7 +580,8 @@ int swa_oracle_backward_gqa(const uint16_t* q, const uint16_t* k, const uint16_t
                 for (int j = 0; j < T; ++j) {
                     const int i_end = (j + reach < T - 1) ? j + reach : T - 1;
                     bwd_key_row(kh + (size_t)j * D, vp + (size_t)j * D, qh, lse, delta, dout, dlse, b, h,
-                                T, H, D, j, i_end, inv_sqrt_d, dkh + (size_t)j * D, dvp + (size_t)j * D);
+                                T, H, D, j, i_end, doc ? doc + (size_t)b * T : NULL, inv_sqrt_d,
+                                dkh + (size_t)j * D, dvp + (size_t)j * D);
                 }
 
                 /* dq rows of head h. */
@@ -658,6 +664,20 @@ done:
  * key row j, the queries in [j, j + W - 1] of every query head of its group), so it equals the full
  * backward's value bit for bit.  Returns 0, or -1 on bad arguments / allocation failure.
  */
+/* Without document ids: the causal window alone. */
+int swa_oracle_backward_gqa(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                            const int64_t* ids, const uint16_t* table, int vocab,
+                            const uint16_t* x, int C, const uint16_t* Wg,
+                            int B, int T, int H, int Hkv, int D, int window, double rope_base,
+                            double eps, int round_bf16, int use_rope, int use_qknorm,
+                            int window_convention, const double* dout, const double* dlse,
+                            double* dq, double* dk, double* dv, double* dve, double* dx,
+                            double* dWg) {
+    return swa_oracle_backward_doc_gqa(q, k, v, ids, table, vocab, x, C, Wg, B, T, H, Hkv, D, window,
+                                       rope_base, eps, round_bf16, use_rope, use_qknorm,
+                                       window_convention, NULL, dout, dlse, dq, dk, dv, dve, dx, dWg);
+}
+
 int swa_oracle_backward_rows_gqa(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                  const int64_t* ids, const uint16_t* table, int vocab,
                                  const uint16_t* x, int C, const uint16_t* Wg,
@@ -744,7 +764,7 @@ int swa_oracle_backward_rows_gqa(const uint16_t* q, const uint16_t* k, const uin
                         const double* gi = dout + (((size_t)b * T + i) * H + h) * (size_t)D;
                         const double gl = dlse ? dlse[((size_t)b * H + h) * T + i] : 0.0;
                         bwd_query_row(qh + (size_t)i * D, gi, gl, kh, vp, T, D, i, W, window_convention,
-                                      inv_sqrt_d, s, &lse[i], &delta[i],
+                                      NULL, inv_sqrt_d, s, &lse[i], &delta[i],
                                       need[i] == 2 ? dqh + (size_t)i * D : NULL);
                     }
                     free(s);
@@ -755,7 +775,7 @@ int swa_oracle_backward_rows_gqa(const uint16_t* q, const uint16_t* k, const uin
                     if (!kneed[j]) continue;
                     const int i_end = (j + reach < T - 1) ? j + reach : T - 1;
                     bwd_key_row(kh + (size_t)j * D, vp + (size_t)j * D, qh, lse, delta, dout, dlse, b, h,
-                                T, H, D, j, i_end, inv_sqrt_d, dkh + (size_t)j * D, dvp + (size_t)j * D);
+                                T, H, D, j, i_end, NULL, inv_sqrt_d, dkh + (size_t)j * D, dvp + (size_t)j * D);
                 }
                 double* xr = (double*)malloc(sizeof(double) * (size_t)D);
                 if (xr == NULL) { rc = -1; break; }

@@ -73,3 +73,74 @@ def test_first_row_of_each_document_is_its_own_value():
     starts = [0] + [t for t in range(1, T) if doc[0, t] != doc[0, t - 1]]
     for t in starts:
         assert np.abs(o[0, t] - vp[0, t]).max() < 1e-12
+
+
+# ------------------------------------------------------------------- the gradient with documents
+
+def _fd_grads(d, window, dout, dlse, doc):
+    """Central differences of the brute-force forward with its own document mask."""
+    inp = {k: (v.numpy().copy() if k == "ids" else v.double().numpy().copy()) for k, v in d.items()}
+
+    def loss():
+        o, l = brute.forward(inp, window, doc=doc)
+        return float(np.sum(o * dout) + np.sum(l * dlse))
+
+    out = {}
+    for name in ("q", "k", "v"):
+        a = inp[name]
+        g = np.zeros_like(a)
+        for idx in np.ndindex(a.shape):
+            old = a[idx]
+            h = 1e-5 * max(1.0, abs(old))
+            a[idx] = old + h
+            lp = loss()
+            a[idx] = old - h
+            lm = loss()
+            a[idx] = old
+            g[idx] = (lp - lm) / (2 * h)
+        out[name] = g
+    return out
+
+
+@pytest.mark.parametrize("window", [0, 3])
+def test_gradient_with_documents_matches_central_differences(window):
+    B, T, H, D = 1, 9, 2, 8
+    d = _layer(B, T, H, D, False, 40 + window)
+    doc = torch.tensor([[0, 0, 0, 1, 1, 1, 1, 2, 2]])
+    g = torch.Generator().manual_seed(window)
+    dout = torch.randn((B, T, H, D), generator=g, dtype=torch.float64).numpy()
+    dlse = torch.randn((B, H, T), generator=g, dtype=torch.float64).numpy()
+    got = oracle.backward(d, dout, window, dlse=dlse, doc=doc)
+    fd = _fd_grads(d, window, dout, dlse, doc)
+    for key, name in (("dq", "q"), ("dk", "k"), ("dv", "v")):
+        assert np.all(np.abs(got[key] - fd[name]) <= 1e-7 + 1e-6 * np.abs(fd[name])), key
+
+
+def test_gradient_with_one_document_is_the_plain_gradient_bit_for_bit():
+    B, T, H, D = 2, 30, 3, 16
+    d = _layer(B, T, H, D, True, 9)
+    g = torch.Generator().manual_seed(2)
+    dout = torch.randn((B, T, H, D), generator=g, dtype=torch.float64).numpy()
+    dlse = torch.randn((B, H, T), generator=g, dtype=torch.float64).numpy()
+    a = oracle.backward(d, dout, 7, dlse=dlse)
+    b = oracle.backward(d, dout, 7, dlse=dlse, doc=torch.zeros((B, T), dtype=torch.int64))
+    for key in a:
+        assert np.array_equal(a[key], b[key]), key
+
+
+def test_gradient_of_each_document_is_the_gradient_on_its_own_slice():
+    """In fp64 the documents are independent layers (relative positions only), so each one's
+    gradient equals the plain gradient of the layer run on its slice alone."""
+    B, T, H, D, W = 1, 50, 2, 16, 12
+    d = _layer(B, T, H, D, True, 13)
+    doc = torch.zeros((B, T), dtype=torch.int64)
+    doc[0, 22:] = 1
+    g = torch.Generator().manual_seed(3)
+    dout = torch.randn((B, T, H, D), generator=g, dtype=torch.float64).numpy()
+    dlse = torch.randn((B, H, T), generator=g, dtype=torch.float64).numpy()
+    full = oracle.backward(d, dout, W, dlse=dlse, doc=doc)
+    for s0, e0 in ((0, 22), (22, 50)):
+        part = {k: (v[:, s0:e0].contiguous() if k in ("q", "k", "v", "ids", "x") else v) for k, v in d.items()}
+        gp = oracle.backward(part, dout[:, s0:e0], W, dlse=dlse[:, :, s0:e0])
+        for key in ("dq", "dk", "dv", "dve", "dx"):
+            assert np.abs(full[key][:, s0:e0] - gp[key]).max() < 1e-11, (key, s0)

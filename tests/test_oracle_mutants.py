@@ -113,12 +113,15 @@ QKV_MUTANTS = {
 DOC_MUTANTS = {
     "doc compared with the first position": ("doc_b[j] == doc_b[i]", "doc_b[j] == doc_b[0]"),
     "previous document leaks in": ("doc_b[j] == doc_b[i]", "(doc_b[j] == doc_b[i] || doc_b[j] + 1 == doc_b[i])"),
+    "backward key pass ignores documents": ("if (doc_b != NULL && doc_b[i] != doc_b[j]) continue;", ";"),
 }
 
 DOC_PIN_FUNCS = [
     lambda: dpins.test_documents_match_bruteforce(7, True),
     dpins.test_each_document_is_the_layer_on_its_own_slice,
     dpins.test_first_row_of_each_document_is_its_own_value,
+    lambda: dpins.test_gradient_with_documents_matches_central_differences(3),
+    dpins.test_gradient_of_each_document_is_the_gradient_on_its_own_slice,
 ]
 
 QKV_PIN_FUNCS = [
