@@ -31,8 +31,9 @@
 //                         dgate_x = dz Wg^T and dWg = gate_x^T dz (fixed summation order).
 // The two tensor-core kernels use seven products per (query tile, key tile) pair instead of
 // five so that neither needs fp32 atomics: dQ is owned by the query-tile kernel, dK and dV by the
-// key-tile kernel.  Every tensor-core operand form here (A from tensor memory or shared memory, B
-// K-major or MN-major, P-style bf16 pairs in tensor memory) is one the forward kernel uses.
+// key-tile kernel.  The tensor-core operand forms here are A from tensor memory (bf16 pairs written
+// by the warps, as the forward feeds P) or from shared memory (K-major, 128-byte swizzle), and B
+// K-major or MN-major from shared memory.
 #pragma once
 
 #include <cuda.h>
