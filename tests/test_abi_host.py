@@ -196,3 +196,21 @@ def test_fused_projection_workspace_and_validation():
     assert call(D=96) == swa.SWA_ERR_UNSUPPORTED
     assert swa.swa_attn_qkv_prologue(A, A, None, None, None, A, A, B, T, C, H, Hkv, D, 1e4, 1e-6, A, n,
                                      None) == swa.SWA_ERR_INVALID_ARG
+
+
+def test_header_is_plain_c():
+    """include/swa_attn.h compiles as C99 (no C++ or torch types at the boundary), and every entry
+    point it declares can be taken by address from C (the source goes to gcc on stdin)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no gcc")
+    names = sorted(_declared_symbols())
+    src = ('#include "swa_attn.h"\n'
+           "typedef void (*swa_fn)(void);\n"
+           "swa_fn swa_entry_points[] = {\n" + "".join(f"    (swa_fn)&{n},\n" for n in names) + "};\n")
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-fsyntax-only",
+                        "-I", os.path.join(ROOT, "include"), "-x", "c", "-"], input=src, capture_output=True,
+                       text=True)
+    assert r.returncode == 0, r.stderr
