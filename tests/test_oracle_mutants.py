@@ -142,6 +142,13 @@ def _failing_pins(funcs=None):
     return failed
 
 
+def _scratch():
+    """Mutant builds go to a git-ignored directory inside the repository."""
+    d = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), ".pytest_cache", "mutants")
+    os.makedirs(d, exist_ok=True)
+    return d
+
+
 def _build_mutant(old, new, tmp):
     src = open(obuild.SRC).read()
     assert src.count(old) == 1, f"mutation anchor not found: {old!r}"
@@ -156,7 +163,7 @@ def _build_mutant(old, new, tmp):
 @pytest.mark.parametrize("name", sorted(BACKWARD_MUTANTS))
 def test_planted_backward_mistake_is_caught(name):
     old, new = BACKWARD_MUTANTS[name]
-    with tempfile.TemporaryDirectory() as tmp:
+    with tempfile.TemporaryDirectory(dir=_scratch()) as tmp:
         oracle._swap_library(_build_mutant(old, new, tmp))
         try:
             assert _failing_pins(BACKWARD_PIN_FUNCS) >= 1, f"no pin caught the planted mistake: {name}"
@@ -167,7 +174,7 @@ def test_planted_backward_mistake_is_caught(name):
 @pytest.mark.parametrize("name", sorted(QKV_MUTANTS))
 def test_planted_projection_mistake_is_caught(name):
     old, new = QKV_MUTANTS[name]
-    with tempfile.TemporaryDirectory() as tmp:
+    with tempfile.TemporaryDirectory(dir=_scratch()) as tmp:
         oracle._swap_library(_build_mutant(old, new, tmp))
         try:
             assert _failing_pins(QKV_PIN_FUNCS) >= 1, f"no pin caught the planted mistake: {name}"
@@ -178,7 +185,7 @@ def test_planted_projection_mistake_is_caught(name):
 @pytest.mark.parametrize("name", sorted(DOC_MUTANTS))
 def test_planted_document_mask_mistake_is_caught(name):
     old, new = DOC_MUTANTS[name]
-    with tempfile.TemporaryDirectory() as tmp:
+    with tempfile.TemporaryDirectory(dir=_scratch()) as tmp:
         oracle._swap_library(_build_mutant(old, new, tmp))
         try:
             assert _failing_pins(DOC_PIN_FUNCS) >= 1, f"no pin caught the planted mistake: {name}"
@@ -199,7 +206,7 @@ def test_planted_mistake_is_caught(name):
     old, new = MUTANTS[name]
     src = open(obuild.SRC).read()
     assert src.count(old) == 1, f"mutation anchor not found: {old!r}"
-    with tempfile.TemporaryDirectory() as tmp:
+    with tempfile.TemporaryDirectory(dir=_scratch()) as tmp:
         c = os.path.join(tmp, "mutant.c")
         so = os.path.join(tmp, "libmutant.so")
         open(c, "w").write(src.replace(old, new))
