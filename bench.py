@@ -116,7 +116,7 @@ class ClockSampler:
                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, index: int, period_s: float = 0.02):
+    def __init__(self, index: int, period_s: float = 0.001):
         self.index = index
         self.period = period_s
         self.samples = []
@@ -627,6 +627,90 @@ def run_forward_x(args, s):
     return 0
 
 
+def run_sssl(args):
+    """The SSSL stack of the d24 model at one point of the length sweep: 24 consecutive layer
+    calls (swa_attn_fwd, the public call, library workspace) with windows S,S,S,L (S = T/2,
+    L = T), value embeddings on even layers, H = 12, D = 128, B = 32768 / T.  Every layer has its
+    own inputs (about 0.4 GB per layer, 9.7 GB in all, so L2 never serves a later layer).  One
+    timed step = all 24 calls.  Metric: TFLOP/s over the stack's unmasked pairs (4 D per pair)
+    and tokens/s = B T / step time.  Inputs are drawn on the device from a seeded generator
+    (N(0,1) bf16; ids uniform over the vocabulary; Wg N(0, 0.02)), the shapes and distributions
+    of the workload; the parity tests check the same stack drawn on the host."""
+    import torch
+    import causal_sliding_window_swa_b200 as swa
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU path)")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    T = args.sssl_T
+    B = 32768 // T
+    H, D = 12, 128
+    shapes = workloads.sssl_layer_shapes(B, T, H, D)
+    gen = torch.Generator(device=dev).manual_seed(workloads.SSSL_SEED)
+    bf = lambda *shp, std=1.0: (torch.randn(shp, generator=gen, device=dev) * std).to(torch.bfloat16)
+    layers = []
+    for s in shapes:
+        L = dict(q=bf(B, T, H, D), k=bf(B, T, H, D), v=bf(B, T, H, D), ve=None, gate_x=None, Wg=None)
+        if s.ve:
+            ids = torch.randint(0, workloads.VOCAB, (B, T), generator=gen, device=dev)
+            table = bf(workloads.VOCAB, H * D)
+            L["ve"] = table[ids].view(B, T, H, D)
+            del table
+            L["gate_x"] = bf(B, T, workloads.GATE_CHANNELS)
+            L["Wg"] = bf(workloads.GATE_CHANNELS, H, std=workloads.WG_STD)
+        layers.append((s, L))
+    out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    st = stream.cuda_stream
+    P = lambda t: None if t is None else t.data_ptr()
+    calls = [(P(L["q"]), P(L["k"]), P(L["v"]), P(L["ve"]), P(L["gate_x"]), P(L["Wg"]), out.data_ptr(),
+              lse.data_ptr(), B, T, H, D, s.window, 10000.0, 1e-6, st) for s, L in layers]
+
+    def step():
+        for a in calls:
+            rc = swa.swa_attn_fwd(*a)
+            if rc != 0:
+                raise swa.SwaError(rc, "swa_attn_fwd")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    swa.check_device_status(stream)
+    K = args.steps
+    sampler = ClockSampler(0).start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    swa.check_device_status(stream)
+    ms = e0.elapsed_time(e1) / K
+    flops = sum(flops_per_step(s) for s in shapes)
+    tf = flops / (ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    line = {
+        "metric": "SSSL stack (24 layers S,S,S,L) attention fwd TFLOP/s (unmasked pairs) & tokens/s",
+        "value": tf, "unit": "TFLOP/s", "n_gpus": 1, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 drawn on the device; VE on even layers)",
+        "config": {"workload": f"SSSL stack B={B} T={T} H={H} D={D}, 24 layers S={T // 2},S,S,L={T}",
+                   "l2": "no flush: each layer's inputs (0.3-0.4 GB) exceed the 126 MB L2"},
+        "tokens_per_s": B * T / (ms * 1e-3),
+        "stack_tflop": flops / 1e12,
+        "roofline": {"bound": "tensor", "achieved": tf, "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
+                     "frac": tf / float(peaks["bf16_tflops"]), "traffic": None,
+                     "note": f"whole stack of public calls; peak = {peak_src} dense bf16 (burst)"},
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -638,10 +722,12 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--reference-budget-s", type=float, default=90.0)
-    ap.add_argument("--mode", choices=["forward", "decode", "backward", "forward_x"], default="forward",
+    ap.add_argument("--mode", choices=["forward", "decode", "backward", "forward_x", "sssl"], default="forward",
                     help="decode: time one KV-cache generation step; backward: time the layer's "
                          "gradient; forward_x: the layer from its input x (fused projection); "
-                         "default: the layer forward")
+                         "sssl: the 24-layer S,S,S,L stack at --sssl-T; default: the layer forward")
+    ap.add_argument("--sssl-T", type=int, default=2048, choices=[1024, 2048, 4096, 8192, 16384],
+                    help="sequence length of the SSSL stack (B = 32768 / T)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -654,6 +740,8 @@ def main(argv=None):
         return run_backward(args, s)
     if args.mode == "forward_x":
         return run_forward_x(args, s)
+    if args.mode == "sssl":
+        return run_sssl(args)
     if args.impl == "reference":
         return run_reference(args, s)
     return run_ours(args, s)

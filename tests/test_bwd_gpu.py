@@ -8,7 +8,9 @@ them, the gradient passed straight through the rounding.
 Tolerance, per gradient tensor, from the arithmetic of the kernels: P and dS enter the tensor-core
 products as bf16 (relative rounding 2^-9 per term), delta uses the bf16 output of the forward, and
 the big gradients are written as bf16 (2^-9); with fp32 accumulation this gives relative L2 errors
-of a few 1e-3.  The bar is relative L2 <= 2e-2 and max |error| <= 5e-2 max |reference|.
+of a few 1e-3.  Measured on B200: relative L2 2.2e-3 to 2.7e-3 for dq, dk, dv, dve and 1.5e-3
+for dgate_x and dWg; max |error| at most 4.7e-3 of the tensor's maximum.  The bar, about twice
+those, is relative L2 <= 6e-3 and max |error| <= 2e-2 max |reference|.
 """
 import numpy as np
 import pytest
@@ -20,8 +22,8 @@ import workloads
 
 pytestmark = pytest.mark.gpu
 
-REL_L2 = 2e-2
-MAX_REL = 5e-2
+REL_L2 = 6e-3
+MAX_REL = 2e-2
 
 
 @pytest.fixture(autouse=True)

@@ -37,13 +37,26 @@ def test_gpt2_124m_full():
 
 
 @pytest.mark.parametrize("s", [workloads.D24_S, workloads.D24_L_VE], ids=["d24_S", "d24_L_VE"])
-def test_d24_full_size_sampled_rows(s):
+def test_d24_full_size_every_element(s):
+    """The d24 layers at full size (16, 2048, 12, 128): every element of out and lse against the
+    oracle (a few seconds of the oracle on the host's cores)."""
+    err = parity.check_full(s)
+    print(f"{s.name}: {err}")
+
+
+@pytest.mark.parametrize("s", [workloads.TINY, workloads.GPT2, workloads.D24_S, workloads.D24_L_VE],
+                         ids=["tiny", "gpt2_124m", "d24_S", "d24_L_VE"])
+def test_named_workloads_against_pure_fp64_at_sampled_rows(s):
+    """Against the oracle's pure fp64 mode (no bf16 rounding of qhat, khat, v' anywhere), at edge
+    and random rows of several (b, h) slices: the output within the layer's bar, the LSE within the
+    pure-mode bar derived in tests/parity.py.  (The SSSL stack has the same check per layer.)"""
     d = workloads.make_layer(s)
     dev = parity.to_device(d)
     out, lse = parity.run_gpu(s, dev)
-    rows = workloads.sample_rows(s, n_random=6, seed=7,
-                                 bh_pairs=[(0, 0), (3, 5), (7, 11), (15, 0), (15, 11), (9, 6)])
-    parity.check_rows(s, d, out, lse, rows)
+    pairs = [(0, 0), (s.B - 1, s.H - 1), (s.B // 2, s.H // 2)]
+    rows = workloads.sample_rows(s, n_random=8, seed=17, bh_pairs=pairs)
+    err = parity.check_rows(s, d, out, lse, rows, pure=True)
+    print(f"{s.name} vs pure fp64: {err}")
 
 
 # ---------------------------------------------------- full compare on mid-size shapes
