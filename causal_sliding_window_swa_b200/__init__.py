@@ -58,6 +58,10 @@ def _load() -> ctypes.CDLL:
     lib.swa_attn_prologue.restype = I
     lib.swa_attn_attention.argtypes = [P, I, P, P, I, I, I, I, I, P, Z, P]
     lib.swa_attn_attention.restype = I
+    lib.swa_attn_prologue_fast.argtypes = [P, P, P, P, P, P, I, I, I, I, F, F, P, Z, P]
+    lib.swa_attn_prologue_fast.restype = I
+    lib.swa_attn_attention_q.argtypes = [P, P, I, P, P, I, I, I, I, I, F, P, Z, P]
+    lib.swa_attn_attention_q.restype = I
     lib.swa_attn_strerror.argtypes = [I]
     lib.swa_attn_strerror.restype = ctypes.c_char_p
     lib.swa_attn_last_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
@@ -157,6 +161,17 @@ def swa_attn_prologue(q, k, v, ve, gate_x, Wg, B, T, H, D, rope_base, eps, works
 
 def swa_attn_attention(v, has_ve, out, lse, B, T, H, D, window, workspace, ws_bytes, stream) -> int:
     return _lib.swa_attn_attention(v, int(has_ve), out, lse, B, T, H, D, window, workspace, ws_bytes, stream)
+
+
+def swa_attn_prologue_fast(q, k, v, ve, gate_x, Wg, B, T, H, D, rope_base, eps, workspace, ws_bytes,
+                           stream) -> int:
+    return _lib.swa_attn_prologue_fast(q, k, v, ve, gate_x, Wg, B, T, H, D, rope_base, eps, workspace,
+                                       ws_bytes, stream)
+
+
+def swa_attn_attention_q(q, v, has_ve, out, lse, B, T, H, D, window, eps, workspace, ws_bytes, stream) -> int:
+    return _lib.swa_attn_attention_q(q, v, int(has_ve), out, lse, B, T, H, D, window, eps, workspace, ws_bytes,
+                                     stream)
 
 
 def swa_attn_strerror(status: int) -> str:
@@ -438,7 +453,8 @@ def check_device_status(stream=None) -> None:
 __all__ = [
     "forward", "decode", "backward", "qkv_prologue", "forward_x", "check_device_status", "SwaError", "LIB_PATH", "load",
     "swa_attn_fwd", "swa_attn_fwd_ws", "swa_attn_fwd_noalloc", "swa_attn_noalloc_scratch_bytes", "swa_attn_workspace_bytes", "swa_attn_workspace_offset", "swa_attn_rope_table", "swa_attn_prologue",
-    "swa_attn_attention", "swa_attn_strerror", "swa_attn_last_device_status",
+    "swa_attn_attention", "swa_attn_prologue_fast", "swa_attn_attention_q", "swa_attn_strerror",
+    "swa_attn_last_device_status",
     "swa_attn_set_wait_limit_ms", "swa_attn_selftest_wait", "swa_attn_version",
     "swa_attn_decode", "swa_attn_decode_workspace_bytes", "swa_attn_fwd_gqa",
     "swa_attn_bwd", "swa_attn_bwd_gqa", "swa_attn_bwd_workspace_bytes",

@@ -39,6 +39,16 @@
 // the unrounded sum.  P is rounded to bf16 toward zero (one byte-permute per pair); because the
 // normaliser is the sum of the same rounded values, the rounding bias cancels in the weights.
 // One exponential in four is evaluated by a polynomial on the FMA pipe to offload the MUFU unit.
+//
+// Query prologue inside the kernel (QPRO).  With QPRO the producer loads the RAW query tile and the
+// softmax warps apply RoPE + RMS to it in shared memory (rope_fast.cuh, thread (row r, quarter c)
+// owning the rotation pairs of quarter c of row r; the four partial sums of squares of a row meet in
+// shared memory) before the MMA thread copies it into tensor memory, so qhat never goes through
+// HBM.  The softmax warps transform the next item's tile right after the last softmax tile of the
+// current item, while the tensor pipe runs that item's last PV product, and write the current
+// item's output afterwards; the next item's first score product then follows the PV product on the
+// pipe without a gap.  Without QPRO the query tile in HBM is already normalised (the fused
+// projection path and the staged entry point).
 #pragma once
 
 #include <cuda.h>
@@ -46,6 +56,7 @@
 #include <cstdint>
 
 #include "ptx.cuh"
+#include "rope_fast.cuh"
 
 namespace swa {
 
@@ -63,9 +74,10 @@ struct FwdCfg {
     static constexpr int SMEM_OUT = TILE_BYTES;        // output tile staged for the TMA store
     static constexpr int SMEM_BAR = 512;
     static constexpr int SMEM_LX = 4 * 128 * 8;        // row-sum exchange between the four threads of a row
+    static constexpr int SMEM_QX = 2 * 4 * 128 * 4;    // query sums of squares, double-buffered by item
     // Dynamic shared memory is declared 1024-byte aligned (the 128-byte swizzle atom repeats every
     // 1024 bytes); the kernel checks the alignment on entry instead of reserving slack for it.
-    static constexpr int SMEM_TOTAL = SMEM_Q + SMEM_KV + SMEM_OUT + SMEM_BAR + SMEM_LX;
+    static constexpr int SMEM_TOTAL = SMEM_Q + SMEM_KV + SMEM_OUT + SMEM_BAR + SMEM_LX + SMEM_QX;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_O = NSB * 128;
     static constexpr uint32_t COL_Q = COL_O + D;       // Q as bf16 pairs: D / 2 columns
@@ -87,13 +99,16 @@ struct FwdParams {
     float* lse;            // (B,H,T) or null
     int* sched;            // [0] next item, [1] CTAs done; zero before the launch, reset after
     unsigned long long wait_limit_ns;
+    const float2* tabf;    // fp32 RoPE table (cos, sin) per (t, i) (QPRO)
+    float inv_d;           // 1 / D (QPRO)
+    float eps;             // RMS epsilon (QPRO)
 };
 
 // Wait sites recorded in the status word on timeout.
 enum : unsigned int {
     kSiteQFull = 1, kSiteKvEmpty = 2, kSiteKvFull = 3, kSiteSFull = 4, kSitePFull = 5,
     kSiteOFull = 6, kSiteDrain = 7, kSiteQEmpty = 8, kSiteOEmpty = 9, kSiteItem = 10,
-    kSiteRowSum = 11, kSiteOStage = 12
+    kSiteRowSum = 11, kSiteOStage = 12, kSiteQSum = 13, kSiteQReady = 14
 };
 
 // Decoded work item: query tile [q0, q0 + 127] of (b, h) and the key tiles lo..hi of its band.
@@ -190,7 +205,7 @@ __device__ __forceinline__ uint32_t softmax_pair_poly(uint32_t s0, uint32_t s1, 
     return w;
 }
 
-template <int D>
+template <int D, bool QPRO>
 __global__ void __launch_bounds__(576, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -221,9 +236,13 @@ __global__ void __launch_bounds__(576, 1)
     uint64_t* b_pfull = bars + 13 + C::NSB;      // [NSB]
     uint64_t* b_kvfull = bars + 13 + 2 * C::NSB;            // [NS]
     uint64_t* b_kvempty = bars + 13 + 2 * C::NSB + C::NS;   // [NS]
-    int* s_item = reinterpret_cast<int*>(bars + 13 + 2 * C::NSB + 2 * C::NS);   // [2]
+    uint64_t* b_qss = bars + 13 + 2 * C::NSB + 2 * C::NS;        // query partial sums posted (QPRO)
+    uint64_t* b_qready = b_qss + 1;                               // query tile normalised (QPRO)
+    int* s_item = reinterpret_cast<int*>(b_qready + 1);           // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_item + 2);
     float2* s_lx = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(bars) + C::SMEM_BAR);   // [4][128]
+    float* s_qx = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(s_lx) + C::SMEM_LX);    // [2][4][128]
+    static_assert(13 + 2 * C::NSB + 2 * C::NS + 2 <= (C::SMEM_BAR - 16) / 8, "barrier area");
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -256,6 +275,8 @@ __global__ void __launch_bounds__(576, 1)
             mbar_init(smem_u32(b_kvfull + s), 1);
             mbar_init(smem_u32(b_kvempty + s), 1);
         }
+        mbar_init(smem_u32(b_qss), C::SOFTMAX_THREADS);
+        mbar_init(smem_u32(b_qready), C::SOFTMAX_THREADS);
         fence_barrier_init();
     }
     if (warp == kMmaWarp) {
@@ -409,7 +430,14 @@ __global__ void __launch_bounds__(576, 1)
                 const Item m = decode_item(p, it);
                 // Q into tensor memory (after the previous item's score products on the same pipe),
                 // then its shared-memory buffer goes back to the producer.
-                if (!(ok = mbar_wait(smem_u32(b_qfull), uses & 1u, lim, kSiteQFull))) break;
+                if (QPRO) {
+                    // the softmax warps wrote the normalised tile (generic proxy, fenced to the async
+                    // proxy before their arrive)
+                    if (!(ok = mbar_wait(smem_u32(b_qready), uses & 1u, lim, kSiteQReady))) break;
+                    tc_fence_after();
+                } else {
+                    if (!(ok = mbar_wait(smem_u32(b_qfull), uses & 1u, lim, kSiteQFull))) break;
+                }
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     tmem_cp_128x256b(tmem + C::COL_Q + 8u * kk,
@@ -443,17 +471,72 @@ __global__ void __launch_bounds__(576, 1)
         // one thread issues the output tile's TMA store
         const bool is_store = (warp == kSoftmaxWarp0 && lane == 0);
         bool ok = true;
-        for (uint32_t k = 0; ok; ++k) {
-            const uint32_t slot = k & 1u;
-            int it = 0;
+
+        // The k-th item from the scheduler's slots (k & 1); -1 when none is left.
+        auto fetch = [&](uint32_t kk) -> int {
+            const uint32_t slot = kk & 1u;
+            int v = 0;
+            bool w = true;
             if (lane == 0) {
-                ok = mbar_wait(smem_u32(b_itfull + slot), (k >> 1) & 1u, lim, kSiteItem);
-                it = s_item[slot];
+                w = mbar_wait(smem_u32(b_itfull + slot), (kk >> 1) & 1u, lim, kSiteItem);
+                v = s_item[slot];
                 mbar_arrive(smem_u32(b_itempty + slot));
             }
-            ok = __all_sync(0xffffffffu, ok);
-            it = __shfl_sync(0xffffffffu, it, 0);
-            if (!ok || it < 0) break;
+            const bool all = __all_sync(0xffffffffu, w);
+            ok = ok && all;
+            v = __shfl_sync(0xffffffffu, v, 0);
+            return ok ? v : -1;
+        };
+
+        // RoPE + RMS of the k-th item's raw query tile in shared memory (QPRO).  This thread: row r,
+        // rotation pairs [cq QP, cq QP + QP), i.e. the QP elements from column cq QP and the QP
+        // elements from column D/2 + cq QP, in the tile's 128-byte-swizzled layout.
+        auto q_transform = [&](const Item& mq, uint32_t kk) -> bool {
+            constexpr int QP = D / 8;
+            constexpr int NW = QP / 8;                  // 16-byte words per half (2 or 1)
+            const int t = min(mq.q0 + r, p.T - 1);      // rows past T hold zeros; any table row does
+            float4 cs[QP / 2];
+            const float4* tp = reinterpret_cast<const float4*>(p.tabf + (long long)t * (D / 2) + cq * QP);
+#pragma unroll
+            for (int e = 0; e < QP / 2; ++e) cs[e] = __ldg(tp + e);
+            uint32_t offa[NW], offb[NW];
+#pragma unroll
+            for (int e = 0; e < NW; ++e) {
+                // element column -> (128-byte chunk, 16-byte unit)
+                const int ca = cq * QP + 8 * e, cb = D / 2 + cq * QP + 8 * e;
+                offa[e] = (uint32_t)((ca >> 6) * C::CHUNK_BYTES + r * 128 + ((((ca & 63) >> 3) ^ (r & 7)) << 4));
+                offb[e] = (uint32_t)((cb >> 6) * C::CHUNK_BYTES + r * 128 + ((((cb & 63) >> 3) ^ (r & 7)) << 4));
+            }
+            bool w = mbar_wait(smem_u32(b_qfull), kk & 1u, lim, kSiteQFull);
+            if (!__all_sync(0xffffffffu, w)) return false;
+            uint4 qa[NW], qb[NW];
+#pragma unroll
+            for (int e = 0; e < NW; ++e) {
+                qa[e] = *reinterpret_cast<const uint4*>(sQ + offa[e]);
+                qb[e] = *reinterpret_cast<const uint4*>(sQ + offb[e]);
+            }
+            float* xs = s_qx + (kk & 1u) * 512u;
+            xs[cq * 128 + r] = quarter_sumsq<NW>(qa, qb);
+            mbar_arrive(smem_u32(b_qss));
+            w = mbar_wait(smem_u32(b_qss), kk & 1u, lim, kSiteQSum);
+            if (!__all_sync(0xffffffffu, w)) return false;
+            const float rs = rms_scale4(xs[r], xs[128 + r], xs[256 + r], xs[384 + r], p.inv_d, p.eps);
+            uint4 oa[NW], ob[NW];
+            rope_quarter<NW>(qa, qb, cs, rs, oa, ob);
+#pragma unroll
+            for (int e = 0; e < NW; ++e) {
+                *reinterpret_cast<uint4*>(sQ + offa[e]) = oa[e];
+                *reinterpret_cast<uint4*>(sQ + offb[e]) = ob[e];
+            }
+            fence_proxy_async_smem();                   // the tensor core reads the tile next
+            mbar_arrive(smem_u32(b_qready));
+            return true;
+        };
+
+        uint32_t k = 0;
+        int it = fetch(0);
+        if (QPRO && it >= 0) ok = q_transform(decode_item(p, it), 0);
+        while (ok && it >= 0) {
             const Item m = decode_item(p, it);
             const int qi = m.q0 + r;              // this thread's query position
             uint64_t l2[4], lr2[4];
@@ -507,6 +590,21 @@ __global__ void __launch_bounds__(576, 1)
                 mbar_arrive(smem_u32(b_pfull + buf));
             }
             if (!ok) break;
+            // This thread's partial row sums (few registers stay live across the next step).
+            float l = 0.f, lr = 0.f;
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                float u0, u1, w0, w1;
+                f2_unpack(l2[a], u0, u1);
+                f2_unpack(lr2[a], w0, w1);
+                l += u0 + u1;
+                lr += w0 + w1;
+            }
+            // The next item's query tile, while the tensor pipe runs this item's last PV product.
+            ++k;
+            const int it_next = fetch(k);
+            if (QPRO && ok && it_next >= 0) ok = q_transform(decode_item(p, it_next), k);
+            if (!ok) break;
             {
                 const bool w = mbar_wait(smem_u32(b_ofull), o_uses & 1u, lim, kSiteOFull);
                 ok = __all_sync(0xffffffffu, w);
@@ -529,15 +627,6 @@ __global__ void __launch_bounds__(576, 1)
             ++o_uses;
             // Row sums: columns 1-3 post their partial sums, column 0 adds them and posts the
             // totals; two mbarriers with bounded waits order the exchange.
-            float l = 0.f, lr = 0.f;
-#pragma unroll
-            for (int a = 0; a < 4; ++a) {
-                float u0, u1, w0, w1;
-                f2_unpack(l2[a], u0, u1);
-                f2_unpack(lr2[a], w0, w1);
-                l += u0 + u1;
-                lr += w0 + w1;
-            }
             const uint32_t xpar = (o_uses - 1u) & 1u;
             if (cq != 0) {
                 s_lx[cq * 128 + r] = make_float2(l, lr);
@@ -598,7 +687,7 @@ __global__ void __launch_bounds__(576, 1)
             if (qi < p.T && cq == 0 && p.lse != nullptr)
                 p.lse[((long long)m.b * p.H + m.h) * p.T + qi] = p.m0 + logf(l);
             ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
+            it = it_next;
         }
     }
 

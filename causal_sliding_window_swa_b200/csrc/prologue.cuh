@@ -65,7 +65,8 @@ __global__ void gate_kernel(const __nv_bfloat16* __restrict__ gate_x, const __nv
 
 // RoPE tables, one entry per (t, i):
 //   tab32[t*D/2 + i] = (c_hi, c_lo, s_hi, s_lo) fp32, each piece with a 16-bit significand;
-//   tab64[t*D/2 + i] = (cos, sin) fp64, read only by the fp64 path.
+//   tab64[t*D/2 + i] = (cos, sin) fp64, read only by the fp64 path;
+//   tabf[t*D/2 + i]  = (cos, sin) rounded to fp32, for the fp32 prologue (rope_fast.cuh).
 __device__ __forceinline__ float round_sig16(double x) {
     // nearest float with at most 16 significant bits (8 low mantissa bits cleared)
     const float f = (float)x;
@@ -73,8 +74,8 @@ __device__ __forceinline__ float round_sig16(double x) {
     return __uint_as_float((u + 0x80u) & 0xffffff00u);
 }
 
-__global__ void rope_table_kernel(float4* __restrict__ tab32, double2* __restrict__ tab64, int T,
-                                  int D, double base) {
+__global__ void rope_table_kernel(float4* __restrict__ tab32, double2* __restrict__ tab64,
+                                  float2* __restrict__ tabf, int T, int D, double base) {
     const int half = D / 2;
     const long long n = (long long)T * half;
     for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
@@ -88,6 +89,7 @@ __global__ void rope_table_kernel(float4* __restrict__ tab32, double2* __restric
         const float c_lo = round_sig16(c - (double)c_hi), s_lo = round_sig16(s - (double)s_hi);
         tab32[idx] = make_float4(c_hi, c_lo, s_hi, s_lo);
         tab64[idx] = make_double2(c, s);
+        tabf[idx] = make_float2((float)c, (float)s);
     }
 }
 

@@ -18,6 +18,7 @@
 #include "decode.cuh"
 #include "prologue.cuh"
 #include "qkv_gemm.cuh"
+#include "rope_fast.cuh"
 
 // ------------------------------------------------------------------ failure-detection self-test
 
@@ -111,11 +112,12 @@ constexpr size_t kAlign = 1024;
 size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct WsLayout {
-    size_t qh, kh, vp, gate, tab32, tab64, sched, total;
+    size_t qh, kh, vp, gate, tab32, tab64, tabf, sched, total;
 };
 
 // qhat | khat | v' and gate (value-embedding layers only) | RoPE table fp32 pieces |
-// RoPE table fp64 | attention scheduler counters, each section 1024-byte aligned.
+// RoPE table fp64 | RoPE table fp32 (cos, sin) | attention scheduler counters, each section
+// 1024-byte aligned.
 WsLayout ws_layout(const Shape& s, bool has_ve) {
     WsLayout w{};
     const size_t tensor = round_up((size_t)s.n * 2);
@@ -127,7 +129,8 @@ WsLayout ws_layout(const Shape& s, bool has_ve) {
     w.gate = w.vp + (has_ve ? kv_tensor : 0);
     w.tab32 = w.gate + (has_ve ? round_up((size_t)s.B * s.T * s.Hkv * sizeof(float2)) : 0);
     w.tab64 = w.tab32 + round_up(pairs * sizeof(float4));
-    w.sched = w.tab64 + round_up(pairs * sizeof(double2));
+    w.tabf = w.tab64 + round_up(pairs * sizeof(double2));
+    w.sched = w.tabf + round_up(pairs * sizeof(float2));
     w.total = w.sched + kAlign;
     return w;
 }
@@ -173,9 +176,13 @@ int device_ready(int* dev_out) {
         }
         if (checked[dev] == 1) {
             const int smem_attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
-            if (cudaFuncSetAttribute(swa::attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            if (cudaFuncSetAttribute(swa::attn_fwd_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      swa::FwdCfg<64>::SMEM_TOTAL) != cudaSuccess ||
-                cudaFuncSetAttribute(swa::attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                cudaFuncSetAttribute(swa::attn_fwd_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     swa::FwdCfg<128>::SMEM_TOTAL) != cudaSuccess ||
+                cudaFuncSetAttribute(swa::attn_fwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     swa::FwdCfg<64>::SMEM_TOTAL) != cudaSuccess ||
+                cudaFuncSetAttribute(swa::attn_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      swa::FwdCfg<128>::SMEM_TOTAL) != cudaSuccess ||
                 cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<64>, (cudaFuncAttribute)smem_attr,
                                      swa::BwdCfg<64>::DQ_SMEM) != cudaSuccess ||
@@ -251,8 +258,8 @@ int launch_rope_table(uint8_t* ws, const WsLayout& L, const Shape& s, float rope
     const int threads = 256;
     const long long blocks = std::min<long long>((n + threads - 1) / threads, 148ll * 16);
     swa::rope_table_kernel<<<(unsigned)blocks, threads, 0, st>>>(
-        reinterpret_cast<float4*>(ws + L.tab32), reinterpret_cast<double2*>(ws + L.tab64), s.T, s.D,
-        (double)rope_base);
+        reinterpret_cast<float4*>(ws + L.tab32), reinterpret_cast<double2*>(ws + L.tab64),
+        reinterpret_cast<float2*>(ws + L.tabf), s.T, s.D, (double)rope_base);
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
@@ -326,12 +333,66 @@ int launch_prologue(const void* q, const void* k, const void* v, const void* ve,
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
-int launch_attention(int dev, const void* v, bool has_ve, void* out, float* lse, const Shape& s,
-                     int window, uint8_t* ws, const WsLayout& L, cudaStream_t st) {
+// The fp32 prologue (rope_fast.cuh): the gate on value-embedding layers, then one launch whose
+// blocks write qhat (when q is given), khat and v' (value-embedding layers) into the workspace.
+// It also zeroes the attention kernel's scheduler counters.
+int launch_prologue_fast(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                         const void* Wg, uint8_t* ws, const WsLayout& L, const Shape& s, float eps,
+                         cudaStream_t st) {
+    using bf = __nv_bfloat16;
+    const bool has_ve = ve != nullptr;
+    const int n_kv_rows = s.B * s.T * s.Hkv;
+    float2* gate = reinterpret_cast<float2*>(ws + L.gate);
+    if (has_ve) {
+        const int gblocks = (int)std::min<long long>(((long long)n_kv_rows + 255) / 256, 148ll * 8);
+        swa::gate_kernel<<<gblocks, 256, 0, st>>>(static_cast<const bf*>(gate_x), static_cast<const bf*>(Wg),
+                                                   gate, n_kv_rows, s.Hkv, make_fastdiv(s.Hkv), 32);
+    }
+    swa::FastProParams p{};
+    p.q = static_cast<const bf*>(q);
+    p.k = static_cast<const bf*>(k);
+    p.v = static_cast<const bf*>(v);
+    p.ve = static_cast<const bf*>(ve);
+    p.gate = gate;
+    p.qh = reinterpret_cast<bf*>(ws + L.qh);
+    p.kh = reinterpret_cast<bf*>(ws + L.kh);
+    p.vp = reinterpret_cast<bf*>(ws + L.vp);
+    p.tabf = reinterpret_cast<const float2*>(ws + L.tabf);
+    p.n_q = q ? s.B * s.T * s.H : 0;
+    p.n_k = n_kv_rows;
+    p.n_v = has_ve ? n_kv_rows : 0;
+    p.nb_q = (p.n_q + 63) / 64;
+    p.nb_k = (p.n_k + 63) / 64;
+    const long long nb_v = ((long long)p.n_v * s.D / 32 + 255) / 256;
+    p.H = s.H;
+    p.Hkv = s.Hkv;
+    p.T = s.T;
+    p.inv_d = 1.0f / (float)s.D;
+    p.eps = eps;
+    p.sched = reinterpret_cast<int*>(ws + L.sched);
+    const long long blocks = (long long)p.nb_q + p.nb_k + nb_v;
+    if (blocks >= (1ll << 31)) return SWA_ERR_UNSUPPORTED;
+    if (s.D == 128) {
+        if (has_ve) swa::prologue_fast_kernel<128, true><<<(unsigned)blocks, 256, 0, st>>>(p);
+        else swa::prologue_fast_kernel<128, false><<<(unsigned)blocks, 256, 0, st>>>(p);
+    } else {
+        if (has_ve) swa::prologue_fast_kernel<64, true><<<(unsigned)blocks, 256, 0, st>>>(p);
+        else swa::prologue_fast_kernel<64, false><<<(unsigned)blocks, 256, 0, st>>>(p);
+    }
+    return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+// The attention kernel.  q_raw non-null: the kernel reads the raw q (B,T,H,D) and applies RoPE + RMS
+// to each query tile itself (the fp32 prologue's arithmetic; the RoPE table must be in the
+// workspace); q_raw null: it reads qhat from the workspace.  khat (and v' on value-embedding
+// layers) always come from the workspace.
+int launch_attention(int dev, const void* q_raw, const void* v, bool has_ve, void* out, float* lse,
+                     const Shape& s, int window, float eps, uint8_t* ws, const WsLayout& L, cudaStream_t st) {
     CUtensorMap tq, tk, tv, to;
     const void* vsrc = has_ve ? static_cast<const void*>(ws + L.vp) : v;
+    const void* qsrc = q_raw ? q_raw : static_cast<const void*>(ws + L.qh);
     // q and out have H heads, k and v Hkv heads
-    if (!make_tile_map(&tq, ws + L.qh, s, s.H) || !make_tile_map(&tk, ws + L.kh, s, s.Hkv) ||
+    if (!make_tile_map(&tq, qsrc, s, s.H) || !make_tile_map(&tk, ws + L.kh, s, s.Hkv) ||
         !make_tile_map(&tv, vsrc, s, s.Hkv) || !make_tile_map(&to, out, s, s.H))
         return SWA_ERR_CUDA;
     swa::FwdParams p{};
@@ -354,11 +415,18 @@ int launch_attention(int dev, const void* v, bool has_ve, void* out, float* lse,
     p.lse = lse;
     p.sched = reinterpret_cast<int*>(ws + L.sched);
     p.wait_limit_ns = wait_limit_ns();
+    p.tabf = reinterpret_cast<const float2*>(ws + L.tabf);
+    p.inv_d = 1.0f / (float)s.D;
+    p.eps = eps;
     const dim3 grid((unsigned)std::min(p.n_items, g_num_sms[dev]));
-    if (s.D == 128)
-        swa::attn_fwd_kernel<128><<<grid, swa::FwdCfg<128>::THREADS, swa::FwdCfg<128>::SMEM_TOTAL, st>>>(tq, tk, tv, to, p);
-    else
-        swa::attn_fwd_kernel<64><<<grid, swa::FwdCfg<64>::THREADS, swa::FwdCfg<64>::SMEM_TOTAL, st>>>(tq, tk, tv, to, p);
+#define SWA_ATTN(DD, QP) \
+    swa::attn_fwd_kernel<DD, QP><<<grid, swa::FwdCfg<DD>::THREADS, swa::FwdCfg<DD>::SMEM_TOTAL, st>>>(tq, tk, tv, to, p)
+    if (s.D == 128) {
+        if (q_raw) SWA_ATTN(128, true); else SWA_ATTN(128, false);
+    } else {
+        if (q_raw) SWA_ATTN(64, true); else SWA_ATTN(64, false);
+    }
+#undef SWA_ATTN
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
@@ -497,9 +565,10 @@ int launch_backward(int dev, const void* q, const void* k, const void* v, const 
     using bf = __nv_bfloat16;
     const bool has_ve = ve != nullptr;
     int rc;
-    // qhat, khat, v' and the gate exactly as the forward computed them.
+    // qhat, khat, v' and the gate exactly as the forward computed them (the fp32 prologue's
+    // arithmetic, which the forward's attention kernel applies to the query tiles in place).
     if ((rc = launch_rope_table(ws, L.f, s, rope_base, st)) != SWA_OK) return rc;
-    if ((rc = launch_prologue(q, k, v, ve, gate_x, Wg, ws, L.f, s, eps, st)) != SWA_OK) return rc;
+    if ((rc = launch_prologue_fast(q, k, v, ve, gate_x, Wg, ws, L.f, s, eps, st)) != SWA_OK) return rc;
 
     int* sched4 = reinterpret_cast<int*>(ws + L.f.sched) + 4;
     float2* rowstat = reinterpret_cast<float2*>(ws + L.rowstat);
@@ -603,6 +672,8 @@ struct DevCache {
     int tab_T = -1, tab_D = -1;
     float tab_base = 0.f;
     size_t tab_off = (size_t)-1;
+    cudaEvent_t last_use = nullptr;       // recorded after the last call's launches
+    cudaStream_t last_stream = nullptr;   // the stream of that call
 };
 DevCache g_cache[64];
 
@@ -696,8 +767,8 @@ int swa_attn_attention(const void* v, int has_ve, void* out, float* lse, int B, 
     if (ws_bytes < L.total) return SWA_ERR_NO_MEMORY;
     int dev;
     if ((rc = device_ready(&dev)) != SWA_OK) return rc;
-    return launch_attention(dev, v, has_ve != 0, out, lse, s, window, static_cast<uint8_t*>(workspace), L,
-                            reinterpret_cast<cudaStream_t>(stream));
+    return launch_attention(dev, nullptr, v, has_ve != 0, out, lse, s, window, 0.f,
+                            static_cast<uint8_t*>(workspace), L, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int swa_attn_fwd_ws(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
@@ -711,11 +782,48 @@ int swa_attn_fwd_ws(const void* q, const void* k, const void* v, const void* ve,
     if (rc != SWA_OK) return rc;
     rc = swa_attn_rope_table(B, T, H, D, ve != nullptr, rope_base, workspace, ws_bytes, stream);
     if (rc != SWA_OK) return rc;
-    rc = swa_attn_prologue(q, k, v, ve, gate_x, Wg, B, T, H, D, rope_base, eps, workspace, ws_bytes,
-                           stream);
+    rc = swa_attn_prologue_fast(nullptr, k, v, ve, gate_x, Wg, B, T, H, D, rope_base, eps, workspace,
+                                ws_bytes, stream);
     if (rc != SWA_OK) return rc;
-    return swa_attn_attention(v, ve != nullptr, out, lse, B, T, H, D, window, workspace, ws_bytes,
-                              stream);
+    return swa_attn_attention_q(q, v, ve != nullptr, out, lse, B, T, H, D, window, eps, workspace,
+                                ws_bytes, stream);
+}
+
+int swa_attn_prologue_fast(const void* q, const void* k, const void* v, const void* ve,
+                           const void* gate_x, const void* Wg, int B, int T, int H, int D,
+                           float rope_base, float eps, void* workspace, size_t ws_bytes,
+                           swa_stream_t stream) {
+    Shape s;
+    int rc = check_sizes(B, T, H, D, &s);
+    // q may be null here (khat and v' only); the others follow the layer's rules
+    if (rc == SWA_OK) rc = check_layer_args(q ? q : k, k, v, ve, gate_x, Wg, rope_base, eps);
+    if (rc != SWA_OK) return rc;
+    if (!workspace) return SWA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return SWA_ERR_MISALIGNED;
+    const WsLayout L = ws_layout(s, ve != nullptr);
+    if (ws_bytes < L.total) return SWA_ERR_NO_MEMORY;
+    int dev;
+    if ((rc = device_ready(&dev)) != SWA_OK) return rc;
+    return launch_prologue_fast(q, k, v, ve, gate_x, Wg, static_cast<uint8_t*>(workspace), L, s, eps,
+                                reinterpret_cast<cudaStream_t>(stream));
+}
+
+int swa_attn_attention_q(const void* q, const void* v, int has_ve, void* out, float* lse, int B, int T,
+                         int H, int D, int window, float eps, void* workspace, size_t ws_bytes,
+                         swa_stream_t stream) {
+    Shape s;
+    int rc = check_sizes(B, T, H, D, &s);
+    if (rc != SWA_OK) return rc;
+    if (!q || !workspace || (!has_ve && !v)) return SWA_ERR_INVALID_ARG;
+    if (!std::isfinite(eps) || eps < 0.f) return SWA_ERR_INVALID_ARG;
+    if ((rc = check_outputs(out, lse)) != SWA_OK) return rc;
+    if (!aligned(q, 16) || !aligned(workspace, 16) || (!has_ve && !aligned(v, 16))) return SWA_ERR_MISALIGNED;
+    const WsLayout L = ws_layout(s, has_ve != 0);
+    if (ws_bytes < L.total) return SWA_ERR_NO_MEMORY;
+    int dev;
+    if ((rc = device_ready(&dev)) != SWA_OK) return rc;
+    return launch_attention(dev, q, v, has_ve != 0, out, lse, s, window, eps, static_cast<uint8_t*>(workspace),
+                            L, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int swa_attn_fwd_gqa(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
@@ -737,6 +845,20 @@ int swa_attn_fwd_gqa(const void* q, const void* k, const void* v, const void* ve
     (void)limit;
     std::lock_guard<std::mutex> lk(g_cache_mu);
     DevCache& c = g_cache[dev];
+    // The cached workspace (and its RoPE table) may still be in use by the previous call's kernels
+    // on another stream: this stream waits for them before it touches, reuses or frees it.
+    if (c.last_use != nullptr && c.last_stream != st) {
+        if (cudaStreamWaitEvent(st, c.last_use, 0) != cudaSuccess) {
+            cudaGetLastError();
+            return SWA_ERR_CUDA;
+        }
+    }
+    if (c.last_use == nullptr &&
+        cudaEventCreateWithFlags(&c.last_use, cudaEventDisableTiming) != cudaSuccess) {
+        cudaGetLastError();
+        c.last_use = nullptr;
+        return SWA_ERR_CUDA;
+    }
     if (c.bytes < L.total) {
         if (c.ptr) cudaFreeAsync(c.ptr, st);
         c.ptr = nullptr;
@@ -758,8 +880,15 @@ int swa_attn_fwd_gqa(const void* q, const void* k, const void* v, const void* ve
         c.tab_base = rope_base;
         c.tab_off = L.tab32;
     }
-    if ((rc = launch_prologue(q, k, v, ve, gate_x, Wg, ws, L, s, eps, st)) != SWA_OK) return rc;
-    return launch_attention(dev, v, has_ve, out, lse, s, window, ws, L, st);
+    rc = launch_prologue_fast(nullptr, k, v, ve, gate_x, Wg, ws, L, s, eps, st);
+    if (rc == SWA_OK) rc = launch_attention(dev, q, v, has_ve, out, lse, s, window, eps, ws, L, st);
+    // Recorded after whatever was enqueued, also on failure, so the next call orders after it.
+    if (cudaEventRecord(c.last_use, st) != cudaSuccess) {
+        cudaGetLastError();
+        if (rc == SWA_OK) rc = SWA_ERR_CUDA;
+    }
+    c.last_stream = st;
+    return rc;
 }
 
 int swa_attn_fwd(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
@@ -818,7 +947,7 @@ int swa_attn_fwd_x(const void* x, const void* Wqkv, const void* ve, const void* 
     if ((rc = launch_qkv(dev, x, Wqkv, ve, Wg, C, s, eps, ws, L, ws + L.qh, ws + L.kh, ws + L.vp,
                          reinterpret_cast<int*>(ws + L.sched), st)) != SWA_OK)
         return rc;
-    return launch_attention(dev, nullptr, true, out, lse, s, window, ws, L, st);
+    return launch_attention(dev, nullptr, nullptr, true, out, lse, s, window, 0.f, ws, L, st);
 }
 
 // ---------------------------------------------------------------------------- backward
@@ -1019,6 +1148,7 @@ void* g_static_ptr[64] = {nullptr};
 
 // Once per device, with that device current: the device address of the scratch array.
 int static_scratch(int dev, uint8_t** out) {
+    if (dev < 0 || dev >= 64) return SWA_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lk(g_static_mu);
     if (g_static_ptr[dev] == nullptr) {
         void* p = nullptr;
@@ -1053,9 +1183,10 @@ extern "C" int swa_attn_fwd_noalloc(const void* q, const void* k, const void* v,
     uint8_t* ws = nullptr;
     if ((rc = static_scratch(dev, &ws)) != SWA_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    // Every section of the scratch this call reads is written earlier in the same call
-    // (table, then qhat/khat/v'), so nothing needs clearing between calls.
+    // Every section of the scratch this call reads is written earlier in the same call (the RoPE
+    // tables, then khat / v' and the gate; the prologue also zeroes the attention kernel's
+    // scheduler counters), so nothing left by an earlier call is read.
     if ((rc = launch_rope_table(ws, L, s, rope_base, st)) != SWA_OK) return rc;
-    if ((rc = launch_prologue(q, k, v, ve, gate_x, Wg, ws, L, s, eps, st)) != SWA_OK) return rc;
-    return launch_attention(dev, v, has_ve, out, lse, s, window, ws, L, st);
+    if ((rc = launch_prologue_fast(nullptr, k, v, ve, gate_x, Wg, ws, L, s, eps, st)) != SWA_OK) return rc;
+    return launch_attention(dev, q, v, has_ve, out, lse, s, window, eps, ws, L, st);
 }

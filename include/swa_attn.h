@@ -31,6 +31,14 @@
  * Streams: calls are asynchronous on `stream` (NULL = the legacy default stream) and never
  * synchronise the host, except swa_attn_last_device_status().
  *
+ * Precision of the forward calls (swa_attn_fwd, _gqa, _ws, _noalloc): the prologue runs in fp32
+ * and rounds qhat, khat and v' to bf16 once (round to nearest even); each of those elements is the
+ * bf16 rounding of a value within a few fp32 ulps of its exact value, so it is the correctly
+ * rounded bf16 or, for elements that lie that close to a rounding midpoint, one bf16 ulp from it.
+ * The query prologue runs inside the attention kernel on each query tile (qhat never goes through
+ * HBM).  swa_attn_prologue() is the exactly rounded prologue (every element the correctly rounded
+ * bf16 of its exact value), used by the staged path and the decode step.
+ *
  * Errors: a negative swa_status.  Arguments are validated before anything is enqueued; a
  * rejected call has no effect.  Waits inside the kernels are bounded: if one expires, the
  * kernel records SWA_ERR_TIMEOUT in a per-device status word and exits cleanly; read it with
@@ -82,10 +90,13 @@ typedef enum swa_status {
  * eps          >= 0 and finite (1e-6 here).
  * stream       CUDA stream (NULL = legacy default stream).
  *
- * Scratch: the library keeps one workspace per device (qhat, khat, v' and the RoPE table),
+ * Scratch: the library keeps one workspace per device (khat, v', the gates and the RoPE table),
  * grown on demand with stream-ordered allocation on `stream` and kept until the library is
- * unloaded.  Calls that may overlap on different streams must use swa_attn_fwd_ws() with
- * separate workspaces.
+ * unloaded.  Each call records an event after its kernels; a call on another stream first makes
+ * its stream wait for that event, so calls on different streams that share the workspace run one
+ * after the other on the GPU (callers that want them to overlap use swa_attn_fwd_ws() with
+ * separate workspaces).  Launches: the gate kernel (value-embedding layers), the k / v prologue
+ * kernel and the attention kernel, plus the RoPE table when T, D or rope_base changes.
  */
 SWA_API int swa_attn_fwd(const void* q, const void* k, const void* v,
                  const void* ve, const void* gate_x, const void* Wg,
@@ -112,9 +123,11 @@ SWA_API size_t swa_attn_workspace_bytes(int B, int T, int H, int D, int has_ve);
 
 /*
  * Byte offset of one section of the workspace, for callers that read the prologue's results
- * (e.g. to keep them for a backward pass) after swa_attn_prologue():
- *   SWA_WS_QHAT, SWA_WS_KHAT   bf16 (B,T,H,D): rms(rope(q)), rms(rope(k)), each element the
- *                              correctly rounded bf16 (nearest, ties to even) of its exact value;
+ * (e.g. to keep them for a backward pass) after swa_attn_prologue() or swa_attn_prologue_fast():
+ *   SWA_WS_QHAT, SWA_WS_KHAT   bf16 (B,T,H,D): rms(rope(q)), rms(rope(k)); after
+ *                              swa_attn_prologue() each element is the correctly rounded bf16
+ *                              (nearest, ties to even) of its exact value, after
+ *                              swa_attn_prologue_fast() it is within one bf16 ulp of that;
  *   SWA_WS_VPRIME              bf16 (B,T,H,D): v + 2 sigmoid(gate_x . Wg) ve, same rounding
  *                              (value-embedding layers only);
  *   SWA_WS_ROPE_TABLE          the RoPE table (internal format).
@@ -125,8 +138,10 @@ SWA_API size_t swa_attn_workspace_offset(int B, int T, int H, int D, int has_ve,
 
 /*
  * Same as swa_attn_fwd() with caller-owned device scratch: `workspace` (16-byte aligned,
- * at least swa_attn_workspace_bytes() bytes) holds qhat, khat, v' and the RoPE table, which
- * is rebuilt on every call (one small extra kernel).  Nothing is allocated.  SWA_ERR_NO_MEMORY if ws_bytes is too small.
+ * at least swa_attn_workspace_bytes() bytes) holds khat, v', the gates and the RoPE table, which
+ * is rebuilt on every call (one small extra kernel).  It runs swa_attn_rope_table(),
+ * swa_attn_prologue_fast() with q = NULL and swa_attn_attention_q().  Nothing is allocated.
+ * SWA_ERR_NO_MEMORY if ws_bytes is too small.
  */
 SWA_API int swa_attn_fwd_ws(const void* q, const void* k, const void* v,
                     const void* ve, const void* gate_x, const void* Wg,
@@ -145,8 +160,18 @@ SWA_API int swa_attn_fwd_ws(const void* q, const void* k, const void* v,
  * swa_attn_prologue: RoPE + RMS norm of q and k, gate + add of the value embedding, into the
  *   workspace (same sizes and rules as swa_attn_fwd_ws).  Uses the table already in the
  *   workspace; it does not rebuild it.
- * swa_attn_attention: the windowed attention on a workspace that swa_attn_prologue() filled
- *   for the same B, T, H, D and value-embedding setting (`v` is read directly when has_ve == 0).
+ * swa_attn_attention: the windowed attention on a workspace that swa_attn_prologue() (or
+ *   swa_attn_prologue_fast() with q) filled for the same B, T, H, D and value-embedding setting
+ *   (`v` is read directly when has_ve == 0).
+ * swa_attn_prologue_fast: the forward's fp32 prologue (precision: see the top of this file) into
+ *   the workspace: khat, and v' with its gate on value-embedding layers; qhat too when q is not
+ *   NULL (q = NULL is the forward's key/value pass).  Needs the RoPE table in the workspace.  It
+ *   also resets the scheduler counters that the attention kernels take their work from.
+ * swa_attn_attention_q: the windowed attention reading the RAW q (B,T,H,D) and applying RoPE + RMS
+ *   (eps as for the prologue) to each query tile inside the kernel, with khat (and v') from a
+ *   workspace that swa_attn_prologue_fast() filled; its qhat equals, bit for bit, the one
+ *   swa_attn_prologue_fast() writes for the same q.
+ * All of them: asynchronous on `stream`, validation before any launch, errors as swa_attn_fwd_ws.
  */
 SWA_API int swa_attn_rope_table(int B, int T, int H, int D, int has_ve, float rope_base,
                                 void* workspace, size_t ws_bytes, swa_stream_t stream);
@@ -160,20 +185,33 @@ SWA_API int swa_attn_attention(const void* v, int has_ve, void* out, float* lse,
                        int B, int T, int H, int D, int window,
                        void* workspace, size_t ws_bytes, swa_stream_t stream);
 
+SWA_API int swa_attn_prologue_fast(const void* q, const void* k, const void* v,
+                                   const void* ve, const void* gate_x, const void* Wg,
+                                   int B, int T, int H, int D, float rope_base, float eps,
+                                   void* workspace, size_t ws_bytes, swa_stream_t stream);
+
+SWA_API int swa_attn_attention_q(const void* q, const void* v, int has_ve, void* out, float* lse,
+                                 int B, int T, int H, int D, int window, float eps,
+                                 void* workspace, size_t ws_bytes, swa_stream_t stream);
+
 /*
  * swa_attn_fwd_noalloc: swa_attn_fwd() for callers that cannot allocate device memory on the
  * call path -- a plugin whose host framework owns all device memory and forbids allocation
  * inside its execute call, or a latency-critical loop where an allocation (which may
  * synchronise the device) is not allowed.  The pages have no counterpart of this entry point.
  *
- * The caller passes inputs and outputs exactly as for swa_attn_fwd(); the scratch (qhat, khat,
- * v' and the RoPE table) lives in a fixed device array compiled into the library,
- * swa_attn_noalloc_scratch_bytes() bytes (64 MiB), which every GPU that loads the library holds
- * until the process exits.  Nothing is allocated or freed by the call.
+ * The caller passes inputs and outputs exactly as for swa_attn_fwd(), and the call computes the
+ * same result with the same kernels; the scratch (khat, v', the gates and the RoPE table) lives in
+ * a fixed device array compiled into the library, swa_attn_noalloc_scratch_bytes() bytes (64 MiB).
+ * Nothing is allocated or freed by the call itself.
+ *   - CUDA loads the library's device code, and with it the array, on a device when the library
+ *     is first used there (lazy module loading): from then on that device holds the 64 MiB until
+ *     the process exits, and that first use may itself allocate.  The first call of
+ *     swa_attn_fwd_noalloc() on a device also looks up the array's device address (a runtime query,
+ *     once per device, with that device current).  Callers that must not allocate make one warm-up
+ *     call on each device outside their no-allocation region and before any stream capture.
  *   - Sizes whose workspace (swa_attn_workspace_bytes()) exceeds that array are rejected with
  *     SWA_ERR_NO_MEMORY before anything is enqueued.
- *   - The first call on a device looks up the array's device address (a runtime query, once per
- *     device, with that device current); make that first call before any stream capture.
  *   - All calls on a device share the one array and it keeps the last call's contents; every
  *     byte a call reads is written earlier in that call.  Calls that overlap on the GPU (other
  *     streams, other host threads) race on it: serialise them.

@@ -11,7 +11,11 @@ moves that score, and so the LSE of a row that sees few keys: for unit-RMS opera
 rounding errors (uniform, up to 2^-9 relative) give the score a standard deviation of
 2^-9 sqrt(2/3) ~ 1.6e-3; the oracle's own parity and pure modes differ by up to 6e-3 at row 0 of
 the d24 layers.  The pure-mode LSE bar is therefore 1.5e-2 (about nine standard deviations of
-that single-score deviation), stated here and asserted alongside the 1e-3 parity-mode bar."""
+that single-score deviation), stated here and asserted alongside the 1e-3 parity-mode bar.  The
+same rounding of v' (half a bf16 ulp, 2^-9 relative, on values up to |v + 2 ve| ~ 5 here) can move
+an output that one key dominates by about 1e-2 on its own, so the pure-mode max-abs bar is 3e-2
+(the parity bar plus that term); the relative L2 bar stays 5e-3.  Measured worst cases against pure
+fp64: max-abs 0.025, relative L2 3.2e-3, LSE 8.1e-3 (the SSSL stack)."""
 from __future__ import annotations
 
 from typing import Dict, Optional
@@ -26,6 +30,7 @@ OUT_MAX_ABS = 2e-2
 OUT_REL_L2 = 5e-3
 LSE_MAX_ABS = 1e-3
 LSE_MAX_ABS_PURE = 1.5e-2
+OUT_MAX_ABS_PURE = 3e-2
 
 
 def to_device(d: Dict[str, torch.Tensor], device="cuda"):
@@ -48,7 +53,7 @@ def run_gpu(s: workloads.LayerShape, dev: Dict, *, nan_fill=True, window=None, *
 
 
 def compare(out_gpu: np.ndarray, lse_gpu: np.ndarray, out_ref: np.ndarray, lse_ref: np.ndarray,
-            what: str = "", lse_tol: float = LSE_MAX_ABS):
+            what: str = "", lse_tol: float = LSE_MAX_ABS, max_abs_tol: float = OUT_MAX_ABS):
     assert np.isfinite(out_gpu).all(), f"{what}: non-finite output (unwritten element?)"
     assert np.isfinite(lse_gpu).all(), f"{what}: non-finite lse (unwritten element?)"
     err = np.abs(out_gpu - out_ref)
@@ -56,7 +61,7 @@ def compare(out_gpu: np.ndarray, lse_gpu: np.ndarray, out_ref: np.ndarray, lse_r
     rel_l2 = float(np.linalg.norm(out_gpu - out_ref) / max(np.linalg.norm(out_ref), 1e-30))
     lse_err = float(np.abs(lse_gpu - lse_ref).max()) if lse_ref.size else 0.0
     msg = f"{what}: max_abs={max_abs:.3e} rel_l2={rel_l2:.3e} lse_max_abs={lse_err:.3e}"
-    assert max_abs <= OUT_MAX_ABS, msg
+    assert max_abs <= max_abs_tol, msg
     assert rel_l2 <= OUT_REL_L2, msg
     assert lse_err <= lse_tol, msg
     return dict(max_abs=max_abs, rel_l2=rel_l2, lse_max_abs=lse_err)
@@ -83,4 +88,27 @@ def check_rows(s: workloads.LayerShape, d: Dict, out: torch.Tensor, lse: torch.T
     l = lse[b.cuda(), h.cuda(), i.cuda()].cpu().numpy()
     assert torch.isfinite(out).all().item() and torch.isfinite(lse).all().item(), f"{s.name}: non-finite"
     return compare(o, l, ref_o, ref_l, s.name + (" (sampled rows, pure fp64)" if pure else " (sampled rows)"),
-                   lse_tol=LSE_MAX_ABS_PURE if pure else LSE_MAX_ABS)
+                   lse_tol=LSE_MAX_ABS_PURE if pure else LSE_MAX_ABS,
+                   max_abs_tol=OUT_MAX_ABS_PURE if pure else OUT_MAX_ABS)
+
+
+def bf16_ulp_keys(a_bf16: torch.Tensor) -> np.ndarray:
+    """Signed integer keys of bf16 values, consecutive for neighbouring representable values
+    (+0 and -0 share key 0)."""
+    u = a_bf16.contiguous().view(torch.int16).cpu().numpy().astype(np.int32) & 0xFFFF
+    mag = u & 0x7FFF
+    return np.where(u & 0x8000, -mag, mag)
+
+
+def ulp_compare(got: torch.Tensor, ref: np.ndarray, what: str, max_fraction: float):
+    """got (bf16) against the oracle's bf16-valued ref (parity mode): every element within one bf16
+    ulp, and the fraction of one-ulp differences at most max_fraction.  Returns that count."""
+    ref_bf = torch.from_numpy(np.ascontiguousarray(ref)).to(torch.bfloat16)
+    assert np.array_equal(ref_bf.double().numpy(), ref), f"{what}: oracle output not bf16-valued"
+    dist = np.abs(bf16_ulp_keys(got.cpu()).reshape(-1) - bf16_ulp_keys(ref_bf).reshape(-1))
+    n_diff = int((dist > 0).sum())
+    frac = n_diff / max(1, dist.size)
+    print(f"{what}: {n_diff} of {dist.size} elements differ by one bf16 ulp ({frac:.2e}), max {int(dist.max())}")
+    assert int(dist.max()) <= 1, f"{what}: an element is {int(dist.max())} bf16 ulps from the oracle"
+    assert frac <= max_fraction, f"{what}: {frac:.2e} of the elements differ by one ulp"
+    return n_diff

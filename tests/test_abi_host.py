@@ -99,6 +99,22 @@ def test_stage_entry_points_reject_bad_arguments():
     assert swa.swa_attn_attention(None, 0, A, A, 1, 16, 1, 64, 0, A, need, None) == swa.SWA_ERR_INVALID_ARG
     assert swa.swa_attn_attention(A, 0, A, A, 1, 16, 1, 64, 0, A, need - 1, None) == swa.SWA_ERR_NO_MEMORY
     assert swa.swa_attn_attention(A, 0, A, A, 1, 16, 1, 80, 0, A, need, None) == swa.SWA_ERR_UNSUPPORTED
+    # the fp32 prologue: q may be NULL (key/value pass), k may not
+    assert swa.swa_attn_prologue_fast(None, A, A, None, None, None, 1, 16, 1, 64, 1e4, 1e-6, A, need - 1, None) \
+        == swa.SWA_ERR_NO_MEMORY
+    assert swa.swa_attn_prologue_fast(None, None, A, None, None, None, 1, 16, 1, 64, 1e4, 1e-6, A, need, None) \
+        == swa.SWA_ERR_INVALID_ARG
+    assert swa.swa_attn_prologue_fast(A + 2, A, A, None, None, None, 1, 16, 1, 64, 1e4, 1e-6, A, need, None) \
+        == swa.SWA_ERR_MISALIGNED
+    assert swa.swa_attn_prologue_fast(None, A, A, A, None, None, 1, 16, 1, 64, 1e4, 1e-6, A, need, None) \
+        == swa.SWA_ERR_INVALID_ARG
+    # the attention from the raw q
+    assert swa.swa_attn_attention_q(None, A, 0, A, A, 1, 16, 1, 64, 0, 1e-6, A, need, None) == swa.SWA_ERR_INVALID_ARG
+    assert swa.swa_attn_attention_q(A, A, 0, A, A, 1, 16, 1, 64, 0, 1e-6, A, need - 1, None) == swa.SWA_ERR_NO_MEMORY
+    assert swa.swa_attn_attention_q(A + 8, A, 0, A, A, 1, 16, 1, 64, 0, 1e-6, A, need, None) == swa.SWA_ERR_MISALIGNED
+    assert swa.swa_attn_attention_q(A, A, 0, A, A, 1, 16, 1, 64, 0, -1.0, A, need, None) == swa.SWA_ERR_INVALID_ARG
+    assert swa.swa_attn_attention_q(A, A, 0, A, A, 1, 16, 1, 128 + 64, 0, 1e-6, A, need, None) \
+        == swa.SWA_ERR_UNSUPPORTED
 
 
 def test_wait_limit_setter():

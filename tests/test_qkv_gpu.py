@@ -2,12 +2,16 @@
 run from its input x (swa_attn_fwd_x), through the C ABI, against the fp64 oracle.
 
 What is compared:
-  * qhat, khat, v' element by element with ``oracle.qkv_prologue(parity=True)``: the projection
-    x Wqkv^T summed in fp64, RoPE, RMS and the gated value embedding, rounded once to bf16.  The
-    kernel keeps the projection in an fp32 tensor-memory accumulator, so an element whose exact
-    value lies within the accumulator's rounding error of a bf16 rounding midpoint may round the
-    other way: every element must be within one bf16 ulp, and such one-ulp differences must stay
-    rare (the count is reported).
+  * qhat, khat, v' element by element with the oracle (``oracle.qkv_prologue``): the projection
+    x Wqkv^T summed in fp64, RoPE, RMS and the gated value embedding.  The kernel keeps the
+    projection in an fp32 tensor-memory accumulator, so its q, k, v carry the accumulation error
+    of a C-term fp32 sum, |dy| <= C 2^-23 sum_c |x_c W_c| (the textbook bound for any summation
+    order, with a factor 2 to spare); an output near zero can therefore be several bf16 ulps of
+    itself away while being only a tiny absolute distance from the exact value.  The check is that
+    bound carried through the prologue: every element within half a bf16 ulp of the exact value
+    (the oracle's pure mode) plus r (|dy_a| + |dy_b|) + |qhat| sum|y||dy| / (ss + D eps) plus a few
+    fp32 roundings for q / k heads, and plus |dy| for v heads; the elements that differ from the
+    correctly rounded value (the oracle's parity mode) are counted and must stay rare.
   * out and lse of ``swa_attn_fwd_x`` against the oracle's attention on the oracle's own rounded
     qhat, khat, v' (its prologue switched off by the test-only flags), at the forward tolerances
     (max-abs 2e-2, relative L2 5e-3, LSE 1e-3).
@@ -31,7 +35,7 @@ pytestmark = pytest.mark.gpu
 
 swa = pytest.importorskip("causal_sliding_window_swa_b200")
 
-ULP_MISMATCH_MAX_FRACTION = 5e-3
+MISMATCH_MAX_FRACTION = 5e-3
 
 
 @pytest.fixture(autouse=True)
@@ -55,24 +59,44 @@ def _draw(B, T, C, H, Hkv, D, ve, seed, vocab=997):
     return d
 
 
-def _ulp_keys(a_bf16: torch.Tensor) -> np.ndarray:
-    """Signed integer keys of bf16 values, consecutive for neighbouring representable values
-    (+0 and -0 share key 0)."""
-    u = a_bf16.view(torch.int16).cpu().numpy().astype(np.int32) & 0xFFFF
-    mag = u & 0x7FFF
-    return np.where(u & 0x8000, -mag, mag)
+def _check_bound(got, exact, rounded, bound, what):
+    """|got - exact| <= half a bf16 ulp of got + bound, elementwise; differences from the correctly
+    rounded value counted (and rare)."""
+    g = got.double().cpu().numpy()
+    half_ulp = np.ldexp(1.0, np.frexp(np.abs(g))[1] - 9)
+    excess = np.abs(g - exact) - half_ulp - bound
+    n_diff = int((g != rounded).sum())
+    print(f"{what}: {n_diff} of {g.size} elements differ from the correctly rounded value; "
+          f"worst margin to the bound {excess.max():.3e}")
+    assert excess.max() <= 0.0, f"{what}: an element is {excess.max():.3e} beyond its bound"
+    assert n_diff <= MISMATCH_MAX_FRACTION * g.size, f"{what}: {n_diff} elements differ"
 
 
-def _ulp_compare(got: torch.Tensor, ref: np.ndarray, what: str):
-    ref_bf = torch.from_numpy(ref).to(torch.bfloat16)   # the oracle's values are bf16 already
-    assert np.array_equal(ref_bf.double().numpy(), ref), f"{what}: oracle output not bf16-valued"
-    dist = np.abs(_ulp_keys(got.cpu()) - _ulp_keys(ref_bf))
-    n_diff = int((dist > 0).sum())
-    frac = n_diff / max(1, dist.size)
-    print(f"{what}: {n_diff} of {dist.size} elements differ by one bf16 ulp ({frac:.2e}), max {int(dist.max())}")
-    assert int(dist.max()) <= 1, f"{what}: an element is {int(dist.max())} bf16 ulps from the oracle"
-    assert frac <= ULP_MISMATCH_MAX_FRACTION, f"{what}: {frac:.2e} of the elements differ by one ulp"
-    return n_diff
+def _check_projection(d, B, T, C, H, Hkv, D, qh, kh, vp, eps=1e-6):
+    x = d["x"].double().numpy().reshape(B, T, C)
+    Wm = d["W"].double().numpy()
+    y = x @ Wm.T                                    # (B, T, N), exact products, fp64 sum
+    dy = C * 2.0 ** -23 * (np.abs(x) @ np.abs(Wm).T)
+    px = oracle.qkv_prologue(d["x"], d["W"], H, Hkv, D, ids=d.get("ids"), table=d.get("table"),
+                             Wg=d.get("Wg"), parity=False)
+    pr = oracle.qkv_prologue(d["x"], d["W"], H, Hkv, D, ids=d.get("ids"), table=d.get("table"),
+                             Wg=d.get("Wg"), parity=True)
+    eps = float(np.float32(eps))
+    for name, heads, off, got, ex, rd in (("qhat", H, 0, qh, px[0], pr[0]), ("khat", Hkv, H * D, kh, px[1], pr[1])):
+        yh = y[..., off:off + heads * D].reshape(B, T, heads, D)
+        dyh = dy[..., off:off + heads * D].reshape(B, T, heads, D)
+        swap = lambda a: np.concatenate([a[..., D // 2:], a[..., :D // 2]], axis=-1)   # RoPE partner
+        ss = (yh ** 2).sum(-1, keepdims=True)
+        r = 1.0 / np.sqrt(ss / D + eps)
+        dss = 2.0 * (np.abs(yh) * dyh).sum(-1, keepdims=True)
+        bound = (r * (dyh + swap(dyh)) + np.abs(ex) * dss / (ss + D * eps)
+                 + 2.0 ** -20 * (r * (np.abs(yh) + np.abs(swap(yh))) + np.abs(ex)))
+        _check_bound(got, ex, rd, bound, name)
+    yv = y[..., (H + Hkv) * D:].reshape(B, T, Hkv, D)
+    dyv = dy[..., (H + Hkv) * D:].reshape(B, T, Hkv, D)
+    ve = d["ve"].double().numpy() if "ve" in d else np.zeros_like(yv)
+    bound = dyv + 2.0 ** -20 * (np.abs(px[2]) + 2.0 * np.abs(ve))
+    _check_bound(vp, px[2], pr[2], bound, "v'")
 
 
 CASES = [
@@ -86,16 +110,12 @@ CASES = [
 
 
 @pytest.mark.parametrize("B,T,C,H,Hkv,D,ve", CASES)
-def test_qkv_prologue_within_one_ulp_of_the_oracle(B, T, C, H, Hkv, D, ve):
+def test_qkv_prologue_within_the_accumulation_bound(B, T, C, H, Hkv, D, ve):
     d = _draw(B, T, C, H, Hkv, D, ve, seed=B * 1000 + T + C + D)
     g = {k: v.cuda() for k, v in d.items() if k in ("x", "W", "ve", "Wg")}
     qh, kh, vp = swa.qkv_prologue(g["x"], g["W"], H, Hkv, D, ve=g.get("ve"), Wg=g.get("Wg"))
     swa.check_device_status()
-    rq, rk, rv = oracle.qkv_prologue(d["x"], d["W"], H, Hkv, D, ids=d.get("ids"), table=d.get("table"),
-                                     Wg=d.get("Wg"), parity=True)
-    _ulp_compare(qh, rq, "qhat")
-    _ulp_compare(kh, rk, "khat")
-    _ulp_compare(vp, rv, "v'")
+    _check_projection(d, B, T, C, H, Hkv, D, qh, kh, vp)
 
 
 @pytest.mark.parametrize("B,T,C,H,Hkv,D,ve,window", [
