@@ -46,7 +46,7 @@ UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["causal_sliding_window_swa_b200/csrc/attn_fwd.cuh",
                   "causal_sliding_window_swa_b200/csrc/ptx.cuh",
-                  "causal_sliding_window_swa_b200/csrc/rope_fast.cuh"]
+                  "causal_sliding_window_swa_b200/csrc/rope_exact.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
 
 
@@ -274,9 +274,9 @@ def run_ours(args, s0):
     stream = torch.cuda.current_stream(dev)
     st = stream.cuda_stream
     P = lambda t: None if t is None else t.data_ptr()
-    # the stages of swa_attn_fwd_ws (the same kernels swa_attn_fwd runs): the key/value fp32
-    # prologue (with the gate on value-embedding layers), then the attention kernel that reads the
-    # raw q and normalises each query tile itself
+    # the stages of swa_attn_fwd_ws (the same kernels swa_attn_fwd runs): the key/value prologue
+    # (with the gate on value-embedding layers), then the attention kernel that reads the raw q and
+    # normalises each query tile itself
     args_pro = (None, P(x["k"]), P(x["v"]), P(x["ve"]), P(x["gate_x"]), P(x["Wg"]),
                 s.B, s.T, s.H, s.D, 10000.0, 1e-6, ws.data_ptr(), nbytes, st)
     args_att = (P(x["q"]), P(x["v"]), int(s.ve), out.data_ptr(), lse.data_ptr(), s.B, s.T, s.H, s.D, s.window,
@@ -297,7 +297,7 @@ def run_ours(args, s0):
     def step(e=None):
         if e is not None:
             e[0].record(stream)
-        check(swa.swa_attn_prologue_fast(*args_pro), "swa_attn_prologue_fast")
+        check(swa.swa_attn_prologue(*args_pro), "swa_attn_prologue")
         if e is not None:
             e[1].record(stream)
         check(swa.swa_attn_attention_q(*args_att), "swa_attn_attention_q")

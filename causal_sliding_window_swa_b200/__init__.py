@@ -58,8 +58,6 @@ def _load() -> ctypes.CDLL:
     lib.swa_attn_prologue.restype = I
     lib.swa_attn_attention.argtypes = [P, I, P, P, I, I, I, I, I, P, Z, P]
     lib.swa_attn_attention.restype = I
-    lib.swa_attn_prologue_fast.argtypes = [P, P, P, P, P, P, I, I, I, I, F, F, P, Z, P]
-    lib.swa_attn_prologue_fast.restype = I
     lib.swa_attn_attention_q.argtypes = [P, P, I, P, P, I, I, I, I, I, F, P, Z, P]
     lib.swa_attn_attention_q.restype = I
     lib.swa_attn_strerror.argtypes = [I]
@@ -68,6 +66,8 @@ def _load() -> ctypes.CDLL:
     lib.swa_attn_last_device_status.restype = I
     lib.swa_attn_fwd_gqa.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, F, P]
     lib.swa_attn_fwd_gqa.restype = I
+    lib.swa_attn_fwd_doc.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, F, P]
+    lib.swa_attn_fwd_doc.restype = I
     lib.swa_attn_decode_workspace_bytes.argtypes = [I, I, I, I, I, I]
     lib.swa_attn_decode_workspace_bytes.restype = Z
     lib.swa_attn_decode.argtypes = [P, P, P, P, P, P, P, P, I, P, P, I, I, I, I, I, F, F, P, Z, P]
@@ -163,12 +163,6 @@ def swa_attn_attention(v, has_ve, out, lse, B, T, H, D, window, workspace, ws_by
     return _lib.swa_attn_attention(v, int(has_ve), out, lse, B, T, H, D, window, workspace, ws_bytes, stream)
 
 
-def swa_attn_prologue_fast(q, k, v, ve, gate_x, Wg, B, T, H, D, rope_base, eps, workspace, ws_bytes,
-                           stream) -> int:
-    return _lib.swa_attn_prologue_fast(q, k, v, ve, gate_x, Wg, B, T, H, D, rope_base, eps, workspace,
-                                       ws_bytes, stream)
-
-
 def swa_attn_attention_q(q, v, has_ve, out, lse, B, T, H, D, window, eps, workspace, ws_bytes, stream) -> int:
     return _lib.swa_attn_attention_q(q, v, int(has_ve), out, lse, B, T, H, D, window, eps, workspace, ws_bytes,
                                      stream)
@@ -187,6 +181,12 @@ def swa_attn_last_device_status(stream=None) -> Tuple[int, int]:
 def swa_attn_fwd_gqa(q, k, v, ve, gate_x, Wg, out, lse, B, T, H, Hkv, D, window, rope_base, eps,
                      stream) -> int:
     return _lib.swa_attn_fwd_gqa(q, k, v, ve, gate_x, Wg, out, lse, B, T, H, Hkv, D, window, rope_base,
+                                 eps, stream)
+
+
+def swa_attn_fwd_doc(q, k, v, ve, gate_x, Wg, doc, out, lse, B, T, H, Hkv, D, window, rope_base, eps,
+                     stream) -> int:
+    return _lib.swa_attn_fwd_doc(q, k, v, ve, gate_x, Wg, doc, out, lse, B, T, H, Hkv, D, window, rope_base,
                                  eps, stream)
 
 
@@ -287,12 +287,14 @@ def _check_qkv(q, k, v, ve, gate_x, Wg):
 
 def forward(q, k, v, window: int = 0, ve=None, gate_x=None, Wg=None, rope_base: float = 10000.0,
             eps: float = 1e-6, *, out=None, lse=None, with_lse: bool = True, workspace=None,
-            stream=None):
+            stream=None, doc=None):
     """One attention layer.  q bf16 (B,T,H,D); k, v (and ve) bf16 (B,T,Hkv,D) CUDA tensors, Hkv
     dividing H (grouped-query attention when Hkv < H: C call swa_attn_fwd_gqa); gate_x (B,T,32);
     Wg [32,Hkv].  Returns (out bf16 (B,T,H,D), lse fp32 (B,H,T) or None).
     ``workspace``: optional uint8 CUDA tensor of at least ``swa_attn_workspace_bytes`` bytes
-    (then nothing is allocated by the library; multi-head layers only)."""
+    (then nothing is allocated by the library; multi-head layers only).
+    ``doc``: optional int32 CUDA tensor (B, T) of document ids (C call swa_attn_fwd_doc): a key is
+    then visible only inside the query's document, a maximal run of equal ids."""
     import torch
     B, T, H, Hkv, D = _check_qkv(q, k, v, ve, gate_x, Wg)
     if out is None:
@@ -300,6 +302,16 @@ def forward(q, k, v, window: int = 0, ve=None, gate_x=None, Wg=None, rope_base: 
     if with_lse and lse is None:
         lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
     st = _stream_handle(stream)
+    if doc is not None:
+        if tuple(doc.shape) != (B, T) or doc.dtype != torch.int32 or not doc.is_cuda or not doc.is_contiguous():
+            raise ValueError(f"doc must be a contiguous CUDA int32 tensor of shape {(B, T)}")
+        if workspace is not None:
+            raise ValueError("the document-masked call uses the library workspace")
+        rc = swa_attn_fwd_doc(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(doc), _ptr(out),
+                              _ptr(lse), B, T, H, Hkv, D, int(window), float(rope_base), float(eps), st)
+        if rc != SWA_OK:
+            raise SwaError(rc, "swa_attn_fwd_doc")
+        return out, lse
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(out), _ptr(lse),
             B, T, H, D, int(window), float(rope_base), float(eps))
     if Hkv != H:
@@ -453,10 +465,10 @@ def check_device_status(stream=None) -> None:
 __all__ = [
     "forward", "decode", "backward", "qkv_prologue", "forward_x", "check_device_status", "SwaError", "LIB_PATH", "load",
     "swa_attn_fwd", "swa_attn_fwd_ws", "swa_attn_fwd_noalloc", "swa_attn_noalloc_scratch_bytes", "swa_attn_workspace_bytes", "swa_attn_workspace_offset", "swa_attn_rope_table", "swa_attn_prologue",
-    "swa_attn_attention", "swa_attn_prologue_fast", "swa_attn_attention_q", "swa_attn_strerror",
+    "swa_attn_attention", "swa_attn_attention_q", "swa_attn_strerror",
     "swa_attn_last_device_status",
     "swa_attn_set_wait_limit_ms", "swa_attn_selftest_wait", "swa_attn_version",
-    "swa_attn_decode", "swa_attn_decode_workspace_bytes", "swa_attn_fwd_gqa",
+    "swa_attn_decode", "swa_attn_decode_workspace_bytes", "swa_attn_fwd_gqa", "swa_attn_fwd_doc",
     "swa_attn_bwd", "swa_attn_bwd_gqa", "swa_attn_bwd_workspace_bytes",
     "swa_attn_fwd_x", "swa_attn_qkv_prologue", "swa_attn_fwd_x_workspace_bytes",
 ]

@@ -41,10 +41,10 @@
 // One exponential in four is evaluated by a polynomial on the FMA pipe to offload the MUFU unit.
 //
 // Query prologue inside the kernel (QPRO).  With QPRO the producer loads the RAW query tile and the
-// softmax warps apply RoPE + RMS to it in shared memory (rope_fast.cuh, thread (row r, quarter c)
-// owning the rotation pairs of quarter c of row r; the four partial sums of squares of a row meet in
-// shared memory) before the MMA thread copies it into tensor memory, so qhat never goes through
-// HBM.  The softmax warps transform the next item's tile right after the last softmax tile of the
+// softmax warps apply RoPE + RMS to it in shared memory (rope_exact.cuh, thread (row r, quarter c)
+// owning the rotation pairs of quarter c of row r; the four fp64 partial sums of squares of a row
+// meet in shared memory) before the MMA thread copies it into tensor memory, so qhat never goes
+// through HBM; its bits equal those of the standalone prologue kernel.  The softmax warps transform the next item's tile right after the last softmax tile of the
 // current item, while the tensor pipe runs that item's last PV product, and write the current
 // item's output afterwards; the next item's first score product then follows the PV product on the
 // pipe without a gap.  Without QPRO the query tile in HBM is already normalised (the fused
@@ -56,7 +56,7 @@
 #include <cstdint>
 
 #include "ptx.cuh"
-#include "rope_fast.cuh"
+#include "rope_exact.cuh"
 
 namespace swa {
 
@@ -74,7 +74,7 @@ struct FwdCfg {
     static constexpr int SMEM_OUT = TILE_BYTES;        // output tile staged for the TMA store
     static constexpr int SMEM_BAR = 512;
     static constexpr int SMEM_LX = 4 * 128 * 8;        // row-sum exchange between the four threads of a row
-    static constexpr int SMEM_QX = 2 * 4 * 128 * 4;    // query sums of squares, double-buffered by item
+    static constexpr int SMEM_QX = 2 * 4 * 128 * 8;    // fp64 query sums of squares, double-buffered by item
     // Dynamic shared memory is declared 1024-byte aligned (the 128-byte swizzle atom repeats every
     // 1024 bytes); the kernel checks the alignment on entry instead of reserving slack for it.
     static constexpr int SMEM_TOTAL = SMEM_Q + SMEM_KV + SMEM_OUT + SMEM_BAR + SMEM_LX + SMEM_QX;
@@ -99,9 +99,10 @@ struct FwdParams {
     float* lse;            // (B,H,T) or null
     int* sched;            // [0] next item, [1] CTAs done; zero before the launch, reset after
     unsigned long long wait_limit_ns;
-    const float2* tabf;    // fp32 RoPE table (cos, sin) per (t, i) (QPRO)
-    float inv_d;           // 1 / D (QPRO)
-    float eps;             // RMS epsilon (QPRO)
+    const double2* tab64;  // fp64 RoPE table (cos, sin) per (t, i) (QPRO)
+    double inv_d;          // 1 / D (QPRO)
+    double eps;            // RMS epsilon (QPRO)
+    const int* dstart;     // (B, T) start of each position's document (document mask), or null
 };
 
 // Wait sites recorded in the status word on timeout.
@@ -132,6 +133,9 @@ __device__ __forceinline__ Item decode_item(const FwdParams& p, int it) {
     m.q0 = qt * 128;
     m.lo = max(0, m.q0 - p.W + 1) / 128;
     m.hi = min(m.q0 + 127, p.T - 1) / 128;
+    // Document mask: no key before the first query row's document start is visible to any row of
+    // the tile (starts never decrease along the sequence), so those key tiles are skipped too.
+    if (p.dstart != nullptr) m.lo = max(m.lo, p.dstart[(long long)m.b * p.T + m.q0] / 128);
     return m;
 }
 
@@ -205,8 +209,9 @@ __device__ __forceinline__ uint32_t softmax_pair_poly(uint32_t s0, uint32_t s1, 
     return w;
 }
 
-template <int D, bool QPRO>
-__global__ void __launch_bounds__(576, 1)
+// 576 threads, one CTA per SM: 112 registers per thread fit the register file (576 x 112 <= 64 K).
+template <int D, bool QPRO, bool DOC = false>
+__global__ void __maxnreg__(112)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                     const FwdParams p) {
@@ -241,7 +246,7 @@ __global__ void __launch_bounds__(576, 1)
     int* s_item = reinterpret_cast<int*>(b_qready + 1);           // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_item + 2);
     float2* s_lx = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(bars) + C::SMEM_BAR);   // [4][128]
-    float* s_qx = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(s_lx) + C::SMEM_LX);    // [2][4][128]
+    double* s_qx = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(s_lx) + C::SMEM_LX);   // [2][4][128]
     static_assert(13 + 2 * C::NSB + 2 * C::NS + 2 <= (C::SMEM_BAR - 16) / 8, "barrier area");
 
     const int warp = threadIdx.x >> 5;
@@ -495,10 +500,6 @@ __global__ void __launch_bounds__(576, 1)
             constexpr int QP = D / 8;
             constexpr int NW = QP / 8;                  // 16-byte words per half (2 or 1)
             const int t = min(mq.q0 + r, p.T - 1);      // rows past T hold zeros; any table row does
-            float4 cs[QP / 2];
-            const float4* tp = reinterpret_cast<const float4*>(p.tabf + (long long)t * (D / 2) + cq * QP);
-#pragma unroll
-            for (int e = 0; e < QP / 2; ++e) cs[e] = __ldg(tp + e);
             uint32_t offa[NW], offb[NW];
 #pragma unroll
             for (int e = 0; e < NW; ++e) {
@@ -507,6 +508,10 @@ __global__ void __launch_bounds__(576, 1)
                 offa[e] = (uint32_t)((ca >> 6) * C::CHUNK_BYTES + r * 128 + ((((ca & 63) >> 3) ^ (r & 7)) << 4));
                 offb[e] = (uint32_t)((cb >> 6) * C::CHUNK_BYTES + r * 128 + ((((cb & 63) >> 3) ^ (r & 7)) << 4));
             }
+            const double2* tab = p.tab64 + (long long)t * (D / 2) + cq * QP;
+            // warm this thread's table entries while the tile is in flight
+#pragma unroll
+            for (int e = 0; e < QP; e += 4) asm volatile("prefetch.global.L1 [%0];" ::"l"(tab + e));
             bool w = mbar_wait(smem_u32(b_qfull), kk & 1u, lim, kSiteQFull);
             if (!__all_sync(0xffffffffu, w)) return false;
             uint4 qa[NW], qb[NW];
@@ -515,14 +520,14 @@ __global__ void __launch_bounds__(576, 1)
                 qa[e] = *reinterpret_cast<const uint4*>(sQ + offa[e]);
                 qb[e] = *reinterpret_cast<const uint4*>(sQ + offb[e]);
             }
-            float* xs = s_qx + (kk & 1u) * 512u;
-            xs[cq * 128 + r] = quarter_sumsq<NW>(qa, qb);
+            double* xs = s_qx + (kk & 1u) * 512u;
+            xs[cq * 128 + r] = quarter_sumsq64<NW>(qa, qb);
             mbar_arrive(smem_u32(b_qss));
             w = mbar_wait(smem_u32(b_qss), kk & 1u, lim, kSiteQSum);
             if (!__all_sync(0xffffffffu, w)) return false;
-            const float rs = rms_scale4(xs[r], xs[128 + r], xs[256 + r], xs[384 + r], p.inv_d, p.eps);
+            const double rs = rms_scale64(xs[r], xs[128 + r], xs[256 + r], xs[384 + r], p.inv_d, p.eps);
             uint4 oa[NW], ob[NW];
-            rope_quarter<NW>(qa, qb, cs, rs, oa, ob);
+            rope_quarter64<NW>(qa, qb, tab, rs, oa, ob);
 #pragma unroll
             for (int e = 0; e < NW; ++e) {
                 *reinterpret_cast<uint4*>(sQ + offa[e]) = oa[e];
@@ -539,6 +544,13 @@ __global__ void __launch_bounds__(576, 1)
         while (ok && it >= 0) {
             const Item m = decode_item(p, it);
             const int qi = m.q0 + r;              // this thread's query position
+            // Document mask: this row's document start, and the largest start among the warp's
+            // rows (warp-uniform test of whether a key block needs the per-element mask).
+            int ds = 0, ds_w = 0;
+            if constexpr (DOC) {
+                ds = __ldg(p.dstart + (long long)m.b * p.T + min(qi, p.T - 1));
+                ds_w = __reduce_max_sync(0xffffffffu, ds);
+            }
             uint64_t l2[4], lr2[4];
 #pragma unroll
             for (int a = 0; a < 4; ++a) l2[a] = lr2[a] = 0ull;
@@ -551,7 +563,7 @@ __global__ void __launch_bounds__(576, 1)
                 if (++s_buf == (uint32_t)C::NSB) s_buf = 0;
                 tc_fence_after();
                 const int k0 = j * C::BN + 32 * cq;    // first key of this thread's 32 columns
-                const bool need_mask = (k0 + 31 > m.q0) || (m.q0 + C::BM - 1 - k0 >= p.W);
+                const bool need_mask = (k0 + 31 > m.q0) || (m.q0 + C::BM - 1 - k0 >= p.W) || (DOC && k0 < ds_w);
                 const uint32_t colS = buf * 128u + 32u * (uint32_t)cq;
                 // The 32 scores in two 16-column blocks, both loaded before any arithmetic; P of
                 // the 32 keys packs into 16 words written over the first 16 of these columns.
@@ -572,8 +584,10 @@ __global__ void __launch_bounds__(576, 1)
                         for (int e = 0; e < 16; e += 2) {
                             const int kv = k0 + cbase + e;
                             // masked scores become -inf in log2 units, so exp gives exactly 0
-                            const uint32_t m0 = ((unsigned)(qi - kv) >= (unsigned)p.W) ? 0xff800000u : sv[e];
-                            const uint32_t m1 = ((unsigned)(qi - kv - 1) >= (unsigned)p.W) ? 0xff800000u : sv[e + 1];
+                            const uint32_t m0 = ((unsigned)(qi - kv) >= (unsigned)p.W || (DOC && kv < ds))
+                                                    ? 0xff800000u : sv[e];
+                            const uint32_t m1 = ((unsigned)(qi - kv - 1) >= (unsigned)p.W || (DOC && kv + 1 < ds))
+                                                    ? 0xff800000u : sv[e + 1];
                             pk[pkbase + (e >> 1)] =
                                 softmax_pair_mufu(m0, m1, c1x2, nc2x2, l2[e >> 1 & 3], lr2[e >> 1 & 3]);
                         }

@@ -18,7 +18,8 @@
 #include "decode.cuh"
 #include "prologue.cuh"
 #include "qkv_gemm.cuh"
-#include "rope_fast.cuh"
+#include "rope_exact.cuh"
+#include "docmask.cuh"
 
 // ------------------------------------------------------------------ failure-detection self-test
 
@@ -112,13 +113,13 @@ constexpr size_t kAlign = 1024;
 size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct WsLayout {
-    size_t qh, kh, vp, gate, tab32, tab64, tabf, sched, total;
+    size_t qh, kh, vp, gate, tab32, tab64, sched, dstart, total;
 };
 
 // qhat | khat | v' and gate (value-embedding layers only) | RoPE table fp32 pieces |
-// RoPE table fp64 | RoPE table fp32 (cos, sin) | attention scheduler counters, each section
-// 1024-byte aligned.
-WsLayout ws_layout(const Shape& s, bool has_ve) {
+// RoPE table fp64 | attention scheduler counters | document starts (B, T) int32
+// (document-masked calls only), each section 1024-byte aligned.
+WsLayout ws_layout(const Shape& s, bool has_ve, bool has_doc = false) {
     WsLayout w{};
     const size_t tensor = round_up((size_t)s.n * 2);
     const size_t kv_tensor = round_up((size_t)s.B * s.T * s.Hkv * s.D * 2);
@@ -129,9 +130,9 @@ WsLayout ws_layout(const Shape& s, bool has_ve) {
     w.gate = w.vp + (has_ve ? kv_tensor : 0);
     w.tab32 = w.gate + (has_ve ? round_up((size_t)s.B * s.T * s.Hkv * sizeof(float2)) : 0);
     w.tab64 = w.tab32 + round_up(pairs * sizeof(float4));
-    w.tabf = w.tab64 + round_up(pairs * sizeof(double2));
-    w.sched = w.tabf + round_up(pairs * sizeof(float2));
-    w.total = w.sched + kAlign;
+    w.sched = w.tab64 + round_up(pairs * sizeof(double2));
+    w.dstart = w.sched + kAlign;
+    w.total = w.dstart + (has_doc ? round_up((size_t)s.B * s.T * sizeof(int)) : 0);
     return w;
 }
 
@@ -183,6 +184,10 @@ int device_ready(int* dev_out) {
                 cudaFuncSetAttribute(swa::attn_fwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      swa::FwdCfg<64>::SMEM_TOTAL) != cudaSuccess ||
                 cudaFuncSetAttribute(swa::attn_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     swa::FwdCfg<128>::SMEM_TOTAL) != cudaSuccess ||
+                cudaFuncSetAttribute(swa::attn_fwd_kernel<64, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     swa::FwdCfg<64>::SMEM_TOTAL) != cudaSuccess ||
+                cudaFuncSetAttribute(swa::attn_fwd_kernel<128, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      swa::FwdCfg<128>::SMEM_TOTAL) != cudaSuccess ||
                 cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<64>, (cudaFuncAttribute)smem_attr,
                                      swa::BwdCfg<64>::DQ_SMEM) != cudaSuccess ||
@@ -258,89 +263,19 @@ int launch_rope_table(uint8_t* ws, const WsLayout& L, const Shape& s, float rope
     const int threads = 256;
     const long long blocks = std::min<long long>((n + threads - 1) / threads, 148ll * 16);
     swa::rope_table_kernel<<<(unsigned)blocks, threads, 0, st>>>(
-        reinterpret_cast<float4*>(ws + L.tab32), reinterpret_cast<double2*>(ws + L.tab64),
-        reinterpret_cast<float2*>(ws + L.tabf), s.T, s.D, (double)rope_base);
+        reinterpret_cast<float4*>(ws + L.tab32), reinterpret_cast<double2*>(ws + L.tab64), s.T, s.D,
+        (double)rope_base);
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
+// The prologue (rope_exact.cuh): the gate on value-embedding layers, then one launch whose blocks
+// write qhat (when q is given), khat and v' (value-embedding layers) into the workspace, each
+// element exactly rounded.  It also zeroes the attention kernel's scheduler counters.
 int launch_prologue(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
                     const void* Wg, uint8_t* ws, const WsLayout& L, const Shape& s, float eps,
                     cudaStream_t st) {
     using bf = __nv_bfloat16;
     const bool has_ve = ve != nullptr;
-    const int n_rows = s.B * s.T * s.H;
-    const int n_kv_rows = s.B * s.T * s.Hkv;
-    const swa::FastDiv divH = make_fastdiv(s.H), divT = make_fastdiv(s.T);
-    float2* gate = reinterpret_cast<float2*>(ws + L.gate);
-    if (has_ve) {
-        const int gblocks = (int)std::min<long long>(((long long)n_kv_rows + 255) / 256, 148ll * 8);
-        swa::gate_kernel<<<gblocks, 256, 0, st>>>(static_cast<const bf*>(gate_x), static_cast<const bf*>(Wg),
-                                                   gate, n_kv_rows, s.Hkv, make_fastdiv(s.Hkv), 32);
-    }
-    const long long threads_total = (long long)n_rows * (s.D / 8);
-    const int threads = 256;
-    const long long blocks = std::min<long long>((threads_total + threads - 1) / threads, 148ll * 3 * 4);
-    const bf* qp = static_cast<const bf*>(q);
-    const bf* kp = static_cast<const bf*>(k);
-    const bf* vpi = static_cast<const bf*>(v);
-    const bf* vep = static_cast<const bf*>(ve);
-    bf* qh = reinterpret_cast<bf*>(ws + L.qh);
-    bf* kh = reinterpret_cast<bf*>(ws + L.kh);
-    bf* vp = reinterpret_cast<bf*>(ws + L.vp);
-    const float4* t32 = reinterpret_cast<const float4*>(ws + L.tab32);
-    const double2* t64 = reinterpret_cast<const double2*>(ws + L.tab64);
-    int* sched = reinterpret_cast<int*>(ws + L.sched);
-    const unsigned g = (unsigned)blocks;
-    const double e = (double)eps;
-    if (s.Hkv != s.H) {
-        // Grouped-query attention: the query rows (H heads) and the key/value rows (Hkv heads) are
-        // two passes over their own rows.
-        const swa::FastDiv divK = make_fastdiv(s.Hkv);
-        const unsigned gk = (unsigned)std::min<long long>(((long long)n_kv_rows * (s.D / 8) + threads - 1) / threads,
-                                                          148ll * 3 * 4);
-#define SWA_PRO_GQA(DD, VE)                                                                                  \
-    swa::prologue_kernel<DD, VE, 1><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, \
-                                                           n_rows, s.T, s.H, divT, divH, e);                 \
-    swa::prologue_kernel<DD, VE, 2><<<gk, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, \
-                                                            n_kv_rows, s.T, s.Hkv, divT, divK, e)
-        if (s.D == 128) {
-            if (has_ve) {
-                SWA_PRO_GQA(128, true);
-            } else {
-                SWA_PRO_GQA(128, false);
-            }
-        } else {
-            if (has_ve) {
-                SWA_PRO_GQA(64, true);
-            } else {
-                SWA_PRO_GQA(64, false);
-            }
-        }
-#undef SWA_PRO_GQA
-        return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
-    }
-    if (s.D == 128) {
-        if (has_ve)
-            swa::prologue_kernel<128, true><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, divT, divH, e);
-        else
-            swa::prologue_kernel<128, false><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, divT, divH, e);
-    } else {
-        if (has_ve)
-            swa::prologue_kernel<64, true><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, divT, divH, e);
-        else
-            swa::prologue_kernel<64, false><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, divT, divH, e);
-    }
-    return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
-}
-
-// The fp32 prologue (rope_fast.cuh): the gate on value-embedding layers, then one launch whose
-// blocks write qhat (when q is given), khat and v' (value-embedding layers) into the workspace.
-// It also zeroes the attention kernel's scheduler counters.
-int launch_prologue_fast(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
-                         const void* Wg, uint8_t* ws, const WsLayout& L, const Shape& s, float eps,
-                         cudaStream_t st) {
-    using bf = __nv_bfloat16;
-    const bool has_ve = ve != nullptr;
     const int n_kv_rows = s.B * s.T * s.Hkv;
     float2* gate = reinterpret_cast<float2*>(ws + L.gate);
     if (has_ve) {
@@ -348,7 +283,7 @@ int launch_prologue_fast(const void* q, const void* k, const void* v, const void
         swa::gate_kernel<<<gblocks, 256, 0, st>>>(static_cast<const bf*>(gate_x), static_cast<const bf*>(Wg),
                                                    gate, n_kv_rows, s.Hkv, make_fastdiv(s.Hkv), 32);
     }
-    swa::FastProParams p{};
+    swa::ExactProParams p{};
     p.q = static_cast<const bf*>(q);
     p.k = static_cast<const bf*>(k);
     p.v = static_cast<const bf*>(v);
@@ -357,7 +292,7 @@ int launch_prologue_fast(const void* q, const void* k, const void* v, const void
     p.qh = reinterpret_cast<bf*>(ws + L.qh);
     p.kh = reinterpret_cast<bf*>(ws + L.kh);
     p.vp = reinterpret_cast<bf*>(ws + L.vp);
-    p.tabf = reinterpret_cast<const float2*>(ws + L.tabf);
+    p.tab64 = reinterpret_cast<const double2*>(ws + L.tab64);
     p.n_q = q ? s.B * s.T * s.H : 0;
     p.n_k = n_kv_rows;
     p.n_v = has_ve ? n_kv_rows : 0;
@@ -367,27 +302,28 @@ int launch_prologue_fast(const void* q, const void* k, const void* v, const void
     p.H = s.H;
     p.Hkv = s.Hkv;
     p.T = s.T;
-    p.inv_d = 1.0f / (float)s.D;
-    p.eps = eps;
+    p.inv_d = 1.0 / (double)s.D;
+    p.eps = (double)eps;
     p.sched = reinterpret_cast<int*>(ws + L.sched);
     const long long blocks = (long long)p.nb_q + p.nb_k + nb_v;
     if (blocks >= (1ll << 31)) return SWA_ERR_UNSUPPORTED;
     if (s.D == 128) {
-        if (has_ve) swa::prologue_fast_kernel<128, true><<<(unsigned)blocks, 256, 0, st>>>(p);
-        else swa::prologue_fast_kernel<128, false><<<(unsigned)blocks, 256, 0, st>>>(p);
+        if (has_ve) swa::prologue_exact_kernel<128, true><<<(unsigned)blocks, 256, 0, st>>>(p);
+        else swa::prologue_exact_kernel<128, false><<<(unsigned)blocks, 256, 0, st>>>(p);
     } else {
-        if (has_ve) swa::prologue_fast_kernel<64, true><<<(unsigned)blocks, 256, 0, st>>>(p);
-        else swa::prologue_fast_kernel<64, false><<<(unsigned)blocks, 256, 0, st>>>(p);
+        if (has_ve) swa::prologue_exact_kernel<64, true><<<(unsigned)blocks, 256, 0, st>>>(p);
+        else swa::prologue_exact_kernel<64, false><<<(unsigned)blocks, 256, 0, st>>>(p);
     }
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
 // The attention kernel.  q_raw non-null: the kernel reads the raw q (B,T,H,D) and applies RoPE + RMS
-// to each query tile itself (the fp32 prologue's arithmetic; the RoPE table must be in the
+// to each query tile itself (the prologue's exact arithmetic; the RoPE table must be in the
 // workspace); q_raw null: it reads qhat from the workspace.  khat (and v' on value-embedding
 // layers) always come from the workspace.
 int launch_attention(int dev, const void* q_raw, const void* v, bool has_ve, void* out, float* lse,
-                     const Shape& s, int window, float eps, uint8_t* ws, const WsLayout& L, cudaStream_t st) {
+                     const Shape& s, int window, float eps, uint8_t* ws, const WsLayout& L, cudaStream_t st,
+                     const int* dstart = nullptr) {
     CUtensorMap tq, tk, tv, to;
     const void* vsrc = has_ve ? static_cast<const void*>(ws + L.vp) : v;
     const void* qsrc = q_raw ? q_raw : static_cast<const void*>(ws + L.qh);
@@ -415,16 +351,20 @@ int launch_attention(int dev, const void* q_raw, const void* v, bool has_ve, voi
     p.lse = lse;
     p.sched = reinterpret_cast<int*>(ws + L.sched);
     p.wait_limit_ns = wait_limit_ns();
-    p.tabf = reinterpret_cast<const float2*>(ws + L.tabf);
-    p.inv_d = 1.0f / (float)s.D;
-    p.eps = eps;
+    p.tab64 = reinterpret_cast<const double2*>(ws + L.tab64);
+    p.inv_d = 1.0 / (double)s.D;
+    p.eps = (double)eps;
+    p.dstart = dstart;
     const dim3 grid((unsigned)std::min(p.n_items, g_num_sms[dev]));
-#define SWA_ATTN(DD, QP) \
-    swa::attn_fwd_kernel<DD, QP><<<grid, swa::FwdCfg<DD>::THREADS, swa::FwdCfg<DD>::SMEM_TOTAL, st>>>(tq, tk, tv, to, p)
-    if (s.D == 128) {
-        if (q_raw) SWA_ATTN(128, true); else SWA_ATTN(128, false);
+#define SWA_ATTN(DD, QP, DC) \
+    swa::attn_fwd_kernel<DD, QP, DC><<<grid, swa::FwdCfg<DD>::THREADS, swa::FwdCfg<DD>::SMEM_TOTAL, st>>>(tq, tk, tv, to, p)
+    if (dstart) {
+        if (!q_raw) return SWA_ERR_INVALID_ARG;
+        if (s.D == 128) SWA_ATTN(128, true, true); else SWA_ATTN(64, true, true);
+    } else if (s.D == 128) {
+        if (q_raw) SWA_ATTN(128, true, false); else SWA_ATTN(128, false, false);
     } else {
-        if (q_raw) SWA_ATTN(64, true); else SWA_ATTN(64, false);
+        if (q_raw) SWA_ATTN(64, true, false); else SWA_ATTN(64, false, false);
     }
 #undef SWA_ATTN
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
@@ -565,10 +505,9 @@ int launch_backward(int dev, const void* q, const void* k, const void* v, const 
     using bf = __nv_bfloat16;
     const bool has_ve = ve != nullptr;
     int rc;
-    // qhat, khat, v' and the gate exactly as the forward computed them (the fp32 prologue's
-    // arithmetic, which the forward's attention kernel applies to the query tiles in place).
+    // qhat, khat, v' and the gate exactly as the forward computed them.
     if ((rc = launch_rope_table(ws, L.f, s, rope_base, st)) != SWA_OK) return rc;
-    if ((rc = launch_prologue_fast(q, k, v, ve, gate_x, Wg, ws, L.f, s, eps, st)) != SWA_OK) return rc;
+    if ((rc = launch_prologue(q, k, v, ve, gate_x, Wg, ws, L.f, s, eps, st)) != SWA_OK) return rc;
 
     int* sched4 = reinterpret_cast<int*>(ws + L.f.sched) + 4;
     float2* rowstat = reinterpret_cast<float2*>(ws + L.rowstat);
@@ -743,7 +682,8 @@ int swa_attn_prologue(const void* q, const void* k, const void* v, const void* v
                       swa_stream_t stream) {
     Shape s;
     int rc = check_sizes(B, T, H, D, &s);
-    if (rc == SWA_OK) rc = check_layer_args(q, k, v, ve, gate_x, Wg, rope_base, eps);
+    // q may be null (khat and v' only); the others follow the layer's rules
+    if (rc == SWA_OK) rc = check_layer_args(q ? q : k, k, v, ve, gate_x, Wg, rope_base, eps);
     if (rc != SWA_OK) return rc;
     if (!workspace) return SWA_ERR_INVALID_ARG;
     if (!aligned(workspace, 16)) return SWA_ERR_MISALIGNED;
@@ -782,30 +722,11 @@ int swa_attn_fwd_ws(const void* q, const void* k, const void* v, const void* ve,
     if (rc != SWA_OK) return rc;
     rc = swa_attn_rope_table(B, T, H, D, ve != nullptr, rope_base, workspace, ws_bytes, stream);
     if (rc != SWA_OK) return rc;
-    rc = swa_attn_prologue_fast(nullptr, k, v, ve, gate_x, Wg, B, T, H, D, rope_base, eps, workspace,
-                                ws_bytes, stream);
+    rc = swa_attn_prologue(nullptr, k, v, ve, gate_x, Wg, B, T, H, D, rope_base, eps, workspace, ws_bytes,
+                           stream);
     if (rc != SWA_OK) return rc;
     return swa_attn_attention_q(q, v, ve != nullptr, out, lse, B, T, H, D, window, eps, workspace,
                                 ws_bytes, stream);
-}
-
-int swa_attn_prologue_fast(const void* q, const void* k, const void* v, const void* ve,
-                           const void* gate_x, const void* Wg, int B, int T, int H, int D,
-                           float rope_base, float eps, void* workspace, size_t ws_bytes,
-                           swa_stream_t stream) {
-    Shape s;
-    int rc = check_sizes(B, T, H, D, &s);
-    // q may be null here (khat and v' only); the others follow the layer's rules
-    if (rc == SWA_OK) rc = check_layer_args(q ? q : k, k, v, ve, gate_x, Wg, rope_base, eps);
-    if (rc != SWA_OK) return rc;
-    if (!workspace) return SWA_ERR_INVALID_ARG;
-    if (!aligned(workspace, 16)) return SWA_ERR_MISALIGNED;
-    const WsLayout L = ws_layout(s, ve != nullptr);
-    if (ws_bytes < L.total) return SWA_ERR_NO_MEMORY;
-    int dev;
-    if ((rc = device_ready(&dev)) != SWA_OK) return rc;
-    return launch_prologue_fast(q, k, v, ve, gate_x, Wg, static_cast<uint8_t*>(workspace), L, s, eps,
-                                reinterpret_cast<cudaStream_t>(stream));
 }
 
 int swa_attn_attention_q(const void* q, const void* v, int has_ve, void* out, float* lse, int B, int T,
@@ -826,20 +747,21 @@ int swa_attn_attention_q(const void* q, const void* v, int has_ve, void* out, fl
                             L, reinterpret_cast<cudaStream_t>(stream));
 }
 
-int swa_attn_fwd_gqa(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
-                     const void* Wg, void* out, float* lse, int B, int T, int H, int Hkv, int D,
-                     int window, float rope_base, float eps, swa_stream_t stream) {
-    Shape s;
-    int rc = check_sizes(B, T, H, D, &s);
-    if (rc == SWA_OK) rc = check_kv_heads(Hkv, &s);
-    if (rc == SWA_OK) rc = check_layer_args(q, k, v, ve, gate_x, Wg, rope_base, eps);
-    if (rc == SWA_OK) rc = check_outputs(out, lse);
-    if (rc != SWA_OK) return rc;
+}  // extern "C"
+
+namespace {
+
+// The forward with the library-owned workspace of the current device (validated arguments).
+int fwd_library_ws(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                   const void* Wg, const int* doc, void* out, float* lse, const Shape& s, int window,
+                   float rope_base, float eps, swa_stream_t stream) {
+    int rc;
     int dev;
     if ((rc = device_ready(&dev)) != SWA_OK) return rc;
+    const int T = s.T, D = s.D;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const bool has_ve = ve != nullptr;
-    const WsLayout L = ws_layout(s, has_ve);
+    const WsLayout L = ws_layout(s, has_ve, doc != nullptr);
 
     const unsigned long long limit = wait_limit_ns();   // read before taking the cache lock
     (void)limit;
@@ -880,8 +802,15 @@ int swa_attn_fwd_gqa(const void* q, const void* k, const void* v, const void* ve
         c.tab_base = rope_base;
         c.tab_off = L.tab32;
     }
-    rc = launch_prologue_fast(nullptr, k, v, ve, gate_x, Wg, ws, L, s, eps, st);
-    if (rc == SWA_OK) rc = launch_attention(dev, q, v, has_ve, out, lse, s, window, eps, ws, L, st);
+    int* dstart = doc ? reinterpret_cast<int*>(ws + L.dstart) : nullptr;
+    if (doc) {
+        swa::doc_start_kernel<<<s.B, 1024, 0, st>>>(doc, dstart, s.T);
+        rc = cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+    } else {
+        rc = SWA_OK;
+    }
+    if (rc == SWA_OK) rc = launch_prologue(nullptr, k, v, ve, gate_x, Wg, ws, L, s, eps, st);
+    if (rc == SWA_OK) rc = launch_attention(dev, q, v, has_ve, out, lse, s, window, eps, ws, L, st, dstart);
     // Recorded after whatever was enqueued, also on failure, so the next call orders after it.
     if (cudaEventRecord(c.last_use, st) != cudaSuccess) {
         cudaGetLastError();
@@ -889,6 +818,36 @@ int swa_attn_fwd_gqa(const void* q, const void* k, const void* v, const void* ve
     }
     c.last_stream = st;
     return rc;
+}
+
+}  // namespace
+
+extern "C" {
+
+int swa_attn_fwd_gqa(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                     const void* Wg, void* out, float* lse, int B, int T, int H, int Hkv, int D,
+                     int window, float rope_base, float eps, swa_stream_t stream) {
+    Shape s;
+    int rc = check_sizes(B, T, H, D, &s);
+    if (rc == SWA_OK) rc = check_kv_heads(Hkv, &s);
+    if (rc == SWA_OK) rc = check_layer_args(q, k, v, ve, gate_x, Wg, rope_base, eps);
+    if (rc == SWA_OK) rc = check_outputs(out, lse);
+    if (rc != SWA_OK) return rc;
+    return fwd_library_ws(q, k, v, ve, gate_x, Wg, nullptr, out, lse, s, window, rope_base, eps, stream);
+}
+
+int swa_attn_fwd_doc(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                     const void* Wg, const int* doc, void* out, float* lse, int B, int T, int H, int Hkv,
+                     int D, int window, float rope_base, float eps, swa_stream_t stream) {
+    Shape s;
+    int rc = check_sizes(B, T, H, D, &s);
+    if (rc == SWA_OK) rc = check_kv_heads(Hkv, &s);
+    if (rc == SWA_OK) rc = check_layer_args(q, k, v, ve, gate_x, Wg, rope_base, eps);
+    if (rc == SWA_OK) rc = check_outputs(out, lse);
+    if (rc != SWA_OK) return rc;
+    if (!doc) return SWA_ERR_INVALID_ARG;
+    if (!aligned(doc, 4)) return SWA_ERR_MISALIGNED;
+    return fwd_library_ws(q, k, v, ve, gate_x, Wg, doc, out, lse, s, window, rope_base, eps, stream);
 }
 
 int swa_attn_fwd(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
@@ -1187,6 +1146,6 @@ extern "C" int swa_attn_fwd_noalloc(const void* q, const void* k, const void* v,
     // tables, then khat / v' and the gate; the prologue also zeroes the attention kernel's
     // scheduler counters), so nothing left by an earlier call is read.
     if ((rc = launch_rope_table(ws, L, s, rope_base, st)) != SWA_OK) return rc;
-    if ((rc = launch_prologue_fast(nullptr, k, v, ve, gate_x, Wg, ws, L, s, eps, st)) != SWA_OK) return rc;
+    if ((rc = launch_prologue(nullptr, k, v, ve, gate_x, Wg, ws, L, s, eps, st)) != SWA_OK) return rc;
     return launch_attention(dev, q, v, has_ve, out, lse, s, window, eps, ws, L, st);
 }

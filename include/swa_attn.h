@@ -31,13 +31,11 @@
  * Streams: calls are asynchronous on `stream` (NULL = the legacy default stream) and never
  * synchronise the host, except swa_attn_last_device_status().
  *
- * Precision of the forward calls (swa_attn_fwd, _gqa, _ws, _noalloc): the prologue runs in fp32
- * and rounds qhat, khat and v' to bf16 once (round to nearest even); each of those elements is the
- * bf16 rounding of a value within a few fp32 ulps of its exact value, so it is the correctly
- * rounded bf16 or, for elements that lie that close to a rounding midpoint, one bf16 ulp from it.
- * The query prologue runs inside the attention kernel on each query tile (qhat never goes through
- * HBM).  swa_attn_prologue() is the exactly rounded prologue (every element the correctly rounded
- * bf16 of its exact value), used by the staged path and the decode step.
+ * Precision: the prologue evaluates qhat, khat and v' in fp64 and rounds each to bf16 once
+ * (nearest, ties to even), so every element is the correctly rounded bf16 of its exact value
+ * (except within about 2^-50 of a rounding midpoint).  In the forward calls (swa_attn_fwd, _gqa,
+ * _doc, _ws, _noalloc) the query prologue runs inside the attention kernel on each raw query tile,
+ * so qhat never goes through HBM; it gives the same bits as swa_attn_prologue() with q.
  *
  * Errors: a negative swa_status.  Arguments are validated before anything is enqueued; a
  * rejected call has no effect.  Waits inside the kernels are bounded: if one expires, the
@@ -118,16 +116,32 @@ SWA_API int swa_attn_fwd_gqa(const void* q, const void* k, const void* v,
                              int B, int T, int H, int Hkv, int D, int window,
                              float rope_base, float eps, swa_stream_t stream);
 
+/*
+ * Document-boundary mask (packed documents; the pages list variable-length attention among the
+ * changes that were tried: intelliparadigm "GPT-2 for $73", section 7).  As swa_attn_fwd_gqa, plus
+ * doc: int32 (B, T) device array of document ids.  A document is a maximal run of equal ids along
+ * a sequence (number packed documents in order: ids that never repeat across runs); key j is
+ * visible to query i iff 0 <= i - j < window and j is in i's document.  RoPE positions stay the
+ * sequence positions 0..T-1.  Key tiles before the first query row's document start are skipped.
+ * Uses the library-owned workspace (plus B*T int32 document starts), with its stream ordering.
+ * Errors as swa_attn_fwd_gqa; SWA_ERR_INVALID_ARG if doc is NULL, SWA_ERR_MISALIGNED if it is
+ * not 4-byte aligned.
+ */
+SWA_API int swa_attn_fwd_doc(const void* q, const void* k, const void* v,
+                             const void* ve, const void* gate_x, const void* Wg, const int* doc,
+                             void* out, float* lse,
+                             int B, int T, int H, int Hkv, int D, int window,
+                             float rope_base, float eps, swa_stream_t stream);
+
 /* Bytes of caller workspace swa_attn_fwd_ws() needs for these sizes (0 on invalid sizes). */
 SWA_API size_t swa_attn_workspace_bytes(int B, int T, int H, int D, int has_ve);
 
 /*
  * Byte offset of one section of the workspace, for callers that read the prologue's results
- * (e.g. to keep them for a backward pass) after swa_attn_prologue() or swa_attn_prologue_fast():
- *   SWA_WS_QHAT, SWA_WS_KHAT   bf16 (B,T,H,D): rms(rope(q)), rms(rope(k)); after
- *                              swa_attn_prologue() each element is the correctly rounded bf16
- *                              (nearest, ties to even) of its exact value, after
- *                              swa_attn_prologue_fast() it is within one bf16 ulp of that;
+ * (e.g. to keep them for a backward pass) after swa_attn_prologue():
+ *   SWA_WS_QHAT, SWA_WS_KHAT   bf16 (B,T,H,D): rms(rope(q)), rms(rope(k)), each element the
+ *                              correctly rounded bf16 (nearest, ties to even) of its exact value
+ *                              (qhat only when swa_attn_prologue() was given q);
  *   SWA_WS_VPRIME              bf16 (B,T,H,D): v + 2 sigmoid(gate_x . Wg) ve, same rounding
  *                              (value-embedding layers only);
  *   SWA_WS_ROPE_TABLE          the RoPE table (internal format).
@@ -140,7 +154,7 @@ SWA_API size_t swa_attn_workspace_offset(int B, int T, int H, int D, int has_ve,
  * Same as swa_attn_fwd() with caller-owned device scratch: `workspace` (16-byte aligned,
  * at least swa_attn_workspace_bytes() bytes) holds khat, v', the gates and the RoPE table, which
  * is rebuilt on every call (one small extra kernel).  It runs swa_attn_rope_table(),
- * swa_attn_prologue_fast() with q = NULL and swa_attn_attention_q().  Nothing is allocated.
+ * swa_attn_prologue() with q = NULL and swa_attn_attention_q().  Nothing is allocated.
  * SWA_ERR_NO_MEMORY if ws_bytes is too small.
  */
 SWA_API int swa_attn_fwd_ws(const void* q, const void* k, const void* v,
@@ -158,19 +172,17 @@ SWA_API int swa_attn_fwd_ws(const void* q, const void* k, const void* v,
  *   rope_base, so a caller that keeps one workspace for many calls of the same T, D and base
  *   builds it once (swa_attn_fwd does that with its own workspace).
  * swa_attn_prologue: RoPE + RMS norm of q and k, gate + add of the value embedding, into the
- *   workspace (same sizes and rules as swa_attn_fwd_ws).  Uses the table already in the
- *   workspace; it does not rebuild it.
- * swa_attn_attention: the windowed attention on a workspace that swa_attn_prologue() (or
- *   swa_attn_prologue_fast() with q) filled for the same B, T, H, D and value-embedding setting
- *   (`v` is read directly when has_ve == 0).
- * swa_attn_prologue_fast: the forward's fp32 prologue (precision: see the top of this file) into
- *   the workspace: khat, and v' with its gate on value-embedding layers; qhat too when q is not
- *   NULL (q = NULL is the forward's key/value pass).  Needs the RoPE table in the workspace.  It
- *   also resets the scheduler counters that the attention kernels take their work from.
+ *   workspace (same sizes and rules as swa_attn_fwd_ws; precision: see the top of this file).
+ *   q may be NULL: then only khat and v' (the forward's key/value pass; the forward normalises the
+ *   query tiles inside the attention kernel).  Uses the table already in the workspace; it does not
+ *   rebuild it.  It also resets the scheduler counters the attention kernels take their work from.
+ * swa_attn_attention: the windowed attention on a workspace that swa_attn_prologue() with q
+ *   filled for the same B, T, H, D and value-embedding setting (`v` is read directly when
+ *   has_ve == 0).
  * swa_attn_attention_q: the windowed attention reading the RAW q (B,T,H,D) and applying RoPE + RMS
  *   (eps as for the prologue) to each query tile inside the kernel, with khat (and v') from a
- *   workspace that swa_attn_prologue_fast() filled; its qhat equals, bit for bit, the one
- *   swa_attn_prologue_fast() writes for the same q.
+ *   workspace that swa_attn_prologue() filled; its qhat equals, bit for bit, the one
+ *   swa_attn_prologue() writes for the same q.
  * All of them: asynchronous on `stream`, validation before any launch, errors as swa_attn_fwd_ws.
  */
 SWA_API int swa_attn_rope_table(int B, int T, int H, int D, int has_ve, float rope_base,
@@ -184,11 +196,6 @@ SWA_API int swa_attn_prologue(const void* q, const void* k, const void* v,
 SWA_API int swa_attn_attention(const void* v, int has_ve, void* out, float* lse,
                        int B, int T, int H, int D, int window,
                        void* workspace, size_t ws_bytes, swa_stream_t stream);
-
-SWA_API int swa_attn_prologue_fast(const void* q, const void* k, const void* v,
-                                   const void* ve, const void* gate_x, const void* Wg,
-                                   int B, int T, int H, int D, float rope_base, float eps,
-                                   void* workspace, size_t ws_bytes, swa_stream_t stream);
 
 SWA_API int swa_attn_attention_q(const void* q, const void* v, int has_ve, void* out, float* lse,
                                  int B, int T, int H, int D, int window, float eps,

@@ -99,14 +99,14 @@ def test_stage_entry_points_reject_bad_arguments():
     assert swa.swa_attn_attention(None, 0, A, A, 1, 16, 1, 64, 0, A, need, None) == swa.SWA_ERR_INVALID_ARG
     assert swa.swa_attn_attention(A, 0, A, A, 1, 16, 1, 64, 0, A, need - 1, None) == swa.SWA_ERR_NO_MEMORY
     assert swa.swa_attn_attention(A, 0, A, A, 1, 16, 1, 80, 0, A, need, None) == swa.SWA_ERR_UNSUPPORTED
-    # the fp32 prologue: q may be NULL (key/value pass), k may not
-    assert swa.swa_attn_prologue_fast(None, A, A, None, None, None, 1, 16, 1, 64, 1e4, 1e-6, A, need - 1, None) \
+    # the prologue: q may be NULL (key/value pass), k may not
+    assert swa.swa_attn_prologue(None, A, A, None, None, None, 1, 16, 1, 64, 1e4, 1e-6, A, need - 1, None) \
         == swa.SWA_ERR_NO_MEMORY
-    assert swa.swa_attn_prologue_fast(None, None, A, None, None, None, 1, 16, 1, 64, 1e4, 1e-6, A, need, None) \
+    assert swa.swa_attn_prologue(None, None, A, None, None, None, 1, 16, 1, 64, 1e4, 1e-6, A, need, None) \
         == swa.SWA_ERR_INVALID_ARG
-    assert swa.swa_attn_prologue_fast(A + 2, A, A, None, None, None, 1, 16, 1, 64, 1e4, 1e-6, A, need, None) \
+    assert swa.swa_attn_prologue(A + 2, A, A, None, None, None, 1, 16, 1, 64, 1e4, 1e-6, A, need, None) \
         == swa.SWA_ERR_MISALIGNED
-    assert swa.swa_attn_prologue_fast(None, A, A, A, None, None, 1, 16, 1, 64, 1e4, 1e-6, A, need, None) \
+    assert swa.swa_attn_prologue(None, A, A, A, None, None, 1, 16, 1, 64, 1e4, 1e-6, A, need, None) \
         == swa.SWA_ERR_INVALID_ARG
     # the attention from the raw q
     assert swa.swa_attn_attention_q(None, A, 0, A, A, 1, 16, 1, 64, 0, 1e-6, A, need, None) == swa.SWA_ERR_INVALID_ARG
@@ -115,6 +115,21 @@ def test_stage_entry_points_reject_bad_arguments():
     assert swa.swa_attn_attention_q(A, A, 0, A, A, 1, 16, 1, 64, 0, -1.0, A, need, None) == swa.SWA_ERR_INVALID_ARG
     assert swa.swa_attn_attention_q(A, A, 0, A, A, 1, 16, 1, 128 + 64, 0, 1e-6, A, need, None) \
         == swa.SWA_ERR_UNSUPPORTED
+
+
+def test_document_forward_rejects_bad_arguments():
+    base = dict(q=A, k=A, v=A, ve=None, gate_x=None, Wg=None, doc=A, out=A, lse=A, B=1, T=16, H=2, Hkv=1, D=64,
+                window=0, rope_base=1e4, eps=1e-6, stream=None)
+
+    def call(**kw):
+        a = dict(base)
+        a.update(kw)
+        return swa.swa_attn_fwd_doc(*a.values())
+    assert call(doc=None) == swa.SWA_ERR_INVALID_ARG
+    assert call(doc=A + 2) == swa.SWA_ERR_MISALIGNED
+    assert call(Hkv=3) == swa.SWA_ERR_INVALID_ARG
+    assert call(D=80) == swa.SWA_ERR_UNSUPPORTED
+    assert call(q=None) == swa.SWA_ERR_INVALID_ARG
 
 
 def test_wait_limit_setter():
