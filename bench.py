@@ -5,9 +5,8 @@ Metric: attention-forward TFLOP/s counted over unmasked (query, key) pairs (4*D 
 2D for q.k, 2D for p*v), with tokens/s and the fraction of the dense-BF16 tensor peak, on the
 nanochat d24 full-window layer with value embeddings (B=16, T=2048, H=12, D=128, W=2048).
 
-One step = one whole layer forward (the gate and the RoPE + RMS / value-embedding prologue of k
-and v, then the windowed attention kernel, which applies RoPE + RMS to each raw query tile itself
-and writes out and the LSE) on inputs already resident in HBM.  Inputs are seeded synthetic
+One step = one whole layer forward (RoPE + RMS QK-norm + VE gate prologue, then the windowed
+attention with its LSE) on inputs already resident in HBM.  Inputs are seeded synthetic
 N(0,1) bf16 tensors shaped like the layer; they are larger than the 126 MB L2, so no flush
 is needed between steps.
 
@@ -45,8 +44,7 @@ METRIC = "attention fwd TFLOP/s (unmasked pairs) & tokens/s, d24 T=2048; % of BF
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["causal_sliding_window_swa_b200/csrc/attn_fwd.cuh",
-                  "causal_sliding_window_swa_b200/csrc/ptx.cuh",
-                  "causal_sliding_window_swa_b200/csrc/rope_exact.cuh"]
+                  "causal_sliding_window_swa_b200/csrc/ptx.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
 
 
@@ -274,13 +272,12 @@ def run_ours(args, s0):
     stream = torch.cuda.current_stream(dev)
     st = stream.cuda_stream
     P = lambda t: None if t is None else t.data_ptr()
-    # the stages of swa_attn_fwd_ws (the same kernels swa_attn_fwd runs): the key/value prologue
-    # (with the gate on value-embedding layers), then the attention kernel that reads the raw q and
-    # normalises each query tile itself
-    args_pro = (None, P(x["k"]), P(x["v"]), P(x["ve"]), P(x["gate_x"]), P(x["Wg"]),
+    # the stages of swa_attn_fwd_ws (the same kernels swa_attn_fwd runs): the prologue (with the
+    # gate on value-embedding layers), then the attention kernel
+    args_pro = (P(x["q"]), P(x["k"]), P(x["v"]), P(x["ve"]), P(x["gate_x"]), P(x["Wg"]),
                 s.B, s.T, s.H, s.D, 10000.0, 1e-6, ws.data_ptr(), nbytes, st)
-    args_att = (P(x["q"]), P(x["v"]), int(s.ve), out.data_ptr(), lse.data_ptr(), s.B, s.T, s.H, s.D, s.window,
-                1e-6, ws.data_ptr(), nbytes, st)
+    args_att = (P(x["v"]), int(s.ve), out.data_ptr(), lse.data_ptr(), s.B, s.T, s.H, s.D, s.window,
+                ws.data_ptr(), nbytes, st)
 
     def check(rc, what):
         if rc != 0:
@@ -300,7 +297,7 @@ def run_ours(args, s0):
         check(swa.swa_attn_prologue(*args_pro), "swa_attn_prologue")
         if e is not None:
             e[1].record(stream)
-        check(swa.swa_attn_attention_q(*args_att), "swa_attn_attention_q")
+        check(swa.swa_attn_attention(*args_att), "swa_attn_attention")
         if e is not None:
             e[2].record(stream)
 
@@ -378,7 +375,7 @@ def run_ours(args, s0):
         "pct_bf16_peak": 100.0 * value / world / peak,
         "peak_source": f"{peak_src} bf16_tflops (burst)",
         "stage_ms": {"prologue": pro_ms_max, "attention": att_ms_max},
-        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128, true>", "achieved": achieved,
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "traffic": recorded_traffic(args.workload),
                      "note": f"4*D flops per unmasked pair / mean attention launch time; peak = "
@@ -388,7 +385,7 @@ def run_ours(args, s0):
                               "frac": prologue_bytes(s) / (pro_ms_max * 1e-3) / 1e9 / float(peaks["hbm_gbs"])},
         "e2e": {"value": world * fl / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": (3 if s.ve else 2) * K,   # (gate,) key/value prologue, attention
+        "gpu_launches": (3 if s.ve else 2) * K,   # (gate,) prologue, attention
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -402,10 +399,10 @@ def run_ours(args, s0):
 
 
 def prologue_bytes(s: workloads.LayerShape) -> float:
-    """Algorithmic bytes of the key/value prologue stage (the query prologue runs inside the
-    attention kernel): read k (+ v, ve, gate_x, Wg), write khat (+ v')."""
+    """Algorithmic bytes of the prologue stage: read q, k (+ v, ve, gate_x, Wg), write qhat, khat
+    (+ v')."""
     n = s.n_elems * 2
-    b = n + n                   # k in; khat out
+    b = 2 * n + 2 * n           # q, k in; qhat, khat out
     if s.ve:
         b += 3 * n + s.B * s.T * 32 * 2 + 32 * s.H * 2   # v, ve in; v' out; gate_x, Wg
     return float(b)

@@ -58,8 +58,6 @@ def _load() -> ctypes.CDLL:
     lib.swa_attn_prologue.restype = I
     lib.swa_attn_attention.argtypes = [P, I, P, P, I, I, I, I, I, P, Z, P]
     lib.swa_attn_attention.restype = I
-    lib.swa_attn_attention_q.argtypes = [P, P, I, P, P, I, I, I, I, I, F, P, Z, P]
-    lib.swa_attn_attention_q.restype = I
     lib.swa_attn_strerror.argtypes = [I]
     lib.swa_attn_strerror.restype = ctypes.c_char_p
     lib.swa_attn_last_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
@@ -74,11 +72,16 @@ def _load() -> ctypes.CDLL:
     lib.swa_attn_decode.restype = I
     lib.swa_attn_decode_gqa.argtypes = [P, P, P, P, P, P, P, P, I, P, P, I, I, I, I, I, I, F, F, P, Z, P]
     lib.swa_attn_decode_gqa.restype = I
+    lib.swa_attn_decode_doc.argtypes = [P, P, P, P, P, P, P, P, I, P, P, P, I, I, I, I, I, I, F, F, P, Z, P]
+    lib.swa_attn_decode_doc.restype = I
     lib.swa_attn_bwd_workspace_bytes.argtypes = [I, I, I, I, I, I]
     lib.swa_attn_bwd_workspace_bytes.restype = Z
     lib.swa_attn_bwd_gqa.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
                                      I, I, I, I, I, I, F, F, P, Z, P]
     lib.swa_attn_bwd_gqa.restype = I
+    lib.swa_attn_bwd_doc.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
+                                     I, I, I, I, I, I, F, F, P, Z, P]
+    lib.swa_attn_bwd_doc.restype = I
     lib.swa_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
                                  I, I, I, I, I, F, F, P, Z, P]
     lib.swa_attn_bwd.restype = I
@@ -161,11 +164,6 @@ def swa_attn_prologue(q, k, v, ve, gate_x, Wg, B, T, H, D, rope_base, eps, works
 
 def swa_attn_attention(v, has_ve, out, lse, B, T, H, D, window, workspace, ws_bytes, stream) -> int:
     return _lib.swa_attn_attention(v, int(has_ve), out, lse, B, T, H, D, window, workspace, ws_bytes, stream)
-
-
-def swa_attn_attention_q(q, v, has_ve, out, lse, B, T, H, D, window, eps, workspace, ws_bytes, stream) -> int:
-    return _lib.swa_attn_attention_q(q, v, int(has_ve), out, lse, B, T, H, D, window, eps, workspace, ws_bytes,
-                                     stream)
 
 
 def swa_attn_strerror(status: int) -> str:
@@ -332,10 +330,13 @@ def forward(q, k, v, window: int = 0, ve=None, gate_x=None, Wg=None, rope_base: 
 
 
 def decode(q, k, v, k_cache, v_cache, pos: int, window: int, ve=None, gate_x=None, Wg=None,
-           rope_base: float = 1e4, eps: float = 1e-6, out=None, lse=None, workspace=None, stream=None):
+           rope_base: float = 1e4, eps: float = 1e-6, out=None, lse=None, workspace=None, stream=None,
+           doc_start=None):
     """One generation step (C call swa_attn_decode, or swa_attn_decode_gqa when k has fewer heads
     than q) on torch tensors: q (B,H,D), k, v (B,Hkv,D) bf16 of the new token at position ``pos``;
     k_cache, v_cache (B,Tmax,Hkv,D) bf16, updated in place at ``pos``.
+    ``doc_start``: optional int32 CUDA tensor (B,) with the first position of each sequence's
+    current document (C call swa_attn_decode_doc).
     Returns (out (B,H,D) bf16, lse (B,H) fp32).  Raises SwaError on a nonzero status."""
     import torch
     B, H, D = q.shape
@@ -349,6 +350,16 @@ def decode(q, k, v, k_cache, v_cache, pos: int, window: int, ve=None, gate_x=Non
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     st = _stream_handle(stream)
+    if doc_start is not None:
+        if tuple(doc_start.shape) != (B,) or doc_start.dtype != torch.int32 or not doc_start.is_cuda:
+            raise ValueError(f"doc_start must be a CUDA int32 tensor of shape {(B,)}")
+        rc = _lib.swa_attn_decode_doc(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(k_cache),
+                                      _ptr(v_cache), int(pos), _ptr(doc_start), _ptr(out), _ptr(lse), B, Tmax, H,
+                                      Hkv, D, int(window), float(rope_base), float(eps), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), st)
+        if rc != SWA_OK:
+            raise SwaError(rc, "swa_attn_decode_doc")
+        return out, lse
     if Hkv == H:
         rc = swa_attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(k_cache),
                              _ptr(v_cache), int(pos), _ptr(out), _ptr(lse), B, Tmax, H, D, int(window),
@@ -364,14 +375,21 @@ def decode(q, k, v, k_cache, v_cache, pos: int, window: int, ve=None, gate_x=Non
     return out, lse
 
 
+def swa_attn_bwd_doc(q, k, v, ve, gate_x, Wg, doc, out, lse, dout, dlse, dq, dk, dv, dve, dgate_x, dWg,
+                     B, T, H, Hkv, D, window, rope_base, eps, workspace, ws_bytes, stream) -> int:
+    return _lib.swa_attn_bwd_doc(q, k, v, ve, gate_x, Wg, doc, out, lse, dout, dlse, dq, dk, dv, dve, dgate_x,
+                                 dWg, B, T, H, Hkv, D, window, rope_base, eps, workspace, ws_bytes, stream)
+
+
 def backward(q, k, v, out, lse, dout, window: int = 0, dlse=None, ve=None, gate_x=None, Wg=None,
-             rope_base: float = 10000.0, eps: float = 1e-6, *, workspace=None, stream=None):
+             rope_base: float = 10000.0, eps: float = 1e-6, *, workspace=None, stream=None, doc=None):
     """Gradient of one layer (C call swa_attn_bwd_gqa) for the loss sum(dout * out) +
     sum(dlse * lse).  q, k, v, ve, gate_x, Wg as for ``forward``; out bf16 (B,T,H,D) and lse fp32
     (B,H,T) are that call's outputs; dout bf16 (B,T,H,D); dlse fp32 (B,H,T) or None.
     Returns a dict: dq bf16 (B,T,H,D), dk, dv bf16 (B,T,Hkv,D) and, on value-embedding layers,
-    dve bf16 (B,T,Hkv,D), dgate_x fp32 (B,T,32), dWg fp32 [32,Hkv].  Raises SwaError on a nonzero
-    status."""
+    dve bf16 (B,T,Hkv,D), dgate_x fp32 (B,T,32), dWg fp32 [32,Hkv].  ``doc``: the int32 (B, T)
+    document ids of a document-masked forward (C call swa_attn_bwd_doc).  Raises SwaError on a
+    nonzero status."""
     import torch
     B, T, H, Hkv, D = _check_qkv(q, k, v, ve, gate_x, Wg)
     for name, t in (("out", out), ("dout", dout)):
@@ -390,13 +408,16 @@ def backward(q, k, v, out, lse, dout, window: int = 0, dlse=None, ve=None, gate_
     need = swa_attn_bwd_workspace_bytes(B, T, H, Hkv, D, ve is not None)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    rc = swa_attn_bwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(out), _ptr(lse),
-                          _ptr(dout), _ptr(dlse), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g.get("dve")),
-                          _ptr(g.get("dgate_x")), _ptr(g.get("dWg")), B, T, H, Hkv, D, int(window),
-                          float(rope_base), float(eps), _ptr(workspace),
+    if doc is not None and (tuple(doc.shape) != (B, T) or doc.dtype != torch.int32 or not doc.is_cuda
+                            or not doc.is_contiguous()):
+        raise ValueError(f"doc must be a contiguous CUDA int32 tensor of shape {(B, T)}")
+    rc = swa_attn_bwd_doc(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(doc), _ptr(out),
+                          _ptr(lse), _ptr(dout), _ptr(dlse), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
+                          _ptr(g.get("dve")), _ptr(g.get("dgate_x")), _ptr(g.get("dWg")), B, T, H, Hkv, D,
+                          int(window), float(rope_base), float(eps), _ptr(workspace),
                           workspace.numel() * workspace.element_size(), _stream_handle(stream))
     if rc != SWA_OK:
-        raise SwaError(rc, "swa_attn_bwd_gqa")
+        raise SwaError(rc, "swa_attn_bwd_doc" if doc is not None else "swa_attn_bwd_gqa")
     return g
 
 
@@ -465,10 +486,10 @@ def check_device_status(stream=None) -> None:
 __all__ = [
     "forward", "decode", "backward", "qkv_prologue", "forward_x", "check_device_status", "SwaError", "LIB_PATH", "load",
     "swa_attn_fwd", "swa_attn_fwd_ws", "swa_attn_fwd_noalloc", "swa_attn_noalloc_scratch_bytes", "swa_attn_workspace_bytes", "swa_attn_workspace_offset", "swa_attn_rope_table", "swa_attn_prologue",
-    "swa_attn_attention", "swa_attn_attention_q", "swa_attn_strerror",
+    "swa_attn_attention", "swa_attn_strerror",
     "swa_attn_last_device_status",
     "swa_attn_set_wait_limit_ms", "swa_attn_selftest_wait", "swa_attn_version",
     "swa_attn_decode", "swa_attn_decode_workspace_bytes", "swa_attn_fwd_gqa", "swa_attn_fwd_doc",
-    "swa_attn_bwd", "swa_attn_bwd_gqa", "swa_attn_bwd_workspace_bytes",
+    "swa_attn_bwd", "swa_attn_bwd_gqa", "swa_attn_bwd_doc", "swa_attn_bwd_workspace_bytes",
     "swa_attn_fwd_x", "swa_attn_qkv_prologue", "swa_attn_fwd_x_workspace_bytes",
 ]

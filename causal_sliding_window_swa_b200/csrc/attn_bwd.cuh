@@ -95,6 +95,8 @@ struct BwdParams {
     float* dvp;            // (B, T, Hkv, D) fp32: dL/dv'
     int* sched;            // [0] next item, [1] CTAs done; zero before the launch, reset after
     unsigned long long wait_limit_ns;
+    const int* dstart;     // (B, T) first position of each position's document, or null (no mask)
+    const int* dend;       // (B, T) last position of each position's document, or null
 };
 
 // Wait sites recorded in the status word on timeout (distinct from the forward's).
@@ -124,6 +126,8 @@ __device__ __forceinline__ BwdQItem bwd_q_item(const BwdParams& p, int it) {
     m.q0 = qt * 128;
     m.lo = max(0, m.q0 - p.W + 1) / 128;
     m.hi = min(m.q0 + 127, p.T - 1) / 128;
+    // Document mask: keys before the first row's document start are seen by no row of the tile.
+    if (p.dstart != nullptr) m.lo = max(m.lo, p.dstart[(long long)m.b * p.T + m.q0] / 128);
     return m;
 }
 
@@ -148,6 +152,8 @@ __device__ __forceinline__ BwdKvItem bwd_kv_item(const BwdParams& p, int it) {
     m.k0 = kt * 128;
     m.lo = kt;
     m.hi = min(m.k0 + 127 + p.W - 1, p.T - 1) / 128;
+    // Document mask: queries past the last key's document end see no key of the tile.
+    if (p.dend != nullptr) m.hi = min(m.hi, p.dend[(long long)m.b * p.T + min(m.k0 + 127, p.T - 1)] / 128);
     return m;
 }
 
@@ -213,7 +219,7 @@ __global__ void bwd_rowstat_kernel(const __nv_bfloat16* __restrict__ out, const 
 //   so while the warps work on tile g the tensor pipe runs dQ(g - 1) and S(g + 1), and only dP(g + 1)
 //   waits for them.  S(g + 2) overwrites the buffer whose dS(g) the dQ(g) product issued just
 //   before it reads (products execute in issue order).
-template <int D>
+template <int D, bool DOC = false>
 __global__ void __launch_bounds__(576, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -452,6 +458,8 @@ __global__ void __launch_bounds__(576, 1)
             if (!ok || it < 0) break;
             const BwdQItem m = bwd_q_item(p, it);
             const int qi = m.q0 + r;
+            // document mask: this row sees no key before its document's start
+            const int ds = DOC ? __ldg(p.dstart + (long long)m.b * p.T + min(qi, p.T - 1)) : 0;
             const float2 rs = p.rowstat[((long long)m.b * p.H + m.h) * p.Tp + qi];
             const float nl = -rs.x, dl = rs.y;
             for (int j = m.lo; j <= m.hi; ++j, ++g) {
@@ -475,8 +483,8 @@ __global__ void __launch_bounds__(576, 1)
                         const int kv = k0 + 16 * hb + e;
                         float p0 = ex2_approx(fmaf(__uint_as_float(sv[hb][e]), p.c1, nl));
                         float p1 = ex2_approx(fmaf(__uint_as_float(sv[hb][e + 1]), p.c1, nl));
-                        if ((unsigned)(qi - kv) >= (unsigned)p.W) p0 = 0.f;
-                        if ((unsigned)(qi - kv - 1) >= (unsigned)p.W) p1 = 0.f;
+                        if ((unsigned)(qi - kv) >= (unsigned)p.W || (DOC && kv < ds)) p0 = 0.f;
+                        if ((unsigned)(qi - kv - 1) >= (unsigned)p.W || (DOC && kv + 1 < ds)) p1 = 0.f;
                         const float d0 = p0 * (__uint_as_float(dv[hb][e]) - dl);
                         const float d1 = p1 * (__uint_as_float(dv[hb][e + 1]) - dl);
                         pk[8 * hb + (e >> 1)] = pack_bf16x2(d0, d1);
@@ -533,7 +541,7 @@ __global__ void __launch_bounds__(576, 1)
 //     S^T(0) dP^T(0) | [P^T(0)] dV(0) S^T(1) [dS^T(0)] dK(0) dP^T(1) | [P^T(1)] dV(1) S^T(2) ...
 //   so phase A of step s + 1 waits only for dV(s) and S^T(s + 1), and phase B for dK(s) and
 //   dP^T(s + 1); each overwrite of a buffer follows, in issue order, the product that reads it.
-template <int D>
+template <int D, bool DOC = false>
 __global__ void __launch_bounds__(576, 1)
     attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -785,6 +793,8 @@ __global__ void __launch_bounds__(576, 1)
             if (!ok || it < 0) break;
             const BwdKvItem m = bwd_kv_item(p, it);
             const int key = m.k0 + r;
+            // document mask: no query past this key's document end sees it
+            const int de = DOC ? __ldg(p.dend + (long long)m.b * p.T + min(key, p.T - 1)) : 0;
             const int nq = m.hi - m.lo + 1;
             const int n_steps = p.G * nq;
             for (int s = 0; s < n_steps; ++s, ++g) {
@@ -814,8 +824,8 @@ __global__ void __launch_bounds__(576, 1)
                         const float2 r0 = rs[c], r1 = rs[c + 1];
                         float p0 = ex2_approx(fmaf(__uint_as_float(sv[c >> 4][c & 15]), p.c1, -r0.x));
                         float p1 = ex2_approx(fmaf(__uint_as_float(sv[c >> 4][(c & 15) + 1]), p.c1, -r1.x));
-                        if ((unsigned)(qc0 + c - key) >= (unsigned)p.W) p0 = 0.f;
-                        if ((unsigned)(qc0 + c + 1 - key) >= (unsigned)p.W) p1 = 0.f;
+                        if ((unsigned)(qc0 + c - key) >= (unsigned)p.W || (DOC && qc0 + c > de)) p0 = 0.f;
+                        if ((unsigned)(qc0 + c + 1 - key) >= (unsigned)p.W || (DOC && qc0 + c + 1 > de)) p1 = 0.f;
                         pv[c] = p0;
                         pv[c + 1] = p1;
                         pp[c >> 1] = pack_bf16x2(p0, p1);

@@ -39,16 +39,6 @@
 // the unrounded sum.  P is rounded to bf16 toward zero (one byte-permute per pair); because the
 // normaliser is the sum of the same rounded values, the rounding bias cancels in the weights.
 // One exponential in four is evaluated by a polynomial on the FMA pipe to offload the MUFU unit.
-//
-// Query prologue inside the kernel (QPRO).  With QPRO the producer loads the RAW query tile and the
-// softmax warps apply RoPE + RMS to it in shared memory (rope_exact.cuh, thread (row r, quarter c)
-// owning the rotation pairs of quarter c of row r; the four fp64 partial sums of squares of a row
-// meet in shared memory) before the MMA thread copies it into tensor memory, so qhat never goes
-// through HBM; its bits equal those of the standalone prologue kernel.  The softmax warps transform the next item's tile right after the last softmax tile of the
-// current item, while the tensor pipe runs that item's last PV product, and write the current
-// item's output afterwards; the next item's first score product then follows the PV product on the
-// pipe without a gap.  Without QPRO the query tile in HBM is already normalised (the fused
-// projection path and the staged entry point).
 #pragma once
 
 #include <cuda.h>
@@ -56,7 +46,6 @@
 #include <cstdint>
 
 #include "ptx.cuh"
-#include "rope_exact.cuh"
 
 namespace swa {
 
@@ -74,10 +63,9 @@ struct FwdCfg {
     static constexpr int SMEM_OUT = TILE_BYTES;        // output tile staged for the TMA store
     static constexpr int SMEM_BAR = 512;
     static constexpr int SMEM_LX = 4 * 128 * 8;        // row-sum exchange between the four threads of a row
-    static constexpr int SMEM_QX = 2 * 4 * 128 * 8;    // fp64 query sums of squares, double-buffered by item
     // Dynamic shared memory is declared 1024-byte aligned (the 128-byte swizzle atom repeats every
     // 1024 bytes); the kernel checks the alignment on entry instead of reserving slack for it.
-    static constexpr int SMEM_TOTAL = SMEM_Q + SMEM_KV + SMEM_OUT + SMEM_BAR + SMEM_LX + SMEM_QX;
+    static constexpr int SMEM_TOTAL = SMEM_Q + SMEM_KV + SMEM_OUT + SMEM_BAR + SMEM_LX;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_O = NSB * 128;
     static constexpr uint32_t COL_Q = COL_O + D;       // Q as bf16 pairs: D / 2 columns
@@ -99,9 +87,6 @@ struct FwdParams {
     float* lse;            // (B,H,T) or null
     int* sched;            // [0] next item, [1] CTAs done; zero before the launch, reset after
     unsigned long long wait_limit_ns;
-    const double2* tab64;  // fp64 RoPE table (cos, sin) per (t, i) (QPRO)
-    double inv_d;          // 1 / D (QPRO)
-    double eps;            // RMS epsilon (QPRO)
     const int* dstart;     // (B, T) start of each position's document (document mask), or null
 };
 
@@ -109,7 +94,7 @@ struct FwdParams {
 enum : unsigned int {
     kSiteQFull = 1, kSiteKvEmpty = 2, kSiteKvFull = 3, kSiteSFull = 4, kSitePFull = 5,
     kSiteOFull = 6, kSiteDrain = 7, kSiteQEmpty = 8, kSiteOEmpty = 9, kSiteItem = 10,
-    kSiteRowSum = 11, kSiteOStage = 12, kSiteQSum = 13, kSiteQReady = 14
+    kSiteRowSum = 11, kSiteOStage = 12
 };
 
 // Decoded work item: query tile [q0, q0 + 127] of (b, h) and the key tiles lo..hi of its band.
@@ -209,9 +194,8 @@ __device__ __forceinline__ uint32_t softmax_pair_poly(uint32_t s0, uint32_t s1, 
     return w;
 }
 
-// 576 threads, one CTA per SM: 112 registers per thread fit the register file (576 x 112 <= 64 K).
-template <int D, bool QPRO, bool DOC = false>
-__global__ void __maxnreg__(112)
+template <int D, bool DOC = false>
+__global__ void __launch_bounds__(576, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                     const FwdParams p) {
@@ -241,13 +225,10 @@ __global__ void __maxnreg__(112)
     uint64_t* b_pfull = bars + 13 + C::NSB;      // [NSB]
     uint64_t* b_kvfull = bars + 13 + 2 * C::NSB;            // [NS]
     uint64_t* b_kvempty = bars + 13 + 2 * C::NSB + C::NS;   // [NS]
-    uint64_t* b_qss = bars + 13 + 2 * C::NSB + 2 * C::NS;        // query partial sums posted (QPRO)
-    uint64_t* b_qready = b_qss + 1;                               // query tile normalised (QPRO)
-    int* s_item = reinterpret_cast<int*>(b_qready + 1);           // [2]
+    int* s_item = reinterpret_cast<int*>(bars + 13 + 2 * C::NSB + 2 * C::NS);   // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_item + 2);
     float2* s_lx = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(bars) + C::SMEM_BAR);   // [4][128]
-    double* s_qx = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(s_lx) + C::SMEM_LX);   // [2][4][128]
-    static_assert(13 + 2 * C::NSB + 2 * C::NS + 2 <= (C::SMEM_BAR - 16) / 8, "barrier area");
+    static_assert(13 + 2 * C::NSB + 2 * C::NS <= (C::SMEM_BAR - 16) / 8, "barrier area");
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -280,8 +261,6 @@ __global__ void __maxnreg__(112)
             mbar_init(smem_u32(b_kvfull + s), 1);
             mbar_init(smem_u32(b_kvempty + s), 1);
         }
-        mbar_init(smem_u32(b_qss), C::SOFTMAX_THREADS);
-        mbar_init(smem_u32(b_qready), C::SOFTMAX_THREADS);
         fence_barrier_init();
     }
     if (warp == kMmaWarp) {
@@ -435,14 +414,7 @@ __global__ void __maxnreg__(112)
                 const Item m = decode_item(p, it);
                 // Q into tensor memory (after the previous item's score products on the same pipe),
                 // then its shared-memory buffer goes back to the producer.
-                if (QPRO) {
-                    // the softmax warps wrote the normalised tile (generic proxy, fenced to the async
-                    // proxy before their arrive)
-                    if (!(ok = mbar_wait(smem_u32(b_qready), uses & 1u, lim, kSiteQReady))) break;
-                    tc_fence_after();
-                } else {
-                    if (!(ok = mbar_wait(smem_u32(b_qfull), uses & 1u, lim, kSiteQFull))) break;
-                }
+                if (!(ok = mbar_wait(smem_u32(b_qfull), uses & 1u, lim, kSiteQFull))) break;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     tmem_cp_128x256b(tmem + C::COL_Q + 8u * kk,
@@ -493,54 +465,8 @@ __global__ void __maxnreg__(112)
             return ok ? v : -1;
         };
 
-        // RoPE + RMS of the k-th item's raw query tile in shared memory (QPRO).  This thread: row r,
-        // rotation pairs [cq QP, cq QP + QP), i.e. the QP elements from column cq QP and the QP
-        // elements from column D/2 + cq QP, in the tile's 128-byte-swizzled layout.
-        auto q_transform = [&](const Item& mq, uint32_t kk) -> bool {
-            constexpr int QP = D / 8;
-            constexpr int NW = QP / 8;                  // 16-byte words per half (2 or 1)
-            const int t = min(mq.q0 + r, p.T - 1);      // rows past T hold zeros; any table row does
-            uint32_t offa[NW], offb[NW];
-#pragma unroll
-            for (int e = 0; e < NW; ++e) {
-                // element column -> (128-byte chunk, 16-byte unit)
-                const int ca = cq * QP + 8 * e, cb = D / 2 + cq * QP + 8 * e;
-                offa[e] = (uint32_t)((ca >> 6) * C::CHUNK_BYTES + r * 128 + ((((ca & 63) >> 3) ^ (r & 7)) << 4));
-                offb[e] = (uint32_t)((cb >> 6) * C::CHUNK_BYTES + r * 128 + ((((cb & 63) >> 3) ^ (r & 7)) << 4));
-            }
-            const double2* tab = p.tab64 + (long long)t * (D / 2) + cq * QP;
-            // warm this thread's table entries while the tile is in flight
-#pragma unroll
-            for (int e = 0; e < QP; e += 4) asm volatile("prefetch.global.L1 [%0];" ::"l"(tab + e));
-            bool w = mbar_wait(smem_u32(b_qfull), kk & 1u, lim, kSiteQFull);
-            if (!__all_sync(0xffffffffu, w)) return false;
-            uint4 qa[NW], qb[NW];
-#pragma unroll
-            for (int e = 0; e < NW; ++e) {
-                qa[e] = *reinterpret_cast<const uint4*>(sQ + offa[e]);
-                qb[e] = *reinterpret_cast<const uint4*>(sQ + offb[e]);
-            }
-            double* xs = s_qx + (kk & 1u) * 512u;
-            xs[cq * 128 + r] = quarter_sumsq64<NW>(qa, qb);
-            mbar_arrive(smem_u32(b_qss));
-            w = mbar_wait(smem_u32(b_qss), kk & 1u, lim, kSiteQSum);
-            if (!__all_sync(0xffffffffu, w)) return false;
-            const double rs = rms_scale64(xs[r], xs[128 + r], xs[256 + r], xs[384 + r], p.inv_d, p.eps);
-            uint4 oa[NW], ob[NW];
-            rope_quarter64<NW>(qa, qb, tab, rs, oa, ob);
-#pragma unroll
-            for (int e = 0; e < NW; ++e) {
-                *reinterpret_cast<uint4*>(sQ + offa[e]) = oa[e];
-                *reinterpret_cast<uint4*>(sQ + offb[e]) = ob[e];
-            }
-            fence_proxy_async_smem();                   // the tensor core reads the tile next
-            mbar_arrive(smem_u32(b_qready));
-            return true;
-        };
-
         uint32_t k = 0;
         int it = fetch(0);
-        if (QPRO && it >= 0) ok = q_transform(decode_item(p, it), 0);
         while (ok && it >= 0) {
             const Item m = decode_item(p, it);
             const int qi = m.q0 + r;              // this thread's query position
@@ -614,10 +540,9 @@ __global__ void __maxnreg__(112)
                 l += u0 + u1;
                 lr += w0 + w1;
             }
-            // The next item's query tile, while the tensor pipe runs this item's last PV product.
+            // The next item (read early: its slot frees the scheduler's next publication).
             ++k;
             const int it_next = fetch(k);
-            if (QPRO && ok && it_next >= 0) ok = q_transform(decode_item(p, it_next), k);
             if (!ok) break;
             {
                 const bool w = mbar_wait(smem_u32(b_ofull), o_uses & 1u, lim, kSiteOFull);

@@ -160,12 +160,14 @@ struct Raw<2> {
 // per warp (keys w, w+4, ..., w+28 of the block): the warp loads their K and V pieces first, then
 // reduces the eight dot products together, so sixteen loads per lane are in flight at once.
 // Partial results: part[(row * n_chunks + chunk) * (D + 2) + d] = sum_j p_j v'_j[d],
-// [.. + D] = sum_j p_j.
+// [.. + D] = sum_j p_j.  With doc_start (one int per sequence: the first position of the new
+// token's document; document-boundary mask) the keys before it are skipped: a chunk that lies
+// entirely before it writes zeros.
 template <int D>
 __global__ void __launch_bounds__(128) decode_attn_kernel(
     const __nv_bfloat16* __restrict__ qh, const __nv_bfloat16* __restrict__ k_cache,
     const __nv_bfloat16* __restrict__ v_cache, float* __restrict__ part, int H, int Hkv, int Tmax,
-    int lo, int n_keys, int n_chunks, float c1, float c2) {
+    int lo, int n_keys, int n_chunks, float c1, float c2, const int* __restrict__ doc_start) {
     constexpr int DPL = D / 32;          // features per lane
     constexpr int U = 8;                 // keys per warp per iteration
     const int row = (int)(blockIdx.x / (unsigned)n_chunks);    // b*H + h
@@ -185,8 +187,10 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
 #pragma unroll
     for (int e = 0; e < DPL; ++e) o[e] = 0.f;
     float l = 0.f;
-    const int key_begin = chunk * kDecodeChunk;
-    const int key_end = min(key_begin + kDecodeChunk, n_keys);
+    // first key of this chunk, past the document start if there is one (key index j is position lo + j)
+    const int jmin = doc_start != nullptr ? max(0, min(__ldg(doc_start + b), lo + n_keys - 1) - lo) : 0;
+    const int key_begin = max(chunk * kDecodeChunk, jmin);
+    const int key_end = min(chunk * kDecodeChunk + kDecodeChunk, n_keys);
     const int hk = h / (H / Hkv);                           // key/value head of this query head
     const long long stride = (long long)Hkv * D;            // between consecutive positions
     const __nv_bfloat16* kbase = k_cache + ((long long)b * Tmax + lo) * stride + (long long)hk * D + lane * DPL;

@@ -65,7 +65,7 @@ __global__ void gate_kernel(const __nv_bfloat16* __restrict__ gate_x, const __nv
 
 // RoPE tables, one entry per (t, i):
 //   tab32[t*D/2 + i] = (c_hi, c_lo, s_hi, s_lo) fp32, each piece with a 16-bit significand;
-//   tab64[t*D/2 + i] = (cos, sin) fp64 (the prologue of rope_exact.cuh; the fallback here).
+//   tab64[t*D/2 + i] = (cos, sin) fp64, read only by the fp64 path.
 __device__ __forceinline__ float round_sig16(double x) {
     // nearest float with at most 16 significant bits (8 low mantissa bits cleared)
     const float f = (float)x;
@@ -215,6 +215,99 @@ __device__ __forceinline__ uint2 gated_add4(const uint2& vw, const uint2& ew, fl
                         ((uint32_t)bf16_rn_bits(fma(g64, (double)e4[e + 1], (double)v[e + 1])) << 16);
     }
     return make_uint2(w[0], w[1]);
+}
+
+// PARTS selects the outputs: bit 0 qhat, bit 1 khat and v' (v' only on value-embedding layers).
+// The multi-head layer runs both in one pass (PARTS = 3, rows (b,t,h) of all inputs); with
+// grouped-query attention the query rows (H heads) and the key/value rows (Hkv heads) are two
+// passes over their own row sets, `H` being that pass's head count.
+template <int D, bool HAS_VE, int PARTS = 3>
+__global__ void __launch_bounds__(256, 3) prologue_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+    const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ ve,
+    const float2* __restrict__ gate,
+    __nv_bfloat16* __restrict__ qh, __nv_bfloat16* __restrict__ kh, __nv_bfloat16* __restrict__ vp,
+    const float4* __restrict__ tab32, const double2* __restrict__ tab64, int* __restrict__ sched,
+    int n_rows, int T, int H, FastDiv divT, FastDiv divH, double eps) {
+    constexpr int TPR = D / 8;           // threads per row (16 or 8); divides 32
+    constexpr int LOG_TPR = (D == 128) ? 4 : 3;
+    constexpr int HALF = D / 2;
+    const long long gtid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    // Every thread of a warp runs the same number of iterations, so the shuffles always see the
+    // full warp; rows past the end are computed on zeros and not stored.
+    const long long n_iter = ((long long)n_rows * TPR + stride - 1) / stride;
+    // The attention kernel that follows takes its work items from this counter.
+    if (gtid == 0) {
+        sched[0] = 0;
+        sched[1] = 0;
+    }
+    for (long long it = 0; it < n_iter; ++it) {
+        const long long tid = gtid + it * stride;
+        const int row_raw = (int)(tid >> LOG_TPR);           // (b*T + t)*H + h, < 2^31
+        const int c = (int)(tid & (TPR - 1));
+        const bool valid = row_raw < n_rows;
+        const int row = valid ? row_raw : 0;
+        const int bt = fdiv(row, divH);
+        const int t = bt - fdiv(bt, divT) * T;
+        const int i0 = 4 * c;
+        const long long off = (long long)row * D;
+
+        // Every load of this row chunk is issued before any arithmetic.
+        constexpr bool DO_Q = (PARTS & 1) != 0, DO_KV = (PARTS & 2) != 0;
+        uint2 raw[8];
+        float2 gw = make_float2(0.f, 0.f);
+        if (valid) {
+            if (DO_Q) {
+                raw[0] = ldg_stream8(q + off + i0);
+                raw[1] = ldg_stream8(q + off + HALF + i0);
+            }
+            if (DO_KV) {
+                raw[2] = ldg_stream8(k + off + i0);
+                raw[3] = ldg_stream8(k + off + HALF + i0);
+            }
+            if (HAS_VE && DO_KV) {
+                raw[4] = ldg_stream8(v + off + i0);
+                raw[5] = ldg_stream8(v + off + HALF + i0);
+                raw[6] = ldg_stream8(ve + off + i0);
+                raw[7] = ldg_stream8(ve + off + HALF + i0);
+                gw = __ldg(gate + row);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) raw[e] = make_uint2(0u, 0u);
+        }
+        if (!DO_Q) raw[0] = raw[1] = make_uint2(0u, 0u);
+        if (!DO_KV || !HAS_VE)
+#pragma unroll
+            for (int e = 4; e < 8; ++e) raw[e] = make_uint2(0u, 0u);
+        if (!DO_KV) raw[2] = raw[3] = make_uint2(0u, 0u);
+        float4 cs[4];
+        {
+            const float4* tp = tab32 + (long long)t * HALF + i0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) cs[e] = __ldg(tp + e);
+        }
+        const double2* t64 = tab64 + (long long)t * HALF + i0;
+        uint2 o0, o1, o2, o3;
+        if (DO_Q) rope_rms_pairs4<D>(raw[0], raw[1], cs, t64, eps, o0, o1);
+        if (DO_KV) rope_rms_pairs4<D>(raw[2], raw[3], cs, t64, eps, o2, o3);
+        if (valid) {
+            if (DO_Q) {
+                *reinterpret_cast<uint2*>(qh + off + i0) = o0;
+                *reinterpret_cast<uint2*>(qh + off + HALF + i0) = o1;
+            }
+            if (DO_KV) {
+                *reinterpret_cast<uint2*>(kh + off + i0) = o2;
+                *reinterpret_cast<uint2*>(kh + off + HALF + i0) = o3;
+            }
+            if (HAS_VE && DO_KV) {
+                const double g64 = (double)gw.x + (double)gw.y;
+                *reinterpret_cast<uint2*>(vp + off + i0) = gated_add4(raw[4], raw[6], gw.x, gw.y, g64);
+                *reinterpret_cast<uint2*>(vp + off + HALF + i0) = gated_add4(raw[5], raw[7], gw.x, gw.y, g64);
+            }
+        }
+    }
 }
 
 }  // namespace swa

@@ -18,7 +18,6 @@
 #include "decode.cuh"
 #include "prologue.cuh"
 #include "qkv_gemm.cuh"
-#include "rope_exact.cuh"
 #include "docmask.cuh"
 
 // ------------------------------------------------------------------ failure-detection self-test
@@ -185,10 +184,6 @@ int device_ready(int* dev_out) {
                                      swa::FwdCfg<64>::SMEM_TOTAL) != cudaSuccess ||
                 cudaFuncSetAttribute(swa::attn_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      swa::FwdCfg<128>::SMEM_TOTAL) != cudaSuccess ||
-                cudaFuncSetAttribute(swa::attn_fwd_kernel<64, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     swa::FwdCfg<64>::SMEM_TOTAL) != cudaSuccess ||
-                cudaFuncSetAttribute(swa::attn_fwd_kernel<128, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     swa::FwdCfg<128>::SMEM_TOTAL) != cudaSuccess ||
                 cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<64>, (cudaFuncAttribute)smem_attr,
                                      swa::BwdCfg<64>::DQ_SMEM) != cudaSuccess ||
                 cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<128>, (cudaFuncAttribute)smem_attr,
@@ -196,6 +191,14 @@ int device_ready(int* dev_out) {
                 cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<64>, (cudaFuncAttribute)smem_attr,
                                      swa::BwdCfg<64>::KV_SMEM) != cudaSuccess ||
                 cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<128>, (cudaFuncAttribute)smem_attr,
+                                     swa::BwdCfg<128>::KV_SMEM) != cudaSuccess ||
+                cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<64, true>, (cudaFuncAttribute)smem_attr,
+                                     swa::BwdCfg<64>::DQ_SMEM) != cudaSuccess ||
+                cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<128, true>, (cudaFuncAttribute)smem_attr,
+                                     swa::BwdCfg<128>::DQ_SMEM) != cudaSuccess ||
+                cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<64, true>, (cudaFuncAttribute)smem_attr,
+                                     swa::BwdCfg<64>::KV_SMEM) != cudaSuccess ||
+                cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<128, true>, (cudaFuncAttribute)smem_attr,
                                      swa::BwdCfg<128>::KV_SMEM) != cudaSuccess) {
                 cudaGetLastError();
                 checked[dev] = 0;
@@ -268,65 +271,83 @@ int launch_rope_table(uint8_t* ws, const WsLayout& L, const Shape& s, float rope
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
-// The prologue (rope_exact.cuh): the gate on value-embedding layers, then one launch whose blocks
-// write qhat (when q is given), khat and v' (value-embedding layers) into the workspace, each
-// element exactly rounded.  It also zeroes the attention kernel's scheduler counters.
 int launch_prologue(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
                     const void* Wg, uint8_t* ws, const WsLayout& L, const Shape& s, float eps,
                     cudaStream_t st) {
     using bf = __nv_bfloat16;
     const bool has_ve = ve != nullptr;
+    const int n_rows = s.B * s.T * s.H;
     const int n_kv_rows = s.B * s.T * s.Hkv;
+    const swa::FastDiv divH = make_fastdiv(s.H), divT = make_fastdiv(s.T);
     float2* gate = reinterpret_cast<float2*>(ws + L.gate);
     if (has_ve) {
         const int gblocks = (int)std::min<long long>(((long long)n_kv_rows + 255) / 256, 148ll * 8);
         swa::gate_kernel<<<gblocks, 256, 0, st>>>(static_cast<const bf*>(gate_x), static_cast<const bf*>(Wg),
                                                    gate, n_kv_rows, s.Hkv, make_fastdiv(s.Hkv), 32);
     }
-    swa::ExactProParams p{};
-    p.q = static_cast<const bf*>(q);
-    p.k = static_cast<const bf*>(k);
-    p.v = static_cast<const bf*>(v);
-    p.ve = static_cast<const bf*>(ve);
-    p.gate = gate;
-    p.qh = reinterpret_cast<bf*>(ws + L.qh);
-    p.kh = reinterpret_cast<bf*>(ws + L.kh);
-    p.vp = reinterpret_cast<bf*>(ws + L.vp);
-    p.tab64 = reinterpret_cast<const double2*>(ws + L.tab64);
-    p.n_q = q ? s.B * s.T * s.H : 0;
-    p.n_k = n_kv_rows;
-    p.n_v = has_ve ? n_kv_rows : 0;
-    p.nb_q = (p.n_q + 63) / 64;
-    p.nb_k = (p.n_k + 63) / 64;
-    const long long nb_v = ((long long)p.n_v * s.D / 32 + 255) / 256;
-    p.H = s.H;
-    p.Hkv = s.Hkv;
-    p.T = s.T;
-    p.inv_d = 1.0 / (double)s.D;
-    p.eps = (double)eps;
-    p.sched = reinterpret_cast<int*>(ws + L.sched);
-    const long long blocks = (long long)p.nb_q + p.nb_k + nb_v;
-    if (blocks >= (1ll << 31)) return SWA_ERR_UNSUPPORTED;
+    const long long threads_total = (long long)n_rows * (s.D / 8);
+    const int threads = 256;
+    const long long blocks = std::min<long long>((threads_total + threads - 1) / threads, 148ll * 3 * 4);
+    const bf* qp = static_cast<const bf*>(q);
+    const bf* kp = static_cast<const bf*>(k);
+    const bf* vpi = static_cast<const bf*>(v);
+    const bf* vep = static_cast<const bf*>(ve);
+    bf* qh = reinterpret_cast<bf*>(ws + L.qh);
+    bf* kh = reinterpret_cast<bf*>(ws + L.kh);
+    bf* vp = reinterpret_cast<bf*>(ws + L.vp);
+    const float4* t32 = reinterpret_cast<const float4*>(ws + L.tab32);
+    const double2* t64 = reinterpret_cast<const double2*>(ws + L.tab64);
+    int* sched = reinterpret_cast<int*>(ws + L.sched);
+    const unsigned g = (unsigned)blocks;
+    const double e = (double)eps;
+    if (s.Hkv != s.H) {
+        // Grouped-query attention: the query rows (H heads) and the key/value rows (Hkv heads) are
+        // two passes over their own rows.
+        const swa::FastDiv divK = make_fastdiv(s.Hkv);
+        const unsigned gk = (unsigned)std::min<long long>(((long long)n_kv_rows * (s.D / 8) + threads - 1) / threads,
+                                                          148ll * 3 * 4);
+#define SWA_PRO_GQA(DD, VE)                                                                                  \
+    swa::prologue_kernel<DD, VE, 1><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, \
+                                                           n_rows, s.T, s.H, divT, divH, e);                 \
+    swa::prologue_kernel<DD, VE, 2><<<gk, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, \
+                                                            n_kv_rows, s.T, s.Hkv, divT, divK, e)
+        if (s.D == 128) {
+            if (has_ve) {
+                SWA_PRO_GQA(128, true);
+            } else {
+                SWA_PRO_GQA(128, false);
+            }
+        } else {
+            if (has_ve) {
+                SWA_PRO_GQA(64, true);
+            } else {
+                SWA_PRO_GQA(64, false);
+            }
+        }
+#undef SWA_PRO_GQA
+        return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+    }
     if (s.D == 128) {
-        if (has_ve) swa::prologue_exact_kernel<128, true><<<(unsigned)blocks, 256, 0, st>>>(p);
-        else swa::prologue_exact_kernel<128, false><<<(unsigned)blocks, 256, 0, st>>>(p);
+        if (has_ve)
+            swa::prologue_kernel<128, true><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, divT, divH, e);
+        else
+            swa::prologue_kernel<128, false><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, divT, divH, e);
     } else {
-        if (has_ve) swa::prologue_exact_kernel<64, true><<<(unsigned)blocks, 256, 0, st>>>(p);
-        else swa::prologue_exact_kernel<64, false><<<(unsigned)blocks, 256, 0, st>>>(p);
+        if (has_ve)
+            swa::prologue_kernel<64, true><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, divT, divH, e);
+        else
+            swa::prologue_kernel<64, false><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, divT, divH, e);
     }
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
-// The attention kernel.  q_raw non-null: the kernel reads the raw q (B,T,H,D) and applies RoPE + RMS
-// to each query tile itself (the prologue's exact arithmetic; the RoPE table must be in the
-// workspace); q_raw null: it reads qhat from the workspace.  khat (and v' on value-embedding
-// layers) always come from the workspace.
-int launch_attention(int dev, const void* q_raw, const void* v, bool has_ve, void* out, float* lse,
-                     const Shape& s, int window, float eps, uint8_t* ws, const WsLayout& L, cudaStream_t st,
-                     const int* dstart = nullptr) {
+// The attention kernel on the workspace's qhat, khat (and v' on value-embedding layers; `v` itself
+// otherwise).  dstart: the document starts (B, T) of a document-masked call, or null.
+int launch_attention(int dev, const void* v, bool has_ve, void* out, float* lse, const Shape& s, int window,
+                     uint8_t* ws, const WsLayout& L, cudaStream_t st, const int* dstart = nullptr) {
     CUtensorMap tq, tk, tv, to;
     const void* vsrc = has_ve ? static_cast<const void*>(ws + L.vp) : v;
-    const void* qsrc = q_raw ? q_raw : static_cast<const void*>(ws + L.qh);
+    const void* qsrc = ws + L.qh;
     // q and out have H heads, k and v Hkv heads
     if (!make_tile_map(&tq, qsrc, s, s.H) || !make_tile_map(&tk, ws + L.kh, s, s.Hkv) ||
         !make_tile_map(&tv, vsrc, s, s.Hkv) || !make_tile_map(&to, out, s, s.H))
@@ -351,20 +372,14 @@ int launch_attention(int dev, const void* q_raw, const void* v, bool has_ve, voi
     p.lse = lse;
     p.sched = reinterpret_cast<int*>(ws + L.sched);
     p.wait_limit_ns = wait_limit_ns();
-    p.tab64 = reinterpret_cast<const double2*>(ws + L.tab64);
-    p.inv_d = 1.0 / (double)s.D;
-    p.eps = (double)eps;
     p.dstart = dstart;
     const dim3 grid((unsigned)std::min(p.n_items, g_num_sms[dev]));
-#define SWA_ATTN(DD, QP, DC) \
-    swa::attn_fwd_kernel<DD, QP, DC><<<grid, swa::FwdCfg<DD>::THREADS, swa::FwdCfg<DD>::SMEM_TOTAL, st>>>(tq, tk, tv, to, p)
-    if (dstart) {
-        if (!q_raw) return SWA_ERR_INVALID_ARG;
-        if (s.D == 128) SWA_ATTN(128, true, true); else SWA_ATTN(64, true, true);
-    } else if (s.D == 128) {
-        if (q_raw) SWA_ATTN(128, true, false); else SWA_ATTN(128, false, false);
+#define SWA_ATTN(DD, DC) \
+    swa::attn_fwd_kernel<DD, DC><<<grid, swa::FwdCfg<DD>::THREADS, swa::FwdCfg<DD>::SMEM_TOTAL, st>>>(tq, tk, tv, to, p)
+    if (s.D == 128) {
+        if (dstart) SWA_ATTN(128, true); else SWA_ATTN(128, false);
     } else {
-        if (q_raw) SWA_ATTN(64, true, false); else SWA_ATTN(64, false, false);
+        if (dstart) SWA_ATTN(64, true); else SWA_ATTN(64, false);
     }
 #undef SWA_ATTN
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
@@ -468,7 +483,7 @@ int launch_qkv(int dev, const void* x, const void* Wqkv, const void* ve, const v
 // layers only).  The backward kernels' scheduler counters are ints 4..7 of the counter section.
 struct BwdLayout {
     WsLayout f;
-    size_t rowstat, dqh, dkh, dvp, dz, wgp, total;
+    size_t rowstat, dqh, dkh, dvp, dz, wgp, dstart, dend, total;
     int Tp, wg_blocks, wg_rows;
 };
 
@@ -493,6 +508,11 @@ BwdLayout bwd_layout(const Shape& s, bool has_ve) {
     o += has_ve ? round_up((size_t)n_bt * s.Hkv * 4) : 0;
     w.wgp = o;
     o += has_ve ? round_up((size_t)w.wg_blocks * 32 * s.Hkv * 4) : 0;
+    // document starts and ends (document-masked calls; a few bytes per position, always reserved)
+    w.dstart = o;
+    o += round_up((size_t)n_bt * 4);
+    w.dend = o;
+    o += round_up((size_t)n_bt * 4);
     w.total = o;
     return w;
 }
@@ -501,7 +521,7 @@ int launch_backward(int dev, const void* q, const void* k, const void* v, const 
                     const void* gate_x, const void* Wg, const void* out, const float* lse,
                     const void* dout, const float* dlse, void* dq, void* dk, void* dv, void* dve,
                     float* dgate_x, float* dWg, const Shape& s, int window, float rope_base, float eps,
-                    uint8_t* ws, const BwdLayout& L, cudaStream_t st) {
+                    uint8_t* ws, const BwdLayout& L, cudaStream_t st, const int* doc = nullptr) {
     using bf = __nv_bfloat16;
     const bool has_ve = ve != nullptr;
     int rc;
@@ -543,6 +563,12 @@ int launch_backward(int dev, const void* q, const void* k, const void* v, const 
     p.dkh = reinterpret_cast<float*>(ws + L.dkh);
     p.dvp = reinterpret_cast<float*>(ws + L.dvp);
     p.wait_limit_ns = wait_limit_ns();
+    if (doc) {
+        p.dstart = reinterpret_cast<int*>(ws + L.dstart);
+        p.dend = reinterpret_cast<int*>(ws + L.dend);
+        swa::doc_start_kernel<<<s.B, 1024, 0, st>>>(doc, reinterpret_cast<int*>(ws + L.dstart),
+                                                   reinterpret_cast<int*>(ws + L.dend), s.T);
+    }
     const long long slice_bytes = 4ll * s.T * s.D;   // two bf16 (T, D) slices
     // Query tiles: chunks of (b, h) slices whose K and V' fit in ~40 MB of L2.
     swa::BwdParams pq = p;
@@ -557,15 +583,18 @@ int launch_backward(int dev, const void* q, const void* k, const void* v, const 
     pk.sched = sched4 + 2;
     const dim3 gq((unsigned)std::min(pq.n_items, g_num_sms[dev]));
     const dim3 gk((unsigned)std::min(pk.n_items, g_num_sms[dev]));
+#define SWA_BWD_TC(DD, DC)                                                                                  \
+    do {                                                                                                    \
+        using C = swa::BwdCfg<DD>;                                                                          \
+        swa::attn_bwd_dq_kernel<DD, DC><<<gq, C::THREADS, C::DQ_SMEM, st>>>(tq, tk, tv, tdo, pq);            \
+        swa::attn_bwd_dkv_kernel<DD, DC><<<gk, C::THREADS, C::KV_SMEM, st>>>(tq, tk, tv, tdo, pk);           \
+    } while (0)
     if (s.D == 128) {
-        using C = swa::BwdCfg<128>;
-        swa::attn_bwd_dq_kernel<128><<<gq, C::THREADS, C::DQ_SMEM, st>>>(tq, tk, tv, tdo, pq);
-        swa::attn_bwd_dkv_kernel<128><<<gk, C::THREADS, C::KV_SMEM, st>>>(tq, tk, tv, tdo, pk);
+        if (doc) SWA_BWD_TC(128, true); else SWA_BWD_TC(128, false);
     } else {
-        using C = swa::BwdCfg<64>;
-        swa::attn_bwd_dq_kernel<64><<<gq, C::THREADS, C::DQ_SMEM, st>>>(tq, tk, tv, tdo, pq);
-        swa::attn_bwd_dkv_kernel<64><<<gk, C::THREADS, C::KV_SMEM, st>>>(tq, tk, tv, tdo, pk);
+        if (doc) SWA_BWD_TC(64, true); else SWA_BWD_TC(64, false);
     }
+#undef SWA_BWD_TC
 
     // The prologue in reverse.
     const double2* t64 = reinterpret_cast<const double2*>(ws + L.f.tab64);
@@ -682,8 +711,7 @@ int swa_attn_prologue(const void* q, const void* k, const void* v, const void* v
                       swa_stream_t stream) {
     Shape s;
     int rc = check_sizes(B, T, H, D, &s);
-    // q may be null (khat and v' only); the others follow the layer's rules
-    if (rc == SWA_OK) rc = check_layer_args(q ? q : k, k, v, ve, gate_x, Wg, rope_base, eps);
+    if (rc == SWA_OK) rc = check_layer_args(q, k, v, ve, gate_x, Wg, rope_base, eps);
     if (rc != SWA_OK) return rc;
     if (!workspace) return SWA_ERR_INVALID_ARG;
     if (!aligned(workspace, 16)) return SWA_ERR_MISALIGNED;
@@ -707,8 +735,8 @@ int swa_attn_attention(const void* v, int has_ve, void* out, float* lse, int B, 
     if (ws_bytes < L.total) return SWA_ERR_NO_MEMORY;
     int dev;
     if ((rc = device_ready(&dev)) != SWA_OK) return rc;
-    return launch_attention(dev, nullptr, v, has_ve != 0, out, lse, s, window, 0.f,
-                            static_cast<uint8_t*>(workspace), L, reinterpret_cast<cudaStream_t>(stream));
+    return launch_attention(dev, v, has_ve != 0, out, lse, s, window, static_cast<uint8_t*>(workspace), L,
+                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 int swa_attn_fwd_ws(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
@@ -722,29 +750,9 @@ int swa_attn_fwd_ws(const void* q, const void* k, const void* v, const void* ve,
     if (rc != SWA_OK) return rc;
     rc = swa_attn_rope_table(B, T, H, D, ve != nullptr, rope_base, workspace, ws_bytes, stream);
     if (rc != SWA_OK) return rc;
-    rc = swa_attn_prologue(nullptr, k, v, ve, gate_x, Wg, B, T, H, D, rope_base, eps, workspace, ws_bytes,
-                           stream);
+    rc = swa_attn_prologue(q, k, v, ve, gate_x, Wg, B, T, H, D, rope_base, eps, workspace, ws_bytes, stream);
     if (rc != SWA_OK) return rc;
-    return swa_attn_attention_q(q, v, ve != nullptr, out, lse, B, T, H, D, window, eps, workspace,
-                                ws_bytes, stream);
-}
-
-int swa_attn_attention_q(const void* q, const void* v, int has_ve, void* out, float* lse, int B, int T,
-                         int H, int D, int window, float eps, void* workspace, size_t ws_bytes,
-                         swa_stream_t stream) {
-    Shape s;
-    int rc = check_sizes(B, T, H, D, &s);
-    if (rc != SWA_OK) return rc;
-    if (!q || !workspace || (!has_ve && !v)) return SWA_ERR_INVALID_ARG;
-    if (!std::isfinite(eps) || eps < 0.f) return SWA_ERR_INVALID_ARG;
-    if ((rc = check_outputs(out, lse)) != SWA_OK) return rc;
-    if (!aligned(q, 16) || !aligned(workspace, 16) || (!has_ve && !aligned(v, 16))) return SWA_ERR_MISALIGNED;
-    const WsLayout L = ws_layout(s, has_ve != 0);
-    if (ws_bytes < L.total) return SWA_ERR_NO_MEMORY;
-    int dev;
-    if ((rc = device_ready(&dev)) != SWA_OK) return rc;
-    return launch_attention(dev, q, v, has_ve != 0, out, lse, s, window, eps, static_cast<uint8_t*>(workspace),
-                            L, reinterpret_cast<cudaStream_t>(stream));
+    return swa_attn_attention(v, ve != nullptr, out, lse, B, T, H, D, window, workspace, ws_bytes, stream);
 }
 
 }  // extern "C"
@@ -804,13 +812,13 @@ int fwd_library_ws(const void* q, const void* k, const void* v, const void* ve, 
     }
     int* dstart = doc ? reinterpret_cast<int*>(ws + L.dstart) : nullptr;
     if (doc) {
-        swa::doc_start_kernel<<<s.B, 1024, 0, st>>>(doc, dstart, s.T);
+        swa::doc_start_kernel<<<s.B, 1024, 0, st>>>(doc, dstart, nullptr, s.T);
         rc = cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
     } else {
         rc = SWA_OK;
     }
-    if (rc == SWA_OK) rc = launch_prologue(nullptr, k, v, ve, gate_x, Wg, ws, L, s, eps, st);
-    if (rc == SWA_OK) rc = launch_attention(dev, q, v, has_ve, out, lse, s, window, eps, ws, L, st, dstart);
+    if (rc == SWA_OK) rc = launch_prologue(q, k, v, ve, gate_x, Wg, ws, L, s, eps, st);
+    if (rc == SWA_OK) rc = launch_attention(dev, v, has_ve, out, lse, s, window, ws, L, st, dstart);
     // Recorded after whatever was enqueued, also on failure, so the next call orders after it.
     if (cudaEventRecord(c.last_use, st) != cudaSuccess) {
         cudaGetLastError();
@@ -906,7 +914,7 @@ int swa_attn_fwd_x(const void* x, const void* Wqkv, const void* ve, const void* 
     if ((rc = launch_qkv(dev, x, Wqkv, ve, Wg, C, s, eps, ws, L, ws + L.qh, ws + L.kh, ws + L.vp,
                          reinterpret_cast<int*>(ws + L.sched), st)) != SWA_OK)
         return rc;
-    return launch_attention(dev, nullptr, nullptr, true, out, lse, s, window, 0.f, ws, L, st);
+    return launch_attention(dev, nullptr, true, out, lse, s, window, ws, L, st);
 }
 
 // ---------------------------------------------------------------------------- backward
@@ -917,11 +925,12 @@ size_t swa_attn_bwd_workspace_bytes(int B, int T, int H, int Hkv, int D, int has
     return bwd_layout(s, has_ve != 0).total;
 }
 
-int swa_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
-                     const void* Wg, const void* out, const float* lse, const void* dout,
+int swa_attn_bwd_doc(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                     const void* Wg, const int* doc, const void* out, const float* lse, const void* dout,
                      const float* dlse, void* dq, void* dk, void* dv, void* dve, float* dgate_x,
                      float* dWg, int B, int T, int H, int Hkv, int D, int window, float rope_base,
                      float eps, void* workspace, size_t ws_bytes, swa_stream_t stream) {
+    if (doc != nullptr && !aligned(doc, 4)) return SWA_ERR_MISALIGNED;
     Shape s;
     int rc = check_sizes(B, T, H, D, &s);
     if (rc == SWA_OK) rc = check_kv_heads(Hkv, &s);
@@ -941,7 +950,16 @@ int swa_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* ve
     if ((rc = device_ready(&dev)) != SWA_OK) return rc;
     return launch_backward(dev, q, k, v, ve, gate_x, Wg, out, lse, dout, dlse, dq, dk, dv, dve, dgate_x, dWg, s,
                            window, rope_base, eps, static_cast<uint8_t*>(workspace), L,
-                           reinterpret_cast<cudaStream_t>(stream));
+                           reinterpret_cast<cudaStream_t>(stream), doc);
+}
+
+int swa_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                     const void* Wg, const void* out, const float* lse, const void* dout,
+                     const float* dlse, void* dq, void* dk, void* dv, void* dve, float* dgate_x,
+                     float* dWg, int B, int T, int H, int Hkv, int D, int window, float rope_base,
+                     float eps, void* workspace, size_t ws_bytes, swa_stream_t stream) {
+    return swa_attn_bwd_doc(q, k, v, ve, gate_x, Wg, nullptr, out, lse, dout, dlse, dq, dk, dv, dve, dgate_x,
+                            dWg, B, T, H, Hkv, D, window, rope_base, eps, workspace, ws_bytes, stream);
 }
 
 int swa_attn_bwd(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
@@ -969,11 +987,12 @@ size_t swa_attn_decode_workspace_bytes(int B, int Tmax, int H, int D, int has_ve
     return round_up((size_t)rows * D * 2) + round_up((size_t)(rows * n_chunks * (D + 2)) * sizeof(float));
 }
 
-int swa_attn_decode_gqa(const void* q, const void* k, const void* v, const void* ve,
+int swa_attn_decode_doc(const void* q, const void* k, const void* v, const void* ve,
                         const void* gate_x, const void* Wg, void* k_cache, void* v_cache, int pos,
-                        void* out, float* lse, int B, int Tmax, int H, int Hkv, int D, int window,
-                        float rope_base, float eps, void* workspace, size_t ws_bytes,
+                        const int* doc_start, void* out, float* lse, int B, int Tmax, int H, int Hkv,
+                        int D, int window, float rope_base, float eps, void* workspace, size_t ws_bytes,
                         swa_stream_t stream) {
+    if (doc_start != nullptr && !aligned(doc_start, 4)) return SWA_ERR_MISALIGNED;
     Shape s;
     int rc = check_sizes(B, Tmax, H, D, &s);
     if (rc == SWA_OK) rc = check_kv_heads(Hkv, &s);
@@ -1045,13 +1064,24 @@ int swa_attn_decode_gqa(const void* q, const void* k, const void* v, const void*
     const bf* vcc = static_cast<const bf*>(v_cache);
     bf* o = static_cast<bf*>(out);
     if (D == 128) {
-        swa::decode_attn_kernel<128><<<grid, 128, 0, st>>>(qc, kcc, vcc, part, H, Hkv, Tmax, lo, n_keys, n_chunks, c1, c2);
+        swa::decode_attn_kernel<128><<<grid, 128, 0, st>>>(qc, kcc, vcc, part, H, Hkv, Tmax, lo, n_keys, n_chunks, c1, c2,
+                                                           doc_start);
         swa::decode_combine_kernel<128><<<rows, 128, 0, st>>>(part, o, lse, n_chunks, (float)m0);
     } else {
-        swa::decode_attn_kernel<64><<<grid, 128, 0, st>>>(qc, kcc, vcc, part, H, Hkv, Tmax, lo, n_keys, n_chunks, c1, c2);
+        swa::decode_attn_kernel<64><<<grid, 128, 0, st>>>(qc, kcc, vcc, part, H, Hkv, Tmax, lo, n_keys, n_chunks, c1, c2,
+                                                          doc_start);
         swa::decode_combine_kernel<64><<<rows, 64, 0, st>>>(part, o, lse, n_chunks, (float)m0);
     }
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+int swa_attn_decode_gqa(const void* q, const void* k, const void* v, const void* ve,
+                        const void* gate_x, const void* Wg, void* k_cache, void* v_cache, int pos,
+                        void* out, float* lse, int B, int Tmax, int H, int Hkv, int D, int window,
+                        float rope_base, float eps, void* workspace, size_t ws_bytes,
+                        swa_stream_t stream) {
+    return swa_attn_decode_doc(q, k, v, ve, gate_x, Wg, k_cache, v_cache, pos, nullptr, out, lse, B, Tmax, H, Hkv,
+                               D, window, rope_base, eps, workspace, ws_bytes, stream);
 }
 
 int swa_attn_decode(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
@@ -1146,6 +1176,6 @@ extern "C" int swa_attn_fwd_noalloc(const void* q, const void* k, const void* v,
     // tables, then khat / v' and the gate; the prologue also zeroes the attention kernel's
     // scheduler counters), so nothing left by an earlier call is read.
     if ((rc = launch_rope_table(ws, L, s, rope_base, st)) != SWA_OK) return rc;
-    if ((rc = launch_prologue(nullptr, k, v, ve, gate_x, Wg, ws, L, s, eps, st)) != SWA_OK) return rc;
-    return launch_attention(dev, q, v, has_ve, out, lse, s, window, eps, ws, L, st);
+    if ((rc = launch_prologue(q, k, v, ve, gate_x, Wg, ws, L, s, eps, st)) != SWA_OK) return rc;
+    return launch_attention(dev, v, has_ve, out, lse, s, window, ws, L, st);
 }

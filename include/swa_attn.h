@@ -31,11 +31,9 @@
  * Streams: calls are asynchronous on `stream` (NULL = the legacy default stream) and never
  * synchronise the host, except swa_attn_last_device_status().
  *
- * Precision: the prologue evaluates qhat, khat and v' in fp64 and rounds each to bf16 once
- * (nearest, ties to even), so every element is the correctly rounded bf16 of its exact value
- * (except within about 2^-50 of a rounding midpoint).  In the forward calls (swa_attn_fwd, _gqa,
- * _doc, _ws, _noalloc) the query prologue runs inside the attention kernel on each raw query tile,
- * so qhat never goes through HBM; it gives the same bits as swa_attn_prologue() with q.
+ * Precision: every qhat, khat and v' element the prologue writes is the correctly rounded bf16
+ * (nearest, ties to even) of its exact value, so the tensor-core operands do not depend on how the
+ * arithmetic is organised.
  *
  * Errors: a negative swa_status.  Arguments are validated before anything is enqueued; a
  * rejected call has no effect.  Waits inside the kernels are bounded: if one expires, the
@@ -88,13 +86,13 @@ typedef enum swa_status {
  * eps          >= 0 and finite (1e-6 here).
  * stream       CUDA stream (NULL = legacy default stream).
  *
- * Scratch: the library keeps one workspace per device (khat, v', the gates and the RoPE table),
+ * Scratch: the library keeps one workspace per device (qhat, khat, v', the gates, the RoPE table),
  * grown on demand with stream-ordered allocation on `stream` and kept until the library is
  * unloaded.  Each call records an event after its kernels; a call on another stream first makes
  * its stream wait for that event, so calls on different streams that share the workspace run one
  * after the other on the GPU (callers that want them to overlap use swa_attn_fwd_ws() with
- * separate workspaces).  Launches: the gate kernel (value-embedding layers), the k / v prologue
- * kernel and the attention kernel, plus the RoPE table when T, D or rope_base changes.
+ * separate workspaces).  Launches: the gate kernel (value-embedding layers), the prologue kernel
+ * and the attention kernel, plus the RoPE table when T, D or rope_base changes.
  */
 SWA_API int swa_attn_fwd(const void* q, const void* k, const void* v,
                  const void* ve, const void* gate_x, const void* Wg,
@@ -140,8 +138,7 @@ SWA_API size_t swa_attn_workspace_bytes(int B, int T, int H, int D, int has_ve);
  * Byte offset of one section of the workspace, for callers that read the prologue's results
  * (e.g. to keep them for a backward pass) after swa_attn_prologue():
  *   SWA_WS_QHAT, SWA_WS_KHAT   bf16 (B,T,H,D): rms(rope(q)), rms(rope(k)), each element the
- *                              correctly rounded bf16 (nearest, ties to even) of its exact value
- *                              (qhat only when swa_attn_prologue() was given q);
+ *                              correctly rounded bf16 (nearest, ties to even) of its exact value;
  *   SWA_WS_VPRIME              bf16 (B,T,H,D): v + 2 sigmoid(gate_x . Wg) ve, same rounding
  *                              (value-embedding layers only);
  *   SWA_WS_ROPE_TABLE          the RoPE table (internal format).
@@ -152,9 +149,9 @@ SWA_API size_t swa_attn_workspace_offset(int B, int T, int H, int D, int has_ve,
 
 /*
  * Same as swa_attn_fwd() with caller-owned device scratch: `workspace` (16-byte aligned,
- * at least swa_attn_workspace_bytes() bytes) holds khat, v', the gates and the RoPE table, which
+ * at least swa_attn_workspace_bytes() bytes) holds qhat, khat, v', the gates and the RoPE table, which
  * is rebuilt on every call (one small extra kernel).  It runs swa_attn_rope_table(),
- * swa_attn_prologue() with q = NULL and swa_attn_attention_q().  Nothing is allocated.
+ * swa_attn_prologue() and swa_attn_attention().  Nothing is allocated.
  * SWA_ERR_NO_MEMORY if ws_bytes is too small.
  */
 SWA_API int swa_attn_fwd_ws(const void* q, const void* k, const void* v,
@@ -172,17 +169,11 @@ SWA_API int swa_attn_fwd_ws(const void* q, const void* k, const void* v,
  *   rope_base, so a caller that keeps one workspace for many calls of the same T, D and base
  *   builds it once (swa_attn_fwd does that with its own workspace).
  * swa_attn_prologue: RoPE + RMS norm of q and k, gate + add of the value embedding, into the
- *   workspace (same sizes and rules as swa_attn_fwd_ws; precision: see the top of this file).
- *   q may be NULL: then only khat and v' (the forward's key/value pass; the forward normalises the
- *   query tiles inside the attention kernel).  Uses the table already in the workspace; it does not
- *   rebuild it.  It also resets the scheduler counters the attention kernels take their work from.
- * swa_attn_attention: the windowed attention on a workspace that swa_attn_prologue() with q
- *   filled for the same B, T, H, D and value-embedding setting (`v` is read directly when
- *   has_ve == 0).
- * swa_attn_attention_q: the windowed attention reading the RAW q (B,T,H,D) and applying RoPE + RMS
- *   (eps as for the prologue) to each query tile inside the kernel, with khat (and v') from a
- *   workspace that swa_attn_prologue() filled; its qhat equals, bit for bit, the one
- *   swa_attn_prologue() writes for the same q.
+ *   workspace (same sizes and rules as swa_attn_fwd_ws).  Uses the table already in the
+ *   workspace; it does not rebuild it.  It also resets the scheduler counters the attention kernel
+ *   takes its work from.
+ * swa_attn_attention: the windowed attention on a workspace that swa_attn_prologue() filled
+ *   for the same B, T, H, D and value-embedding setting (`v` is read directly when has_ve == 0).
  * All of them: asynchronous on `stream`, validation before any launch, errors as swa_attn_fwd_ws.
  */
 SWA_API int swa_attn_rope_table(int B, int T, int H, int D, int has_ve, float rope_base,
@@ -197,9 +188,6 @@ SWA_API int swa_attn_attention(const void* v, int has_ve, void* out, float* lse,
                        int B, int T, int H, int D, int window,
                        void* workspace, size_t ws_bytes, swa_stream_t stream);
 
-SWA_API int swa_attn_attention_q(const void* q, const void* v, int has_ve, void* out, float* lse,
-                                 int B, int T, int H, int D, int window, float eps,
-                                 void* workspace, size_t ws_bytes, swa_stream_t stream);
 
 /*
  * swa_attn_fwd_noalloc: swa_attn_fwd() for callers that cannot allocate device memory on the
@@ -208,7 +196,7 @@ SWA_API int swa_attn_attention_q(const void* q, const void* v, int has_ve, void*
  * synchronise the device) is not allowed.  The pages have no counterpart of this entry point.
  *
  * The caller passes inputs and outputs exactly as for swa_attn_fwd(), and the call computes the
- * same result with the same kernels; the scratch (khat, v', the gates and the RoPE table) lives in
+ * same result with the same kernels; the scratch (qhat, khat, v', the gates and the RoPE table) lives in
  * a fixed device array compiled into the library, swa_attn_noalloc_scratch_bytes() bytes (64 MiB).
  * Nothing is allocated or freed by the call itself.
  *   - CUDA loads the library's device code, and with it the array, on a device when the library
@@ -285,6 +273,22 @@ SWA_API int swa_attn_decode_gqa(const void* q, const void* k, const void* v, con
                                 size_t ws_bytes, swa_stream_t stream);
 
 /*
+ * One generation step of the document-masked layer: as swa_attn_decode_gqa, plus doc_start, an
+ * int32 (B,) device array with the first position of each sequence's current document (the
+ * document the new token at `pos` belongs to; values above pos are read as pos).  The new token
+ * attends to the cached keys [max(pos - W + 1, doc_start[b]), pos] (the document-boundary mask of
+ * swa_attn_fwd_doc, row pos).  doc_start = NULL is swa_attn_decode_gqa.  SWA_ERR_MISALIGNED if
+ * doc_start is not 4-byte aligned.
+ */
+SWA_API int swa_attn_decode_doc(const void* q, const void* k, const void* v,
+                                const void* ve, const void* gate_x, const void* Wg,
+                                void* k_cache, void* v_cache, int pos, const int* doc_start,
+                                void* out, float* lse,
+                                int B, int Tmax, int H, int Hkv, int D, int window,
+                                float rope_base, float eps,
+                                void* workspace, size_t ws_bytes, swa_stream_t stream);
+
+/*
  * The layer from its input x: the bias-free q, k, v projection fused with the prologue, then the
  * attention of swa_attn_fwd_gqa.  The pages form q, k, v of each layer as linear maps of the
  * layer input ("Let's reproduce GPT-2 (124M)" notes, section 3, the attention listing;
@@ -351,6 +355,22 @@ SWA_API int swa_attn_bwd_gqa(const void* q, const void* k, const void* v, const 
                              void* dve, float* dgate_x, float* dWg, int B, int T, int H, int Hkv,
                              int D, int window, float rope_base, float eps, void* workspace,
                              size_t ws_bytes, swa_stream_t stream);
+
+/*
+ * The backward of the document-masked layer (swa_attn_fwd_doc): as swa_attn_bwd_gqa, plus doc, the
+ * same int32 (B, T) document ids the forward took (documents are maximal runs of equal ids).  The
+ * query-tile kernel skips key tiles before the tile's first document start and masks keys before
+ * each row's document start; the key-tile kernel skips query tiles past the tile's last document end
+ * and masks queries past each key's document end.  Workspace: swa_attn_bwd_workspace_bytes() (it
+ * reserves the document starts and ends).  doc = NULL is swa_attn_bwd_gqa.  SWA_ERR_MISALIGNED if
+ * doc is not 4-byte aligned.
+ */
+SWA_API int swa_attn_bwd_doc(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                             const void* Wg, const int* doc, const void* out, const float* lse,
+                             const void* dout, const float* dlse, void* dq, void* dk, void* dv, void* dve,
+                             float* dgate_x, float* dWg, int B, int T, int H, int Hkv, int D, int window,
+                             float rope_base, float eps, void* workspace, size_t ws_bytes,
+                             swa_stream_t stream);
 /* The multi-head layer: swa_attn_bwd_gqa with Hkv = H. */
 SWA_API int swa_attn_bwd(const void* q, const void* k, const void* v, const void* ve,
                          const void* gate_x, const void* Wg, const void* out, const float* lse,

@@ -99,22 +99,6 @@ def test_stage_entry_points_reject_bad_arguments():
     assert swa.swa_attn_attention(None, 0, A, A, 1, 16, 1, 64, 0, A, need, None) == swa.SWA_ERR_INVALID_ARG
     assert swa.swa_attn_attention(A, 0, A, A, 1, 16, 1, 64, 0, A, need - 1, None) == swa.SWA_ERR_NO_MEMORY
     assert swa.swa_attn_attention(A, 0, A, A, 1, 16, 1, 80, 0, A, need, None) == swa.SWA_ERR_UNSUPPORTED
-    # the prologue: q may be NULL (key/value pass), k may not
-    assert swa.swa_attn_prologue(None, A, A, None, None, None, 1, 16, 1, 64, 1e4, 1e-6, A, need - 1, None) \
-        == swa.SWA_ERR_NO_MEMORY
-    assert swa.swa_attn_prologue(None, None, A, None, None, None, 1, 16, 1, 64, 1e4, 1e-6, A, need, None) \
-        == swa.SWA_ERR_INVALID_ARG
-    assert swa.swa_attn_prologue(A + 2, A, A, None, None, None, 1, 16, 1, 64, 1e4, 1e-6, A, need, None) \
-        == swa.SWA_ERR_MISALIGNED
-    assert swa.swa_attn_prologue(None, A, A, A, None, None, 1, 16, 1, 64, 1e4, 1e-6, A, need, None) \
-        == swa.SWA_ERR_INVALID_ARG
-    # the attention from the raw q
-    assert swa.swa_attn_attention_q(None, A, 0, A, A, 1, 16, 1, 64, 0, 1e-6, A, need, None) == swa.SWA_ERR_INVALID_ARG
-    assert swa.swa_attn_attention_q(A, A, 0, A, A, 1, 16, 1, 64, 0, 1e-6, A, need - 1, None) == swa.SWA_ERR_NO_MEMORY
-    assert swa.swa_attn_attention_q(A + 8, A, 0, A, A, 1, 16, 1, 64, 0, 1e-6, A, need, None) == swa.SWA_ERR_MISALIGNED
-    assert swa.swa_attn_attention_q(A, A, 0, A, A, 1, 16, 1, 64, 0, -1.0, A, need, None) == swa.SWA_ERR_INVALID_ARG
-    assert swa.swa_attn_attention_q(A, A, 0, A, A, 1, 16, 1, 128 + 64, 0, 1e-6, A, need, None) \
-        == swa.SWA_ERR_UNSUPPORTED
 
 
 def test_document_forward_rejects_bad_arguments():
@@ -173,7 +157,8 @@ def test_decode_workspace_and_validation():
 
 def test_backward_workspace_and_validation():
     # forward sections + row statistics (B*H*Tp float2) + dqhat (fp32) + dkhat, dv' (fp32, Hkv heads)
-    # [+ dz and the dWg partial sums on value-embedding layers], each section 1024-byte aligned
+    # [+ dz and the dWg partial sums on value-embedding layers] + document starts and ends (B*T int32
+    # each), each section 1024-byte aligned
     B, T, H, Hkv, D = 2, 200, 4, 2, 64
     up = lambda x: (x + 1023) // 1024 * 1024
     fwd = swa.swa_attn_workspace_bytes(B, T, H, D, 0)
@@ -181,7 +166,8 @@ def test_backward_workspace_and_validation():
     Tp = 256
     kv_fwd = up(B * T * Hkv * D * 2)
     assert n0 == (fwd - 2 * up(B * T * H * D * 2) + 2 * kv_fwd + up(B * T * H * D * 2) - kv_fwd
-                  + up(B * H * Tp * 8) + up(B * T * H * D * 4) + 2 * up(B * T * Hkv * D * 4))
+                  + up(B * H * Tp * 8) + up(B * T * H * D * 4) + 2 * up(B * T * Hkv * D * 4)
+                  + 2 * up(B * T * 4))
     n1 = swa.swa_attn_bwd_workspace_bytes(B, T, H, Hkv, D, 1)
     assert n1 > n0 + up(B * T * Hkv * 4)
     assert swa.swa_attn_bwd_workspace_bytes(B, T, H, 3, D, 0) == 0     # 3 does not divide 4

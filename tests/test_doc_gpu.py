@@ -86,3 +86,91 @@ def test_one_token_documents_return_their_own_value():
     assert torch.equal(out.cpu(), d["v"])
     ro, rl = oracle.forward(d, 0, parity=True, doc=doc)
     assert np.abs(lse.cpu().numpy() - rl).max() <= parity.LSE_MAX_ABS
+
+
+# ------------------------------------------------------------------ backward with documents
+
+@pytest.mark.parametrize("B,T,H,Hkv,D,window,ve,cuts", [
+    (1, 520, 4, 2, 128, 0, True, 4),
+    (2, 300, 2, 2, 64, 100, False, 3),
+    (1, 700, 2, 2, 128, 200, True, 9),
+])
+def test_document_backward_matches_the_oracle(B, T, H, Hkv, D, window, ve, cuts):
+    """The gradient of sum(dout * out) + sum(dlse * lse) through the document-masked layer, every
+    element against the oracle's backward with the same document ids (parity mode), at the
+    backward's bar (relative L2 6e-3, max error 2e-2 of the tensor's maximum)."""
+    s = workloads.LayerShape(B=B, T=T, H=H, D=D, window=window, ve=ve, seed=T + 3 * cuts, vocab=1000,
+                             kv_heads=Hkv)
+    d = workloads.make_layer(s)
+    doc = _docs(B, T, cuts, seed=11 * cuts)
+    g = torch.Generator().manual_seed(70_000 + T)
+    dout = torch.randn((B, T, H, D), generator=g).to(torch.bfloat16)
+    dlse = torch.randn((B, H, T), generator=g)
+    gi = {k: (v.cuda() if v is not None else None) for k, v in workloads.gpu_side_inputs(d).items()}
+    docd = doc.to(torch.int32).cuda()
+    out, lse = swa.forward(gi["q"], gi["k"], gi["v"], window, gi["ve"], gi["gate_x"], gi["Wg"], doc=docd)
+    got = swa.backward(gi["q"], gi["k"], gi["v"], out, lse, dout.cuda(), window, dlse=dlse.cuda(), ve=gi["ve"],
+                       gate_x=gi["gate_x"], Wg=gi["Wg"], doc=docd)
+    swa.check_device_status()
+    ref = oracle.backward(d, dout, window, dlse=dlse, parity=True, doc=doc)
+    for key, rk in (("dq", "dq"), ("dk", "dk"), ("dv", "dv"), ("dve", "dve"), ("dgate_x", "dx"), ("dWg", "dWg")):
+        if key not in got:
+            continue
+        a = got[key].float().cpu().numpy().astype(np.float64)
+        b = ref[rk]
+        rel = float(np.linalg.norm(a - b) / np.linalg.norm(b))
+        mx = float(np.abs(a - b).max() / np.abs(b).max())
+        print(f"doc backward {key}: rel_l2={rel:.3e} max_rel={mx:.3e}")
+        assert rel <= 6e-3 and mx <= 2e-2, (key, rel, mx)
+
+
+def test_document_backward_with_one_document_equals_the_plain_backward():
+    s = workloads.LayerShape(B=1, T=333, H=2, D=128, window=150, ve=True, seed=21, vocab=1000)
+    d = workloads.make_layer(s)
+    g = torch.Generator().manual_seed(5)
+    dout = torch.randn((1, 333, 2, 128), generator=g).to(torch.bfloat16).cuda()
+    gi = {k: (v.cuda() if v is not None else None) for k, v in workloads.gpu_side_inputs(d).items()}
+    out, lse = swa.forward(gi["q"], gi["k"], gi["v"], 150, gi["ve"], gi["gate_x"], gi["Wg"])
+    a = swa.backward(gi["q"], gi["k"], gi["v"], out, lse, dout, 150, ve=gi["ve"], gate_x=gi["gate_x"], Wg=gi["Wg"])
+    b = swa.backward(gi["q"], gi["k"], gi["v"], out, lse, dout, 150, ve=gi["ve"], gate_x=gi["gate_x"], Wg=gi["Wg"],
+                     doc=torch.zeros((1, 333), dtype=torch.int32, device="cuda"))
+    swa.check_device_status()
+    for key in a:
+        assert torch.equal(a[key], b[key]), key
+
+
+# ------------------------------------------------------------------ decode with documents
+
+@pytest.mark.parametrize("B,T,H,Hkv,D,window,ve,cuts", [
+    (2, 200, 2, 2, 128, 0, True, 4),
+    (1, 260, 4, 2, 64, 50, False, 6),
+])
+def test_document_decode_sequence_matches_the_oracle(B, T, H, Hkv, D, window, ve, cuts):
+    """A whole sequence generated token by token through swa_attn_decode_doc, each step given the
+    first position of its token's document: step pos returns the oracle's forward row pos with the
+    same document ids, at the forward's tolerances."""
+    s = workloads.LayerShape(B=B, T=T, H=H, D=D, window=window, ve=ve, seed=T + cuts, vocab=1000, kv_heads=Hkv)
+    d = workloads.make_layer(s)
+    doc = _docs(B, T, cuts, seed=5 * cuts)
+    dev = parity.to_device(d)
+    # first position of each position's document (a run of equal ids), computed here on the host
+    start = torch.zeros((B, T), dtype=torch.int32)
+    for b in range(B):
+        for t in range(1, T):
+            start[b, t] = start[b, t - 1] if doc[b, t] == doc[b, t - 1] else t
+    k_cache = torch.zeros((B, T, Hkv, D), dtype=torch.bfloat16, device="cuda")
+    v_cache = torch.zeros_like(k_cache)
+    out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
+    ws = torch.empty(swa.swa_attn_decode_workspace_bytes(B, T, H, D, ve, window), dtype=torch.uint8, device="cuda")
+    for pos in range(T):
+        tok = {n: (None if dev[n] is None else dev[n][:, pos].contiguous()) for n in ("q", "k", "v", "ve", "gate_x")}
+        o, l = swa.decode(tok["q"], tok["k"], tok["v"], k_cache, v_cache, pos, window, ve=tok["ve"],
+                          gate_x=tok["gate_x"], Wg=dev["Wg"], workspace=ws,
+                          doc_start=start[:, pos].contiguous().cuda())
+        out[:, pos] = o
+        lse[:, :, pos] = l
+    swa.check_device_status()
+    ro, rl = oracle.forward(d, window, parity=True, doc=doc)
+    print(parity.compare(out.float().cpu().numpy(), lse.cpu().numpy(), ro, rl,
+                         f"doc decode ({B},{T},{H}/{Hkv},{D}) W={window}"))
