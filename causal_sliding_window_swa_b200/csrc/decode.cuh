@@ -23,7 +23,8 @@
 
 namespace swa {
 
-constexpr int kDecodeChunk = 128;        // keys per CTA of the attention kernel
+constexpr int kDecodeChunk = 128;        // fewest keys per CTA of the attention kernel (the host picks
+                                         // a multiple of 32 from here up to fill the GPU's CTA slots)
 
 // Prologue of the new token: rows r = b*H + h (H = the head count of this pass); D/8 threads per
 // row as in the prefill prologue.  PARTS: bit 0 qhat (to the workspace), bit 1 khat and v' (to the
@@ -167,7 +168,7 @@ template <int D>
 __global__ void __launch_bounds__(128) decode_attn_kernel(
     const __nv_bfloat16* __restrict__ qh, const __nv_bfloat16* __restrict__ k_cache,
     const __nv_bfloat16* __restrict__ v_cache, float* __restrict__ part, int H, int Hkv, int Tmax,
-    int lo, int n_keys, int n_chunks, float c1, float c2, const int* __restrict__ doc_start) {
+    int lo, int n_keys, int n_chunks, int chunk_keys, float c1, float c2, const int* __restrict__ doc_start) {
     constexpr int DPL = D / 32;          // features per lane
     constexpr int U = 8;                 // keys per warp per iteration
     const int row = (int)(blockIdx.x / (unsigned)n_chunks);    // b*H + h
@@ -189,8 +190,8 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(
     float l = 0.f;
     // first key of this chunk, past the document start if there is one (key index j is position lo + j)
     const int jmin = doc_start != nullptr ? max(0, min(__ldg(doc_start + b), lo + n_keys - 1) - lo) : 0;
-    const int key_begin = max(chunk * kDecodeChunk, jmin);
-    const int key_end = min(chunk * kDecodeChunk + kDecodeChunk, n_keys);
+    const int key_begin = max(chunk * chunk_keys, jmin);
+    const int key_end = min(chunk * chunk_keys + chunk_keys, n_keys);
     const int hk = h / (H / Hkv);                           // key/value head of this query head
     const long long stride = (long long)Hkv * D;            // between consecutive positions
     const __nv_bfloat16* kbase = k_cache + ((long long)b * Tmax + lo) * stride + (long long)hk * D + lane * DPL;

@@ -130,6 +130,45 @@ __device__ __forceinline__ bool near_midpoint_8ulp(float x) {
     return ((__float_as_uint(x) + 8u - 0x8000u) & 0xfff0u) == 0u;
 }
 
+// Two rotation pairs (A0, B0), (A1, B1) of one row, scaled by r (r64 in fp64): the bf16 words
+// (a'_0, a'_1) and (b'_0, b'_1), each element the correctly rounded bf16 of its exact value.
+// w0, w1 = (c_hi, c_lo, s_hi, s_lo) of the two pairs; t64 their fp64 (cos, sin), read only by the
+// rare fp64 path.
+__device__ __forceinline__ void rope_2pairs_exact(float A0, float B0, float A1, float B1, const float4& w0,
+                                                  const float4& w1, const double2* __restrict__ t64, float r,
+                                                  double r64, uint32_t& wa, uint32_t& wb) {
+    const float A[2] = {A0, A1}, Bv[2] = {B0, B1};
+    const float4 w[2] = {w0, w1};
+    float xa[2], xb[2];
+    bool slow = false;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        // products with a 16-bit piece are exact; one rounding per fma, one per add
+        const float ra = fmaf(A[u], w[u].x, -(Bv[u] * w[u].z)) + fmaf(A[u], w[u].y, -(Bv[u] * w[u].w));
+        const float rb = fmaf(A[u], w[u].z, Bv[u] * w[u].x) + fmaf(A[u], w[u].w, Bv[u] * w[u].y);
+        xa[u] = ra * r;
+        xb[u] = rb * r;
+        const float small = r * (fabsf(A[u]) + fabsf(Bv[u])) * 0x1p-8f;
+        slow |= near_midpoint_8ulp(xa[u]) | near_midpoint_8ulp(xb[u]) | (fabsf(xa[u]) < small) |
+                (fabsf(xb[u]) < small);
+    }
+    wa = pack_bf16x2(xa[0], xa[1]);
+    wb = pack_bf16x2(xb[0], xb[1]);
+    if (slow) {
+        // Rare: these two pairs in fp64, rounded once.
+        uint16_t oa[2], ob[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const double2 tw = t64[u];
+            const double Ad = (double)A[u], Bd = (double)Bv[u];
+            oa[u] = bf16_rn_bits((Ad * tw.x - Bd * tw.y) * r64);
+            ob[u] = bf16_rn_bits((Ad * tw.y + Bd * tw.x) * r64);
+        }
+        wa = oa[0] | ((uint32_t)oa[1] << 16);
+        wb = ob[0] | ((uint32_t)ob[1] << 16);
+    }
+}
+
 // One group of D/8 consecutive threads handles one (b, t, h) row.  Thread c of the group owns
 // pairs i in [4c, 4c+4): elements i (in `lo_raw`) and i + D/2 (in `hi_raw`).
 template <int D>
@@ -153,38 +192,8 @@ __device__ __forceinline__ void rope_rms_pairs4(const uint2& lo_raw, const uint2
     const float r = (float)r64;
     uint32_t wa[2], wb[2];
 #pragma unroll
-    for (int e = 0; e < 4; e += 2) {
-        float xa[2], xb[2];
-        bool slow = false;
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const float4 w = cs[e + u];   // (c_hi, c_lo, s_hi, s_lo)
-            const float A = a[e + u], Bv = b[e + u];
-            // products with a 16-bit piece are exact; one rounding per fma, one per add
-            const float ra = fmaf(A, w.x, -(Bv * w.z)) + fmaf(A, w.y, -(Bv * w.w));
-            const float rb = fmaf(A, w.z, Bv * w.x) + fmaf(A, w.w, Bv * w.y);
-            xa[u] = ra * r;
-            xb[u] = rb * r;
-            const float small = r * (fabsf(A) + fabsf(Bv)) * 0x1p-8f;
-            slow |= near_midpoint_8ulp(xa[u]) | near_midpoint_8ulp(xb[u]) |
-                    (fabsf(xa[u]) < small) | (fabsf(xb[u]) < small);
-        }
-        wa[e >> 1] = pack_bf16x2(xa[0], xa[1]);
-        wb[e >> 1] = pack_bf16x2(xb[0], xb[1]);
-        if (slow) {
-            // Rare: these two pairs in fp64, rounded once.
-            uint16_t oa[2], ob[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const double2 w = tab64[e + u];
-                const double A = (double)a[e + u], Bv = (double)b[e + u];
-                oa[u] = bf16_rn_bits((A * w.x - Bv * w.y) * r64);
-                ob[u] = bf16_rn_bits((A * w.y + Bv * w.x) * r64);
-            }
-            wa[e >> 1] = oa[0] | ((uint32_t)oa[1] << 16);
-            wb[e >> 1] = ob[0] | ((uint32_t)ob[1] << 16);
-        }
-    }
+    for (int e = 0; e < 4; e += 2)
+        rope_2pairs_exact(a[e], b[e], a[e + 1], b[e + 1], cs[e], cs[e + 1], tab64 + e, r, r64, wa[e >> 1], wb[e >> 1]);
     out_lo = make_uint2(wa[0], wa[1]);
     out_hi = make_uint2(wb[0], wb[1]);
 }

@@ -15,6 +15,7 @@
 #include "swa_attn.h"
 #include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
+#include "attn_fwd_wide.cuh"
 #include "decode.cuh"
 #include "prologue.cuh"
 #include "qkv_gemm.cuh"
@@ -184,6 +185,10 @@ int device_ready(int* dev_out) {
                                      swa::FwdCfg<64>::SMEM_TOTAL) != cudaSuccess ||
                 cudaFuncSetAttribute(swa::attn_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      swa::FwdCfg<128>::SMEM_TOTAL) != cudaSuccess ||
+                cudaFuncSetAttribute(swa::attn_fwd_wide_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     swa::WideCfg::SMEM_TOTAL) != cudaSuccess ||
+                cudaFuncSetAttribute(swa::attn_fwd_wide_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     swa::WideCfg::SMEM_TOTAL) != cudaSuccess ||
                 cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<64>, (cudaFuncAttribute)smem_attr,
                                      swa::BwdCfg<64>::DQ_SMEM) != cudaSuccess ||
                 cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<128>, (cudaFuncAttribute)smem_attr,
@@ -376,11 +381,15 @@ int launch_attention(int dev, const void* v, bool has_ve, void* out, float* lse,
     const dim3 grid((unsigned)std::min(p.n_items, g_num_sms[dev]));
 #define SWA_ATTN(DD, DC) \
     swa::attn_fwd_kernel<DD, DC><<<grid, swa::FwdCfg<DD>::THREADS, swa::FwdCfg<DD>::SMEM_TOTAL, st>>>(tq, tk, tv, to, p)
+#define SWA_ATTN_WIDE(DC) \
+    swa::attn_fwd_wide_kernel<DC><<<grid, swa::WideCfg::THREADS, swa::WideCfg::SMEM_TOTAL, st>>>(tq, tk, tv, to, p)
     if (s.D == 128) {
-        if (dstart) SWA_ATTN(128, true); else SWA_ATTN(128, false);
+        // 256-key score products (attn_fwd_wide.cuh)
+        if (dstart) SWA_ATTN_WIDE(true); else SWA_ATTN_WIDE(false);
     } else {
         if (dstart) SWA_ATTN(64, true); else SWA_ATTN(64, false);
     }
+#undef SWA_ATTN_WIDE
 #undef SWA_ATTN
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
@@ -1054,7 +1063,37 @@ int swa_attn_decode_doc(const void* q, const void* k, const void* v, const void*
     const int W = (window <= 0 || window >= Tmax) ? Tmax : window;
     const int lo = std::max(0, pos - W + 1);
     const int n_keys = pos - lo + 1;
-    const int n_chunks = (n_keys + swa::kDecodeChunk - 1) / swa::kDecodeChunk;
+    // Keys per CTA: the multiple of 32 (at least kDecodeChunk) whose grid fills the GPU's resident
+    // CTA slots best over whole waves (fewer, fuller waves; ties to the smaller chunk).
+    int chunk_keys = swa::kDecodeChunk;
+    {
+        static int per_sm[64][2] = {{0}};
+        int& cached = per_sm[dev][D == 128 ? 1 : 0];
+        if (cached == 0) {
+            int n = 0;
+            const cudaError_t e = D == 128
+                ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, swa::decode_attn_kernel<128>, 128, 0)
+                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, swa::decode_attn_kernel<64>, 128, 0);
+            if (e != cudaSuccess || n < 1) {
+                cudaGetLastError();
+                n = 1;
+            }
+            cached = n;
+        }
+        const long long slots = (long long)cached * g_num_sms[dev];
+        double best = -1.0;
+        for (int ck = swa::kDecodeChunk; ck <= 1024; ck += 32) {
+            const long long ctas = (long long)rows * ((n_keys + ck - 1) / ck);
+            const long long waves = (ctas + slots - 1) / slots;
+            const double fill = (double)ctas / (double)(waves * slots);
+            if (fill > best + 1e-9) {
+                best = fill;
+                chunk_keys = ck;
+            }
+            if (ck >= n_keys) break;
+        }
+    }
+    const int n_chunks = (n_keys + chunk_keys - 1) / chunk_keys;
     const double log2e = 1.4426950408889634;
     const double m0 = std::sqrt((double)D) * (1.0 + 1.0 / 64.0);
     const float c1 = (float)(log2e / std::sqrt((double)D)), c2 = (float)(m0 * log2e);
@@ -1064,12 +1103,12 @@ int swa_attn_decode_doc(const void* q, const void* k, const void* v, const void*
     const bf* vcc = static_cast<const bf*>(v_cache);
     bf* o = static_cast<bf*>(out);
     if (D == 128) {
-        swa::decode_attn_kernel<128><<<grid, 128, 0, st>>>(qc, kcc, vcc, part, H, Hkv, Tmax, lo, n_keys, n_chunks, c1, c2,
-                                                           doc_start);
+        swa::decode_attn_kernel<128><<<grid, 128, 0, st>>>(qc, kcc, vcc, part, H, Hkv, Tmax, lo, n_keys, n_chunks,
+                                                           chunk_keys, c1, c2, doc_start);
         swa::decode_combine_kernel<128><<<rows, 128, 0, st>>>(part, o, lse, n_chunks, (float)m0);
     } else {
-        swa::decode_attn_kernel<64><<<grid, 128, 0, st>>>(qc, kcc, vcc, part, H, Hkv, Tmax, lo, n_keys, n_chunks, c1, c2,
-                                                          doc_start);
+        swa::decode_attn_kernel<64><<<grid, 128, 0, st>>>(qc, kcc, vcc, part, H, Hkv, Tmax, lo, n_keys, n_chunks,
+                                                          chunk_keys, c1, c2, doc_start);
         swa::decode_combine_kernel<64><<<rows, 64, 0, st>>>(part, o, lse, n_chunks, (float)m0);
     }
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
