@@ -375,7 +375,7 @@ def run_ours(args, s0):
         "pct_bf16_peak": 100.0 * value / world / peak,
         "peak_source": f"{peak_src} bf16_tflops (burst)",
         "stage_ms": {"prologue": pro_ms_max, "attention": att_ms_max},
-        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>", "achieved": achieved,
+        "roofline": {"bound": "tensor", "kernel": f"attn_fwd_kernel<{s.D}>", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "traffic": recorded_traffic(args.workload),
                      "note": f"4*D flops per unmasked pair / mean attention launch time; peak = "

@@ -154,8 +154,10 @@ __device__ __forceinline__ uint32_t softmax_pair_mufu(uint32_t s0, uint32_t s1, 
 // relative error on that interval (Remez exchange fitted for this library, 7.5e-5 in fp32);
 // 2^n applied by adding n to the exponent field.  Valid for x in [-126, 0].
 // Pair j of every 8 consecutive key pairs takes the polynomial when bit j of this mask is set
-// (unmasked tiles only); the rest go to MUFU.
-constexpr uint32_t kPolyPairMask = 0x88u;
+// (unmasked tiles only); the rest go to MUFU.  All pairs go to MUFU: with the tile loop bound by
+// the issue of its tensor-core products, sending 2 pairs of 8 to the polynomial measured 3-4%
+// slower on B200 at D = 128 (the extra FMA-pipe instructions cost more than the MUFU time saved).
+constexpr uint32_t kPolyPairMask = 0x00u;
 
 struct PolyConsts {
     uint64_t shift, c3, c2, c1, c0;

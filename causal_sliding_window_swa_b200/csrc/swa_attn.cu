@@ -15,7 +15,6 @@
 #include "swa_attn.h"
 #include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
-#include "attn_fwd_wide.cuh"
 #include "decode.cuh"
 #include "prologue.cuh"
 #include "qkv_gemm.cuh"
@@ -185,10 +184,6 @@ int device_ready(int* dev_out) {
                                      swa::FwdCfg<64>::SMEM_TOTAL) != cudaSuccess ||
                 cudaFuncSetAttribute(swa::attn_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      swa::FwdCfg<128>::SMEM_TOTAL) != cudaSuccess ||
-                cudaFuncSetAttribute(swa::attn_fwd_wide_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     swa::WideCfg::SMEM_TOTAL) != cudaSuccess ||
-                cudaFuncSetAttribute(swa::attn_fwd_wide_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     swa::WideCfg::SMEM_TOTAL) != cudaSuccess ||
                 cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<64>, (cudaFuncAttribute)smem_attr,
                                      swa::BwdCfg<64>::DQ_SMEM) != cudaSuccess ||
                 cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<128>, (cudaFuncAttribute)smem_attr,
@@ -381,15 +376,11 @@ int launch_attention(int dev, const void* v, bool has_ve, void* out, float* lse,
     const dim3 grid((unsigned)std::min(p.n_items, g_num_sms[dev]));
 #define SWA_ATTN(DD, DC) \
     swa::attn_fwd_kernel<DD, DC><<<grid, swa::FwdCfg<DD>::THREADS, swa::FwdCfg<DD>::SMEM_TOTAL, st>>>(tq, tk, tv, to, p)
-#define SWA_ATTN_WIDE(DC) \
-    swa::attn_fwd_wide_kernel<DC><<<grid, swa::WideCfg::THREADS, swa::WideCfg::SMEM_TOTAL, st>>>(tq, tk, tv, to, p)
     if (s.D == 128) {
-        // 256-key score products (attn_fwd_wide.cuh)
-        if (dstart) SWA_ATTN_WIDE(true); else SWA_ATTN_WIDE(false);
+        if (dstart) SWA_ATTN(128, true); else SWA_ATTN(128, false);
     } else {
         if (dstart) SWA_ATTN(64, true); else SWA_ATTN(64, false);
     }
-#undef SWA_ATTN_WIDE
 #undef SWA_ATTN
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
