@@ -49,8 +49,9 @@ __global__ void __launch_bounds__(256) decode_prologue_kernel(
         const double theta = pow(base, -2.0 * (double)i / (double)D);
         double sn, cs;
         sincos((double)pos * theta, &sn, &cs);
-        const float c_hi = round_sig16(cs), s_hi = round_sig16(sn);
-        const float c_lo = round_sig16(cs - (double)c_hi), s_lo = round_sig16(sn - (double)s_hi);
+        float c_hi, c_lo, s_hi, s_lo;
+        rope_split(cs, c_hi, c_lo);
+        rope_split(sn, s_hi, s_lo);
         s_tab32[i] = make_float4(c_hi, c_lo, s_hi, s_lo);
         s_tab64[i] = make_double2(cs, sn);
     }
@@ -108,8 +109,8 @@ __global__ void __launch_bounds__(256) decode_prologue_kernel(
 #pragma unroll
         for (int e = 0; e < 4; ++e) cs4[e] = s_tab32[i0 + e];
         uint2 o0, o1, o2, o3;
-        if (DO_Q) rope_rms_pairs4<D>(raw[0], raw[1], cs4, s_tab64 + i0, eps, o0, o1);
-        if (DO_KV) rope_rms_pairs4<D>(raw[2], raw[3], cs4, s_tab64 + i0, eps, o2, o3);
+        if (DO_Q) rope_rms_exact4<D>(raw[0], raw[1], cs4, s_tab64 + i0, eps, o0, o1);
+        if (DO_KV) rope_rms_exact4<D>(raw[2], raw[3], cs4, s_tab64 + i0, eps, o2, o3);
         if (valid && DO_Q) {
             *reinterpret_cast<uint2*>(qh + in_off + i0) = o0;
             *reinterpret_cast<uint2*>(qh + in_off + HALF + i0) = o1;

@@ -10,15 +10,18 @@
 // exact value of its definition, so the tensor-core operands do not depend on how the arithmetic
 // is organised (an fp32-only pipeline flips the last bf16 bit of ~1e-4 of the elements, which
 // moves single attention scores by ~1e-3).  The common path runs in fp32 with a proven error
-// bound; a pair whose fp32 result could round differently from the exact one is recomputed in
-// fp64 (a fraction of a percent of them).
+// bound; an element whose fp32 result could round differently from the exact one (a few in 10^4)
+// is listed and recomputed in fp64 by a second, small kernel that overwrites it.
 //   norm: r = 1 / sqrt(ss / D + eps) from the sum of squares of the raw inputs (the rotation
 //     preserves it) in fp64, where each square and the sum are exact; the inverse square root by
 //     two Newton-Raphson steps from the hardware estimate, then rounded once to fp32.
-//   rotation: cos and sin are stored as two pieces with 16-bit significands (remainder below
-//     2^-33), so every product a * piece is exact in fp32 for a bf16 input a; x = ra * r is then
-//     within 4 of its own ulps of the exact value whenever |x| >= 2^-8 r (|a| + |b|).  The test
-//     window is 8 ulps, and smaller |x| (partial cancellation) always take the fp64 path.
+//   rotation: cos and sin are stored as a head with a 16-bit significand, so that a * head is
+//     exact in fp32 for a bf16 input a, and the fp32 remainder (|c - head - tail| < 2^-40).  With
+//     S = |a| + |b|: the head term a c_hi - b s_hi is one fma of exact operands (error 2^-24 of
+//     itself), the tail term costs at most 2^-39 S, the table 2^-40 S, so ra is within
+//     2^-23 |ra| + 2^-38 S of the exact rotation and x = ra * r within 2^-22 |x| + 2^-38 S r, i.e.
+//     within 5 of its own ulps whenever |x| >= 2^-14 S r.  The test window is 8 ulps, and smaller
+//     |x| (partial cancellation, a few in 10^5 elements) always take the fp64 path.
 //   gate: z = x[:32] . Wg[:, h] and g = 2 sigmoid(z) in fp64 by a separate one-thread-per-row
 //     kernel, stored split as g_hi + g_lo (fp32); v' = (v + g_hi ve) + g_lo ve with two fp32
 //     roundings: within 1 ulp of the exact value unless |v'| < 2^-16 |g ve|.
@@ -64,13 +67,20 @@ __global__ void gate_kernel(const __nv_bfloat16* __restrict__ gate_x, const __nv
 }
 
 // RoPE tables, one entry per (t, i):
-//   tab32[t*D/2 + i] = (c_hi, c_lo, s_hi, s_lo) fp32, each piece with a 16-bit significand;
+//   tab32[t*D/2 + i] = (c_hi, c_lo, s_hi, s_lo) fp32: c_hi with a 16-bit significand, c_lo the
+//     fp32 of the remainder c - c_hi (likewise s);
 //   tab64[t*D/2 + i] = (cos, sin) fp64, read only by the fp64 path.
 __device__ __forceinline__ float round_sig16(double x) {
     // nearest float with at most 16 significant bits (8 low mantissa bits cleared)
     const float f = (float)x;
     const uint32_t u = __float_as_uint(f);
     return __uint_as_float((u + 0x80u) & 0xffffff00u);
+}
+
+// c -> (hi, lo): hi = c to 16 significant bits, lo = fp32(c - hi); |c - hi - lo| <= 2^-40 |c|.
+__device__ __forceinline__ void rope_split(double c, float& hi, float& lo) {
+    hi = round_sig16(c);
+    lo = (float)(c - (double)hi);
 }
 
 __global__ void rope_table_kernel(float4* __restrict__ tab32, double2* __restrict__ tab64, int T,
@@ -84,8 +94,9 @@ __global__ void rope_table_kernel(float4* __restrict__ tab32, double2* __restric
         const double theta = pow(base, -2.0 * (double)i / (double)D);
         double s, c;
         sincos((double)t * theta, &s, &c);
-        const float c_hi = round_sig16(c), s_hi = round_sig16(s);
-        const float c_lo = round_sig16(c - (double)c_hi), s_lo = round_sig16(s - (double)s_hi);
+        float c_hi, c_lo, s_hi, s_lo;
+        rope_split(c, c_hi, c_lo);
+        rope_split(s, s_hi, s_lo);
         tab32[idx] = make_float4(c_hi, c_lo, s_hi, s_lo);
         tab64[idx] = make_double2(c, s);
     }
@@ -130,54 +141,58 @@ __device__ __forceinline__ bool near_midpoint_8ulp(float x) {
     return ((__float_as_uint(x) + 8u - 0x8000u) & 0xfff0u) == 0u;
 }
 
-// Two rotation pairs (A0, B0), (A1, B1) of one row, scaled by r (r64 in fp64): the bf16 words
-// (a'_0, a'_1) and (b'_0, b'_1), each element the correctly rounded bf16 of its exact value.
-// w0, w1 = (c_hi, c_lo, s_hi, s_lo) of the two pairs; t64 their fp64 (cos, sin), read only by the
-// rare fp64 path.
-__device__ __forceinline__ void rope_2pairs_exact(float A0, float B0, float A1, float B1, const float4& w0,
-                                                  const float4& w1, const double2* __restrict__ t64, float r,
-                                                  double r64, uint32_t& wa, uint32_t& wb) {
-    const float A[2] = {A0, A1}, Bv[2] = {B0, B1};
-    const float4 w[2] = {w0, w1};
-    float xa[2], xb[2];
-    bool slow = false;
+// Fast path of four rotation pairs (a_e, b_e) = (element i0 + e, element i0 + e + D/2) of one
+// row, scaled by r: the bf16 words of (a'_0..a'_3) and (b'_0..b'_3) rounded from fp32, and a mask
+// with bit e set where pair e could round differently from its exact value (near a bf16 rounding
+// midpoint, or partial cancellation).  No branch: the caller repairs masked pairs afterwards.
+__device__ __forceinline__ uint32_t rope_rms_fast4(const float (&a)[4], const float (&b)[4], const float4 (&w)[4],
+                                                   float r, uint2& out_lo, uint2& out_hi) {
+    float xa[4], xb[4];
+    uint32_t mask = 0u;
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        // products with a 16-bit piece are exact; one rounding per fma, one per add
-        const float ra = fmaf(A[u], w[u].x, -(Bv[u] * w[u].z)) + fmaf(A[u], w[u].y, -(Bv[u] * w[u].w));
-        const float rb = fmaf(A[u], w[u].z, Bv[u] * w[u].x) + fmaf(A[u], w[u].w, Bv[u] * w[u].y);
-        xa[u] = ra * r;
-        xb[u] = rb * r;
-        const float small = r * (fabsf(A[u]) + fabsf(Bv[u])) * 0x1p-8f;
-        slow |= near_midpoint_8ulp(xa[u]) | near_midpoint_8ulp(xb[u]) | (fabsf(xa[u]) < small) |
-                (fabsf(xb[u]) < small);
+    for (int e = 0; e < 4; ++e) {
+        // head products are exact (one rounding per head fma); tail terms are 2^-16 smaller
+        const float ra = fmaf(a[e], w[e].x, -(b[e] * w[e].z)) + fmaf(a[e], w[e].y, -(b[e] * w[e].w));
+        const float rb = fmaf(a[e], w[e].z, b[e] * w[e].x) + fmaf(a[e], w[e].w, b[e] * w[e].y);
+        xa[e] = ra * r;
+        xb[e] = rb * r;
+        const float small = r * (fabsf(a[e]) + fabsf(b[e])) * 0x1p-14f;
+        const bool slow = near_midpoint_8ulp(xa[e]) | near_midpoint_8ulp(xb[e]) | (fabsf(xa[e]) < small) |
+                          (fabsf(xb[e]) < small);
+        mask |= (slow ? 1u : 0u) << e;
     }
-    wa = pack_bf16x2(xa[0], xa[1]);
-    wb = pack_bf16x2(xb[0], xb[1]);
-    if (slow) {
-        // Rare: these two pairs in fp64, rounded once.
-        uint16_t oa[2], ob[2];
+    out_lo = make_uint2(pack_bf16x2(xa[0], xa[1]), pack_bf16x2(xa[2], xa[3]));
+    out_hi = make_uint2(pack_bf16x2(xb[0], xb[1]), pack_bf16x2(xb[2], xb[3]));
+    return mask;
+}
+
+// Replaces 16-bit element e (0..3) of a 4-element bf16 word pair.
+__device__ __forceinline__ void set_bf16_elem(uint2& w, int e, uint16_t v) {
+    uint32_t& word = (e >> 1) ? w.y : w.x;
+    word = (e & 1) ? ((word & 0x0000ffffu) | ((uint32_t)v << 16)) : ((word & 0xffff0000u) | v);
+}
+
+// The masked pairs of rope_rms_fast4 in fp64, rounded once: ((a cos - b sin) r64, (a sin + b cos) r64).
+__device__ __noinline__ void rope_rms_repair4(const float (&a)[4], const float (&b)[4], const double2* __restrict__ t64,
+                                              double r64, uint32_t mask, uint2& out_lo, uint2& out_hi) {
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const double2 tw = t64[u];
-            const double Ad = (double)A[u], Bd = (double)Bv[u];
-            oa[u] = bf16_rn_bits((Ad * tw.x - Bd * tw.y) * r64);
-            ob[u] = bf16_rn_bits((Ad * tw.y + Bd * tw.x) * r64);
-        }
-        wa = oa[0] | ((uint32_t)oa[1] << 16);
-        wb = ob[0] | ((uint32_t)ob[1] << 16);
+    for (int e = 0; e < 4; ++e) {
+        if (!((mask >> e) & 1u)) continue;
+        const double2 tw = t64[e];
+        const double Ad = (double)a[e], Bd = (double)b[e];
+        set_bf16_elem(out_lo, e, bf16_rn_bits((Ad * tw.x - Bd * tw.y) * r64));
+        set_bf16_elem(out_hi, e, bf16_rn_bits((Ad * tw.y + Bd * tw.x) * r64));
     }
 }
 
 // One group of D/8 consecutive threads handles one (b, t, h) row.  Thread c of the group owns
-// pairs i in [4c, 4c+4): elements i (in `lo_raw`) and i + D/2 (in `hi_raw`).
+// pairs i in [4c, 4c+4): elements i (in `lo_raw`) and i + D/2 (in `hi_raw`).  Returns the mask of
+// pairs still to be repaired (rope_rms_repair4 with the returned r64).
 template <int D>
-__device__ __forceinline__ void rope_rms_pairs4(const uint2& lo_raw, const uint2& hi_raw,
-                                                const float4 (&cs)[4],
-                                                const double2* __restrict__ tab64, double eps,
-                                                uint2& out_lo, uint2& out_hi) {
+__device__ __forceinline__ uint32_t rope_rms_pairs4(const uint2& lo_raw, const uint2& hi_raw, const float4 (&cs)[4],
+                                                    double eps, float (&a)[4], float (&b)[4], uint2& out_lo,
+                                                    uint2& out_hi, double& r64) {
     constexpr int TPR = D / 8;
-    float a[4], b[4];
     unpack4(lo_raw, a);
     unpack4(hi_raw, b);
     double ss = 0.0;
@@ -188,42 +203,193 @@ __device__ __forceinline__ void rope_rms_pairs4(const uint2& lo_raw, const uint2
     }
 #pragma unroll
     for (int m = TPR / 2; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-    const double r64 = rsqrt_newton(ss * (1.0 / (double)D) + eps);
-    const float r = (float)r64;
-    uint32_t wa[2], wb[2];
-#pragma unroll
-    for (int e = 0; e < 4; e += 2)
-        rope_2pairs_exact(a[e], b[e], a[e + 1], b[e + 1], cs[e], cs[e + 1], tab64 + e, r, r64, wa[e >> 1], wb[e >> 1]);
-    out_lo = make_uint2(wa[0], wa[1]);
-    out_hi = make_uint2(wb[0], wb[1]);
+    r64 = rsqrt_newton(ss * (1.0 / (double)D) + eps);
+    return rope_rms_fast4(a, b, cs, (float)r64, out_lo, out_hi);
 }
 
 // v' = v + g ve for 4 elements: (v + g_hi ve) + g_lo ve in fp32 (two roundings, within 1 ulp
-// unless |v'| < 2^-16 |g ve|); fp64 when that could cross a bf16 rounding midpoint.
-__device__ __forceinline__ uint2 gated_add4(const uint2& vw, const uint2& ew, float g_hi, float g_lo,
-                                            double g64) {
+// unless |v'| < 2^-16 |g ve|).  Returns the mask of elements that could cross a bf16 rounding
+// midpoint (repaired in fp64 by gated_repair4).
+__device__ __forceinline__ uint32_t gated_fast4(const uint2& vw, const uint2& ew, float g_hi, float g_lo, uint2& out) {
     float v[4], e4[4];
     unpack4(vw, v);
     unpack4(ew, e4);
-    uint32_t w[2];
-    bool slow = false;
+    float x[4];
+    uint32_t mask = 0u;
 #pragma unroll
-    for (int e = 0; e < 4; e += 2) {
-        float x[2];
+    for (int e = 0; e < 4; ++e) {
+        x[e] = fmaf(g_lo, e4[e], fmaf(g_hi, e4[e], v[e]));
+        const bool slow = near_midpoint_8ulp(x[e]) | (fabsf(x[e]) < fabsf(g_hi * e4[e]) * 0x1p-16f);
+        mask |= (slow ? 1u : 0u) << e;
+    }
+    out = make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]));
+    return mask;
+}
+
+__device__ __noinline__ void gated_repair4(const uint2& vw, const uint2& ew, double g64, uint32_t mask, uint2& out) {
+    float v[4], e4[4];
+    unpack4(vw, v);
+    unpack4(ew, e4);
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            x[u] = fmaf(g_lo, e4[e + u], fmaf(g_hi, e4[e + u], v[e + u]));
-            slow |= near_midpoint_8ulp(x[u]) | (fabsf(x[u]) < fabsf(g_hi * e4[e + u]) * 0x1p-16f);
+    for (int e = 0; e < 4; ++e)
+        if ((mask >> e) & 1u) set_bf16_elem(out, e, bf16_rn_bits(fma(g64, (double)e4[e], (double)v[e])));
+}
+
+// The two steps together, for callers with few rows (the decode step).
+template <int D>
+__device__ __forceinline__ void rope_rms_exact4(const uint2& lo_raw, const uint2& hi_raw, const float4 (&cs)[4],
+                                                const double2* __restrict__ t64, double eps, uint2& out_lo,
+                                                uint2& out_hi) {
+    float a[4], b[4];
+    double r64;
+    const uint32_t m = rope_rms_pairs4<D>(lo_raw, hi_raw, cs, eps, a, b, out_lo, out_hi, r64);
+    if (m) rope_rms_repair4(a, b, t64, r64, m, out_lo, out_hi);
+}
+
+__device__ __forceinline__ uint2 gated_add4(const uint2& vw, const uint2& ew, float g_hi, float g_lo, double g64) {
+    uint2 out;
+    const uint32_t m = gated_fast4(vw, ew, g_hi, g_lo, out);
+    if (m) gated_repair4(vw, ew, g64, m, out);
+    return out;
+}
+
+// ------------------------------------------------------------------ deferred repairs
+// The prologue kernel writes every output from its fp32 fast path.  For a row chunk (D/8 threads
+// per row; four rotation pairs and eight v' elements per thread) with elements that fast path
+// cannot certify, it lists (chunk, flags) in its block's list: flag bits 0-3 qhat pairs i0 + e
+// (elements i0 + e and i0 + e + D/2), bits 4-7 khat pairs, bits 8-11 v' elements i0 + e, bits
+// 12-15 v' elements i0 + D/2 + e.  prologue_fix_kernel recomputes the flagged elements in fp64 and
+// overwrites them.  A block whose list overflows (inputs built to sit on rounding midpoints) has
+// every element of its row chunks recomputed instead.  An item carries the rows' fp64 r (the fast
+// path already has it), so that a repair needs only the chunk's own inputs.
+constexpr int kFixPerBlock = 256;
+
+struct __align__(16) FixItem {
+    uint32_t chunk_lo;     // row chunk index, low 32 bits
+    uint32_t code;         // flag bits | (chunk index >> 32) << 16
+    uint32_t pad0, pad1;
+    double rq, rk;         // r of the chunk's qhat row and khat row (fp64)
+};
+
+struct FixParams {
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* k;
+    const __nv_bfloat16* v;
+    const __nv_bfloat16* ve;
+    const float2* gate;
+    __nv_bfloat16* qh;
+    __nv_bfloat16* kh;
+    __nv_bfloat16* vp;
+    const double2* tab64;
+    int T, H, Hkv, D;
+    double eps;
+    // the prologue pass these lists belong to
+    int heads;                 // heads of its rows (H, or Hkv for the key/value pass)
+    uint32_t all_flags;        // flag bits of the outputs it computes
+    long long n_chunks;        // rows * D / 8
+    long long stride;          // its grid's thread count
+    int n_iter;                // loop iterations of each of its threads
+};
+
+// 1 / sqrt(ss / D + eps) of one row in fp64: exact squares, fp64 sums.  All loads are issued
+// before the arithmetic.
+template <int D>
+__device__ __forceinline__ double row_r64(const __nv_bfloat16* __restrict__ x, double eps) {
+    uint4 u[D / 8];
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) u[j] = *reinterpret_cast<const uint4*>(x + 8 * j);
+    double s0 = 0.0, s1 = 0.0;
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) {
+        float f[4], g[4];
+        unpack4(make_uint2(u[j].x, u[j].y), f);
+        unpack4(make_uint2(u[j].z, u[j].w), g);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            s0 = fma((double)f[e], (double)f[e], s0);
+            s1 = fma((double)g[e], (double)g[e], s1);
         }
-        w[e >> 1] = pack_bf16x2(x[0], x[1]);
     }
-    if (slow) {
+    return rsqrt_newton((s0 + s1) * (1.0 / (double)D) + eps);
+}
+
+// The flagged elements of one row chunk in fp64, each rounded once: the rotation with the fp64
+// table scaled by the row's r; v + g ve with g = g_hi + g_lo.  The loads of a tensor's row and of
+// the chunk's four pairs are issued together.
+template <int D>
+__device__ void prologue_fix_chunk(long long chunk, uint32_t flags, const FixParams& p, const double* r_known) {
+    constexpr int TPR = D / 8, HALF = D / 2;
+    const uint32_t row = (uint32_t)(chunk / TPR);
+    const int i0 = 4 * (int)(chunk % TPR);
+    const long long base = (long long)row * D;
+    const uint32_t t = (row / (uint32_t)p.heads) % (uint32_t)p.T;
+    const double2* tw = p.tab64 + (long long)t * HALF + i0;
+#pragma unroll 1
+    for (int tensor = 0; tensor < 2; ++tensor) {
+        const uint32_t m = (flags >> (4 * tensor)) & 15u;
+        if (m == 0u) continue;
+        const __nv_bfloat16* x = (tensor == 0 ? p.q : p.k) + base;
+        __nv_bfloat16* dst = (tensor == 0 ? p.qh : p.kh) + base;
+        double2 cs[4];
 #pragma unroll
-        for (int e = 0; e < 4; e += 2)
-            w[e >> 1] = (uint32_t)bf16_rn_bits(fma(g64, (double)e4[e], (double)v[e])) |
-                        ((uint32_t)bf16_rn_bits(fma(g64, (double)e4[e + 1], (double)v[e + 1])) << 16);
+        for (int e = 0; e < 4; ++e) cs[e] = tw[e];
+        float a[4], b[4];
+        unpack4(*reinterpret_cast<const uint2*>(x + i0), a);
+        unpack4(*reinterpret_cast<const uint2*>(x + HALF + i0), b);
+        const double r64 = r_known != nullptr ? r_known[tensor] : row_r64<D>(x, p.eps);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (!((m >> e) & 1u)) continue;
+            const double A = (double)a[e], B = (double)b[e];
+            dst[i0 + e] = __ushort_as_bfloat16(bf16_rn_bits((A * cs[e].x - B * cs[e].y) * r64));
+            dst[HALF + i0 + e] = __ushort_as_bfloat16(bf16_rn_bits((A * cs[e].y + B * cs[e].x) * r64));
+        }
     }
-    return make_uint2(w[0], w[1]);
+    const uint32_t mv = flags >> 8;
+    if (mv != 0u) {
+        const float2 g = p.gate[row];
+        float v[8], e8[8];
+        unpack4(*reinterpret_cast<const uint2*>(p.v + base + i0), *reinterpret_cast<float(*)[4]>(v));
+        unpack4(*reinterpret_cast<const uint2*>(p.v + base + HALF + i0), *reinterpret_cast<float(*)[4]>(v + 4));
+        unpack4(*reinterpret_cast<const uint2*>(p.ve + base + i0), *reinterpret_cast<float(*)[4]>(e8));
+        unpack4(*reinterpret_cast<const uint2*>(p.ve + base + HALF + i0), *reinterpret_cast<float(*)[4]>(e8 + 4));
+        const double g64 = (double)g.x + (double)g.y;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            if (!((mv >> e) & 1u)) continue;
+            const int i = e < 4 ? i0 + e : HALF + i0 + e - 4;
+            p.vp[base + i] = __ushort_as_bfloat16(bf16_rn_bits(fma(g64, (double)e8[e], (double)v[e])));
+        }
+    }
+}
+
+// One warp per prologue block's list (a single wave for the usual grid); its lanes take the
+// list's items.  An overflowed list (count > kFixPerBlock) has its warp walk all the row chunks
+// of that block instead.
+template <int D>
+__global__ void __launch_bounds__(256) prologue_fix_kernel(const int* __restrict__ counts, const FixItem* __restrict__ items,
+                                                           int n_lists, const __grid_constant__ FixParams p) {
+    const int lane = (int)(threadIdx.x & 31u);
+    const int n_warps = (int)((gridDim.x * blockDim.x) >> 5);
+    for (int list = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); list < n_lists; list += n_warps) {
+        // the count and the lane's first item are read together; slots past the count are ignored
+        const int cnt = __ldg(counts + list);
+        FixItem it = items[(long long)list * kFixPerBlock + lane];
+        if (cnt <= kFixPerBlock) {
+            for (int slot = lane; slot < cnt; slot += 32) {
+                if (slot != lane) it = items[(long long)list * kFixPerBlock + slot];
+                const double r[2] = {it.rq, it.rk};
+                prologue_fix_chunk<D>((long long)it.chunk_lo | ((long long)(it.code >> 16) << 32), it.code & 0xffffu,
+                                      p, r);
+            }
+        } else {
+            // the block's threads handled chunks list * 256 + u + it * stride, u < 256, it < n_iter
+            for (long long j = lane; j < 256ll * p.n_iter; j += 32) {
+                const long long c = (long long)list * 256 + (j & 255) + (j >> 8) * p.stride;
+                if (c < p.n_chunks) prologue_fix_chunk<D>(c, p.all_flags, p, nullptr);
+            }
+        }
+    }
 }
 
 // PARTS selects the outputs: bit 0 qhat, bit 1 khat and v' (v' only on value-embedding layers).
@@ -236,8 +402,9 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(
     const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ ve,
     const float2* __restrict__ gate,
     __nv_bfloat16* __restrict__ qh, __nv_bfloat16* __restrict__ kh, __nv_bfloat16* __restrict__ vp,
-    const float4* __restrict__ tab32, const double2* __restrict__ tab64, int* __restrict__ sched,
-    int n_rows, int T, int H, FastDiv divT, FastDiv divH, double eps) {
+    const float4* __restrict__ tab32, int* __restrict__ sched,
+    int n_rows, int T, int H, FastDiv divT, FastDiv divH, double eps, int* __restrict__ fix_counts,
+    FixItem* __restrict__ fix_items) {
     constexpr int TPR = D / 8;           // threads per row (16 or 8); divides 32
     constexpr int LOG_TPR = (D == 128) ? 4 : 3;
     constexpr int HALF = D / 2;
@@ -251,6 +418,11 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(
         sched[0] = 0;
         sched[1] = 0;
     }
+    // This block's list of row chunks to repair (prologue_fix_kernel).
+    __shared__ int s_nfix;
+    __shared__ FixItem s_fix[kFixPerBlock];
+    if (threadIdx.x == 0) s_nfix = 0;
+    __syncthreads();
     for (long long it = 0; it < n_iter; ++it) {
         const long long tid = gtid + it * stride;
         const int row_raw = (int)(tid >> LOG_TPR);           // (b*T + t)*H + h, < 2^31
@@ -297,10 +469,20 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(
 #pragma unroll
             for (int e = 0; e < 4; ++e) cs[e] = __ldg(tp + e);
         }
-        const double2* t64 = tab64 + (long long)t * HALF + i0;
-        uint2 o0, o1, o2, o3;
-        if (DO_Q) rope_rms_pairs4<D>(raw[0], raw[1], cs, t64, eps, o0, o1);
-        if (DO_KV) rope_rms_pairs4<D>(raw[2], raw[3], cs, t64, eps, o2, o3);
+        // Fast path for every output of the row chunk (one branch-free block); a chunk with
+        // elements it cannot certify goes on the block's repair list.
+        uint2 o0, o1, o2, o3, o4 = make_uint2(0u, 0u), o5 = make_uint2(0u, 0u);
+        uint32_t mq = 0u, mk = 0u, mv = 0u;
+        double rq = 0.0, rk = 0.0;
+        {
+            float a[4], b[4];
+            if (DO_Q) mq = rope_rms_pairs4<D>(raw[0], raw[1], cs, eps, a, b, o0, o1, rq);
+            if (DO_KV) mk = rope_rms_pairs4<D>(raw[2], raw[3], cs, eps, a, b, o2, o3, rk);
+        }
+        if (HAS_VE && DO_KV) {
+            mv = gated_fast4(raw[4], raw[6], gw.x, gw.y, o4);
+            mv |= gated_fast4(raw[5], raw[7], gw.x, gw.y, o5) << 4;
+        }
         if (valid) {
             if (DO_Q) {
                 *reinterpret_cast<uint2*>(qh + off + i0) = o0;
@@ -311,12 +493,29 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(
                 *reinterpret_cast<uint2*>(kh + off + HALF + i0) = o3;
             }
             if (HAS_VE && DO_KV) {
-                const double g64 = (double)gw.x + (double)gw.y;
-                *reinterpret_cast<uint2*>(vp + off + i0) = gated_add4(raw[4], raw[6], gw.x, gw.y, g64);
-                *reinterpret_cast<uint2*>(vp + off + HALF + i0) = gated_add4(raw[5], raw[7], gw.x, gw.y, g64);
+                *reinterpret_cast<uint2*>(vp + off + i0) = o4;
+                *reinterpret_cast<uint2*>(vp + off + HALF + i0) = o5;
+            }
+        }
+        const uint32_t fw = valid ? (mq | (mk << 4) | (mv << 8)) : 0u;
+        if (fw != 0u) {
+            const int slot = atomicAdd(&s_nfix, 1);
+            if (slot < kFixPerBlock) {
+                FixItem item;
+                item.chunk_lo = (uint32_t)tid;
+                item.code = fw | ((uint32_t)(tid >> 32) << 16);
+                item.pad0 = item.pad1 = 0u;
+                item.rq = rq;
+                item.rk = rk;
+                s_fix[slot] = item;
             }
         }
     }
+    __syncthreads();
+    const int nf = s_nfix;
+    for (int i = threadIdx.x; i < min(nf, kFixPerBlock); i += blockDim.x)
+        fix_items[(long long)blockIdx.x * kFixPerBlock + i] = s_fix[i];
+    if (threadIdx.x == 0) fix_counts[blockIdx.x] = nf;
 }
 
 }  // namespace swa

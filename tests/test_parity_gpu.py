@@ -236,3 +236,27 @@ def test_prologue_bit_exact_other_constants(rope_base, eps):
     qh, kh, vp = oracle.prologue(d, rope_base=rope_base, eps=float(np.float32(eps)), parity=True)
     for name, ref in (("qh", qh), ("kh", kh), ("vp", vp)):
         assert (got[name] != _bits_of(ref)).sum().item() == 0, name
+
+
+def test_prologue_dense_repairs_overflow_the_repair_lists():
+    """Every v' element on a bf16 rounding tie: v in [1, 2), ve = 2^-8 (half a bf16 ulp there) and
+    Wg = 0 (gate 2 sigmoid(0) = 1, so v' = v + 2^-8 exactly).  The fast path flags all of them, far
+    more than a prologue block's repair list holds (three row chunks per thread at this size), so
+    the repair kernel recomputes those blocks' chunks whole; every element must still be v rounded
+    to nearest even, element by element, as the oracle gives."""
+    import oracle
+    s = LS(1, 4096, 16, 128, 0, True, seed=44)
+    d = workloads.make_layer(s)
+    g = torch.Generator().manual_seed(44)
+    mant = torch.randint(0, 128, d["v"].shape, generator=g, dtype=torch.int32)
+    d["v"] = ((0x3F80 | mant).to(torch.int16)).view(torch.bfloat16)          # 1 + m / 128
+    d["table"] = torch.full_like(d["table"], 2.0 ** -8)
+    d["Wg"] = torch.zeros_like(d["Wg"])
+    got = _prologue_on_gpu(s, parity.to_device(d))
+    _, _, vp = oracle.prologue(d, eps=float(np.float32(1e-6)), parity=True)
+    v = d["v"].float()
+    even = (mant % 2 == 0)
+    expect = torch.where(even, v, v + 2.0 ** -7)                              # ties to even
+    assert torch.equal(torch.from_numpy(vp).float(), expect)                 # the oracle agrees
+    mism = (got["vp"] != _bits_of(vp)).sum().item()
+    assert mism == 0, f"v': {mism} of {vp.size} values differ"
