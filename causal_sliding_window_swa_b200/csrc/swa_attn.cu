@@ -215,7 +215,11 @@ int device_ready(int* dev_out) {
                 cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<64, true>, (cudaFuncAttribute)smem_attr,
                                      swa::BwdCfg<64>::KV_SMEM) != cudaSuccess ||
                 cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<128, true>, (cudaFuncAttribute)smem_attr,
-                                     swa::BwdCfg<128>::KV_SMEM) != cudaSuccess) {
+                                     swa::BwdCfg<128>::KV_SMEM) != cudaSuccess ||
+                cudaFuncSetAttribute(swa::decode_attn_kernel<64>, (cudaFuncAttribute)smem_attr,
+                                     swa::DecCfg<64>::SMEM) != cudaSuccess ||
+                cudaFuncSetAttribute(swa::decode_attn_kernel<128>, (cudaFuncAttribute)smem_attr,
+                                     swa::DecCfg<128>::SMEM) != cudaSuccess) {
                 cudaGetLastError();
                 checked[dev] = 0;
                 return SWA_ERR_CUDA;
@@ -871,6 +875,94 @@ int fwd_library_ws(const void* q, const void* k, const void* v, const void* ve, 
 
 }  // namespace
 
+// The caches (B, Tmax, Hkv, D) bf16 as 3-D {D, Hkv, B * Tmax}; box = D features x 1 head x KB
+// positions, no swizzle.  Positions past B * Tmax read as zeros.
+bool make_cache_map(CUtensorMap* m, const void* base, int B, int Tmax, int Hkv, int D, int kb) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)B * Tmax};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)D, 1, (cuuint32_t)kb};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Attention of the new tokens over the window keys [lo, lo + n_keys): a cluster of n_chunks CTAs
+// per row b*H + h.  n_chunks (at most 8, the portable cluster size) is the number of the GPU's
+// resident CTA slots per row, so that one wave streams the whole window; each CTA takes whole
+// KB-key tiles.
+template <int D>
+int launch_decode_attention_d(int dev, const void* qh, const void* k_cache, const void* v_cache, const int* doc_start,
+                              void* out, float* lse, int B, int Tmax, int H, int Hkv, int lo, int n_keys,
+                              cudaStream_t st) {
+    using C = swa::DecCfg<D>;
+    CUtensorMap tk, tv;
+    if (!make_cache_map(&tk, k_cache, B, Tmax, Hkv, D, C::KB) || !make_cache_map(&tv, v_cache, B, Tmax, Hkv, D, C::KB))
+        return SWA_ERR_CUDA;
+    static int per_sm[64] = {0};
+    if (per_sm[dev] == 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, swa::decode_attn_kernel<D>, C::THREADS, C::SMEM) !=
+                cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = 1;
+        }
+        per_sm[dev] = n;
+    }
+    const long long rows = (long long)B * H;
+    const long long slots = (long long)per_sm[dev] * g_num_sms[dev];
+    const int n_tiles = (n_keys + C::KB - 1) / C::KB;
+    int n_chunks = (int)std::max<long long>(1, std::min<long long>(slots / rows, swa::kDecodeMaxCluster));
+    n_chunks = std::min(n_chunks, n_tiles);
+    const int tiles_per_chunk = (n_tiles + n_chunks - 1) / n_chunks;
+    n_chunks = (n_tiles + tiles_per_chunk - 1) / tiles_per_chunk;
+    swa::DecParams p{};
+    p.qh = static_cast<const __nv_bfloat16*>(qh);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    p.doc_start = doc_start;
+    p.H = H;
+    p.Hkv = Hkv;
+    p.Tmax = Tmax;
+    p.lo = lo;
+    p.n_keys = n_keys;
+    p.tiles_per_chunk = tiles_per_chunk;
+    const double log2e = 1.4426950408889634;
+    const double m0 = std::sqrt((double)D) * (1.0 + 1.0 / 64.0);
+    p.c1 = (float)(log2e / std::sqrt((double)D));
+    p.c2 = (float)(m0 * log2e);
+    p.m0 = (float)m0;
+    p.wait_limit_ns = wait_limit_ns();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(rows * n_chunks));
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)n_chunks;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    // may start before the prologue kernel ends (the kernel waits where it reads that kernel's output)
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, swa::decode_attn_kernel<D>, tk, tv, p) != cudaSuccess) return SWA_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+int launch_decode_attention(int dev, const void* qh, const void* k_cache, const void* v_cache, const int* doc_start,
+                            void* out, float* lse, int B, int Tmax, int H, int Hkv, int D, int lo, int n_keys,
+                            cudaStream_t st) {
+    return D == 128 ? launch_decode_attention_d<128>(dev, qh, k_cache, v_cache, doc_start, out, lse, B, Tmax, H, Hkv,
+                                                     lo, n_keys, st)
+                    : launch_decode_attention_d<64>(dev, qh, k_cache, v_cache, doc_start, out, lse, B, Tmax, H, Hkv,
+                                                    lo, n_keys, st);
+}
+
 extern "C" {
 
 int swa_attn_fwd_gqa(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
@@ -1014,18 +1106,15 @@ int swa_attn_bwd(const void* q, const void* k, const void* v, const void* ve, co
 
 // ------------------------------------------------------------- decode step with a KV cache
 //
-// Workspace: qhat of the new token (B*H*D bf16) | chunk partials (B*H*n_chunks*(D+2) fp32), each
-// section 1024-byte aligned; n_chunks covers the largest window the call can see, min(window,
-// Tmax) keys.
+// Workspace: qhat of the new token (B*H*D bf16), 1024-byte aligned.  The chunks of a row are
+// combined inside their cluster, so nothing else is stored.
 
 size_t swa_attn_decode_workspace_bytes(int B, int Tmax, int H, int D, int has_ve, int window) {
     Shape s;
     if (check_sizes(B, Tmax, H, D, &s) != SWA_OK) return 0;
-    const long long rows = (long long)B * H;
-    const int W = (window <= 0 || window >= Tmax) ? Tmax : window;
-    const long long n_chunks = (W + swa::kDecodeChunk - 1) / swa::kDecodeChunk;
     (void)has_ve;
-    return round_up((size_t)rows * D * 2) + round_up((size_t)(rows * n_chunks * (D + 2)) * sizeof(float));
+    (void)window;
+    return round_up((size_t)B * H * D * 2);
 }
 
 int swa_attn_decode_doc(const void* q, const void* k, const void* v, const void* ve,
@@ -1051,7 +1140,6 @@ int swa_attn_decode_doc(const void* q, const void* k, const void* v, const void*
     const int rows = B * H;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     bf* qh = reinterpret_cast<bf*>(ws);
-    float* part = reinterpret_cast<float*>(ws + round_up((size_t)rows * D * 2));
     {
         const int rows_per_block = 256 / (D / 8);
         const int blocks = std::max(1, std::min((rows + rows_per_block - 1) / rows_per_block, 148 * 8));
@@ -1095,55 +1183,7 @@ int swa_attn_decode_doc(const void* q, const void* k, const void* v, const void*
     const int W = (window <= 0 || window >= Tmax) ? Tmax : window;
     const int lo = std::max(0, pos - W + 1);
     const int n_keys = pos - lo + 1;
-    // Keys per CTA: the multiple of 32 (at least kDecodeChunk) whose grid fills the GPU's resident
-    // CTA slots best over whole waves (fewer, fuller waves; ties to the smaller chunk).
-    int chunk_keys = swa::kDecodeChunk;
-    {
-        static int per_sm[64][2] = {{0}};
-        int& cached = per_sm[dev][D == 128 ? 1 : 0];
-        if (cached == 0) {
-            int n = 0;
-            const cudaError_t e = D == 128
-                ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, swa::decode_attn_kernel<128>, 128, 0)
-                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, swa::decode_attn_kernel<64>, 128, 0);
-            if (e != cudaSuccess || n < 1) {
-                cudaGetLastError();
-                n = 1;
-            }
-            cached = n;
-        }
-        const long long slots = (long long)cached * g_num_sms[dev];
-        double best = -1.0;
-        for (int ck = swa::kDecodeChunk; ck <= 1024; ck += 32) {
-            const long long ctas = (long long)rows * ((n_keys + ck - 1) / ck);
-            const long long waves = (ctas + slots - 1) / slots;
-            const double fill = (double)ctas / (double)(waves * slots);
-            if (fill > best + 1e-9) {
-                best = fill;
-                chunk_keys = ck;
-            }
-            if (ck >= n_keys) break;
-        }
-    }
-    const int n_chunks = (n_keys + chunk_keys - 1) / chunk_keys;
-    const double log2e = 1.4426950408889634;
-    const double m0 = std::sqrt((double)D) * (1.0 + 1.0 / 64.0);
-    const float c1 = (float)(log2e / std::sqrt((double)D)), c2 = (float)(m0 * log2e);
-    const unsigned grid = (unsigned)((long long)rows * n_chunks);
-    const bf* qc = qh;
-    const bf* kcc = static_cast<const bf*>(k_cache);
-    const bf* vcc = static_cast<const bf*>(v_cache);
-    bf* o = static_cast<bf*>(out);
-    if (D == 128) {
-        swa::decode_attn_kernel<128><<<grid, 128, 0, st>>>(qc, kcc, vcc, part, H, Hkv, Tmax, lo, n_keys, n_chunks,
-                                                           chunk_keys, c1, c2, doc_start);
-        swa::decode_combine_kernel<128><<<rows, 128, 0, st>>>(part, o, lse, n_chunks, (float)m0);
-    } else {
-        swa::decode_attn_kernel<64><<<grid, 128, 0, st>>>(qc, kcc, vcc, part, H, Hkv, Tmax, lo, n_keys, n_chunks,
-                                                          chunk_keys, c1, c2, doc_start);
-        swa::decode_combine_kernel<64><<<rows, 64, 0, st>>>(part, o, lse, n_chunks, (float)m0);
-    }
-    return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+    return launch_decode_attention(dev, qh, k_cache, v_cache, doc_start, out, lse, B, Tmax, H, Hkv, D, lo, n_keys, st);
 }
 
 int swa_attn_decode_gqa(const void* q, const void* k, const void* v, const void* ve,

@@ -130,11 +130,10 @@ def test_selftest_wait_rejects_limits_out_of_range():
 
 
 def test_decode_workspace_and_validation():
-    # qhat (B*H*D bf16) + chunk partials for the largest window, each section 1024-byte aligned
+    # qhat (B*H*D bf16), 1024-byte aligned; the chunks of a row are combined inside their cluster
     n = swa.swa_attn_decode_workspace_bytes(2, 1000, 3, 64, 0, 0)
-    chunks = (1000 + 127) // 128
-    assert n == 1024 + ((2 * 3 * chunks * 66 * 4 + 1023) // 1024) * 1024
-    assert swa.swa_attn_decode_workspace_bytes(2, 1000, 3, 64, 0, 200) < n
+    assert n == 1024
+    assert swa.swa_attn_decode_workspace_bytes(16, 1000, 12, 128, 1, 200) == 16 * 12 * 128 * 2
     assert swa.swa_attn_decode_workspace_bytes(2, 1000, 3, 96, 0, 0) == 0
     need = swa.swa_attn_decode_workspace_bytes(1, 16, 1, 64, 0, 0)
     base = dict(q=A, k=A, v=A, ve=None, gate_x=None, Wg=None, k_cache=A, v_cache=A, out=A, lse=A,
@@ -159,12 +158,12 @@ def test_backward_workspace_and_validation():
     # forward sections + row statistics (B*H*Tp float2) + dqhat (fp32) + dkhat, dv' (fp32, Hkv heads)
     # [+ dz and the dWg partial sums on value-embedding layers] + document starts and ends (B*T int32
     # each), each section 1024-byte aligned.  The forward's prologue repair lists (an int count and
-    # 512 (chunk, flags) items per block of each prologue pass; 256-thread blocks, D/8 threads per
-    # row, at most 1776 blocks a pass) take two passes under grouped-query attention, one otherwise.
+    # 256 32-byte items per block of each prologue pass; 256-thread blocks, D/8 threads per row, at
+    # most 1776 blocks a pass) take two passes under grouped-query attention, one otherwise.
     B, T, H, Hkv, D = 2, 200, 4, 2, 64
     up = lambda x: (x + 1023) // 1024 * 1024
     blocks = lambda rows: max(1, min((rows * (D // 8) + 255) // 256, 1776))
-    fix = lambda lists: up(lists * 4) + up(lists * 512 * 8)
+    fix = lambda lists: up(lists * 4) + up(lists * 256 * 32)
     fwd = swa.swa_attn_workspace_bytes(B, T, H, D, 0)
     n0 = swa.swa_attn_bwd_workspace_bytes(B, T, H, Hkv, D, 0)
     Tp = 256

@@ -22,6 +22,9 @@ CASES = [
     # grouped-query layers: caches with Hkv heads, query head h reads key/value head h / (H/Hkv)
     workloads.LayerShape(B=2, T=180, H=4, D=64, window=50, ve=True, seed=15, kv_heads=2, name="decode gqa D64 H4/2 W50 VE"),
     workloads.LayerShape(B=1, T=260, H=6, D=128, window=0, ve=False, seed=16, kv_heads=3, name="decode gqa D128 H6/3 full"),
+    # many rows: few chunks per row, each longer than the four-stage tile ring
+    workloads.LayerShape(B=8, T=600, H=12, D=128, window=0, ve=True, seed=17, name="decode D128 96 rows full VE"),
+    workloads.LayerShape(B=16, T=1000, H=12, D=64, window=700, ve=False, seed=18, name="decode D64 192 rows W700"),
 ]
 
 
