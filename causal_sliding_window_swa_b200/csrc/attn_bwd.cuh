@@ -25,8 +25,9 @@
 //                         P^T first and dS^T second, so that dV += P^T dO and the next S^T run
 //                         while dS^T is formed, and dK += dS^T Q and the next dP^T while the next
 //                         P^T is.
-//   bwd_qk_rows_kernel    dq (dk) = RoPE^T applied to the RMS backward of dqhat (dkhat).
-//   bwd_v_rows_kernel     dv = dv', dve = g dv', dz = (dv' . ve) g (1 - g / 2) per row.
+//   Both tensor-core kernels end each item with the prologue in reverse for their rows: dq (dk)
+//   = RoPE^T applied to the RMS backward of dqhat (dkhat), with the row sums exchanged between
+//   the four threads of a row; dv = dv', dve = g dv', dz = (dv' . ve) g (1 - g / 2).
 //   bwd_gate_x_kernel, bwd_wg_partial_kernel, bwd_wg_final_kernel
 //                         dgate_x = dz Wg^T and dWg = gate_x^T dz (fixed summation order).
 // The two tensor-core kernels use seven products per (query tile, key tile) pair instead of
@@ -63,14 +64,17 @@ struct BwdCfg {
     static constexpr uint32_t TMEM_COLS = 512;
     // query-tile kernel: Q | dO | NS-stage ring of K and V' tiles | barriers
     static constexpr int DQ_NS = (D == 128) ? 4 : 10;
-    static constexpr int DQ_SMEM = 2 * TILE_BYTES + DQ_NS * TILE_BYTES + SMEM_BAR;
+    static constexpr int DQ_RED = 2 * 4 * 128 * 8;      // row-sum exchange, two buffers of [4][128] float2
+    static constexpr int THETA_BYTES = 512;            // theta_i, fp64, i < D / 2
+    static constexpr int DQ_SMEM = 2 * TILE_BYTES + DQ_NS * TILE_BYTES + SMEM_BAR + DQ_RED + THETA_BYTES;
     static constexpr uint32_t DQ_COL_S = 0;            // S(0) | S(1), each then dS as bf16 pairs
     static constexpr uint32_t DQ_COL_DP = 256;
     static constexpr uint32_t DQ_COL_DQ = 384;         // D fp32 columns
     // key-tile kernel: K | V' | NS stages of (Q tile, dO tile, 128 row statistics) | barriers
     static constexpr int STAGE_BYTES = 2 * TILE_BYTES + 1024;
     static constexpr int KV_NS = (D == 128) ? 2 : 5;
-    static constexpr int KV_SMEM = 2 * TILE_BYTES + KV_NS * STAGE_BYTES + SMEM_BAR;
+    static constexpr int KV_RED = 2 * 4 * 128 * 16;     // row-sum exchange, two buffers of [4][128] float4
+    static constexpr int KV_SMEM = 2 * TILE_BYTES + KV_NS * STAGE_BYTES + SMEM_BAR + KV_RED + THETA_BYTES;
     static constexpr uint32_t KV_COL_ST = 0;           // S^T, then P^T as bf16 pairs
     static constexpr uint32_t KV_COL_DPT = 128;        // dP^T, then dS^T as bf16 pairs
     static constexpr uint32_t KV_COL_DV = 256;
@@ -90,9 +94,18 @@ struct BwdParams {
     float c1;              // log2(e) / sqrt(D): raw score -> log2 units
     float inv_sqrt_d;
     const float2* rowstat; // (B, H, Tp): (lse log2 e, delta - dlse); padding rows (+inf, 0)
-    float* dqh;            // (B, T, H, D) fp32: dL/dqhat
-    float* dkh;            // (B, T, Hkv, D) fp32: dL/dkhat
-    float* dvp;            // (B, T, Hkv, D) fp32: dL/dv'
+    // the prologue in reverse, applied in the epilogues
+    const __nv_bfloat16* xq;   // (B, T, H, D) raw q
+    const __nv_bfloat16* xk;   // (B, T, Hkv, D) raw k
+    const __nv_bfloat16* ve;   // (B, T, Hkv, D) value embedding, or null
+    const float2* gate;        // (B, T, Hkv) gate as (g_hi, g_lo), or null
+    double rope_base;          // theta_i = rope_base^(-2 i / D)
+    float eps;
+    __nv_bfloat16* dq;         // (B, T, H, D)
+    __nv_bfloat16* dk;         // (B, T, Hkv, D)
+    __nv_bfloat16* dv;         // (B, T, Hkv, D)
+    __nv_bfloat16* dve;        // (B, T, Hkv, D), value-embedding layers
+    float* dz;                 // (B, T, Hkv): dL/dz of the gate's logit, value-embedding layers
     int* sched;            // [0] next item, [1] CTAs done; zero before the launch, reset after
     unsigned long long wait_limit_ns;
     const int* dstart;     // (B, T) first position of each position's document, or null (no mask)
@@ -103,7 +116,7 @@ struct BwdParams {
 enum : unsigned int {
     kSiteBwdQFull = 40, kSiteBwdQEmpty = 41, kSiteBwdKvFull = 42, kSiteBwdKvEmpty = 43,
     kSiteBwdSFull = 44, kSiteBwdPFull = 45, kSiteBwdOFull = 46, kSiteBwdOEmpty = 47,
-    kSiteBwdItem = 48, kSiteBwdDrain = 49, kSiteBwdStage = 50
+    kSiteBwdItem = 48, kSiteBwdDrain = 49, kSiteBwdStage = 50, kSiteBwdRed = 51
 };
 
 // Query-tile item: tile [q0, q0 + 127] of (b, h) and the key tiles lo..hi of its band; order as
@@ -162,6 +175,112 @@ __device__ __forceinline__ BwdKvItem bwd_kv_item(const BwdParams& p, int it) {
 template <int D>
 __device__ __forceinline__ uint64_t kmajor_step(int kk) {
     return (uint64_t)(((kk >> 2) * BwdCfg<D>::CHUNK_BYTES + (kk & 3) * 32) >> 4);
+}
+
+// ------------------------------------------------------------------- epilogue helpers
+// An epilogue thread owns NP = D / 8 rotation pairs of one row, i in [i0, i0 + NP) with
+// i0 = NP * (output quarter): elements i and i + D/2, so the rotation needs no other thread; the
+// row sums are exchanged through shared memory between the four threads of the row.
+
+template <int NP>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NP]) {
+    if constexpr (NP == 16)
+        tmem_ld16(taddr, r);
+    else
+        tmem_ld8(taddr, r);
+}
+
+// NP consecutive bf16 at p (16-byte aligned) -> fp32.
+template <int NP>
+__device__ __forceinline__ void load_bf16_row(const __nv_bfloat16* p, float (&x)[NP]) {
+#pragma unroll
+    for (int q = 0; q < NP / 8; ++q) {
+        const uint4 u = *reinterpret_cast<const uint4*>(p + 8 * q);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            x[8 * q + 2 * e] = __uint_as_float(w[e] << 16);
+            x[8 * q + 2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+        }
+    }
+}
+
+// The same load kept packed (NP / 2 registers) until unpack_bf16_row.
+template <int NP>
+__device__ __forceinline__ void load_bf16_raw(const __nv_bfloat16* p, uint4 (&u)[NP / 8]) {
+#pragma unroll
+    for (int q = 0; q < NP / 8; ++q) u[q] = *reinterpret_cast<const uint4*>(p + 8 * q);
+}
+
+template <int NP>
+__device__ __forceinline__ void unpack_bf16_row(const uint4 (&u)[NP / 8], float (&x)[NP]) {
+#pragma unroll
+    for (int q = 0; q < NP / 8; ++q) {
+        const uint32_t w[4] = {u[q].x, u[q].y, u[q].z, u[q].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            x[8 * q + 2 * e] = __uint_as_float(w[e] << 16);
+            x[8 * q + 2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+        }
+    }
+}
+
+template <int NP>
+__device__ __forceinline__ void store_bf16_row(__nv_bfloat16* p, const float (&y)[NP]) {
+#pragma unroll
+    for (int q = 0; q < NP / 8; ++q)
+        *reinterpret_cast<uint4*>(p + 8 * q) =
+            make_uint4(pack_bf16x2(y[8 * q], y[8 * q + 1]), pack_bf16x2(y[8 * q + 2], y[8 * q + 3]),
+                       pack_bf16x2(y[8 * q + 4], y[8 * q + 5]), pack_bf16x2(y[8 * q + 6], y[8 * q + 7]));
+}
+
+// RMS backward then RoPE transposed, for this thread's pairs: g = dL/dxhat (ga at i, gb at
+// i + D/2), x the raw input row, tab its RoPE (cos, sin).  With u = R^T g (ua = ga c + gb s,
+// ub = gb c - ga s), the row sums ss = sum x^2 and xu = sum x . u give
+// dx = r u - r^3 (xu / D) x, r = 1 / sqrt(ss / D + eps).  Phase 1 returns this thread's partial
+// sums and fills ua, ub; phase 2 takes the row's sums.
+// cos and sin of t theta_i for this thread's NP frequencies (theta from shared memory, fp64): the
+// angle is formed and reduced to [-pi, pi] in fp64 (error below 1e-11), then evaluated on the
+// special-function unit in fp32 (absolute error about 1e-6, well inside the gradient's tolerance).
+template <int NP>
+__device__ __forceinline__ void rope_cs_fast(int t, const double* __restrict__ theta, float (&c)[NP], float (&sn)[NP]) {
+    constexpr double kTwoPi = 6.283185307179586;
+    constexpr double kInvTwoPi = 0.15915494309189535;
+#pragma unroll
+    for (int e = 0; e < NP; ++e) {
+        const double a = (double)t * theta[e];
+        const double red = fma(-rint(a * kInvTwoPi), kTwoPi, a);
+        __sincosf((float)red, &sn[e], &c[e]);
+    }
+}
+
+template <int NP>
+__device__ __forceinline__ void rms_rope_bwd_partial(const float (&ga)[NP], const float (&gb)[NP],
+                                                     const float (&xa)[NP], const float (&xb)[NP],
+                                                     const float (&cc)[NP], const float (&ssn)[NP], float (&ua)[NP],
+                                                     float (&ub)[NP], float& ss, float& xu) {
+    ss = 0.f;
+    xu = 0.f;
+#pragma unroll
+    for (int e = 0; e < NP; ++e) {
+        const float c = cc[e], sn = ssn[e];
+        ua[e] = ga[e] * c + gb[e] * sn;
+        ub[e] = gb[e] * c - ga[e] * sn;
+        ss += xa[e] * xa[e] + xb[e] * xb[e];
+        xu += xa[e] * ua[e] + xb[e] * ub[e];
+    }
+}
+
+template <int NP>
+__device__ __forceinline__ void rms_rope_bwd_finish(float ss, float xu, int D, float eps, const float (&ua)[NP],
+                                                    const float (&ub)[NP], float (&xa)[NP], float (&xb)[NP]) {
+    const float rr = rsqrtf(ss / (float)D + eps);
+    const float coef = rr * rr * rr * xu / (float)D;
+#pragma unroll
+    for (int e = 0; e < NP; ++e) {
+        xa[e] = rr * ua[e] - coef * xa[e];
+        xb[e] = rr * ub[e] - coef * xb[e];
+    }
 }
 
 // ------------------------------------------------------------------- row statistics
@@ -246,8 +365,11 @@ __global__ void __launch_bounds__(576, 1)
     uint64_t* b_pfull = bars + 10;               // dS(g) written to tensor memory
     uint64_t* b_kvfull = bars + 11;              // [NS]
     uint64_t* b_kvempty = bars + 11 + NS;        // [NS]
-    int* s_item = reinterpret_cast<int*>(bars + 11 + 2 * NS);   // [2]
+    uint64_t* b_red = bars + 11 + 2 * NS;        // [2] row sums of an epilogue written
+    int* s_item = reinterpret_cast<int*>(bars + 13 + 2 * NS);   // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_item + 2);
+    float2* s_red = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(bars) + C::SMEM_BAR);   // [2][4][128]
+    double* s_theta = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(s_red) + C::DQ_RED);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -272,6 +394,7 @@ __global__ void __launch_bounds__(576, 1)
             mbar_init(smem_u32(b_kvfull + s), 1);
             mbar_init(smem_u32(b_kvempty + s), 1);
         }
+        for (int i = 0; i < 2; ++i) mbar_init(smem_u32(b_red + i), C::SOFTMAX_THREADS);
         fence_barrier_init();
     }
     if (warp == kMmaWarp) {
@@ -284,6 +407,8 @@ __global__ void __launch_bounds__(576, 1)
         tma_prefetch_desc(&tm_v);
         tma_prefetch_desc(&tm_do);
     }
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + D / 2)
+        s_theta[threadIdx.x - 64] = pow(p.rope_base, -2.0 * (double)(threadIdx.x - 64) / (double)D);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -458,6 +583,9 @@ __global__ void __launch_bounds__(576, 1)
             if (!ok || it < 0) break;
             const BwdQItem m = bwd_q_item(p, it);
             const int qi = m.q0 + r;
+            // the epilogue's raw q row, into L2 while the item's tiles are worked on
+            if (cq < D / 64 && qi < p.T)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(p.xq + (((long long)m.b * p.T + qi) * p.H + m.h) * D + 64 * cq));
             // document mask: this row sees no key before its document's start
             const int ds = DOC ? __ldg(p.dstart + (long long)m.b * p.T + min(qi, p.T - 1)) : 0;
             const float2 rs = p.rowstat[((long long)m.b * p.H + m.h) * p.Tp + qi];
@@ -496,30 +624,56 @@ __global__ void __launch_bounds__(576, 1)
                 mbar_arrive(smem_u32(b_pfull));
             }
             if (!ok) break;
+            // The raw q row (the epilogue's input that does not depend on dQ) is fetched while the
+            // item's last dQ product runs.
+            constexpr int NP = D / 8;
+            const int i0 = NP * cq;
+            const bool live = qi < p.T;
+            const int qc = min(qi, p.T - 1);
+            const long long roff = (((long long)m.b * p.T + qc) * p.H + m.h) * D;
+            uint4 xra[NP / 8], xrb[NP / 8];
+            load_bf16_raw<NP>(p.xq + roff + i0, xra);
+            load_bf16_raw<NP>(p.xq + roff + D / 2 + i0, xrb);
             {
                 const bool w = mbar_wait(smem_u32(b_ofull), o_uses & 1u, lim, kSiteBwdOFull);
                 ok = __all_sync(0xffffffffu, w);
             }
             if (!ok) break;
             tc_fence_after();
-            constexpr int OQ = D / 4;   // output columns per thread: 32 or 16
-            uint32_t ov[OQ];
-            tmem_ld16(tmem + lane_base + C::DQ_COL_DQ + (uint32_t)(OQ * cq), *reinterpret_cast<uint32_t(*)[16]>(ov));
-            if constexpr (OQ == 32)
-                tmem_ld16(tmem + lane_base + C::DQ_COL_DQ + (uint32_t)(OQ * cq) + 16u,
-                          *reinterpret_cast<uint32_t(*)[16]>(ov + 16));
+            // dqhat of this thread's pairs (columns i0 .. and D/2 + i0 ..), then dq = RoPE^T of the
+            // RMS backward (the prologue in reverse)
+            uint32_t gau[NP], gbu[NP];
+            tmem_ld_cols<NP>(tmem + lane_base + C::DQ_COL_DQ + (uint32_t)i0, gau);
+            tmem_ld_cols<NP>(tmem + lane_base + C::DQ_COL_DQ + (uint32_t)(D / 2 + i0), gbu);
             tmem_ld_wait();
             tc_fence_before();
             mbar_arrive(smem_u32(b_oempty));
-            ++o_uses;
-            if (qi < p.T) {
-                float4* dst = reinterpret_cast<float4*>(p.dqh + (((long long)m.b * p.T + qi) * p.H + m.h) * D + OQ * cq);
+            const uint32_t e_idx = o_uses++;
+            float xa[NP], xb[NP], cc[NP], sn[NP], ga[NP], gb[NP], ua[NP], ub[NP];
+            unpack_bf16_row<NP>(xra, xa);
+            unpack_bf16_row<NP>(xrb, xb);
+            rope_cs_fast<NP>(qc, s_theta + i0, cc, sn);
 #pragma unroll
-                for (int e = 0; e < OQ / 4; ++e)
-                    dst[e] = make_float4(__uint_as_float(ov[4 * e]) * p.inv_sqrt_d,
-                                         __uint_as_float(ov[4 * e + 1]) * p.inv_sqrt_d,
-                                         __uint_as_float(ov[4 * e + 2]) * p.inv_sqrt_d,
-                                         __uint_as_float(ov[4 * e + 3]) * p.inv_sqrt_d);
+            for (int e = 0; e < NP; ++e) {
+                ga[e] = __uint_as_float(gau[e]) * p.inv_sqrt_d;
+                gb[e] = __uint_as_float(gbu[e]) * p.inv_sqrt_d;
+            }
+            float ss, xu;
+            rms_rope_bwd_partial<NP>(ga, gb, xa, xb, cc, sn, ua, ub, ss, xu);
+            float2* red = s_red + (e_idx & 1u) * 512u;
+            red[cq * 128 + r] = make_float2(ss, xu);
+            mbar_arrive(smem_u32(b_red + (e_idx & 1u)));
+            {
+                const bool w = mbar_wait(smem_u32(b_red + (e_idx & 1u)), (e_idx >> 1) & 1u, lim, kSiteBwdRed);
+                ok = __all_sync(0xffffffffu, w);
+            }
+            if (!ok) break;
+            const float2 t0 = red[r], t1 = red[128 + r], t2 = red[256 + r], t3 = red[384 + r];
+            rms_rope_bwd_finish<NP>((t0.x + t1.x) + (t2.x + t3.x), (t0.y + t1.y) + (t2.y + t3.y), D, p.eps, ua, ub,
+                                    xa, xb);
+            if (live) {
+                store_bf16_row<NP>(p.dq + roff + i0, xa);
+                store_bf16_row<NP>(p.dq + roff + D / 2 + i0, xb);
             }
         }
     }
@@ -570,8 +724,11 @@ __global__ void __launch_bounds__(576, 1)
     uint64_t* b_dsready = bars + 12;             // dS^T(s) written
     uint64_t* b_stfull = bars + 13;              // [NS]
     uint64_t* b_stempty = bars + 13 + NS;        // [NS]
-    int* s_item = reinterpret_cast<int*>(bars + 13 + 2 * NS);
+    uint64_t* b_red = bars + 13 + 2 * NS;        // [2] row sums of an epilogue written
+    int* s_item = reinterpret_cast<int*>(bars + 15 + 2 * NS);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_item + 2);
+    float4* s_red = reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(bars) + C::SMEM_BAR);   // [2][4][128]
+    double* s_theta = reinterpret_cast<double*>(reinterpret_cast<uint8_t*>(s_red) + C::KV_RED);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -598,6 +755,7 @@ __global__ void __launch_bounds__(576, 1)
             mbar_init(smem_u32(b_stfull + s), 1);
             mbar_init(smem_u32(b_stempty + s), 1);
         }
+        for (int i = 0; i < 2; ++i) mbar_init(smem_u32(b_red + i), C::SOFTMAX_THREADS);
         fence_barrier_init();
     }
     if (warp == kMmaWarp) {
@@ -610,6 +768,8 @@ __global__ void __launch_bounds__(576, 1)
         tma_prefetch_desc(&tm_v);
         tma_prefetch_desc(&tm_do);
     }
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + D / 2)
+        s_theta[threadIdx.x - 64] = pow(p.rope_base, -2.0 * (double)(threadIdx.x - 64) / (double)D);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -793,6 +953,12 @@ __global__ void __launch_bounds__(576, 1)
             if (!ok || it < 0) break;
             const BwdKvItem m = bwd_kv_item(p, it);
             const int key = m.k0 + r;
+            // the epilogue's raw k and value-embedding rows, into L2 while the item is worked on
+            if (cq < D / 64 && key < p.T) {
+                const long long o = (((long long)m.b * p.T + key) * p.Hkv + m.hk) * D + 64 * cq;
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(p.xk + o));
+                if (p.ve != nullptr) asm volatile("prefetch.global.L2 [%0];" ::"l"(p.ve + o));
+            }
             // document mask: no query past this key's document end sees it
             const int de = DOC ? __ldg(p.dend + (long long)m.b * p.T + min(key, p.T - 1)) : 0;
             const int nq = m.hi - m.lo + 1;
@@ -858,39 +1024,102 @@ __global__ void __launch_bounds__(576, 1)
                 mbar_arrive(smem_u32(b_dsready));
             }
             if (!ok) break;
+            // dK and dV' of this thread's pairs (columns i0 .. and D/2 + i0 ..); then the prologue in
+            // reverse: dk = RoPE^T of the RMS backward (raw k row), dv = dv', and on value-embedding
+            // layers dve = g dv' and dz = (dv' . ve) g (1 - g / 2), the derivative of g = 2 sigmoid(z)
+            // being 2 sigmoid (1 - sigmoid).  The raw k row (an input that does not depend on the
+            // products) is fetched while the item's last products run.
+            constexpr int NP = D / 8;
+            const int i0 = NP * cq;
+            const bool live = key < p.T;
+            const int kc = min(key, p.T - 1);
+            const long long rrow = ((long long)m.b * p.T + kc) * p.Hkv + m.hk;
+            const long long roff = rrow * D;
+            uint4 xra[NP / 8], xrb[NP / 8], era[NP / 8], erb[NP / 8];
+            load_bf16_raw<NP>(p.xk + roff + i0, xra);
+            load_bf16_raw<NP>(p.xk + roff + D / 2 + i0, xrb);
+            float g = 0.f;
             {
                 const bool w = mbar_wait(smem_u32(b_ofull), o_uses & 1u, lim, kSiteBwdOFull);
                 ok = __all_sync(0xffffffffu, w);
             }
             if (!ok) break;
             tc_fence_after();
-            constexpr int OQ = D / 4;
-            uint32_t ovv[OQ], okk[OQ];
-            tmem_ld16(tmem + lane_base + C::KV_COL_DV + (uint32_t)(OQ * cq), *reinterpret_cast<uint32_t(*)[16]>(ovv));
-            tmem_ld16(tmem + lane_base + C::KV_COL_DK + (uint32_t)(OQ * cq), *reinterpret_cast<uint32_t(*)[16]>(okk));
-            if constexpr (OQ == 32) {
-                tmem_ld16(tmem + lane_base + C::KV_COL_DV + (uint32_t)(OQ * cq) + 16u,
-                          *reinterpret_cast<uint32_t(*)[16]>(ovv + 16));
-                tmem_ld16(tmem + lane_base + C::KV_COL_DK + (uint32_t)(OQ * cq) + 16u,
-                          *reinterpret_cast<uint32_t(*)[16]>(okk + 16));
-            }
-            tmem_ld_wait();
-            tc_fence_before();
-            mbar_arrive(smem_u32(b_oempty));
-            ++o_uses;
-            if (key < p.T) {
-                const long long off = (((long long)m.b * p.T + key) * p.Hkv + m.hk) * D + OQ * cq;
-                float4* dvd = reinterpret_cast<float4*>(p.dvp + off);
-                float4* dkd = reinterpret_cast<float4*>(p.dkh + off);
+            // dV' first: dv = dv', dve = g dv' and this thread's part of dv' . ve
+            float dvve = 0.f;
+            {
+                uint32_t vau[NP], vbu[NP];
+                tmem_ld_cols<NP>(tmem + lane_base + C::KV_COL_DV + (uint32_t)i0, vau);
+                tmem_ld_cols<NP>(tmem + lane_base + C::KV_COL_DV + (uint32_t)(D / 2 + i0), vbu);
+                tmem_ld_wait();
+                float va[NP], vb[NP];
 #pragma unroll
-                for (int e = 0; e < OQ / 4; ++e) {
-                    dvd[e] = make_float4(__uint_as_float(ovv[4 * e]), __uint_as_float(ovv[4 * e + 1]),
-                                         __uint_as_float(ovv[4 * e + 2]), __uint_as_float(ovv[4 * e + 3]));
-                    dkd[e] = make_float4(__uint_as_float(okk[4 * e]) * p.inv_sqrt_d,
-                                         __uint_as_float(okk[4 * e + 1]) * p.inv_sqrt_d,
-                                         __uint_as_float(okk[4 * e + 2]) * p.inv_sqrt_d,
-                                         __uint_as_float(okk[4 * e + 3]) * p.inv_sqrt_d);
+                for (int e = 0; e < NP; ++e) {
+                    va[e] = __uint_as_float(vau[e]);
+                    vb[e] = __uint_as_float(vbu[e]);
                 }
+                if (live) {
+                    store_bf16_row<NP>(p.dv + roff + i0, va);
+                    store_bf16_row<NP>(p.dv + roff + D / 2 + i0, vb);
+                }
+                if (p.ve != nullptr) {
+                    load_bf16_raw<NP>(p.ve + roff + i0, era);
+                    load_bf16_raw<NP>(p.ve + roff + D / 2 + i0, erb);
+                    const float2 gg = p.gate[rrow];
+                    g = gg.x + gg.y;
+                    float ea[NP], eb[NP];
+                    unpack_bf16_row<NP>(era, ea);
+                    unpack_bf16_row<NP>(erb, eb);
+#pragma unroll
+                    for (int e = 0; e < NP; ++e) {
+                        dvve += va[e] * ea[e] + vb[e] * eb[e];
+                        va[e] *= g;
+                        vb[e] *= g;
+                    }
+                    if (live) {
+                        store_bf16_row<NP>(p.dve + roff + i0, va);
+                        store_bf16_row<NP>(p.dve + roff + D / 2 + i0, vb);
+                    }
+                }
+            }
+            // then dK: dk = RoPE^T of the RMS backward, with the raw k row
+            float xa[NP], xb[NP], ua[NP], ub[NP];
+            float ss, xu;
+            {
+                uint32_t kau[NP], kbu[NP];
+                tmem_ld_cols<NP>(tmem + lane_base + C::KV_COL_DK + (uint32_t)i0, kau);
+                tmem_ld_cols<NP>(tmem + lane_base + C::KV_COL_DK + (uint32_t)(D / 2 + i0), kbu);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(smem_u32(b_oempty));
+                unpack_bf16_row<NP>(xra, xa);
+                unpack_bf16_row<NP>(xrb, xb);
+                float ga[NP], gb[NP];
+#pragma unroll
+                for (int e = 0; e < NP; ++e) {
+                    ga[e] = __uint_as_float(kau[e]) * p.inv_sqrt_d;
+                    gb[e] = __uint_as_float(kbu[e]) * p.inv_sqrt_d;
+                }
+                float cc[NP], sn[NP];
+                rope_cs_fast<NP>(kc, s_theta + i0, cc, sn);
+                rms_rope_bwd_partial<NP>(ga, gb, xa, xb, cc, sn, ua, ub, ss, xu);
+            }
+            const uint32_t e_idx = o_uses++;
+            float4* red = s_red + (e_idx & 1u) * 512u;
+            red[cq * 128 + r] = make_float4(ss, xu, dvve, 0.f);
+            mbar_arrive(smem_u32(b_red + (e_idx & 1u)));
+            {
+                const bool w = mbar_wait(smem_u32(b_red + (e_idx & 1u)), (e_idx >> 1) & 1u, lim, kSiteBwdRed);
+                ok = __all_sync(0xffffffffu, w);
+            }
+            if (!ok) break;
+            const float4 t0 = red[r], t1 = red[128 + r], t2 = red[256 + r], t3 = red[384 + r];
+            rms_rope_bwd_finish<NP>((t0.x + t1.x) + (t2.x + t3.x), (t0.y + t1.y) + (t2.y + t3.y), D, p.eps, ua, ub,
+                                    xa, xb);
+            if (live) {
+                store_bf16_row<NP>(p.dk + roff + i0, xa);
+                store_bf16_row<NP>(p.dk + roff + D / 2 + i0, xb);
+                if (p.ve != nullptr && cq == 0) p.dz[rrow] = ((t0.z + t1.z) + (t2.z + t3.z)) * g * (1.f - 0.5f * g);
             }
         }
     }
@@ -903,88 +1132,7 @@ __global__ void __launch_bounds__(576, 1)
     }
 }
 
-// ------------------------------------------------------------- the prologue in reverse
-
-// dL/d(raw row) of q or k from dy = dL/d(normalised row), one warp per (b, t, head) row.
-// With x the raw row, R_t the rotation at position t, r = (|x|^2 / D + eps)^(-1/2) (the rotation
-// keeps the norm) and u = R_t^T dy:  dx = r u - (r^3 / D) (x . u) x.  Lane l holds the pairs
-// (i, i + D/2) for i = l P .. l P + P - 1, P = D / 64.
-template <int D>
-__global__ void bwd_qk_rows_kernel(const __nv_bfloat16* __restrict__ src, const float* __restrict__ dy,
-                                   __nv_bfloat16* __restrict__ dx, const double2* __restrict__ tab64,
-                                   int n_rows, int T, int heads, float eps) {
-    constexpr int P = D / 64;
-    constexpr int HALF = D / 2;
-    const int lane = threadIdx.x & 31;
-    const int warps = gridDim.x * (blockDim.x >> 5);
-    for (int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < n_rows; row += warps) {
-        const int t = (row / heads) % T;
-        const long long base = (long long)row * D;
-        const int i0 = lane * P;
-        float xa[P], xb[P], ua[P], ub[P];
-        float ss = 0.f, xu = 0.f;
-#pragma unroll
-        for (int e = 0; e < P; ++e) {
-            const int i = i0 + e;
-            xa[e] = __bfloat162float(src[base + i]);
-            xb[e] = __bfloat162float(src[base + i + HALF]);
-            const float ga = dy[base + i], gb = dy[base + i + HALF];
-            const double2 cs = tab64[(long long)t * HALF + i];
-            const float c = (float)cs.x, s = (float)cs.y;
-            ua[e] = ga * c + gb * s;
-            ub[e] = gb * c - ga * s;
-            ss += xa[e] * xa[e] + xb[e] * xb[e];
-            xu += xa[e] * ua[e] + xb[e] * ub[e];
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            xu += __shfl_xor_sync(0xffffffffu, xu, o);
-        }
-        const float rr = rsqrtf(ss / (float)D + eps);
-        const float coef = rr * rr * rr * xu / (float)D;
-#pragma unroll
-        for (int e = 0; e < P; ++e) {
-            const int i = i0 + e;
-            dx[base + i] = __float2bfloat16_rn(rr * ua[e] - coef * xa[e]);
-            dx[base + i + HALF] = __float2bfloat16_rn(rr * ub[e] - coef * xb[e]);
-        }
-    }
-}
-
-// dv = dv'; on value-embedding layers dve = g dv' and dz = (dv' . ve) g (1 - g / 2), the
-// derivative of g = 2 sigmoid(z) being 2 sigmoid (1 - sigmoid).  One warp per (b, t, hk) row.
-template <int D, bool HAS_VE>
-__global__ void bwd_v_rows_kernel(const float* __restrict__ dvp, const __nv_bfloat16* __restrict__ ve,
-                                  const float2* __restrict__ gate, __nv_bfloat16* __restrict__ dv,
-                                  __nv_bfloat16* __restrict__ dve, float* __restrict__ dz, int n_rows) {
-    constexpr int E = D / 32;
-    const int lane = threadIdx.x & 31;
-    const int warps = gridDim.x * (blockDim.x >> 5);
-    for (int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < n_rows; row += warps) {
-        const long long base = (long long)row * D + lane * E;
-        float g = 0.f;
-        if constexpr (HAS_VE) {
-            const float2 gg = gate[row];
-            g = gg.x + gg.y;
-        }
-        float acc = 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const float d = dvp[base + e];
-            dv[base + e] = __float2bfloat16_rn(d);
-            if constexpr (HAS_VE) {
-                dve[base + e] = __float2bfloat16_rn(g * d);
-                acc += d * __bfloat162float(ve[base + e]);
-            }
-        }
-        if constexpr (HAS_VE) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (lane == 0) dz[row] = acc * g * (1.f - 0.5f * g);
-        }
-    }
-}
+// ------------------------------------------------------------- the gate in reverse
 
 // dgate_x[bt, c] = sum_hk dz[bt, hk] Wg[c, hk]: one thread per (bt, c).
 __global__ void bwd_gate_x_kernel(const float* __restrict__ dz, const __nv_bfloat16* __restrict__ Wg,

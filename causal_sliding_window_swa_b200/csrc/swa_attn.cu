@@ -528,7 +528,7 @@ int launch_qkv(int dev, const void* x, const void* Wqkv, const void* ve, const v
 // layers only).  The backward kernels' scheduler counters are ints 4..7 of the counter section.
 struct BwdLayout {
     WsLayout f;
-    size_t rowstat, dqh, dkh, dvp, dz, wgp, dstart, dend, total;
+    size_t rowstat, dz, wgp, dstart, dend, total;
     int Tp, wg_blocks, wg_rows;
 };
 
@@ -537,18 +537,11 @@ BwdLayout bwd_layout(const Shape& s, bool has_ve) {
     w.f = ws_layout(s, has_ve);
     w.Tp = ((s.T + 127) / 128) * 128;
     const long long n_bt = (long long)s.B * s.T;
-    const size_t kv_f32 = round_up((size_t)n_bt * s.Hkv * s.D * 4);
     w.wg_rows = 32;
     w.wg_blocks = has_ve ? (int)((n_bt + w.wg_rows - 1) / w.wg_rows) : 0;
     size_t o = w.f.total;
     w.rowstat = o;
     o += round_up((size_t)s.B * s.H * w.Tp * sizeof(float2));
-    w.dqh = o;
-    o += round_up((size_t)s.n * 4);
-    w.dkh = o;
-    o += kv_f32;
-    w.dvp = o;
-    o += kv_f32;
     w.dz = o;
     o += has_ve ? round_up((size_t)n_bt * s.Hkv * 4) : 0;
     w.wgp = o;
@@ -604,9 +597,17 @@ int launch_backward(int dev, const void* q, const void* k, const void* v, const 
     p.c1 = (float)(1.4426950408889634 / std::sqrt((double)s.D));
     p.inv_sqrt_d = (float)(1.0 / std::sqrt((double)s.D));
     p.rowstat = rowstat;
-    p.dqh = reinterpret_cast<float*>(ws + L.dqh);
-    p.dkh = reinterpret_cast<float*>(ws + L.dkh);
-    p.dvp = reinterpret_cast<float*>(ws + L.dvp);
+    p.xq = static_cast<const bf*>(q);
+    p.xk = static_cast<const bf*>(k);
+    p.ve = static_cast<const bf*>(ve);
+    p.gate = has_ve ? reinterpret_cast<const float2*>(ws + L.f.gate) : nullptr;
+    p.rope_base = (double)rope_base;
+    p.eps = eps;
+    p.dq = static_cast<bf*>(dq);
+    p.dk = static_cast<bf*>(dk);
+    p.dv = static_cast<bf*>(dv);
+    p.dve = static_cast<bf*>(dve);
+    p.dz = has_ve ? reinterpret_cast<float*>(ws + L.dz) : nullptr;
     p.wait_limit_ns = wait_limit_ns();
     if (doc) {
         p.dstart = reinterpret_cast<int*>(ws + L.dstart);
@@ -641,29 +642,8 @@ int launch_backward(int dev, const void* q, const void* k, const void* v, const 
     }
 #undef SWA_BWD_TC
 
-    // The prologue in reverse.
-    const double2* t64 = reinterpret_cast<const double2*>(ws + L.f.tab64);
-    const int n_q = s.B * s.T * s.H, n_kv = s.B * s.T * s.Hkv;
-    const int bq = std::min((n_q + 7) / 8, 148 * 16), bkv = std::min((n_kv + 7) / 8, 148 * 16);
-    const float2* gate = reinterpret_cast<const float2*>(ws + L.f.gate);
+    // The rest of the prologue in reverse: the gate's inputs from dz (the epilogues did the rows).
     float* dz = reinterpret_cast<float*>(ws + L.dz);
-#define SWA_BWD_ROWS(DD)                                                                                          \
-    swa::bwd_qk_rows_kernel<DD><<<bq, 256, 0, st>>>(static_cast<const bf*>(q), p.dqh, static_cast<bf*>(dq), t64,  \
-                                                   n_q, s.T, s.H, eps);                                            \
-    swa::bwd_qk_rows_kernel<DD><<<bkv, 256, 0, st>>>(static_cast<const bf*>(k), p.dkh, static_cast<bf*>(dk), t64, \
-                                                    n_kv, s.T, s.Hkv, eps);                                        \
-    if (has_ve)                                                                                                   \
-        swa::bwd_v_rows_kernel<DD, true><<<bkv, 256, 0, st>>>(p.dvp, static_cast<const bf*>(ve), gate,            \
-                                                             static_cast<bf*>(dv), static_cast<bf*>(dve), dz, n_kv); \
-    else                                                                                                          \
-        swa::bwd_v_rows_kernel<DD, false><<<bkv, 256, 0, st>>>(p.dvp, nullptr, nullptr, static_cast<bf*>(dv),     \
-                                                              nullptr, nullptr, n_kv)
-    if (s.D == 128) {
-        SWA_BWD_ROWS(128);
-    } else {
-        SWA_BWD_ROWS(64);
-    }
-#undef SWA_BWD_ROWS
     if (has_ve) {
         const long long n_bt = (long long)s.B * s.T;
         const int bgx = (int)std::min<long long>((n_bt * 32 + 255) / 256, 148ll * 16);

@@ -155,7 +155,7 @@ def test_decode_workspace_and_validation():
 
 
 def test_backward_workspace_and_validation():
-    # forward sections + row statistics (B*H*Tp float2) + dqhat (fp32) + dkhat, dv' (fp32, Hkv heads)
+    # forward sections + row statistics (B*H*Tp float2)
     # [+ dz and the dWg partial sums on value-embedding layers] + document starts and ends (B*T int32
     # each), each section 1024-byte aligned.  The forward's prologue repair lists (an int count and
     # 256 32-byte items per block of each prologue pass; 256-thread blocks, D/8 threads per row, at
@@ -171,8 +171,7 @@ def test_backward_workspace_and_validation():
     fix_mha, fix_gqa = fix(blocks(B * T * H)), fix(blocks(B * T * H) + blocks(B * T * Hkv))
     assert n0 == (fwd - 2 * up(B * T * H * D * 2) + 2 * kv_fwd + up(B * T * H * D * 2) - kv_fwd
                   - fix_mha + fix_gqa
-                  + up(B * H * Tp * 8) + up(B * T * H * D * 4) + 2 * up(B * T * Hkv * D * 4)
-                  + 2 * up(B * T * 4))
+                  + up(B * H * Tp * 8) + 2 * up(B * T * 4))
     n1 = swa.swa_attn_bwd_workspace_bytes(B, T, H, Hkv, D, 1)
     assert n1 > n0 + up(B * T * Hkv * 4)
     assert swa.swa_attn_bwd_workspace_bytes(B, T, H, 3, D, 0) == 0     # 3 does not divide 4
