@@ -280,6 +280,9 @@ __global__ void __launch_bounds__(576, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const unsigned long long lim = p.wait_limit_ns;
+    // Launched as a programmatic dependent of the prologue: the setup above overlapped its tail;
+    // nothing it wrote (qhat, khat, v', the item counter) is touched before this wait.
+    grid_dependency_wait();
 
     if (warp == kProducerWarp) {
         // ========================= scheduler + TMA producer =========================

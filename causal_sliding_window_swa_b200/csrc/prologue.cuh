@@ -48,21 +48,39 @@ __device__ __forceinline__ int fdiv(int n, const FastDiv& f) {
 }
 
 // Gate of every (b, t, h) row: g = 2 sigmoid(sum_{c<32} x[b,t,c] Wg[c,h]) in fp64, stored as
-// (g_hi, g_lo) = (fp32(g), fp32(g - g_hi)).  Token bt's 32 gate channels start at
-// gate_x + bt * x_stride (32 for the contiguous slice, C for the full layer input).
+// (g_hi, g_lo) = (fp32(g), fp32(g - g_hi)) at gate[bt * H + h].  One thread per token bt: its 32
+// gate channels (at gate_x + bt * x_stride: 32 for the contiguous slice, C for the full layer
+// input) are loaded once, and the heads are taken four at a time, each sum over c in order.  Wg
+// (32 x H) is staged in shared memory as fp64 (32 H doubles of dynamic shared memory) when
+// wg_smem is set, else read from global memory.
 __global__ void gate_kernel(const __nv_bfloat16* __restrict__ gate_x, const __nv_bfloat16* __restrict__ Wg,
-                            float2* __restrict__ gate, int n_rows, int H, FastDiv divH, int x_stride) {
-    for (int row = blockIdx.x * blockDim.x + threadIdx.x; row < n_rows; row += gridDim.x * blockDim.x) {
-        const int bt = fdiv(row, divH);
-        const int h = row - bt * H;
+                            float2* __restrict__ gate, int n_tokens, int H, int x_stride, int wg_smem) {
+    extern __shared__ double s_wg[];   // [32][H]
+    grid_dependents_launch();          // the prologue kernel may launch (it waits for this one)
+    if (wg_smem)
+        for (int i = threadIdx.x; i < 32 * H; i += blockDim.x) s_wg[i] = (double)__bfloat162float(Wg[i]);
+    __syncthreads();
+    auto wg = [&](int i) -> double { return wg_smem ? s_wg[i] : (double)__bfloat162float(Wg[i]); };
+    for (int bt = blockIdx.x * blockDim.x + threadIdx.x; bt < n_tokens; bt += gridDim.x * blockDim.x) {
         const __nv_bfloat16* xr = gate_x + (long long)bt * x_stride;
-        double z = 0.0;
-#pragma unroll 8
-        for (int c = 0; c < 32; ++c)
-            z = fma((double)__bfloat162float(xr[c]), (double)__bfloat162float(Wg[c * H + h]), z);
-        const double g = 2.0 / (1.0 + exp(-z));
-        const float g_hi = (float)g;
-        gate[row] = make_float2(g_hi, (float)(g - (double)g_hi));
+        double x[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) x[c] = (double)__bfloat162float(xr[c]);
+        for (int h0 = 0; h0 < H; h0 += 4) {
+            double z[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (h0 + u < H) z[u] = fma(x[c], wg(c * H + h0 + u), z[u]);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (h0 + u >= H) break;
+                const double g = 2.0 / (1.0 + exp(-z[u]));
+                const float g_hi = (float)g;
+                gate[(long long)bt * H + h0 + u] = make_float2(g_hi, (float)(g - (double)g_hi));
+            }
+        }
     }
 }
 
@@ -369,6 +387,9 @@ __device__ void prologue_fix_chunk(long long chunk, uint32_t flags, const FixPar
 template <int D>
 __global__ void __launch_bounds__(256) prologue_fix_kernel(const int* __restrict__ counts, const FixItem* __restrict__ items,
                                                            int n_lists, const __grid_constant__ FixParams p) {
+    // a programmatic dependent of the prologue kernel: wait for it, then let the attention launch
+    grid_dependency_wait();
+    grid_dependents_launch();
     const int lane = (int)(threadIdx.x & 31u);
     const int n_warps = (int)((gridDim.x * blockDim.x) >> 5);
     for (int list = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); list < n_lists; list += n_warps) {
@@ -413,6 +434,10 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(
     // Every thread of a warp runs the same number of iterations, so the shuffles always see the
     // full warp; rows past the end are computed on zeros and not stored.
     const long long n_iter = ((long long)n_rows * TPR + stride - 1) / stride;
+    // Launched as a programmatic dependent of the gate kernel: wait for it before any memory
+    // access, then let the repair kernel launch.
+    grid_dependency_wait();
+    grid_dependents_launch();
     // The attention kernel that follows takes its work items from this counter.
     if (gtid == 0) {
         sched[0] = 0;

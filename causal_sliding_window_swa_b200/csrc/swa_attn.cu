@@ -281,6 +281,24 @@ swa::FastDiv make_fastdiv(int d) {
     return f;
 }
 
+// A launch that may start while the kernel before it on the stream still runs (programmatic
+// dependent launch): the kernel waits (griddepcontrol.wait) before it touches memory that kernel
+// wrote, so only the launch latency and its own setup overlap.
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 int launch_rope_table(uint8_t* ws, const WsLayout& L, const Shape& s, float rope_base, cudaStream_t st) {
     const long long n = (long long)s.T * (s.D / 2);
     const int threads = 256;
@@ -303,9 +321,9 @@ int launch_prologue_fix(const int* counts, const swa::FixItem* items, long long 
     fp.n_iter = (int)((fp.n_chunks + fp.stride - 1) / fp.stride);
     const unsigned g = (unsigned)((blocks + 7) / 8);     // a warp per list
     if (fp.D == 128)
-        swa::prologue_fix_kernel<128><<<g, 256, 0, st>>>(counts, items, (int)blocks, fp);
+        launch_pdl(swa::prologue_fix_kernel<128>, dim3(g), dim3(256), 0, st, counts, items, (int)blocks, fp);
     else
-        swa::prologue_fix_kernel<64><<<g, 256, 0, st>>>(counts, items, (int)blocks, fp);
+        launch_pdl(swa::prologue_fix_kernel<64>, dim3(g), dim3(256), 0, st, counts, items, (int)blocks, fp);
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
@@ -319,9 +337,11 @@ int launch_prologue(const void* q, const void* k, const void* v, const void* ve,
     const swa::FastDiv divH = make_fastdiv(s.H), divT = make_fastdiv(s.T);
     float2* gate = reinterpret_cast<float2*>(ws + L.gate);
     if (has_ve) {
-        const int gblocks = (int)std::min<long long>(((long long)n_kv_rows + 255) / 256, 148ll * 8);
-        swa::gate_kernel<<<gblocks, 256, 0, st>>>(static_cast<const bf*>(gate_x), static_cast<const bf*>(Wg),
-                                                   gate, n_kv_rows, s.Hkv, make_fastdiv(s.Hkv), 32);
+        const int n_tok = s.B * s.T;
+        const int gblocks = (int)std::min<long long>(((long long)n_tok + 127) / 128, 148ll * 16);
+        const int wg_smem = 32 * s.Hkv * (int)sizeof(double) <= 48 * 1024;
+        swa::gate_kernel<<<gblocks, 128, wg_smem ? 32 * s.Hkv * sizeof(double) : 0, st>>>(
+            static_cast<const bf*>(gate_x), static_cast<const bf*>(Wg), gate, n_tok, s.Hkv, 32, wg_smem);
     }
     const long long threads_total = (long long)n_rows * (s.D / 8);
     const int threads = 256;
@@ -374,14 +394,14 @@ int launch_prologue(const void* q, const void* k, const void* v, const void* ve,
     }
     if (s.D == 128) {
         if (has_ve)
-            swa::prologue_kernel<128, true><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, sched, n_rows, s.T, s.H, divT, divH, e, fixc, fixi);
+            launch_pdl(swa::prologue_kernel<128, true, 3>, dim3(g), dim3(threads), 0, st, qp, kp, vpi, vep, (const float2*)gate, qh, kh, vp, t32, sched, n_rows, s.T, s.H, divT, divH, e, fixc, fixi);
         else
-            swa::prologue_kernel<128, false><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, sched, n_rows, s.T, s.H, divT, divH, e, fixc, fixi);
+            launch_pdl(swa::prologue_kernel<128, false, 3>, dim3(g), dim3(threads), 0, st, qp, kp, vpi, vep, (const float2*)gate, qh, kh, vp, t32, sched, n_rows, s.T, s.H, divT, divH, e, fixc, fixi);
     } else {
         if (has_ve)
-            swa::prologue_kernel<64, true><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, sched, n_rows, s.T, s.H, divT, divH, e, fixc, fixi);
+            launch_pdl(swa::prologue_kernel<64, true, 3>, dim3(g), dim3(threads), 0, st, qp, kp, vpi, vep, (const float2*)gate, qh, kh, vp, t32, sched, n_rows, s.T, s.H, divT, divH, e, fixc, fixi);
         else
-            swa::prologue_kernel<64, false><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, sched, n_rows, s.T, s.H, divT, divH, e, fixc, fixi);
+            launch_pdl(swa::prologue_kernel<64, false, 3>, dim3(g), dim3(threads), 0, st, qp, kp, vpi, vep, (const float2*)gate, qh, kh, vp, t32, sched, n_rows, s.T, s.H, divT, divH, e, fixc, fixi);
     }
     return launch_prologue_fix(fixc, fixi, g, n_rows, s.H, 0x00ffu | ve_flags, fp, st);
 }
@@ -420,7 +440,8 @@ int launch_attention(int dev, const void* v, bool has_ve, void* out, float* lse,
     p.dstart = dstart;
     const dim3 grid((unsigned)std::min(p.n_items, g_num_sms[dev]));
 #define SWA_ATTN(DD, DC) \
-    swa::attn_fwd_kernel<DD, DC><<<grid, swa::FwdCfg<DD>::THREADS, swa::FwdCfg<DD>::SMEM_TOTAL, st>>>(tq, tk, tv, to, p)
+    launch_pdl(swa::attn_fwd_kernel<DD, DC>, grid, dim3(swa::FwdCfg<DD>::THREADS), swa::FwdCfg<DD>::SMEM_TOTAL, st, tq, tk, \
+               tv, to, p)
     if (s.D == 128) {
         if (dstart) SWA_ATTN(128, true); else SWA_ATTN(128, false);
     } else {
@@ -479,10 +500,10 @@ int launch_qkv(int dev, const void* x, const void* Wqkv, const void* ve, const v
     }
     float2* gate = reinterpret_cast<float2*>(ws + L.gate);
     if (has_ve) {
-        const int n_kv_rows = (int)(M * s.Hkv);
-        const int gblocks = (int)std::min<long long>(((long long)n_kv_rows + 255) / 256, 148ll * 8);
-        swa::gate_kernel<<<gblocks, 256, 0, st>>>(static_cast<const bf*>(x), static_cast<const bf*>(Wg), gate,
-                                                   n_kv_rows, s.Hkv, make_fastdiv(s.Hkv), C);
+        const int gblocks = (int)std::min<long long>((M + 127) / 128, 148ll * 16);
+        const int wg_smem = 32 * s.Hkv * (int)sizeof(double) <= 48 * 1024;
+        swa::gate_kernel<<<gblocks, 128, wg_smem ? 32 * s.Hkv * sizeof(double) : 0, st>>>(
+            static_cast<const bf*>(x), static_cast<const bf*>(Wg), gate, (int)M, s.Hkv, C, wg_smem);
     }
     const int N = (s.H + 2 * s.Hkv) * s.D;
     const int BN = ((s.H * s.D) % 256 == 0 && (s.Hkv * s.D) % 256 == 0) ? 256 : 128;
