@@ -38,7 +38,8 @@
 // applies sum to one (a row with one visible key returns that key's v' unchanged); the LSE uses
 // the unrounded sum.  P is rounded to bf16 toward zero (one byte-permute per pair); because the
 // normaliser is the sum of the same rounded values, the rounding bias cancels in the weights.
-// One exponential in four is evaluated by a polynomial on the FMA pipe to offload the MUFU unit.
+// Every exponential runs on MUFU (a polynomial on the FMA pipe is kept behind a zero mask: sending
+// part of the pairs to it measured slower, the loop being bound by the issue of its products).
 #pragma once
 
 #include <cuda.h>
@@ -62,15 +63,21 @@ struct FwdCfg {
     static constexpr int SMEM_KV = NS * TILE_BYTES;
     static constexpr int SMEM_OUT = TILE_BYTES;        // output tile staged for the TMA store
     static constexpr int SMEM_BAR = 512;
-    static constexpr int SMEM_LX = 4 * 128 * 8;        // row-sum exchange between the four threads of a row
+    // Softmax threads per tile row (NQ) and the key columns each takes (CW).  Four is the most
+    // that fits: 128 NQ softmax threads plus the MMA and producer warps must stay within 1024.
+    static constexpr int NQ = 4;
+    static constexpr int CW = 128 / NQ;
+    static constexpr int SMEM_LX = NQ * 128 * 8;       // row-sum exchange between the NQ threads of a row
     // Dynamic shared memory is declared 1024-byte aligned (the 128-byte swizzle atom repeats every
     // 1024 bytes); the kernel checks the alignment on entry instead of reserving slack for it.
     static constexpr int SMEM_TOTAL = SMEM_Q + SMEM_KV + SMEM_OUT + SMEM_BAR + SMEM_LX;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_O = NSB * 128;
     static constexpr uint32_t COL_Q = COL_O + D;       // Q as bf16 pairs: D / 2 columns
-    static constexpr int THREADS = 576;
-    static constexpr int SOFTMAX_THREADS = 512;
+    static constexpr int SOFTMAX_THREADS = 128 * NQ;
+    static constexpr int SOFTMAX_WARPS = SOFTMAX_THREADS / 32;
+    static constexpr int THREADS = 64 + SOFTMAX_THREADS;
+    static_assert(CW == 16 || CW == 32, "softmax column split");
 };
 
 struct FwdParams {
@@ -197,7 +204,7 @@ __device__ __forceinline__ uint32_t softmax_pair_poly(uint32_t s0, uint32_t s1, 
 }
 
 template <int D, bool DOC = false>
-__global__ void __launch_bounds__(576, 1)
+__global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                     const FwdParams p) {
@@ -239,7 +246,7 @@ __global__ void __launch_bounds__(576, 1)
     constexpr int kMmaWarp = 0;
     constexpr int kProducerWarp = 1;
     constexpr int kSoftmaxWarp0 = 2;
-    constexpr uint32_t kItemConsumers = 1 + 16;  // the MMA thread and lane 0 of each softmax warp
+    constexpr uint32_t kItemConsumers = 1 + C::SOFTMAX_WARPS;  // the MMA thread and lane 0 of each softmax warp
 
     if (threadIdx.x == 32) {
         mbar_init(smem_u32(b_qfull), 1);
@@ -247,7 +254,7 @@ __global__ void __launch_bounds__(576, 1)
         mbar_init(smem_u32(b_ofull), 1);
         mbar_init(smem_u32(b_oempty), C::SOFTMAX_THREADS);
         mbar_init(smem_u32(b_mdrain), 1);
-        mbar_init(smem_u32(b_lxa), 3 * 128);
+        mbar_init(smem_u32(b_lxa), (C::NQ - 1) * 128);
         mbar_init(smem_u32(b_lxb), 128);
         mbar_init(smem_u32(b_ostaged), C::SOFTMAX_THREADS);
         mbar_init(smem_u32(b_ofree), 1);
@@ -400,8 +407,8 @@ __global__ void __launch_bounds__(576, 1)
                 const uint64_t db = dv + (uint64_t)((sv * C::TILE_BYTES) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk)
-                    mma_ts(d_o, pa + (kk >> 1) * 32 + (kk & 1) * 8, db + (uint64_t)((kk * 16 * 128) >> 4),
-                           idesc_pv, (j > m.lo || kk > 0) ? 1u : 0u);
+                    mma_ts(d_o, pa + (uint32_t)(C::CW * (16 * kk / C::CW) + (16 * kk % C::CW) / 2),
+                           db + (uint64_t)((kk * 16 * 128) >> 4), idesc_pv, (j > m.lo || kk > 0) ? 1u : 0u);
                 mma_commit(smem_u32(b_kvempty + sv));
                 if (j == m.hi) mma_commit(smem_u32(b_ofull));
                 ++p_cnt;
@@ -493,13 +500,14 @@ __global__ void __launch_bounds__(576, 1)
                 ++s_cnt;
                 if (++s_buf == (uint32_t)C::NSB) s_buf = 0;
                 tc_fence_after();
-                const int k0 = j * C::BN + 32 * cq;    // first key of this thread's 32 columns
-                const bool need_mask = (k0 + 31 > m.q0) || (m.q0 + C::BM - 1 - k0 >= p.W) || (DOC && k0 < ds_w);
-                const uint32_t colS = buf * 128u + 32u * (uint32_t)cq;
+                const int k0 = j * C::BN + C::CW * cq;   // first key of this thread's CW columns
+                const bool need_mask =
+                    (k0 + C::CW - 1 > m.q0) || (m.q0 + C::BM - 1 - k0 >= p.W) || (DOC && k0 < ds_w);
+                const uint32_t colS = buf * 128u + (uint32_t)(C::CW * cq);
                 // The 32 scores in two 16-column blocks, both loaded before any arithmetic; P of
                 // the 32 keys packs into 16 words written over the first 16 of these columns.
-                uint32_t sq[2][16];
-                uint32_t pk[16];
+                uint32_t sq[C::CW / 16][16];
+                uint32_t pk[C::CW / 2];
                 auto block = [&](const uint32_t (&sv)[16], int cbase, int pkbase) {
                     if (!need_mask) {
 #pragma unroll
@@ -525,11 +533,15 @@ __global__ void __launch_bounds__(576, 1)
                     }
                 };
                 tmem_ld16(tmem + lane_base + colS + 0, sq[0]);
-                tmem_ld16(tmem + lane_base + colS + 16, sq[1]);
+                if constexpr (C::CW == 32) tmem_ld16(tmem + lane_base + colS + 16, sq[C::CW / 16 - 1]);
                 tmem_ld_wait();
                 block(sq[0], 0, 0);
-                block(sq[1], 16, 8);
-                tmem_st16(tmem + lane_base + colS + 0, pk);
+                if constexpr (C::CW == 32) {
+                    block(sq[C::CW / 16 - 1], 16, 8);
+                    tmem_st16(tmem + lane_base + colS + 0, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+                } else {
+                    tmem_st8(tmem + lane_base + colS + 0, *reinterpret_cast<const uint32_t(*)[8]>(pk));
+                }
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(smem_u32(b_pfull + buf));
@@ -556,14 +568,16 @@ __global__ void __launch_bounds__(576, 1)
             if (!ok) break;
             tc_fence_after();
             // Read this thread's quarter of the O row, then release O to the next item.
-            constexpr int OQ = D / 4;             // output columns per thread: 32 or 16
+            constexpr int OQ = D / C::NQ;         // output columns per thread: 8 to 32
             uint32_t ov[OQ];
             if constexpr (OQ == 32) {
                 tmem_ld16(tmem + lane_base + C::COL_O + (uint32_t)(OQ * cq), *reinterpret_cast<uint32_t(*)[16]>(ov));
                 tmem_ld16(tmem + lane_base + C::COL_O + (uint32_t)(OQ * cq) + 16u,
                           *reinterpret_cast<uint32_t(*)[16]>(ov + 16));
-            } else {
+            } else if constexpr (OQ == 16) {
                 tmem_ld16(tmem + lane_base + C::COL_O + (uint32_t)(OQ * cq), *reinterpret_cast<uint32_t(*)[16]>(ov));
+            } else {
+                tmem_ld8(tmem + lane_base + C::COL_O + (uint32_t)(OQ * cq), *reinterpret_cast<uint32_t(*)[8]>(ov));
             }
             tmem_ld_wait();
             tc_fence_before();
@@ -582,7 +596,7 @@ __global__ void __launch_bounds__(576, 1)
             } else {
                 ok = mbar_wait(smem_u32(b_lxa), xpar, lim, kSiteRowSum);
 #pragma unroll
-                for (int c = 1; c < 4; ++c) {
+                for (int c = 1; c < C::NQ; ++c) {
                     const float2 t = s_lx[c * 128 + r];
                     l += t.x;
                     lr += t.y;
