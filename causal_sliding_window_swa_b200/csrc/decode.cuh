@@ -179,8 +179,8 @@ struct Raw<2> {
 // ------------------------------------------------------------------- attention of the new token
 //
 // One CTA per (row b*H + h, chunk of the window), the chunks of a row forming one thread-block
-// cluster, launched so that it may start while the prologue kernel runs (it waits for that kernel
-// before reading qhat and before loading the tile with the new token).  A producer warp streams the chunk's K and V' tiles (KB keys x D, 8 KB each) from the
+// cluster, launched so that it may start while the token prologue runs: it forms qhat itself and
+// waits for that kernel only before it loads the tile with the new token.  A producer warp streams the chunk's K and V' tiles (KB keys x D, 8 KB each) from the
 // caches into a four-stage shared-memory ring with TMA; four consumer warps take KB / 4 keys of
 // each tile.  Lane l holds features [l DPL, (l + 1) DPL) of qhat; a warp's NK partial dot
 // products are summed over the lanes by a butterfly that halves the set of keys at each of the
@@ -231,7 +231,9 @@ __device__ __forceinline__ float warp_sum_keys(float (&v)[NK], int lane) {
 }
 
 struct DecParams {
-    const __nv_bfloat16* qh;     // (B*H, D) qhat of the new tokens
+    const __nv_bfloat16* q;      // (B*H, D) raw q of the new tokens (qhat is formed here)
+    double rope_base, eps;
+    int pos;                     // position of the new tokens
     __nv_bfloat16* out;          // (B*H, D)
     float* lse;                  // (B*H) or null
     const int* doc_start;        // (B) or null
@@ -258,6 +260,9 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS) decode_attn_kernel(const _
     float* s_l = reinterpret_cast<float*>(smem + C::OFF_L);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* empty = full + C::NS;
+    __shared__ float4 s_tab32[D / 2];
+    __shared__ double2 s_tab64[D / 2];
+    __shared__ __align__(16) __nv_bfloat16 s_qh[D];
 
     const int warp = (int)(threadIdx.x >> 5), lane = (int)(threadIdx.x & 31u);
     const uint32_t rank = cluster_ctarank(), n_ranks = cluster_nctarank();
@@ -303,13 +308,41 @@ __global__ void __launch_bounds__(DecCfg<D>::THREADS) decode_attn_kernel(const _
             }
         }
     } else {
-        float q[DPL];
-        grid_dependency_wait();                                    // qhat comes from the prologue kernel
-        {
-            const __nv_bfloat16* qr = p.qh + (long long)row * D + lane * DPL;
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) q[e] = __bfloat162float(qr[e]);
+        // qhat of this row, formed here while the first tiles load: the RoPE row of `pos` (one
+        // entry per thread of the first D/2), then the prologue's exact-rounding rotation and
+        // RMS on warp 0 (D/8 lanes per row; the other lanes compute copies), as the prefill and
+        // token prologues do, so qhat is bit-identical to theirs.
+        if ((int)threadIdx.x < D / 2) {
+            const int i = (int)threadIdx.x;
+            const double theta = pow(p.rope_base, -2.0 * (double)i / (double)D);
+            double sn, cs;
+            sincos((double)p.pos * theta, &sn, &cs);
+            float c_hi, c_lo, s_hi, s_lo;
+            rope_split(cs, c_hi, c_lo);
+            rope_split(sn, s_hi, s_lo);
+            s_tab32[i] = make_float4(c_hi, c_lo, s_hi, s_lo);
+            s_tab64[i] = make_double2(cs, sn);
         }
+        asm volatile("bar.sync 1, %0;" ::"r"(32 * C::CONSUMERS) : "memory");
+        if (warp == 0) {
+            constexpr int TPR = D / 8;
+            const int c = lane % TPR, i0 = 4 * c;
+            const __nv_bfloat16* qr = p.q + (long long)row * D;
+            const uint2 lo_raw = ldg_stream8(qr + i0), hi_raw = ldg_stream8(qr + D / 2 + i0);
+            float4 cs4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) cs4[e] = s_tab32[i0 + e];
+            uint2 o_lo, o_hi;
+            rope_rms_exact4<D>(lo_raw, hi_raw, cs4, s_tab64 + i0, p.eps, o_lo, o_hi);
+            if (lane < TPR) {
+                *reinterpret_cast<uint2*>(s_qh + i0) = o_lo;
+                *reinterpret_cast<uint2*>(s_qh + D / 2 + i0) = o_hi;
+            }
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(32 * C::CONSUMERS) : "memory");
+        float q[DPL];
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) q[e] = __bfloat162float(s_qh[lane * DPL + e]);
         float o[DPL];
 #pragma unroll
         for (int e = 0; e < DPL; ++e) o[e] = 0.f;

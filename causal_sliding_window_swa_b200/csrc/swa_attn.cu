@@ -895,9 +895,9 @@ bool make_cache_map(CUtensorMap* m, const void* base, int B, int Tmax, int Hkv, 
 // resident CTA slots per row, so that one wave streams the whole window; each CTA takes whole
 // KB-key tiles.
 template <int D>
-int launch_decode_attention_d(int dev, const void* qh, const void* k_cache, const void* v_cache, const int* doc_start,
-                              void* out, float* lse, int B, int Tmax, int H, int Hkv, int lo, int n_keys,
-                              cudaStream_t st) {
+int launch_decode_attention_d(int dev, const void* q, const void* k_cache, const void* v_cache, const int* doc_start,
+                              void* out, float* lse, int B, int Tmax, int H, int Hkv, int lo, int n_keys, int pos,
+                              double rope_base, double eps, cudaStream_t st) {
     using C = swa::DecCfg<D>;
     CUtensorMap tk, tv;
     if (!make_cache_map(&tk, k_cache, B, Tmax, Hkv, D, C::KB) || !make_cache_map(&tv, v_cache, B, Tmax, Hkv, D, C::KB))
@@ -920,7 +920,10 @@ int launch_decode_attention_d(int dev, const void* qh, const void* k_cache, cons
     const int tiles_per_chunk = (n_tiles + n_chunks - 1) / n_chunks;
     n_chunks = (n_tiles + tiles_per_chunk - 1) / tiles_per_chunk;
     swa::DecParams p{};
-    p.qh = static_cast<const __nv_bfloat16*>(qh);
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.rope_base = rope_base;
+    p.eps = eps;
+    p.pos = pos;
     p.out = static_cast<__nv_bfloat16*>(out);
     p.lse = lse;
     p.doc_start = doc_start;
@@ -955,13 +958,13 @@ int launch_decode_attention_d(int dev, const void* qh, const void* k_cache, cons
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
-int launch_decode_attention(int dev, const void* qh, const void* k_cache, const void* v_cache, const int* doc_start,
-                            void* out, float* lse, int B, int Tmax, int H, int Hkv, int D, int lo, int n_keys,
-                            cudaStream_t st) {
-    return D == 128 ? launch_decode_attention_d<128>(dev, qh, k_cache, v_cache, doc_start, out, lse, B, Tmax, H, Hkv,
-                                                     lo, n_keys, st)
-                    : launch_decode_attention_d<64>(dev, qh, k_cache, v_cache, doc_start, out, lse, B, Tmax, H, Hkv,
-                                                    lo, n_keys, st);
+int launch_decode_attention(int dev, const void* q, const void* k_cache, const void* v_cache, const int* doc_start,
+                            void* out, float* lse, int B, int Tmax, int H, int Hkv, int D, int lo, int n_keys, int pos,
+                            double rope_base, double eps, cudaStream_t st) {
+    return D == 128 ? launch_decode_attention_d<128>(dev, q, k_cache, v_cache, doc_start, out, lse, B, Tmax, H, Hkv,
+                                                     lo, n_keys, pos, rope_base, eps, st)
+                    : launch_decode_attention_d<64>(dev, q, k_cache, v_cache, doc_start, out, lse, B, Tmax, H, Hkv,
+                                                    lo, n_keys, pos, rope_base, eps, st);
 }
 
 extern "C" {
@@ -1138,12 +1141,10 @@ int swa_attn_decode_doc(const void* q, const void* k, const void* v, const void*
     if ((rc = device_ready(&dev)) != SWA_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     using bf = __nv_bfloat16;
-    const int rows = B * H;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    bf* qh = reinterpret_cast<bf*>(ws);
+    bf* qh = reinterpret_cast<bf*>(ws);   // unused by the key/value pass (qhat is formed by the attention kernel)
     {
         const int rows_per_block = 256 / (D / 8);
-        const int blocks = std::max(1, std::min((rows + rows_per_block - 1) / rows_per_block, 148 * 8));
         const bf* qp = static_cast<const bf*>(q);
         const bf* kp = static_cast<const bf*>(k);
         const bf* vp = static_cast<const bf*>(v);
@@ -1153,21 +1154,12 @@ int swa_attn_decode_doc(const void* q, const void* k, const void* v, const void*
         bf* kc = static_cast<bf*>(k_cache);
         bf* vc = static_cast<bf*>(v_cache);
         const double base = (double)rope_base, e = (double)eps;
-        // grouped-query layers: the query rows and the key/value rows (Hkv heads) as two passes
         const int kv_rows = B * Hkv;
         const int kv_blocks = std::max(1, std::min((kv_rows + rows_per_block - 1) / rows_per_block, 148 * 8));
+    // The token prologue writes khat and v' to the caches; the attention kernel forms qhat itself.
 #define SWA_DEC_PRO(DD, VE)                                                                               \
-    do {                                                                                                  \
-    if (Hkv == H) {                                                                                       \
-        swa::decode_prologue_kernel<DD, VE><<<blocks, 256, 0, st>>>(qp, kp, vp, vep, gx, wg, qh, kc, vc, rows, \
-                                                                    H, Tmax, pos, base, e);               \
-    } else {                                                                                              \
-        swa::decode_prologue_kernel<DD, VE, 1><<<blocks, 256, 0, st>>>(qp, kp, vp, vep, gx, wg, qh, kc, vc,   \
-                                                                       rows, H, Tmax, pos, base, e);      \
-        swa::decode_prologue_kernel<DD, VE, 2><<<kv_blocks, 256, 0, st>>>(qp, kp, vp, vep, gx, wg, qh, kc, vc, \
-                                                                          kv_rows, Hkv, Tmax, pos, base, e); \
-    }                                                                                                     \
-    } while (0)
+    swa::decode_prologue_kernel<DD, VE, 2><<<kv_blocks, 256, 0, st>>>(qp, kp, vp, vep, gx, wg, qh, kc, vc,     \
+                                                                      kv_rows, Hkv, Tmax, pos, base, e)
         if (D == 128) {
             if (has_ve)
                 SWA_DEC_PRO(128, true);
@@ -1184,7 +1176,8 @@ int swa_attn_decode_doc(const void* q, const void* k, const void* v, const void*
     const int W = (window <= 0 || window >= Tmax) ? Tmax : window;
     const int lo = std::max(0, pos - W + 1);
     const int n_keys = pos - lo + 1;
-    return launch_decode_attention(dev, qh, k_cache, v_cache, doc_start, out, lse, B, Tmax, H, Hkv, D, lo, n_keys, st);
+    return launch_decode_attention(dev, q, k_cache, v_cache, doc_start, out, lse, B, Tmax, H, Hkv, D, lo, n_keys, pos,
+                                   (double)rope_base, (double)eps, st);
 }
 
 int swa_attn_decode_gqa(const void* q, const void* k, const void* v, const void* ve,
