@@ -252,7 +252,9 @@ SWA_API int swa_attn_last_device_status(swa_stream_t stream, unsigned int* detai
  *   workspace    device memory of at least swa_attn_decode_workspace_bytes(B, Tmax, H, D, has_ve,
  *                window) bytes, 16-byte aligned, caller-owned and not retained.
  * Scores, exponentials and weighted sums are fp32 (no bf16 rounding of the weights).  The call is
- * asynchronous on `stream` (two kernels: the prologue, then one cluster of CTAs per row for the attention); arguments are validated before anything is enqueued.  Errors: SWA_ERR_INVALID_ARG (null pointer, pos outside [0, Tmax), bad rope_base /
+ * asynchronous on `stream` (two kernels: the token's key/value prologue, then one cluster of CTAs
+ * per row for the attention, which also forms qhat); arguments are validated before anything is
+ * enqueued.  Errors: SWA_ERR_INVALID_ARG (null pointer, pos outside [0, Tmax), bad rope_base /
  * eps, partial value-embedding set), SWA_ERR_UNSUPPORTED (D not 64/128, sizes beyond int32),
  * SWA_ERR_MISALIGNED, SWA_ERR_NO_MEMORY (workspace too small), SWA_ERR_CUDA.
  */
