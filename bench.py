@@ -367,30 +367,58 @@ def run_ours(args, s0):
     pro_ms_max = reduce_max(pro_ms, dev)
 
     # ---------------- end to end through the public call, host buffers, copies inside
+    # Every step copies all of its inputs in from pinned host memory, runs swa.forward and reads
+    # out and lse back.  Two sets of device buffers: step i's copy-in (its own stream) overlaps
+    # step i-1's layer call and read-back (a third stream), as a training or serving loop would
+    # pipeline them; the link carries both directions at once.
     E = max(1, min(args.e2e_steps, K))
-    h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    h_lse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
-    xin = {k: (None if v is None else torch.empty_like(v)) for k, v in x.items()}
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    bufs = []
+    for _ in range(2):
+        bufs.append({
+            "x": {k: (None if v is None else torch.empty_like(v)) for k, v in x.items()},
+            "out": torch.empty_like(out), "lse": torch.empty_like(lse),
+            "h_out": torch.empty(out.shape, dtype=out.dtype, pin_memory=True),
+            "h_lse": torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True),
+            "in": torch.cuda.Event(), "done": torch.cuda.Event(), "read": torch.cuda.Event(),
+            "used": False})
 
-    def e2e_step():
-        for k, v in host.items():
-            if v is not None:
-                xin[k].copy_(v, non_blocking=True)
+    def e2e_step(i):
+        b = bufs[i & 1]
+        if b["used"]:
+            s_in.wait_event(b["done"])          # the layer call two steps back has read these inputs
+        with torch.cuda.stream(s_in):
+            for k, v in host.items():
+                if v is not None:
+                    b["x"][k].copy_(v, non_blocking=True)
+        b["in"].record(s_in)
+        stream.wait_event(b["in"])
+        if b["used"]:
+            stream.wait_event(b["read"])        # its out / lse have been read back
+        xin = b["x"]
         swa.forward(xin["q"], xin["k"], xin["v"], s.window, xin["ve"], xin["gate_x"], xin["Wg"],
-                    out=out, lse=lse)
-        h_out.copy_(out, non_blocking=True)
-        h_lse.copy_(lse, non_blocking=True)
+                    out=b["out"], lse=b["lse"])
+        b["done"].record(stream)
+        s_out.wait_event(b["done"])
+        with torch.cuda.stream(s_out):
+            b["h_out"].copy_(b["out"], non_blocking=True)
+            b["h_lse"].copy_(b["lse"], non_blocking=True)
+        b["read"].record(s_out)
+        b["used"] = True
 
-    for _ in range(3):
-        e2e_step()
+    for i in range(3):
+        e2e_step(i)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(E):
-        e2e_step()
+    s_in.wait_event(e0)
+    for i in range(E):
+        e2e_step(i)
+    for b in bufs:
+        stream.wait_event(b["read"])
     e1.record(stream)
     torch.cuda.synchronize(dev)
     swa.check_device_status(stream)
