@@ -452,7 +452,7 @@ def run_ours(args, s0):
                               "frac": prologue_bytes(s) / (pro_ms_max * 1e-3) / 1e9 / float(peaks["hbm_gbs"])},
         "e2e": {"value": world * fl / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": (4 if s.ve else 3) * K,   # (gate,) prologue, prologue repairs, attention
+        "gpu_launches": (3 if s.ve else 2) * K,   # (gate,) prologue with its repairs, attention
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -610,9 +610,9 @@ def run_backward(args, s):
     flops = 2.5 * flops_per_step(s)
     tf = flops / (ms * 1e-3) / 1e12
     peaks, peak_src = load_peaks()
-    # RoPE table, prologue, prologue repairs, row statistics, dQ, dK/dV; on value-embedding
-    # layers also the gate and the three gate-gradient kernels
-    launches = 6 + (4 if s.ve else 0)
+    # RoPE table, prologue, row statistics, dQ, dK/dV; on value-embedding layers also the gate and
+    # the three gate-gradient kernels
+    launches = 5 + (4 if s.ve else 0)
     line = {
         "metric": "attention backward TFLOP/s (10 D flops per visible pair)",
         "value": tf, "unit": "TFLOP/s", "n_gpus": 1, "steps": K, "warmup": args.warmup,
@@ -774,8 +774,8 @@ def run_sssl(args):
         "roofline": {"bound": "tensor", "achieved": tf, "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
                      "frac": tf / float(peaks["bf16_tflops"]), "traffic": None,
                      "note": f"whole stack of public calls; peak = {peak_src} dense bf16 (burst)"},
-        # per layer: (gate,) prologue, prologue repairs, attention
-        "gpu_launches": sum(4 if ls.ve else 3 for ls in shapes) * K,
+        # per layer: (gate,) prologue with its repairs, attention
+        "gpu_launches": sum(3 if ls.ve else 2 for ls in shapes) * K,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

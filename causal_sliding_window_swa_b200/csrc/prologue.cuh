@@ -11,7 +11,7 @@
 // is organised (an fp32-only pipeline flips the last bf16 bit of ~1e-4 of the elements, which
 // moves single attention scores by ~1e-3).  The common path runs in fp32 with a proven error
 // bound; an element whose fp32 result could round differently from the exact one (a few in 10^4)
-// is listed and recomputed in fp64 by a second, small kernel that overwrites it.
+// is listed, and its block recomputes it in fp64 and overwrites it after its last row chunk.
 //   norm: r = 1 / sqrt(ss / D + eps) from the sum of squares of the raw inputs (the rotation
 //     preserves it) in fp64, where each square and the sum are exact; the inverse square root by
 //     two Newton-Raphson steps from the hardware estimate, then rounded once to fp32.
@@ -272,15 +272,16 @@ __device__ __forceinline__ uint2 gated_add4(const uint2& vw, const uint2& ew, fl
 }
 
 // ------------------------------------------------------------------ deferred repairs
-// The prologue kernel writes every output from its fp32 fast path.  For a row chunk (D/8 threads
-// per row; four rotation pairs and eight v' elements per thread) with elements that fast path
-// cannot certify, it lists (chunk, flags) in its block's list: flag bits 0-3 qhat pairs i0 + e
-// (elements i0 + e and i0 + e + D/2), bits 4-7 khat pairs, bits 8-11 v' elements i0 + e, bits
-// 12-15 v' elements i0 + D/2 + e.  prologue_fix_kernel recomputes the flagged elements in fp64 and
-// overwrites them.  A block whose list overflows (inputs built to sit on rounding midpoints) has
-// every element of its row chunks recomputed instead.  An item carries the rows' fp64 r (the fast
+// The prologue kernel writes every output from its fp32 fast path.  A row chunk (D/8 threads per
+// row; four rotation pairs and eight v' elements per thread) with elements that fast path cannot
+// certify goes on its block's shared-memory list as (chunk, flags): flag bits 0-3 qhat pairs
+// i0 + e (elements i0 + e and i0 + e + D/2), bits 4-7 khat pairs, bits 8-11 v' elements i0 + e,
+// bits 12-15 v' elements i0 + D/2 + e.  The grid is a single wave of blocks, so each block
+// repairs its list once, after its last chunk: its threads recompute the listed elements in fp64
+// and overwrite them.  A block whose list overflows (inputs built to sit on rounding midpoints)
+// recomputes every element of its row chunks instead.  An item carries the rows' fp64 r (the fast
 // path already has it), so that a repair needs only the chunk's own inputs.
-constexpr int kFixPerBlock = 256;
+constexpr int kFixPerBlock = 1024;
 
 struct __align__(16) FixItem {
     uint32_t chunk_lo;     // row chunk index, low 32 bits
@@ -299,14 +300,9 @@ struct FixParams {
     __nv_bfloat16* kh;
     __nv_bfloat16* vp;
     const double2* tab64;
-    int T, H, Hkv, D;
+    int T;
+    int heads;                 // heads of the pass's rows (H, or Hkv for the key/value pass)
     double eps;
-    // the prologue pass these lists belong to
-    int heads;                 // heads of its rows (H, or Hkv for the key/value pass)
-    uint32_t all_flags;        // flag bits of the outputs it computes
-    long long n_chunks;        // rows * D / 8
-    long long stride;          // its grid's thread count
-    int n_iter;                // loop iterations of each of its threads
 };
 
 // 1 / sqrt(ss / D + eps) of one row in fp64: exact squares, fp64 sums.  All loads are issued
@@ -333,9 +329,10 @@ __device__ __forceinline__ double row_r64(const __nv_bfloat16* __restrict__ x, d
 
 // The flagged elements of one row chunk in fp64, each rounded once: the rotation with the fp64
 // table scaled by the row's r; v + g ve with g = g_hi + g_lo.  The loads of a tensor's row and of
-// the chunk's four pairs are issued together.
+// the chunk's four pairs are issued together.  Out of line: it runs for a few chunks in 10^4.
 template <int D>
-__device__ void prologue_fix_chunk(long long chunk, uint32_t flags, const FixParams& p, const double* r_known) {
+__device__ __noinline__ void prologue_fix_chunk(long long chunk, uint32_t flags, const FixParams& p,
+                                                double rq, double rk, bool r_known) {
     constexpr int TPR = D / 8, HALF = D / 2;
     const uint32_t row = (uint32_t)(chunk / TPR);
     const int i0 = 4 * (int)(chunk % TPR);
@@ -354,7 +351,7 @@ __device__ void prologue_fix_chunk(long long chunk, uint32_t flags, const FixPar
         float a[4], b[4];
         unpack4(*reinterpret_cast<const uint2*>(x + i0), a);
         unpack4(*reinterpret_cast<const uint2*>(x + HALF + i0), b);
-        const double r64 = r_known != nullptr ? r_known[tensor] : row_r64<D>(x, p.eps);
+        const double r64 = r_known ? (tensor == 0 ? rq : rk) : row_r64<D>(x, p.eps);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             if (!((m >> e) & 1u)) continue;
@@ -381,38 +378,6 @@ __device__ void prologue_fix_chunk(long long chunk, uint32_t flags, const FixPar
     }
 }
 
-// One warp per prologue block's list (a single wave for the usual grid); its lanes take the
-// list's items.  An overflowed list (count > kFixPerBlock) has its warp walk all the row chunks
-// of that block instead.
-template <int D>
-__global__ void __launch_bounds__(256) prologue_fix_kernel(const int* __restrict__ counts, const FixItem* __restrict__ items,
-                                                           int n_lists, const __grid_constant__ FixParams p) {
-    // a programmatic dependent of the prologue kernel: wait for it, then let the attention launch
-    grid_dependency_wait();
-    grid_dependents_launch();
-    const int lane = (int)(threadIdx.x & 31u);
-    const int n_warps = (int)((gridDim.x * blockDim.x) >> 5);
-    for (int list = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); list < n_lists; list += n_warps) {
-        // the count and the lane's first item are read together; slots past the count are ignored
-        const int cnt = __ldg(counts + list);
-        FixItem it = items[(long long)list * kFixPerBlock + lane];
-        if (cnt <= kFixPerBlock) {
-            for (int slot = lane; slot < cnt; slot += 32) {
-                if (slot != lane) it = items[(long long)list * kFixPerBlock + slot];
-                const double r[2] = {it.rq, it.rk};
-                prologue_fix_chunk<D>((long long)it.chunk_lo | ((long long)(it.code >> 16) << 32), it.code & 0xffffu,
-                                      p, r);
-            }
-        } else {
-            // the block's threads handled chunks list * 256 + u + it * stride, u < 256, it < n_iter
-            for (long long j = lane; j < 256ll * p.n_iter; j += 32) {
-                const long long c = (long long)list * 256 + (j & 255) + (j >> 8) * p.stride;
-                if (c < p.n_chunks) prologue_fix_chunk<D>(c, p.all_flags, p, nullptr);
-            }
-        }
-    }
-}
-
 // PARTS selects the outputs: bit 0 qhat, bit 1 khat and v' (v' only on value-embedding layers).
 // The multi-head layer runs both in one pass (PARTS = 3, rows (b,t,h) of all inputs); with
 // grouped-query attention the query rows (H heads) and the key/value rows (Hkv heads) are two
@@ -423,19 +388,19 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(
     const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ ve,
     const float2* __restrict__ gate,
     __nv_bfloat16* __restrict__ qh, __nv_bfloat16* __restrict__ kh, __nv_bfloat16* __restrict__ vp,
-    const float4* __restrict__ tab32, int* __restrict__ sched,
-    int n_rows, int T, int H, FastDiv divT, FastDiv divH, double eps, int* __restrict__ fix_counts,
-    FixItem* __restrict__ fix_items) {
+    const float4* __restrict__ tab32, const double2* __restrict__ tab64, int* __restrict__ sched,
+    int n_rows, int T, int H, FastDiv divT, FastDiv divH, double eps) {
     constexpr int TPR = D / 8;           // threads per row (16 or 8); divides 32
     constexpr int LOG_TPR = (D == 128) ? 4 : 3;
     constexpr int HALF = D / 2;
+    constexpr bool DO_Q = (PARTS & 1) != 0, DO_KV = (PARTS & 2) != 0;
     const long long gtid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
     const long long stride = (long long)gridDim.x * blockDim.x;
     // Every thread of a warp runs the same number of iterations, so the shuffles always see the
     // full warp; rows past the end are computed on zeros and not stored.
     const long long n_iter = ((long long)n_rows * TPR + stride - 1) / stride;
     // Launched as a programmatic dependent of the gate kernel: wait for it before any memory
-    // access, then let the repair kernel launch.
+    // access, then let the attention kernel launch (it waits for this grid to finish).
     grid_dependency_wait();
     grid_dependents_launch();
     // The attention kernel that follows takes its work items from this counter.
@@ -443,7 +408,7 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(
         sched[0] = 0;
         sched[1] = 0;
     }
-    // This block's list of row chunks to repair (prologue_fix_kernel).
+    // This block's list of row chunks to repair once all of them are written.
     __shared__ int s_nfix;
     __shared__ FixItem s_fix[kFixPerBlock];
     if (threadIdx.x == 0) s_nfix = 0;
@@ -460,7 +425,6 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(
         const long long off = (long long)row * D;
 
         // Every load of this row chunk is issued before any arithmetic.
-        constexpr bool DO_Q = (PARTS & 1) != 0, DO_KV = (PARTS & 2) != 0;
         uint2 raw[8];
         float2 gw = make_float2(0.f, 0.f);
         if (valid) {
@@ -536,11 +500,25 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(
             }
         }
     }
+    // The repairs: after the barrier every fast-path store of the block is ordered before them.
     __syncthreads();
     const int nf = s_nfix;
-    for (int i = threadIdx.x; i < min(nf, kFixPerBlock); i += blockDim.x)
-        fix_items[(long long)blockIdx.x * kFixPerBlock + i] = s_fix[i];
-    if (threadIdx.x == 0) fix_counts[blockIdx.x] = nf;
+    if (nf == 0) return;
+    const FixParams fp{q, k, v, ve, gate, qh, kh, vp, tab64, T, H, eps};
+    if (nf <= kFixPerBlock) {
+        for (int i = threadIdx.x; i < nf; i += blockDim.x) {
+            const FixItem item = s_fix[i];
+            prologue_fix_chunk<D>((long long)item.chunk_lo | ((long long)(item.code >> 16) << 32), item.code & 0xffffu,
+                                  fp, item.rq, item.rk, true);
+        }
+    } else {
+        constexpr uint32_t all = ((PARTS & 1) ? 0x000fu : 0u) | ((PARTS & 2) ? 0x00f0u : 0u) |
+                                 ((PARTS & 2) && HAS_VE ? 0xff00u : 0u);
+        for (long long it = 0; it < n_iter; ++it) {
+            const long long tid = gtid + it * stride;
+            if (tid < (long long)n_rows * TPR) prologue_fix_chunk<D>(tid, all, fp, 0.0, 0.0, false);
+        }
+    }
 }
 
 }  // namespace swa

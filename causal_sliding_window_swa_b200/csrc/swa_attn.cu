@@ -112,25 +112,18 @@ constexpr size_t kAlign = 1024;
 size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct WsLayout {
-    size_t qh, kh, vp, gate, tab32, tab64, sched, dstart, fixc, fixi, total;
+    size_t qh, kh, vp, gate, tab32, tab64, sched, dstart, total;
 };
 
 // Grid of one prologue pass over `rows` rows: 256-thread blocks, D / 8 threads per row, at most
-// three resident blocks per SM times four waves.
+// one wave of three resident blocks per SM (each block repairs its own list at its end).
 long long prologue_blocks(long long rows, int D) {
-    return std::max<long long>(1, std::min<long long>((rows * (D / 8) + 255) / 256, 148ll * 3 * 4));
-}
-
-// Repair lists of the prologue: one per block of its pass(es).
-int prologue_fix_lists(const Shape& s) {
-    const long long rows = (long long)s.B * s.T * s.H, kv_rows = (long long)s.B * s.T * s.Hkv;
-    return (int)(prologue_blocks(rows, s.D) + (s.Hkv != s.H ? prologue_blocks(kv_rows, s.D) : 0));
+    return std::max<long long>(1, std::min<long long>((rows * (D / 8) + 255) / 256, 148ll * 3));
 }
 
 // qhat | khat | v' and gate (value-embedding layers only) | RoPE table fp32 pieces |
 // RoPE table fp64 | attention scheduler counters | document starts (B, T) int32
-// (document-masked calls only) | prologue repair-list counts (one int per prologue block of each
-// pass) | repair-list items, each section 1024-byte aligned.
+// (document-masked calls only), each section 1024-byte aligned.
 WsLayout ws_layout(const Shape& s, bool has_ve, bool has_doc = false) {
     WsLayout w{};
     const size_t tensor = round_up((size_t)s.n * 2);
@@ -144,10 +137,7 @@ WsLayout ws_layout(const Shape& s, bool has_ve, bool has_doc = false) {
     w.tab64 = w.tab32 + round_up(pairs * sizeof(float4));
     w.sched = w.tab64 + round_up(pairs * sizeof(double2));
     w.dstart = w.sched + kAlign;
-    w.fixc = w.dstart + (has_doc ? round_up((size_t)s.B * s.T * sizeof(int)) : 0);
-    const size_t lists = (size_t)prologue_fix_lists(s);
-    w.fixi = w.fixc + round_up(lists * sizeof(int));
-    w.total = w.fixi + round_up(lists * swa::kFixPerBlock * sizeof(swa::FixItem));
+    w.total = w.dstart + (has_doc ? round_up((size_t)s.B * s.T * sizeof(int)) : 0);
     return w;
 }
 
@@ -309,24 +299,6 @@ int launch_rope_table(uint8_t* ws, const WsLayout& L, const Shape& s, float rope
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
-// The deferred fp64 repairs of one prologue pass (grid `blocks`, `rows` rows of `heads` heads,
-// outputs `all_flags`): one thread per list slot.
-int launch_prologue_fix(const int* counts, const swa::FixItem* items, long long blocks, long long rows, int heads,
-                        uint32_t all_flags, swa::FixParams fp, cudaStream_t st) {
-    if (cudaGetLastError() != cudaSuccess) return SWA_ERR_CUDA;
-    fp.heads = heads;
-    fp.all_flags = all_flags;
-    fp.n_chunks = rows * (fp.D / 8);
-    fp.stride = blocks * 256;
-    fp.n_iter = (int)((fp.n_chunks + fp.stride - 1) / fp.stride);
-    const unsigned g = (unsigned)((blocks + 7) / 8);     // a warp per list
-    if (fp.D == 128)
-        launch_pdl(swa::prologue_fix_kernel<128>, dim3(g), dim3(256), 0, st, counts, items, (int)blocks, fp);
-    else
-        launch_pdl(swa::prologue_fix_kernel<64>, dim3(g), dim3(256), 0, st, counts, items, (int)blocks, fp);
-    return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
-}
-
 int launch_prologue(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
                     const void* Wg, uint8_t* ws, const WsLayout& L, const Shape& s, float eps,
                     cudaStream_t st) {
@@ -336,6 +308,8 @@ int launch_prologue(const void* q, const void* k, const void* v, const void* ve,
     const int n_kv_rows = s.B * s.T * s.Hkv;
     const swa::FastDiv divH = make_fastdiv(s.H), divT = make_fastdiv(s.T);
     float2* gate = reinterpret_cast<float2*>(ws + L.gate);
+    const int threads = 256;
+    const long long blocks = prologue_blocks(n_rows, s.D);
     if (has_ve) {
         const int n_tok = s.B * s.T;
         const int gblocks = (int)std::min<long long>(((long long)n_tok + 127) / 128, 148ll * 16);
@@ -343,10 +317,6 @@ int launch_prologue(const void* q, const void* k, const void* v, const void* ve,
         swa::gate_kernel<<<gblocks, 128, wg_smem ? 32 * s.Hkv * sizeof(double) : 0, st>>>(
             static_cast<const bf*>(gate_x), static_cast<const bf*>(Wg), gate, n_tok, s.Hkv, 32, wg_smem);
     }
-    const long long threads_total = (long long)n_rows * (s.D / 8);
-    const int threads = 256;
-    const long long blocks = prologue_blocks(n_rows, s.D);
-    (void)threads_total;
     const bf* qp = static_cast<const bf*>(q);
     const bf* kp = static_cast<const bf*>(k);
     const bf* vpi = static_cast<const bf*>(v);
@@ -357,10 +327,6 @@ int launch_prologue(const void* q, const void* k, const void* v, const void* ve,
     const float4* t32 = reinterpret_cast<const float4*>(ws + L.tab32);
     const double2* t64 = reinterpret_cast<const double2*>(ws + L.tab64);
     int* sched = reinterpret_cast<int*>(ws + L.sched);
-    int* fixc = reinterpret_cast<int*>(ws + L.fixc);
-    swa::FixItem* fixi = reinterpret_cast<swa::FixItem*>(ws + L.fixi);
-    swa::FixParams fp{qp, kp, vpi, vep, gate, qh, kh, vp, t64, s.T, s.H, s.Hkv, s.D, (double)eps, 0, 0u, 0, 0, 0};
-    const uint32_t ve_flags = has_ve ? 0xff00u : 0u;
     const unsigned g = (unsigned)blocks;
     const double e = (double)eps;
     if (s.Hkv != s.H) {
@@ -369,10 +335,10 @@ int launch_prologue(const void* q, const void* k, const void* v, const void* ve,
         const swa::FastDiv divK = make_fastdiv(s.Hkv);
         const unsigned gk = (unsigned)prologue_blocks(n_kv_rows, s.D);
 #define SWA_PRO_GQA(DD, VE)                                                                                  \
-    swa::prologue_kernel<DD, VE, 1><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, sched,      \
-                                                           n_rows, s.T, s.H, divT, divH, e, fixc, fixi); \
-    swa::prologue_kernel<DD, VE, 2><<<gk, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, sched,     \
-                                                            n_kv_rows, s.T, s.Hkv, divT, divK, e, fixc + g, fixi + (long long)g * swa::kFixPerBlock)
+    swa::prologue_kernel<DD, VE, 1><<<g, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, \
+                                                           n_rows, s.T, s.H, divT, divH, e);                 \
+    swa::prologue_kernel<DD, VE, 2><<<gk, threads, 0, st>>>(qp, kp, vpi, vep, gate, qh, kh, vp, t32, t64, sched, \
+                                                            n_kv_rows, s.T, s.Hkv, divT, divK, e)
         if (s.D == 128) {
             if (has_ve) {
                 SWA_PRO_GQA(128, true);
@@ -387,23 +353,18 @@ int launch_prologue(const void* q, const void* k, const void* v, const void* ve,
             }
         }
 #undef SWA_PRO_GQA
-        const int rc = launch_prologue_fix(fixc, fixi, g, n_rows, s.H, 0x000fu, fp, st);
-        return rc != SWA_OK ? rc
-                            : launch_prologue_fix(fixc + g, fixi + (long long)g * swa::kFixPerBlock, gk, n_kv_rows,
-                                                  s.Hkv, 0x00f0u | ve_flags, fp, st);
+        return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
     }
+#define SWA_PRO(DD, VE)                                                                                          \
+    launch_pdl(swa::prologue_kernel<DD, VE, 3>, dim3(g), dim3(threads), 0, st, qp, kp, vpi, vep, (const float2*)gate, \
+               qh, kh, vp, t32, t64, sched, n_rows, s.T, s.H, divT, divH, e)
     if (s.D == 128) {
-        if (has_ve)
-            launch_pdl(swa::prologue_kernel<128, true, 3>, dim3(g), dim3(threads), 0, st, qp, kp, vpi, vep, (const float2*)gate, qh, kh, vp, t32, sched, n_rows, s.T, s.H, divT, divH, e, fixc, fixi);
-        else
-            launch_pdl(swa::prologue_kernel<128, false, 3>, dim3(g), dim3(threads), 0, st, qp, kp, vpi, vep, (const float2*)gate, qh, kh, vp, t32, sched, n_rows, s.T, s.H, divT, divH, e, fixc, fixi);
+        if (has_ve) SWA_PRO(128, true); else SWA_PRO(128, false);
     } else {
-        if (has_ve)
-            launch_pdl(swa::prologue_kernel<64, true, 3>, dim3(g), dim3(threads), 0, st, qp, kp, vpi, vep, (const float2*)gate, qh, kh, vp, t32, sched, n_rows, s.T, s.H, divT, divH, e, fixc, fixi);
-        else
-            launch_pdl(swa::prologue_kernel<64, false, 3>, dim3(g), dim3(threads), 0, st, qp, kp, vpi, vep, (const float2*)gate, qh, kh, vp, t32, sched, n_rows, s.T, s.H, divT, divH, e, fixc, fixi);
+        if (has_ve) SWA_PRO(64, true); else SWA_PRO(64, false);
     }
-    return launch_prologue_fix(fixc, fixi, g, n_rows, s.H, 0x00ffu | ve_flags, fp, st);
+#undef SWA_PRO
+    return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
 // The attention kernel on the workspace's qhat, khat (and v' on value-embedding layers; `v` itself

@@ -157,20 +157,14 @@ def test_decode_workspace_and_validation():
 def test_backward_workspace_and_validation():
     # forward sections + row statistics (B*H*Tp float2)
     # [+ dz and the dWg partial sums on value-embedding layers] + document starts and ends (B*T int32
-    # each), each section 1024-byte aligned.  The forward's prologue repair lists (an int count and
-    # 256 32-byte items per block of each prologue pass; 256-thread blocks, D/8 threads per row, at
-    # most 1776 blocks a pass) take two passes under grouped-query attention, one otherwise.
+    # each), each section 1024-byte aligned.
     B, T, H, Hkv, D = 2, 200, 4, 2, 64
     up = lambda x: (x + 1023) // 1024 * 1024
-    blocks = lambda rows: max(1, min((rows * (D // 8) + 255) // 256, 1776))
-    fix = lambda lists: up(lists * 4) + up(lists * 256 * 32)
     fwd = swa.swa_attn_workspace_bytes(B, T, H, D, 0)
     n0 = swa.swa_attn_bwd_workspace_bytes(B, T, H, Hkv, D, 0)
     Tp = 256
     kv_fwd = up(B * T * Hkv * D * 2)
-    fix_mha, fix_gqa = fix(blocks(B * T * H)), fix(blocks(B * T * H) + blocks(B * T * Hkv))
     assert n0 == (fwd - 2 * up(B * T * H * D * 2) + 2 * kv_fwd + up(B * T * H * D * 2) - kv_fwd
-                  - fix_mha + fix_gqa
                   + up(B * H * Tp * 8) + 2 * up(B * T * 4))
     n1 = swa.swa_attn_bwd_workspace_bytes(B, T, H, Hkv, D, 1)
     assert n1 > n0 + up(B * T * Hkv * 4)

@@ -241,9 +241,9 @@ def test_prologue_bit_exact_other_constants(rope_base, eps):
 def test_prologue_dense_repairs_overflow_the_repair_lists():
     """Every v' element on a bf16 rounding tie: v in [1, 2), ve = 2^-8 (half a bf16 ulp there) and
     Wg = 0 (gate 2 sigmoid(0) = 1, so v' = v + 2^-8 exactly).  The fast path flags all of them, far
-    more than a prologue block's repair list holds (three row chunks per thread at this size), so
-    the repair kernel recomputes those blocks' chunks whole; every element must still be v rounded
-    to nearest even, element by element, as the oracle gives."""
+    more than a prologue block's repair list holds (ten row chunks per thread at this size, 1024
+    list slots per block), so each block recomputes all its chunks in fp64; every element must
+    still be v rounded to nearest even, element by element, as the oracle gives."""
     import oracle
     s = LS(1, 4096, 16, 128, 0, True, seed=44)
     d = workloads.make_layer(s)
