@@ -537,6 +537,43 @@ BwdLayout bwd_layout(const Shape& s, bool has_ve) {
     return w;
 }
 
+// A second stream per device for kernels of one call that do not depend on the kernels before
+// them on the caller's stream: they are forked from the caller's stream (an event recorded there,
+// waited on here) and joined back the same way, so everything the caller enqueued earlier happens
+// before them and everything after the join happens after them.  Calls that share the side stream
+// serialise their side kernels on it.
+std::mutex g_side_mu;                 // guards the creation of the side streams
+std::mutex g_side_mu_call[64];        // held by a call while it uses its device's side stream
+cudaStream_t g_side[64] = {nullptr};
+
+// `to` waits for everything enqueued on `from` so far.  The event is released at once; CUDA keeps
+// it until the wait is resolved.
+int stream_wait(cudaStream_t to, cudaStream_t from) {
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+        cudaGetLastError();
+        return SWA_ERR_CUDA;
+    }
+    const bool ok = cudaEventRecord(e, from) == cudaSuccess && cudaStreamWaitEvent(to, e, 0) == cudaSuccess;
+    cudaEventDestroy(e);
+    if (!ok) {
+        cudaGetLastError();
+        return SWA_ERR_CUDA;
+    }
+    return SWA_OK;
+}
+
+int side_stream(int dev, cudaStream_t* out) {
+    std::lock_guard<std::mutex> lk(g_side_mu);
+    if (g_side[dev] == nullptr && cudaStreamCreateWithFlags(&g_side[dev], cudaStreamNonBlocking) != cudaSuccess) {
+        cudaGetLastError();
+        g_side[dev] = nullptr;
+        return SWA_ERR_CUDA;
+    }
+    *out = g_side[dev];
+    return SWA_OK;
+}
+
 int launch_backward(int dev, const void* q, const void* k, const void* v, const void* ve,
                     const void* gate_x, const void* Wg, const void* out, const float* lse,
                     const void* dout, const float* dlse, void* dq, void* dk, void* dv, void* dve,
@@ -545,22 +582,30 @@ int launch_backward(int dev, const void* q, const void* k, const void* v, const 
     using bf = __nv_bfloat16;
     const bool has_ve = ve != nullptr;
     int rc;
-    // qhat, khat, v' and the gate exactly as the forward computed them.
-    if ((rc = launch_rope_table(ws, L.f, s, rope_base, st)) != SWA_OK) return rc;
-    if ((rc = launch_prologue(q, k, v, ve, gate_x, Wg, ws, L.f, s, eps, st)) != SWA_OK) return rc;
-
+    // The row statistics need only out, dout, lse and dlse: they run on the side stream while the
+    // caller's stream recomputes the prologue, and the tensor-core kernels wait for both.  The
+    // side stream is held for the whole call, so that its kernels are this call's alone.
+    std::lock_guard<std::mutex> side_lk(g_side_mu_call[dev]);
+    cudaStream_t side = nullptr;
+    if ((rc = side_stream(dev, &side)) != SWA_OK) return rc;
+    if ((rc = stream_wait(side, st)) != SWA_OK) return rc;
     int* sched4 = reinterpret_cast<int*>(ws + L.f.sched) + 4;
     float2* rowstat = reinterpret_cast<float2*>(ws + L.rowstat);
     {
         const long long rows = (long long)s.B * s.H * L.Tp;
         const int blocks = (int)((rows * (s.D / 8) + 255) / 256);   // D / 8 lanes per row
         if (s.D == 128)
-            swa::bwd_rowstat_kernel<128><<<blocks, 256, 0, st>>>(static_cast<const bf*>(out), static_cast<const bf*>(dout),
-                                                                 lse, dlse, rowstat, s.B, s.T, s.H, L.Tp, sched4);
+            swa::bwd_rowstat_kernel<128><<<blocks, 256, 0, side>>>(static_cast<const bf*>(out), static_cast<const bf*>(dout),
+                                                                   lse, dlse, rowstat, s.B, s.T, s.H, L.Tp, sched4);
         else
-            swa::bwd_rowstat_kernel<64><<<blocks, 256, 0, st>>>(static_cast<const bf*>(out), static_cast<const bf*>(dout),
-                                                                lse, dlse, rowstat, s.B, s.T, s.H, L.Tp, sched4);
+            swa::bwd_rowstat_kernel<64><<<blocks, 256, 0, side>>>(static_cast<const bf*>(out), static_cast<const bf*>(dout),
+                                                                  lse, dlse, rowstat, s.B, s.T, s.H, L.Tp, sched4);
+        if (cudaGetLastError() != cudaSuccess) return SWA_ERR_CUDA;
     }
+    // qhat, khat, v' and the gate exactly as the forward computed them.
+    if ((rc = launch_rope_table(ws, L.f, s, rope_base, st)) != SWA_OK) return rc;
+    if ((rc = launch_prologue(q, k, v, ve, gate_x, Wg, ws, L.f, s, eps, st)) != SWA_OK) return rc;
+    if ((rc = stream_wait(st, side)) != SWA_OK) return rc;
 
     CUtensorMap tq, tk, tv, tdo;
     const void* vsrc = has_ve ? static_cast<const void*>(ws + L.f.vp) : v;
@@ -627,14 +672,18 @@ int launch_backward(int dev, const void* q, const void* k, const void* v, const 
     // The rest of the prologue in reverse: the gate's inputs from dz (the epilogues did the rows).
     float* dz = reinterpret_cast<float*>(ws + L.dz);
     if (has_ve) {
+        // dgate_x on the caller's stream, dWg (two steps) on the side stream; both only read dz.
+        if ((rc = stream_wait(side, st)) != SWA_OK) return rc;
         const long long n_bt = (long long)s.B * s.T;
         const int bgx = (int)std::min<long long>((n_bt * 32 + 255) / 256, 148ll * 16);
         swa::bwd_gate_x_kernel<<<bgx, 256, 0, st>>>(dz, static_cast<const bf*>(Wg), dgate_x, n_bt, s.Hkv);
         float* part = reinterpret_cast<float*>(ws + L.wgp);
-        swa::bwd_wg_partial_kernel<<<L.wg_blocks, 256, 0, st>>>(dz, static_cast<const bf*>(gate_x), part, n_bt,
-                                                                s.Hkv, L.wg_rows);
+        swa::bwd_wg_partial_kernel<<<L.wg_blocks, 256, 0, side>>>(dz, static_cast<const bf*>(gate_x), part, n_bt,
+                                                                  s.Hkv, L.wg_rows);
         const int n = 32 * s.Hkv;
-        swa::bwd_wg_final_kernel<<<n, 256, 0, st>>>(part, dWg, L.wg_blocks, n);
+        swa::bwd_wg_final_kernel<<<n, 256, 0, side>>>(part, dWg, L.wg_blocks, n);
+        if (cudaGetLastError() != cudaSuccess) return SWA_ERR_CUDA;
+        if ((rc = stream_wait(st, side)) != SWA_OK) return rc;
     }
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
