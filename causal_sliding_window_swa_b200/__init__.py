@@ -85,6 +85,9 @@ def _load() -> ctypes.CDLL:
     lib.swa_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
                                  I, I, I, I, I, F, F, P, Z, P]
     lib.swa_attn_bwd.restype = I
+    lib.swa_attn_bwd_saved.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P,
+                                       I, I, I, I, I, F, F, P, Z, P]
+    lib.swa_attn_bwd_saved.restype = I
     lib.swa_attn_fwd_x_workspace_bytes.argtypes = [I, I, I, I, I]
     lib.swa_attn_fwd_x_workspace_bytes.restype = Z
     lib.swa_attn_qkv_prologue.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, F, P, Z, P]
@@ -212,6 +215,12 @@ def swa_attn_bwd(q, k, v, ve, gate_x, Wg, out, lse, dout, dlse, dq, dk, dv, dve,
                  B, T, H, D, window, rope_base, eps, workspace, ws_bytes, stream) -> int:
     return _lib.swa_attn_bwd(q, k, v, ve, gate_x, Wg, out, lse, dout, dlse, dq, dk, dv, dve, dgate_x, dWg,
                              B, T, H, D, window, rope_base, eps, workspace, ws_bytes, stream)
+
+
+def swa_attn_bwd_saved(q, k, v, ve, gate_x, Wg, out, lse, dout, dlse, dq, dk, dv, dve, dgate_x, dWg,
+                       B, T, H, D, window, rope_base, eps, workspace, ws_bytes, stream) -> int:
+    return _lib.swa_attn_bwd_saved(q, k, v, ve, gate_x, Wg, out, lse, dout, dlse, dq, dk, dv, dve, dgate_x, dWg,
+                                   B, T, H, D, window, rope_base, eps, workspace, ws_bytes, stream)
 
 
 def swa_attn_fwd_x_workspace_bytes(B, T, H, Hkv, D) -> int:
@@ -382,14 +391,17 @@ def swa_attn_bwd_doc(q, k, v, ve, gate_x, Wg, doc, out, lse, dout, dlse, dq, dk,
 
 
 def backward(q, k, v, out, lse, dout, window: int = 0, dlse=None, ve=None, gate_x=None, Wg=None,
-             rope_base: float = 10000.0, eps: float = 1e-6, *, workspace=None, stream=None, doc=None):
+             rope_base: float = 10000.0, eps: float = 1e-6, *, workspace=None, stream=None, doc=None,
+             saved: bool = False):
     """Gradient of one layer (C call swa_attn_bwd_gqa) for the loss sum(dout * out) +
     sum(dlse * lse).  q, k, v, ve, gate_x, Wg as for ``forward``; out bf16 (B,T,H,D) and lse fp32
     (B,H,T) are that call's outputs; dout bf16 (B,T,H,D); dlse fp32 (B,H,T) or None.
     Returns a dict: dq bf16 (B,T,H,D), dk, dv bf16 (B,T,Hkv,D) and, on value-embedding layers,
     dve bf16 (B,T,Hkv,D), dgate_x fp32 (B,T,32), dWg fp32 [32,Hkv].  ``doc``: the int32 (B, T)
-    document ids of a document-masked forward (C call swa_attn_bwd_doc).  Raises SwaError on a
-    nonzero status."""
+    document ids of a document-masked forward (C call swa_attn_bwd_doc).  ``saved``: `workspace`
+    (swa_attn_bwd_workspace_bytes() bytes) was passed to the ``forward(..., workspace=...)`` call
+    that produced out and lse, so the prologue is not recomputed (C call swa_attn_bwd_saved;
+    multi-head, no document mask).  Raises SwaError on a nonzero status."""
     import torch
     B, T, H, Hkv, D = _check_qkv(q, k, v, ve, gate_x, Wg)
     for name, t in (("out", out), ("dout", dout)):
@@ -411,6 +423,17 @@ def backward(q, k, v, out, lse, dout, window: int = 0, dlse=None, ve=None, gate_
     if doc is not None and (tuple(doc.shape) != (B, T) or doc.dtype != torch.int32 or not doc.is_cuda
                             or not doc.is_contiguous()):
         raise ValueError(f"doc must be a contiguous CUDA int32 tensor of shape {(B, T)}")
+    if saved:
+        if Hkv != H or doc is not None or workspace is None:
+            raise ValueError("saved=True needs the forward's workspace, Hkv == H and no document mask")
+        rc = swa_attn_bwd_saved(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(out), _ptr(lse),
+                                _ptr(dout), _ptr(dlse), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g.get("dve")),
+                                _ptr(g.get("dgate_x")), _ptr(g.get("dWg")), B, T, H, D, int(window), float(rope_base),
+                                float(eps), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _stream_handle(stream))
+        if rc != SWA_OK:
+            raise SwaError(rc, "swa_attn_bwd_saved")
+        return g
     rc = swa_attn_bwd_doc(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(doc), _ptr(out),
                           _ptr(lse), _ptr(dout), _ptr(dlse), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
                           _ptr(g.get("dve")), _ptr(g.get("dgate_x")), _ptr(g.get("dWg")), B, T, H, Hkv, D,
@@ -490,6 +513,6 @@ __all__ = [
     "swa_attn_last_device_status",
     "swa_attn_set_wait_limit_ms", "swa_attn_selftest_wait", "swa_attn_version",
     "swa_attn_decode", "swa_attn_decode_workspace_bytes", "swa_attn_fwd_gqa", "swa_attn_fwd_doc",
-    "swa_attn_bwd", "swa_attn_bwd_gqa", "swa_attn_bwd_doc", "swa_attn_bwd_workspace_bytes",
+    "swa_attn_bwd", "swa_attn_bwd_saved", "swa_attn_bwd_gqa", "swa_attn_bwd_doc", "swa_attn_bwd_workspace_bytes",
     "swa_attn_fwd_x", "swa_attn_qkv_prologue", "swa_attn_fwd_x_workspace_bytes",
 ]

@@ -578,7 +578,8 @@ int launch_backward(int dev, const void* q, const void* k, const void* v, const 
                     const void* gate_x, const void* Wg, const void* out, const float* lse,
                     const void* dout, const float* dlse, void* dq, void* dk, void* dv, void* dve,
                     float* dgate_x, float* dWg, const Shape& s, int window, float rope_base, float eps,
-                    uint8_t* ws, const BwdLayout& L, cudaStream_t st, const int* doc = nullptr) {
+                    uint8_t* ws, const BwdLayout& L, cudaStream_t st, const int* doc = nullptr,
+                    bool prologue_saved = false) {
     using bf = __nv_bfloat16;
     const bool has_ve = ve != nullptr;
     int rc;
@@ -602,9 +603,12 @@ int launch_backward(int dev, const void* q, const void* k, const void* v, const 
                                                                   lse, dlse, rowstat, s.B, s.T, s.H, L.Tp, sched4);
         if (cudaGetLastError() != cudaSuccess) return SWA_ERR_CUDA;
     }
-    // qhat, khat, v' and the gate exactly as the forward computed them.
-    if ((rc = launch_rope_table(ws, L.f, s, rope_base, st)) != SWA_OK) return rc;
-    if ((rc = launch_prologue(q, k, v, ve, gate_x, Wg, ws, L.f, s, eps, st)) != SWA_OK) return rc;
+    // qhat, khat, v' and the gate exactly as the forward computed them (unless the caller's forward
+    // left them in this workspace).
+    if (!prologue_saved) {
+        if ((rc = launch_rope_table(ws, L.f, s, rope_base, st)) != SWA_OK) return rc;
+        if ((rc = launch_prologue(q, k, v, ve, gate_x, Wg, ws, L.f, s, eps, st)) != SWA_OK) return rc;
+    }
     if ((rc = stream_wait(st, side)) != SWA_OK) return rc;
 
     CUtensorMap tq, tk, tv, tdo;
@@ -1072,11 +1076,17 @@ size_t swa_attn_bwd_workspace_bytes(int B, int T, int H, int Hkv, int D, int has
     return bwd_layout(s, has_ve != 0).total;
 }
 
-int swa_attn_bwd_doc(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
-                     const void* Wg, const int* doc, const void* out, const float* lse, const void* dout,
-                     const float* dlse, void* dq, void* dk, void* dv, void* dve, float* dgate_x,
-                     float* dWg, int B, int T, int H, int Hkv, int D, int window, float rope_base,
-                     float eps, void* workspace, size_t ws_bytes, swa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The backward entry points after argument checks; prologue_saved: qhat, khat, v', the gates and
+// the RoPE tables are already in the workspace (left there by swa_attn_fwd_ws).
+int bwd_checked(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                const void* Wg, const int* doc, const void* out, const float* lse, const void* dout,
+                const float* dlse, void* dq, void* dk, void* dv, void* dve, float* dgate_x,
+                float* dWg, int B, int T, int H, int Hkv, int D, int window, float rope_base,
+                float eps, void* workspace, size_t ws_bytes, swa_stream_t stream, bool prologue_saved) {
     if (doc != nullptr && !aligned(doc, 4)) return SWA_ERR_MISALIGNED;
     Shape s;
     int rc = check_sizes(B, T, H, D, &s);
@@ -1097,7 +1107,29 @@ int swa_attn_bwd_doc(const void* q, const void* k, const void* v, const void* ve
     if ((rc = device_ready(&dev)) != SWA_OK) return rc;
     return launch_backward(dev, q, k, v, ve, gate_x, Wg, out, lse, dout, dlse, dq, dk, dv, dve, dgate_x, dWg, s,
                            window, rope_base, eps, static_cast<uint8_t*>(workspace), L,
-                           reinterpret_cast<cudaStream_t>(stream), doc);
+                           reinterpret_cast<cudaStream_t>(stream), doc, prologue_saved);
+}
+
+}  // namespace
+
+extern "C" {
+
+int swa_attn_bwd_doc(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                     const void* Wg, const int* doc, const void* out, const float* lse, const void* dout,
+                     const float* dlse, void* dq, void* dk, void* dv, void* dve, float* dgate_x,
+                     float* dWg, int B, int T, int H, int Hkv, int D, int window, float rope_base,
+                     float eps, void* workspace, size_t ws_bytes, swa_stream_t stream) {
+    return bwd_checked(q, k, v, ve, gate_x, Wg, doc, out, lse, dout, dlse, dq, dk, dv, dve, dgate_x, dWg, B, T, H,
+                       Hkv, D, window, rope_base, eps, workspace, ws_bytes, stream, false);
+}
+
+int swa_attn_bwd_saved(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,
+                       const void* Wg, const void* out, const float* lse, const void* dout, const float* dlse,
+                       void* dq, void* dk, void* dv, void* dve, float* dgate_x, float* dWg, int B, int T,
+                       int H, int D, int window, float rope_base, float eps, void* workspace, size_t ws_bytes,
+                       swa_stream_t stream) {
+    return bwd_checked(q, k, v, ve, gate_x, Wg, nullptr, out, lse, dout, dlse, dq, dk, dv, dve, dgate_x, dWg, B, T,
+                       H, H, D, window, rope_base, eps, workspace, ws_bytes, stream, true);
 }
 
 int swa_attn_bwd_gqa(const void* q, const void* k, const void* v, const void* ve, const void* gate_x,

@@ -373,6 +373,23 @@ SWA_API int swa_attn_bwd_doc(const void* q, const void* k, const void* v, const 
                              float* dgate_x, float* dWg, int B, int T, int H, int Hkv, int D, int window,
                              float rope_base, float eps, void* workspace, size_t ws_bytes,
                              swa_stream_t stream);
+/*
+ * swa_attn_bwd_saved: the multi-head backward (as swa_attn_bwd) for a caller that keeps the
+ * forward's activations.  Use it when `workspace` (swa_attn_bwd_workspace_bytes() bytes, which
+ * covers swa_attn_workspace_bytes()) was passed to the swa_attn_fwd_ws() call that produced `out`
+ * and `lse`, with the same q, k, v, ve, gate_x, Wg, sizes, rope_base and eps, and nothing has
+ * written to it since.  That call left qhat, khat, v', the gates and the RoPE tables at the
+ * offsets this backward reads, so the prologue is not recomputed.  The gradients are bit-identical
+ * to swa_attn_bwd's.  The call cannot check that the workspace holds this layer's forward state:
+ * any other content gives wrong gradients (every access stays inside the workspace).
+ */
+SWA_API int swa_attn_bwd_saved(const void* q, const void* k, const void* v, const void* ve,
+                               const void* gate_x, const void* Wg, const void* out, const float* lse,
+                               const void* dout, const float* dlse, void* dq, void* dk, void* dv,
+                               void* dve, float* dgate_x, float* dWg, int B, int T, int H, int D,
+                               int window, float rope_base, float eps, void* workspace, size_t ws_bytes,
+                               swa_stream_t stream);
+
 /* The multi-head layer: swa_attn_bwd_gqa with Hkv = H. */
 SWA_API int swa_attn_bwd(const void* q, const void* k, const void* v, const void* ve,
                          const void* gate_x, const void* Wg, const void* out, const float* lse,

@@ -170,3 +170,71 @@ def test_backward_is_deterministic_and_leaves_its_inputs_alone():
         assert torch.equal(runs[0][k], runs[1][k]), k
     for k, v in before.items():
         assert torch.equal(v, ins[k]), k
+
+
+def test_concurrent_calls_on_two_streams_match_serial():
+    """Two host threads, each with its own stream and workspace, run backward calls at the same
+    time.  The row statistics and the dWg sums of every call go through the library's per-device
+    side stream, forked from and joined back into the caller's stream.  Every gradient must equal
+    that of a serial call bit for bit."""
+    import threading
+    prepared = []
+    for s, d, dout, dlse in (_case(1, 520, 2, 128, 100, True, seed=71), _case(2, 300, 2, 64, 0, True, seed=72)):
+        gi = {k: (v.cuda() if v is not None else None) for k, v in workloads.gpu_side_inputs(d).items()}
+        out, lse = swa.forward(gi["q"], gi["k"], gi["v"], s.window, ve=gi["ve"], gate_x=gi["gate_x"], Wg=gi["Wg"])
+        prepared.append((s, gi, out, lse, dout.cuda(), dlse.cuda()))
+
+    def call(pp, stream):
+        s, gi, out, lse, dout, dlse = pp
+        with torch.cuda.stream(stream):
+            return swa.backward(gi["q"], gi["k"], gi["v"], out, lse, dout, s.window, dlse=dlse, ve=gi["ve"],
+                                gate_x=gi["gate_x"], Wg=gi["Wg"], stream=stream)
+
+    main = torch.cuda.current_stream()
+    ref = [call(pp, main) for pp in prepared]
+    torch.cuda.synchronize()
+    swa.check_device_status()
+    results = [[], []]
+    errors = []
+
+    def worker(i):
+        try:
+            st = torch.cuda.Stream()
+            for _ in range(4):
+                results[i].append(call(prepared[i], st))
+            st.synchronize()
+        except Exception as e:  # reported below, on the test's thread
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    torch.cuda.synchronize()
+    swa.check_device_status()
+    for i in range(2):
+        assert len(results[i]) == 4
+        for g in results[i]:
+            for name, want in ref[i].items():
+                assert torch.equal(g[name], want), (i, name)
+
+
+@pytest.mark.parametrize("B,T,H,D,window,ve", [(1, 520, 2, 128, 100, True), (2, 300, 2, 64, 0, False)])
+def test_saved_activations_match_recompute(B, T, H, D, window, ve):
+    """backward(saved=True) on the workspace the forward wrote (qhat, khat, v', the gates and the
+    RoPE tables stay there) gives the recomputing backward's gradients bit for bit."""
+    s, d, dout, dlse = _case(B, T, H, D, window, ve, seed=81)
+    gi = {k: (v.cuda() if v is not None else None) for k, v in workloads.gpu_side_inputs(d).items()}
+    ws = torch.empty(swa.swa_attn_bwd_workspace_bytes(B, T, H, H, D, int(ve)), dtype=torch.uint8, device="cuda")
+    out, lse = swa.forward(gi["q"], gi["k"], gi["v"], s.window, ve=gi["ve"], gate_x=gi["gate_x"], Wg=gi["Wg"],
+                           workspace=ws)
+    kw = dict(dlse=dlse.cuda(), ve=gi["ve"], gate_x=gi["gate_x"], Wg=gi["Wg"])
+    ref = swa.backward(gi["q"], gi["k"], gi["v"], out, lse, dout.cuda(), s.window, **kw)
+    got = swa.backward(gi["q"], gi["k"], gi["v"], out, lse, dout.cuda(), s.window, **kw, workspace=ws, saved=True)
+    torch.cuda.synchronize()
+    swa.check_device_status()
+    assert set(got) == set(ref)
+    for name in ref:
+        assert torch.equal(got[name], ref[name]), name
