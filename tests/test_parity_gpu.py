@@ -253,10 +253,15 @@ def test_prologue_dense_repairs_overflow_the_repair_lists():
     d["table"] = torch.full_like(d["table"], 2.0 ** -8)
     d["Wg"] = torch.zeros_like(d["Wg"])
     got = _prologue_on_gpu(s, parity.to_device(d))
-    _, _, vp = oracle.prologue(d, eps=float(np.float32(1e-6)), parity=True)
+    qh, kh, vp = oracle.prologue(d, eps=float(np.float32(1e-6)), parity=True)
     v = d["v"].float()
     even = (mant % 2 == 0)
     expect = torch.where(even, v, v + 2.0 ** -7)                              # ties to even
     assert torch.equal(torch.from_numpy(vp).float(), expect)                 # the oracle agrees
     mism = (got["vp"] != _bits_of(vp)).sum().item()
     assert mism == 0, f"v': {mism} of {vp.size} values differ"
+    # the overflowing blocks recompute qhat and khat of all their chunks in fp64 as well
+    for name, ref in (("qh", qh), ("kh", kh)):
+        mism = (got[name] != _bits_of(ref)).sum().item()
+        assert mism == 0, f"{name}: {mism} of {ref.size} values differ"
+
