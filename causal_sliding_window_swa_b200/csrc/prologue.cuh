@@ -101,8 +101,10 @@ __device__ __forceinline__ void rope_split(double c, float& hi, float& lo) {
     lo = (float)(c - (double)hi);
 }
 
-__global__ void rope_table_kernel(float4* __restrict__ tab32, double2* __restrict__ tab64, int T,
-                                  int D, double base) {
+// tab2 (optional, for the fused projection's epilogue): (c_hi + c_lo, s_hi + s_lo) summed in fp32,
+// the values that epilogue uses; tab64 may then be null (the fused path keeps tab2 in its place).
+__global__ void rope_table_kernel(float4* __restrict__ tab32, double2* __restrict__ tab64, float2* __restrict__ tab2,
+                                  int T, int D, double base) {
     const int half = D / 2;
     const long long n = (long long)T * half;
     for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
@@ -116,7 +118,8 @@ __global__ void rope_table_kernel(float4* __restrict__ tab32, double2* __restric
         rope_split(c, c_hi, c_lo);
         rope_split(s, s_hi, s_lo);
         tab32[idx] = make_float4(c_hi, c_lo, s_hi, s_lo);
-        tab64[idx] = make_double2(c, s);
+        if (tab64 != nullptr) tab64[idx] = make_double2(c, s);
+        if (tab2 != nullptr) tab2[idx] = make_float2(c_hi + c_lo, s_hi + s_lo);
     }
 }
 

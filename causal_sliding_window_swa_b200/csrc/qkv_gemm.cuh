@@ -65,7 +65,7 @@ struct QkvParams {
     int n_ntiles;          // (H + 2 Hkv) D / BN
     int n_tiles;           // ceil(M / 128) * n_ntiles
     float eps;
-    const float4* tab32;   // RoPE table (c_hi, c_lo, s_hi, s_lo) per (t, i)
+    const float2* tab2;    // RoPE (c, s) per (t, i): the fp32 sums c_hi + c_lo, s_hi + s_lo
     const float2* gate;    // (B*T, Hkv) (g_hi, g_lo), value-embedding layers
     const __nv_bfloat16* ve;   // (B*T, Hkv, D), value-embedding layers
     __nv_bfloat16* qh;     // (B*T, H, D)
@@ -103,7 +103,7 @@ __device__ __forceinline__ void qkv_head_row(uint32_t taddr, bool is_v, bool liv
         }
         const float r = (float)(1.0 / sqrt((double)ss / (double)D + (double)p.eps));
         // pass 2: rotate 16 pairs at a time, scale, round, store
-        const float4* tab = p.tab32 + (long long)t * HALF;
+        const float2* tab = p.tab2 + (long long)t * HALF;
 #pragma unroll
         for (int i0 = 0; i0 < HALF; i0 += 16) {
             uint32_t a[16], b[16];
@@ -114,8 +114,8 @@ __device__ __forceinline__ void qkv_head_row(uint32_t taddr, bool is_v, bool liv
             uint32_t wa[8], wb[8];
 #pragma unroll
             for (int e = 0; e < 16; e += 2) {
-                const float4 t0 = tab[i0 + e], t1 = tab[i0 + e + 1];
-                const float c0 = t0.x + t0.y, s0 = t0.z + t0.w, c1 = t1.x + t1.y, s1 = t1.z + t1.w;
+                const float2 t0 = tab[i0 + e], t1 = tab[i0 + e + 1];
+                const float c0 = t0.x, s0 = t0.y, c1 = t1.x, s1 = t1.y;
                 const float a0 = __uint_as_float(a[e]), b0 = __uint_as_float(b[e]);
                 const float a1 = __uint_as_float(a[e + 1]), b1 = __uint_as_float(b[e + 1]);
                 wa[e >> 1] = pack_bf16x2((a0 * c0 - b0 * s0) * r, (a1 * c1 - b1 * s1) * r);

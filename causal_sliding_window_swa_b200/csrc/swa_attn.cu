@@ -289,13 +289,16 @@ void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
     cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-int launch_rope_table(uint8_t* ws, const WsLayout& L, const Shape& s, float rope_base, cudaStream_t st) {
+// fused: the fused projection's table, (c, s) as fp32 sums in the section that otherwise holds the
+// fp64 table (which only the prologue's repairs read).
+int launch_rope_table(uint8_t* ws, const WsLayout& L, const Shape& s, float rope_base, cudaStream_t st,
+                      bool fused = false) {
     const long long n = (long long)s.T * (s.D / 2);
     const int threads = 256;
     const long long blocks = std::min<long long>((n + threads - 1) / threads, 148ll * 16);
     swa::rope_table_kernel<<<(unsigned)blocks, threads, 0, st>>>(
-        reinterpret_cast<float4*>(ws + L.tab32), reinterpret_cast<double2*>(ws + L.tab64), s.T, s.D,
-        (double)rope_base);
+        reinterpret_cast<float4*>(ws + L.tab32), fused ? nullptr : reinterpret_cast<double2*>(ws + L.tab64),
+        fused ? reinterpret_cast<float2*>(ws + L.tab64) : nullptr, s.T, s.D, (double)rope_base);
     return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
@@ -480,7 +483,7 @@ int launch_qkv(int dev, const void* x, const void* Wqkv, const void* ve, const v
     p.n_ntiles = (N + BN - 1) / BN;
     p.n_tiles = (int)((M + 127) / 128) * p.n_ntiles;
     p.eps = eps;
-    p.tab32 = reinterpret_cast<const float4*>(ws + L.tab32);
+    p.tab2 = reinterpret_cast<const float2*>(ws + L.tab64);
     p.gate = has_ve ? gate : nullptr;
     p.ve = static_cast<const bf*>(ve);
     p.qh = static_cast<bf*>(qh);
@@ -1040,7 +1043,7 @@ int swa_attn_qkv_prologue(const void* x, const void* Wqkv, const void* ve, const
     if ((rc = device_ready(&dev)) != SWA_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    if ((rc = launch_rope_table(ws, L, s, rope_base, st)) != SWA_OK) return rc;
+    if ((rc = launch_rope_table(ws, L, s, rope_base, st, true)) != SWA_OK) return rc;
     return launch_qkv(dev, x, Wqkv, ve, Wg, C, s, eps, ws, L, qh, kh, vp, nullptr, st);
 }
 
@@ -1061,7 +1064,7 @@ int swa_attn_fwd_x(const void* x, const void* Wqkv, const void* ve, const void* 
     if ((rc = device_ready(&dev)) != SWA_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    if ((rc = launch_rope_table(ws, L, s, rope_base, st)) != SWA_OK) return rc;
+    if ((rc = launch_rope_table(ws, L, s, rope_base, st, true)) != SWA_OK) return rc;
     if ((rc = launch_qkv(dev, x, Wqkv, ve, Wg, C, s, eps, ws, L, ws + L.qh, ws + L.kh, ws + L.vp,
                          reinterpret_cast<int*>(ws + L.sched), st)) != SWA_OK)
         return rc;

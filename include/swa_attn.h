@@ -305,7 +305,9 @@ SWA_API int swa_attn_decode_doc(const void* q, const void* k, const void* v,
  * swa_attn_qkv_prologue writes qh bf16 (B, T, H, D), kh and vp bf16 (B, T, Hkv, D) (caller buffers);
  * swa_attn_fwd_x writes out bf16 (B, T, H, D) and lse fp32 (B, H, T) (NULL = skip) with qhat, khat,
  * v' kept in the workspace.  workspace: at least swa_attn_fwd_x_workspace_bytes(B, T, H, Hkv, D)
- * bytes, 16-byte aligned, nothing kept between calls.  Asynchronous on `stream`; arguments are
+ * bytes, 16-byte aligned, nothing kept between calls.  Both calls leave the workspace's RoPE table
+ * in their own form (fp32 cos and sin, no fp64 copy): on a workspace they used, call
+ * swa_attn_rope_table() again before swa_attn_prologue().  Asynchronous on `stream`; arguments are
  * validated before anything is enqueued.  Errors: SWA_ERR_INVALID_ARG (null pointer, ve / Wg not
  * both set, C < 32 with the value embedding, Hkv not dividing H, bad rope_base / eps),
  * SWA_ERR_UNSUPPORTED (D not 64 / 128, C not a multiple of 8, sizes beyond int32),
