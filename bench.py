@@ -111,6 +111,18 @@ class L2Flush:
 L2_NOTE = "flushed between steps (256 MB write, then a 256 MB read of another buffer; outside the timed events)"
 
 
+def drain(dev):
+    """Wait for the device while the clock sampler keeps sampling: poll an event recorded after
+    the enqueued work and sleep between polls (one blocking synchronize can keep the sampler
+    thread from running until the work is done)."""
+    import torch
+    ev = torch.cuda.Event()
+    ev.record(torch.cuda.current_stream(dev))
+    while not ev.query():
+        time.sleep(0.0005)
+    torch.cuda.synchronize(dev)
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -351,7 +363,7 @@ def run_ours(args, s0):
             flush(i)
         step(ev[i])
     t_end.record(stream)
-    torch.cuda.synchronize(dev)
+    drain(dev)
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
@@ -534,7 +546,7 @@ def run_decode(args, s):
         evs[i][0].record(stream)
         step()
         evs[i][1].record(stream)
-    torch.cuda.synchronize(dev)
+    drain(dev)
     clocks = sampler.stop()
     swa.check_device_status(stream)
     ms = sum(a.elapsed_time(b) for a, b in evs) / K
@@ -603,7 +615,7 @@ def run_backward(args, s):
         evs[i][0].record(stream)
         step()
         evs[i][1].record(stream)
-    torch.cuda.synchronize(dev)
+    drain(dev)
     clocks = sampler.stop()
     swa.check_device_status(stream)
     ms = sum(a.elapsed_time(b) for a, b in evs) / K
@@ -699,7 +711,7 @@ def run_forward_x(args, s):
         evs[i][0].record(stream)
         step()
         evs[i][1].record(stream)
-    torch.cuda.synchronize(dev)
+    drain(dev)
     clocks = sampler.stop()
     swa.check_device_status(stream)
     ms = sum(a.elapsed_time(b) for a, b in evs) / K
@@ -783,7 +795,7 @@ def run_sssl(args):
     for _ in range(K):
         step()
     e1.record(stream)
-    torch.cuda.synchronize(dev)
+    drain(dev)
     clocks = sampler.stop()
     swa.check_device_status(stream)
     ms = e0.elapsed_time(e1) / K
