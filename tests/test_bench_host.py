@@ -1,0 +1,42 @@
+"""Host-side checks of bench.py's arithmetic (no GPU): the algorithmic flop count of each workload
+against the GFLOP column of the baseline table (4 D flops per unmasked query-key pair, pairs
+W (W + 1) / 2 + (T - W) W per (b, h)), the SSSL stack totals, and the L2 note of each workload."""
+import pytest
+
+import bench
+import workloads
+
+
+@pytest.mark.parametrize("s,gflop", [
+    (workloads.TINY, 0.034),
+    (workloads.GPT2, 12.90),
+    (workloads.D24_S, 154.67),
+    (workloads.D24_L_VE, 206.26),
+], ids=["tiny", "gpt2_124m", "d24_S", "d24_L_VE"])
+def test_flops_match_the_baseline_table(s, gflop):
+    got = bench.flops_per_step(s) / 1e9
+    assert abs(got - gflop) <= 0.006 * gflop + 1e-3, (s.name, got, gflop)
+
+
+def test_unmasked_pairs_closed_form_and_brute_force():
+    # brute force over a small (b, h) slice: pairs (i, j) with 0 <= i - j < W
+    for T, W in ((7, 3), (16, 16), (130, 40), (257, 1)):
+        s = workloads.LayerShape(B=2, T=T, H=3, D=64, window=W, ve=False, seed=0, name="x")
+        brute = sum(1 for i in range(T) for j in range(T) if 0 <= i - j < min(W, T))
+        assert s.unmasked_pairs() == 2 * 3 * brute
+
+
+@pytest.mark.parametrize("T,tflop", [(1024, 2.01), (2048, 4.02), (4096, 8.04), (8192, 16.08), (16384, 32.16)])
+def test_sssl_stack_flops_match_the_baseline_table(T, tflop):
+    shapes = workloads.sssl_layer_shapes(32768 // T, T, 12, 128)
+    assert len(shapes) == 24
+    got = sum(bench.flops_per_step(s) for s in shapes) / 1e12
+    assert abs(got - tflop) <= 0.006 * tflop, (T, got, tflop)
+
+
+def test_l2_note_follows_the_input_size():
+    # d24 inputs (q, k, v, ve: 403 MB) exceed the 126 MB L2, the GPT-2 124M layer's (38 MB) do not
+    assert bench.input_bytes(workloads.D24_L_VE) > bench.L2_BYTES
+    assert bench.config_of(workloads.D24_L_VE, 1)["l2"].startswith("no flush")
+    assert bench.input_bytes(workloads.GPT2) < bench.L2_BYTES
+    assert "flushed between steps" in bench.config_of(workloads.GPT2, 1)["l2"]
