@@ -1,6 +1,7 @@
 """Host-side checks of bench.py's arithmetic (no GPU): the algorithmic flop count of each workload
-against the GFLOP column of the baseline table (4 D flops per unmasked query-key pair, pairs
-W (W + 1) / 2 + (T - W) W per (b, h)), the SSSL stack totals, and the L2 note of each workload."""
+(4 D flops per unmasked query-key pair, W (W + 1) / 2 + (T - W) W pairs per (b, h)) against the
+GFLOP each layer shape gives by hand, the 24-layer S,S,S,L stack totals, and the L2 note of each
+workload."""
 import pytest
 
 import bench
@@ -13,7 +14,7 @@ import workloads
     (workloads.D24_S, 154.67),
     (workloads.D24_L_VE, 206.26),
 ], ids=["tiny", "gpt2_124m", "d24_S", "d24_L_VE"])
-def test_flops_match_the_baseline_table(s, gflop):
+def test_flops_match_the_hand_counts(s, gflop):
     got = bench.flops_per_step(s) / 1e9
     assert abs(got - gflop) <= 0.006 * gflop + 1e-3, (s.name, got, gflop)
 
@@ -27,7 +28,7 @@ def test_unmasked_pairs_closed_form_and_brute_force():
 
 
 @pytest.mark.parametrize("T,tflop", [(1024, 2.01), (2048, 4.02), (4096, 8.04), (8192, 16.08), (16384, 32.16)])
-def test_sssl_stack_flops_match_the_baseline_table(T, tflop):
+def test_sssl_stack_flops_match_the_hand_counts(T, tflop):
     shapes = workloads.sssl_layer_shapes(32768 // T, T, 12, 128)
     assert len(shapes) == 24
     got = sum(bench.flops_per_step(s) for s in shapes) / 1e12
