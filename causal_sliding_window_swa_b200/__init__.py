@@ -403,6 +403,8 @@ def backward(q, k, v, out, lse, dout, window: int = 0, dlse=None, ve=None, gate_
     that produced out and lse, so the prologue is not recomputed (C call swa_attn_bwd_saved;
     multi-head, no document mask).  Raises SwaError on a nonzero status."""
     import torch
+    if saved and (workspace is None or doc is not None):
+        raise ValueError("saved=True needs the forward's workspace, Hkv == H and no document mask")
     B, T, H, Hkv, D = _check_qkv(q, k, v, ve, gate_x, Wg)
     for name, t in (("out", out), ("dout", dout)):
         if tuple(t.shape) != (B, T, H, D) or t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
@@ -424,7 +426,7 @@ def backward(q, k, v, out, lse, dout, window: int = 0, dlse=None, ve=None, gate_
                             or not doc.is_contiguous()):
         raise ValueError(f"doc must be a contiguous CUDA int32 tensor of shape {(B, T)}")
     if saved:
-        if Hkv != H or doc is not None or workspace is None:
+        if Hkv != H:
             raise ValueError("saved=True needs the forward's workspace, Hkv == H and no document mask")
         rc = swa_attn_bwd_saved(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(out), _ptr(lse),
                                 _ptr(dout), _ptr(dlse), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g.get("dve")),

@@ -189,6 +189,57 @@ def test_backward_workspace_and_validation():
     assert call(eps=-1.0) == swa.SWA_ERR_INVALID_ARG
 
 
+def test_saved_backward_and_document_backward_validation():
+    # swa_attn_bwd_saved takes the multi-head backward's arguments and checks them the same way;
+    # swa_attn_bwd_doc also wants a 4-byte aligned document-id array.
+    B, T, H, D = 2, 200, 4, 64
+    n0 = swa.swa_attn_bwd_workspace_bytes(B, T, H, H, D, 0)
+    base = dict(q=A, k=A, v=A, ve=None, gate_x=None, Wg=None, out=A, lse=A, dout=A, dlse=None, dq=A, dk=A,
+                dv=A, dve=None, dgate_x=None, dWg=None, B=B, T=T, H=H, D=D, window=0,
+                rope_base=1e4, eps=1e-6, workspace=A, ws_bytes=n0, stream=None)
+
+    def saved(**kw):
+        return swa.swa_attn_bwd_saved(*dict(base, **kw).values())
+    assert saved(dout=None) == swa.SWA_ERR_INVALID_ARG
+    assert saved(workspace=None) == swa.SWA_ERR_INVALID_ARG
+    assert saved(dve=A) == swa.SWA_ERR_INVALID_ARG
+    assert saved(dq=A + 8) == swa.SWA_ERR_MISALIGNED
+    assert saved(ws_bytes=n0 - 1) == swa.SWA_ERR_NO_MEMORY
+    assert saved(D=80) == swa.SWA_ERR_UNSUPPORTED
+    assert saved(rope_base=0.0) == swa.SWA_ERR_INVALID_ARG
+
+    def doc(**kw):
+        a = dict(base, **kw)
+        return swa._lib.swa_attn_bwd_doc(a["q"], a["k"], a["v"], a["ve"], a["gate_x"], a["Wg"], a.get("doc", A),
+                                         a["out"], a["lse"], a["dout"], a["dlse"], a["dq"], a["dk"], a["dv"],
+                                         a["dve"], a["dgate_x"], a["dWg"], a["B"], a["T"], a["H"], a.get("Hkv", H),
+                                         a["D"], a["window"], a["rope_base"], a["eps"], a["workspace"],
+                                         a["ws_bytes"], a["stream"])
+    assert doc(doc=A + 2) == swa.SWA_ERR_MISALIGNED
+    assert doc(Hkv=3) == swa.SWA_ERR_INVALID_ARG
+    assert doc(ws_bytes=n0 - 1) == swa.SWA_ERR_NO_MEMORY
+
+
+def test_document_decode_rejects_a_misaligned_id_array():
+    need = swa.swa_attn_decode_workspace_bytes(1, 16, 1, 64, 0, 0)
+
+    def call(doc, Hkv=1):
+        return swa._lib.swa_attn_decode_doc(A, A, A, None, None, None, A, A, 3, doc, A, A, 1, 16, 1, Hkv, 64, 0,
+                                            1e4, 1e-6, A, need, None)
+    assert call(A + 2) == swa.SWA_ERR_MISALIGNED
+    assert call(A, Hkv=2) == swa.SWA_ERR_INVALID_ARG
+
+
+def test_saved_backward_binding_wants_the_forward_workspace():
+    # the check runs before any tensor is looked at or any workspace is allocated
+    import torch
+    t = torch.zeros(1)
+    with pytest.raises(ValueError, match="saved=True"):
+        swa.backward(t, t, t, t, t, t, saved=True)
+    with pytest.raises(ValueError, match="saved=True"):
+        swa.backward(t, t, t, t, t, t, saved=True, workspace=t, doc=t)
+
+
 def test_fused_projection_workspace_and_validation():
     B, T, H, Hkv, D, C = 2, 100, 4, 2, 64, 256
     n = swa.swa_attn_fwd_x_workspace_bytes(B, T, H, Hkv, D)
