@@ -264,6 +264,26 @@ def _stream_handle(stream):
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
 
 
+def _want(name, t, shape, dtype, device=None):
+    """t must be a contiguous CUDA tensor of `shape` and `dtype` (on `device` when given): the C
+    calls take bare pointers and cannot check sizes, so a wrong tensor is refused here."""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, not {t.dtype}")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the layer's inputs on {device}")
+
+
+def _want_workspace(ws, device):
+    if not ws.is_cuda or not ws.is_contiguous() or ws.device != device:
+        raise ValueError(f"workspace must be a contiguous CUDA tensor on {device}")
+
+
 def _check_qkv(q, k, v, ve, gate_x, Wg):
     """Shapes of a layer call: q (B,T,H,D); k, v and ve (B,T,Hkv,D) with Hkv dividing H (Hkv == H
     for the multi-head layer); gate_x (B,T,32); Wg [32,Hkv].  Returns (B, T, H, Hkv, D)."""
@@ -289,6 +309,9 @@ def _check_qkv(q, k, v, ve, gate_x, Wg):
             raise ValueError(f"Wg must be a contiguous bf16 [32, {Hkv}] tensor")
     elif gate_x is not None or Wg is not None:
         raise ValueError("ve, gate_x and Wg go together")
+    for name, t in (("k", k), ("v", v), ("ve", ve), ("gate_x", gate_x), ("Wg", Wg)):
+        if t is not None and t.device != q.device:
+            raise ValueError(f"{name} is on {t.device}, q on {q.device}")
     return B, T, H, Hkv, D
 
 
@@ -304,83 +327,97 @@ def forward(q, k, v, window: int = 0, ve=None, gate_x=None, Wg=None, rope_base: 
     then visible only inside the query's document, a maximal run of equal ids."""
     import torch
     B, T, H, Hkv, D = _check_qkv(q, k, v, ve, gate_x, Wg)
+    dev = q.device
     if out is None:
         out = torch.empty_like(q)
+    _want("out", out, (B, T, H, D), torch.bfloat16, dev)
     if with_lse and lse is None:
-        lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
-    st = _stream_handle(stream)
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+    if lse is not None:
+        _want("lse", lse, (B, H, T), torch.float32, dev)
+    if workspace is not None:
+        _want_workspace(workspace, dev)
     if doc is not None:
-        if tuple(doc.shape) != (B, T) or doc.dtype != torch.int32 or not doc.is_cuda or not doc.is_contiguous():
-            raise ValueError(f"doc must be a contiguous CUDA int32 tensor of shape {(B, T)}")
+        _want("doc", doc, (B, T), torch.int32, dev)
         if workspace is not None:
             raise ValueError("the document-masked call uses the library workspace")
-        rc = swa_attn_fwd_doc(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(doc), _ptr(out),
-                              _ptr(lse), B, T, H, Hkv, D, int(window), float(rope_base), float(eps), st)
-        if rc != SWA_OK:
-            raise SwaError(rc, "swa_attn_fwd_doc")
-        return out, lse
-    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(out), _ptr(lse),
-            B, T, H, D, int(window), float(rope_base), float(eps))
-    if Hkv != H:
-        if workspace is not None:
-            raise ValueError("a caller workspace is supported for multi-head layers only")
-        rc = swa_attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(out),
-                              _ptr(lse), B, T, H, Hkv, D, int(window), float(rope_base), float(eps), st)
-        if rc != SWA_OK:
-            raise SwaError(rc, "swa_attn_fwd_gqa")
-        return out, lse
-    if workspace is None:
-        rc = swa_attn_fwd(*args, st)
-    else:
-        rc = swa_attn_fwd_ws(*args, _ptr(workspace), workspace.numel() * workspace.element_size(), st)
+    if Hkv != H and workspace is not None:
+        raise ValueError("a caller workspace is supported for multi-head layers only")
+    with torch.cuda.device(dev):
+        st = _stream_handle(stream)
+        if doc is not None:
+            rc = swa_attn_fwd_doc(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(doc),
+                                  _ptr(out), _ptr(lse), B, T, H, Hkv, D, int(window), float(rope_base), float(eps),
+                                  st)
+            name = "swa_attn_fwd_doc"
+        elif Hkv != H:
+            rc = swa_attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(out),
+                                  _ptr(lse), B, T, H, Hkv, D, int(window), float(rope_base), float(eps), st)
+            name = "swa_attn_fwd_gqa"
+        else:
+            args = (_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(out), _ptr(lse),
+                    B, T, H, D, int(window), float(rope_base), float(eps))
+            if workspace is None:
+                rc = swa_attn_fwd(*args, st)
+            else:
+                rc = swa_attn_fwd_ws(*args, _ptr(workspace), workspace.numel() * workspace.element_size(), st)
+            name = "swa_attn_fwd"
     if rc != SWA_OK:
-        raise SwaError(rc, "swa_attn_fwd")
+        raise SwaError(rc, name)
     return out, lse
 
 
 def decode(q, k, v, k_cache, v_cache, pos: int, window: int, ve=None, gate_x=None, Wg=None,
            rope_base: float = 1e4, eps: float = 1e-6, out=None, lse=None, workspace=None, stream=None,
            doc_start=None):
-    """One generation step (C call swa_attn_decode, or swa_attn_decode_gqa when k has fewer heads
-    than q) on torch tensors: q (B,H,D), k, v (B,Hkv,D) bf16 of the new token at position ``pos``;
-    k_cache, v_cache (B,Tmax,Hkv,D) bf16, updated in place at ``pos``.
+    """One generation step (C call swa_attn_decode_doc, which with no ``doc_start`` is
+    swa_attn_decode, or swa_attn_decode_gqa when k has fewer heads than q) on torch tensors:
+    q (B,H,D), k, v (B,Hkv,D) bf16 of the new token at position ``pos``; ve (B,Hkv,D), gate_x
+    (B,32), Wg [32,Hkv] on value-embedding layers; k_cache, v_cache (B,Tmax,Hkv,D) bf16, updated
+    in place at ``pos``.  Every tensor is checked against these shapes before the call.
     ``doc_start``: optional int32 CUDA tensor (B,) with the first position of each sequence's
     current document (C call swa_attn_decode_doc).
     Returns (out (B,H,D) bf16, lse (B,H) fp32).  Raises SwaError on a nonzero status."""
     import torch
+    if q.dim() != 3 or k.dim() != 3 or k_cache.dim() != 4:
+        raise ValueError("q must be (B, H, D), k and v (B, Hkv, D), the caches (B, Tmax, Hkv, D)")
     B, H, D = q.shape
     Hkv = k.shape[1]
     Tmax = k_cache.shape[1]
+    dev = q.device
+    bf = torch.bfloat16
+    _want("q", q, (B, H, D), bf)
+    for name, t in (("k", k), ("v", v)):
+        _want(name, t, (B, Hkv, D), bf, dev)
+    for name, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+        _want(name, t, (B, Tmax, Hkv, D), bf, dev)
+    if (ve is None) != (gate_x is None) or (ve is None) != (Wg is None):
+        raise ValueError("ve, gate_x and Wg go together")
+    if ve is not None:
+        _want("ve", ve, (B, Hkv, D), bf, dev)
+        _want("gate_x", gate_x, (B, 32), bf, dev)
+        _want("Wg", Wg, (32, Hkv), bf, dev)
     if out is None:
         out = torch.empty_like(q)
+    _want("out", out, (B, H, D), bf, dev)
     if lse is None:
-        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+        lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    _want("lse", lse, (B, H), torch.float32, dev)
     need = swa_attn_decode_workspace_bytes(B, Tmax, H, D, ve is not None, window)
     if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    st = _stream_handle(stream)
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _want_workspace(workspace, dev)
     if doc_start is not None:
-        if tuple(doc_start.shape) != (B,) or doc_start.dtype != torch.int32 or not doc_start.is_cuda:
-            raise ValueError(f"doc_start must be a CUDA int32 tensor of shape {(B,)}")
+        _want("doc_start", doc_start, (B,), torch.int32, dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        st = _stream_handle(stream)
         rc = _lib.swa_attn_decode_doc(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(k_cache),
                                       _ptr(v_cache), int(pos), _ptr(doc_start), _ptr(out), _ptr(lse), B, Tmax, H,
-                                      Hkv, D, int(window), float(rope_base), float(eps), _ptr(workspace),
-                                      workspace.numel() * workspace.element_size(), st)
-        if rc != SWA_OK:
-            raise SwaError(rc, "swa_attn_decode_doc")
-        return out, lse
-    if Hkv == H:
-        rc = swa_attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(k_cache),
-                             _ptr(v_cache), int(pos), _ptr(out), _ptr(lse), B, Tmax, H, D, int(window),
-                             float(rope_base), float(eps), _ptr(workspace),
-                             workspace.numel() * workspace.element_size(), st)
-    else:
-        rc = _lib.swa_attn_decode_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg),
-                                      _ptr(k_cache), _ptr(v_cache), int(pos), _ptr(out), _ptr(lse), B,
-                                      Tmax, H, Hkv, D, int(window), float(rope_base), float(eps),
-                                      _ptr(workspace), workspace.numel() * workspace.element_size(), st)
+                                      Hkv, D, int(window), float(rope_base), float(eps), _ptr(workspace), ws_bytes,
+                                      st)
     if rc != SWA_OK:
-        raise SwaError(rc, "swa_attn_decode")
+        raise SwaError(rc, "swa_attn_decode_doc" if doc_start is not None else "swa_attn_decode")
     return out, lse
 
 
@@ -406,14 +443,14 @@ def backward(q, k, v, out, lse, dout, window: int = 0, dlse=None, ve=None, gate_
     if saved and (workspace is None or doc is not None):
         raise ValueError("saved=True needs the forward's workspace, Hkv == H and no document mask")
     B, T, H, Hkv, D = _check_qkv(q, k, v, ve, gate_x, Wg)
+    dev = q.device
     for name, t in (("out", out), ("dout", dout)):
-        if tuple(t.shape) != (B, T, H, D) or t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {(B, T, H, D)}")
-    for name, t in (("lse", lse), ("dlse", dlse)):
-        if t is None and name == "dlse":
-            continue
-        if tuple(t.shape) != (B, H, T) or t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous CUDA fp32 tensor of shape {(B, H, T)}")
+        _want(name, t, (B, T, H, D), torch.bfloat16, dev)
+    _want("lse", lse, (B, H, T), torch.float32, dev)
+    if dlse is not None:
+        _want("dlse", dlse, (B, H, T), torch.float32, dev)
+    if workspace is not None:
+        _want_workspace(workspace, dev)
     g = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v))
     if ve is not None:
         g.update(dve=torch.empty_like(ve),
@@ -422,17 +459,22 @@ def backward(q, k, v, out, lse, dout, window: int = 0, dlse=None, ve=None, gate_
     need = swa_attn_bwd_workspace_bytes(B, T, H, Hkv, D, ve is not None)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    if doc is not None and (tuple(doc.shape) != (B, T) or doc.dtype != torch.int32 or not doc.is_cuda
-                            or not doc.is_contiguous()):
-        raise ValueError(f"doc must be a contiguous CUDA int32 tensor of shape {(B, T)}")
+    if doc is not None:
+        _want("doc", doc, (B, T), torch.int32, dev)
+    if saved and Hkv != H:
+        raise ValueError("saved=True needs the forward's workspace, Hkv == H and no document mask")
+    with torch.cuda.device(dev):
+        return _backward_call(q, k, v, ve, gate_x, Wg, doc, out, lse, dout, dlse, g, B, T, H, Hkv, D, window,
+                              rope_base, eps, workspace, _stream_handle(stream), saved)
+
+
+def _backward_call(q, k, v, ve, gate_x, Wg, doc, out, lse, dout, dlse, g, B, T, H, Hkv, D, window, rope_base,
+                   eps, workspace, st, saved):
     if saved:
-        if Hkv != H:
-            raise ValueError("saved=True needs the forward's workspace, Hkv == H and no document mask")
         rc = swa_attn_bwd_saved(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(out), _ptr(lse),
                                 _ptr(dout), _ptr(dlse), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g.get("dve")),
                                 _ptr(g.get("dgate_x")), _ptr(g.get("dWg")), B, T, H, D, int(window), float(rope_base),
-                                float(eps), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                _stream_handle(stream))
+                                float(eps), _ptr(workspace), workspace.numel() * workspace.element_size(), st)
         if rc != SWA_OK:
             raise SwaError(rc, "swa_attn_bwd_saved")
         return g
@@ -440,7 +482,7 @@ def backward(q, k, v, out, lse, dout, window: int = 0, dlse=None, ve=None, gate_
                           _ptr(lse), _ptr(dout), _ptr(dlse), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
                           _ptr(g.get("dve")), _ptr(g.get("dgate_x")), _ptr(g.get("dWg")), B, T, H, Hkv, D,
                           int(window), float(rope_base), float(eps), _ptr(workspace),
-                          workspace.numel() * workspace.element_size(), _stream_handle(stream))
+                          workspace.numel() * workspace.element_size(), st)
     if rc != SWA_OK:
         raise SwaError(rc, "swa_attn_bwd_doc" if doc is not None else "swa_attn_bwd_gqa")
     return g
@@ -448,19 +490,17 @@ def backward(q, k, v, out, lse, dout, window: int = 0, dlse=None, ve=None, gate_
 
 def _check_x_w(x, Wqkv, H, Hkv, D, ve, Wg):
     import torch
-    if x.dim() != 3 or x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous():
-        raise ValueError("x must be a contiguous CUDA bf16 (B, T, C) tensor")
+    if x.dim() != 3:
+        raise ValueError("x must be a (B, T, C) tensor")
     B, T, C = x.shape
     N = (H + 2 * Hkv) * D
-    if tuple(Wqkv.shape) != (N, C) or Wqkv.dtype != torch.bfloat16 or not Wqkv.is_contiguous():
-        raise ValueError(f"Wqkv must be a contiguous bf16 [{N}, {C}] tensor")
+    _want("x", x, (B, T, C), torch.bfloat16)
+    _want("Wqkv", Wqkv, (N, C), torch.bfloat16, x.device)
     if (ve is None) != (Wg is None):
         raise ValueError("ve and Wg go together")
     if ve is not None:
-        if tuple(ve.shape) != (B, T, Hkv, D) or ve.dtype != torch.bfloat16 or not ve.is_contiguous():
-            raise ValueError(f"ve must be a contiguous bf16 {(B, T, Hkv, D)} tensor")
-        if tuple(Wg.shape) != (32, Hkv) or Wg.dtype != torch.bfloat16 or not Wg.is_contiguous():
-            raise ValueError(f"Wg must be a contiguous bf16 [32, {Hkv}] tensor")
+        _want("ve", ve, (B, T, Hkv, D), torch.bfloat16, x.device)
+        _want("Wg", Wg, (32, Hkv), torch.bfloat16, x.device)
     return B, T, C
 
 
@@ -475,8 +515,9 @@ def qkv_prologue(x, Wqkv, H: int, Hkv: int, D: int, ve=None, Wg=None, rope_base:
     vp = torch.empty((B, T, Hkv, D), dtype=torch.bfloat16, device=x.device)
     need = swa_attn_fwd_x_workspace_bytes(B, T, H, Hkv, D)
     ws = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
-    rc = swa_attn_qkv_prologue(_ptr(x), _ptr(Wqkv), _ptr(ve), _ptr(Wg), _ptr(qh), _ptr(kh), _ptr(vp), B, T, C, H,
-                               Hkv, D, float(rope_base), float(eps), _ptr(ws), need, _stream_handle(stream))
+    with torch.cuda.device(x.device):
+        rc = swa_attn_qkv_prologue(_ptr(x), _ptr(Wqkv), _ptr(ve), _ptr(Wg), _ptr(qh), _ptr(kh), _ptr(vp), B, T, C,
+                                   H, Hkv, D, float(rope_base), float(eps), _ptr(ws), need, _stream_handle(stream))
     if rc != SWA_OK:
         raise SwaError(rc, "swa_attn_qkv_prologue")
     return qh, kh, vp
@@ -493,9 +534,11 @@ def forward_x(x, Wqkv, H: int, Hkv: int, D: int, window: int = 0, ve=None, Wg=No
     need = swa_attn_fwd_x_workspace_bytes(B, T, H, Hkv, D)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
-    rc = swa_attn_fwd_x(_ptr(x), _ptr(Wqkv), _ptr(ve), _ptr(Wg), _ptr(out), _ptr(lse), B, T, C, H, Hkv, D,
-                        int(window), float(rope_base), float(eps), _ptr(workspace),
-                        workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _want_workspace(workspace, x.device)
+    with torch.cuda.device(x.device):
+        rc = swa_attn_fwd_x(_ptr(x), _ptr(Wqkv), _ptr(ve), _ptr(Wg), _ptr(out), _ptr(lse), B, T, C, H, Hkv, D,
+                            int(window), float(rope_base), float(eps), _ptr(workspace),
+                            workspace.numel() * workspace.element_size(), _stream_handle(stream))
     if rc != SWA_OK:
         raise SwaError(rc, "swa_attn_fwd_x")
     return out, lse

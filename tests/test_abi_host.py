@@ -280,3 +280,19 @@ def test_header_is_plain_c():
                         "-I", os.path.join(ROOT, "include"), "-x", "c", "-"], input=src, capture_output=True,
                        text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_binding_tensor_checks():
+    # the helper the tensor-level calls use before handing bare pointers to the C calls
+    import torch
+    t = torch.zeros((2, 3), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="out is required"):
+        swa._want("out", None, (2, 3), torch.bfloat16)
+    with pytest.raises(ValueError, match=r"shape \(2, 4\), not \(2, 3\)"):
+        swa._want("out", t, (2, 4), torch.bfloat16)
+    with pytest.raises(ValueError, match="must be torch.float32"):
+        swa._want("lse", t, (2, 3), torch.float32)
+    with pytest.raises(ValueError, match="contiguous CUDA"):
+        swa._want("out", t, (2, 3), torch.bfloat16)
+    with pytest.raises(ValueError, match="workspace"):
+        swa._want_workspace(torch.zeros(16, dtype=torch.uint8), torch.device("cpu"))
