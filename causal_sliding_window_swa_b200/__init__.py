@@ -14,6 +14,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+import threading
 from typing import Optional, Tuple
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -104,13 +105,17 @@ def _load() -> ctypes.CDLL:
 
 
 _lib_handle: Optional[ctypes.CDLL] = None
+_lib_lock = threading.Lock()
 
 
 def load() -> ctypes.CDLL:
-    """Load libswa_attn.so (once); raises ImportError/OSError if it is missing or stale."""
+    """Load libswa_attn.so (once, also when several threads make their first call together);
+    raises ImportError/OSError if it is missing or stale."""
     global _lib_handle
     if _lib_handle is None:
-        _lib_handle = _load()
+        with _lib_lock:
+            if _lib_handle is None:
+                _lib_handle = _load()
     return _lib_handle
 
 

@@ -159,65 +159,74 @@ bool set_qkv_smem() {
            cudaFuncSetAttribute(swa::qkv_gemm_kernel<64, 128, false>, a, swa::QkvCfg<128>::SMEM_TOTAL) == cudaSuccess;
 }
 
+// Device `dev` must be compute capability 10.0; its SM count goes to g_num_sms[dev].  On such a
+// device, raises the dynamic shared memory limit of every kernel that uses more than 48 KB.
+// Returns 1 (ready), 2 (not sm_100) or a negative status.
+int check_device(int dev) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return SWA_ERR_CUDA;
+    }
+    if (major != 10 || minor != 0) return 2;
+    const int smem_attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
+    if (cudaFuncSetAttribute(swa::attn_fwd_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             swa::FwdCfg<64>::SMEM_TOTAL) != cudaSuccess ||
+        cudaFuncSetAttribute(swa::attn_fwd_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             swa::FwdCfg<128>::SMEM_TOTAL) != cudaSuccess ||
+        cudaFuncSetAttribute(swa::attn_fwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             swa::FwdCfg<64>::SMEM_TOTAL) != cudaSuccess ||
+        cudaFuncSetAttribute(swa::attn_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             swa::FwdCfg<128>::SMEM_TOTAL) != cudaSuccess ||
+        cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<64>, (cudaFuncAttribute)smem_attr,
+                             swa::BwdCfg<64>::DQ_SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<128>, (cudaFuncAttribute)smem_attr,
+                             swa::BwdCfg<128>::DQ_SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<64>, (cudaFuncAttribute)smem_attr,
+                             swa::BwdCfg<64>::KV_SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<128>, (cudaFuncAttribute)smem_attr,
+                             swa::BwdCfg<128>::KV_SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<64, true>, (cudaFuncAttribute)smem_attr,
+                             swa::BwdCfg<64>::DQ_SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<128, true>, (cudaFuncAttribute)smem_attr,
+                             swa::BwdCfg<128>::DQ_SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<64, true>, (cudaFuncAttribute)smem_attr,
+                             swa::BwdCfg<64>::KV_SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<128, true>, (cudaFuncAttribute)smem_attr,
+                             swa::BwdCfg<128>::KV_SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(swa::decode_attn_kernel<64>, (cudaFuncAttribute)smem_attr,
+                             swa::DecCfg<64>::SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(swa::decode_attn_kernel<128>, (cudaFuncAttribute)smem_attr,
+                             swa::DecCfg<128>::SMEM) != cudaSuccess) {
+        cudaGetLastError();
+        return SWA_ERR_CUDA;
+    }
+    return 1;
+}
+
+// Per-device state of device_ready: 0 not yet checked, 1 ready, 2 unsupported.  The first call
+// on a device checks it under g_dev_mu; g_num_sms[dev] is written before the state is published.
+std::mutex g_dev_mu;
+std::atomic<int> g_dev_state[64];
+
 int device_ready(int* dev_out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();
         return SWA_ERR_NO_DEVICE;
     }
-    static int checked[64] = {0};   // 0 unknown, 1 ok, 2 unsupported
     if (dev < 0 || dev >= 64) return SWA_ERR_UNSUPPORTED;
-    if (checked[dev] == 0) {
-        int major = 0, minor = 0;
-        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
-            cudaGetLastError();
-            return SWA_ERR_CUDA;
-        }
-        checked[dev] = (major == 10 && minor == 0) ? 1 : 2;
-        if (cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-            cudaGetLastError();
-            checked[dev] = 0;
-            return SWA_ERR_CUDA;
-        }
-        if (checked[dev] == 1) {
-            const int smem_attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
-            if (cudaFuncSetAttribute(swa::attn_fwd_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     swa::FwdCfg<64>::SMEM_TOTAL) != cudaSuccess ||
-                cudaFuncSetAttribute(swa::attn_fwd_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     swa::FwdCfg<128>::SMEM_TOTAL) != cudaSuccess ||
-                cudaFuncSetAttribute(swa::attn_fwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     swa::FwdCfg<64>::SMEM_TOTAL) != cudaSuccess ||
-                cudaFuncSetAttribute(swa::attn_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     swa::FwdCfg<128>::SMEM_TOTAL) != cudaSuccess ||
-                cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<64>, (cudaFuncAttribute)smem_attr,
-                                     swa::BwdCfg<64>::DQ_SMEM) != cudaSuccess ||
-                cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<128>, (cudaFuncAttribute)smem_attr,
-                                     swa::BwdCfg<128>::DQ_SMEM) != cudaSuccess ||
-                cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<64>, (cudaFuncAttribute)smem_attr,
-                                     swa::BwdCfg<64>::KV_SMEM) != cudaSuccess ||
-                cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<128>, (cudaFuncAttribute)smem_attr,
-                                     swa::BwdCfg<128>::KV_SMEM) != cudaSuccess ||
-                cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<64, true>, (cudaFuncAttribute)smem_attr,
-                                     swa::BwdCfg<64>::DQ_SMEM) != cudaSuccess ||
-                cudaFuncSetAttribute(swa::attn_bwd_dq_kernel<128, true>, (cudaFuncAttribute)smem_attr,
-                                     swa::BwdCfg<128>::DQ_SMEM) != cudaSuccess ||
-                cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<64, true>, (cudaFuncAttribute)smem_attr,
-                                     swa::BwdCfg<64>::KV_SMEM) != cudaSuccess ||
-                cudaFuncSetAttribute(swa::attn_bwd_dkv_kernel<128, true>, (cudaFuncAttribute)smem_attr,
-                                     swa::BwdCfg<128>::KV_SMEM) != cudaSuccess ||
-                cudaFuncSetAttribute(swa::decode_attn_kernel<64>, (cudaFuncAttribute)smem_attr,
-                                     swa::DecCfg<64>::SMEM) != cudaSuccess ||
-                cudaFuncSetAttribute(swa::decode_attn_kernel<128>, (cudaFuncAttribute)smem_attr,
-                                     swa::DecCfg<128>::SMEM) != cudaSuccess) {
-                cudaGetLastError();
-                checked[dev] = 0;
-                return SWA_ERR_CUDA;
-            }
-        }
+    int state = g_dev_state[dev].load(std::memory_order_acquire);
+    if (state == 0) {
+        std::lock_guard<std::mutex> lk(g_dev_mu);
+        state = g_dev_state[dev].load(std::memory_order_relaxed);
+        if (state == 0 && (state = check_device(dev)) < 0) return state;
+        g_dev_state[dev].store(state, std::memory_order_release);
     }
     *dev_out = dev;
-    return checked[dev] == 1 ? SWA_OK : SWA_ERR_UNSUPPORTED;
+    return state == 1 ? SWA_OK : SWA_ERR_UNSUPPORTED;
 }
 
 // ---------------------------------------------------------------------- TMA descriptors
@@ -919,18 +928,19 @@ int launch_decode_attention_d(int dev, const void* q, const void* k_cache, const
     CUtensorMap tk, tv;
     if (!make_cache_map(&tk, k_cache, B, Tmax, Hkv, D, C::KB) || !make_cache_map(&tv, v_cache, B, Tmax, Hkv, D, C::KB))
         return SWA_ERR_CUDA;
-    static int per_sm[64] = {0};
-    if (per_sm[dev] == 0) {
-        int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, swa::decode_attn_kernel<D>, C::THREADS, C::SMEM) !=
-                cudaSuccess || n < 1) {
+    // resident CTAs per SM, found once per device (threads that race here store the same value)
+    static std::atomic<int> per_sm[64];
+    int n_per_sm = per_sm[dev].load(std::memory_order_relaxed);
+    if (n_per_sm == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n_per_sm, swa::decode_attn_kernel<D>, C::THREADS,
+                                                          C::SMEM) != cudaSuccess || n_per_sm < 1) {
             cudaGetLastError();
-            n = 1;
+            n_per_sm = 1;
         }
-        per_sm[dev] = n;
+        per_sm[dev].store(n_per_sm, std::memory_order_relaxed);
     }
     const long long rows = (long long)B * H;
-    const long long slots = (long long)per_sm[dev] * g_num_sms[dev];
+    const long long slots = (long long)n_per_sm * g_num_sms[dev];
     const int n_tiles = (n_keys + C::KB - 1) / C::KB;
     int n_chunks = (int)std::max<long long>(1, std::min<long long>(slots / rows, swa::kDecodeMaxCluster));
     n_chunks = std::min(n_chunks, n_tiles);

@@ -1,6 +1,10 @@
 """The tensor-level calls refuse tensors whose shape, dtype or device does not match the layer
 before any C call: the C ABI takes bare pointers and could not see the mistake, which would turn
 into writes outside the caller's buffers.  No kernel is launched here."""
+import os
+import subprocess
+import sys
+
 import pytest
 import torch
 
@@ -75,3 +79,37 @@ def test_fused_projection_refuses_wrong_weights():
         swa.forward_x(x, W.cpu(), H, H, D)
     with pytest.raises(ValueError, match="workspace"):
         swa.forward_x(x, W, H, H, D, workspace=torch.empty(1 << 20, dtype=torch.uint8))
+
+
+def test_first_calls_from_several_threads():
+    # A fresh process whose first library calls come from four threads at once, each on its own
+    # stream: the lazy load, the per-device checks and the shared workspace are set up once and
+    # every thread gets the serial result bit for bit.
+    code = """
+import threading, torch
+import causal_sliding_window_swa_b200 as swa
+torch.cuda.set_device(0)
+g = torch.Generator().manual_seed(1)
+q, k, v = (torch.randn(2, 300, 2, 64, generator=g).to(torch.bfloat16).cuda() for _ in range(3))
+torch.cuda.synchronize()
+res = [None] * 4
+go = threading.Barrier(4)
+def run(i):
+    torch.cuda.set_device(0)
+    s = torch.cuda.Stream()
+    go.wait()
+    with torch.cuda.stream(s):
+        res[i] = swa.forward(q, k, v, 100)
+    s.synchronize()
+ts = [threading.Thread(target=run, args=(i,)) for i in range(4)]
+[t.start() for t in ts]
+[t.join() for t in ts]
+ref = swa.forward(q, k, v, 100)
+torch.cuda.synchronize()
+swa.check_device_status()
+assert all(torch.equal(r[0], ref[0]) and torch.equal(r[1], ref[1]) for r in res)
+print("threads ok")
+"""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and "threads ok" in r.stdout, r.stdout + r.stderr
