@@ -31,6 +31,11 @@
  * Streams: calls are asynchronous on `stream` (NULL = the legacy default stream) and never
  * synchronise the host, except swa_attn_last_device_status().
  *
+ * Threads: calls may come from several host threads at once.  The per-device setup of the first
+ * call, the library-owned workspace and the backward's side stream are guarded by locks, and a
+ * call that reuses the library workspace on another stream first waits, on the device, for the
+ * previous call that used it.  Caller-owned workspaces are the caller's to keep apart.
+ *
  * Precision: every qhat, khat and v' element the prologue writes is the correctly rounded bf16
  * (nearest, ties to even) of its exact value, so the tensor-core operands do not depend on how the
  * arithmetic is organised.
