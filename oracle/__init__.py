@@ -5,15 +5,17 @@ TEST INFRASTRUCTURE.  Only the tests, ``__graft_entry__.smoke()`` and the CPU-ba
 ``bench.py`` may import this package.  It shares no code with the CUDA library and never
 imports it.
 
-Two independent implementations live here:
+Two independent implementations live here.  The C oracle (``swa_oracle.c``, fp64, one query
+row at a time) backs the functions of this module:
 
-* ``forward`` / ``prologue``: the C oracle (``swa_oracle.c``), one query row at a time, fp64.
+* ``forward`` / ``prologue``: the layer and its prologue.
 * ``qkv_prologue``: the bias-free q, k, v projection of the layer input x followed by the same
   prologue (the fused projection).
 * ``backward``: the gradient of the same layer (chain rule through the five steps in
-  reverse), also in ``swa_oracle.c``; ``backward_rows`` gives the same values at sampled rows.
-* ``brute.py``: a NumPy fp64 restatement that materialises the full T x T score matrix, used
-  as the brute-force pin of the C oracle on small shapes.
+  reverse); ``backward_rows`` gives the same values at sampled rows.
+
+``brute.py`` is the second: a NumPy fp64 restatement that materialises the full T x T score
+matrix, used as the brute-force pin of the C oracle on small shapes.
 
 Each function cites the passage of the pages it follows in ``swa_oracle.c``'s header.
 Readings taken where the pages are silent (pair layout and sign of RoPE, window boundary,
