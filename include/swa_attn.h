@@ -88,7 +88,9 @@ typedef enum swa_status {
  * B, T, H      >= 1;  D in {64, 128};  B*T*H*D < 2^31.
  * window       keys visible to a query, counting itself; <= 0 or >= T is full causal.
  * rope_base    > 0 and finite (10000 in the pages' models).
- * eps          >= 0 and finite (1e-6 here).
+ * eps          >= 0 and finite (1e-6 here).  At eps = 0 an all-zero q or k head row has no
+ *              normalised value (0/0 in the definition): such inputs are outside the domain and
+ *              their results are unspecified.
  * stream       CUDA stream (NULL = legacy default stream).
  *
  * Scratch: the library keeps one workspace per device (qhat, khat, v', the gates, the RoPE table),
