@@ -41,3 +41,44 @@ def test_l2_note_follows_the_input_size():
     assert bench.config_of(workloads.D24_L_VE, 1)["l2"].startswith("no flush")
     assert bench.input_bytes(workloads.GPT2) < bench.L2_BYTES
     assert "flushed between steps" in bench.config_of(workloads.GPT2, 1)["l2"]
+
+
+def _fake_nvml(clocks, reasons_attr, bits):
+    import itertools
+    import types
+    seq = itertools.cycle(clocks)
+    nv = types.SimpleNamespace(NVML_CLOCK_SM=1, nvmlInit=lambda: None,
+                               nvmlDeviceGetHandleByIndex=lambda i: ("gpu", i),
+                               nvmlDeviceGetMaxClockInfo=lambda h, c: 1965,
+                               nvmlDeviceGetClockInfo=lambda h, c: next(seq))
+    setattr(nv, reasons_attr, lambda h: bits)
+    return nv
+
+
+@pytest.mark.parametrize("reasons_attr", ["nvmlDeviceGetCurrentClocksEventReasons",
+                                          "nvmlDeviceGetCurrentClocksThrottleReasons"])
+def test_clock_sampler_reads_clocks_and_reasons(monkeypatch, reasons_attr):
+    # NVML faked on the host: clocks cycle 1965 / 1965 / 1800 MHz, reasons gpu_idle + sw_power_cap
+    # + hw_slowdown; gpu_idle is not a throttle and is dropped, the rest are named.
+    import sys
+    import time
+    monkeypatch.setitem(sys.modules, "pynvml", _fake_nvml([1965, 1965, 1800], reasons_attr, 0x1 | 0x4 | 0x8))
+    s = bench.ClockSampler(0, period_s=0.001).start()
+    assert s.ok
+    time.sleep(0.05)
+    r = s.stop()
+    assert r["sm_max_mhz"] == 1965 and r["samples"] >= 3
+    assert r["sm_mhz"] == 1965                      # the median of a 2:1 mix
+    assert r["reasons"] == ["hw_slowdown", "sw_power_cap"]
+
+
+def test_clock_sampler_without_nvml(monkeypatch):
+    import sys
+    import types
+
+    def fail():
+        raise RuntimeError("no NVML")
+    monkeypatch.setitem(sys.modules, "pynvml", types.SimpleNamespace(nvmlInit=fail))
+    s = bench.ClockSampler(0).start()
+    assert not s.ok
+    assert s.stop() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
