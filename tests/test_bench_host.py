@@ -82,3 +82,16 @@ def test_clock_sampler_without_nvml(monkeypatch):
     s = bench.ClockSampler(0).start()
     assert not s.ok
     assert s.stop() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+
+def test_recorded_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
+    # the committed ncu traffic is reported only for the kernel source it was captured on
+    import json
+    f = tmp_path / "traffic.json"
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    assert bench.recorded_traffic("d24_L_VE") is None                      # no file
+    f.write_text(json.dumps({"d24_L_VE": {"kernel_sha256": bench.kernel_hash(), "dram_bytes_per_launch": 123}}))
+    assert bench.recorded_traffic("d24_L_VE") == 123
+    assert bench.recorded_traffic("gpt2_124m") is None                     # another workload
+    f.write_text(json.dumps({"d24_L_VE": {"kernel_sha256": "0" * 64, "dram_bytes_per_launch": 123}}))
+    assert bench.recorded_traffic("d24_L_VE") is None                      # the kernel changed since
