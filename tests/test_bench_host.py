@@ -95,3 +95,54 @@ def test_recorded_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
     assert bench.recorded_traffic("gpt2_124m") is None                     # another workload
     f.write_text(json.dumps({"d24_L_VE": {"kernel_sha256": "0" * 64, "dram_bytes_per_launch": 123}}))
     assert bench.recorded_traffic("d24_L_VE") is None                      # the kernel changed since
+
+
+def _bench(*argv, env=None):
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    e = dict(os.environ)
+    e.update(env or {})
+    return subprocess.run([sys.executable, os.path.join(root, "bench.py"), *argv], cwd=root, env=e,
+                          capture_output=True, text=True, timeout=600)
+
+
+def test_reference_arm_line():
+    # The reference arm is the oracle on the host cores, so it runs here: one JSON line with the
+    # GPU arm's metric, unit and workload, impl "reference", its CPU sample, and an e2e entry
+    # without device copies.
+    import json
+    r = _bench("--impl", "reference", "--steps", "1", "--warmup", "3")
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["higher_is_better"] is True
+    assert line["metric"].startswith("attention fwd TFLOP/s") and line["n_gpus"] == 1
+    assert line["config"]["workload"] == "d24 L+VE (16,2048,12,128) W=2048"
+    assert line["steps"] == 1 and line["warmup"] == 3 and line["value"] > 0
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    r = _bench("--impl", "reference", "--steps", "1", "--warmup", "3", "--gpus", "2",
+               env=dict(RANK="1", WORLD_SIZE="2", LOCAL_RANK="1"))
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_bench_refuses_short_warmup():
+    r = _bench("--steps", "1", "--warmup", "2")
+    assert r.returncode != 0 and "--warmup must be >= 3" in r.stderr
+
+
+def test_gpu_arm_without_a_device_fails_loudly():
+    # no CPU path: without CUDA the product arm exits non-zero and prints no result line
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is visible")
+    r = _bench("--steps", "1", "--warmup", "3")
+    assert r.returncode != 0 and "{" not in r.stdout and "needs a CUDA device" in r.stderr
