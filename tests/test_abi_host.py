@@ -296,3 +296,51 @@ def test_binding_tensor_checks():
         swa._want("out", t, (2, 3), torch.bfloat16)
     with pytest.raises(ValueError, match="workspace"):
         swa._want_workspace(torch.zeros(16, dtype=torch.uint8), torch.device("cpu"))
+
+
+def test_c_program_links_and_calls_the_library(tmp_path):
+    """A plain C99 program includes the header, links libswa_attn.so and calls it: the version,
+    strerror, the workspace size, arguments refused before any device work, and (on a machine
+    without a GPU) a valid call that reports SWA_ERR_NO_DEVICE instead of computing anything."""
+    import shutil
+    import subprocess
+    import torch
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no gcc")
+    lib_dir = os.path.dirname(swa.LIB_PATH)
+    no_gpu = int(not torch.cuda.is_available())
+    src = tmp_path / "use_swa.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <stdint.h>
+#include "swa_attn.h"
+
+int main(void) {
+    void* a = (void*)(uintptr_t)0x7f0000000000ull;   /* aligned, never dereferenced */
+    float* l = (float*)a;
+    if (swa_attn_version() < 100) return 1;
+    if (swa_attn_workspace_bytes(1, 16, 1, 96, 0) != 0) return 2;
+    if (swa_attn_workspace_bytes(1, 16, 1, 64, 0) == 0) return 3;
+    if (swa_attn_fwd(a, a, a, NULL, NULL, NULL, a, l, 0, 16, 1, 64, 0, 1e4f, 1e-6f, NULL) != SWA_ERR_INVALID_ARG)
+        return 4;
+    if (swa_attn_fwd(a, a, a, NULL, NULL, NULL, a, l, 1, 16, 1, 96, 0, 1e4f, 1e-6f, NULL) != SWA_ERR_UNSUPPORTED)
+        return 5;
+    if (swa_attn_fwd((char*)a + 2, a, a, NULL, NULL, NULL, a, l, 1, 16, 1, 64, 0, 1e4f, 1e-6f, NULL) !=
+        SWA_ERR_MISALIGNED)
+        return 6;
+    if (NO_GPU && swa_attn_fwd(a, a, a, NULL, NULL, NULL, a, l, 1, 16, 1, 64, 0, 1e4f, 1e-6f, NULL) !=
+        SWA_ERR_NO_DEVICE)
+        return 7;
+    printf("%s\n", swa_attn_strerror(SWA_ERR_MISALIGNED));
+    return 0;
+}
+''')
+    exe = tmp_path / "use_swa"
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", f"-DNO_GPU={no_gpu}", "-I",
+                        os.path.join(ROOT, "include"), str(src), "-L", lib_dir, "-lswa_attn",
+                        f"-Wl,-rpath,{lib_dir}", "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0, (run.returncode, run.stderr)
+    assert run.stdout.strip() == swa.swa_attn_strerror(swa.SWA_ERR_MISALIGNED)
