@@ -344,3 +344,21 @@ int main(void) {
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert run.returncode == 0, (run.returncode, run.stderr)
     assert run.stdout.strip() == swa.swa_attn_strerror(swa.SWA_ERR_MISALIGNED)
+
+
+def test_readme_usage_matches_the_binding():
+    # every call in the README's usage block binds to the binding's signature (names, order and
+    # keywords), so the documented API cannot drift from the code
+    import ast
+    import inspect
+    txt = open(os.path.join(ROOT, "README.md")).read()
+    block = txt.split("```python", 1)[1].split("```", 1)[0]
+    calls = [n for n in ast.walk(ast.parse(block)) if isinstance(n, ast.Call)
+             and isinstance(n.func, ast.Attribute) and isinstance(n.func.value, ast.Name) and n.func.value.id == "swa"]
+    assert len(calls) >= 8
+    for c in calls:
+        fn = getattr(swa, c.func.attr)
+        sig = inspect.signature(fn)
+        args = [object()] * len(c.args)
+        kwargs = {k.arg: object() for k in c.keywords}
+        sig.bind(*args, **kwargs)      # raises TypeError on a mismatch
