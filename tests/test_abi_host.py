@@ -362,3 +362,47 @@ def test_readme_usage_matches_the_binding():
         args = [object()] * len(c.args)
         kwargs = {k.arg: object() for k in c.keywords}
         sig.bind(*args, **kwargs)      # raises TypeError on a mismatch
+
+
+def _prototypes():
+    """name -> list of parameter type strings, from the SWA_API declarations of include/*.h."""
+    protos = {}
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if not f.endswith(".h"):
+            continue
+        txt = re.sub(r"/\*.*?\*/", "", open(os.path.join(inc, f)).read(), flags=re.S)
+        for m in re.finditer(r"SWA_API\s+[\w\s\*]+?\b(swa_\w+)\s*\(([^)]*)\)\s*;", txt):
+            params = [p.strip() for p in m.group(2).split(",")]
+            protos[m.group(1)] = [] if params == ["void"] else params
+    return protos
+
+
+def _ctype_of(param: str):
+    p = re.sub(r"\b(const|restrict)\b", " ", param)
+    if "*" in p or re.search(r"\bswa_stream_t\b", p):
+        return "pointer"
+    for key, name in (("size_t", "size_t"), ("unsigned", "uint"), ("double", "double"), ("float", "float"),
+                      ("int", "int")):
+        if re.search(rf"\b{key}\b", p):
+            return name
+    raise AssertionError(f"unmapped C parameter type: {param!r}")
+
+
+def test_binding_argtypes_match_the_header():
+    # the ctypes signature of every entry point the binding declares has the header's arity and
+    # parameter kinds, so no call can pass an argument in the wrong slot or width
+    lib = swa.load()
+    kinds = {ctypes.c_int: "int", ctypes.c_uint: "uint", ctypes.c_float: "float", ctypes.c_double: "double",
+             ctypes.c_size_t: "size_t", ctypes.c_void_p: "pointer", ctypes.c_char_p: "pointer"}
+    checked = 0
+    for name, params in _prototypes().items():
+        fn = getattr(lib, name)
+        if fn.argtypes is None:
+            continue
+        assert len(fn.argtypes) == len(params), (name, len(fn.argtypes), len(params))
+        for t, p in zip(fn.argtypes, params):
+            got = kinds.get(t, "pointer" if issubclass(t, (ctypes._Pointer, ctypes.c_void_p)) else repr(t))
+            assert got == _ctype_of(p), (name, p, t)
+        checked += 1
+    assert checked == len(_prototypes()) >= 28      # every declared entry point has argtypes
