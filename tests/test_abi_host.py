@@ -406,3 +406,20 @@ def test_binding_argtypes_match_the_header():
             assert got == _ctype_of(p), (name, p, t)
         checked += 1
     assert checked == len(_prototypes()) >= 28      # every declared entry point has argtypes
+
+
+def test_binding_restypes_match_the_header():
+    lib = swa.load()
+    inc = os.path.join(ROOT, "include")
+    want = {"int": ctypes.c_int, "size_t": ctypes.c_size_t, "const char*": ctypes.c_char_p}
+    n = 0
+    for f in os.listdir(inc):
+        if not f.endswith(".h"):
+            continue
+        txt = re.sub(r"/\*.*?\*/", "", open(os.path.join(inc, f)).read(), flags=re.S)
+        for m in re.finditer(r"SWA_API\s+([\w\s\*]+?)\s*\b(swa_\w+)\s*\(", txt):
+            ret = re.sub(r"\s+", " ", m.group(1)).replace(" *", "*").strip()
+            assert ret in want, (m.group(2), ret)
+            assert getattr(lib, m.group(2)).restype is want[ret], (m.group(2), ret)
+            n += 1
+    assert n >= 28
