@@ -42,22 +42,41 @@ def _runtime(name):
     return p if os.path.isabs(p) and os.path.exists(p) else None
 
 
-@pytest.mark.parametrize("kind", ["address", "undefined"])
-def test_oracle_pins_under_a_sanitizer(kind):
+# A one-element heap overflow planted in the row buffer of the attention step: the address
+# sanitizer run must report it (the check is not vacuous).
+OVERFLOW = ("            double* o = (double*)malloc(sizeof(double) * (size_t)D);",
+            "            double* o = (double*)malloc(sizeof(double) * (size_t)(D - 1));")
+
+
+def _run_pins(kind, src_text):
     rt = _runtime("libasan.so" if kind == "address" else "libubsan.so")
     if rt is None:
         pytest.skip(f"no {kind} sanitizer runtime")
     scratch = os.path.join(ROOT, ".pytest_cache", "sanitized")
     os.makedirs(scratch, exist_ok=True)
     with tempfile.TemporaryDirectory(dir=scratch) as tmp:
+        c = os.path.join(tmp, "oracle_san.c")
         so = os.path.join(tmp, "liboracle_san.so")
+        open(c, "w").write(src_text)
         flags = ["-fsanitize=address", "-fno-omit-frame-pointer"] if kind == "address" else \
             ["-fsanitize=undefined,bounds", "-fno-sanitize-recover=all"]
         subprocess.run(["gcc", "-O1", "-g", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fPIC", "-shared",
-                        *flags, "-o", so, obuild.SRC, "-lm"], check=True)
+                        *flags, "-o", so, c, "-lm"], check=True)
         env = dict(os.environ, ASAN_OPTIONS="detect_leaks=0")
         # the runtime goes first; libstdc++ with it, so the sanitizer finds the C++ runtime it wraps
         env["LD_PRELOAD"] = " ".join(p for p in (rt, _runtime("libstdc++.so")) if p)
-        r = subprocess.run([sys.executable, "-c", PINS, so], cwd=ROOT, env=env, capture_output=True, text=True,
-                           timeout=600)
+        return subprocess.run([sys.executable, "-c", PINS, so], cwd=ROOT, env=env, capture_output=True,
+                              text=True, timeout=600)
+
+
+@pytest.mark.parametrize("kind", ["address", "undefined"])
+def test_oracle_pins_under_a_sanitizer(kind):
+    r = _run_pins(kind, open(obuild.SRC).read())
     assert r.returncode == 0 and "pins ok under" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]
+
+
+def test_planted_overflow_is_reported():
+    src = open(obuild.SRC).read()
+    assert src.count(OVERFLOW[0]) == 1
+    r = _run_pins("address", src.replace(*OVERFLOW))
+    assert r.returncode != 0 and "heap-buffer-overflow" in r.stderr, r.stderr[-2000:]
