@@ -423,3 +423,33 @@ def test_binding_restypes_match_the_header():
             assert getattr(lib, m.group(2)).restype is want[ret], (m.group(2), ret)
             n += 1
     assert n >= 28
+
+
+def test_fuzzed_forward_arguments_get_a_documented_status():
+    # Random sizes, pointer alignments and null patterns: every call returns one of the header's
+    # statuses without touching memory; on a machine without a GPU, arguments that pass validation
+    # end in SWA_ERR_NO_DEVICE (no compute anywhere else).
+    import torch
+    from hypothesis import given, settings, strategies as st
+    codes = {swa.SWA_OK, swa.SWA_ERR_INVALID_ARG, swa.SWA_ERR_UNSUPPORTED, swa.SWA_ERR_MISALIGNED,
+             swa.SWA_ERR_CUDA, swa.SWA_ERR_TIMEOUT, swa.SWA_ERR_NO_MEMORY, swa.SWA_ERR_NO_DEVICE}
+    no_gpu = not torch.cuda.is_available()
+    sizes = st.integers(min_value=-3, max_value=1 << 20)
+    ptr = st.one_of(st.none(), st.sampled_from([A, A + 2, A + 8, A + 16]))
+
+    @settings(max_examples=300, deadline=None)
+    @given(q=ptr, k=ptr, v=ptr, ve=ptr, gx=ptr, wg=ptr, out=ptr, lse=ptr, B=sizes, T=sizes, H=sizes,
+           D=st.sampled_from([0, 32, 64, 96, 128, 256]), window=sizes,
+           base=st.sampled_from([1e4, 0.0, -1.0, float("inf"), float("nan")]),
+           eps=st.sampled_from([1e-6, 0.0, -1e-6, float("nan")]))
+    def check(q, k, v, ve, gx, wg, out, lse, B, T, H, D, window, base, eps):
+        rc = swa.swa_attn_fwd(q, k, v, ve, gx, wg, out, lse, B, T, H, D, window, base, eps, None)
+        assert rc in codes
+        valid = (None not in (q, k, v, out) and len({ve is None, gx is None, wg is None}) == 1
+                 and B >= 1 and T >= 1 and H >= 1 and D in (64, 128) and B * T * H * D < (1 << 31)
+                 and B <= 65535 and H <= 65535 and base > 0 and base != float("inf") and eps >= 0
+                 and all(p % 16 == 0 for p in (q, k, v, out)) and (lse is None or lse % 4 == 0)
+                 and (ve is None or (ve % 16 == 0 and gx % 2 == 0 and wg % 2 == 0)))
+        assert (rc == swa.SWA_ERR_NO_DEVICE) == (valid and no_gpu) or not no_gpu, (rc, valid)
+
+    check()
