@@ -453,3 +453,57 @@ def test_fuzzed_forward_arguments_get_a_documented_status():
         assert (rc == swa.SWA_ERR_NO_DEVICE) == (valid and no_gpu) or not no_gpu, (rc, valid)
 
     check()
+
+
+def test_fuzzed_decode_arguments_get_a_documented_status():
+    import torch
+    from hypothesis import given, settings, strategies as st
+    no_gpu = not torch.cuda.is_available()
+    ptr = st.one_of(st.none(), st.sampled_from([A, A + 4, A + 16]))
+
+    @settings(max_examples=300, deadline=None)
+    @given(q=ptr, kc=ptr, vc=ptr, ws=ptr, out=ptr, ve=st.sampled_from([None, A]), B=st.integers(-1, 40),
+           Tmax=st.integers(-1, 5000), H=st.integers(-1, 16), Hkv=st.integers(-1, 16), D=st.sampled_from([64, 96, 128]),
+           pos=st.integers(-2, 5001), ws_extra=st.integers(-2048, 2048))
+    def check(q, kc, vc, ws, out, ve, B, Tmax, H, Hkv, D, pos, ws_extra):
+        need = swa.swa_attn_decode_workspace_bytes(max(B, 1), max(Tmax, 1), max(H, 1), D, ve is not None, 0)
+        ws_bytes = max(0, need + ws_extra)
+        rc = swa._lib.swa_attn_decode_gqa(q, A, A, ve, ve, ve, kc, vc, pos, out, A, B, Tmax, H, Hkv, D, 0,
+                                          1e4, 1e-6, ws, ws_bytes, None)
+        valid = (None not in (q, kc, vc, ws, out) and B >= 1 and Tmax >= 1 and H >= 1 and D in (64, 128)
+                 and 1 <= Hkv <= H and H % Hkv == 0 and 0 <= pos < Tmax
+                 and all(p % 16 == 0 for p in (q, kc, vc, ws, out)) and ws_bytes >= need)
+        assert rc in range(-7, 1)
+        if no_gpu:
+            assert (rc == swa.SWA_ERR_NO_DEVICE) == valid, (rc, valid)
+
+    check()
+
+
+def test_fuzzed_backward_arguments_get_a_documented_status():
+    import torch
+    from hypothesis import given, settings, strategies as st
+    no_gpu = not torch.cuda.is_available()
+    ptr = st.one_of(st.none(), st.sampled_from([A, A + 4, A + 16]))
+
+    @settings(max_examples=300, deadline=None)
+    @given(out=ptr, lse=ptr, dout=ptr, dq=ptr, dk=ptr, ws=ptr, has_ve=st.booleans(),
+           vegrads=st.sampled_from([0, 1, 3]), B=st.integers(-1, 8), T=st.integers(-1, 3000),
+           H=st.integers(-1, 12), Hkv=st.integers(-1, 12), D=st.sampled_from([64, 96, 128]),
+           ws_extra=st.integers(-2048, 2048))
+    def check(out, lse, dout, dq, dk, ws, has_ve, vegrads, B, T, H, Hkv, D, ws_extra):
+        ve = A if has_ve else None
+        dve, dgx, dwg = [(A, A, A), (A, None, None), (None, None, None)][{3: 0, 1: 1, 0: 2}[vegrads]]
+        need = swa.swa_attn_bwd_workspace_bytes(max(B, 1), max(T, 1), max(H, 1), max(Hkv, 1), D, int(has_ve))
+        ws_bytes = max(0, need + ws_extra)
+        rc = swa.swa_attn_bwd_gqa(A, A, A, ve, ve, ve, out, lse, dout, None, dq, dk, A, dve, dgx, dwg, B, T, H,
+                                  Hkv, D, 0, 1e4, 1e-6, ws, ws_bytes, None)
+        valid = (None not in (out, lse, dout, dq, dk, ws) and B >= 1 and T >= 1 and H >= 1 and D in (64, 128)
+                 and 1 <= Hkv <= H and H % Hkv == 0 and vegrads == (3 if has_ve else 0)
+                 and all(p % 16 == 0 for p in (out, dout, dq, dk, ws)) and lse % 4 == 0 and need > 0
+                 and ws_bytes >= need)
+        assert rc in range(-7, 1)
+        if no_gpu:
+            assert (rc == swa.SWA_ERR_NO_DEVICE) == valid, (rc, valid)
+
+    check()
