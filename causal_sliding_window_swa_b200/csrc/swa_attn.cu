@@ -440,11 +440,12 @@ bool make_matrix_map(CUtensorMap* m, const void* base, long long rows, int cols,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int check_qkv_args(const void* x, const void* Wqkv, const void* ve, const void* Wg, int C, float rope_base,
-                   float eps) {
+int check_qkv_args(const void* x, const void* Wqkv, const void* ve, const void* Wg, const Shape& s, int C,
+                   float rope_base, float eps) {
     if (!x || !Wqkv) return SWA_ERR_INVALID_ARG;
     if ((ve == nullptr) != (Wg == nullptr)) return SWA_ERR_INVALID_ARG;
     if (C < 8 || (C % 8) != 0) return SWA_ERR_UNSUPPORTED;   // 16-byte rows for the tensor maps
+    if ((long long)s.B * s.T * C >= (1ll << 31)) return SWA_ERR_UNSUPPORTED;   // int32 indexing of x
     if (ve != nullptr && C < 32) return SWA_ERR_INVALID_ARG;  // the gate reads 32 channels
     if (!std::isfinite(rope_base) || !(rope_base > 0.f)) return SWA_ERR_INVALID_ARG;
     if (!std::isfinite(eps) || eps < 0.f) return SWA_ERR_INVALID_ARG;
@@ -1043,7 +1044,7 @@ int swa_attn_qkv_prologue(const void* x, const void* Wqkv, const void* ve, const
     Shape s;
     int rc = check_sizes(B, T, H, D, &s);
     if (rc == SWA_OK) rc = check_kv_heads(Hkv, &s);
-    if (rc == SWA_OK) rc = check_qkv_args(x, Wqkv, ve, Wg, C, rope_base, eps);
+    if (rc == SWA_OK) rc = check_qkv_args(x, Wqkv, ve, Wg, s, C, rope_base, eps);
     if (rc != SWA_OK) return rc;
     if (!qh || !kh || !vp || !workspace) return SWA_ERR_INVALID_ARG;
     if (!aligned(qh, 16) || !aligned(kh, 16) || !aligned(vp, 16) || !aligned(workspace, 16)) return SWA_ERR_MISALIGNED;
@@ -1063,7 +1064,7 @@ int swa_attn_fwd_x(const void* x, const void* Wqkv, const void* ve, const void* 
     Shape s;
     int rc = check_sizes(B, T, H, D, &s);
     if (rc == SWA_OK) rc = check_kv_heads(Hkv, &s);
-    if (rc == SWA_OK) rc = check_qkv_args(x, Wqkv, ve, Wg, C, rope_base, eps);
+    if (rc == SWA_OK) rc = check_qkv_args(x, Wqkv, ve, Wg, s, C, rope_base, eps);
     if (rc == SWA_OK) rc = check_outputs(out, lse);
     if (rc != SWA_OK) return rc;
     if (!workspace) return SWA_ERR_INVALID_ARG;

@@ -317,7 +317,7 @@ SWA_API int swa_attn_decode_doc(const void* q, const void* k, const void* v,
  * swa_attn_rope_table() again before swa_attn_prologue().  Asynchronous on `stream`; arguments are
  * validated before anything is enqueued.  Errors: SWA_ERR_INVALID_ARG (null pointer, ve / Wg not
  * both set, C < 32 with the value embedding, Hkv not dividing H, bad rope_base / eps),
- * SWA_ERR_UNSUPPORTED (D not 64 / 128, C not a multiple of 8, sizes beyond int32),
+ * SWA_ERR_UNSUPPORTED (D not 64 / 128, C not a multiple of 8, B T H D or B T C at least 2^31),
  * SWA_ERR_MISALIGNED, SWA_ERR_NO_MEMORY, SWA_ERR_CUDA.
  */
 SWA_API size_t swa_attn_fwd_x_workspace_bytes(int B, int T, int H, int Hkv, int D);

@@ -262,6 +262,13 @@ def test_fused_projection_workspace_and_validation():
     assert call(D=96) == swa.SWA_ERR_UNSUPPORTED
     assert swa.swa_attn_qkv_prologue(A, A, None, None, None, A, A, B, T, C, H, Hkv, D, 1e4, 1e-6, A, n,
                                      None) == swa.SWA_ERR_INVALID_ARG
+    # x with B T C = 2^31 elements (small B T H D): refused before the device is looked at
+    big = dict(B=2, T=1 << 14, C=1 << 16, H=1, Hkv=1, D=64)
+    nb = swa.swa_attn_fwd_x_workspace_bytes(2, 1 << 14, 1, 1, 64)
+    assert nb > 0
+    assert call(**big, ws_bytes=nb) == swa.SWA_ERR_UNSUPPORTED
+    assert swa.swa_attn_qkv_prologue(A, A, None, None, A, A, A, 2, 1 << 14, 1 << 16, 1, 1, 64, 1e4, 1e-6, A, nb,
+                                     None) == swa.SWA_ERR_UNSUPPORTED
 
 
 def test_header_is_plain_c():
@@ -502,6 +509,33 @@ def test_fuzzed_backward_arguments_get_a_documented_status():
                  and 1 <= Hkv <= H and H % Hkv == 0 and vegrads == (3 if has_ve else 0)
                  and all(p % 16 == 0 for p in (out, dout, dq, dk, ws)) and lse % 4 == 0 and need > 0
                  and ws_bytes >= need)
+        assert rc in range(-7, 1)
+        if no_gpu:
+            assert (rc == swa.SWA_ERR_NO_DEVICE) == valid, (rc, valid)
+
+    check()
+
+
+def test_fuzzed_fused_layer_arguments_get_a_documented_status():
+    # including inputs x too large for int32 indexing (B T C >= 2^31), refused before any work
+    import torch
+    from hypothesis import given, settings, strategies as st
+    no_gpu = not torch.cuda.is_available()
+    ptr = st.one_of(st.none(), st.sampled_from([A, A + 4, A + 16]))
+
+    @settings(max_examples=300, deadline=None)
+    @given(x=ptr, w=ptr, ws=ptr, out=ptr, ve=st.sampled_from([None, A]), wg=st.sampled_from([None, A]),
+           B=st.integers(-1, 1 << 12), T=st.integers(-1, 1 << 14), C=st.sampled_from([0, 12, 16, 32, 768, 1536, 1 << 16]),
+           H=st.integers(1, 12), Hkv=st.integers(1, 12), D=st.sampled_from([64, 96, 128]),
+           ws_extra=st.integers(-2048, 2048))
+    def check(x, w, ws, out, ve, wg, B, T, C, H, Hkv, D, ws_extra):
+        need = swa.swa_attn_fwd_x_workspace_bytes(max(B, 1), max(T, 1), H, Hkv, D)
+        ws_bytes = max(0, need + ws_extra)
+        rc = swa.swa_attn_fwd_x(x, w, ve, wg, out, A, B, T, C, H, Hkv, D, 0, 1e4, 1e-6, ws, ws_bytes, None)
+        valid = (None not in (x, w, ws, out) and B >= 1 and T >= 1 and D in (64, 128) and H % Hkv == 0
+                 and Hkv <= H and B * T * H * D < (1 << 31) and (ve is None) == (wg is None)
+                 and C >= 8 and C % 8 == 0 and (ve is None or C >= 32) and B * T * C < (1 << 31)
+                 and all(p % 16 == 0 for p in (x, w, ws, out)) and need > 0 and ws_bytes >= need)
         assert rc in range(-7, 1)
         if no_gpu:
             assert (rc == swa.SWA_ERR_NO_DEVICE) == valid, (rc, valid)
