@@ -262,10 +262,14 @@ def _ptr(t) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
-def _stream_handle(stream):
+def _stream_handle(stream, device=None):
+    """The CUDA stream handle of `stream` (None = the current stream).  A torch stream must belong
+    to `device`, the inputs' GPU, when that is given."""
     import torch
     if stream is None:
         stream = torch.cuda.current_stream()
+    if device is not None and getattr(stream, "device", device) != device:
+        raise ValueError(f"stream is on {stream.device}, the inputs on {device}")
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
 
 
@@ -349,7 +353,7 @@ def forward(q, k, v, window: int = 0, ve=None, gate_x=None, Wg=None, rope_base: 
     if Hkv != H and workspace is not None:
         raise ValueError("a caller workspace is supported for multi-head layers only")
     with torch.cuda.device(dev):
-        st = _stream_handle(stream)
+        st = _stream_handle(stream, dev)
         if doc is not None:
             rc = swa_attn_fwd_doc(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(doc),
                                   _ptr(out), _ptr(lse), B, T, H, Hkv, D, int(window), float(rope_base), float(eps),
@@ -416,7 +420,7 @@ def decode(q, k, v, k_cache, v_cache, pos: int, window: int, ve=None, gate_x=Non
         _want("doc_start", doc_start, (B,), torch.int32, dev)
     ws_bytes = workspace.numel() * workspace.element_size()
     with torch.cuda.device(dev):
-        st = _stream_handle(stream)
+        st = _stream_handle(stream, dev)
         rc = _lib.swa_attn_decode_doc(_ptr(q), _ptr(k), _ptr(v), _ptr(ve), _ptr(gate_x), _ptr(Wg), _ptr(k_cache),
                                       _ptr(v_cache), int(pos), _ptr(doc_start), _ptr(out), _ptr(lse), B, Tmax, H,
                                       Hkv, D, int(window), float(rope_base), float(eps), _ptr(workspace), ws_bytes,
@@ -470,7 +474,7 @@ def backward(q, k, v, out, lse, dout, window: int = 0, dlse=None, ve=None, gate_
         raise ValueError("saved=True needs the forward's workspace, Hkv == H and no document mask")
     with torch.cuda.device(dev):
         return _backward_call(q, k, v, ve, gate_x, Wg, doc, out, lse, dout, dlse, g, B, T, H, Hkv, D, window,
-                              rope_base, eps, workspace, _stream_handle(stream), saved)
+                              rope_base, eps, workspace, _stream_handle(stream, dev), saved)
 
 
 def _backward_call(q, k, v, ve, gate_x, Wg, doc, out, lse, dout, dlse, g, B, T, H, Hkv, D, window, rope_base,
@@ -522,7 +526,8 @@ def qkv_prologue(x, Wqkv, H: int, Hkv: int, D: int, ve=None, Wg=None, rope_base:
     ws = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
     with torch.cuda.device(x.device):
         rc = swa_attn_qkv_prologue(_ptr(x), _ptr(Wqkv), _ptr(ve), _ptr(Wg), _ptr(qh), _ptr(kh), _ptr(vp), B, T, C,
-                                   H, Hkv, D, float(rope_base), float(eps), _ptr(ws), need, _stream_handle(stream))
+                                   H, Hkv, D, float(rope_base), float(eps), _ptr(ws), need,
+                                   _stream_handle(stream, x.device))
     if rc != SWA_OK:
         raise SwaError(rc, "swa_attn_qkv_prologue")
     return qh, kh, vp
@@ -543,7 +548,7 @@ def forward_x(x, Wqkv, H: int, Hkv: int, D: int, window: int = 0, ve=None, Wg=No
     with torch.cuda.device(x.device):
         rc = swa_attn_fwd_x(_ptr(x), _ptr(Wqkv), _ptr(ve), _ptr(Wg), _ptr(out), _ptr(lse), B, T, C, H, Hkv, D,
                             int(window), float(rope_base), float(eps), _ptr(workspace),
-                            workspace.numel() * workspace.element_size(), _stream_handle(stream))
+                            workspace.numel() * workspace.element_size(), _stream_handle(stream, x.device))
     if rc != SWA_OK:
         raise SwaError(rc, "swa_attn_fwd_x")
     return out, lse

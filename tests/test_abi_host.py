@@ -541,3 +541,14 @@ def test_fuzzed_fused_layer_arguments_get_a_documented_status():
             assert (rc == swa.SWA_ERR_NO_DEVICE) == valid, (rc, valid)
 
     check()
+
+
+def test_stream_handle_checks_the_device():
+    # a torch stream must be on the inputs' GPU; a raw handle has no device to check
+    import types
+    import torch
+    dev0, dev1 = torch.device("cuda", 0), torch.device("cuda", 1)
+    with pytest.raises(ValueError, match="stream is on cuda:1"):
+        swa._stream_handle(types.SimpleNamespace(device=dev1, cuda_stream=1234), dev0)
+    assert swa._stream_handle(types.SimpleNamespace(device=dev0, cuda_stream=99), dev0) == 99
+    assert swa._stream_handle(5678, dev0) == 5678
