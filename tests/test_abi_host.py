@@ -552,3 +552,37 @@ def test_stream_handle_checks_the_device():
         swa._stream_handle(types.SimpleNamespace(device=dev1, cuda_stream=1234), dev0)
     assert swa._stream_handle(types.SimpleNamespace(device=dev0, cuda_stream=99), dev0) == 99
     assert swa._stream_handle(5678, dev0) == 5678
+
+
+def test_fuzzed_stage_arguments_get_a_documented_status():
+    # the stage entry points (RoPE table, prologue, attention) on random arguments
+    import torch
+    from hypothesis import given, settings, strategies as st
+    no_gpu = not torch.cuda.is_available()
+    ptr = st.one_of(st.none(), st.sampled_from([A, A + 4, A + 16]))
+
+    @settings(max_examples=300, deadline=None)
+    @given(v=ptr, out=ptr, lse=ptr, ws=ptr, has_ve=st.booleans(), B=st.integers(-1, 16), T=st.integers(-1, 4096),
+           H=st.integers(-1, 16), D=st.sampled_from([64, 96, 128]), base=st.sampled_from([1e4, 0.0, float("nan")]),
+           ws_extra=st.integers(-2048, 2048))
+    def check(v, out, lse, ws, has_ve, B, T, H, D, base, ws_extra):
+        need = swa.swa_attn_workspace_bytes(max(B, 1), max(T, 1), max(H, 1), D, int(has_ve))
+        wsb = max(0, need + ws_extra)
+        sizes_ok = B >= 1 and T >= 1 and H >= 1 and D in (64, 128)
+        ws_ok = ws is not None and ws % 16 == 0 and need > 0 and wsb >= need
+        ve = A if has_ve else None
+        rcs = {
+            "rope": (swa.swa_attn_rope_table(B, T, H, D, int(has_ve), base, ws, wsb, None),
+                     sizes_ok and base > 0 and ws_ok),
+            "prologue": (swa.swa_attn_prologue(A, A, A, ve, ve, ve, B, T, H, D, base, 1e-6, ws, wsb, None),
+                         sizes_ok and base > 0 and ws_ok),
+            "attention": (swa.swa_attn_attention(v, int(has_ve), out, lse, B, T, H, D, 0, ws, wsb, None),
+                          sizes_ok and ws_ok and out is not None and out % 16 == 0
+                          and (lse is None or lse % 4 == 0) and (has_ve or (v is not None and v % 16 == 0))),
+        }
+        for name, (rc, valid) in rcs.items():
+            assert rc in range(-7, 1), name
+            if no_gpu:
+                assert (rc == swa.SWA_ERR_NO_DEVICE) == valid, (name, rc, valid)
+
+    check()
