@@ -206,6 +206,18 @@ def swa_attn_decode(q, k, v, ve, gate_x, Wg, k_cache, v_cache, pos, out, lse, B,
                                 window, rope_base, eps, workspace, ws_bytes, stream)
 
 
+def swa_attn_decode_gqa(q, k, v, ve, gate_x, Wg, k_cache, v_cache, pos, out, lse, B, Tmax, H, Hkv, D, window,
+                        rope_base, eps, workspace, ws_bytes, stream) -> int:
+    return _lib.swa_attn_decode_gqa(q, k, v, ve, gate_x, Wg, k_cache, v_cache, pos, out, lse, B, Tmax, H, Hkv,
+                                    D, window, rope_base, eps, workspace, ws_bytes, stream)
+
+
+def swa_attn_decode_doc(q, k, v, ve, gate_x, Wg, k_cache, v_cache, pos, doc_start, out, lse, B, Tmax, H, Hkv, D,
+                        window, rope_base, eps, workspace, ws_bytes, stream) -> int:
+    return _lib.swa_attn_decode_doc(q, k, v, ve, gate_x, Wg, k_cache, v_cache, pos, doc_start, out, lse, B, Tmax,
+                                    H, Hkv, D, window, rope_base, eps, workspace, ws_bytes, stream)
+
+
 def swa_attn_bwd_workspace_bytes(B, T, H, Hkv, D, has_ve) -> int:
     return int(_lib.swa_attn_bwd_workspace_bytes(B, T, H, Hkv, D, int(has_ve)))
 
@@ -562,12 +574,14 @@ def check_device_status(stream=None) -> None:
 
 
 __all__ = [
-    "forward", "decode", "backward", "qkv_prologue", "forward_x", "check_device_status", "SwaError", "LIB_PATH", "load",
-    "swa_attn_fwd", "swa_attn_fwd_ws", "swa_attn_fwd_noalloc", "swa_attn_noalloc_scratch_bytes", "swa_attn_workspace_bytes", "swa_attn_workspace_offset", "swa_attn_rope_table", "swa_attn_prologue",
-    "swa_attn_attention", "swa_attn_strerror",
-    "swa_attn_last_device_status",
-    "swa_attn_set_wait_limit_ms", "swa_attn_selftest_wait", "swa_attn_version",
-    "swa_attn_decode", "swa_attn_decode_workspace_bytes", "swa_attn_fwd_gqa", "swa_attn_fwd_doc",
-    "swa_attn_bwd", "swa_attn_bwd_saved", "swa_attn_bwd_gqa", "swa_attn_bwd_doc", "swa_attn_bwd_workspace_bytes",
-    "swa_attn_fwd_x", "swa_attn_qkv_prologue", "swa_attn_fwd_x_workspace_bytes",
+    "forward", "decode", "backward", "qkv_prologue", "forward_x", "check_device_status", "SwaError",
+    "LIB_PATH", "load", "swa_attn_fwd", "swa_attn_fwd_ws", "swa_attn_fwd_noalloc",
+    "swa_attn_noalloc_scratch_bytes", "swa_attn_workspace_bytes", "swa_attn_workspace_offset",
+    "swa_attn_rope_table", "swa_attn_prologue", "swa_attn_attention", "swa_attn_strerror",
+    "swa_attn_last_device_status", "swa_attn_set_wait_limit_ms", "swa_attn_selftest_wait", "swa_attn_version",
+    "swa_attn_decode", "swa_attn_decode_gqa", "swa_attn_decode_doc", "swa_attn_decode_workspace_bytes",
+    "swa_attn_fwd_gqa", "swa_attn_fwd_doc",
+    "swa_attn_bwd", "swa_attn_bwd_saved", "swa_attn_bwd_gqa", "swa_attn_bwd_doc",
+    "swa_attn_bwd_workspace_bytes", "swa_attn_fwd_x", "swa_attn_qkv_prologue",
+    "swa_attn_fwd_x_workspace_bytes",
 ]

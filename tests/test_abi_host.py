@@ -586,3 +586,16 @@ def test_fuzzed_stage_arguments_get_a_documented_status():
                 assert (rc == swa.SWA_ERR_NO_DEVICE) == valid, (name, rc, valid)
 
     check()
+
+
+def test_every_entry_point_has_a_binding_of_the_same_name():
+    # one Python function per C entry point, taking the C inputs in order; an `unsigned int*`
+    # out-parameter is returned by the Python function instead of passed in
+    import inspect
+    lib = swa.load()
+    for name, params in _prototypes().items():
+        fn = getattr(swa, name, None)
+        assert callable(fn) and name in swa.__all__, name
+        inputs = [p for p in params if not re.match(r"unsigned\s+int\s*\*", p)]
+        assert len(inspect.signature(fn).parameters) == len(inputs), name
+        assert len(params) == len(getattr(lib, name).argtypes), name
