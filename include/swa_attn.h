@@ -85,7 +85,7 @@ typedef enum swa_status {
  *              otherwise all three set (else SWA_ERR_INVALID_ARG).
  * out          bf16 (B,T,H,D), written.
  * lse          fp32 (B,H,T), written; NULL skips it.
- * B, T, H      >= 1;  D in {64, 128};  B*T*H*D < 2^31.
+ * B, T, H      >= 1;  D in {64, 128};  B*T*H*D < 2^31;  B, H <= 65535 (else SWA_ERR_UNSUPPORTED).
  * window       keys visible to a query, counting itself; <= 0 or >= T is full causal.
  * rope_base    > 0 and finite (10000 in the pages' models).
  * eps          >= 0 and finite (1e-6 here).  At eps = 0 an all-zero q or k head row has no
