@@ -146,3 +146,15 @@ def test_gpu_arm_without_a_device_fails_loudly():
         pytest.skip("a CUDA device is visible")
     r = _bench("--steps", "1", "--warmup", "3")
     assert r.returncode != 0 and "{" not in r.stdout and "needs a CUDA device" in r.stderr
+
+
+def test_input_bytes_and_config_by_hand():
+    # d24 L+VE reads q, k, v and ve: 4 x 16 x 2048 x 12 x 128 bf16 = 402.65 MB; GPT-2 124M reads
+    # q, k, v: 3 x 8 x 1024 x 12 x 64 bf16 = 37.7 MB
+    assert bench.input_bytes(workloads.D24_L_VE) == 4 * 16 * 2048 * 12 * 128 * 2
+    assert bench.input_bytes(workloads.GPT2) == 3 * 8 * 1024 * 12 * 64 * 2
+    c = bench.config_of(workloads.D24_L_VE, 1)
+    assert (c["B_per_gpu"], c["T"], c["H"], c["D"], c["window"], c["value_embeddings"]) == (16, 2048, 12, 128, 2048, True)
+    assert c["workload"] == "d24 L+VE (16,2048,12,128) W=2048" and c["global_batch"] == 16
+    assert "403 MB" in c["l2"]
+    assert bench.config_of(workloads.D24_L_VE, 4)["global_batch"] == 64     # weak scaling: B per GPU fixed
