@@ -158,3 +158,16 @@ def test_input_bytes_and_config_by_hand():
     assert c["workload"] == "d24 L+VE (16,2048,12,128) W=2048" and c["global_batch"] == 16
     assert "403 MB" in c["l2"]
     assert bench.config_of(workloads.D24_L_VE, 4)["global_batch"] == 64     # weak scaling: B per GPU fixed
+
+
+def test_sssl_stack_recipe():
+    # S,S,S,L windows (S = T/2), value embeddings on even layers, and every layer drawn in turn
+    # from one generator: no two layers share inputs, so L2 cannot serve a later layer's data
+    shapes = workloads.sssl_layer_shapes(2, 64, 2, 64, n_layers=8)
+    assert [s.window for s in shapes] == [32, 32, 32, 64] * 2
+    assert [s.ve for s in shapes] == [True, False] * 4
+    stack = workloads.sssl_stack(2, 64, 2, 64, n_layers=8)
+    hashes = [workloads.sha256_of(d) for _, d in stack]
+    assert len(set(hashes)) == 8
+    again = [workloads.sha256_of(d) for _, d in workloads.sssl_stack(2, 64, 2, 64, n_layers=8)]
+    assert hashes == again                                       # seeded: the same stack every run
